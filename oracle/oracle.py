@@ -1,0 +1,209 @@
+"""ctypes front end of the fp64 C oracle (oracle/slay_oracle.c).
+
+TEST INFRASTRUCTURE ONLY: used by tests/, the package smoke check and the
+benchmark's CPU-baseline leg.  Arguments are numpy arrays; everything is
+converted to C-contiguous float64 before the call.  The parameter set
+(omega, anchors, s, wt) is drawn by the oracle's own Philox from the seed.
+"""
+import ctypes as C
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = C.CDLL(path)
+        dp = C.POINTER(C.c_double)
+        i64p = C.POINTER(C.c_int64)
+        u32p = C.POINTER(C.c_uint32)
+        L.orc_philox4x32_10.argtypes = [u32p, u32p, u32p]
+        L.orc_philox4x32_10.restype = None
+        L.orc_gauss_laguerre.argtypes = [C.c_int, dp, dp]
+        L.orc_gauss_laguerre.restype = C.c_int
+        L.orc_sketch_params.argtypes = [C.c_int, C.c_int, C.c_int, C.c_uint64, C.c_double,
+                                        dp, dp, dp, dp]
+        L.orc_sketch_params.restype = C.c_int
+        L.orc_yat_kernel.argtypes = [C.c_double, C.c_double]
+        L.orc_yat_kernel.restype = C.c_double
+        L.orc_quad_kernel.argtypes = [C.c_double, C.c_int, C.c_double]
+        L.orc_quad_kernel.restype = C.c_double
+        par = [dp, dp, dp, dp]
+        L.orc_feature_map.argtypes = [dp, C.c_int64, C.c_int, C.c_int, C.c_int] + par + [dp]
+        L.orc_feature_map.restype = None
+        shp = [C.c_int] * 7
+        L.orc_attn_quadratic.argtypes = [dp, dp, dp] + shp + par + [C.c_double, C.c_int, dp, dp]
+        L.orc_attn_quadratic.restype = None
+        L.orc_attn_quadratic_rows.argtypes = ([dp, dp, dp] + shp + par +
+                                              [C.c_double, C.c_int, i64p, C.c_int, dp, dp])
+        L.orc_attn_quadratic_rows.restype = None
+        L.orc_attn_recurrent.argtypes = [dp, dp, dp] + shp + par + [C.c_double, C.c_int, dp, dp]
+        L.orc_attn_recurrent.restype = None
+        L.orc_decode_step.argtypes = ([dp, dp, dp, dp, dp, dp] + [C.c_int] * 5 + par +
+                                      [C.c_double])
+        L.orc_decode_step.restype = None
+        L.orc_attn_causal_bwd.argtypes = [dp, dp, dp, dp] + shp + par + [C.c_double, dp, dp, dp]
+        L.orc_attn_causal_bwd.restype = None
+        L.orc_attn_causal_bwd_rows.argtypes = ([dp, dp, dp, dp] + shp + par +
+                                               [C.c_double, i64p, C.c_int, dp, dp, dp])
+        L.orc_attn_causal_bwd_rows.restype = None
+        L.orc_num_threads.argtypes = []
+        L.orc_num_threads.restype = C.c_int
+        _lib = L
+    return _lib
+
+
+def _d(a):
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _p(a):
+    return a.ctypes.data_as(C.POINTER(C.c_double))
+
+
+def num_threads() -> int:
+    return lib().orc_num_threads()
+
+
+def philox4x32_10(ctr, key):
+    c = (C.c_uint32 * 4)(*[int(x) & 0xffffffff for x in ctr])
+    k = (C.c_uint32 * 2)(*[int(x) & 0xffffffff for x in key])
+    o = (C.c_uint32 * 4)()
+    lib().orc_philox4x32_10(c, k, o)
+    return [int(x) for x in o]
+
+
+def gauss_laguerre(R: int):
+    t = np.zeros(R)
+    w = np.zeros(R)
+    if lib().orc_gauss_laguerre(R, _p(t), _p(w)) != 0:
+        raise ValueError("gauss_laguerre failed for R=%d" % R)
+    return t, w
+
+
+class Params:
+    """Sketch parameters of one (D, R, m, seed, eps) key, drawn by the oracle."""
+
+    def __init__(self, D, R, m, seed, eps):
+        F = R * m
+        self.D, self.R, self.m, self.seed, self.eps, self.F = D, R, m, seed, eps, F
+        self.omega = np.zeros((F, D))
+        self.anchors = np.zeros((F, D))
+        self.s = np.zeros(R)
+        self.wt = np.zeros(R)
+        rc = lib().orc_sketch_params(D, R, m, C.c_uint64(seed), eps, _p(self.omega),
+                                     _p(self.anchors), _p(self.s), _p(self.wt))
+        if rc != 0:
+            raise ValueError("sketch_params failed")
+
+    def args(self):
+        return [_p(self.omega), _p(self.anchors), _p(self.s), _p(self.wt)]
+
+
+def sketch_params(D, R, m, seed, eps) -> Params:
+    return Params(D, R, m, seed, eps)
+
+
+def yat_kernel(x, eps):
+    return lib().orc_yat_kernel(float(x), float(eps))
+
+
+def quad_kernel(x, R, eps):
+    return lib().orc_quad_kernel(float(x), int(R), float(eps))
+
+
+def feature_map(x, P: Params):
+    x = _d(x)
+    n = x.size // P.D
+    phi = np.zeros((n, P.F))
+    lib().orc_feature_map(_p(x), n, P.D, P.R, P.m, *P.args(), _p(phi))
+    return phi.reshape(x.shape[:-1] + (P.F,))
+
+
+def _shape4(q, v):
+    B, H, L, D = q.shape
+    return B, H, L, D, v.shape[-1]
+
+
+def attn_quadratic(q, k, v, P: Params, causal: bool):
+    q, k, v = _d(q), _d(k), _d(v)
+    B, H, L, D, Dv = _shape4(q, v)
+    out = np.zeros((B, H, L, Dv))
+    den = np.zeros((B, H, L))
+    lib().orc_attn_quadratic(_p(q), _p(k), _p(v), B, H, L, D, Dv, P.R, P.m, *P.args(),
+                             P.eps, int(causal), _p(out), _p(den))
+    return out, den
+
+
+def attn_quadratic_rows(q, k, v, P: Params, causal: bool, rows):
+    q, k, v = _d(q), _d(k), _d(v)
+    B, H, L, D, Dv = _shape4(q, v)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    nr = rows.size
+    out = np.zeros((B, H, nr, Dv))
+    den = np.zeros((B, H, nr))
+    lib().orc_attn_quadratic_rows(_p(q), _p(k), _p(v), B, H, L, D, Dv, P.R, P.m, *P.args(),
+                                  P.eps, int(causal),
+                                  rows.ctypes.data_as(C.POINTER(C.c_int64)), nr,
+                                  _p(out), _p(den))
+    return out, den
+
+
+def attn_recurrent(q, k, v, P: Params, causal: bool):
+    q, k, v = _d(q), _d(k), _d(v)
+    B, H, L, D, Dv = _shape4(q, v)
+    out = np.zeros((B, H, L, Dv))
+    den = np.zeros((B, H, L))
+    lib().orc_attn_recurrent(_p(q), _p(k), _p(v), B, H, L, D, Dv, P.R, P.m, *P.args(),
+                             P.eps, int(causal), _p(out), _p(den))
+    return out, den
+
+
+def decode_step(q, k, v, S, z, P: Params):
+    """Returns (out, S_new, z_new); inputs are not modified."""
+    q, k, v = _d(q), _d(k), _d(v)
+    S = _d(S).copy()
+    z = _d(z).copy()
+    N = q.size // P.D
+    Dv = v.shape[-1]
+    out = np.zeros(v.shape)
+    lib().orc_decode_step(_p(q), _p(k), _p(v), _p(S), _p(z), _p(out), N, P.D, Dv, P.R, P.m,
+                          *P.args(), P.eps)
+    return out, S, z
+
+
+def attn_causal_bwd(q, k, v, dout, P: Params):
+    q, k, v, g = _d(q), _d(k), _d(v), _d(dout)
+    B, H, L, D, Dv = _shape4(q, v)
+    dq = np.zeros(q.shape)
+    dk = np.zeros(k.shape)
+    dv = np.zeros(v.shape)
+    lib().orc_attn_causal_bwd(_p(q), _p(k), _p(v), _p(g), B, H, L, D, Dv, P.R, P.m, *P.args(),
+                              P.eps, _p(dq), _p(dk), _p(dv))
+    return dq, dk, dv
+
+
+def attn_causal_bwd_rows(q, k, v, dout, P: Params, rows):
+    q, k, v, g = _d(q), _d(k), _d(v), _d(dout)
+    B, H, L, D, Dv = _shape4(q, v)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    nr = rows.size
+    dq = np.zeros((B, H, nr, D))
+    dk = np.zeros((B, H, nr, D))
+    dv = np.zeros((B, H, nr, Dv))
+    lib().orc_attn_causal_bwd_rows(_p(q), _p(k), _p(v), _p(g), B, H, L, D, Dv, P.R, P.m,
+                                   *P.args(), P.eps,
+                                   rows.ctypes.data_as(C.POINTER(C.c_int64)), nr,
+                                   _p(dq), _p(dk), _p(dv))
+    return dq, dk, dv
+
+
+__all__ = ["lib", "num_threads", "philox4x32_10", "gauss_laguerre", "Params", "sketch_params",
+           "yat_kernel", "quad_kernel", "feature_map", "attn_quadratic", "attn_quadratic_rows",
+           "attn_recurrent", "decode_step", "attn_causal_bwd", "attn_causal_bwd_rows"]

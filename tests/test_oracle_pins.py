@@ -1,0 +1,341 @@
+"""Pins of the fp64 oracle to facts fixed outside the oracle itself (CPU only).
+
+Each test checks the oracle against a published known-answer vector, a library
+routine, a closed form, an invariant or a brute-force special case, chosen so that a
+plausible slip (a dropped term, a wrong sign or index, a transposed operand, an
+exclusive instead of inclusive causal sum) fails at least one of them.
+
+Method source: "SLAY: Geometry-Aware Spherical Linearized Attention with Yat-Kernel"
+(abstract; nubint.ai review, "Proposed method" steps 1-6).
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ------------------------------------------------------------------ Philox
+
+def _kat_rows():
+    rows = []
+    with open(os.path.join(GOLDEN, "philox4x32_10_kat.txt")) as fh:
+        for line in fh:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            w = [int(x, 16) for x in line.split()]
+            rows.append((w[0:4], w[4:6], w[6:10]))
+    return rows
+
+
+def test_philox_known_answers():
+    rows = _kat_rows()
+    assert len(rows) == 3
+    for ctr, key, out in rows:
+        assert O.philox4x32_10(ctr, key) == out
+
+
+# --------------------------------------------------------- Gauss-Laguerre
+
+@pytest.mark.parametrize("R", list(range(1, 17)))
+def test_gauss_laguerre_moments(R):
+    # The R-point rule integrates e^{-t} t^k exactly for k < 2R: int = k!.
+    t, w = O.gauss_laguerre(R)
+    for k in range(2 * R):
+        got = float(np.sum(w * t ** k))
+        assert abs(got - math.factorial(k)) <= 1e-11 * math.factorial(k), (R, k, got)
+    # ... and not for k = 2R (the degree is exactly 2R-1): the remainder is
+    # (R!)^2 > 0, so the rule falls short of (2R)! by exactly (R!)^2.
+    got = float(np.sum(w * t ** (2 * R)))
+    want = math.factorial(2 * R) - math.factorial(R) ** 2
+    assert abs(got - want) <= 1e-9 * math.factorial(2 * R)
+
+
+def test_gauss_laguerre_two_point_closed_form():
+    t, w = O.gauss_laguerre(2)
+    r2 = math.sqrt(2.0)
+    np.testing.assert_allclose(t, [2 - r2, 2 + r2], rtol=1e-15)
+    np.testing.assert_allclose(w, [(2 + r2) / 4, (2 - r2) / 4], rtol=1e-14)
+
+
+@pytest.mark.parametrize("R", [1, 2, 3, 4, 5, 8, 12, 16, 24, 32])
+def test_gauss_laguerre_matches_library_rule(R):
+    t, w = O.gauss_laguerre(R)
+    tn, wn = np.polynomial.laguerre.laggauss(R)
+    np.testing.assert_allclose(t, tn, rtol=1e-12)
+    np.testing.assert_allclose(w, wn, rtol=1e-9, atol=1e-300)
+
+
+# ------------------------------------------------------- Yat kernel, quadrature
+
+def test_yat_kernel_on_sphere_matches_definition():
+    # (q.k)^2 / (|q-k|^2 + eps) evaluated from the vectors equals x^2/(2-2x+eps).
+    rng = np.random.default_rng(0)
+    eps = 1e-6
+    for _ in range(50):
+        q = rng.standard_normal(7); q /= np.linalg.norm(q)
+        k = rng.standard_normal(7); k /= np.linalg.norm(k)
+        direct = float(q @ k) ** 2 / (float(np.sum((q - k) ** 2)) + eps)
+        assert O.yat_kernel(float(q @ k), eps) == pytest.approx(direct, rel=1e-9)
+    assert O.yat_kernel(-1.0, eps) == pytest.approx(1.0 / (4.0 + eps), rel=1e-15)
+    assert O.yat_kernel(0.0, eps) == 0.0
+    assert O.yat_kernel(1.0, eps) == pytest.approx(1.0 / eps, rel=1e-12)
+
+
+def test_yat_kernel_positive_definite_and_bounded():
+    # The abstract states PD and boundedness on the sphere.
+    rng = np.random.default_rng(1)
+    X = rng.standard_normal((60, 5))
+    X /= np.linalg.norm(X, axis=1, keepdims=True)
+    G = X @ X.T
+    eps = 1e-2
+    K = np.vectorize(lambda x: O.yat_kernel(min(x, 1.0), eps))(G)
+    ev = np.linalg.eigvalsh(K)
+    assert ev.min() > -1e-9 * ev.max()
+    assert K.max() <= 1.0 / eps * (1 + 1e-12)
+
+
+@pytest.mark.parametrize("x", [-1.0, -0.5, 0.3, 0.5, 0.8])
+def test_quadrature_converges_from_below(x):
+    # Gauss-Laguerre error for f(t) = e^{ct} is (R!)^2/(2R)! c^{2R} e^{c xi} > 0, so the
+    # quadrature kernel stays at or below the closed form and approaches it as R grows.
+    eps = 1e-6
+    exact = O.yat_kernel(x, eps)
+    errs = []
+    for R in (2, 4, 8, 16, 32):
+        q = O.quad_kernel(x, R, eps)
+        errs.append((q - exact) / exact)
+        assert q <= exact * (1 + 1e-12)
+    assert all(abs(errs[i + 1]) < abs(errs[i]) or abs(errs[i]) < 1e-12 for i in range(4))
+    assert abs(errs[-1]) < 1e-8
+
+
+def test_quadrature_zero_at_x_zero():
+    for R in (1, 4, 8):
+        assert O.quad_kernel(0.0, R, 1e-6) == 0.0
+
+
+# ----------------------------------------------------------------- phi
+
+def test_sketch_params_shapes_and_marginals():
+    P = O.sketch_params(D=64, R=4, m=256, seed=1234, eps=1e-6)
+    assert P.omega.shape == (1024, 64) and P.anchors.shape == (1024, 64)
+    # fp32 rounding of the draws
+    assert np.array_equal(P.omega, P.omega.astype(np.float32).astype(np.float64))
+    assert np.array_equal(P.anchors, P.anchors.astype(np.float32).astype(np.float64))
+    # omega ~ N(0,1), anchors ~ N(0, 1/D): moments within a few standard errors
+    n = P.omega.size
+    assert abs(P.omega.mean()) < 4 / math.sqrt(n)
+    assert abs(P.omega.var() - 1.0) < 4 * math.sqrt(2.0 / n)
+    assert abs(P.anchors.var() * 64 - 1.0) < 4 * math.sqrt(2.0 / n)
+    # fourth moment of a standard normal is 3 (catches a uniform or wrong-scale draw)
+    assert abs(np.mean(P.omega ** 4) - 3.0) < 0.1
+    # independence of omega and anchors
+    assert abs(np.corrcoef(P.omega.ravel(), P.anchors.ravel())[0, 1]) < 4 / math.sqrt(n)
+    # quadrature tables
+    t, w = O.gauss_laguerre(4)
+    np.testing.assert_allclose(P.s, t / (2 + 1e-6), rtol=1e-15)
+    np.testing.assert_allclose(P.wt, w / (2 + 1e-6), rtol=1e-15)
+    # different seeds give different draws; same seed is reproducible
+    P2 = O.sketch_params(D=64, R=4, m=256, seed=1234, eps=1e-6)
+    P3 = O.sketch_params(D=64, R=4, m=256, seed=1235, eps=1e-6)
+    assert np.array_equal(P.omega, P2.omega)
+    assert not np.array_equal(P.omega, P3.omega)
+
+
+def test_phi_strictly_positive_and_scale_invariant():
+    P = O.sketch_params(D=64, R=4, m=64, seed=3, eps=1e-6)
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((40, 64))
+    phi = O.feature_map(x, P)
+    assert phi.shape == (40, 256)
+    assert (phi > 0).all()
+    np.testing.assert_allclose(O.feature_map(3.7 * x, P), phi, rtol=1e-9)
+    np.testing.assert_allclose(O.feature_map(1e-3 * x, P), phi, rtol=1e-9)
+    # a zero row is degenerate: x^ = 0, every anchor factor is 0
+    z = O.feature_map(np.zeros((1, 64)), P)
+    assert (z == 0).all()
+
+
+@pytest.mark.parametrize("x", [0.35, -0.4])
+def test_phi_monte_carlo_mean_per_node(x):
+    # For unit q, k with q.k = x, omega ~ N(0,I), a ~ N(0,I/D):
+    #   E[exp(sqrt(2s) w.q - s) exp(sqrt(2s) w.k - s)] = exp(2 s x)
+    #   E[(a.q)^2 (a.k)^2] = (1 + 2 x^2) / D^2        (Isserlis)
+    # so m * mean_j phi_{rj}(q) phi_{rj}(k) -> wt_r exp(2 s_r x) (1 + 2x^2)/D^2.
+    D, R, m = 4, 3, 200000
+    P = O.sketch_params(D=D, R=R, m=m, seed=11, eps=1e-6)
+    q = np.array([1.0, 0.0, 0.0, 0.0])
+    k = np.array([x, math.sqrt(1 - x * x), 0.0, 0.0])
+    pq = O.feature_map(q[None], P)[0]
+    pk = O.feature_map(k[None], P)[0]
+    prod = (pq * pk).reshape(R, m) * m
+    for r in range(R):
+        want = P.wt[r] * math.exp(2 * P.s[r] * x) * (1 + 2 * x * x) / D ** 2
+        mean = prod[r].mean()
+        sem = prod[r].std() / math.sqrt(m)
+        assert abs(mean - want) < 4.5 * sem, (r, mean, want, sem)
+        assert sem < 0.2 * want  # informative even for the heavy-tailed top node
+
+
+# ------------------------------------------------------------ contraction
+
+def _small(seed, B=2, H=2, L=37, D=16, Dv=8):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, H, L, D))
+    k = rng.standard_normal((B, H, L, D))
+    v = rng.standard_normal((B, H, L, Dv))
+    return q, k, v
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_quadratic_equals_recurrent(causal):
+    q, k, v = _small(3)
+    P = O.sketch_params(D=16, R=3, m=8, seed=5, eps=1e-6)
+    o1, d1 = O.attn_quadratic(q, k, v, P, causal)
+    o2, d2 = O.attn_recurrent(q, k, v, P, causal)
+    np.testing.assert_allclose(o1, o2, rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(d1, d2, rtol=1e-11)
+
+
+def test_rows_variant_equals_full():
+    q, k, v = _small(4, L=50)
+    P = O.sketch_params(D=16, R=2, m=8, seed=6, eps=1e-6)
+    rows = np.array([0, 3, 17, 49])
+    for causal in (True, False):
+        o, d = O.attn_quadratic(q, k, v, P, causal)
+        orow, drow = O.attn_quadratic_rows(q, k, v, P, causal, rows)
+        np.testing.assert_allclose(orow, o[:, :, rows], rtol=1e-13, atol=1e-15)
+        np.testing.assert_allclose(drow, d[:, :, rows], rtol=1e-13)
+
+
+def test_uniform_keys_closed_form():
+    # All keys equal: a_ij = a_i for every j, so the causal output is the running mean
+    # of v scaled by (i+1) a_i / ((i+1) a_i + eps).
+    L, D, Dv, eps = 20, 16, 5, 1e-3
+    rng = np.random.default_rng(8)
+    q = rng.standard_normal((1, 1, L, D))
+    k = np.repeat(rng.standard_normal((1, 1, 1, D)), L, axis=2)
+    v = rng.standard_normal((1, 1, L, Dv))
+    P = O.sketch_params(D=D, R=2, m=4, seed=9, eps=eps)
+    out, den = O.attn_quadratic(q, k, v, P, True)
+    a = (O.feature_map(q[0, 0], P) @ O.feature_map(k[0, 0, :1], P).T)[:, 0]
+    for i in range(L):
+        n = i + 1
+        want = v[0, 0, :n].mean(axis=0) * (n * a[i]) / (n * a[i] + eps)
+        np.testing.assert_allclose(out[0, 0, i], want, rtol=1e-12)
+        assert den[0, 0, i] == pytest.approx(n * a[i], rel=1e-12)
+
+
+def test_single_token_closed_form():
+    D, Dv, eps = 8, 3, 0.05
+    rng = np.random.default_rng(10)
+    q = rng.standard_normal((1, 1, 1, D))
+    k = rng.standard_normal((1, 1, 1, D))
+    v = rng.standard_normal((1, 1, 1, Dv))
+    P = O.sketch_params(D=D, R=2, m=4, seed=1, eps=eps)
+    a = float(O.feature_map(q[0, 0], P)[0] @ O.feature_map(k[0, 0], P)[0])
+    for causal in (True, False):
+        out, den = O.attn_quadratic(q, k, v, P, causal)
+        np.testing.assert_allclose(out[0, 0, 0], v[0, 0, 0] * a / (a + eps), rtol=1e-13)
+
+
+def test_weights_nonnegative_and_sum_to_one():
+    # With v = identity (Dv = L) output row i is the weight vector alpha_i.
+    L, D = 24, 8
+    rng = np.random.default_rng(12)
+    q = rng.standard_normal((1, 1, L, D))
+    k = rng.standard_normal((1, 1, L, D))
+    v = np.eye(L)[None, None]
+    P = O.sketch_params(D=D, R=3, m=6, seed=2, eps=1e-6)
+    for causal in (True, False):
+        out, den = O.attn_quadratic(q, k, v, P, causal)
+        W = out[0, 0]
+        assert (W >= 0).all()
+        if causal:
+            assert (np.triu(W, 1) == 0).all()
+            assert (np.diag(W) > 0).all()
+        np.testing.assert_allclose(W.sum(axis=1), den[0, 0] / (den[0, 0] + 1e-6), rtol=1e-12)
+        assert (np.abs(W.sum(axis=1) - 1) < 1e-4).all()
+
+
+def test_bidir_last_row_and_permutation():
+    q, k, v = _small(13, B=1, H=1, L=30)
+    P = O.sketch_params(D=16, R=2, m=8, seed=4, eps=1e-6)
+    oc, _ = O.attn_quadratic(q, k, v, P, True)
+    ob, _ = O.attn_quadratic(q, k, v, P, False)
+    np.testing.assert_allclose(ob[0, 0, -1], oc[0, 0, -1], rtol=1e-12)
+    perm = np.random.default_rng(0).permutation(30)
+    op, _ = O.attn_quadratic(q, k[:, :, perm], v[:, :, perm], P, False)
+    np.testing.assert_allclose(op, ob, rtol=1e-11)
+    assert not np.allclose(oc[0, 0, :-1], ob[0, 0, :-1])
+
+
+# ------------------------------------------------------------------ decode
+
+def test_decode_chain_reproduces_causal_and_resumes():
+    q, k, v = _small(14, B=2, H=3, L=25)
+    P = O.sketch_params(D=16, R=2, m=8, seed=7, eps=1e-6)
+    oc, _ = O.attn_quadratic(q, k, v, P, True)
+    S = np.zeros((2, 3, P.F, 8))
+    z = np.zeros((2, 3, P.F))
+    ckpt = None
+    for i in range(25):
+        out, S, z = O.decode_step(q[:, :, i], k[:, :, i], v[:, :, i], S, z, P)
+        np.testing.assert_allclose(out, oc[:, :, i], rtol=1e-11, atol=1e-14)
+        if i == 11:
+            ckpt = (S.copy(), z.copy())
+    S2, z2 = ckpt
+    for i in range(12, 25):
+        out, S2, z2 = O.decode_step(q[:, :, i], k[:, :, i], v[:, :, i], S2, z2, P)
+    np.testing.assert_array_equal(S2, S)
+    np.testing.assert_array_equal(z2, z)
+
+
+# ---------------------------------------------------------------- backward
+
+def test_backward_matches_finite_differences():
+    B, H, L, D, Dv = 1, 1, 9, 6, 4
+    rng = np.random.default_rng(15)
+    q = rng.standard_normal((B, H, L, D))
+    k = rng.standard_normal((B, H, L, D))
+    v = rng.standard_normal((B, H, L, Dv))
+    g = rng.standard_normal((B, H, L, Dv))
+    P = O.sketch_params(D=D, R=2, m=3, seed=8, eps=1e-3)
+
+    def loss(q_, k_, v_):
+        out, _ = O.attn_quadratic(q_, k_, v_, P, True)
+        return float(np.sum(out * g))
+
+    dq, dk, dv = O.attn_causal_bwd(q, k, v, g, P)
+    h = 1e-6
+    for name, x, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        fd = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp = x.copy(); xp[idx] += h
+            xm = x.copy(); xm[idx] -= h
+            args_p = {"q": q, "k": k, "v": v}; args_p[name] = xp
+            args_m = {"q": q, "k": k, "v": v}; args_m[name] = xm
+            fd[idx] = (loss(**{a + "_": b for a, b in args_p.items()}) -
+                       loss(**{a + "_": b for a, b in args_m.items()})) / (2 * h)
+        err = np.linalg.norm(fd - grad) / np.linalg.norm(fd)
+        assert err < 1e-7, (name, err)
+
+
+def test_backward_rows_variant_equals_full():
+    q, k, v = _small(16, B=1, H=2, L=21, D=8, Dv=4)
+    g = np.random.default_rng(17).standard_normal(v.shape)
+    P = O.sketch_params(D=8, R=2, m=5, seed=9, eps=1e-6)
+    dq, dk, dv = O.attn_causal_bwd(q, k, v, g, P)
+    rows = np.array([0, 5, 20])
+    rq, rk, rv = O.attn_causal_bwd_rows(q, k, v, g, P, rows)
+    np.testing.assert_allclose(rq, dq[:, :, rows], rtol=1e-10, atol=1e-14)
+    np.testing.assert_allclose(rk, dk[:, :, rows], rtol=1e-10, atol=1e-14)
+    np.testing.assert_allclose(rv, dv[:, :, rows], rtol=1e-10, atol=1e-14)
