@@ -1,0 +1,440 @@
+#!/usr/bin/env python
+"""Benchmark of the SLAY causal forward (spherical Yat-kernel linear attention) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload causal_16k|causal_2k|bidir_vision|fwd_8k|bwd_8k|decode|feature_map]
+
+One step = one pass of the whole forward path (feature map of q and k, causal contraction,
+normalisation) over one batch of synthetic inputs already resident in HBM.  Default
+workload: B=1, H=16, L=16384, D=Dv=64, R=4 nodes, m=64 features per node (F=256), bf16
+inputs, fp32 state.  Multi-GPU (torchrun): every rank runs its own batch (weak scaling,
+no collective on the data path); the timed region is bracketed by barriers and the
+reported time is the max over ranks.
+
+Prints one JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle (the only
+reference this method has) on the host cores instead.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from kernelized_linear_attention_unit_b200 import workloads as W  # noqa: E402
+
+METRIC = "SLAY causal fwd tokens/s at L=16k on 1 B200; % of tensor-core/HBM roofline"
+
+WORKLOADS = {
+    "causal_16k": (W.CAUSAL_16K, "causal"),
+    "causal_2k": (W.CAUSAL_2K, "causal"),
+    "bidir_vision": (W.BIDIR_VISION, "bidir"),
+    "fwd_8k": (W.FWDBWD_8K, "causal"),
+    "bwd_8k": (W.FWDBWD_8K, "bwd"),
+    "decode": (W.DECODE, "decode"),
+    "feature_map": (W.CAUSAL_16K, "feature_map"),
+}
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+L2_FLUSH_BYTES = 256 << 20
+C_CHUNK = 64
+
+
+# ----------------------------------------------------------------- helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def alu_peak_tflops(sm_mhz):
+    # FP32 FFMA: 148 SMs x 128 lanes x 2 flop per clock
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+def kernel_work(name, w, op):
+    """Algorithmic work of one launch of kernel `name`: (amount, unit, bound).
+
+    Per-unit figures (token-head = one row of one (b, h) slice; D = Dv = 64):
+      feature map     bytes: x read (2 B/elem) + phi written in its own dtype
+      causal fwd      flop: 8DF + 4F Dv + (C+1)(F+Dv) per token-head, C = 64
+      bidir fwd       flop: 8DF + 4F Dv per token-head
+    """
+    D, Dv, F = w.D, w.Dv, w.F
+    th = w.B * w.H * w.L                    # token-heads in the batch
+    if name in ("tc_causal_out",):
+        return th * (8 * D * F + 4 * F * Dv + (C_CHUNK + 1) * (F + Dv)), "flop", "tensor"
+    if name in ("tc_causal_state",):
+        return th * (4 * D * F + 2 * F * Dv), "flop", "tensor"
+    if name in ("tc_bidir_out",):
+        return th * (4 * D * F + 2 * F * Dv), "flop", "tensor"
+    if name in ("tc_bidir_state",):
+        return th * (4 * D * F + 2 * F * Dv), "flop", "tensor"
+    if name == "tc_feature_map":
+        return th * (D * 2 + F * 2), "byte", "hbm"
+    if name == "simt_feature_map":
+        return th * (D * 2 + F * 4), "byte", "hbm"
+    if name == "simt_chunk_state":
+        return th * 2 * F * (Dv + 1), "flop", "alu"
+    if name == "simt_chunk_out":
+        if op == "bidir":
+            return th * 2 * F * (Dv + 1), "flop", "alu"
+        return th * ((C_CHUNK + 1) * (F + Dv + 1) + 2 * F * (Dv + 1)), "flop", "alu"
+    if name == "simt_scan":
+        nc = (w.L + C_CHUNK - 1) // C_CHUNK
+        return w.B * w.H * nc * F * (Dv + 1) * 4 * 2, "byte", "hbm"
+    if name == "simt_decode":
+        per = F * Dv * 4 * 2 + F * 4 * 2 + (2 * D + 2 * Dv) * 2
+        return w.B * w.H * per, "byte", "hbm"
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while the GPU is loaded."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="slay_clk_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    rows.append((float(parts[2]), float(parts[3]), parts[6:10]))
+                except ValueError:
+                    continue
+        os.remove(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, flags in rows for i, f in enumerate(flags)
+                          if f.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------ CPU oracle leg
+
+def oracle_sample(w, op, max_heads):
+    """Time the fp64 oracle's O(L) form on `h` full-length (b, h) slices.
+
+    Returns (seconds, token-equivalents processed, threads, description)."""
+    import oracle as O
+    P = O.sketch_params(w.D, w.R, w.m, w.sketch_seed, float(np.float32(w.eps)))
+    threads = O.num_threads()
+    if op == "decode":
+        n = min(w.B * w.H, max(64, 16 * threads))
+        q, k, v, S, z = W.gen_decode(w, Bt=1, H=n)
+        t0 = time.perf_counter()
+        O.decode_step(q, k, v, S, z, P)
+        dt = time.perf_counter() - t0
+        return dt, n, threads, "%d of %d (b,h) decode states" % (n, w.B * w.H)
+    h = max(1, min(w.H, max_heads))
+    q, k, v = W.gen_qkv(w, B=1, H=h)
+    t0 = time.perf_counter()
+    if op == "feature_map":
+        O.feature_map(q, P)
+        O.feature_map(k, P)
+    else:
+        O.attn_recurrent(q, k, v, P, op != "bidir")
+    dt = time.perf_counter() - t0
+    tokens = h / w.H * w.L          # token-equivalents (a token carries H heads)
+    return dt, tokens, threads, "%d of %d heads of one sequence at L=%d, O(L) fp64 form" % (
+        h, w.H, w.L)
+
+
+def run_reference(args, w, op):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cores = os.cpu_count() or 1
+    max_heads = max(1, min(w.H, cores))
+    times, units = [], 0.0
+    for i in range(args.warmup + args.steps):
+        dt, u, threads, desc = oracle_sample(w, op, max_heads if i else 1)
+        if i >= args.warmup:
+            times.append(dt)
+            units += u
+    val = units / sum(times)
+    unit = "tokens/s" if op != "decode" else "decode-steps/s"
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": unit,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w, op),
+            "cpu_baseline": {"value": val, "unit": unit, "cores": threads, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w, op):
+    return {"workload": w.name if op not in ("bwd", "feature_map") else "%s_%s" % (w.name, op),
+            "B": w.B, "H": w.H, "L": w.L, "D": w.D, "Dv": w.Dv, "R": w.R, "m": w.m, "F": w.F,
+            "op": op, "eps": w.eps, "sketch_seed": w.sketch_seed,
+            "l2": "flushed between timed steps (256 MiB write outside the timed events)"}
+
+
+# ----------------------------------------------------------------- GPU leg
+
+def run_ours(args, w, op):
+    import torch
+    import torch.distributed as dist
+    from kernelized_linear_attention_unit_b200 import binding as bd
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    eps = float(np.float32(w.eps))
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    def to_dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev).to(tdt)
+
+    def pinned(t):
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t)
+        return h
+
+    # inputs: each rank draws its own batch (data seed offset by rank)
+    wr = W.Workload(**{**w.__dict__, "data_seed": w.data_seed + 1000 * rank})
+    if op == "decode":
+        qn, kn, vn, Sn, zn = W.gen_decode(wr)
+        q, k, v = to_dev(qn), to_dev(kn), to_dev(vn)
+        S = torch.from_numpy(Sn).to(dev)
+        z = torch.from_numpy(zn).to(dev)
+        out = torch.empty(v.shape, device=dev, dtype=tdt)
+        host_in = [pinned(x.cpu()) for x in (q, k, v)]
+        dev_in = [q, k, v]
+
+        def step():
+            bd.slay_decode_step(q, k, v, S, z, out, w.R, w.m, w.sketch_seed, eps)
+        units_per_step = w.B * w.H
+        unit = "decode-steps/s"
+    elif op == "feature_map":
+        qn, kn, _ = W.gen_qkv(wr)
+        x = to_dev(np.concatenate([qn.reshape(-1, w.D), kn.reshape(-1, w.D)]))
+        out = torch.empty((x.shape[0], w.F), device=dev, dtype=tdt)
+        host_in, dev_in = [pinned(x.cpu())], [x]
+
+        def step():
+            bd.slay_feature_map(x, out, w.R, w.m, w.sketch_seed, eps)
+        units_per_step = w.B * w.L
+        unit = "tokens/s"
+    else:
+        qn, kn, vn = W.gen_qkv(wr)
+        q, k, v = to_dev(qn), to_dev(kn), to_dev(vn)
+        out = torch.empty(v.shape, device=dev, dtype=tdt)
+        den = torch.empty(v.shape[:-1], device=dev, dtype=torch.float32)
+        host_in, dev_in = [pinned(x.cpu()) for x in (q, k, v)], [q, k, v]
+        if op == "bwd":
+            g = to_dev(W.gen_dout(wr))
+            ws = bd.alloc_workspace(bd.OP_CAUSAL_BWD, tdt, w.B, w.H, w.L, w.D, w.Dv, w.R, w.m, dev)
+            wsf = bd.alloc_workspace(bd.OP_CAUSAL_FWD, tdt, w.B, w.H, w.L, w.D, w.Dv, w.R, w.m, dev)
+            bd.slay_attn_causal_fwd(q, k, v, out, den, w.R, w.m, w.sketch_seed, eps, wsf)
+            dq = torch.empty(q.shape, device=dev, dtype=torch.float32)
+            dk = torch.empty_like(dq)
+            dv = torch.empty(v.shape, device=dev, dtype=torch.float32)
+            host_in.append(pinned(g.cpu()))
+            dev_in.append(g)
+
+            def step():
+                bd.slay_attn_causal_bwd(q, k, v, out, den, g, dq, dk, dv, w.R, w.m,
+                                        w.sketch_seed, eps, ws)
+        else:
+            opc = bd.OP_BIDIR_FWD if op == "bidir" else bd.OP_CAUSAL_FWD
+            ws = bd.alloc_workspace(opc, tdt, w.B, w.H, w.L, w.D, w.Dv, w.R, w.m, dev)
+            fn = bd.slay_attn_bidir_fwd if op == "bidir" else bd.slay_attn_causal_fwd
+
+            def step():
+                fn(q, k, v, out, den, w.R, w.m, w.sketch_seed, eps, ws)
+        units_per_step = w.B * w.L
+        unit = "tokens/s"
+    result = dq if op == "bwd" else out
+    host_out = torch.empty(result.shape, dtype=result.dtype, pin_memory=True)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    bd.slay_prepare(w.D, w.R, w.m, w.sketch_seed, eps)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- device-timed region: inputs resident in HBM, L2 flushed between steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clk = ClockSampler(local)
+    clk.start()
+    time.sleep(0.3)
+    bd.slay_trace_enable(True)
+    bd.slay_trace_read()
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    bd.slay_trace_enable(False)
+    trace = bd.slay_trace_read()
+    clocks = clk.stop()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    value = world * units_per_step * args.steps / (total_ms / 1e3)
+
+    # ---- end to end through the same public call: H2D of inputs, the call, D2H of result
+    h2d = sum(x.numel() * x.element_size() for x in host_in)
+    d2h = host_out.numel() * host_out.element_size()
+    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        e_starts[i].record(stream)
+        for hsrc, dtgt in zip(host_in, dev_in):
+            dtgt.copy_(hsrc, non_blocking=True)
+        step()
+        host_out.copy_(result, non_blocking=True)
+        e_ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends))
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = world * units_per_step * args.steps / (e2e_ms / 1e3)
+
+    # ---- roofline of the dominant kernel (largest total device time in the timed region)
+    peaks, peak_src = load_peaks()
+    per = {}
+    for name, ms in trace:
+        per.setdefault(name, []).append(ms)
+    roofline = None
+    kernels = {n: {"launches": len(v), "total_ms": sum(v), "avg_us": 1e3 * sum(v) / len(v)}
+               for n, v in per.items()}
+    if per:
+        dom = max(per, key=lambda n: sum(per[n]))
+        avg_s = sum(per[dom]) / len(per[dom]) / 1e3
+        wk = kernel_work(dom, w, op)
+        if wk is not None:
+            amount, kind, bound = wk
+            if bound == "hbm":
+                achieved, peak, u = amount / avg_s / 1e9, peaks["hbm_gbs"], "GB/s"
+            elif bound == "tensor":
+                achieved, peak, u = amount / avg_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+            else:
+                achieved = amount / avg_s / 1e12
+                peak = alu_peak_tflops(peaks.get("sm_max_mhz", 1965.0))
+                u = "TFLOP/s"
+            roofline = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak,
+                        "unit": u, "frac": achieved / peak, "traffic": None,
+                        "peak_source": peak_src + (" (fp32 FFMA: 148 SMs x 128 x 2 x max clock)"
+                                                   if bound == "alu" else ""),
+                        "algorithmic_%s_per_launch" % kind: amount,
+                        "avg_launch_us": avg_s * 1e6}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cores = os.cpu_count() or 1
+        dt, u, threads, desc = oracle_sample(w, op, max(1, min(w.H, cores)))
+        cpu = {"value": u / dt, "unit": unit, "cores": threads, "kind": "oracle", "sample": desc,
+               "seconds": dt}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+                "config": config_of(w, op),
+                "e2e": {"value": e2e, "unit": unit, "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h},
+                "gpu_launches": len(trace),
+                "roofline": roofline, "kernels": kernels, "clocks": clocks,
+                "cpu_baseline": cpu}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="causal_16k", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    w, op = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w, op)
+    return run_ours(args, w, op)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

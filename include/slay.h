@@ -1,0 +1,167 @@
+/*
+ * slay.h -- C ABI of libslay.so: SLAY spherical Yat-kernel linear attention on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method ("SLAY: Geometry-Aware Spherical Linearized Attention with Yat-Kernel",
+ * arXiv 2602.04915; abstract, and the nubint.ai review, section "Proposed method"):
+ *   x^ = x / max(|x|, 1e-12)                           (queries/keys on the sphere)
+ *   K(q,k) = x^2 / (2 - 2x + eps), x = q^ . k^         (spherical Yat kernel)
+ *   1/(2-2x+eps) = int e^{-s(2+eps)} e^{2sx} ds         (Bernstein / Laplace)
+ *   R-node Gauss-Laguerre rule (t_r, w_r) after t=(2+eps)s:
+ *       s_r = t_r/(2+eps), wt_r = w_r/(2+eps)
+ *   phi_{r*m+j}(x) = sqrt(wt_r/m) exp(sqrt(2 s_r) omega_{rj}.x^ - s_r) (a_{rj}.x^)^2
+ *       (positive random feature x anchor feature, fused by an elementwise sketch)
+ *   out_i = phi(q_i)^T S_i / (phi(q_i)^T z_i + eps),
+ *       S_i = sum_{j in J(i)} phi(k_j) v_j^T, z_i = sum_{j in J(i)} phi(k_j)
+ *   with J(i) = {j <= i} (causal) or all j (bidirectional).  F = R*m features.
+ *
+ * Sketch parameters: omega_{f,d} ~ N(0,1), a_{f,d} ~ N(0,1)/sqrt(D), f = r*m+j, drawn
+ * from `seed` with Philox4x32-10 (Salmon et al., SC'11): counter (f*D+d, tag, 0, 0),
+ * tag 0 for omega and 1 for anchors, key (seed & 0xffffffff, seed >> 32); one normal
+ * per counter by Box-Muller on the first two words mapped to (0,1) as (w + 1/2) 2^-32,
+ * computed in double and rounded to float.  The same draw serves q and k and every
+ * batch and head.
+ *
+ * Conventions for every entry point:
+ *   - Device pointers are caller-owned CUDA device memory; the library never frees or
+ *     keeps them.  Tensors are contiguous row-major: [B,H,L,D] has D innermost.
+ *     Every tensor base must be 16-byte aligned; `workspace` must be 256-byte aligned.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous on it: a returned SLAY_OK means the work was enqueued.
+ *   - dtype SLAY_F32: inputs/outputs fp32, all arithmetic fp32 on CUDA cores.
+ *     dtype SLAY_BF16: q,k,v,out (and dout) bf16; arithmetic with fp32 accumulation,
+ *     states S and z always fp32; gradients fp32.
+ *   - Supported: D == Dv == 64, 1 <= R <= 16, 1 <= m, F = R*m <= 1024 (F % 16 == 0 on
+ *     the bf16 tensor-core path; other F run on CUDA cores), eps > 0 and finite.
+ *   - Errors are status codes, never exceptions or aborts.  On any error nothing is
+ *     enqueued.  The library owns only its sketch-parameter cache: one small device
+ *     buffer per (device, D, R, m, seed, eps), created on first use (synchronous
+ *     allocation and upload; call slay_prepare before capturing a stream into a CUDA
+ *     graph) and held until the process exits.  The cache is thread-safe.
+ *   - Empty work (L == 0, n_rows == 0, B*H == 0) returns SLAY_OK and enqueues nothing.
+ */
+#ifndef SLAY_H
+#define SLAY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SLAY_OK = 0,
+    SLAY_ERR_INVALID_ARG = 1,   /* NULL pointer, misalignment, bad size, workspace too small */
+    SLAY_ERR_UNSUPPORTED = 2,   /* a size or dtype combination this build does not offer */
+    SLAY_ERR_CUDA = 3,          /* a CUDA runtime error (launch, allocation of the cache, no device) */
+    SLAY_ERR_TIMEOUT = 4,       /* reserved: no kernel of this library waits on another CTA */
+    SLAY_ERR_NO_MEMORY = 5      /* host allocation failed */
+} slay_status;
+
+typedef enum { SLAY_F32 = 0, SLAY_BF16 = 1 } slay_dtype;
+
+typedef enum {
+    SLAY_OP_FEATURE_MAP = 0,
+    SLAY_OP_CAUSAL_FWD = 1,
+    SLAY_OP_BIDIR_FWD = 2,
+    SLAY_OP_CAUSAL_BWD = 3,
+    SLAY_OP_DECODE = 4
+} slay_op;
+
+/* Feature map phi (review, "Proposed method", steps 1, 3, 4, 5).
+ * x   : device [n_rows, D] in `in_dt` (rows need not be unit length; they are
+ *       projected onto the sphere inside, a zero row maps to phi = 0).
+ * phi : device [n_rows, R*m] in `out_dt`, written; feature index f = r*m + j.
+ * in_dt/out_dt: (F32,F32), (BF16,BF16) or (BF16,F32).  No workspace. */
+slay_status slay_feature_map(const void* x, void* phi, int64_t n_rows, int D,
+                             slay_dtype in_dt, slay_dtype out_dt, int R, int m,
+                             uint64_t seed, float eps, void* stream);
+
+/* Causal SLAY attention forward (review, "Proposed method", step 6: the linear
+ * contraction with prefix states, no LxL matrix; abstract: O(L) time and memory).
+ * q,k : device [B,H,L,D], v : device [B,H,L,Dv], all in `dt`.
+ * out : device [B,H,L,Dv] in `dt`, written.
+ * den : device [B,H,L] fp32 or NULL; if given, den_i = phi(q_i)^T z_i (without eps)
+ *       is written (the backward needs it).
+ * workspace/ws_bytes: device scratch of at least
+ *       slay_workspace_bytes(SLAY_OP_CAUSAL_FWD, dt, B, H, L, D, Dv, R, m) bytes;
+ *       its contents on entry are ignored and on exit undefined. */
+slay_status slay_attn_causal_fwd(const void* q, const void* k, const void* v, void* out,
+                                 float* den, int B, int H, int L, int D, int Dv,
+                                 slay_dtype dt, int R, int m, uint64_t seed, float eps,
+                                 void* workspace, size_t ws_bytes, void* stream);
+
+/* Bidirectional SLAY attention forward: as above with S, z summed over all keys
+ * (review, "Proposed method", step 6, non-causal form).  Same arguments; workspace
+ * size from slay_workspace_bytes(SLAY_OP_BIDIR_FWD, ...). */
+slay_status slay_attn_bidir_fwd(const void* q, const void* k, const void* v, void* out,
+                                float* den, int B, int H, int L, int D, int Dv,
+                                slay_dtype dt, int R, int m, uint64_t seed, float eps,
+                                void* workspace, size_t ws_bytes, void* stream);
+
+/* Backward of the causal forward: gradients of sum_i <dout_i, out_i> with respect to
+ * q, k, v, through the contraction, the normaliser, phi and the sphere projection.
+ * The pages give no backward; it is the derivative of the forward above.  omega and
+ * anchors are fixed random draws and get no gradient.
+ * out, den : the forward's outputs for the same inputs (out in `dt`, den fp32).
+ * dout     : device [B,H,L,Dv] in `dt`.
+ * dq, dk   : device [B,H,L,D] fp32, dv : device [B,H,L,Dv] fp32, all written.
+ * workspace: slay_workspace_bytes(SLAY_OP_CAUSAL_BWD, ...) bytes. */
+slay_status slay_attn_causal_bwd(const void* q, const void* k, const void* v,
+                                 const void* out, const float* den, const void* dout,
+                                 float* dq, float* dk, float* dv,
+                                 int B, int H, int L, int D, int Dv,
+                                 slay_dtype dt, int R, int m, uint64_t seed, float eps,
+                                 void* workspace, size_t ws_bytes, void* stream);
+
+/* One recurrent decode step for Bt*H independent sequences (abstract: linear time
+ * and memory; the O(1)-per-token form of the causal contraction), inclusive:
+ *   S += phi(k) v^T;  z += phi(k);  out = phi(q)^T S / (phi(q)^T z + eps)
+ * q,k : device [Bt,H,D], v : device [Bt,H,Dv] in `dt`; out : device [Bt,H,Dv] in `dt`.
+ * S   : device [Bt,H,F,Dv] fp32, z : device [Bt,H,F] fp32, updated in place
+ *       (caller-owned; a checkpoint is a copy of S, z and the key (D,R,m,seed,eps)).
+ * No workspace. */
+slay_status slay_decode_step(const void* q, const void* k, const void* v,
+                             float* S, float* z, void* out,
+                             int Bt, int H, int D, int Dv, slay_dtype dt,
+                             int R, int m, uint64_t seed, float eps, void* stream);
+
+/* Workspace bytes an entry point needs for these sizes (0 if none; SIZE_MAX if the
+ * sizes are unsupported).  Feature map and decode need none. */
+size_t slay_workspace_bytes(slay_op op, slay_dtype dt, int B, int H, int L, int D, int Dv,
+                            int R, int m);
+
+/* Create (if absent) the device copy of the sketch parameters of this key on the
+ * current device: synchronous; lets a caller warm the cache before stream capture. */
+slay_status slay_prepare(int D, int R, int m, uint64_t seed, float eps);
+
+/* Host copy of the sketch parameters the kernels use, for tests and checkpoints:
+ * omega_host, anchors_host [R*m, D] float (each may be NULL), s_host, w_host [R] double
+ * (each may be NULL): s_r = t_r/(2+eps), w_host[r] = wt_r = w_r/(2+eps).  Host only:
+ * needs no GPU. */
+slay_status slay_sketch_params(int D, int R, int m, uint64_t seed, float eps,
+                               float* omega_host, float* anchors_host,
+                               double* s_host, double* w_host);
+
+/* Per-launch timing for profiling: while enabled (on != 0), every kernel this library
+ * launches is bracketed by a pair of CUDA events recorded on its stream.  Host-side
+ * bookkeeping only; results are unchanged.  Not for use during stream capture. */
+slay_status slay_trace_enable(int on);
+
+/* Waits for the recorded events, writes up to `cap` records (kernel name: a static
+ * string owned by the library; duration in milliseconds, -1 if unavailable) into
+ * names[] / ms[] (either may be NULL), clears the record list and returns the number of
+ * records that were pending (which may exceed cap). */
+int slay_trace_read(const char** names, float* ms, int cap);
+
+/* Static description of a status code. */
+const char* slay_status_string(slay_status st);
+
+/* Text of the last CUDA error seen by this thread inside the library ("" if none). */
+const char* slay_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SLAY_H */

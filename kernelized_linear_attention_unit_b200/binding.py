@@ -1,0 +1,238 @@
+"""Thin ctypes binding of libslay.so (the C ABI declared in include/slay.h).
+
+Argument marshalling only: each function checks the torch tensors it is given
+(device, dtype, contiguity, shape), passes their device pointers and the current CUDA
+stream to the C entry point of the same name, and raises SlayError on a non-zero
+status.  Every step of the computation runs in the library's CUDA kernels; there is no
+Python or CPU fallback, and the first call raises if the library is missing.
+"""
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libslay.so")
+
+SLAY_OK, SLAY_ERR_INVALID_ARG, SLAY_ERR_UNSUPPORTED, SLAY_ERR_CUDA, SLAY_ERR_TIMEOUT, \
+    SLAY_ERR_NO_MEMORY = range(6)
+SLAY_F32, SLAY_BF16 = 0, 1
+OP_FEATURE_MAP, OP_CAUSAL_FWD, OP_BIDIR_FWD, OP_CAUSAL_BWD, OP_DECODE = range(5)
+
+EXPORTS = ["slay_feature_map", "slay_attn_causal_fwd", "slay_attn_bidir_fwd",
+           "slay_attn_causal_bwd", "slay_decode_step", "slay_workspace_bytes", "slay_prepare",
+           "slay_sketch_params", "slay_status_string", "slay_last_error", "slay_trace_enable",
+           "slay_trace_read"]
+
+
+class SlayError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        msg = "%s: %s" % (where, lib().slay_status_string(status).decode())
+        detail = lib().slay_last_error().decode()
+        if status == SLAY_ERR_CUDA and detail:
+            msg += " (%s)" % detail
+        super().__init__(msg)
+
+
+_lib = None
+
+
+def lib():
+    """Load libslay.so once; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError("libslay.so not found at %s: build it with "
+                           "`python -m kernelized_linear_attention_unit_b200.build`" % LIB_PATH)
+    L = C.CDLL(LIB_PATH)
+    vp, i32, i64, u64, f32, sz = C.c_void_p, C.c_int, C.c_int64, C.c_uint64, C.c_float, C.c_size_t
+    L.slay_feature_map.argtypes = [vp, vp, i64, i32, i32, i32, i32, i32, u64, f32, vp]
+    attn = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, u64, f32, vp, sz, vp]
+    L.slay_attn_causal_fwd.argtypes = attn
+    L.slay_attn_bidir_fwd.argtypes = attn
+    L.slay_attn_causal_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
+                                       i32, i32, i32, i32, u64, f32, vp, sz, vp]
+    L.slay_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                   u64, f32, vp]
+    L.slay_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32]
+    L.slay_workspace_bytes.restype = sz
+    L.slay_prepare.argtypes = [i32, i32, i32, u64, f32]
+    L.slay_sketch_params.argtypes = [i32, i32, i32, u64, f32, vp, vp, vp, vp]
+    L.slay_status_string.argtypes = [i32]
+    L.slay_status_string.restype = C.c_char_p
+    L.slay_last_error.argtypes = []
+    L.slay_last_error.restype = C.c_char_p
+    L.slay_trace_enable.argtypes = [i32]
+    L.slay_trace_enable.restype = i32
+    L.slay_trace_read.argtypes = [C.POINTER(C.c_char_p), C.POINTER(C.c_float), i32]
+    L.slay_trace_read.restype = i32
+    for name in ("slay_feature_map", "slay_attn_causal_fwd", "slay_attn_bidir_fwd",
+                 "slay_attn_causal_bwd", "slay_decode_step", "slay_prepare",
+                 "slay_sketch_params"):
+        getattr(L, name).restype = i32
+    _lib = L
+    return _lib
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return SLAY_F32
+    if t.dtype == torch.bfloat16:
+        return SLAY_BF16
+    raise TypeError("dtype %s not supported (float32 or bfloat16)" % t.dtype)
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _check(t, name, dtype=None, shape=None):
+    if t is None:
+        raise ValueError("%s is required" % name)
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), tuple(shape)))
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return C.c_void_p(s.cuda_stream)
+
+
+def _raise(status, where):
+    if status != SLAY_OK:
+        raise SlayError(status, where)
+
+
+def slay_workspace_bytes(op, dtype, B, H, L, D, Dv, R, m) -> int:
+    dt = dtype if isinstance(dtype, int) else _dt(torch.empty(0, dtype=dtype))
+    n = lib().slay_workspace_bytes(op, dt, B, H, L, D, Dv, R, m)
+    if n == C.c_size_t(-1).value:
+        raise SlayError(SLAY_ERR_UNSUPPORTED, "slay_workspace_bytes")
+    return int(n)
+
+
+def alloc_workspace(op, dtype, B, H, L, D, Dv, R, m, device=None):
+    """Caller-owned workspace of the size the library asks for (torch allocation)."""
+    n = slay_workspace_bytes(op, dtype, B, H, L, D, Dv, R, m)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def slay_prepare(D, R, m, seed, eps):
+    _raise(lib().slay_prepare(D, R, m, seed, eps), "slay_prepare")
+
+
+def slay_sketch_params(D, R, m, seed, eps):
+    """Host copy of (omega [F,D] f32, anchors [F,D] f32, s [R] f64, wt [R] f64)."""
+    import numpy as np
+    F = R * m
+    om = np.zeros((F, D), dtype=np.float32)
+    an = np.zeros((F, D), dtype=np.float32)
+    s = np.zeros(R, dtype=np.float64)
+    w = np.zeros(R, dtype=np.float64)
+    _raise(lib().slay_sketch_params(D, R, m, seed, eps, om.ctypes.data, an.ctypes.data,
+                                    s.ctypes.data, w.ctypes.data), "slay_sketch_params")
+    return om, an, s, w
+
+
+def slay_trace_enable(on: bool):
+    _raise(lib().slay_trace_enable(1 if on else 0), "slay_trace_enable")
+
+
+def slay_trace_read(cap: int = 1 << 16):
+    """List of (kernel name, milliseconds) for the launches recorded since the last read."""
+    names = (C.c_char_p * cap)()
+    ms = (C.c_float * cap)()
+    n = lib().slay_trace_read(names, ms, cap)
+    return [(names[i].decode(), float(ms[i])) for i in range(min(n, cap))]
+
+
+def slay_feature_map(x, phi, R, m, seed, eps, stream=None):
+    """phi[n, R*m] = phi(x[n, D]); x f32 -> phi f32, x bf16 -> phi bf16 or f32."""
+    _check(x, "x")
+    _check(phi, "phi")
+    D = x.shape[-1]
+    n = x.numel() // D if D else 0
+    if phi.numel() != n * R * m or phi.shape[-1] != R * m:
+        raise ValueError("phi must have %d rows of %d features" % (n, R * m))
+    _raise(lib().slay_feature_map(_ptr(x), _ptr(phi), n, D, _dt(x), _dt(phi), R, m, seed, eps,
+                                  _stream(stream)), "slay_feature_map")
+
+
+def _attn(fn, name, op, q, k, v, out, den, R, m, seed, eps, workspace, stream):
+    _check(q, "q")
+    B, H, L, D = q.shape
+    Dv = v.shape[-1]
+    _check(k, "k", q.dtype, (B, H, L, D))
+    _check(v, "v", q.dtype, (B, H, L, Dv))
+    _check(out, "out", q.dtype, (B, H, L, Dv))
+    if den is not None:
+        _check(den, "den", torch.float32, (B, H, L))
+    dt = _dt(q)
+    need = slay_workspace_bytes(op, dt, B, H, L, D, Dv, R, m)
+    if workspace is None:
+        workspace = alloc_workspace(op, dt, B, H, L, D, Dv, R, m, q.device)
+    _check(workspace, "workspace")
+    wbytes = workspace.numel() * workspace.element_size()
+    if wbytes < need:
+        raise ValueError("workspace has %d bytes, %d needed" % (wbytes, need))
+    _raise(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(den), B, H, L, D, Dv, dt, R, m, seed,
+              eps, _ptr(workspace), wbytes, _stream(stream)), name)
+
+
+def slay_attn_causal_fwd(q, k, v, out, den, R, m, seed, eps, workspace=None, stream=None):
+    _attn(lib().slay_attn_causal_fwd, "slay_attn_causal_fwd", OP_CAUSAL_FWD, q, k, v, out, den,
+          R, m, seed, eps, workspace, stream)
+
+
+def slay_attn_bidir_fwd(q, k, v, out, den, R, m, seed, eps, workspace=None, stream=None):
+    _attn(lib().slay_attn_bidir_fwd, "slay_attn_bidir_fwd", OP_BIDIR_FWD, q, k, v, out, den,
+          R, m, seed, eps, workspace, stream)
+
+
+def slay_attn_causal_bwd(q, k, v, out, den, dout, dq, dk, dv, R, m, seed, eps, workspace=None,
+                         stream=None):
+    _check(q, "q")
+    B, H, L, D = q.shape
+    Dv = v.shape[-1]
+    _check(k, "k", q.dtype, (B, H, L, D))
+    _check(v, "v", q.dtype, (B, H, L, Dv))
+    _check(out, "out", q.dtype, (B, H, L, Dv))
+    _check(den, "den", torch.float32, (B, H, L))
+    _check(dout, "dout", q.dtype, (B, H, L, Dv))
+    _check(dq, "dq", torch.float32, (B, H, L, D))
+    _check(dk, "dk", torch.float32, (B, H, L, D))
+    _check(dv, "dv", torch.float32, (B, H, L, Dv))
+    dt = _dt(q)
+    need = slay_workspace_bytes(OP_CAUSAL_BWD, dt, B, H, L, D, Dv, R, m)
+    if workspace is None:
+        workspace = alloc_workspace(OP_CAUSAL_BWD, dt, B, H, L, D, Dv, R, m, q.device)
+    wbytes = workspace.numel() * workspace.element_size()
+    if wbytes < need:
+        raise ValueError("workspace has %d bytes, %d needed" % (wbytes, need))
+    _raise(lib().slay_attn_causal_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(den), _ptr(dout),
+                                      _ptr(dq), _ptr(dk), _ptr(dv), B, H, L, D, Dv, dt, R, m,
+                                      seed, eps, _ptr(workspace), wbytes, _stream(stream)),
+           "slay_attn_causal_bwd")
+
+
+def slay_decode_step(q, k, v, S, z, out, R, m, seed, eps, stream=None):
+    _check(q, "q")
+    Bt, H, D = q.shape
+    Dv = v.shape[-1]
+    F = R * m
+    _check(k, "k", q.dtype, (Bt, H, D))
+    _check(v, "v", q.dtype, (Bt, H, Dv))
+    _check(S, "S", torch.float32, (Bt, H, F, Dv))
+    _check(z, "z", torch.float32, (Bt, H, F))
+    _check(out, "out", q.dtype, (Bt, H, Dv))
+    _raise(lib().slay_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(S), _ptr(z), _ptr(out), Bt, H,
+                                  D, Dv, _dt(q), R, m, seed, eps, _stream(stream)),
+           "slay_decode_step")

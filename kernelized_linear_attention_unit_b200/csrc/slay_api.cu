@@ -1,0 +1,332 @@
+// slay_api.cu -- C ABI entry points of libslay.so: argument checks, the per-key
+// sketch-parameter cache and dispatch to the kernels.  See include/slay.h for the
+// contract of each entry point.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "slay.h"
+#include "slay_internal.h"
+#include "slay_tc.h"
+
+namespace slay {
+namespace {
+
+thread_local std::string g_last_error;
+
+slay_status cuda_fail(cudaError_t e)
+{
+    g_last_error = cudaGetErrorString(e);
+    return SLAY_ERR_CUDA;
+}
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+using Key = std::tuple<int, int, int, int, uint64_t, uint32_t>;  // device, D, R, m, seed, eps bits
+
+struct Entry {
+    void* dev = nullptr;
+    Params P{};
+};
+
+std::mutex g_mu;
+std::map<Key, Entry>& cache()
+{
+    static std::map<Key, Entry>* c = new std::map<Key, Entry>();  // held until exit
+    return *c;
+}
+
+uint32_t float_bits(float x)
+{
+    uint32_t b;
+    std::memcpy(&b, &x, sizeof b);
+    return b;
+}
+
+uint16_t to_bf16_bits(float x)
+{
+    uint32_t b = float_bits(x);
+    b += 0x7FFFu + ((b >> 16) & 1u);
+    return static_cast<uint16_t>(b >> 16);
+}
+
+// Build (or find) the device copy of the key's parameters on the current device.
+slay_status get_params(int D, int R, int m, uint64_t seed, float eps, Params* out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    const Key key{dev, D, R, m, seed, float_bits(eps)};
+    std::lock_guard<std::mutex> lock(g_mu);
+    auto it = cache().find(key);
+    if (it != cache().end()) { *out = it->second.P; return SLAY_OK; }
+
+    const int F = R * m;
+    std::vector<float> om(static_cast<size_t>(F) * D), an(static_cast<size_t>(F) * D);
+    double s[kMaxR], wt[kMaxR];
+    if (!draw_sketch(D, R, m, seed, static_cast<double>(eps), om.data(), an.data(), s, wt))
+        return SLAY_ERR_INVALID_ARG;
+    const size_t nF = static_cast<size_t>(F) * D;
+    // layout: omT | anT | om | an (fp32), then wB (bf16 tensor-core operand)
+    const size_t wb_elems = tc_wb_elems(D, R, m);
+    const size_t bytes = 4 * nF * sizeof(float) + wb_elems * sizeof(uint16_t);
+    std::vector<unsigned char> host(bytes);
+    float* h = reinterpret_cast<float*>(host.data());
+    for (int f = 0; f < F; ++f)
+        for (int d = 0; d < D; ++d) {
+            h[static_cast<size_t>(d) * F + f] = om[static_cast<size_t>(f) * D + d];
+            h[nF + static_cast<size_t>(d) * F + f] = an[static_cast<size_t>(f) * D + d];
+        }
+    std::memcpy(h + 2 * nF, om.data(), nF * sizeof(float));
+    std::memcpy(h + 3 * nF, an.data(), nF * sizeof(float));
+    uint16_t* wb = reinterpret_cast<uint16_t*>(h + 4 * nF);
+    if (wb_elems) {
+        std::vector<uint16_t> omb(nF), anb(nF);
+        for (size_t i = 0; i < nF; ++i) { omb[i] = to_bf16_bits(om[i]); anb[i] = to_bf16_bits(an[i]); }
+        tc_pack_wb(D, R, m, omb.data(), anb.data(), wb);
+    }
+
+    Entry ent;
+    e = cudaMalloc(&ent.dev, bytes);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaMemcpy(ent.dev, host.data(), bytes, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) { cudaFree(ent.dev); return cuda_fail(e); }
+    float* d = static_cast<float*>(ent.dev);
+    Params& P = ent.P;
+    P.omT = d;
+    P.anT = d + nF;
+    P.om = d + 2 * nF;
+    P.an = d + 3 * nF;
+    P.wB = wb_elems ? reinterpret_cast<const uint16_t*>(d + 4 * nF) : nullptr;
+    P.D = D; P.R = R; P.m = m; P.F = F;
+    const double log2e = 1.4426950408889634073599246810019;
+    for (int r = 0; r < kMaxR; ++r) {
+        if (r < R) {
+            const double c = std::sqrt(wt[r] / m);
+            const double sq = std::sqrt(2.0 * s[r]);
+            P.a2[r] = static_cast<float>(sq * log2e);
+            P.b2[r] = static_cast<float>(std::log2(c) - s[r] * log2e);
+            P.sq[r] = static_cast<float>(sq);
+            P.c[r] = static_cast<float>(c);
+        } else {
+            P.a2[r] = P.b2[r] = P.sq[r] = P.c[r] = 0.0f;
+        }
+    }
+    cache()[key] = ent;
+    *out = P;
+    return SLAY_OK;
+}
+
+bool eps_ok(float eps) { return std::isfinite(eps) && eps > 0.0f; }
+bool dtype_ok(slay_dtype d) { return d == SLAY_F32 || d == SLAY_BF16; }
+
+slay_status check_shape(int D, int Dv, int R, int m)
+{
+    if (D <= 0 || Dv <= 0 || R <= 0 || m <= 0) return SLAY_ERR_INVALID_ARG;
+    if (D != kD || Dv != kD) return SLAY_ERR_UNSUPPORTED;
+    if (R > kMaxR || static_cast<int64_t>(R) * m > kMaxF) return SLAY_ERR_UNSUPPORTED;
+    return SLAY_OK;
+}
+
+slay_status check_attn(const void* q, const void* k, const void* v, const void* out, int B,
+                       int H, int L, int D, int Dv, slay_dtype dt, int R, int m, float eps)
+{
+    if (B < 0 || H < 0 || L < 0) return SLAY_ERR_INVALID_ARG;
+    slay_status s = check_shape(D, Dv, R, m);
+    if (s != SLAY_OK) return s;
+    if (!dtype_ok(dt) || !eps_ok(eps)) return SLAY_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(B) * H * L == 0) return SLAY_OK;
+    if (!q || !k || !v || !out) return SLAY_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+        return SLAY_ERR_INVALID_ARG;
+    // grid limits of the launches: (b,h) and 64-token chunks index grid y/z dimensions
+    if (static_cast<int64_t>(B) * H > 65535 || (static_cast<int64_t>(L) + 63) / 64 > 65535)
+        return SLAY_ERR_UNSUPPORTED;
+    return SLAY_OK;
+}
+
+size_t attn_ws(slay_op op, slay_dtype dt, int B, int H, int L, int Dv, int R, int m)
+{
+    const int F = R * m;
+    if (dt == SLAY_BF16 && tc_supported(op, B, H, L, R, m))
+        return tc_workspace_bytes(op, B, H, L, R, m);
+    switch (op) {
+        case SLAY_OP_CAUSAL_FWD: return simt_ws_causal(B, H, L, Dv, F);
+        case SLAY_OP_BIDIR_FWD: return simt_ws_bidir(B, H, L, Dv, F);
+        case SLAY_OP_CAUSAL_BWD: return simt_ws_bwd(B, H, L, Dv, F);
+        default: return 0;
+    }
+}
+
+slay_status attn_fwd(const void* q, const void* k, const void* v, void* out, float* den, int B,
+                     int H, int L, int D, int Dv, slay_dtype dt, int R, int m, uint64_t seed,
+                     float eps, void* ws, size_t ws_bytes, void* stream, bool causal)
+{
+    slay_status s = check_attn(q, k, v, out, B, H, L, D, Dv, dt, R, m, eps);
+    if (s != SLAY_OK) return s;
+    if (static_cast<int64_t>(B) * H * L == 0) return SLAY_OK;
+    if (den && !aligned(den, 4)) return SLAY_ERR_INVALID_ARG;
+    const slay_op op = causal ? SLAY_OP_CAUSAL_FWD : SLAY_OP_BIDIR_FWD;
+    const size_t need = attn_ws(op, dt, B, H, L, Dv, R, m);
+    if (need > 0 && (!ws || ws_bytes < need || !aligned(ws, 256))) return SLAY_ERR_INVALID_ARG;
+    Params P;
+    if ((s = get_params(D, R, m, seed, eps, &P)) != SLAY_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (dt == SLAY_BF16 && tc_supported(op, B, H, L, R, m))
+        e = tc_attn_fwd(q, k, v, out, den, B, H, L, P, eps, causal, ws, st);
+    else
+        e = simt_attn_fwd(q, k, v, out, den, B, H, L, dt, P, eps, causal, ws, st);
+    return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
+}
+
+}  // namespace
+}  // namespace slay
+
+using namespace slay;
+
+extern "C" {
+
+slay_status slay_feature_map(const void* x, void* phi, int64_t n_rows, int D, slay_dtype in_dt,
+                             slay_dtype out_dt, int R, int m, uint64_t seed, float eps,
+                             void* stream)
+{
+    if (n_rows < 0) return SLAY_ERR_INVALID_ARG;
+    slay_status s = check_shape(D, kD, R, m);
+    if (s != SLAY_OK) return s;
+    if (!dtype_ok(in_dt) || !dtype_ok(out_dt) || !eps_ok(eps)) return SLAY_ERR_INVALID_ARG;
+    if (in_dt == SLAY_F32 && out_dt == SLAY_BF16) return SLAY_ERR_UNSUPPORTED;
+    if (n_rows == 0) return SLAY_OK;
+    if (!x || !phi || !aligned(x, 16) || !aligned(phi, 16)) return SLAY_ERR_INVALID_ARG;
+    if (n_rows > (int64_t(1) << 36)) return SLAY_ERR_UNSUPPORTED;
+    Params P;
+    if ((s = get_params(D, R, m, seed, eps, &P)) != SLAY_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (in_dt == SLAY_BF16 && out_dt == SLAY_BF16 && tc_supported(SLAY_OP_FEATURE_MAP, 1, 1, 1, R, m))
+        e = tc_feature_map(x, phi, n_rows, P, st);
+    else
+        e = simt_feature_map(x, phi, n_rows, in_dt, out_dt, P, st);
+    return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
+}
+
+slay_status slay_attn_causal_fwd(const void* q, const void* k, const void* v, void* out,
+                                 float* den, int B, int H, int L, int D, int Dv, slay_dtype dt,
+                                 int R, int m, uint64_t seed, float eps, void* workspace,
+                                 size_t ws_bytes, void* stream)
+{
+    return attn_fwd(q, k, v, out, den, B, H, L, D, Dv, dt, R, m, seed, eps, workspace, ws_bytes,
+                    stream, true);
+}
+
+slay_status slay_attn_bidir_fwd(const void* q, const void* k, const void* v, void* out,
+                                float* den, int B, int H, int L, int D, int Dv, slay_dtype dt,
+                                int R, int m, uint64_t seed, float eps, void* workspace,
+                                size_t ws_bytes, void* stream)
+{
+    return attn_fwd(q, k, v, out, den, B, H, L, D, Dv, dt, R, m, seed, eps, workspace, ws_bytes,
+                    stream, false);
+}
+
+slay_status slay_attn_causal_bwd(const void* q, const void* k, const void* v, const void* out,
+                                 const float* den, const void* dout, float* dq, float* dk,
+                                 float* dv, int B, int H, int L, int D, int Dv, slay_dtype dt,
+                                 int R, int m, uint64_t seed, float eps, void* workspace,
+                                 size_t ws_bytes, void* stream)
+{
+    slay_status s = check_attn(q, k, v, out, B, H, L, D, Dv, dt, R, m, eps);
+    if (s != SLAY_OK) return s;
+    if (static_cast<int64_t>(B) * H * L == 0) return SLAY_OK;
+    if (!den || !dout || !dq || !dk || !dv) return SLAY_ERR_INVALID_ARG;
+    if (!aligned(den, 4) || !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) ||
+        !aligned(dv, 16))
+        return SLAY_ERR_INVALID_ARG;
+    const size_t need = attn_ws(SLAY_OP_CAUSAL_BWD, dt, B, H, L, Dv, R, m);
+    if (need > 0 && (!workspace || ws_bytes < need || !aligned(workspace, 256)))
+        return SLAY_ERR_INVALID_ARG;
+    Params P;
+    if ((s = get_params(D, R, m, seed, eps, &P)) != SLAY_OK) return s;
+    cudaError_t e = simt_attn_causal_bwd(q, k, v, out, den, dout, dq, dk, dv, B, H, L, dt, P, eps,
+                                         workspace, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
+}
+
+slay_status slay_decode_step(const void* q, const void* k, const void* v, float* S, float* z,
+                             void* out, int Bt, int H, int D, int Dv, slay_dtype dt, int R, int m,
+                             uint64_t seed, float eps, void* stream)
+{
+    if (Bt < 0 || H < 0) return SLAY_ERR_INVALID_ARG;
+    slay_status s = check_shape(D, Dv, R, m);
+    if (s != SLAY_OK) return s;
+    if (!dtype_ok(dt) || !eps_ok(eps)) return SLAY_ERR_INVALID_ARG;
+    const int64_t N = static_cast<int64_t>(Bt) * H;
+    if (N == 0) return SLAY_OK;
+    if (N > (1 << 30)) return SLAY_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !S || !z || !out) return SLAY_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(S, 16) ||
+        !aligned(z, 16) || !aligned(out, 16))
+        return SLAY_ERR_INVALID_ARG;
+    Params P;
+    if ((s = get_params(D, R, m, seed, eps, &P)) != SLAY_OK) return s;
+    cudaError_t e = simt_decode_step(q, k, v, S, z, out, static_cast<int>(N), dt, P, eps,
+                                     static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
+}
+
+size_t slay_workspace_bytes(slay_op op, slay_dtype dt, int B, int H, int L, int D, int Dv, int R,
+                            int m)
+{
+    if (B < 0 || H < 0 || L < 0 || !dtype_ok(dt)) return SIZE_MAX;
+    if (check_shape(D, Dv, R, m) != SLAY_OK) return SIZE_MAX;
+    if (op == SLAY_OP_FEATURE_MAP || op == SLAY_OP_DECODE) return 0;
+    if (op != SLAY_OP_CAUSAL_FWD && op != SLAY_OP_BIDIR_FWD && op != SLAY_OP_CAUSAL_BWD)
+        return SIZE_MAX;
+    if (static_cast<int64_t>(B) * H * L == 0) return 0;
+    return attn_ws(op, dt, B, H, L, Dv, R, m);
+}
+
+slay_status slay_prepare(int D, int R, int m, uint64_t seed, float eps)
+{
+    slay_status s = check_shape(D, kD, R, m);
+    if (s != SLAY_OK) return s;
+    if (!eps_ok(eps)) return SLAY_ERR_INVALID_ARG;
+    Params P;
+    return get_params(D, R, m, seed, eps, &P);
+}
+
+slay_status slay_sketch_params(int D, int R, int m, uint64_t seed, float eps, float* omega_host,
+                               float* anchors_host, double* s_host, double* w_host)
+{
+    if (D <= 0 || D > 4096 || R <= 0 || R > kMaxR || m <= 0 || !eps_ok(eps))
+        return SLAY_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(R) * m * D > (int64_t(1) << 31)) return SLAY_ERR_UNSUPPORTED;
+    if (!draw_sketch(D, R, m, seed, static_cast<double>(eps), omega_host, anchors_host, s_host,
+                     w_host))
+        return SLAY_ERR_INVALID_ARG;
+    return SLAY_OK;
+}
+
+const char* slay_status_string(slay_status st)
+{
+    switch (st) {
+        case SLAY_OK: return "ok";
+        case SLAY_ERR_INVALID_ARG: return "invalid argument";
+        case SLAY_ERR_UNSUPPORTED: return "unsupported size or dtype";
+        case SLAY_ERR_CUDA: return "CUDA error";
+        case SLAY_ERR_TIMEOUT: return "timeout";
+        case SLAY_ERR_NO_MEMORY: return "out of host memory";
+    }
+    return "unknown status";
+}
+
+const char* slay_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

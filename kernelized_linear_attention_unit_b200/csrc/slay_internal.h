@@ -1,0 +1,76 @@
+// slay_internal.h -- declarations shared by the files of libslay.so (not installed).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "slay.h"
+
+namespace slay {
+
+constexpr int kMaxR = 16;
+constexpr int kMaxF = 1024;
+constexpr int kD = 64;  // head dimension this build supports (D == Dv == 64)
+
+// Device view of one sketch-parameter key.  The node constants travel by value.
+struct Params {
+    const float* omT;    // [D][F]   omega transposed (feature index fastest)
+    const float* anT;    // [D][F]   anchors transposed
+    const float* om;     // [F][D]   omega, row per feature
+    const float* an;     // [F][D]   anchors, row per feature
+    const uint16_t* wB;  // [F/16][2][16][D] bf16 (see tensor-core path), may be null
+    int D, R, m, F;
+    // phi_f = exp2(a2[r] * u + b2[r]) * p^2 with u = omega_f . x^, p = a_f . x^, where
+    // a2 = sqrt(2 s_r) log2(e), b2 = log2(sqrt(wt_r/m)) - s_r log2(e).
+    float a2[kMaxR];
+    float b2[kMaxR];
+    // For the backward: sq = sqrt(2 s_r), c = sqrt(wt_r/m).
+    float sq[kMaxR];
+    float c[kMaxR];
+};
+
+// ---- per-launch timing (slay_trace.cpp) ----
+// Brackets the kernel launched inside its scope with CUDA events while tracing is on.
+class TraceScope {
+public:
+    TraceScope(const char* name, cudaStream_t st);
+    ~TraceScope();
+    TraceScope(const TraceScope&) = delete;
+    TraceScope& operator=(const TraceScope&) = delete;
+
+private:
+    cudaStream_t st_;
+    int idx_;
+};
+
+// ---- host math (slay_params.cpp): no CUDA calls ----
+void philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]);
+// Nodes/weights of the R-point Gauss-Laguerre rule; false on failure.
+bool gauss_laguerre(int R, double* t, double* w);
+// omega, anchors: [F*D] float, s, wt: [R] double.  false on failure.
+bool draw_sketch(int D, int R, int m, uint64_t seed, double eps, float* omega,
+                 float* anchors, double* s, double* wt);
+
+// ---- CUDA-core kernels (slay_simt.cu) ----
+// Sizes of the workspace carve-outs of the CUDA-core path.
+size_t simt_ws_causal(int B, int H, int L, int Dv, int F);
+size_t simt_ws_bidir(int B, int H, int L, int Dv, int F);
+size_t simt_ws_bwd(int B, int H, int L, int Dv, int F);
+
+cudaError_t simt_feature_map(const void* x, void* phi, int64_t n, slay_dtype in_dt,
+                             slay_dtype out_dt, const Params& P, cudaStream_t st);
+cudaError_t simt_attn_fwd(const void* q, const void* k, const void* v, void* out, float* den,
+                          int B, int H, int L, slay_dtype dt, const Params& P, float eps,
+                          bool causal, void* ws, cudaStream_t st);
+cudaError_t simt_attn_causal_bwd(const void* q, const void* k, const void* v,
+                                 const void* out, const float* den, const void* dout,
+                                 float* dq, float* dk, float* dv, int B, int H, int L,
+                                 slay_dtype dt, const Params& P, float eps, void* ws,
+                                 cudaStream_t st);
+cudaError_t simt_decode_step(const void* q, const void* k, const void* v, float* S, float* z,
+                             void* out, int N, slay_dtype dt, const Params& P, float eps,
+                             cudaStream_t st);
+
+}  // namespace slay

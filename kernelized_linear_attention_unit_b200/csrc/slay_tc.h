@@ -1,0 +1,27 @@
+// slay_tc.h -- tensor-core (tcgen05/TMEM, TMA) path of libslay.so for bf16 inputs.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "slay.h"
+#include "slay_internal.h"
+
+namespace slay {
+
+// Whether the tensor-core path takes this op at these sizes (bf16 mode only).
+bool tc_supported(slay_op op, int B, int H, int L, int R, int m);
+size_t tc_workspace_bytes(slay_op op, int B, int H, int L, int R, int m);
+// Elements of the packed bf16 projection operand (0 when the path is not built).
+size_t tc_wb_elems(int D, int R, int m);
+// Pack bf16 omega / anchors ([F][D] row-major bit patterns) into the operand layout.
+void tc_pack_wb(int D, int R, int m, const uint16_t* om, const uint16_t* an, uint16_t* wb);
+
+cudaError_t tc_feature_map(const void* x, void* phi, int64_t n, const Params& P, cudaStream_t st);
+cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, float* den,
+                        int B, int H, int L, const Params& P, float eps, bool causal, void* ws,
+                        cudaStream_t st);
+
+}  // namespace slay

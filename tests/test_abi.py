@@ -1,0 +1,128 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the header
+declares, draws the same sketch parameters as the oracle's independent Philox, and
+rejects bad arguments before touching the device."""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as O
+from kernelized_linear_attention_unit_b200 import binding as bd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "slay.h")
+
+
+def _declared():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(slay_[a-z0-9_]+)\s*\(", txt)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = bd.lib()
+    names = _declared()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(bd.EXPORTS) == set(names)
+
+
+def test_status_strings():
+    L = bd.lib()
+    for s in range(6):
+        assert L.slay_status_string(s)
+    assert L.slay_status_string(99) == b"unknown status"
+
+
+@pytest.mark.parametrize("D,R,m,seed", [(64, 2, 16, 1234), (64, 4, 64, 1234), (64, 8, 64, 99),
+                                        (16, 3, 5, 2 ** 40 + 17)])
+def test_sketch_params_match_oracle_bitwise(D, R, m, seed):
+    eps = float(np.float32(1e-6))
+    om, an, s, w = bd.slay_sketch_params(D, R, m, seed, eps)
+    P = O.sketch_params(D, R, m, seed, eps)
+    assert np.array_equal(om.astype(np.float64), P.omega)
+    assert np.array_equal(an.astype(np.float64), P.anchors)
+    # quadrature: Golub-Welsch (library) against Newton/bisection (oracle)
+    np.testing.assert_allclose(s, P.s, rtol=1e-13)
+    np.testing.assert_allclose(w, P.wt, rtol=1e-11)
+
+
+@pytest.mark.parametrize("R", list(range(1, 17)))
+def test_library_quadrature_against_library_rule(R):
+    _, _, s, w = bd.slay_sketch_params(4, R, 1, 0, 1.0)
+    tn, wn = np.polynomial.laguerre.laggauss(R)
+    np.testing.assert_allclose(s * 3.0, tn, rtol=1e-12)
+    np.testing.assert_allclose(w * 3.0, wn, rtol=1e-9, atol=1e-300)
+
+
+def test_workspace_bytes():
+    f = bd.slay_workspace_bytes
+    assert f(bd.OP_FEATURE_MAP, bd.SLAY_BF16, 1, 1, 16, 64, 64, 4, 64) == 0
+    assert f(bd.OP_DECODE, bd.SLAY_BF16, 1, 1, 16, 64, 64, 4, 64) == 0
+    assert f(bd.OP_CAUSAL_FWD, bd.SLAY_F32, 0, 8, 1024, 64, 64, 4, 64) == 0
+    for op in (bd.OP_CAUSAL_FWD, bd.OP_BIDIR_FWD, bd.OP_CAUSAL_BWD):
+        for dt in (bd.SLAY_F32, bd.SLAY_BF16):
+            a = f(op, dt, 1, 2, 1000, 64, 64, 4, 64)
+            b = f(op, dt, 1, 2, 2000, 64, 64, 4, 64)
+            assert 0 < a <= b
+            assert a % 256 == 0
+    with pytest.raises(bd.SlayError):
+        f(bd.OP_CAUSAL_FWD, bd.SLAY_F32, 1, 1, 16, 32, 64, 4, 64)
+
+
+def _fake(addr=0x10000):
+    return C.c_void_p(addr)
+
+
+def test_argument_errors_before_any_device_work():
+    L = bd.lib()
+    f = L.slay_attn_causal_fwd
+    good = dict(D=64, Dv=64, R=4, m=64)
+    args = lambda q=_fake(), k=_fake(), v=_fake(), out=_fake(), B=1, H=1, Ln=128, D=64, Dv=64, \
+        dt=bd.SLAY_BF16, R=4, m=64, eps=1e-6, ws=_fake(0x20000), wsb=1 << 40: \
+        (q, k, v, out, None, B, H, Ln, D, Dv, dt, R, m, 1234, eps, ws, wsb, None)
+    assert f(*args(q=None)) == bd.SLAY_ERR_INVALID_ARG
+    assert f(*args(out=None)) == bd.SLAY_ERR_INVALID_ARG
+    assert f(*args(q=_fake(0x10004))) == bd.SLAY_ERR_INVALID_ARG          # misaligned
+    assert f(*args(B=-1)) == bd.SLAY_ERR_INVALID_ARG
+    assert f(*args(D=32)) == bd.SLAY_ERR_UNSUPPORTED
+    assert f(*args(Dv=128)) == bd.SLAY_ERR_UNSUPPORTED
+    assert f(*args(R=17)) == bd.SLAY_ERR_UNSUPPORTED
+    assert f(*args(m=2048)) == bd.SLAY_ERR_UNSUPPORTED
+    assert f(*args(R=0)) == bd.SLAY_ERR_INVALID_ARG
+    assert f(*args(eps=0.0)) == bd.SLAY_ERR_INVALID_ARG
+    assert f(*args(eps=float("nan"))) == bd.SLAY_ERR_INVALID_ARG
+    assert f(*args(dt=7)) == bd.SLAY_ERR_INVALID_ARG
+    assert f(*args(ws=None)) == bd.SLAY_ERR_INVALID_ARG                    # workspace missing
+    assert f(*args(wsb=16)) == bd.SLAY_ERR_INVALID_ARG                     # workspace too small
+    assert f(*args(ws=_fake(0x20010))) == bd.SLAY_ERR_INVALID_ARG          # workspace misaligned
+    # empty work is a no-op even with NULL pointers
+    assert f(*args(q=None, k=None, v=None, out=None, Ln=0)) == bd.SLAY_OK
+    assert f(*args(q=None, k=None, v=None, out=None, B=0)) == bd.SLAY_OK
+    # feature map
+    fm = L.slay_feature_map
+    assert fm(None, _fake(), 10, 64, bd.SLAY_BF16, bd.SLAY_BF16, 4, 64, 1, 1e-6, None) == bd.SLAY_ERR_INVALID_ARG
+    assert fm(_fake(), _fake(), 10, 64, bd.SLAY_F32, bd.SLAY_BF16, 4, 64, 1, 1e-6, None) == bd.SLAY_ERR_UNSUPPORTED
+    assert fm(_fake(), _fake(), -1, 64, bd.SLAY_F32, bd.SLAY_F32, 4, 64, 1, 1e-6, None) == bd.SLAY_ERR_INVALID_ARG
+    assert fm(None, None, 0, 64, bd.SLAY_F32, bd.SLAY_F32, 4, 64, 1, 1e-6, None) == bd.SLAY_OK
+    # decode
+    dc = L.slay_decode_step
+    assert dc(_fake(), _fake(), _fake(), None, _fake(), _fake(), 2, 2, 64, 64, bd.SLAY_BF16, 4, 64,
+              1, 1e-6, None) == bd.SLAY_ERR_INVALID_ARG
+    assert dc(None, None, None, None, None, None, 0, 16, 64, 64, bd.SLAY_BF16, 4, 64, 1, 1e-6,
+              None) == bd.SLAY_OK
+    # backward needs den and the gradients
+    bw = L.slay_attn_causal_bwd
+    assert bw(_fake(), _fake(), _fake(), _fake(), None, _fake(), _fake(), _fake(), _fake(), 1, 1,
+              64, 64, 64, bd.SLAY_BF16, 4, 64, 1, 1e-6, _fake(0x20000), 1 << 40,
+              None) == bd.SLAY_ERR_INVALID_ARG
+
+
+def test_sketch_params_rejects_bad_args():
+    L = bd.lib()
+    assert L.slay_sketch_params(64, 0, 4, 1, 1e-6, None, None, None, None) == bd.SLAY_ERR_INVALID_ARG
+    assert L.slay_sketch_params(64, 4, 4, 1, -1.0, None, None, None, None) == bd.SLAY_ERR_INVALID_ARG
+    assert L.slay_sketch_params(64, 4, 4, 1, 1e-6, None, None, None, None) == bd.SLAY_OK

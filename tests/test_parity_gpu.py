@@ -1,0 +1,268 @@
+"""GPU parity: every entry point of libslay.so against the fp64 oracle.
+
+Inputs come from the shared seeded recipe (kernelized_linear_attention_unit_b200.workloads)
+and are rounded to the mode's dtype before either side sees them, so both compute on the
+same values.  Tolerances (relative L2 error, whole tensor): 1e-5 in fp32 mode and 1.5e-2 in
+bf16-input / fp32-accumulate mode.  Small cases are compared element by element over every
+row; the full-size workloads are compared on sampled rows (ends, chunk and tile borders,
+random rows), in the launch configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from kernelized_linear_attention_unit_b200 import binding as bd
+from kernelized_linear_attention_unit_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-5, "bf16": 1.5e-2}
+TDT = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+def _eps(w):
+    return float(np.float32(w.eps))
+
+
+def dev(x, dt):
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to("cuda").to(TDT[dt])
+
+
+def host(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def rel_l2(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def params(w):
+    return O.sketch_params(w.D, w.R, w.m, w.sketch_seed, _eps(w))
+
+
+def small(dt, R, m, L, B=1, H=2, correlated=False, seed=21):
+    return W.Workload("small", B=B, H=H, L=L, R=R, m=m, dtype=dt, correlated=correlated,
+                      data_seed=seed)
+
+
+# ------------------------------------------------------------- feature map
+
+@pytest.mark.parametrize("dt_in,dt_out,R,m,n", [("f32", "f32", 2, 16, 1000),
+                                                 ("f32", "f32", 4, 64, 130),
+                                                 ("bf16", "bf16", 4, 64, 1000),
+                                                 ("bf16", "f32", 8, 64, 333),
+                                                 ("bf16", "bf16", 8, 64, 4097)])
+def test_feature_map(dt_in, dt_out, R, m, n):
+    w = small(dt_in, R, m, n, B=1, H=1)
+    q, _, _ = W.gen_qkv(w)
+    x = q.reshape(n, 64).copy()
+    x[3] = 0.0                       # degenerate zero row -> phi = 0
+    x[5] *= 37.0                     # rescaled row -> same phi
+    P = params(w)
+    want = O.feature_map(x, P)
+    xt = dev(x, dt_in)
+    phi = torch.empty((n, R * m), device="cuda", dtype=TDT[dt_out])
+    bd.slay_feature_map(xt, phi, R, m, w.sketch_seed, _eps(w))
+    torch.cuda.synchronize()
+    got = host(phi)
+    tol = TOL["bf16"] if "bf16" in (dt_in, dt_out) else TOL["f32"]
+    assert rel_l2(got, want) <= tol
+    assert (got[3] == 0).all()
+    assert (np.delete(got, 3, axis=0) >= 0).all()
+
+
+# ------------------------------------------------------------ forward
+
+def _run_fwd(q, k, v, w, causal):
+    B, H, L, _ = q.shape
+    qt, kt, vt = dev(q, w.dtype), dev(k, w.dtype), dev(v, w.dtype)
+    out = torch.empty((B, H, L, w.Dv), device="cuda", dtype=TDT[w.dtype])
+    den = torch.empty((B, H, L), device="cuda", dtype=torch.float32)
+    fn = bd.slay_attn_causal_fwd if causal else bd.slay_attn_bidir_fwd
+    fn(qt, kt, vt, out, den, w.R, w.m, w.sketch_seed, _eps(w))
+    torch.cuda.synchronize()
+    return host(out), host(den)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("dt,R,m,L", [("f32", 2, 16, 256), ("f32", 2, 16, 1), ("f32", 4, 64, 200),
+                                      ("f32", 3, 16, 129), ("bf16", 4, 64, 300),
+                                      ("bf16", 4, 64, 1), ("bf16", 8, 64, 257),
+                                      ("bf16", 2, 16, 64)])
+def test_attn_fwd_small(dt, R, m, L, causal):
+    w = small(dt, R, m, L)
+    q, k, v = W.gen_qkv(w)
+    q[0, 1, min(2, L - 1)] = 0.0          # zero query: phi = 0, den = 0, out = 0
+    P = params(w)
+    want, wden = O.attn_quadratic(q, k, v, P, causal)
+    got, gden = _run_fwd(q, k, v, w, causal)
+    assert rel_l2(got, want) <= TOL[dt]
+    assert rel_l2(gden, wden) <= TOL[dt]
+    assert np.isfinite(got).all()
+    assert (got[0, 1, min(2, L - 1)] == 0).all()
+
+
+def test_tiny_workload_both_modes():
+    w = W.TINY
+    q, k, v = W.gen_qkv(w)
+    P = params(w)
+    for causal in (True, False):
+        want, wden = O.attn_quadratic(q, k, v, P, causal)
+        got, gden = _run_fwd(q, k, v, w, causal)
+        assert rel_l2(got, want) <= TOL["f32"]
+        assert rel_l2(gden, wden) <= TOL["f32"]
+
+
+FULL = [W.CAUSAL_2K, W.CAUSAL_16K, W.BIDIR_VISION, W.FWDBWD_8K]
+
+
+@pytest.mark.parametrize("w", FULL, ids=[x.name for x in FULL])
+def test_attn_fwd_full_size_sampled(w):
+    q, k, v = W.gen_qkv(w)
+    got, gden = _run_fwd(q, k, v, w, w.causal)
+    assert np.isfinite(got).all() and (gden > 0).all()
+    rows = W.sample_rows(w.L, 24)
+    # oracle on a subset of (b, h) slices at full length
+    bsel, hsel = slice(0, min(w.B, 2)), slice(0, min(w.H, 4))
+    P = params(w)
+    want, wden = O.attn_quadratic_rows(q[bsel, hsel], k[bsel, hsel], v[bsel, hsel], P,
+                                       w.causal, rows)
+    assert rel_l2(got[bsel, hsel][:, :, rows], want) <= TOL[w.dtype]
+    assert rel_l2(gden[bsel, hsel][:, :, rows], wden) <= TOL[w.dtype]
+
+
+def test_bidir_correlated_small():
+    w = small("bf16", 4, 64, 160, B=2, H=3, correlated=True)
+    q, k, v = W.gen_qkv(w)
+    P = params(w)
+    want, _ = O.attn_quadratic(q, k, v, P, False)
+    got, _ = _run_fwd(q, k, v, w, False)
+    assert rel_l2(got, want) <= TOL["bf16"]
+
+
+# ------------------------------------------------------------ backward
+
+def _run_bwd(q, k, v, g, w):
+    B, H, L, _ = q.shape
+    qt, kt, vt, gt = dev(q, w.dtype), dev(k, w.dtype), dev(v, w.dtype), dev(g, w.dtype)
+    out = torch.empty((B, H, L, w.Dv), device="cuda", dtype=TDT[w.dtype])
+    den = torch.empty((B, H, L), device="cuda", dtype=torch.float32)
+    bd.slay_attn_causal_fwd(qt, kt, vt, out, den, w.R, w.m, w.sketch_seed, _eps(w))
+    dq = torch.empty((B, H, L, w.D), device="cuda", dtype=torch.float32)
+    dk = torch.empty_like(dq)
+    dv = torch.empty((B, H, L, w.Dv), device="cuda", dtype=torch.float32)
+    bd.slay_attn_causal_bwd(qt, kt, vt, out, den, gt, dq, dk, dv, w.R, w.m, w.sketch_seed, _eps(w))
+    torch.cuda.synchronize()
+    return host(dq), host(dk), host(dv)
+
+
+@pytest.mark.parametrize("dt,R,m,L", [("f32", 2, 16, 100), ("f32", 4, 64, 130),
+                                      ("bf16", 4, 64, 150), ("bf16", 8, 64, 64),
+                                      ("bf16", 2, 16, 65)])
+def test_attn_bwd_small(dt, R, m, L):
+    w = small(dt, R, m, L)
+    q, k, v = W.gen_qkv(w)
+    g = W.gen_dout(w)
+    P = params(w)
+    wq, wk, wv = O.attn_causal_bwd(q, k, v, g, P)
+    gq, gk, gv = _run_bwd(q, k, v, g, w)
+    assert rel_l2(gq, wq) <= TOL[dt]
+    assert rel_l2(gk, wk) <= TOL[dt]
+    assert rel_l2(gv, wv) <= TOL[dt]
+
+
+def test_attn_bwd_single_token():
+    # L = 1: the only weight is a/(a+eps) ~ 1 - eps/a, so dq and dk are O(eps/a) and come
+    # from the cancellation <v, dn> + delta with delta = -<g, out>/Z.  Rounding `out` to
+    # bf16 (relative 2^-9) swamps that difference, so the case is checked in fp32, where
+    # the same cancellation amplifies fp32 rounding by a/eps: dv to 1e-5, dq and dk to 1e-3.
+    w = small("f32", 2, 16, 1)
+    q, k, v = W.gen_qkv(w)
+    g = W.gen_dout(w)
+    P = params(w)
+    wq, wk, wv = O.attn_causal_bwd(q, k, v, g, P)
+    gq, gk, gv = _run_bwd(q, k, v, g, w)
+    assert rel_l2(gv, wv) <= 1e-5
+    assert rel_l2(gq, wq) <= 1e-3
+    assert rel_l2(gk, wk) <= 1e-3
+
+
+def test_attn_bwd_full_size_sampled():
+    w = W.FWDBWD_8K
+    q, k, v = W.gen_qkv(w)
+    g = W.gen_dout(w)
+    gq, gk, gv = _run_bwd(q, k, v, g, w)
+    assert np.isfinite(gq).all() and np.isfinite(gk).all() and np.isfinite(gv).all()
+    rows = W.sample_rows(w.L, 12)
+    bsel, hsel = slice(0, 1), slice(0, 2)
+    P = params(w)
+    wq, wk, wv = O.attn_causal_bwd_rows(q[bsel, hsel], k[bsel, hsel], v[bsel, hsel],
+                                        g[bsel, hsel], P, rows)
+    assert rel_l2(gq[bsel, hsel][:, :, rows], wq) <= TOL["bf16"]
+    assert rel_l2(gk[bsel, hsel][:, :, rows], wk) <= TOL["bf16"]
+    assert rel_l2(gv[bsel, hsel][:, :, rows], wv) <= TOL["bf16"]
+
+
+# -------------------------------------------------------------- decode
+
+def _run_decode(q, k, v, S, z, w):
+    qt, kt, vt = dev(q, w.dtype), dev(k, w.dtype), dev(v, w.dtype)
+    St = torch.from_numpy(S).cuda()
+    zt = torch.from_numpy(z).cuda()
+    out = torch.empty(v.shape, device="cuda", dtype=TDT[w.dtype])
+    bd.slay_decode_step(qt, kt, vt, St, zt, out, w.R, w.m, w.sketch_seed, _eps(w))
+    torch.cuda.synchronize()
+    return host(out), St.cpu().numpy().astype(np.float64), zt.cpu().numpy().astype(np.float64)
+
+
+@pytest.mark.parametrize("dt,R,m,Bt,H", [("f32", 2, 16, 3, 2), ("f32", 8, 64, 5, 3),
+                                         ("bf16", 4, 64, 7, 2), ("bf16", 8, 64, 9, 16)])
+def test_decode_small(dt, R, m, Bt, H):
+    w = W.Workload("dec", B=Bt, H=H, L=1, R=R, m=m, dtype=dt, data_seed=31)
+    q, k, v, S, z = W.gen_decode(w)
+    P = params(w)
+    wo, wS, wz = O.decode_step(q, k, v, S, z, P)
+    go, gS, gz = _run_decode(q, k, v, S, z, w)
+    tol = TOL[dt]
+    assert rel_l2(go, wo) <= tol
+    assert rel_l2(gS, wS) <= 1e-5 if dt == "f32" else rel_l2(gS, wS) <= tol
+    assert rel_l2(gz, wz) <= 1e-5 if dt == "f32" else rel_l2(gz, wz) <= tol
+
+
+def test_decode_full_size():
+    w = W.DECODE
+    q, k, v, S, z = W.gen_decode(w)
+    go, gS, gz = _run_decode(q, k, v, S, z, w)
+    sel = slice(0, 32)
+    P = params(w)
+    wo, wS, wz = O.decode_step(q[sel], k[sel], v[sel], S[sel], z[sel], P)
+    assert rel_l2(go[sel], wo) <= TOL["bf16"]
+    assert rel_l2(gS[sel], wS) <= TOL["bf16"]
+    assert rel_l2(gz[sel], wz) <= TOL["bf16"]
+    # the state update itself is fp32: the increment phi(k) v^T is tiny next to S ~ N(0,1),
+    # so check the increment separately
+    dS = gS[sel] - S[sel].astype(np.float64)
+    wdS = wS - S[sel].astype(np.float64)
+    assert rel_l2(dS, wdS) <= TOL["bf16"]
+
+
+def test_decode_chain_matches_causal():
+    # L decode steps from S = z = 0 reproduce the causal forward rows (GPU vs oracle).
+    w = small("f32", 2, 16, 40, B=2, H=2)
+    q, k, v = W.gen_qkv(w)
+    P = params(w)
+    want, _ = O.attn_quadratic(q, k, v, P, True)
+    F = w.F
+    St = torch.zeros((2, 2, F, 64), device="cuda")
+    zt = torch.zeros((2, 2, F), device="cuda")
+    outs = []
+    for i in range(w.L):
+        qi, ki, vi = (dev(np.ascontiguousarray(a[:, :, i]), "f32") for a in (q, k, v))
+        o = torch.empty((2, 2, 64), device="cuda")
+        bd.slay_decode_step(qi, ki, vi, St, zt, o, w.R, w.m, w.sketch_seed, _eps(w))
+        outs.append(o)
+    got = torch.stack(outs, dim=2).cpu().numpy()
+    assert rel_l2(got, want) <= TOL["f32"]
