@@ -127,6 +127,30 @@ slay_status slay_decode_step(const void* q, const void* k, const void* v,
                              int Bt, int H, int D, int Dv, slay_dtype dt,
                              int R, int m, uint64_t seed, float eps, void* stream);
 
+/* The causal forward above for callers that cannot allocate device memory: a host that
+ * reserves all of HBM for its own pool at start-up, a plugin that is handed tensors but
+ * no workspace, or a latency-bound loop that must not pay for cudaMalloc's implicit
+ * synchronisation.  The pages of the method have no counterpart of this entry point; it
+ * computes exactly what slay_attn_causal_fwd computes, with the same kernels.
+ * Arguments: as slay_attn_causal_fwd without workspace/ws_bytes.
+ * Memory: allocates nothing.  Its workspace is a file-scope device array of 32 MiB and its
+ *   sketch parameters live in a second one of 2 MiB; every GPU that loads the library
+ *   holds both (34 MiB) until the process exits.  Sizes whose workspace
+ *   (slay_workspace_bytes(SLAY_OP_CAUSAL_FWD, ...)) exceeds 32 MiB are rejected with
+ *   SLAY_ERR_UNSUPPORTED before anything is enqueued.
+ * Set-up: the first call on a device looks up the arrays' device addresses; the first
+ *   call with a new (D, R, m, seed, eps) uploads that key's parameters into the single
+ *   parameter slot with a copy ordered on `stream`.  Make such calls before capturing the
+ *   stream into a graph.
+ * Sharing: all calls on a device share both arrays, which keep the last call's contents
+ *   (no part of them needs to start at zero).  Calls that overlap on the GPU -- on
+ *   different streams, or from different host threads -- race on them; calls in order on
+ *   one stream do not. */
+slay_status slay_attn_causal_fwd_noalloc(const void* q, const void* k, const void* v,
+                                         void* out, float* den, int B, int H, int L, int D,
+                                         int Dv, slay_dtype dt, int R, int m, uint64_t seed,
+                                         float eps, void* stream);
+
 /* Workspace bytes an entry point needs for these sizes (0 if none; SIZE_MAX if the
  * sizes are unsupported).  Feature map and decode need none. */
 size_t slay_workspace_bytes(slay_op op, slay_dtype dt, int B, int H, int L, int D, int Dv,

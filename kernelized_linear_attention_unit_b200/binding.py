@@ -22,7 +22,7 @@ OP_FEATURE_MAP, OP_CAUSAL_FWD, OP_BIDIR_FWD, OP_CAUSAL_BWD, OP_DECODE = range(5)
 EXPORTS = ["slay_feature_map", "slay_attn_causal_fwd", "slay_attn_bidir_fwd",
            "slay_attn_causal_bwd", "slay_decode_step", "slay_workspace_bytes", "slay_prepare",
            "slay_sketch_params", "slay_status_string", "slay_last_error", "slay_trace_enable",
-           "slay_trace_read"]
+           "slay_trace_read", "slay_attn_causal_fwd_noalloc"]
 
 
 class SlayError(RuntimeError):
@@ -52,6 +52,8 @@ def lib():
     attn = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, u64, f32, vp, sz, vp]
     L.slay_attn_causal_fwd.argtypes = attn
     L.slay_attn_bidir_fwd.argtypes = attn
+    L.slay_attn_causal_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                               i32, i32, u64, f32, vp]
     L.slay_attn_causal_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
                                        i32, i32, i32, i32, u64, f32, vp, sz, vp]
     L.slay_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
@@ -70,6 +72,7 @@ def lib():
     L.slay_trace_read.restype = i32
     for name in ("slay_feature_map", "slay_attn_causal_fwd", "slay_attn_bidir_fwd",
                  "slay_attn_causal_bwd", "slay_decode_step", "slay_prepare",
+                 "slay_attn_causal_fwd_noalloc",
                  "slay_sketch_params"):
         getattr(L, name).restype = i32
     _lib = L
@@ -195,6 +198,21 @@ def slay_attn_causal_fwd(q, k, v, out, den, R, m, seed, eps, workspace=None, str
 def slay_attn_bidir_fwd(q, k, v, out, den, R, m, seed, eps, workspace=None, stream=None):
     _attn(lib().slay_attn_bidir_fwd, "slay_attn_bidir_fwd", OP_BIDIR_FWD, q, k, v, out, den,
           R, m, seed, eps, workspace, stream)
+
+
+def slay_attn_causal_fwd_noalloc(q, k, v, out, den, R, m, seed, eps, stream=None):
+    """Causal forward that allocates nothing (library-owned static scratch, 32 MiB max)."""
+    _check(q, "q")
+    B, H, L, D = q.shape
+    Dv = v.shape[-1]
+    _check(k, "k", q.dtype, (B, H, L, D))
+    _check(v, "v", q.dtype, (B, H, L, Dv))
+    _check(out, "out", q.dtype, (B, H, L, Dv))
+    if den is not None:
+        _check(den, "den", torch.float32, (B, H, L))
+    _raise(lib().slay_attn_causal_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(den), B,
+                                              H, L, D, Dv, _dt(q), R, m, seed, eps,
+                                              _stream(stream)), "slay_attn_causal_fwd_noalloc")
 
 
 def slay_attn_causal_bwd(q, k, v, out, den, dout, dq, dk, dv, R, m, seed, eps, workspace=None,

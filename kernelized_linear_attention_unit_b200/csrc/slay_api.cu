@@ -125,6 +125,8 @@ slay_status get_params(int D, int R, int m, uint64_t seed, float eps, Params* ou
     return SLAY_OK;
 }
 
+}  // namespace
+
 bool eps_ok(float eps) { return std::isfinite(eps) && eps > 0.0f; }
 bool dtype_ok(slay_dtype d) { return d == SLAY_F32 || d == SLAY_BF16; }
 
@@ -165,6 +167,8 @@ size_t attn_ws(slay_op op, slay_dtype dt, int B, int H, int L, int Dv, int R, in
         default: return 0;
     }
 }
+
+namespace {
 
 slay_status attn_fwd(const void* q, const void* k, const void* v, void* out, float* den, int B,
                      int H, int L, int D, int Dv, slay_dtype dt, int R, int m, uint64_t seed,

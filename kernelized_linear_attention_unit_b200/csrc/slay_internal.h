@@ -53,6 +53,14 @@ bool gauss_laguerre(int R, double* t, double* w);
 bool draw_sketch(int D, int R, int m, uint64_t seed, double eps, float* omega,
                  float* anchors, double* s, double* wt);
 
+// ---- argument checks and workspace sizing shared by the entry points (slay_api.cu) ----
+bool eps_ok(float eps);
+bool dtype_ok(slay_dtype d);
+slay_status check_shape(int D, int Dv, int R, int m);
+slay_status check_attn(const void* q, const void* k, const void* v, const void* out, int B,
+                       int H, int L, int D, int Dv, slay_dtype dt, int R, int m, float eps);
+size_t attn_ws(slay_op op, slay_dtype dt, int B, int H, int L, int Dv, int R, int m);
+
 // ---- CUDA-core kernels (slay_simt.cu) ----
 // Sizes of the workspace carve-outs of the CUDA-core path.
 size_t simt_ws_causal(int B, int H, int L, int Dv, int F);
