@@ -66,7 +66,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
                 sys.stderr.write(log)
     objs = [o for o, _ in results]
     tmp = LIB + ".tmp.%d" % os.getpid()
-    cmd = [NVCC] + ARCH + ["-shared", "-o", tmp] + objs + ["-lcuda"]
+    cmd = [NVCC] + ARCH + ["-shared", "-o", tmp] + objs
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("link failed: %s\n%s\n%s" % (" ".join(cmd), r.stdout, r.stderr))

@@ -91,7 +91,9 @@ def _run_fwd(q, k, v, w, causal):
 @pytest.mark.parametrize("dt,R,m,L", [("f32", 2, 16, 256), ("f32", 2, 16, 1), ("f32", 4, 64, 200),
                                       ("f32", 3, 16, 129), ("bf16", 4, 64, 300),
                                       ("bf16", 4, 64, 1), ("bf16", 8, 64, 257),
-                                      ("bf16", 2, 16, 64)])
+                                      ("bf16", 2, 16, 64), ("bf16", 2, 64, 129),
+                                      ("bf16", 4, 64, 1000), ("bf16", 2, 64, 2049),
+                                      ("bf16", 4, 64, 128)])
 def test_attn_fwd_small(dt, R, m, L, causal):
     w = small(dt, R, m, L)
     q, k, v = W.gen_qkv(w)
