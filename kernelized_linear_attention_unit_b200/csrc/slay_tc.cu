@@ -5,19 +5,26 @@
 // (b,h) sequence, out_i = phi(q_i)^T S_i / (phi(q_i)^T z_i + eps) with
 // S_i = sum_{j<=i} phi(k_j) v_j^T, z_i = sum_{j<=i} phi(k_j), in 128-token tiles:
 //
-//   U   = X W_t^T                   projection of a 64-feature slice t (omega and anchor
-//                                   rows of W_t), raw bf16 x; the 1/|x| scale is applied in
-//                                   the epilogue, phi = exp2(a2 u/|x| + b2) (p/|x|)^2
-//   P  += phiQ_t phiK_t^T           intra-tile scores, summed over feature slices
+//   U   = X W_n^T                   projection of a 32-feature sub-slice n (its omega and
+//                                   anchor rows), raw bf16 x; the 1/|x| scale is applied in
+//                                   the epilogue: phi = exp2(a2 u/|x| + b2) (p/|x|)^2
+//   P  += phiQ_t phiK_t^T           intra-tile scores, summed over 64-feature slices t
 //   O  += phiQ_t S_t                inter-tile readout with the state entering the tile
 //   O  += tril(P) V                 masked intra-tile term
-//   S  += phiK^T V,  z += phiK^T 1  state update (fp32 in tensor memory)
+//   [S|z] += phiK^T [V|1]           state update, z as extra accumulator columns (fp32 in
+//                                   tensor memory), one N=80 MMA per K step
 //
 // Sequences are split into L-segments so that every SM has work: a first kernel computes
 // each segment's own sum of phi(k) [v, 1]^T, the second starts each segment from the sum
 // of the earlier segments' contributions and produces the outputs.  Neither kernel waits on
-// another CTA.  Every mbarrier wait is bounded in time; a timeout sets an error word in the
-// workspace header and the kernel leaves after its in-flight copies have landed.
+// another CTA.
+//
+// Both kernels are warp-specialised: warp 0 issues TMA copies, warps 1 and 10 issue
+// tcgen05 MMAs (one elected thread each: the issue rate of a single thread, not the tensor
+// pipe, limits narrow MMAs), warps 2-5 and 6-9 are two epilogue groups (one row of a 128-row
+// tile per thread, one TMEM lane each).  Hand-offs go through mbarriers.  Every wait is
+// bounded in time; a timeout sets an error word in the workspace header, later waits give
+// up at once, and the CTA drains before releasing its memory.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -35,59 +42,75 @@ using namespace tc;
 
 namespace {
 
-constexpr int kTile = 128;             // tokens per tile (MMA M)
-constexpr int kSlice = 64;             // features per projection slice
-constexpr int kTileBytes = kTile * 128;  // one [128 rows][64 bf16] swizzled tile = 16 KiB
-constexpr int kThreads = 128;
-constexpr size_t kWsHeader = 256;      // error word + padding at the start of the workspace
+constexpr int kTile = 128;                 // tokens per tile (MMA M)
+constexpr int kSlice = 64;                 // features per phi tile (K of the P MMA)
+constexpr int kSub = 32;                   // features per projection (N = 64 with anchors)
+constexpr int kTileBytes = kTile * 128;    // one [128 rows][64 bf16] swizzled tile = 16 KiB
+constexpr int kWBytes = 64 * 128;          // one projection operand [64 rows][64 bf16] = 8 KiB
+constexpr int kWSlots = 3;                 // output kernel: 3 x 8 KiB projection operands
+constexpr int kThreads = 352;              // 11 warps
+constexpr int kOnesBytes = kTileBytes;     // [128][64] bf16 ones: the z columns of [V | 1]
+constexpr size_t kWsHeader = 256;          // error word + padding at the start of the workspace
 constexpr int kNumSMs = 148;
+constexpr uint64_t kWaitNs = 2000000000ull;
 
 // TMEM column map (one CTA per SM, 512 columns allocated).
-constexpr uint32_t kColU = 0;     // 128: projection of one slice (64 u | 64 p)
-constexpr uint32_t kColP = 128;   // 128: intra-tile scores
-constexpr uint32_t kColO = 256;   // 64 : output numerator
-constexpr uint32_t kColS = 320;   // 2 x 64: state S, feature halves
-constexpr uint32_t kColZ = 448;   // 2 x 16: state z (column 0 of each half is read)
-constexpr uint32_t kColSA = 128;  // state kernel: S at 128.., z at 256..
-constexpr uint32_t kColZA = 256;
+constexpr uint32_t kColU0 = 0;     // 64: q-side projection (32 u | 32 p)
+constexpr uint32_t kColU1 = 64;    // 64: k-side projection
+constexpr uint32_t kColP = 128;    // 128: intra-tile scores
+constexpr uint32_t kColO = 256;    // 64 : output numerator
+constexpr uint32_t kColS = 320;    // 2 x 80: state [S | z], feature halves (z in column 64)
 
-enum { BAR_QK = 0, BAR_V = 1, BAR_W0 = 2, BAR_W1 = 3, BAR_MMA = 4, NUM_BARS = 8 };
-
-struct SmemOut {
-    uint32_t w, q, k, v, phik, phiq, sbf, ones, z, bar, tmem, total;
+// -------------------------------------------------------------- barriers
+enum {
+    B_QK_FULL = 0, B_QK_EMPTY, B_V_FULL, B_V_EMPTY,
+    B_W_FULL0, B_W_FULL1, B_W_FULL2, B_W_FULL3,
+    B_W_EMPTY0, B_W_EMPTY1, B_W_EMPTY2, B_W_EMPTY3,
+    B_U_FULL0, B_U_FULL1, B_U_EMPTY0, B_U_EMPTY1,
+    B_PQ_FULL0, B_PQ_FULL1, B_PQ_EMPTY0, B_PQ_EMPTY1,
+    B_PK_FULL, B_P_FULL, B_PSM_FULL, B_TILE_DONE, B_O_EMPTY, B_SBF_READY,
+    NUM_BARS
 };
 
+struct SmemOut {
+    uint32_t w, q, k, v, phik, phiq, sbf, ones, z, dsum, bar, tmem, total;
+};
+
+// Output kernel: the masked scores P (two [128][64] tiles) reuse the phi(q) double buffer.
 __host__ __device__ inline SmemOut smem_out_layout(int F)
 {
     SmemOut s;
     s.w = 0;
-    s.q = 2 * kTileBytes;
+    s.q = kWSlots * kWBytes;
     s.k = s.q + kTileBytes;
     s.v = s.k + kTileBytes;
-    s.phik = s.v + kTileBytes;
+    s.ones = s.v + kTileBytes;                         // right after V: fixed offset from it
+    s.phik = s.ones + kOnesBytes;
     s.phiq = s.phik + (F / kSlice) * kTileBytes;
-    s.sbf = s.phiq + kTileBytes;
-    s.ones = s.sbf + F * 128;
-    s.z = s.ones + 4096;
-    s.bar = s.z + F * 4;
+    s.sbf = s.phiq + 2 * kTileBytes;
+    s.z = s.sbf + F * 128;
+    s.dsum = s.z + F * 4;
+    s.bar = s.dsum + kTile * 4;
     s.tmem = s.bar + NUM_BARS * 8;
     s.total = s.tmem + 16;
     return s;
 }
 
+// State kernel: two 16 KiB projection operands (64 features each).
+constexpr int kWStateBytes = 2 * kWBytes;
 struct SmemState {
-    uint32_t w, k, v, phik, ones, bar, tmem, total;
+    uint32_t w, k, v, ones, phik, bar, tmem, total;
 };
 
 __host__ __device__ inline SmemState smem_state_layout(int F)
 {
     SmemState s;
     s.w = 0;
-    s.k = 2 * kTileBytes;
+    s.k = 2 * kWStateBytes;
     s.v = s.k + kTileBytes;
-    s.phik = s.v + kTileBytes;
-    s.ones = s.phik + (F / kSlice) * kTileBytes;
-    s.bar = s.ones + 4096;
+    s.ones = s.v + kTileBytes;
+    s.phik = s.ones + kOnesBytes;
+    s.bar = s.phik + (F / kSlice) * kTileBytes;
     s.tmem = s.bar + NUM_BARS * 8;
     s.total = s.tmem + 16;
     return s;
@@ -97,14 +120,39 @@ struct Seg {
     int bh, seg, t_begin, t_end;
 };
 
-__device__ __forceinline__ Seg segment_of(int block, int nseg, int ntiles)
+__device__ __forceinline__ Seg segment_of(int index, int nseg, int ntiles)
 {
     Seg s;
-    s.bh = block / nseg;
-    s.seg = block % nseg;
+    s.bh = index / nseg;
+    s.seg = index % nseg;
     s.t_begin = static_cast<int>((static_cast<int64_t>(s.seg) * ntiles) / nseg);
     s.t_end = static_cast<int>((static_cast<int64_t>(s.seg + 1) * ntiles) / nseg);
     return s;
+}
+
+struct KParams {
+    int L, F, m, nseg, ntiles;
+    float eps;
+    float a2[kMaxR];
+    float b2[kMaxR];
+};
+
+// A waiter that stops waiting (and reports) once any wait of this thread timed out.
+struct Waiter {
+    bool ok = true;
+    __device__ __forceinline__ void wait(uint64_t* bar, uint32_t& phase)
+    {
+        ok = mbar_wait(bar, phase, ok ? kWaitNs : 0) && ok;
+        phase ^= 1u;
+    }
+};
+
+__device__ __forceinline__ void drain_after_failure(bool ok)
+{
+    if (ok) return;
+    const uint64_t t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < 20000000ull) {
+    }
 }
 
 // Sum of squares of one 64-element bf16 row (128 bytes; order does not matter, so the
@@ -130,122 +178,111 @@ __device__ __forceinline__ void row_scale(const unsigned char* row, float& inv, 
     l2inv2 = -2.0f * __log2f(n);
 }
 
-// Epilogue of one projection slice: TMEM columns [colU, colU+64) hold u, [colU+64, +128)
-// hold p for this thread's row.  phi_j = exp2(a u_j + b) p_j^2 with a = a2[r]/|x| and
-// b = b2[r] + 2 log2(1/|x|).  Writes the 64 bf16 values as row `row` of a 128-byte-swizzled
-// K-major tile at `tile_addr`; if zs != nullptr also returns sum_j phi_j zs[j].
-__device__ __forceinline__ float phi_slice_epilogue(uint32_t taddr_row, float a, float b,
-                                                    uint32_t tile_addr, uint32_t row,
-                                                    const float* zs)
+// phi of one 32-feature sub-slice from registers holding u (32) and p (32) of this row:
+// phi_j = exp2(a u_j + b) p_j^2, a = a2[r]/|x|, b = b2[r] + 2 log2(1/|x|).  Stores the 32
+// bf16 values as chunks [4*half, 4*half+4) of row `row` of the swizzled tile at tile_addr.
+// With zs != nullptr returns sum_j phi_j zs[j] (the inter-tile denominator term).
+__device__ __forceinline__ float phi_sub_epilogue(const uint32_t (&ur)[32], const uint32_t (&pr)[32],
+                                                  float a, float b, uint32_t tile_addr,
+                                                  uint32_t row, int half, const float* zs)
 {
     float dz = 0.0f;
+    uint32_t pk[16];
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-        uint32_t ur[32], pr[32];
-        tmem_ld32(taddr_row + kColU + 32 * c, ur);
-        tmem_ld32(taddr_row + kColU + 64 + 32 * c, pr);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-            const float u0 = __uint_as_float(ur[j]), u1 = __uint_as_float(ur[j + 1]);
-            const float p0 = __uint_as_float(pr[j]), p1 = __uint_as_float(pr[j + 1]);
-            const float f0 = ex2(fmaf(a, u0, b)) * p0 * p0;
-            const float f1 = ex2(fmaf(a, u1, b)) * p1 * p1;
-            if (zs) {
-                dz = fmaf(f0, zs[32 * c + j], dz);
-                dz = fmaf(f1, zs[32 * c + j + 1], dz);
-            }
-            pk[j >> 1] = pack_bf16(f0, f1);
+    for (int j = 0; j < 32; j += 2) {
+        const float p0 = __uint_as_float(pr[j]), p1 = __uint_as_float(pr[j + 1]);
+        const float f0 = ex2(fmaf(a, __uint_as_float(ur[j]), b)) * p0 * p0;
+        const float f1 = ex2(fmaf(a, __uint_as_float(ur[j + 1]), b)) * p1 * p1;
+        if (zs) {
+            dz = fmaf(f0, zs[j], dz);
+            dz = fmaf(f1, zs[j + 1], dz);
         }
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            st_shared_v4(tile_addr + sw128_off(row, 4 * c + q), pk[4 * q], pk[4 * q + 1],
-                         pk[4 * q + 2], pk[4 * q + 3]);
+        pk[j >> 1] = pack_bf16(f0, f1);
     }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        st_shared_v4(tile_addr + sw128_off(row, 4 * half + q), pk[4 * q], pk[4 * q + 1],
+                     pk[4 * q + 2], pk[4 * q + 3]);
     return dz;
 }
 
-// After a timed-out wait: give copies and MMAs still in flight time to land (bounded)
-// before the CTA releases its shared and tensor memory.
-__device__ __forceinline__ void drain_after_failure(bool ok)
+// U (64 columns: 32 u then 32 p) = X [128 x 64] . W_n^T [64 x 64]
+__device__ __forceinline__ void issue_projection(uint32_t d_tmem, uint32_t x_addr, uint32_t w_addr)
 {
-    if (ok) return;
-    const uint64_t t0 = global_timer_ns();
-    while (global_timer_ns() - t0 < 20000000ull) {
-    }
-}
-
-struct KParams {
-    int L, F, m, nseg, ntiles;
-    float eps;
-    float a2[kMaxR];
-    float b2[kMaxR];
-};
-
-__device__ __forceinline__ void issue_projection(uint32_t tmem, uint32_t x_addr, uint32_t w_addr)
-{
-    constexpr uint32_t id = idesc_bf16(128, 128, 0, 0);
+    constexpr uint32_t id = idesc_bf16(128, 64, 0, 0);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-        umma_bf16(tmem + kColU, sdesc(x_addr + 32 * kk, 16, 1024, kLayoutSW128),
+        umma_bf16(d_tmem, sdesc(x_addr + 32 * kk, 16, 1024, kLayoutSW128),
                   sdesc(w_addr + 32 * kk, 16, 1024, kLayoutSW128), id, kk > 0 ? 1u : 0u);
 }
 
-// S_h (+)= phiK_h^T V and z_h (+)= phiK_h^T 1 for feature halves h (phiK as an MN-major
-// A operand: 128 features = two 64-feature sub-tiles 16 KiB apart).
-__device__ __forceinline__ void issue_state_update(uint32_t tmem, uint32_t colS, uint32_t colZ,
-                                                   uint32_t phik, uint32_t vaddr, uint32_t ones,
-                                                   int halves, bool first)
+// [S|z]_h (+)= phiK_h^T [V | 1] for feature half h: phiK as an MN-major A operand
+// (128 features = two 64-feature sub-tiles 16 KiB apart); B = V as an MN-major operand of
+// width 80 whose columns 64..79 come from the ones tile at LBO (= ones - V) bytes.
+__device__ __forceinline__ void issue_state_half(uint32_t tmem, uint32_t colS, uint32_t phik,
+                                                 uint32_t vaddr, uint32_t ones, int h, bool first)
 {
-    constexpr uint32_t idS = idesc_bf16(128, 64, 1, 1);
-    constexpr uint32_t idZ = idesc_bf16(128, 16, 1, 0);
-    for (int h = 0; h < halves; ++h) {
-        const uint32_t a0 = phik + 2 * h * kTileBytes;
+    constexpr uint32_t idS = idesc_bf16(128, 80, 1, 1);
+    const uint32_t a0 = phik + 2 * h * kTileBytes;
+    const uint32_t lbo = ones - vaddr;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t ad = sdesc(a0 + 2048 * kk, kTileBytes, 1024, kLayoutSW128);
-            const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-            umma_bf16(tmem + colS + 64 * h, ad, sdesc(vaddr + 2048 * kk, kTileBytes, 1024, kLayoutSW128),
-                      idS, acc);
-            umma_bf16(tmem + colZ + 16 * h, ad, sdesc(ones + 256 * kk, 128, 256, kLayoutNone), idZ,
-                      acc);
-        }
-    }
+    for (int kk = 0; kk < 8; ++kk)
+        umma_bf16(tmem + colS + 80 * h, sdesc(a0 + 2048 * kk, kTileBytes, 1024, kLayoutSW128),
+                  sdesc(vaddr + 2048 * kk, lbo, 1024, kLayoutSW128), idS,
+                  (first && kk == 0) ? 0u : 1u);
 }
 
 __device__ __forceinline__ void fill_ones(unsigned char* ones)
 {
     uint32_t* p = reinterpret_cast<uint32_t*>(ones);
-    for (int i = threadIdx.x; i < 1024; i += blockDim.x) p[i] = 0x3F803F80u;  // bf16 1.0 pairs
+    for (int i = threadIdx.x; i < kOnesBytes / 4; i += blockDim.x) p[i] = 0x3F803F80u;  // bf16 1.0
+}
+
+__device__ __forceinline__ unsigned char* aligned_smem(unsigned char* raw)
+{
+    return reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(raw) + 1023) &
+                                            ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ void warp_arrive(uint64_t* bar)
+{
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
 // ------------------------------------------------------------ state kernel
 // grid = BH * (nseg - 1): segment seg of sequence bh writes
 //   ws_S[bh][seg][f][e] = sum_{t in seg} phi(k_t)_f v_t[e],  ws_z[bh][seg][f] = sum phi(k_t)_f
+// Projections are 64 features wide (N = 128: two packed 32-feature operands), double
+// buffered in TMEM; epilogue group g takes the projections n with n % 2 == g.
 __global__ void __launch_bounds__(kThreads, 1)
 k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                   const __grid_constant__ CUtensorMap tmw, KParams kp, float* __restrict__ wsS,
                   float* __restrict__ wsZ, int* __restrict__ err)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char* sm = reinterpret_cast<unsigned char*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char* sm = aligned_smem(smem_raw);
     const SmemState L = smem_state_layout(kp.F);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L.bar);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L.tmem);
     const uint32_t sbase = smem_u32(sm);
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int NT = kp.F / kSlice, halves = kp.F / 128;
-    // the last segment's sum is never needed
     const Seg sg = segment_of(blockIdx.x + blockIdx.x / (kp.nseg - 1), kp.nseg, kp.ntiles);
-
-    if (warp == 0) {
+    constexpr uint32_t kColUS = 0;     // 2 x 128: projections
+    constexpr uint32_t kColSS = 256;   // 2 x 80 : [S | z]
+    // barrier roles here: QK_* hold K, V_* hold V, W_*0..1 the two operand slots,
+    // PK_FULL = all phiK of a tile written
+    if (warp == 1) {
         tmem_alloc(tslot, 512);
         tmem_relinquish();
     }
     if (tid == 0) {
         for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bar[i], 1);
+        mbar_init(&bar[B_QK_EMPTY], 1 + 8);
+        mbar_init(&bar[B_U_EMPTY0], 4);
+        mbar_init(&bar[B_U_EMPTY1], 4);
+        mbar_init(&bar[B_PK_FULL], 8);
         mbar_fence_init();
         tma_prefetch_desc(&tmk);
         tma_prefetch_desc(&tmv);
@@ -257,91 +294,149 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
-    const uint32_t trow = tmem + ((32u * warp) << 16);
+    Waiter wt;
 
-    auto load_kv = [&](int tile) {
-        mbar_arrive_expect_tx(&bar[BAR_QK], 2 * kTileBytes);
-        tma_load_3d(sm + L.k, &tmk, &bar[BAR_QK], 0, tile * kTile, sg.bh);
-        tma_load_3d(sm + L.v, &tmv, &bar[BAR_QK], 0, tile * kTile, sg.bh);
-    };
-    auto load_w = [&](int slice, int slot) {
-        mbar_arrive_expect_tx(&bar[BAR_W0 + slot], kTileBytes);
-        tma_load_2d(sm + L.w + slot * kTileBytes, &tmw, &bar[BAR_W0 + slot], 0, slice * 128);
-    };
-    if (tid == 0) {
-        load_kv(sg.t_begin);
-        for (int s = 0; s < 2 && s < NT; ++s) load_w(s, s);
-    }
-    bool ok = true;
-    uint32_t ph_kv = 0, ph_w0 = 0, ph_w1 = 0, ph_mma = 0;
-    for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
-        ok = mbar_wait(&bar[BAR_QK], ph_kv, ok ? 2000000000ull : 0) && ok;
-        ph_kv ^= 1;
-        float inv, l2i;
-        row_scale(sm + L.k + tid * 128, inv, l2i);
-        for (int t = 0; t < NT; ++t) {
-            const int slot = t & 1;
-            ok = mbar_wait(&bar[BAR_W0 + slot], slot ? ph_w1 : ph_w0, ok ? 2000000000ull : 0) && ok;
-            if (slot) ph_w1 ^= 1; else ph_w0 ^= 1;
-            if (tid == 0) {
-                tc_fence_after();
-                issue_projection(tmem, sbase + L.k, sbase + L.w + slot * kTileBytes);
-                umma_commit(&bar[BAR_MMA]);
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t ph_ke = 0, ph_ve = 0, ph_we = 0x3u;  // both operand slots start free
+            int n_glob = 0;
+            mbar_arrive_expect_tx(&bar[B_QK_FULL], kTileBytes);
+            tma_load_3d(sm + L.k, &tmk, &bar[B_QK_FULL], 0, sg.t_begin * kTile, sg.bh);
+            mbar_arrive_expect_tx(&bar[B_V_FULL], kTileBytes);
+            tma_load_3d(sm + L.v, &tmv, &bar[B_V_FULL], 0, sg.t_begin * kTile, sg.bh);
+            for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+                for (int n = 0; n < NT; ++n, ++n_glob) {
+                    const int slot = n_glob & 1;
+                    uint32_t ph = (ph_we >> slot) & 1u;
+                    wt.wait(&bar[B_W_EMPTY0 + slot], ph);
+                    ph_we ^= (1u << slot);
+                    mbar_arrive_expect_tx(&bar[B_W_FULL0 + slot], kWStateBytes);
+                    unsigned char* dst = sm + L.w + slot * kWStateBytes;
+                    tma_load_2d(dst, &tmw, &bar[B_W_FULL0 + slot], 0, (2 * n) * 64);
+                    tma_load_2d(dst + kWBytes, &tmw, &bar[B_W_FULL0 + slot], 0, (2 * n + 1) * 64);
+                    if (tile > sg.t_begin && n == 1) {   // V once the previous update is done
+                        wt.wait(&bar[B_V_EMPTY], ph_ve);
+                        mbar_arrive_expect_tx(&bar[B_V_FULL], kTileBytes);
+                        tma_load_3d(sm + L.v, &tmv, &bar[B_V_FULL], 0, tile * kTile, sg.bh);
+                    }
+                }
+                if (tile + 1 < sg.t_end) {
+                    wt.wait(&bar[B_QK_EMPTY], ph_ke);
+                    mbar_arrive_expect_tx(&bar[B_QK_FULL], kTileBytes);
+                    tma_load_3d(sm + L.k, &tmk, &bar[B_QK_FULL], 0, (tile + 1) * kTile, sg.bh);
+                }
             }
-            ok = mbar_wait(&bar[BAR_MMA], ph_mma, ok ? 2000000000ull : 0) && ok;
-            ph_mma ^= 1;
-            tc_fence_after();
-            const int node = (t * kSlice) / kp.m;
-            phi_slice_epilogue(trow, kp.a2[node] * inv, kp.b2[node] + l2i,
-                               sbase + L.phik + t * kTileBytes, tid, nullptr);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            uint32_t ph_kf = 0, ph_vf = 0, ph_wf = 0, ph_ue0 = 1, ph_ue1 = 1, ph_pk = 0;
+            int n_glob = 0;
+            constexpr uint32_t idU = idesc_bf16(128, 128, 0, 0);
+            for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+                wt.wait(&bar[B_QK_FULL], ph_kf);
+                for (int n = 0; n < NT; ++n, ++n_glob) {
+                    const int slot = n_glob & 1;
+                    uint32_t ph = (ph_wf >> slot) & 1u;
+                    wt.wait(&bar[B_W_FULL0 + slot], ph);
+                    ph_wf ^= (1u << slot);
+                    const int b = n & 1;
+                    wt.wait(&bar[B_U_EMPTY0 + b], b ? ph_ue1 : ph_ue0);
+                    tc_fence_after();
+                    const uint32_t w = sbase + L.w + slot * kWStateBytes;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_bf16(tmem + kColUS + 128 * b,
+                                  sdesc(sbase + L.k + 32 * kk, 16, 1024, kLayoutSW128),
+                                  sdesc(w + 32 * kk, 16, 1024, kLayoutSW128), idU, kk > 0 ? 1u : 0u);
+                    umma_commit(&bar[B_U_FULL0 + b]);
+                    umma_commit(&bar[B_W_EMPTY0 + slot]);
+                }
+                umma_commit(&bar[B_QK_EMPTY]);
+                wt.wait(&bar[B_PK_FULL], ph_pk);
+                wt.wait(&bar[B_V_FULL], ph_vf);
+                tc_fence_after();
+                for (int h = 0; h < halves; ++h)
+                    issue_state_half(tmem, kColSS, sbase + L.phik, sbase + L.v, sbase + L.ones, h,
+                                     tile == sg.t_begin);
+                umma_commit(&bar[B_V_EMPTY]);
+                umma_commit(&bar[B_TILE_DONE]);
+            }
+        }
+    } else if (warp < 10) {
+        const int grp = (warp >= 6) ? 1 : 0;
+        const int sp = warp & 3;
+        const uint32_t row = 32u * sp + lane;
+        const uint32_t trow = tmem + ((32u * sp) << 16);
+        uint32_t ph_kf = 0, ph_uf = 0, ph_td = 0;
+        for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+            wt.wait(&bar[B_QK_FULL], ph_kf);
+            float inv, l2i;
+            row_scale(sm + L.k + row * 128, inv, l2i);
+            warp_arrive(&bar[B_QK_EMPTY]);
+            if (tile > sg.t_begin) wt.wait(&bar[B_TILE_DONE], ph_td);  // phiK slots free again
+            for (int n = grp; n < NT; n += 2) {
+                wt.wait(&bar[B_U_FULL0 + grp], ph_uf);
+                tc_fence_after();
+                const int node = (n * kSlice) / kp.m;
+                const float a = kp.a2[node] * inv, b = kp.b2[node] + l2i;
+                const uint32_t col = kColUS + 128 * grp;
+                uint32_t ua[32], pa[32], ub[32], pb[32];
+                tmem_ld32(trow + col, ua);
+                tmem_ld32(trow + col + 32, pa);
+                tmem_ld32(trow + col + 64, ub);
+                tmem_ld32(trow + col + 96, pb);
+                tmem_wait_ld();
+                reg_fence(ua);
+                reg_fence(pa);
+                reg_fence(ub);
+                reg_fence(pb);
+                tc_fence_before();
+                warp_arrive(&bar[B_U_EMPTY0 + grp]);
+                const uint32_t tile_addr = sbase + L.phik + n * kTileBytes;
+                phi_sub_epilogue(ua, pa, a, b, tile_addr, row, 0, nullptr);
+                phi_sub_epilogue(ub, pb, a, b, tile_addr, row, 1, nullptr);
+            }
             fence_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            if (tid == 0 && t + 2 < NT) load_w(t + 2, slot);
+            warp_arrive(&bar[B_PK_FULL]);
         }
-        if (tid == 0) {
-            tc_fence_after();
-            issue_state_update(tmem, kColSA, kColZA, sbase + L.phik, sbase + L.v, sbase + L.ones,
-                               halves, tile == sg.t_begin);
-            umma_commit(&bar[BAR_MMA]);
-        }
-        ok = mbar_wait(&bar[BAR_MMA], ph_mma, ok ? 2000000000ull : 0) && ok;
-        ph_mma ^= 1;
+        // the segment's sums: group 0 writes feature half 0, group 1 half 1
+        wt.wait(&bar[B_TILE_DONE], ph_td);
         tc_fence_after();
-        if (tid == 0 && tile + 1 < sg.t_end) {
-            load_kv(tile + 1);
-            for (int s = 0; s < 2 && s < NT; ++s) load_w(s, s);
+        const size_t segidx = static_cast<size_t>(sg.bh) * kp.nseg + sg.seg;
+        for (int h = grp; h < halves; h += 2) {
+            const int f = 128 * h + row;
+            uint32_t r0[32], r1[32], zr;
+            tmem_ld32(trow + kColSS + 80 * h, r0);
+            tmem_ld32(trow + kColSS + 80 * h + 32, r1);
+            tmem_ld1(trow + kColSS + 80 * h + 64, zr);
+            tmem_wait_ld();
+            reg_fence(r0);
+            reg_fence(r1);
+            reg_fence1(zr);
+            float4* dst = reinterpret_cast<float4*>(wsS + (segidx * kp.F + f) * 64);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                dst[q] = make_float4(__uint_as_float(r0[4 * q]), __uint_as_float(r0[4 * q + 1]),
+                                     __uint_as_float(r0[4 * q + 2]), __uint_as_float(r0[4 * q + 3]));
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                dst[8 + q] = make_float4(__uint_as_float(r1[4 * q]), __uint_as_float(r1[4 * q + 1]),
+                                         __uint_as_float(r1[4 * q + 2]), __uint_as_float(r1[4 * q + 3]));
+            wsZ[segidx * kp.F + f] = __uint_as_float(zr);
         }
     }
-    // write the segment sums: thread = TMEM lane = feature within a half
-    const size_t segidx = static_cast<size_t>(sg.bh) * kp.nseg + sg.seg;
-    for (int h = 0; h < halves; ++h) {
-        const int f = 128 * h + tid;
-        uint32_t r0[32], r1[32], zr;
-        tmem_ld32(trow + kColSA + 64 * h, r0);
-        tmem_ld32(trow + kColSA + 64 * h + 32, r1);
-        tmem_ld1(trow + kColZA + 16 * h, zr);
-        tmem_wait_ld();
-        float4* dst = reinterpret_cast<float4*>(wsS + (segidx * kp.F + f) * 64);
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-            dst[q] = make_float4(__uint_as_float(r0[4 * q]), __uint_as_float(r0[4 * q + 1]),
-                                 __uint_as_float(r0[4 * q + 2]), __uint_as_float(r0[4 * q + 3]));
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-            dst[8 + q] = make_float4(__uint_as_float(r1[4 * q]), __uint_as_float(r1[4 * q + 1]),
-                                     __uint_as_float(r1[4 * q + 2]), __uint_as_float(r1[4 * q + 3]));
-        wsZ[segidx * kp.F + f] = __uint_as_float(zr);
-    }
-    if (!ok) atomicExch(err, 1);
-    drain_after_failure(ok);
+    if (!wt.ok) atomicExch(err, 1);
+    drain_after_failure(wt.ok);
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 512);
+    if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 // ----------------------------------------------------------- output kernel
 // grid = BH * nseg.  One CTA walks the tiles of one segment with the state entering it.
+// Warp 10 issues the projections (q into U0, k into U1, 32 features each); warp 1 issues the
+// score, readout, state and P.V MMAs.  Epilogue group 0 (warps 2-5): phi(q), left half of the
+// masked scores, the output.  Group 1 (warps 6-9): phi(k), right half, the state copy.
 __global__ void __launch_bounds__(kThreads, 1)
 k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                 const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmw,
@@ -349,23 +444,32 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 __nv_bfloat16* __restrict__ out, float* __restrict__ den, int* __restrict__ err)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char* sm = reinterpret_cast<unsigned char*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char* sm = aligned_smem(smem_raw);
     const SmemOut L = smem_out_layout(kp.F);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L.bar);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L.tmem);
     float* zs = reinterpret_cast<float*>(sm + L.z);
+    float* dsum = reinterpret_cast<float*>(sm + L.dsum);
     const uint32_t sbase = smem_u32(sm);
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int NT = kp.F / kSlice, halves = kp.F / 128;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int NT = kp.F / kSlice, NS = kp.F / kSub, halves = kp.F / 128;
     const Seg sg = segment_of(blockIdx.x, kp.nseg, kp.ntiles);
 
-    if (warp == 0) {
+    if (warp == 1) {
         tmem_alloc(tslot, 512);
         tmem_relinquish();
     }
     if (tid == 0) {
         for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bar[i], 1);
+        mbar_init(&bar[B_QK_EMPTY], 1 + 8);
+        mbar_init(&bar[B_U_EMPTY0], 4);
+        mbar_init(&bar[B_U_EMPTY1], 4);
+        mbar_init(&bar[B_PQ_FULL0], 4);
+        mbar_init(&bar[B_PQ_FULL1], 4);
+        mbar_init(&bar[B_PK_FULL], 4);
+        mbar_init(&bar[B_PSM_FULL], 8);
+        mbar_init(&bar[B_O_EMPTY], 4);
+        mbar_init(&bar[B_SBF_READY], 4);
         mbar_fence_init();
         tma_prefetch_desc(&tmq);
         tma_prefetch_desc(&tmk);
@@ -377,242 +481,321 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
-    const uint32_t trow = tmem + ((32u * warp) << 16);
 
-    auto load_qkv = [&](int tile) {
-        mbar_arrive_expect_tx(&bar[BAR_QK], 2 * kTileBytes);
-        tma_load_3d(sm + L.q, &tmq, &bar[BAR_QK], 0, tile * kTile, sg.bh);
-        tma_load_3d(sm + L.k, &tmk, &bar[BAR_QK], 0, tile * kTile, sg.bh);
-        mbar_arrive_expect_tx(&bar[BAR_V], kTileBytes);
-        tma_load_3d(sm + L.v, &tmv, &bar[BAR_V], 0, tile * kTile, sg.bh);
-    };
-    auto load_w = [&](int slice, int slot) {
-        mbar_arrive_expect_tx(&bar[BAR_W0 + slot], kTileBytes);
-        tma_load_2d(sm + L.w + slot * kTileBytes, &tmw, &bar[BAR_W0 + slot], 0, slice * 128);
-    };
-    if (tid == 0) {
-        load_qkv(sg.t_begin);
-        for (int s = 0; s < 2 && s < NT; ++s) load_w(s, s);
-    }
-
-    // state entering the segment: sum of the earlier segments' contributions
-    for (int h = 0; h < halves; ++h) {
-        const int f = 128 * h + tid;
-        float acc[64];
+    // state entering the segment (sum of the earlier segments), by epilogue group 1
+    if (warp >= 6 && warp < 10) {
+        const int sp = warp & 3;
+        const uint32_t row = 32u * sp + lane;
+        const uint32_t trow = tmem + ((32u * sp) << 16);
+        for (int h = 0; h < halves; ++h) {
+            const int f = 128 * h + row;
+            float acc[64];
 #pragma unroll
-        for (int e = 0; e < 64; ++e) acc[e] = 0.0f;
-        float zf = 0.0f;
-        for (int s = 0; s < sg.seg; ++s) {
-            const size_t segidx = static_cast<size_t>(sg.bh) * kp.nseg + s;
-            const float4* src = reinterpret_cast<const float4*>(wsS + (segidx * kp.F + f) * 64);
+            for (int e = 0; e < 64; ++e) acc[e] = 0.0f;
+            float zf = 0.0f;
+            for (int s = 0; s < sg.seg; ++s) {
+                const size_t segidx = static_cast<size_t>(sg.bh) * kp.nseg + s;
+                const float4* src = reinterpret_cast<const float4*>(wsS + (segidx * kp.F + f) * 64);
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const float4 x = src[q];
-                acc[4 * q] += x.x; acc[4 * q + 1] += x.y; acc[4 * q + 2] += x.z; acc[4 * q + 3] += x.w;
+                for (int q = 0; q < 16; ++q) {
+                    const float4 x = src[q];
+                    acc[4 * q] += x.x; acc[4 * q + 1] += x.y; acc[4 * q + 2] += x.z; acc[4 * q + 3] += x.w;
+                }
+                zf += wsZ[segidx * kp.F + f];
             }
-            zf += wsZ[segidx * kp.F + f];
+            uint32_t r[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(acc[e]);
+            tmem_st32(trow + kColS + 80 * h, r);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(acc[32 + e]);
+            tmem_st32(trow + kColS + 80 * h + 32, r);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(zf);
+            tmem_st32(trow + kColS + 80 * h + 64, r);  // z columns (a later half rewrites its own)
+            uint32_t pk[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) pk[e] = pack_bf16(acc[2 * e], acc[2 * e + 1]);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                st_shared_v4(sbase + L.sbf + sw128_off(f, q), pk[4 * q], pk[4 * q + 1],
+                             pk[4 * q + 2], pk[4 * q + 3]);
+            zs[f] = zf;
         }
-        uint32_t r[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(acc[e]);
-        tmem_st32(trow + kColS + 64 * h, r);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(acc[32 + e]);
-        tmem_st32(trow + kColS + 64 * h + 32, r);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(e == 0 ? zf : 0.0f);
-        tmem_st32(trow + kColZ + 16 * h, r);  // columns z_h .. z_h+31 (z_{h+1} is rewritten next)
-        uint32_t pk[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16(acc[2 * e], acc[2 * e + 1]);
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-            st_shared_v4(sbase + L.sbf + sw128_off(f, q), pk[4 * q], pk[4 * q + 1], pk[4 * q + 2],
-                         pk[4 * q + 3]);
-        zs[f] = zf;
+        tmem_wait_st();
     }
-    tmem_wait_st();
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
 
-    bool ok = true;
-    uint32_t ph_qk = 0, ph_v = 0, ph_w0 = 0, ph_w1 = 0, ph_mma = 0;
+    Waiter wt;
     const int64_t rowbase = static_cast<int64_t>(sg.bh) * kp.L;
-    for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
-        ok = mbar_wait(&bar[BAR_QK], ph_qk, ok ? 2000000000ull : 0) && ok;
-        ph_qk ^= 1;
-        float invq, l2q, invk, l2k;
-        row_scale(sm + L.q + tid * 128, invq, l2q);
-        row_scale(sm + L.k + tid * 128, invk, l2k);
-        float den_inter = 0.0f;
-        for (int t = 0; t < NT; ++t) {
-            const int slot = t & 1;
-            const uint32_t waddr = sbase + L.w + slot * kTileBytes;
-            ok = mbar_wait(&bar[BAR_W0 + slot], slot ? ph_w1 : ph_w0, ok ? 2000000000ull : 0) && ok;
-            if (slot) ph_w1 ^= 1; else ph_w0 ^= 1;
-            const int node = (t * kSlice) / kp.m;
-            // q projection -> phiQ_t
-            if (tid == 0) {
-                tc_fence_after();
-                issue_projection(tmem, sbase + L.q, waddr);
-                umma_commit(&bar[BAR_MMA]);
-            }
-            ok = mbar_wait(&bar[BAR_MMA], ph_mma, ok ? 2000000000ull : 0) && ok;
-            ph_mma ^= 1;
-            tc_fence_after();
-            den_inter += phi_slice_epilogue(trow, kp.a2[node] * invq, kp.b2[node] + l2q,
-                                            sbase + L.phiq, tid, zs + t * kSlice);
-            fence_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            // k projection -> phiK_t
-            if (tid == 0) {
-                tc_fence_after();
-                issue_projection(tmem, sbase + L.k, waddr);
-                umma_commit(&bar[BAR_MMA]);
-            }
-            ok = mbar_wait(&bar[BAR_MMA], ph_mma, ok ? 2000000000ull : 0) && ok;
-            ph_mma ^= 1;
-            tc_fence_after();
-            phi_slice_epilogue(trow, kp.a2[node] * invk, kp.b2[node] + l2k,
-                               sbase + L.phik + t * kTileBytes, tid, nullptr);
-            fence_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            // P += phiQ_t phiK_t^T ; O += phiQ_t S_t
-            if (tid == 0) {
-                tc_fence_after();
-                constexpr uint32_t idP = idesc_bf16(128, 128, 0, 0);
-                constexpr uint32_t idO = idesc_bf16(128, 64, 0, 1);
-                const uint32_t aq = sbase + L.phiq;
-                const uint32_t bk = sbase + L.phik + t * kTileBytes;
-                const uint32_t bs = sbase + L.sbf + t * kSlice * 128;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-                    const uint64_t ad = sdesc(aq + 32 * kk, 16, 1024, kLayoutSW128);
-                    umma_bf16(tmem + kColP, ad, sdesc(bk + 32 * kk, 16, 1024, kLayoutSW128), idP, acc);
-                    umma_bf16(tmem + kColO, ad, sdesc(bs + 2048 * kk, kTileBytes, 1024, kLayoutSW128),
-                              idO, acc);
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA
+        if (lane == 0) {
+            uint32_t ph_qke = 0, ph_ve = 0, ph_we = (1u << kWSlots) - 1u;
+            int n_glob = 0;
+            const int vpoint = (NS < kWSlots ? NS : kWSlots) - 1;
+            mbar_arrive_expect_tx(&bar[B_QK_FULL], 2 * kTileBytes);
+            tma_load_3d(sm + L.q, &tmq, &bar[B_QK_FULL], 0, sg.t_begin * kTile, sg.bh);
+            tma_load_3d(sm + L.k, &tmk, &bar[B_QK_FULL], 0, sg.t_begin * kTile, sg.bh);
+            mbar_arrive_expect_tx(&bar[B_V_FULL], kTileBytes);
+            tma_load_3d(sm + L.v, &tmv, &bar[B_V_FULL], 0, sg.t_begin * kTile, sg.bh);
+            for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+                for (int n = 0; n < NS; ++n, ++n_glob) {
+                    const int slot = n_glob % kWSlots;
+                    uint32_t ph = (ph_we >> slot) & 1u;
+                    wt.wait(&bar[B_W_EMPTY0 + slot], ph);
+                    ph_we ^= (1u << slot);
+                    mbar_arrive_expect_tx(&bar[B_W_FULL0 + slot], kWBytes);
+                    tma_load_2d(sm + L.w + slot * kWBytes, &tmw, &bar[B_W_FULL0 + slot], 0, n * 64);
+                    // V of this tile once the previous tile's P.V and state update are done
+                    if (tile > sg.t_begin && n == vpoint) {
+                        wt.wait(&bar[B_V_EMPTY], ph_ve);
+                        mbar_arrive_expect_tx(&bar[B_V_FULL], kTileBytes);
+                        tma_load_3d(sm + L.v, &tmv, &bar[B_V_FULL], 0, tile * kTile, sg.bh);
+                    }
                 }
-                umma_commit(&bar[BAR_MMA]);
+                if (tile + 1 < sg.t_end) {
+                    wt.wait(&bar[B_QK_EMPTY], ph_qke);
+                    mbar_arrive_expect_tx(&bar[B_QK_FULL], 2 * kTileBytes);
+                    tma_load_3d(sm + L.q, &tmq, &bar[B_QK_FULL], 0, (tile + 1) * kTile, sg.bh);
+                    tma_load_3d(sm + L.k, &tmk, &bar[B_QK_FULL], 0, (tile + 1) * kTile, sg.bh);
+                }
             }
-            ok = mbar_wait(&bar[BAR_MMA], ph_mma, ok ? 2000000000ull : 0) && ok;
-            ph_mma ^= 1;
-            tc_fence_after();
-            if (tid == 0 && t + 2 < NT) load_w(t + 2, slot);
         }
-        // state update (asynchronous) while the masked scores are formed
-        ok = mbar_wait(&bar[BAR_V], ph_v, ok ? 2000000000ull : 0) && ok;
-        ph_v ^= 1;
-        if (tid == 0) {
-            tc_fence_after();
-            issue_state_update(tmem, kColS, kColZ, sbase + L.phik, sbase + L.v, sbase + L.ones,
-                               halves, false);
-        }
-        // P epilogue: mask j <= i, row sum, bf16 into the Q/K tile space (K-major, K = 128)
-        float den_intra = 0.0f;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            uint32_t pr[32];
-            tmem_ld32(trow + kColP + 32 * c, pr);
-            tmem_wait_ld();
-            uint32_t pk[16];
-#pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-                const int col = 32 * c + j;
-                const float x0 = (col <= tid) ? __uint_as_float(pr[j]) : 0.0f;
-                const float x1 = (col + 1 <= tid) ? __uint_as_float(pr[j + 1]) : 0.0f;
-                den_intra += x0 + x1;
-                pk[j >> 1] = pack_bf16(x0, x1);
+    } else if (warp == 10) {
+        // --------------------------------------------------- projection issuer
+        if (lane == 0) {
+            uint32_t ph_qkf = 0, ph_wf = 0, ph_ue0 = 1, ph_ue1 = 1;
+            int n_glob = 0;
+            for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+                wt.wait(&bar[B_QK_FULL], ph_qkf);
+                for (int n = 0; n < NS; ++n, ++n_glob) {
+                    const int slot = n_glob % kWSlots;
+                    uint32_t ph = (ph_wf >> slot) & 1u;
+                    wt.wait(&bar[B_W_FULL0 + slot], ph);
+                    ph_wf ^= (1u << slot);
+                    const uint32_t waddr = sbase + L.w + slot * kWBytes;
+                    wt.wait(&bar[B_U_EMPTY0], ph_ue0);
+                    tc_fence_after();
+                    issue_projection(tmem + kColU0, sbase + L.q, waddr);
+                    umma_commit(&bar[B_U_FULL0]);
+                    wt.wait(&bar[B_U_EMPTY1], ph_ue1);
+                    tc_fence_after();
+                    issue_projection(tmem + kColU1, sbase + L.k, waddr);
+                    umma_commit(&bar[B_U_FULL1]);
+                    umma_commit(&bar[B_W_EMPTY0 + slot]);
+                }
+                umma_commit(&bar[B_QK_EMPTY]);
             }
-            const uint32_t base = sbase + ((c < 2) ? L.q : L.k);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                st_shared_v4(base + sw128_off(tid, 4 * (c & 1) + q), pk[4 * q], pk[4 * q + 1],
-                             pk[4 * q + 2], pk[4 * q + 3]);
         }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after();
+    } else if (warp == 1) {
+        // ------------------------------------------------------ main MMA issuer
+        if (lane == 0) {
+            uint32_t ph_vf = 0, ph_pqf0 = 0, ph_pqf1 = 0, ph_pkf = 0, ph_psm = 0, ph_oe = 0,
+                     ph_sbf = 0;
+            constexpr uint32_t idP = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t idO = idesc_bf16(128, 64, 0, 1);
+            for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+                const bool last = tile + 1 == sg.t_end;
+                for (int t = 0; t < NT; ++t) {
+                    const int pslot = t & 1;
+                    wt.wait(&bar[B_PQ_FULL0 + pslot], pslot ? ph_pqf1 : ph_pqf0);
+                    wt.wait(&bar[B_PK_FULL], ph_pkf);
+                    if (t == 0 && tile > sg.t_begin) {
+                        wt.wait(&bar[B_SBF_READY], ph_sbf);
+                        wt.wait(&bar[B_O_EMPTY], ph_oe);
+                    }
+                    tc_fence_after();
+                    const uint32_t aq = sbase + L.phiq + pslot * kTileBytes;
+                    const uint32_t bk = sbase + L.phik + t * kTileBytes;
+                    const uint32_t bs = sbase + L.sbf + t * kSlice * 128;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t a = sbase + ((kk < 4) ? L.q : L.k) + 32 * (kk & 3);
-                umma_bf16(tmem + kColO, sdesc(a, 16, 1024, kLayoutSW128),
-                          sdesc(sbase + L.v + 2048 * kk, kTileBytes, 1024, kLayoutSW128), idO, 1u);
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+                        const uint64_t ad = sdesc(aq + 32 * kk, 16, 1024, kLayoutSW128);
+                        umma_bf16(tmem + kColP, ad, sdesc(bk + 32 * kk, 16, 1024, kLayoutSW128), idP, acc);
+                        umma_bf16(tmem + kColO, ad,
+                                  sdesc(bs + 2048 * kk, kTileBytes, 1024, kLayoutSW128), idO, acc);
+                    }
+                    umma_commit(&bar[B_PQ_EMPTY0 + pslot]);
+                    // state update of a feature half once its phiK slices are in place
+                    if (!last && (t & 1) == 1) {
+                        if (t == 1) wt.wait(&bar[B_V_FULL], ph_vf);
+                        issue_state_half(tmem, kColS, sbase + L.phik, sbase + L.v, sbase + L.ones,
+                                         t >> 1, false);
+                    }
+                }
+                umma_commit(&bar[B_P_FULL]);
+                if (last) wt.wait(&bar[B_V_FULL], ph_vf);
+                wt.wait(&bar[B_PSM_FULL], ph_psm);
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t a = sbase + L.phiq + (kk >> 2) * kTileBytes + 32 * (kk & 3);
+                    umma_bf16(tmem + kColO, sdesc(a, 16, 1024, kLayoutSW128),
+                              sdesc(sbase + L.v + 2048 * kk, kTileBytes, 1024, kLayoutSW128), idO, 1u);
+                }
+                umma_commit(&bar[B_TILE_DONE]);
+                umma_commit(&bar[B_V_EMPTY]);
             }
-            umma_commit(&bar[BAR_MMA]);
         }
-        ok = mbar_wait(&bar[BAR_MMA], ph_mma, ok ? 2000000000ull : 0) && ok;
-        ph_mma ^= 1;
-        tc_fence_after();
-        if (tid == 0 && tile + 1 < sg.t_end) {
-            load_qkv(tile + 1);
-            for (int s = 0; s < 2 && s < NT; ++s) load_w(s, s);
-        }
-        // output epilogue
-        {
-            uint32_t o0[32], o1[32];
-            tmem_ld32(trow + kColO, o0);
-            tmem_ld32(trow + kColO + 32, o1);
-            tmem_wait_ld();
-            const float d = den_intra + den_inter;
-            const float rz = 1.0f / (d + kp.eps);
-            const int row = tile * kTile + tid;
-            if (row < kp.L) {
-                uint4* dst = reinterpret_cast<uint4*>(out + (rowbase + row) * 64);
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    dst[q] = make_uint4(pack_bf16(__uint_as_float(o0[8 * q]) * rz, __uint_as_float(o0[8 * q + 1]) * rz),
-                                        pack_bf16(__uint_as_float(o0[8 * q + 2]) * rz, __uint_as_float(o0[8 * q + 3]) * rz),
-                                        pack_bf16(__uint_as_float(o0[8 * q + 4]) * rz, __uint_as_float(o0[8 * q + 5]) * rz),
-                                        pack_bf16(__uint_as_float(o0[8 * q + 6]) * rz, __uint_as_float(o0[8 * q + 7]) * rz));
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    dst[4 + q] = make_uint4(pack_bf16(__uint_as_float(o1[8 * q]) * rz, __uint_as_float(o1[8 * q + 1]) * rz),
-                                            pack_bf16(__uint_as_float(o1[8 * q + 2]) * rz, __uint_as_float(o1[8 * q + 3]) * rz),
-                                            pack_bf16(__uint_as_float(o1[8 * q + 4]) * rz, __uint_as_float(o1[8 * q + 5]) * rz),
-                                            pack_bf16(__uint_as_float(o1[8 * q + 6]) * rz, __uint_as_float(o1[8 * q + 7]) * rz));
-                if (den) den[rowbase + row] = d;
+    } else {
+        // ----------------------------------------------------------- epilogues
+        const int grp = (warp >= 6) ? 1 : 0;
+        const int sp = warp & 3;
+        const uint32_t row = 32u * sp + lane;
+        const uint32_t trow = tmem + ((32u * sp) << 16);
+        uint32_t ph_qkf = 0, ph_uf = 0, ph_pqe0 = 0, ph_pqe1 = 0, ph_pf = 0, ph_psm = 0, ph_td = 0,
+                 ph_sbf = 0;
+        int uses0 = 0, uses1 = 0;
+        for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+            wt.wait(&bar[B_QK_FULL], ph_qkf);
+            float inv, l2i;
+            row_scale(sm + (grp ? L.k : L.q) + row * 128, inv, l2i);
+            warp_arrive(&bar[B_QK_EMPTY]);
+            if (grp == 0 && tile > sg.t_begin) wt.wait(&bar[B_SBF_READY], ph_sbf);  // zs of this tile
+            float den_inter = 0.0f;
+            for (int t = 0; t < NT; ++t) {
+                const int node = (t * kSlice) / kp.m;
+                const float a = kp.a2[node] * inv, b = kp.b2[node] + l2i;
+                const int pslot = t & 1;
+                for (int half = 0; half < 2; ++half) {
+                    wt.wait(&bar[B_U_FULL0 + grp], ph_uf);
+                    tc_fence_after();
+                    uint32_t ur[32], pr[32];
+                    const uint32_t col = grp ? kColU1 : kColU0;
+                    tmem_ld32(trow + col, ur);
+                    tmem_ld32(trow + col + 32, pr);
+                    tmem_wait_ld();
+                    reg_fence(ur);
+                    reg_fence(pr);
+                    tc_fence_before();
+                    warp_arrive(&bar[B_U_EMPTY0 + grp]);
+                    if (grp == 0) {
+                        if (half == 0) {
+                            int& uses = pslot ? uses1 : uses0;
+                            if (uses > 0) wt.wait(&bar[B_PQ_EMPTY0 + pslot], pslot ? ph_pqe1 : ph_pqe0);
+                            ++uses;
+                        }
+                        den_inter += phi_sub_epilogue(ur, pr, a, b,
+                                                      sbase + L.phiq + pslot * kTileBytes, row, half,
+                                                      zs + t * kSlice + half * kSub);
+                    } else {
+                        phi_sub_epilogue(ur, pr, a, b, sbase + L.phik + t * kTileBytes, row, half,
+                                         nullptr);
+                    }
+                }
+                fence_async_smem();
+                warp_arrive(&bar[grp ? B_PK_FULL : (B_PQ_FULL0 + pslot)]);
             }
-        }
-        // state after the tile -> bf16 operand copy and fp32 z
-        if (tile + 1 < sg.t_end) {
-            for (int h = 0; h < halves; ++h) {
-                const int f = 128 * h + tid;
-                uint32_t r0[32], r1[32], zr;
-                tmem_ld32(trow + kColS + 64 * h, r0);
-                tmem_ld32(trow + kColS + 64 * h + 32, r1);
-                tmem_ld1(trow + kColZ + 16 * h, zr);
+            // masked scores into the phi(q) buffers: group 0 columns 0..63, group 1 64..127
+            wt.wait(&bar[B_P_FULL], ph_pf);
+            tc_fence_after();
+            float dpart = 0.0f;
+            {
+                uint32_t p0[32], p1[32];
+                tmem_ld32(trow + kColP + 64 * grp, p0);
+                tmem_ld32(trow + kColP + 64 * grp + 32, p1);
                 tmem_wait_ld();
+                reg_fence(p0);
+                reg_fence(p1);
                 uint32_t pk[32];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    pk[e] = pack_bf16(__uint_as_float(r0[2 * e]), __uint_as_float(r0[2 * e + 1]));
-                    pk[16 + e] = pack_bf16(__uint_as_float(r1[2 * e]), __uint_as_float(r1[2 * e + 1]));
+                for (int j = 0; j < 32; j += 2) {
+                    const uint32_t c0 = 64u * grp + j;
+                    const float x0 = (c0 <= row) ? __uint_as_float(p0[j]) : 0.0f;
+                    const float x1 = (c0 + 1 <= row) ? __uint_as_float(p0[j + 1]) : 0.0f;
+                    const float y0 = (c0 + 32 <= row) ? __uint_as_float(p1[j]) : 0.0f;
+                    const float y1 = (c0 + 33 <= row) ? __uint_as_float(p1[j + 1]) : 0.0f;
+                    dpart += (x0 + x1) + (y0 + y1);
+                    pk[j >> 1] = pack_bf16(x0, x1);
+                    pk[16 + (j >> 1)] = pack_bf16(y0, y1);
                 }
+                const uint32_t base = sbase + L.phiq + grp * kTileBytes;
 #pragma unroll
                 for (int q = 0; q < 8; ++q)
-                    st_shared_v4(sbase + L.sbf + sw128_off(f, q), pk[4 * q], pk[4 * q + 1],
-                                 pk[4 * q + 2], pk[4 * q + 3]);
-                zs[f] = __uint_as_float(zr);
+                    st_shared_v4(base + sw128_off(row, q), pk[4 * q], pk[4 * q + 1], pk[4 * q + 2],
+                                 pk[4 * q + 3]);
+            }
+            if (grp == 1) dsum[row] = dpart;
+            fence_async_smem();
+            tc_fence_before();
+            warp_arrive(&bar[B_PSM_FULL]);
+            if (grp == 0) {
+                wt.wait(&bar[B_PSM_FULL], ph_psm);  // group 1's partial sums are in dsum
+                wt.wait(&bar[B_TILE_DONE], ph_td);
+                tc_fence_after();
+                uint32_t o0[32], o1[32];
+                tmem_ld32(trow + kColO, o0);
+                tmem_ld32(trow + kColO + 32, o1);
+                tmem_wait_ld();
+                reg_fence(o0);
+                reg_fence(o1);
+                tc_fence_before();
+                warp_arrive(&bar[B_O_EMPTY]);
+                const float d = dpart + dsum[row] + den_inter;
+                const float rz = 1.0f / (d + kp.eps);
+                const int grow = tile * kTile + static_cast<int>(row);
+                if (grow < kp.L) {
+                    uint4* dst = reinterpret_cast<uint4*>(out + (rowbase + grow) * 64);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        dst[q] = make_uint4(
+                            pack_bf16(__uint_as_float(o0[8 * q]) * rz, __uint_as_float(o0[8 * q + 1]) * rz),
+                            pack_bf16(__uint_as_float(o0[8 * q + 2]) * rz, __uint_as_float(o0[8 * q + 3]) * rz),
+                            pack_bf16(__uint_as_float(o0[8 * q + 4]) * rz, __uint_as_float(o0[8 * q + 5]) * rz),
+                            pack_bf16(__uint_as_float(o0[8 * q + 6]) * rz, __uint_as_float(o0[8 * q + 7]) * rz));
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        dst[4 + q] = make_uint4(
+                            pack_bf16(__uint_as_float(o1[8 * q]) * rz, __uint_as_float(o1[8 * q + 1]) * rz),
+                            pack_bf16(__uint_as_float(o1[8 * q + 2]) * rz, __uint_as_float(o1[8 * q + 3]) * rz),
+                            pack_bf16(__uint_as_float(o1[8 * q + 4]) * rz, __uint_as_float(o1[8 * q + 5]) * rz),
+                            pack_bf16(__uint_as_float(o1[8 * q + 6]) * rz, __uint_as_float(o1[8 * q + 7]) * rz));
+                    if (den) den[rowbase + grow] = d;
+                }
+            } else {
+                wt.wait(&bar[B_TILE_DONE], ph_td);
+                tc_fence_after();
+                if (tile + 1 < sg.t_end) {
+                    // state after this tile -> bf16 operand copy and fp32 z
+                    for (int h = 0; h < halves; ++h) {
+                        const int f = 128 * h + row;
+                        uint32_t r0s[32], r1s[32], zr;
+                        tmem_ld32(trow + kColS + 80 * h, r0s);
+                        tmem_ld32(trow + kColS + 80 * h + 32, r1s);
+                        tmem_ld1(trow + kColS + 80 * h + 64, zr);
+                        tmem_wait_ld();
+                        reg_fence(r0s);
+                        reg_fence(r1s);
+                        reg_fence1(zr);
+                        uint32_t pk[32];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            pk[e] = pack_bf16(__uint_as_float(r0s[2 * e]), __uint_as_float(r0s[2 * e + 1]));
+                            pk[16 + e] = pack_bf16(__uint_as_float(r1s[2 * e]), __uint_as_float(r1s[2 * e + 1]));
+                        }
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            st_shared_v4(sbase + L.sbf + sw128_off(f, q), pk[4 * q], pk[4 * q + 1],
+                                         pk[4 * q + 2], pk[4 * q + 3]);
+                        zs[f] = __uint_as_float(zr);
+                    }
+                    fence_async_smem();
+                    tc_fence_before();
+                    warp_arrive(&bar[B_SBF_READY]);
+                }
             }
         }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
     }
-    if (!ok) atomicExch(err, 1);
-    drain_after_failure(ok);
+    if (!wt.ok) atomicExch(err, 1);
+    drain_after_failure(wt.ok);
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 512);
+    if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 // ------------------------------------------------------------------ host side
@@ -651,15 +834,15 @@ bool map_rows(CUtensorMap* m, const void* base, int L, int BH)
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// packed projection operand [F/64][128][64] bf16: per 64-feature slice, 64 omega rows then
-// 64 anchor rows, each row the 64 input dimensions.
+// packed projection operand [F/32][64][64] bf16: per 32-feature sub-slice, 32 omega rows
+// then 32 anchor rows, each row the 64 input dimensions.
 bool map_w(CUtensorMap* m, const void* base, int F)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
-    const cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(F / kSlice) * 128};
+    const cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(F / kSub) * 64};
     const cuuint64_t strides[1] = {128};
-    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t box[2] = {64, 64};
     const cuuint32_t es[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
               es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -707,11 +890,11 @@ size_t tc_wb_elems(int D, int R, int m)
 void tc_pack_wb(int D, int R, int m, const uint16_t* om, const uint16_t* an, uint16_t* wb)
 {
     const int F = R * m;
-    for (int t = 0; t < F / kSlice; ++t)
-        for (int r = 0; r < 128; ++r) {
-            const int f = t * kSlice + (r & 63);
-            const uint16_t* src = (r < 64) ? om : an;
-            std::memcpy(wb + (static_cast<size_t>(t) * 128 + r) * D, src + static_cast<size_t>(f) * D,
+    for (int n = 0; n < F / kSub; ++n)
+        for (int r = 0; r < 64; ++r) {
+            const int f = n * kSub + (r & 31);
+            const uint16_t* src = (r < 32) ? om : an;
+            std::memcpy(wb + (static_cast<size_t>(n) * 64 + r) * D, src + static_cast<size_t>(f) * D,
                         D * sizeof(uint16_t));
         }
 }
