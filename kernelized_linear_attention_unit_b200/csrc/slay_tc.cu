@@ -19,10 +19,12 @@
 // of the earlier segments' contributions and produces the outputs.  Neither kernel waits on
 // another CTA.
 //
-// Both kernels are warp-specialised: warp 0 issues TMA copies, warps 1 and 10 issue
+// Both kernels are warp-specialised: warp 0 issues TMA copies, warps 1, 10 and 11 issue
 // tcgen05 MMAs (one elected thread each: the issue rate of a single thread, not the tensor
 // pipe, limits narrow MMAs), warps 2-5 and 6-9 are two epilogue groups (one row of a 128-row
-// tile per thread, one TMEM lane each).  Hand-offs go through mbarriers.  Every wait is
+// tile per thread, one TMEM lane each).  In the output kernel the denominator is an extra
+// accumulator column: O = [P | phiQ] . [[V | 1]; [S | z]], so no per-element dot product
+// with z is needed and the phi(q) group never waits for the end of a tile.  Hand-offs go through mbarriers.  Every wait is
 // bounded in time; a timeout sets an error word in the workspace header, later waits give
 // up at once, and the CTA drains before releasing its memory.
 #include <cuda.h>
@@ -48,7 +50,7 @@ constexpr int kSub = 32;                   // features per projection (N = 64 wi
 constexpr int kTileBytes = kTile * 128;    // one [128 rows][64 bf16] swizzled tile = 16 KiB
 constexpr int kWBytes = 64 * 128;          // one projection operand [64 rows][64 bf16] = 8 KiB
 constexpr int kWSlots = 3;                 // output kernel: 3 x 8 KiB projection operands
-constexpr int kThreads = 352;              // 11 warps
+constexpr int kThreads = 384;              // 12 warps
 constexpr int kOnesBytes = kTileBytes;     // [128][64] bf16 ones: the z columns of [V | 1]
 constexpr size_t kWsHeader = 256;          // error word + padding at the start of the workspace
 constexpr int kNumSMs = 148;
@@ -58,8 +60,9 @@ constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint32_t kColU0 = 0;     // 64: q-side projection (32 u | 32 p)
 constexpr uint32_t kColU1 = 64;    // 64: k-side projection
 constexpr uint32_t kColP = 128;    // 128: intra-tile scores
-constexpr uint32_t kColO = 256;    // 64 : output numerator
-constexpr uint32_t kColS = 320;    // 2 x 80: state [S | z], feature halves (z in column 64)
+constexpr uint32_t kColO = 256;    // 80 : output [numerator | denominator] (denominator column 64)
+constexpr uint32_t kColS = 336;    // 2 x 80: state [S | z], feature halves (z in column 64)
+constexpr int kStBytes = 80 * 128; // [S | z] rows of one 64-feature slice: 80 columns x 64 features bf16
 
 // -------------------------------------------------------------- barriers
 enum {
@@ -73,10 +76,12 @@ enum {
 };
 
 struct SmemOut {
-    uint32_t w, q, k, v, phik, phiq, sbf, ones, z, dsum, bar, tmem, total;
+    uint32_t w, q, k, v, ones, phik, phiq, st, bar, tmem, total;
 };
 
-// Output kernel: the masked scores P (two [128][64] tiles) reuse the phi(q) double buffer.
+// Output kernel: st = the state entering the tile in bf16, [S | z | 0] with 80 columns, as
+// the B operand of the readout (MN-major, no swizzle: 8x8 core matrices, K groups of 8
+// features 128 bytes apart, N groups of 8 columns F*16 bytes apart).
 __host__ __device__ inline SmemOut smem_out_layout(int F)
 {
     SmemOut s;
@@ -87,10 +92,8 @@ __host__ __device__ inline SmemOut smem_out_layout(int F)
     s.ones = s.v + kTileBytes;                         // right after V: fixed offset from it
     s.phik = s.ones + kOnesBytes;
     s.phiq = s.phik + (F / kSlice) * kTileBytes;
-    s.sbf = s.phiq + 2 * kTileBytes;
-    s.z = s.sbf + F * 128;
-    s.dsum = s.z + F * 4;
-    s.bar = s.dsum + kTile * 4;
+    s.st = s.phiq + 2 * kTileBytes;
+    s.bar = s.st + (F / kSlice) * kStBytes;
     s.tmem = s.bar + NUM_BARS * 8;
     s.total = s.tmem + 16;
     return s;
@@ -433,10 +436,26 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
 }
 
 // ----------------------------------------------------------- output kernel
+// Row f of the state copy [S | z]: columns 0..63 = S[f][:], column 64 = z[f], 65..71 = 0, in
+// the no-swizzle MN-major layout (core matrix (n/8, f/8), row f%8, 16 bytes per row).
+// Nine 16-byte stores; a warp's 32 consecutive features fill 512 contiguous bytes.
+__device__ __forceinline__ void write_state_row(uint32_t st, int F, int f, const float* s, float z)
+{
+    const uint32_t base = st + (f >> 3) * 128 + (f & 7) * 16;
+    const uint32_t sbo = static_cast<uint32_t>(F) * 16;
+#pragma unroll
+    for (int g = 0; g < 8; ++g)
+        st_shared_v4(base + g * sbo, pack_bf16(s[8 * g], s[8 * g + 1]), pack_bf16(s[8 * g + 2], s[8 * g + 3]),
+                     pack_bf16(s[8 * g + 4], s[8 * g + 5]), pack_bf16(s[8 * g + 6], s[8 * g + 7]));
+    st_shared_v4(base + 8 * sbo, pack_bf16(z, 0.0f), 0u, 0u, 0u);
+}
+
 // grid = BH * nseg.  One CTA walks the tiles of one segment with the state entering it.
-// Warp 10 issues the projections (q into U0, k into U1, 32 features each); warp 1 issues the
-// score, readout, state and P.V MMAs.  Epilogue group 0 (warps 2-5): phi(q), left half of the
-// masked scores, the output.  Group 1 (warps 6-9): phi(k), right half, the state copy.
+// Warps 10 / 11 issue the q / k projections (32 features each) into U0 / U1; warp 1 issues
+// the score, readout, state and P.V MMAs.  Epilogue group 0 (warps 2-5) turns q projections
+// into phi(q); group 1 (warps 6-9) turns k projections into phi(k) and then does the end of
+// the tile: the masked scores (bf16, in place in tensor memory), the output and the state
+// copy for the next tile.
 __global__ void __launch_bounds__(kThreads, 1)
 k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                 const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmw,
@@ -448,8 +467,6 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
     const SmemOut L = smem_out_layout(kp.F);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L.bar);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L.tmem);
-    float* zs = reinterpret_cast<float*>(sm + L.z);
-    float* dsum = reinterpret_cast<float*>(sm + L.dsum);
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int NT = kp.F / kSlice, NS = kp.F / kSub, halves = kp.F / 128;
@@ -461,13 +478,14 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
     }
     if (tid == 0) {
         for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bar[i], 1);
-        mbar_init(&bar[B_QK_EMPTY], 1 + 8);
+        mbar_init(&bar[B_QK_EMPTY], 2 + 8);
+        for (int s = 0; s < kWSlots; ++s) mbar_init(&bar[B_W_EMPTY0 + s], 2);
         mbar_init(&bar[B_U_EMPTY0], 4);
         mbar_init(&bar[B_U_EMPTY1], 4);
         mbar_init(&bar[B_PQ_FULL0], 4);
         mbar_init(&bar[B_PQ_FULL1], 4);
         mbar_init(&bar[B_PK_FULL], 4);
-        mbar_init(&bar[B_PSM_FULL], 8);
+        mbar_init(&bar[B_PSM_FULL], 4);
         mbar_init(&bar[B_O_EMPTY], 4);
         mbar_init(&bar[B_SBF_READY], 4);
         mbar_fence_init();
@@ -477,6 +495,10 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         tma_prefetch_desc(&tmw);
     }
     fill_ones(sm + L.ones);
+    {   // the state copy: columns 65..79 stay zero
+        uint4* p = reinterpret_cast<uint4*>(sm + L.st);
+        for (int i = tid; i < NT * kStBytes / 16; i += kThreads) p[i] = make_uint4(0, 0, 0, 0);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -513,14 +535,7 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
 #pragma unroll
             for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(zf);
             tmem_st32(trow + kColS + 80 * h + 64, r);  // z columns (a later half rewrites its own)
-            uint32_t pk[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) pk[e] = pack_bf16(acc[2 * e], acc[2 * e + 1]);
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                st_shared_v4(sbase + L.sbf + sw128_off(f, q), pk[4 * q], pk[4 * q + 1],
-                             pk[4 * q + 2], pk[4 * q + 3]);
-            zs[f] = zf;
+            write_state_row(sbase + L.st, kp.F, f, acc, zf);
         }
         tmem_wait_st();
     }
@@ -565,10 +580,12 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 }
             }
         }
-    } else if (warp == 10) {
-        // --------------------------------------------------- projection issuer
+    } else if (warp >= 10) {
+        // ------------------------------------------ projection issuers (q: 10, k: 11)
         if (lane == 0) {
-            uint32_t ph_qkf = 0, ph_wf = 0, ph_ue0 = 1, ph_ue1 = 1;
+            const int g = warp - 10;
+            const uint32_t xaddr = sbase + (g ? L.k : L.q);
+            uint32_t ph_qkf = 0, ph_wf = 0, ph_ue = 1;
             int n_glob = 0;
             for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
                 wt.wait(&bar[B_QK_FULL], ph_qkf);
@@ -577,15 +594,10 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                     uint32_t ph = (ph_wf >> slot) & 1u;
                     wt.wait(&bar[B_W_FULL0 + slot], ph);
                     ph_wf ^= (1u << slot);
-                    const uint32_t waddr = sbase + L.w + slot * kWBytes;
-                    wt.wait(&bar[B_U_EMPTY0], ph_ue0);
+                    wt.wait(&bar[B_U_EMPTY0 + g], ph_ue);
                     tc_fence_after();
-                    issue_projection(tmem + kColU0, sbase + L.q, waddr);
-                    umma_commit(&bar[B_U_FULL0]);
-                    wt.wait(&bar[B_U_EMPTY1], ph_ue1);
-                    tc_fence_after();
-                    issue_projection(tmem + kColU1, sbase + L.k, waddr);
-                    umma_commit(&bar[B_U_FULL1]);
+                    issue_projection(tmem + (g ? kColU1 : kColU0), xaddr, sbase + L.w + slot * kWBytes);
+                    umma_commit(&bar[B_U_FULL0 + g]);
                     umma_commit(&bar[B_W_EMPTY0 + slot]);
                 }
                 umma_commit(&bar[B_QK_EMPTY]);
@@ -597,7 +609,8 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             uint32_t ph_vf = 0, ph_pqf0 = 0, ph_pqf1 = 0, ph_pkf = 0, ph_psm = 0, ph_oe = 0,
                      ph_sbf = 0;
             constexpr uint32_t idP = idesc_bf16(128, 128, 0, 0);
-            constexpr uint32_t idO = idesc_bf16(128, 64, 0, 1);
+            constexpr uint32_t idO = idesc_bf16(128, 80, 0, 1);
+            constexpr uint32_t idPV = idesc_bf16(128, 80, 0, 1);
             for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
                 const bool last = tile + 1 == sg.t_end;
                 for (int t = 0; t < NT; ++t) {
@@ -611,14 +624,14 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                     tc_fence_after();
                     const uint32_t aq = sbase + L.phiq + pslot * kTileBytes;
                     const uint32_t bk = sbase + L.phik + t * kTileBytes;
-                    const uint32_t bs = sbase + L.sbf + t * kSlice * 128;
+                    const uint32_t bs = sbase + L.st + t * (kSlice / 8) * 128;
+                    const uint32_t st_sbo = static_cast<uint32_t>(kp.F) * 16;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
                         const uint64_t ad = sdesc(aq + 32 * kk, 16, 1024, kLayoutSW128);
                         umma_bf16(tmem + kColP, ad, sdesc(bk + 32 * kk, 16, 1024, kLayoutSW128), idP, acc);
-                        umma_bf16(tmem + kColO, ad,
-                                  sdesc(bs + 2048 * kk, kTileBytes, 1024, kLayoutSW128), idO, acc);
+                        umma_bf16(tmem + kColO, ad, sdesc(bs + 256 * kk, 128, st_sbo, kLayoutNone), idO, acc);
                     }
                     umma_commit(&bar[B_PQ_EMPTY0 + pslot]);
                     // state update of a feature half once its phiK slices are in place
@@ -632,12 +645,11 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 if (last) wt.wait(&bar[B_V_FULL], ph_vf);
                 wt.wait(&bar[B_PSM_FULL], ph_psm);
                 tc_fence_after();
+                const uint32_t lbo = L.ones - L.v;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t a = sbase + L.phiq + (kk >> 2) * kTileBytes + 32 * (kk & 3);
-                    umma_bf16(tmem + kColO, sdesc(a, 16, 1024, kLayoutSW128),
-                              sdesc(sbase + L.v + 2048 * kk, kTileBytes, 1024, kLayoutSW128), idO, 1u);
-                }
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_bf16_ts(tmem + kColO, tmem + kColP + 8 * kk,
+                                 sdesc(sbase + L.v + 2048 * kk, lbo, 1024, kLayoutSW128), idPV, 1u);
                 umma_commit(&bar[B_TILE_DONE]);
                 umma_commit(&bar[B_V_EMPTY]);
             }
@@ -648,16 +660,13 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         const int sp = warp & 3;
         const uint32_t row = 32u * sp + lane;
         const uint32_t trow = tmem + ((32u * sp) << 16);
-        uint32_t ph_qkf = 0, ph_uf = 0, ph_pqe0 = 0, ph_pqe1 = 0, ph_pf = 0, ph_psm = 0, ph_td = 0,
-                 ph_sbf = 0;
+        uint32_t ph_qkf = 0, ph_uf = 0, ph_pqe0 = 0, ph_pqe1 = 0, ph_pf = 0, ph_td = 0;
         int uses0 = 0, uses1 = 0;
         for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
             wt.wait(&bar[B_QK_FULL], ph_qkf);
             float inv, l2i;
             row_scale(sm + (grp ? L.k : L.q) + row * 128, inv, l2i);
             warp_arrive(&bar[B_QK_EMPTY]);
-            if (grp == 0 && tile > sg.t_begin) wt.wait(&bar[B_SBF_READY], ph_sbf);  // zs of this tile
-            float den_inter = 0.0f;
             for (int t = 0; t < NT; ++t) {
                 const int node = (t * kSlice) / kp.m;
                 const float a = kp.a2[node] * inv, b = kp.b2[node] + l2i;
@@ -680,9 +689,8 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                             if (uses > 0) wt.wait(&bar[B_PQ_EMPTY0 + pslot], pslot ? ph_pqe1 : ph_pqe0);
                             ++uses;
                         }
-                        den_inter += phi_sub_epilogue(ur, pr, a, b,
-                                                      sbase + L.phiq + pslot * kTileBytes, row, half,
-                                                      zs + t * kSlice + half * kSub);
+                        phi_sub_epilogue(ur, pr, a, b, sbase + L.phiq + pslot * kTileBytes, row, half,
+                                         nullptr);
                     } else {
                         phi_sub_epilogue(ur, pr, a, b, sbase + L.phik + t * kTileBytes, row, half,
                                          nullptr);
@@ -691,52 +699,46 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 fence_async_smem();
                 warp_arrive(&bar[grp ? B_PK_FULL : (B_PQ_FULL0 + pslot)]);
             }
-            // masked scores into the phi(q) buffers: group 0 columns 0..63, group 1 64..127
-            wt.wait(&bar[B_P_FULL], ph_pf);
-            tc_fence_after();
-            float dpart = 0.0f;
-            {
-                uint32_t p0[32], p1[32];
-                tmem_ld32(trow + kColP + 64 * grp, p0);
-                tmem_ld32(trow + kColP + 64 * grp + 32, p1);
-                tmem_wait_ld();
-                reg_fence(p0);
-                reg_fence(p1);
-                uint32_t pk[32];
+            if (grp == 1) {
+                // masked scores -> bf16 in place (row i keeps keys j <= i), the A operand of P.V
+                wt.wait(&bar[B_P_FULL], ph_pf);
+                tc_fence_after();
 #pragma unroll
-                for (int j = 0; j < 32; j += 2) {
-                    const uint32_t c0 = 64u * grp + j;
-                    const float x0 = (c0 <= row) ? __uint_as_float(p0[j]) : 0.0f;
-                    const float x1 = (c0 + 1 <= row) ? __uint_as_float(p0[j + 1]) : 0.0f;
-                    const float y0 = (c0 + 32 <= row) ? __uint_as_float(p1[j]) : 0.0f;
-                    const float y1 = (c0 + 33 <= row) ? __uint_as_float(p1[j + 1]) : 0.0f;
-                    dpart += (x0 + x1) + (y0 + y1);
-                    pk[j >> 1] = pack_bf16(x0, x1);
-                    pk[16 + (j >> 1)] = pack_bf16(y0, y1);
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t p0[32], p1[32];
+                    tmem_ld32(trow + kColP + 64 * c, p0);
+                    tmem_ld32(trow + kColP + 64 * c + 32, p1);
+                    tmem_wait_ld();
+                    reg_fence(p0);
+                    reg_fence(p1);
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2) {
+                        const uint32_t c0 = 64u * c + j;
+                        pk[j >> 1] = pack_bf16((c0 <= row) ? __uint_as_float(p0[j]) : 0.0f,
+                                               (c0 + 1 <= row) ? __uint_as_float(p0[j + 1]) : 0.0f);
+                        pk[16 + (j >> 1)] = pack_bf16((c0 + 32 <= row) ? __uint_as_float(p1[j]) : 0.0f,
+                                                      (c0 + 33 <= row) ? __uint_as_float(p1[j + 1]) : 0.0f);
+                    }
+                    tmem_st32(trow + kColP + 32 * c, pk);
                 }
-                const uint32_t base = sbase + L.phiq + grp * kTileBytes;
-#pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    st_shared_v4(base + sw128_off(row, q), pk[4 * q], pk[4 * q + 1], pk[4 * q + 2],
-                                 pk[4 * q + 3]);
-            }
-            if (grp == 1) dsum[row] = dpart;
-            fence_async_smem();
-            tc_fence_before();
-            warp_arrive(&bar[B_PSM_FULL]);
-            if (grp == 0) {
-                wt.wait(&bar[B_PSM_FULL], ph_psm);  // group 1's partial sums are in dsum
+                tmem_wait_st();
+                tc_fence_before();
+                warp_arrive(&bar[B_PSM_FULL]);
+                // output: O[:, :64] / (O[:, 64] + eps)
                 wt.wait(&bar[B_TILE_DONE], ph_td);
                 tc_fence_after();
-                uint32_t o0[32], o1[32];
+                uint32_t o0[32], o1[32], dr;
                 tmem_ld32(trow + kColO, o0);
                 tmem_ld32(trow + kColO + 32, o1);
+                tmem_ld1(trow + kColO + 64, dr);
                 tmem_wait_ld();
                 reg_fence(o0);
                 reg_fence(o1);
+                reg_fence1(dr);
                 tc_fence_before();
                 warp_arrive(&bar[B_O_EMPTY]);
-                const float d = dpart + dsum[row] + den_inter;
+                const float d = __uint_as_float(dr);
                 const float rz = 1.0f / (d + kp.eps);
                 const int grow = tile * kTile + static_cast<int>(row);
                 if (grow < kp.L) {
@@ -757,11 +759,8 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                             pack_bf16(__uint_as_float(o1[8 * q + 6]) * rz, __uint_as_float(o1[8 * q + 7]) * rz));
                     if (den) den[rowbase + grow] = d;
                 }
-            } else {
-                wt.wait(&bar[B_TILE_DONE], ph_td);
-                tc_fence_after();
                 if (tile + 1 < sg.t_end) {
-                    // state after this tile -> bf16 operand copy and fp32 z
+                    // state after this tile -> bf16 copy for the next readout
                     for (int h = 0; h < halves; ++h) {
                         const int f = 128 * h + row;
                         uint32_t r0s[32], r1s[32], zr;
@@ -772,17 +771,13 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                         reg_fence(r0s);
                         reg_fence(r1s);
                         reg_fence1(zr);
-                        uint32_t pk[32];
+                        float sv[64];
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            pk[e] = pack_bf16(__uint_as_float(r0s[2 * e]), __uint_as_float(r0s[2 * e + 1]));
-                            pk[16 + e] = pack_bf16(__uint_as_float(r1s[2 * e]), __uint_as_float(r1s[2 * e + 1]));
+                        for (int e = 0; e < 32; ++e) {
+                            sv[e] = __uint_as_float(r0s[e]);
+                            sv[32 + e] = __uint_as_float(r1s[e]);
                         }
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            st_shared_v4(sbase + L.sbf + sw128_off(f, q), pk[4 * q], pk[4 * q + 1],
-                                         pk[4 * q + 2], pk[4 * q + 3]);
-                        zs[f] = __uint_as_float(zr);
+                        write_state_row(sbase + L.st, kp.F, f, sv, __uint_as_float(zr));
                     }
                     fence_async_smem();
                     tc_fence_before();

@@ -59,6 +59,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t phase)
     return done != 0;
 }
 
+// As above, but a thread whose phase is not complete is suspended (up to about `hint_ns`)
+// instead of spinning, so waiting warps do not take issue slots from working warps; it
+// resumes as soon as the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t addr, uint32_t phase, uint32_t hint_ns)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(addr), "r"(phase), "r"(hint_ns)
+        : "memory");
+    return done != 0;
+}
+
 // Bounded wait for the completion of `phase`.  Gives up after `limit_ns` of global time
 // and returns false (the caller records an error and leaves); never spins forever.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase,
@@ -68,8 +84,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase,
     if (mbar_try_wait(addr, phase)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 0; it < (1u << 30); ++it) {
-        if (mbar_try_wait(addr, phase)) return true;
-        if ((it & 63) == 63 && global_timer_ns() - t0 > limit_ns) return false;
+        if (mbar_try_wait_sleep(addr, phase, 100000u)) return true;
+        if (global_timer_ns() - t0 > limit_ns) return false;
     }
     return false;
 }
@@ -220,6 +236,20 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(
             d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+        : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]: A is read from tensor memory (bf16 pairs packed in 32-bit
+// columns, one row per lane, K along the columns); issued by one thread.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(
+            d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
         : "memory");
 }
 
