@@ -99,7 +99,8 @@ __host__ __device__ inline SmemOut smem_out_layout(int F)
     return s;
 }
 
-// State kernel: two 16 KiB projection operands (64 features each).
+// State kernel: two 16 KiB projection operands (64 features each); V and phi(k) are double
+// buffered so that the phi(k) of tile i+1 is written while tile i's state update runs.
 constexpr int kWStateBytes = 2 * kWBytes;
 struct SmemState {
     uint32_t w, k, v, ones, phik, bar, tmem, total;
@@ -110,10 +111,10 @@ __host__ __device__ inline SmemState smem_state_layout(int F)
     SmemState s;
     s.w = 0;
     s.k = 2 * kWStateBytes;
-    s.v = s.k + kTileBytes;
-    s.ones = s.v + kTileBytes;
-    s.phik = s.ones + kOnesBytes;
-    s.bar = s.phik + (F / kSlice) * kTileBytes;
+    s.v = s.k + kTileBytes;                 // 2 buffers
+    s.ones = s.v + 2 * kTileBytes;
+    s.phik = s.ones + kOnesBytes;           // 2 buffers of F/64 tiles
+    s.bar = s.phik + 2 * (F / kSlice) * kTileBytes;
     s.tmem = s.bar + NUM_BARS * 8;
     s.total = s.tmem + 16;
     return s;
@@ -257,7 +258,8 @@ __device__ __forceinline__ void warp_arrive(uint64_t* bar)
 // grid = BH * (nseg - 1): segment seg of sequence bh writes
 //   ws_S[bh][seg][f][e] = sum_{t in seg} phi(k_t)_f v_t[e],  ws_z[bh][seg][f] = sum phi(k_t)_f
 // Projections are 64 features wide (N = 128: two packed 32-feature operands), double
-// buffered in TMEM; epilogue group g takes the projections n with n % 2 == g.
+// buffered in TMEM; epilogue group g takes the projections n with n % 2 == g.  Tile i uses
+// V and phi(k) buffer (i - first) % 2.
 __global__ void __launch_bounds__(kThreads, 1)
 k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                   const __grid_constant__ CUtensorMap tmw, KParams kp, float* __restrict__ wsS,
@@ -271,11 +273,15 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int NT = kp.F / kSlice, halves = kp.F / 128;
+    const uint32_t phik_bytes = NT * kTileBytes;
     const Seg sg = segment_of(blockIdx.x + blockIdx.x / (kp.nseg - 1), kp.nseg, kp.ntiles);
     constexpr uint32_t kColUS = 0;     // 2 x 128: projections
     constexpr uint32_t kColSS = 256;   // 2 x 80 : [S | z]
-    // barrier roles here: QK_* hold K, V_* hold V, W_*0..1 the two operand slots,
-    // PK_FULL = all phiK of a tile written
+    // barrier roles here: QK_* hold the K tile; VF(b) / VE(b) the V buffers; TD(b) = the
+    // state update of a tile in buffer b is done; PK_FULL = all phiK of a tile written
+    uint64_t* VF = &bar[B_PQ_FULL0];
+    uint64_t* VE = &bar[B_PQ_EMPTY0];
+    uint64_t* TD = &bar[B_O_EMPTY];    // B_O_EMPTY, B_SBF_READY
     if (warp == 1) {
         tmem_alloc(tslot, 512);
         tmem_relinquish();
@@ -305,9 +311,10 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             int n_glob = 0;
             mbar_arrive_expect_tx(&bar[B_QK_FULL], kTileBytes);
             tma_load_3d(sm + L.k, &tmk, &bar[B_QK_FULL], 0, sg.t_begin * kTile, sg.bh);
-            mbar_arrive_expect_tx(&bar[B_V_FULL], kTileBytes);
-            tma_load_3d(sm + L.v, &tmv, &bar[B_V_FULL], 0, sg.t_begin * kTile, sg.bh);
+            mbar_arrive_expect_tx(&VF[0], kTileBytes);
+            tma_load_3d(sm + L.v, &tmv, &VF[0], 0, sg.t_begin * kTile, sg.bh);
             for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+                const int nxt = tile + 1 - sg.t_begin;   // local index of the next tile
                 for (int n = 0; n < NT; ++n, ++n_glob) {
                     const int slot = n_glob & 1;
                     uint32_t ph = (ph_we >> slot) & 1u;
@@ -317,10 +324,16 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                     unsigned char* dst = sm + L.w + slot * kWStateBytes;
                     tma_load_2d(dst, &tmw, &bar[B_W_FULL0 + slot], 0, (2 * n) * 64);
                     tma_load_2d(dst + kWBytes, &tmw, &bar[B_W_FULL0 + slot], 0, (2 * n + 1) * 64);
-                    if (tile > sg.t_begin && n == 1) {   // V once the previous update is done
-                        wt.wait(&bar[B_V_EMPTY], ph_ve);
-                        mbar_arrive_expect_tx(&bar[B_V_FULL], kTileBytes);
-                        tma_load_3d(sm + L.v, &tmv, &bar[B_V_FULL], 0, tile * kTile, sg.bh);
+                    // V of the next tile into its buffer once that buffer's last update is done
+                    if (n == NT - 1 && tile + 1 < sg.t_end) {
+                        const int vb = nxt & 1;
+                        if (nxt >= 2) {
+                            uint32_t pv = (ph_ve >> vb) & 1u;
+                            wt.wait(&VE[vb], pv);
+                            ph_ve ^= (1u << vb);
+                        }
+                        mbar_arrive_expect_tx(&VF[vb], kTileBytes);
+                        tma_load_3d(sm + L.v + vb * kTileBytes, &tmv, &VF[vb], 0, (tile + 1) * kTile, sg.bh);
                     }
                 }
                 if (tile + 1 < sg.t_end) {
@@ -336,33 +349,37 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             int n_glob = 0;
             constexpr uint32_t idU = idesc_bf16(128, 128, 0, 0);
             for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+                const int b = (tile - sg.t_begin) & 1;
                 wt.wait(&bar[B_QK_FULL], ph_kf);
                 for (int n = 0; n < NT; ++n, ++n_glob) {
                     const int slot = n_glob & 1;
                     uint32_t ph = (ph_wf >> slot) & 1u;
                     wt.wait(&bar[B_W_FULL0 + slot], ph);
                     ph_wf ^= (1u << slot);
-                    const int b = n & 1;
-                    wt.wait(&bar[B_U_EMPTY0 + b], b ? ph_ue1 : ph_ue0);
+                    const int ub = n & 1;
+                    wt.wait(&bar[B_U_EMPTY0 + ub], ub ? ph_ue1 : ph_ue0);
                     tc_fence_after();
                     const uint32_t w = sbase + L.w + slot * kWStateBytes;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(tmem + kColUS + 128 * b,
+                        umma_bf16(tmem + kColUS + 128 * ub,
                                   sdesc(sbase + L.k + 32 * kk, 16, 1024, kLayoutSW128),
                                   sdesc(w + 32 * kk, 16, 1024, kLayoutSW128), idU, kk > 0 ? 1u : 0u);
-                    umma_commit(&bar[B_U_FULL0 + b]);
+                    umma_commit(&bar[B_U_FULL0 + ub]);
                     umma_commit(&bar[B_W_EMPTY0 + slot]);
                 }
                 umma_commit(&bar[B_QK_EMPTY]);
                 wt.wait(&bar[B_PK_FULL], ph_pk);
-                wt.wait(&bar[B_V_FULL], ph_vf);
+                uint32_t pv = (ph_vf >> b) & 1u;
+                wt.wait(&VF[b], pv);
+                ph_vf ^= (1u << b);
                 tc_fence_after();
                 for (int h = 0; h < halves; ++h)
-                    issue_state_half(tmem, kColSS, sbase + L.phik, sbase + L.v, sbase + L.ones, h,
+                    issue_state_half(tmem, kColSS, sbase + L.phik + b * phik_bytes,
+                                     sbase + L.v + b * kTileBytes, sbase + L.ones, h,
                                      tile == sg.t_begin);
-                umma_commit(&bar[B_V_EMPTY]);
-                umma_commit(&bar[B_TILE_DONE]);
+                umma_commit(&VE[b]);
+                umma_commit(&TD[b]);
             }
         }
     } else if (warp < 10) {
@@ -372,16 +389,21 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         const uint32_t trow = tmem + ((32u * sp) << 16);
         uint32_t ph_kf = 0, ph_uf = 0, ph_td = 0;
         for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+            const int li = tile - sg.t_begin, b = li & 1;
             wt.wait(&bar[B_QK_FULL], ph_kf);
             float inv, l2i;
             row_scale(sm + L.k + row * 128, inv, l2i);
             warp_arrive(&bar[B_QK_EMPTY]);
-            if (tile > sg.t_begin) wt.wait(&bar[B_TILE_DONE], ph_td);  // phiK slots free again
+            if (li >= 2) {   // phiK buffer b free again (update of tile li-2 done)
+                uint32_t pt = (ph_td >> b) & 1u;
+                wt.wait(&TD[b], pt);
+                ph_td ^= (1u << b);
+            }
             for (int n = grp; n < NT; n += 2) {
                 wt.wait(&bar[B_U_FULL0 + grp], ph_uf);
                 tc_fence_after();
                 const int node = (n * kSlice) / kp.m;
-                const float a = kp.a2[node] * inv, b = kp.b2[node] + l2i;
+                const float a = kp.a2[node] * inv, bb = kp.b2[node] + l2i;
                 const uint32_t col = kColUS + 128 * grp;
                 uint32_t ua[32], pa[32], ub[32], pb[32];
                 tmem_ld32(trow + col, ua);
@@ -395,15 +417,19 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 reg_fence(pb);
                 tc_fence_before();
                 warp_arrive(&bar[B_U_EMPTY0 + grp]);
-                const uint32_t tile_addr = sbase + L.phik + n * kTileBytes;
-                phi_sub_epilogue(ua, pa, a, b, tile_addr, row, 0, nullptr);
-                phi_sub_epilogue(ub, pb, a, b, tile_addr, row, 1, nullptr);
+                const uint32_t tile_addr = sbase + L.phik + b * phik_bytes + n * kTileBytes;
+                phi_sub_epilogue(ua, pa, a, bb, tile_addr, row, 0, nullptr);
+                phi_sub_epilogue(ub, pb, a, bb, tile_addr, row, 1, nullptr);
             }
             fence_async_smem();
             warp_arrive(&bar[B_PK_FULL]);
         }
-        // the segment's sums: group 0 writes feature half 0, group 1 half 1
-        wt.wait(&bar[B_TILE_DONE], ph_td);
+        // the segment's sums once the last update is done (it follows all earlier ones)
+        {
+            const int lb = (sg.t_end - 1 - sg.t_begin) & 1;
+            uint32_t pt = (ph_td >> lb) & 1u;
+            wt.wait(&TD[lb], pt);
+        }
         tc_fence_after();
         const size_t segidx = static_cast<size_t>(sg.bh) * kp.nseg + sg.seg;
         for (int h = grp; h < halves; h += 2) {
