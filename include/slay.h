@@ -55,7 +55,7 @@ typedef enum {
     SLAY_ERR_INVALID_ARG = 1,   /* NULL pointer, misalignment, bad size, workspace too small */
     SLAY_ERR_UNSUPPORTED = 2,   /* a size or dtype combination this build does not offer */
     SLAY_ERR_CUDA = 3,          /* a CUDA runtime error (launch, allocation of the cache, no device) */
-    SLAY_ERR_TIMEOUT = 4,       /* reserved: no kernel of this library waits on another CTA */
+    SLAY_ERR_TIMEOUT = 4,       /* a kernel's bounded wait ran out (see slay_kernel_status) */
     SLAY_ERR_NO_MEMORY = 5      /* host allocation failed */
 } slay_status;
 
@@ -150,6 +150,18 @@ slay_status slay_attn_causal_fwd_noalloc(const void* q, const void* k, const voi
                                          void* out, float* den, int B, int H, int L, int D,
                                          int Dv, slay_dtype dt, int R, int m, uint64_t seed,
                                          float eps, void* stream);
+
+/* Kernel status of the last attention call that used `workspace` (or, with workspace ==
+ * NULL, of the last slay_attn_causal_fwd_noalloc call on the current device).
+ * The tensor-core kernels coordinate their warps through shared-memory barriers; every
+ * wait is bounded (2 s).  A wait that runs out makes the kernel stop early, leave its
+ * outputs incomplete and set the status word, the first int of the workspace, which each
+ * attention call clears when it is enqueued.  This call copies the word to the host on
+ * `stream` and synchronizes the stream.  Returns SLAY_ERR_TIMEOUT if the word is set,
+ * SLAY_OK if it is not (or if the no-alloc path never ran on this device),
+ * SLAY_ERR_INVALID_ARG for a workspace that is not 256-byte aligned, SLAY_ERR_CUDA if the
+ * copy fails.  The status of a call is only defined once it has been enqueued. */
+slay_status slay_kernel_status(const void* workspace, void* stream);
 
 /* Workspace bytes an entry point needs for these sizes (0 if none; SIZE_MAX if the
  * sizes are unsupported).  Feature map and decode need none. */

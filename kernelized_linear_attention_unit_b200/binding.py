@@ -22,7 +22,7 @@ OP_FEATURE_MAP, OP_CAUSAL_FWD, OP_BIDIR_FWD, OP_CAUSAL_BWD, OP_DECODE = range(5)
 EXPORTS = ["slay_feature_map", "slay_attn_causal_fwd", "slay_attn_bidir_fwd",
            "slay_attn_causal_bwd", "slay_decode_step", "slay_workspace_bytes", "slay_prepare",
            "slay_sketch_params", "slay_status_string", "slay_last_error", "slay_trace_enable",
-           "slay_trace_read", "slay_attn_causal_fwd_noalloc"]
+           "slay_trace_read", "slay_attn_causal_fwd_noalloc", "slay_kernel_status"]
 
 
 class SlayError(RuntimeError):
@@ -66,6 +66,8 @@ def lib():
     L.slay_status_string.restype = C.c_char_p
     L.slay_last_error.argtypes = []
     L.slay_last_error.restype = C.c_char_p
+    L.slay_kernel_status.argtypes = [vp, vp]
+    L.slay_kernel_status.restype = i32
     L.slay_trace_enable.argtypes = [i32]
     L.slay_trace_enable.restype = i32
     L.slay_trace_read.argtypes = [C.POINTER(C.c_char_p), C.POINTER(C.c_float), i32]
@@ -188,15 +190,18 @@ def _attn(fn, name, op, q, k, v, out, den, R, m, seed, eps, workspace, stream):
         raise ValueError("workspace has %d bytes, %d needed" % (wbytes, need))
     _raise(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(den), B, H, L, D, Dv, dt, R, m, seed,
               eps, _ptr(workspace), wbytes, _stream(stream)), name)
+    return workspace
 
 
 def slay_attn_causal_fwd(q, k, v, out, den, R, m, seed, eps, workspace=None, stream=None):
-    _attn(lib().slay_attn_causal_fwd, "slay_attn_causal_fwd", OP_CAUSAL_FWD, q, k, v, out, den,
+    """Enqueue the causal forward; returns the workspace it used (see slay_kernel_status)."""
+    return _attn(lib().slay_attn_causal_fwd, "slay_attn_causal_fwd", OP_CAUSAL_FWD, q, k, v, out, den,
           R, m, seed, eps, workspace, stream)
 
 
 def slay_attn_bidir_fwd(q, k, v, out, den, R, m, seed, eps, workspace=None, stream=None):
-    _attn(lib().slay_attn_bidir_fwd, "slay_attn_bidir_fwd", OP_BIDIR_FWD, q, k, v, out, den,
+    """Enqueue the bidirectional forward; returns the workspace it used."""
+    return _attn(lib().slay_attn_bidir_fwd, "slay_attn_bidir_fwd", OP_BIDIR_FWD, q, k, v, out, den,
           R, m, seed, eps, workspace, stream)
 
 
@@ -239,6 +244,16 @@ def slay_attn_causal_bwd(q, k, v, out, den, dout, dq, dk, dv, R, m, seed, eps, w
                                       _ptr(dq), _ptr(dk), _ptr(dv), B, H, L, D, Dv, dt, R, m,
                                       seed, eps, _ptr(workspace), wbytes, _stream(stream)),
            "slay_attn_causal_bwd")
+    return workspace
+
+
+def slay_kernel_status(workspace=None, stream=None):
+    """Raise SlayError if a kernel of the last call on `workspace` (None: the last
+    no-alloc causal forward on this device) stopped on a wait that ran out; synchronizes
+    the stream."""
+    if workspace is not None:
+        _check(workspace, "workspace")
+    _raise(lib().slay_kernel_status(_ptr(workspace), _stream(stream)), "slay_kernel_status")
 
 
 def slay_decode_step(q, k, v, S, z, out, R, m, seed, eps, stream=None):

@@ -161,9 +161,9 @@ size_t attn_ws(slay_op op, slay_dtype dt, int B, int H, int L, int Dv, int R, in
     if (dt == SLAY_BF16 && tc_supported(op, B, H, L, R, m))
         return tc_workspace_bytes(op, B, H, L, R, m);
     switch (op) {
-        case SLAY_OP_CAUSAL_FWD: return simt_ws_causal(B, H, L, Dv, F);
-        case SLAY_OP_BIDIR_FWD: return simt_ws_bidir(B, H, L, Dv, F);
-        case SLAY_OP_CAUSAL_BWD: return simt_ws_bwd(B, H, L, Dv, F);
+        case SLAY_OP_CAUSAL_FWD: return kWsHeader + simt_ws_causal(B, H, L, Dv, F);
+        case SLAY_OP_BIDIR_FWD: return kWsHeader + simt_ws_bidir(B, H, L, Dv, F);
+        case SLAY_OP_CAUSAL_BWD: return kWsHeader + simt_ws_bwd(B, H, L, Dv, F);
         default: return 0;
     }
 }
@@ -185,10 +185,14 @@ slay_status attn_fwd(const void* q, const void* k, const void* v, void* out, flo
     if ((s = get_params(D, R, m, seed, eps, &P)) != SLAY_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e;
-    if (dt == SLAY_BF16 && tc_supported(op, B, H, L, R, m))
+    if (dt == SLAY_BF16 && tc_supported(op, B, H, L, R, m)) {
         e = tc_attn_fwd(q, k, v, out, den, B, H, L, P, eps, causal, ws, st);
-    else
-        e = simt_attn_fwd(q, k, v, out, den, B, H, L, dt, P, eps, causal, ws, st);
+    } else {
+        e = cudaMemsetAsync(ws, 0, sizeof(int), st);
+        if (e == cudaSuccess)
+            e = simt_attn_fwd(q, k, v, out, den, B, H, L, dt, P, eps, causal,
+                              static_cast<char*>(ws) + kWsHeader, st);
+    }
     return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
 }
 
@@ -258,8 +262,11 @@ slay_status slay_attn_causal_bwd(const void* q, const void* k, const void* v, co
         return SLAY_ERR_INVALID_ARG;
     Params P;
     if ((s = get_params(D, R, m, seed, eps, &P)) != SLAY_OK) return s;
-    cudaError_t e = simt_attn_causal_bwd(q, k, v, out, den, dout, dq, dk, dv, B, H, L, dt, P, eps,
-                                         workspace, static_cast<cudaStream_t>(stream));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
+    if (e == cudaSuccess)
+        e = simt_attn_causal_bwd(q, k, v, out, den, dout, dq, dk, dv, B, H, L, dt, P, eps,
+                                 static_cast<char*>(workspace) + kWsHeader, st);
     return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
 }
 
@@ -283,6 +290,19 @@ slay_status slay_decode_step(const void* q, const void* k, const void* v, float*
     cudaError_t e = simt_decode_step(q, k, v, S, z, out, static_cast<int>(N), dt, P, eps,
                                      static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
+}
+
+slay_status slay_kernel_status(const void* workspace, void* stream)
+{
+    const void* word = workspace ? workspace : noalloc_status_word();
+    if (!word) return SLAY_OK;
+    if (!aligned(word, 256)) return SLAY_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int flag = 0;
+    cudaError_t e = cudaMemcpyAsync(&flag, word, sizeof(int), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return flag ? SLAY_ERR_TIMEOUT : SLAY_OK;
 }
 
 size_t slay_workspace_bytes(slay_op op, slay_dtype dt, int B, int H, int L, int D, int Dv, int R,

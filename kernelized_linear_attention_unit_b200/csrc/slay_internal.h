@@ -59,7 +59,14 @@ bool dtype_ok(slay_dtype d);
 slay_status check_shape(int D, int Dv, int R, int m);
 slay_status check_attn(const void* q, const void* k, const void* v, const void* out, int B,
                        int H, int L, int D, int Dv, slay_dtype dt, int R, int m, float eps);
+// Every attention workspace starts with a 256-byte header whose first int is the
+// kernel status word: 0 after a call is enqueued, set to 1 by a kernel whose bounded
+// mbarrier wait ran out.  The path's own scratch follows the header.
+constexpr size_t kWsHeader = 256;
 size_t attn_ws(slay_op op, slay_dtype dt, int B, int H, int L, int Dv, int R, int m);
+// Device address of the no-alloc path's status word on the current device, or nullptr
+// when that path has not run on it.
+const void* noalloc_status_word();
 
 // ---- CUDA-core kernels (slay_simt.cu) ----
 // Sizes of the workspace carve-outs of the CUDA-core path.

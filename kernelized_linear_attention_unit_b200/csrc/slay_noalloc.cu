@@ -127,6 +127,15 @@ slay_status load_params(DeviceSlot* slot, int D, int R, int m, uint64_t seed, fl
 }
 
 }  // namespace
+
+const void* noalloc_status_word()
+{
+    std::lock_guard<std::mutex> lock(g_mu);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+    return slots()[dev].scratch;
+}
+
 }  // namespace slay
 
 using namespace slay;
@@ -163,7 +172,8 @@ extern "C" slay_status slay_attn_causal_fwd_noalloc(const void* q, const void* k
     cudaError_t e;
     if (dt == SLAY_BF16 && tc_supported(SLAY_OP_CAUSAL_FWD, B, H, L, R, m))
         e = tc_attn_fwd(q, k, v, out, den, B, H, L, slot.P, eps, true, slot.scratch, st);
-    else
-        e = simt_attn_fwd(q, k, v, out, den, B, H, L, dt, slot.P, eps, true, slot.scratch, st);
+    else if ((e = cudaMemsetAsync(slot.scratch, 0, sizeof(int), st)) == cudaSuccess)
+        e = simt_attn_fwd(q, k, v, out, den, B, H, L, dt, slot.P, eps, true,
+                          slot.scratch + kWsHeader, st);
     return e == cudaSuccess ? SLAY_OK : SLAY_ERR_CUDA;
 }

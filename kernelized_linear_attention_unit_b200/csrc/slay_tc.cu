@@ -50,9 +50,9 @@ constexpr int kSub = 32;                   // features per projection (N = 64 wi
 constexpr int kTileBytes = kTile * 128;    // one [128 rows][64 bf16] swizzled tile = 16 KiB
 constexpr int kWBytes = 64 * 128;          // one projection operand [64 rows][64 bf16] = 8 KiB
 constexpr int kWSlots = 3;                 // output kernel: 3 x 8 KiB projection operands
-constexpr int kThreads = 384;              // 12 warps
+constexpr int kThreads = 384;              // 12 warps (state kernel)
+constexpr int kOutThreads = 512;           // 16 warps (output kernel)
 constexpr int kOnesBytes = kTileBytes;     // [128][64] bf16 ones: the z columns of [V | 1]
-constexpr size_t kWsHeader = 256;          // error word + padding at the start of the workspace
 constexpr int kNumSMs = 148;
 constexpr uint64_t kWaitNs = 2000000000ull;
 
@@ -72,6 +72,7 @@ enum {
     B_U_FULL0, B_U_FULL1, B_U_EMPTY0, B_U_EMPTY1,
     B_PQ_FULL0, B_PQ_FULL1, B_PQ_EMPTY0, B_PQ_EMPTY1,
     B_PK_FULL, B_P_FULL, B_PSM_FULL, B_TILE_DONE, B_O_EMPTY, B_SBF_READY,
+    B_PK_FREE0, B_PK_FREE1, B_PK_FULL1, B_PK_FULL2, B_PK_FULL3,
     NUM_BARS
 };
 
@@ -476,13 +477,21 @@ __device__ __forceinline__ void write_state_row(uint32_t st, int F, int f, const
     st_shared_v4(base + 8 * sbo, pack_bf16(z, 0.0f), 0u, 0u, 0u);
 }
 
+// Output kernel: phi(k) slice t (of at most 4) is signalled on its own barrier, so the
+// phi(k) warps, which may run a tile ahead, never complete a phase the MMA warp has not
+// yet waited for.
+__device__ __forceinline__ uint64_t* pk_full(uint64_t* bar, int t)
+{
+    return &bar[t == 0 ? B_PK_FULL : B_PK_FULL1 + t - 1];
+}
+
 // grid = BH * nseg.  One CTA walks the tiles of one segment with the state entering it.
-// Warps 10 / 11 issue the q / k projections (32 features each) into U0 / U1; warp 1 issues
-// the score, readout, state and P.V MMAs.  Epilogue group 0 (warps 2-5) turns q projections
-// into phi(q); group 1 (warps 6-9) turns k projections into phi(k) and then does the end of
-// the tile: the masked scores (bf16, in place in tensor memory), the output and the state
-// copy for the next tile.
-__global__ void __launch_bounds__(kThreads, 1)
+// Warp 0 loads tiles; warp 1 issues the score, readout, state and P.V MMAs; warps 2 / 3
+// issue the q / k projections (32 features each) into U0 / U1.  Warps 4-7 turn q
+// projections into phi(q), warps 8-11 k projections into phi(k); warps 12-15 finish each
+// tile (masked scores in place in tensor memory as bf16, the state copy for the next
+// readout, the output), so the feature warps move on to the next tile meanwhile.
+__global__ void __launch_bounds__(kOutThreads, 1)
 k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                 const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmw,
                 KParams kp, const float* __restrict__ wsS, const float* __restrict__ wsZ,
@@ -511,6 +520,7 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         mbar_init(&bar[B_PQ_FULL0], 4);
         mbar_init(&bar[B_PQ_FULL1], 4);
         mbar_init(&bar[B_PK_FULL], 4);
+        for (int t = 1; t < 4; ++t) mbar_init(&bar[B_PK_FULL1 + t - 1], 4);
         mbar_init(&bar[B_PSM_FULL], 4);
         mbar_init(&bar[B_O_EMPTY], 4);
         mbar_init(&bar[B_SBF_READY], 4);
@@ -523,234 +533,294 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
     fill_ones(sm + L.ones);
     {   // the state copy: columns 65..79 stay zero
         uint4* p = reinterpret_cast<uint4*>(sm + L.st);
-        for (int i = tid; i < NT * kStBytes / 16; i += kThreads) p[i] = make_uint4(0, 0, 0, 0);
+        for (int i = tid; i < NT * kStBytes / 16; i += kOutThreads) p[i] = make_uint4(0, 0, 0, 0);
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
-
-    // state entering the segment (sum of the earlier segments), by epilogue group 1
-    if (warp >= 6 && warp < 10) {
-        const int sp = warp & 3;
-        const uint32_t row = 32u * sp + lane;
-        const uint32_t trow = tmem + ((32u * sp) << 16);
-        for (int h = 0; h < halves; ++h) {
-            const int f = 128 * h + row;
-            float acc[64];
-#pragma unroll
-            for (int e = 0; e < 64; ++e) acc[e] = 0.0f;
-            float zf = 0.0f;
-            for (int s = 0; s < sg.seg; ++s) {
-                const size_t segidx = static_cast<size_t>(sg.bh) * kp.nseg + s;
-                const float4* src = reinterpret_cast<const float4*>(wsS + (segidx * kp.F + f) * 64);
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const float4 x = src[q];
-                    acc[4 * q] += x.x; acc[4 * q + 1] += x.y; acc[4 * q + 2] += x.z; acc[4 * q + 3] += x.w;
-                }
-                zf += wsZ[segidx * kp.F + f];
-            }
-            uint32_t r[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(acc[e]);
-            tmem_st32(trow + kColS + 80 * h, r);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(acc[32 + e]);
-            tmem_st32(trow + kColS + 80 * h + 32, r);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(zf);
-            tmem_st32(trow + kColS + 80 * h + 64, r);  // z columns (a later half rewrites its own)
-            write_state_row(sbase + L.st, kp.F, f, acc, zf);
-        }
-        tmem_wait_st();
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-
-    Waiter wt;
-    const int64_t rowbase = static_cast<int64_t>(sg.bh) * kp.L;
-    if (warp == 0) {
-        // ---------------------------------------------------------------- TMA
-        if (lane == 0) {
-            uint32_t ph_qke = 0, ph_ve = 0, ph_we = (1u << kWSlots) - 1u;
-            int n_glob = 0;
-            const int vpoint = (NS < kWSlots ? NS : kWSlots) - 1;
-            mbar_arrive_expect_tx(&bar[B_QK_FULL], 2 * kTileBytes);
-            tma_load_3d(sm + L.q, &tmq, &bar[B_QK_FULL], 0, sg.t_begin * kTile, sg.bh);
-            tma_load_3d(sm + L.k, &tmk, &bar[B_QK_FULL], 0, sg.t_begin * kTile, sg.bh);
-            mbar_arrive_expect_tx(&bar[B_V_FULL], kTileBytes);
-            tma_load_3d(sm + L.v, &tmv, &bar[B_V_FULL], 0, sg.t_begin * kTile, sg.bh);
-            for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
-                for (int n = 0; n < NS; ++n, ++n_glob) {
-                    const int slot = n_glob % kWSlots;
-                    uint32_t ph = (ph_we >> slot) & 1u;
-                    wt.wait(&bar[B_W_EMPTY0 + slot], ph);
-                    ph_we ^= (1u << slot);
-                    mbar_arrive_expect_tx(&bar[B_W_FULL0 + slot], kWBytes);
-                    tma_load_2d(sm + L.w + slot * kWBytes, &tmw, &bar[B_W_FULL0 + slot], 0, n * 64);
-                    // V of this tile once the previous tile's P.V and state update are done
-                    if (tile > sg.t_begin && n == vpoint) {
-                        wt.wait(&bar[B_V_EMPTY], ph_ve);
-                        mbar_arrive_expect_tx(&bar[B_V_FULL], kTileBytes);
-                        tma_load_3d(sm + L.v, &tmv, &bar[B_V_FULL], 0, tile * kTile, sg.bh);
+    // registers: 128 per thread at launch; the single-thread issuers of warpgroup 0 give
+    // 32 of theirs to the three epilogue warpgroups (128*96 + 384*136 <= 65536).  Each role
+    // stays inside the branch that set its budget.
+    if (warp < 4) {
+        regs_dec<96>();
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        Waiter wt;
+        if (warp == 0) {
+            // ---------------------------------------------------------------- TMA
+            if (lane == 0) {
+                uint32_t ph_qke = 0, ph_ve = 0, ph_we = (1u << kWSlots) - 1u;
+                int n_glob = 0;
+                const int vpoint = (NS < kWSlots ? NS : kWSlots) - 1;
+                mbar_arrive_expect_tx(&bar[B_QK_FULL], 2 * kTileBytes);
+                tma_load_3d(sm + L.q, &tmq, &bar[B_QK_FULL], 0, sg.t_begin * kTile, sg.bh);
+                tma_load_3d(sm + L.k, &tmk, &bar[B_QK_FULL], 0, sg.t_begin * kTile, sg.bh);
+                mbar_arrive_expect_tx(&bar[B_V_FULL], kTileBytes);
+                tma_load_3d(sm + L.v, &tmv, &bar[B_V_FULL], 0, sg.t_begin * kTile, sg.bh);
+                for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+                    for (int n = 0; n < NS; ++n, ++n_glob) {
+                        const int slot = n_glob % kWSlots;
+                        uint32_t ph = (ph_we >> slot) & 1u;
+                        wt.wait(&bar[B_W_EMPTY0 + slot], ph);
+                        ph_we ^= (1u << slot);
+                        mbar_arrive_expect_tx(&bar[B_W_FULL0 + slot], kWBytes);
+                        tma_load_2d(sm + L.w + slot * kWBytes, &tmw, &bar[B_W_FULL0 + slot], 0, n * 64);
+                        // V of this tile once the previous tile's P.V and state update are done
+                        if (tile > sg.t_begin && n == vpoint) {
+                            wt.wait(&bar[B_V_EMPTY], ph_ve);
+                            mbar_arrive_expect_tx(&bar[B_V_FULL], kTileBytes);
+                            tma_load_3d(sm + L.v, &tmv, &bar[B_V_FULL], 0, tile * kTile, sg.bh);
+                        }
+                    }
+                    if (tile + 1 < sg.t_end) {
+                        wt.wait(&bar[B_QK_EMPTY], ph_qke);
+                        mbar_arrive_expect_tx(&bar[B_QK_FULL], 2 * kTileBytes);
+                        tma_load_3d(sm + L.q, &tmq, &bar[B_QK_FULL], 0, (tile + 1) * kTile, sg.bh);
+                        tma_load_3d(sm + L.k, &tmk, &bar[B_QK_FULL], 0, (tile + 1) * kTile, sg.bh);
                     }
                 }
-                if (tile + 1 < sg.t_end) {
-                    wt.wait(&bar[B_QK_EMPTY], ph_qke);
-                    mbar_arrive_expect_tx(&bar[B_QK_FULL], 2 * kTileBytes);
-                    tma_load_3d(sm + L.q, &tmq, &bar[B_QK_FULL], 0, (tile + 1) * kTile, sg.bh);
-                    tma_load_3d(sm + L.k, &tmk, &bar[B_QK_FULL], 0, (tile + 1) * kTile, sg.bh);
+            }
+        } else if (warp == 1) {
+            // ------------------------------------------------------ main MMA issuer
+            if (lane == 0) {
+                uint32_t ph_vf = 0, ph_pqf0 = 0, ph_pqf1 = 0, ph_pkf = 0, ph_psm = 0, ph_oe = 0,
+                         ph_sbf = 0;
+                constexpr uint32_t idP = idesc_bf16(128, 128, 0, 0);
+                constexpr uint32_t idO = idesc_bf16(128, 80, 0, 1);
+                constexpr uint32_t idPV = idesc_bf16(128, 80, 0, 1);
+                for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+                    const bool last = tile + 1 == sg.t_end;
+                    for (int t = 0; t < NT; ++t) {
+                        const int pslot = t & 1;
+                        wt.wait(&bar[B_PQ_FULL0 + pslot], pslot ? ph_pqf1 : ph_pqf0);
+                        {   // ph_pkf: one phase bit per phiK slice barrier
+                            uint32_t ph = (ph_pkf >> t) & 1u;
+                            wt.wait(pk_full(bar, t), ph);
+                            ph_pkf ^= (1u << t);
+                        }
+                        if (t == 0 && tile > sg.t_begin) {
+                            wt.wait(&bar[B_SBF_READY], ph_sbf);
+                            wt.wait(&bar[B_O_EMPTY], ph_oe);
+                        }
+                        tc_fence_after();
+                        const uint32_t aq = sbase + L.phiq + pslot * kTileBytes;
+                        const uint32_t bk = sbase + L.phik + t * kTileBytes;
+                        const uint32_t bs = sbase + L.st + t * (kSlice / 8) * 128;
+                        const uint32_t st_sbo = static_cast<uint32_t>(kp.F) * 16;
+    #pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+                            const uint64_t ad = sdesc(aq + 32 * kk, 16, 1024, kLayoutSW128);
+                            umma_bf16(tmem + kColP, ad, sdesc(bk + 32 * kk, 16, 1024, kLayoutSW128), idP, acc);
+                            umma_bf16(tmem + kColO, ad, sdesc(bs + 256 * kk, 128, st_sbo, kLayoutNone), idO, acc);
+                        }
+                        umma_commit(&bar[B_PQ_EMPTY0 + pslot]);
+                        // state update of a feature half once its phiK slices are in place; the
+                        // half's phiK slices are free for the next tile once it has been read
+                        if (!last && (t & 1) == 1) {
+                            if (t == 1) wt.wait(&bar[B_V_FULL], ph_vf);
+                            issue_state_half(tmem, kColS, sbase + L.phik, sbase + L.v, sbase + L.ones,
+                                             t >> 1, false);
+                            umma_commit(&bar[B_PK_FREE0 + (t >> 1)]);
+                        }
+                    }
+                    umma_commit(&bar[B_P_FULL]);
+                    if (last) wt.wait(&bar[B_V_FULL], ph_vf);
+                    wt.wait(&bar[B_PSM_FULL], ph_psm);
+                    tc_fence_after();
+                    const uint32_t lbo = L.ones - L.v;
+    #pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_bf16_ts(tmem + kColO, tmem + kColP + 8 * kk,
+                                     sdesc(sbase + L.v + 2048 * kk, lbo, 1024, kLayoutSW128), idPV, 1u);
+                    umma_commit(&bar[B_TILE_DONE]);
+                    umma_commit(&bar[B_V_EMPTY]);
+                }
+            }
+        } else {
+            // ------------------------------------------- projection issuers (q: 2, k: 3)
+            if (lane == 0) {
+                const int g = warp - 2;
+                const uint32_t xaddr = sbase + (g ? L.k : L.q);
+                uint32_t ph_qkf = 0, ph_wf = 0, ph_ue = 1;
+                int n_glob = 0;
+                for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+                    wt.wait(&bar[B_QK_FULL], ph_qkf);
+                    for (int n = 0; n < NS; ++n, ++n_glob) {
+                        const int slot = n_glob % kWSlots;
+                        uint32_t ph = (ph_wf >> slot) & 1u;
+                        wt.wait(&bar[B_W_FULL0 + slot], ph);
+                        ph_wf ^= (1u << slot);
+                        wt.wait(&bar[B_U_EMPTY0 + g], ph_ue);
+                        tc_fence_after();
+                        issue_projection(tmem + (g ? kColU1 : kColU0), xaddr, sbase + L.w + slot * kWBytes);
+                        umma_commit(&bar[B_U_FULL0 + g]);
+                        umma_commit(&bar[B_W_EMPTY0 + slot]);
+                    }
+                    umma_commit(&bar[B_QK_EMPTY]);
                 }
             }
         }
-    } else if (warp >= 10) {
-        // ------------------------------------------ projection issuers (q: 10, k: 11)
-        if (lane == 0) {
-            const int g = warp - 10;
-            const uint32_t xaddr = sbase + (g ? L.k : L.q);
-            uint32_t ph_qkf = 0, ph_wf = 0, ph_ue = 1;
-            int n_glob = 0;
+        if (!wt.ok) atomicExch(err, 1);
+        drain_after_failure(wt.ok);
+    } else {
+        regs_inc<136>();
+        // state entering the segment (sum of the earlier segments), by the tail warps
+        if (warp >= 12) {
+            const int sp = warp & 3;
+            const uint32_t row = 32u * sp + lane;
+            const uint32_t trow = tmem + ((32u * sp) << 16);
+            for (int h = 0; h < halves; ++h) {
+                const int f = 128 * h + row;
+                float acc[64];
+    #pragma unroll
+                for (int e = 0; e < 64; ++e) acc[e] = 0.0f;
+                float zf = 0.0f;
+                for (int s = 0; s < sg.seg; ++s) {
+                    const size_t segidx = static_cast<size_t>(sg.bh) * kp.nseg + s;
+                    const float4* src = reinterpret_cast<const float4*>(wsS + (segidx * kp.F + f) * 64);
+    #pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const float4 x = src[q];
+                        acc[4 * q] += x.x; acc[4 * q + 1] += x.y; acc[4 * q + 2] += x.z; acc[4 * q + 3] += x.w;
+                    }
+                    zf += wsZ[segidx * kp.F + f];
+                }
+                uint32_t r[32];
+    #pragma unroll
+                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(acc[e]);
+                tmem_st32(trow + kColS + 80 * h, r);
+    #pragma unroll
+                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(acc[32 + e]);
+                tmem_st32(trow + kColS + 80 * h + 32, r);
+    #pragma unroll
+                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(zf);
+                tmem_st32(trow + kColS + 80 * h + 64, r);  // z columns (a later half rewrites its own)
+                write_state_row(sbase + L.st, kp.F, f, acc, zf);
+            }
+            tmem_wait_st();
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        Waiter wt;
+        const int64_t rowbase = static_cast<int64_t>(sg.bh) * kp.L;
+        if (warp < 12) {
+            // ------------------------------------------------ feature epilogues
+            const int grp = (warp >= 8) ? 1 : 0;
+            const int sp = warp & 3;
+            const uint32_t row = 32u * sp + lane;
+            const uint32_t trow = tmem + ((32u * sp) << 16);
+            uint32_t ph_qkf = 0, ph_uf = 0, ph_pqe0 = 0, ph_pqe1 = 0, ph_pkf0 = 0, ph_pkf1 = 0;
+            int uses0 = 0, uses1 = 0;
             for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
                 wt.wait(&bar[B_QK_FULL], ph_qkf);
-                for (int n = 0; n < NS; ++n, ++n_glob) {
-                    const int slot = n_glob % kWSlots;
-                    uint32_t ph = (ph_wf >> slot) & 1u;
-                    wt.wait(&bar[B_W_FULL0 + slot], ph);
-                    ph_wf ^= (1u << slot);
-                    wt.wait(&bar[B_U_EMPTY0 + g], ph_ue);
-                    tc_fence_after();
-                    issue_projection(tmem + (g ? kColU1 : kColU0), xaddr, sbase + L.w + slot * kWBytes);
-                    umma_commit(&bar[B_U_FULL0 + g]);
-                    umma_commit(&bar[B_W_EMPTY0 + slot]);
-                }
-                umma_commit(&bar[B_QK_EMPTY]);
-            }
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------------ main MMA issuer
-        if (lane == 0) {
-            uint32_t ph_vf = 0, ph_pqf0 = 0, ph_pqf1 = 0, ph_pkf = 0, ph_psm = 0, ph_oe = 0,
-                     ph_sbf = 0;
-            constexpr uint32_t idP = idesc_bf16(128, 128, 0, 0);
-            constexpr uint32_t idO = idesc_bf16(128, 80, 0, 1);
-            constexpr uint32_t idPV = idesc_bf16(128, 80, 0, 1);
-            for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
-                const bool last = tile + 1 == sg.t_end;
+                float inv, l2i;
+                row_scale(sm + (grp ? L.k : L.q) + row * 128, inv, l2i);
+                warp_arrive(&bar[B_QK_EMPTY]);
                 for (int t = 0; t < NT; ++t) {
+                    const int node = (t * kSlice) / kp.m;
+                    const float a = kp.a2[node] * inv, b = kp.b2[node] + l2i;
                     const int pslot = t & 1;
-                    wt.wait(&bar[B_PQ_FULL0 + pslot], pslot ? ph_pqf1 : ph_pqf0);
-                    wt.wait(&bar[B_PK_FULL], ph_pkf);
-                    if (t == 0 && tile > sg.t_begin) {
-                        wt.wait(&bar[B_SBF_READY], ph_sbf);
-                        wt.wait(&bar[B_O_EMPTY], ph_oe);
-                    }
-                    tc_fence_after();
-                    const uint32_t aq = sbase + L.phiq + pslot * kTileBytes;
-                    const uint32_t bk = sbase + L.phik + t * kTileBytes;
-                    const uint32_t bs = sbase + L.st + t * (kSlice / 8) * 128;
-                    const uint32_t st_sbo = static_cast<uint32_t>(kp.F) * 16;
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-                        const uint64_t ad = sdesc(aq + 32 * kk, 16, 1024, kLayoutSW128);
-                        umma_bf16(tmem + kColP, ad, sdesc(bk + 32 * kk, 16, 1024, kLayoutSW128), idP, acc);
-                        umma_bf16(tmem + kColO, ad, sdesc(bs + 256 * kk, 128, st_sbo, kLayoutNone), idO, acc);
-                    }
-                    umma_commit(&bar[B_PQ_EMPTY0 + pslot]);
-                    // state update of a feature half once its phiK slices are in place
-                    if (!last && (t & 1) == 1) {
-                        if (t == 1) wt.wait(&bar[B_V_FULL], ph_vf);
-                        issue_state_half(tmem, kColS, sbase + L.phik, sbase + L.v, sbase + L.ones,
-                                         t >> 1, false);
-                    }
-                }
-                umma_commit(&bar[B_P_FULL]);
-                if (last) wt.wait(&bar[B_V_FULL], ph_vf);
-                wt.wait(&bar[B_PSM_FULL], ph_psm);
-                tc_fence_after();
-                const uint32_t lbo = L.ones - L.v;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_bf16_ts(tmem + kColO, tmem + kColP + 8 * kk,
-                                 sdesc(sbase + L.v + 2048 * kk, lbo, 1024, kLayoutSW128), idPV, 1u);
-                umma_commit(&bar[B_TILE_DONE]);
-                umma_commit(&bar[B_V_EMPTY]);
-            }
-        }
-    } else {
-        // ----------------------------------------------------------- epilogues
-        const int grp = (warp >= 6) ? 1 : 0;
-        const int sp = warp & 3;
-        const uint32_t row = 32u * sp + lane;
-        const uint32_t trow = tmem + ((32u * sp) << 16);
-        uint32_t ph_qkf = 0, ph_uf = 0, ph_pqe0 = 0, ph_pqe1 = 0, ph_pf = 0, ph_td = 0;
-        int uses0 = 0, uses1 = 0;
-        for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
-            wt.wait(&bar[B_QK_FULL], ph_qkf);
-            float inv, l2i;
-            row_scale(sm + (grp ? L.k : L.q) + row * 128, inv, l2i);
-            warp_arrive(&bar[B_QK_EMPTY]);
-            for (int t = 0; t < NT; ++t) {
-                const int node = (t * kSlice) / kp.m;
-                const float a = kp.a2[node] * inv, b = kp.b2[node] + l2i;
-                const int pslot = t & 1;
-                for (int half = 0; half < 2; ++half) {
-                    wt.wait(&bar[B_U_FULL0 + grp], ph_uf);
-                    tc_fence_after();
-                    uint32_t ur[32], pr[32];
-                    const uint32_t col = grp ? kColU1 : kColU0;
-                    tmem_ld32(trow + col, ur);
-                    tmem_ld32(trow + col + 32, pr);
-                    tmem_wait_ld();
-                    reg_fence(ur);
-                    reg_fence(pr);
-                    tc_fence_before();
-                    warp_arrive(&bar[B_U_EMPTY0 + grp]);
-                    if (grp == 0) {
-                        if (half == 0) {
-                            int& uses = pslot ? uses1 : uses0;
-                            if (uses > 0) wt.wait(&bar[B_PQ_EMPTY0 + pslot], pslot ? ph_pqe1 : ph_pqe0);
-                            ++uses;
+                    for (int half = 0; half < 2; ++half) {
+                        wt.wait(&bar[B_U_FULL0 + grp], ph_uf);
+                        tc_fence_after();
+                        uint32_t ur[32], pr[32];
+                        const uint32_t col = grp ? kColU1 : kColU0;
+                        tmem_ld32(trow + col, ur);
+                        tmem_ld32(trow + col + 32, pr);
+                        tmem_wait_ld();
+                        reg_fence(ur);
+                        reg_fence(pr);
+                        tc_fence_before();
+                        warp_arrive(&bar[B_U_EMPTY0 + grp]);
+                        if (grp == 0) {
+                            if (half == 0) {
+                                int& uses = pslot ? uses1 : uses0;
+                                if (uses > 0) wt.wait(&bar[B_PQ_EMPTY0 + pslot], pslot ? ph_pqe1 : ph_pqe0);
+                                ++uses;
+                            }
+                            phi_sub_epilogue(ur, pr, a, b, sbase + L.phiq + pslot * kTileBytes, row, half,
+                                             nullptr);
+                        } else {
+                            if (half == 0 && pslot == 0 && tile > sg.t_begin)
+                                wt.wait(&bar[B_PK_FREE0 + (t >> 1)], (t >> 1) ? ph_pkf1 : ph_pkf0);
+                            phi_sub_epilogue(ur, pr, a, b, sbase + L.phik + t * kTileBytes, row, half,
+                                             nullptr);
                         }
-                        phi_sub_epilogue(ur, pr, a, b, sbase + L.phiq + pslot * kTileBytes, row, half,
-                                         nullptr);
-                    } else {
-                        phi_sub_epilogue(ur, pr, a, b, sbase + L.phik + t * kTileBytes, row, half,
-                                         nullptr);
                     }
+                    fence_async_smem();
+                    warp_arrive(grp ? pk_full(bar, t) : &bar[B_PQ_FULL0 + pslot]);
                 }
-                fence_async_smem();
-                warp_arrive(&bar[grp ? B_PK_FULL : (B_PQ_FULL0 + pslot)]);
             }
-            if (grp == 1) {
-                // masked scores -> bf16 in place (row i keeps keys j <= i), the A operand of P.V
+        } else {
+            // ------------------------------------------------------------ tile tail
+            const int sp = warp & 3;
+            const uint32_t row = 32u * sp + lane;
+            const uint32_t trow = tmem + ((32u * sp) << 16);
+            uint32_t ph_pf = 0, ph_td = 0;
+            for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+                // masked scores -> bf16 in place (row i keeps keys j <= i), the A operand of P.V.
+                // Key chunk c (32 keys) is below this warp's rows for c < sp, on the diagonal for
+                // c == sp and above it (all zero, not read) for c > sp.
                 wt.wait(&bar[B_P_FULL], ph_pf);
                 tc_fence_after();
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    uint32_t p0[32], p1[32];
-                    tmem_ld32(trow + kColP + 64 * c, p0);
-                    tmem_ld32(trow + kColP + 64 * c + 32, p1);
-                    tmem_wait_ld();
-                    reg_fence(p0);
-                    reg_fence(p1);
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int j = 0; j < 32; j += 2) {
-                        const uint32_t c0 = 64u * c + j;
-                        pk[j >> 1] = pack_bf16((c0 <= row) ? __uint_as_float(p0[j]) : 0.0f,
-                                               (c0 + 1 <= row) ? __uint_as_float(p0[j + 1]) : 0.0f);
-                        pk[16 + (j >> 1)] = pack_bf16((c0 + 32 <= row) ? __uint_as_float(p1[j]) : 0.0f,
-                                                      (c0 + 33 <= row) ? __uint_as_float(p1[j + 1]) : 0.0f);
+    #pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t pk[16];
+                    if (c <= sp) {
+                        uint32_t pv[32];
+                        tmem_ld32(trow + kColP + 32 * c, pv);
+                        tmem_wait_ld();
+                        reg_fence(pv);
+                        if (c < sp) {
+    #pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                pk[j] = pack_bf16(__uint_as_float(pv[2 * j]), __uint_as_float(pv[2 * j + 1]));
+                        } else {
+    #pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                pk[j] = pack_bf16((2 * j <= lane) ? __uint_as_float(pv[2 * j]) : 0.0f,
+                                                  (2 * j + 1 <= lane) ? __uint_as_float(pv[2 * j + 1]) : 0.0f);
+                        }
+                    } else {
+    #pragma unroll
+                        for (int j = 0; j < 16; ++j) pk[j] = 0u;
                     }
-                    tmem_st32(trow + kColP + 32 * c, pk);
+                    tmem_st16(trow + kColP + 16 * c, pk);
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 warp_arrive(&bar[B_PSM_FULL]);
+                if (tile + 1 < sg.t_end) {
+                    // state after this tile (its update finished before the scores did) -> bf16
+                    // copy for the next readout
+                    for (int h = 0; h < halves; ++h) {
+                        const int f = 128 * h + row;
+                        uint32_t r0s[32], r1s[32], zr;
+                        tmem_ld32(trow + kColS + 80 * h, r0s);
+                        tmem_ld32(trow + kColS + 80 * h + 32, r1s);
+                        tmem_ld1(trow + kColS + 80 * h + 64, zr);
+                        tmem_wait_ld();
+                        reg_fence(r0s);
+                        reg_fence(r1s);
+                        reg_fence1(zr);
+                        float sv[64];
+    #pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            sv[e] = __uint_as_float(r0s[e]);
+                            sv[32 + e] = __uint_as_float(r1s[e]);
+                        }
+                        write_state_row(sbase + L.st, kp.F, f, sv, __uint_as_float(zr));
+                    }
+                    fence_async_smem();
+                    tc_fence_before();
+                    warp_arrive(&bar[B_SBF_READY]);
+                }
                 // output: O[:, :64] / (O[:, 64] + eps)
                 wt.wait(&bar[B_TILE_DONE], ph_td);
                 tc_fence_after();
@@ -769,14 +839,14 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 const int grow = tile * kTile + static_cast<int>(row);
                 if (grow < kp.L) {
                     uint4* dst = reinterpret_cast<uint4*>(out + (rowbase + grow) * 64);
-#pragma unroll
+    #pragma unroll
                     for (int q = 0; q < 4; ++q)
                         dst[q] = make_uint4(
                             pack_bf16(__uint_as_float(o0[8 * q]) * rz, __uint_as_float(o0[8 * q + 1]) * rz),
                             pack_bf16(__uint_as_float(o0[8 * q + 2]) * rz, __uint_as_float(o0[8 * q + 3]) * rz),
                             pack_bf16(__uint_as_float(o0[8 * q + 4]) * rz, __uint_as_float(o0[8 * q + 5]) * rz),
                             pack_bf16(__uint_as_float(o0[8 * q + 6]) * rz, __uint_as_float(o0[8 * q + 7]) * rz));
-#pragma unroll
+    #pragma unroll
                     for (int q = 0; q < 4; ++q)
                         dst[4 + q] = make_uint4(
                             pack_bf16(__uint_as_float(o1[8 * q]) * rz, __uint_as_float(o1[8 * q + 1]) * rz),
@@ -785,35 +855,11 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                             pack_bf16(__uint_as_float(o1[8 * q + 6]) * rz, __uint_as_float(o1[8 * q + 7]) * rz));
                     if (den) den[rowbase + grow] = d;
                 }
-                if (tile + 1 < sg.t_end) {
-                    // state after this tile -> bf16 copy for the next readout
-                    for (int h = 0; h < halves; ++h) {
-                        const int f = 128 * h + row;
-                        uint32_t r0s[32], r1s[32], zr;
-                        tmem_ld32(trow + kColS + 80 * h, r0s);
-                        tmem_ld32(trow + kColS + 80 * h + 32, r1s);
-                        tmem_ld1(trow + kColS + 80 * h + 64, zr);
-                        tmem_wait_ld();
-                        reg_fence(r0s);
-                        reg_fence(r1s);
-                        reg_fence1(zr);
-                        float sv[64];
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            sv[e] = __uint_as_float(r0s[e]);
-                            sv[32 + e] = __uint_as_float(r1s[e]);
-                        }
-                        write_state_row(sbase + L.st, kp.F, f, sv, __uint_as_float(zr));
-                    }
-                    fence_async_smem();
-                    tc_fence_before();
-                    warp_arrive(&bar[B_SBF_READY]);
-                }
             }
         }
+        if (!wt.ok) atomicExch(err, 1);
+        drain_after_failure(wt.ok);
     }
-    if (!wt.ok) atomicExch(err, 1);
-    drain_after_failure(wt.ok);
     tc_fence_before();
     __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, 512);
@@ -963,7 +1009,7 @@ cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, 
     if (e != cudaSuccess) return e;
     {
         TraceScope trace_("tc_causal_out", st);
-        k_tc_causal_out<<<BH * nseg, kThreads, sm, st>>>(mq, mk, mv, mw, kp, wsS, wsZ,
+        k_tc_causal_out<<<BH * nseg, kOutThreads, sm, st>>>(mq, mk, mv, mw, kp, wsS, wsZ,
                                                          static_cast<__nv_bfloat16*>(out), den, err);
     }
     return cudaGetLastError();

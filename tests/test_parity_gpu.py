@@ -82,7 +82,8 @@ def _run_fwd(q, k, v, w, causal):
     out = torch.empty((B, H, L, w.Dv), device="cuda", dtype=TDT[w.dtype])
     den = torch.empty((B, H, L), device="cuda", dtype=torch.float32)
     fn = bd.slay_attn_causal_fwd if causal else bd.slay_attn_bidir_fwd
-    fn(qt, kt, vt, out, den, w.R, w.m, w.sketch_seed, _eps(w))
+    ws = fn(qt, kt, vt, out, den, w.R, w.m, w.sketch_seed, _eps(w))
+    bd.slay_kernel_status(ws)          # raises if a kernel stopped on an expired wait
     torch.cuda.synchronize()
     return host(out), host(den)
 
@@ -105,6 +106,22 @@ def test_attn_fwd_small(dt, R, m, L, causal):
     assert rel_l2(gden, wden) <= TOL[dt]
     assert np.isfinite(got).all()
     assert (got[0, 1, min(2, L - 1)] == 0).all()
+
+
+# Enough (b, h) slices that the sequence is cut into few segments, so one CTA walks
+# several 128-token tiles (state carried in tensor memory from tile to tile), with a
+# ragged last tile; and B*H >= 148, where a single segment covers the whole sequence.
+@pytest.mark.parametrize("B,H,L,R,m", [(2, 37, 657, 4, 64), (1, 148, 300, 4, 64),
+                                       (2, 37, 520, 2, 64), (1, 50, 1111, 4, 64)])
+def test_attn_fwd_multi_tile_segments(B, H, L, R, m):
+    w = W.Workload("multitile", B=B, H=H, L=L, R=R, m=m, dtype="bf16", data_seed=17)
+    q, k, v = W.gen_qkv(w)
+    P = params(w)
+    want, wden = O.attn_quadratic(q, k, v, P, True)
+    got, gden = _run_fwd(q, k, v, w, True)
+    assert np.isfinite(got).all()
+    assert rel_l2(got, want) <= TOL["bf16"]
+    assert rel_l2(gden, wden) <= TOL["bf16"]
 
 
 def test_tiny_workload_both_modes():
@@ -156,7 +173,9 @@ def _run_bwd(q, k, v, g, w):
     dq = torch.empty((B, H, L, w.D), device="cuda", dtype=torch.float32)
     dk = torch.empty_like(dq)
     dv = torch.empty((B, H, L, w.Dv), device="cuda", dtype=torch.float32)
-    bd.slay_attn_causal_bwd(qt, kt, vt, out, den, gt, dq, dk, dv, w.R, w.m, w.sketch_seed, _eps(w))
+    ws = bd.slay_attn_causal_bwd(qt, kt, vt, out, den, gt, dq, dk, dv, w.R, w.m, w.sketch_seed,
+                                 _eps(w))
+    bd.slay_kernel_status(ws)
     torch.cuda.synchronize()
     return host(dq), host(dk), host(dv)
 
