@@ -69,7 +69,7 @@ def kernel_work(name, w, op):
     """Algorithmic work of one launch of kernel `name`: (amount, unit, bound).
 
     Per-unit figures (token-head = one row of one (b, h) slice; D = Dv = 64):
-      feature map     bytes: x read (2 B/elem) + phi written in its own dtype
+      feature map     bytes: x read (2 B/elem) + phi written in its own dtype, per row
       causal fwd      flop: 8DF + 4F Dv + (C+1)(F+Dv) per token-head, C = 64
       bidir fwd       flop: 8DF + 4F Dv per token-head
     """
@@ -83,9 +83,13 @@ def kernel_work(name, w, op):
         return th * (4 * D * F + 2 * F * Dv), "flop", "tensor"
     if name in ("tc_bidir_state",):
         return th * (4 * D * F + 2 * F * Dv), "flop", "tensor"
+    # the feature-map workload maps q and k rows (2 th rows, bf16 -> bf16) in one launch;
+    # the CUDA-core attention paths map q and k separately (th rows, fp32 features)
     if name == "tc_feature_map":
-        return th * (D * 2 + F * 2), "byte", "hbm"
+        return 2 * th * (D * 2 + F * 2), "byte", "hbm"
     if name == "simt_feature_map":
+        if op == "feature_map":
+            return 2 * th * (D * 2 + F * 2), "byte", "hbm"
         return th * (D * 2 + F * 4), "byte", "hbm"
     if name == "simt_chunk_state":
         return th * 2 * F * (Dv + 1), "flop", "alu"

@@ -152,13 +152,14 @@ slay_status slay_attn_causal_fwd_noalloc(const void* q, const void* k, const voi
                                          float eps, void* stream);
 
 /* Kernel status of the last attention call that used `workspace` (or, with workspace ==
- * NULL, of the last slay_attn_causal_fwd_noalloc call on the current device).
+ * NULL, of the last slay_attn_causal_fwd_noalloc call and the last slay_feature_map call
+ * on the current device: the library's own status words).
  * The tensor-core kernels coordinate their warps through shared-memory barriers; every
  * wait is bounded (2 s).  A wait that runs out makes the kernel stop early, leave its
  * outputs incomplete and set the status word, the first int of the workspace, which each
  * attention call clears when it is enqueued.  This call copies the word to the host on
  * `stream` and synchronizes the stream.  Returns SLAY_ERR_TIMEOUT if the word is set,
- * SLAY_OK if it is not (or if the no-alloc path never ran on this device),
+ * SLAY_OK if it is not (or if neither of those paths ran on this device),
  * SLAY_ERR_INVALID_ARG for a workspace that is not 256-byte aligned, SLAY_ERR_CUDA if the
  * copy fails.  The status of a call is only defined once it has been enqueued. */
 slay_status slay_kernel_status(const void* workspace, void* stream);

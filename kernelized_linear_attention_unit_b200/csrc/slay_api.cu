@@ -219,7 +219,7 @@ slay_status slay_feature_map(const void* x, void* phi, int64_t n_rows, int D, sl
     if ((s = get_params(D, R, m, seed, eps, &P)) != SLAY_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e;
-    if (in_dt == SLAY_BF16 && out_dt == SLAY_BF16 && tc_supported(SLAY_OP_FEATURE_MAP, 1, 1, 1, R, m))
+    if (in_dt == SLAY_BF16 && out_dt == SLAY_BF16 && P.wB && tc_fmap_supported(D, R, m, n_rows))
         e = tc_feature_map(x, phi, n_rows, P, st);
     else
         e = simt_feature_map(x, phi, n_rows, in_dt, out_dt, P, st);
@@ -294,15 +294,22 @@ slay_status slay_decode_step(const void* q, const void* k, const void* v, float*
 
 slay_status slay_kernel_status(const void* workspace, void* stream)
 {
-    const void* word = workspace ? workspace : noalloc_status_word();
-    if (!word) return SLAY_OK;
-    if (!aligned(word, 256)) return SLAY_ERR_INVALID_ARG;
+    if (workspace && !aligned(workspace, 256)) return SLAY_ERR_INVALID_ARG;
+    // the caller's workspace, or the library's own words: no-alloc scratch and feature map
+    const void* words[2] = {workspace, nullptr};
+    if (!workspace) {
+        words[0] = noalloc_status_word();
+        words[1] = fmap_status_word();
+    }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    int flag = 0;
-    cudaError_t e = cudaMemcpyAsync(&flag, word, sizeof(int), cudaMemcpyDeviceToHost, st);
+    int flags[2] = {0, 0};
+    cudaError_t e = cudaSuccess;
+    for (int i = 0; i < 2 && e == cudaSuccess; ++i)
+        if (words[i])
+            e = cudaMemcpyAsync(&flags[i], words[i], sizeof(int), cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_fail(e);
-    return flag ? SLAY_ERR_TIMEOUT : SLAY_OK;
+    return (flags[0] || flags[1]) ? SLAY_ERR_TIMEOUT : SLAY_OK;
 }
 
 size_t slay_workspace_bytes(slay_op op, slay_dtype dt, int B, int H, int L, int D, int Dv, int R,

@@ -20,7 +20,8 @@ struct Params {
     const float* anT;    // [D][F]   anchors transposed
     const float* om;     // [F][D]   omega, row per feature
     const float* an;     // [F][D]   anchors, row per feature
-    const uint16_t* wB;  // [F/16][2][16][D] bf16 (see tensor-core path), may be null
+    const uint16_t* wB;  // [F/32][64][D] bf16: per 32 features, 32 omega rows then 32
+                         // anchor rows (tensor-core projection operand), may be null
     int D, R, m, F;
     // phi_f = exp2(a2[r] * u + b2[r]) * p^2 with u = omega_f . x^, p = a_f . x^, where
     // a2 = sqrt(2 s_r) log2(e), b2 = log2(sqrt(wt_r/m)) - s_r log2(e).

@@ -37,6 +37,7 @@
 
 #include "slay_tc.h"
 #include "slay_tc_ptx.cuh"
+#include "slay_tc_common.cuh"
 
 namespace slay {
 
@@ -54,7 +55,6 @@ constexpr int kThreads = 384;              // 12 warps (state kernel)
 constexpr int kOutThreads = 512;           // 16 warps (output kernel)
 constexpr int kOnesBytes = kTileBytes;     // [128][64] bf16 ones: the z columns of [V | 1]
 constexpr int kNumSMs = 148;
-constexpr uint64_t kWaitNs = 2000000000ull;
 
 // TMEM column map (one CTA per SM, 512 columns allocated).
 constexpr uint32_t kColU0 = 0;     // 64: q-side projection (32 u | 32 p)
@@ -142,47 +142,6 @@ struct KParams {
     float b2[kMaxR];
 };
 
-// A waiter that stops waiting (and reports) once any wait of this thread timed out.
-struct Waiter {
-    bool ok = true;
-    __device__ __forceinline__ void wait(uint64_t* bar, uint32_t& phase)
-    {
-        ok = mbar_wait(bar, phase, ok ? kWaitNs : 0) && ok;
-        phase ^= 1u;
-    }
-};
-
-__device__ __forceinline__ void drain_after_failure(bool ok)
-{
-    if (ok) return;
-    const uint64_t t0 = global_timer_ns();
-    while (global_timer_ns() - t0 < 20000000ull) {
-    }
-}
-
-// Sum of squares of one 64-element bf16 row (128 bytes; order does not matter, so the
-// swizzle is irrelevant) -> (1/|x|, 2 log2(1/|x|)) with the 1e-12 norm guard.
-__device__ __forceinline__ void row_scale(const unsigned char* row, float& inv, float& l2inv2)
-{
-    const uint4* p = reinterpret_cast<const uint4*>(row);
-    float s = 0.0f;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        const uint4 w = p[c];
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float lo = __uint_as_float(ws[e] << 16);
-            const float hi = __uint_as_float(ws[e] & 0xFFFF0000u);
-            s = fmaf(lo, lo, s);
-            s = fmaf(hi, hi, s);
-        }
-    }
-    const float n = fmaxf(sqrtf(s), 1e-12f);
-    inv = 1.0f / n;
-    l2inv2 = -2.0f * __log2f(n);
-}
-
 // phi of one 32-feature sub-slice from registers holding u (32) and p (32) of this row:
 // phi_j = exp2(a u_j + b) p_j^2, a = a2[r]/|x|, b = b2[r] + 2 log2(1/|x|).  Stores the 32
 // bf16 values as chunks [4*half, 4*half+4) of row `row` of the swizzled tile at tile_addr.
@@ -243,17 +202,6 @@ __device__ __forceinline__ void fill_ones(unsigned char* ones)
     for (int i = threadIdx.x; i < kOnesBytes / 4; i += blockDim.x) p[i] = 0x3F803F80u;  // bf16 1.0
 }
 
-__device__ __forceinline__ unsigned char* aligned_smem(unsigned char* raw)
-{
-    return reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(raw) + 1023) &
-                                            ~uintptr_t(1023));
-}
-
-__device__ __forceinline__ void warp_arrive(uint64_t* bar)
-{
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-}
 
 // ------------------------------------------------------------ state kernel
 // grid = BH * (nseg - 1): segment seg of sequence bh writes
@@ -867,25 +815,6 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
 
 // ------------------------------------------------------------------ host side
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn()
-{
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
 // [BH][L][64] bf16 viewed as a 3-D tensor, 128-token x 64 boxes, 128-byte swizzle;
 // rows past L read as zero.
 bool map_rows(CUtensorMap* m, const void* base, int L, int BH)
@@ -964,11 +893,6 @@ void tc_pack_wb(int D, int R, int m, const uint16_t* om, const uint16_t* an, uin
             std::memcpy(wb + (static_cast<size_t>(n) * 64 + r) * D, src + static_cast<size_t>(f) * D,
                         D * sizeof(uint16_t));
         }
-}
-
-cudaError_t tc_feature_map(const void*, void*, int64_t, const Params&, cudaStream_t)
-{
-    return cudaErrorNotSupported;
 }
 
 cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, float* den, int B,

@@ -19,7 +19,11 @@ size_t tc_wb_elems(int D, int R, int m);
 // Pack bf16 omega / anchors ([F][D] row-major bit patterns) into the operand layout.
 void tc_pack_wb(int D, int R, int m, const uint16_t* om, const uint16_t* an, uint16_t* wb);
 
+// Feature map bf16 -> bf16 on tensor cores: D == 64, m % 32 == 0, F % 128 == 0, F <= 512.
+bool tc_fmap_supported(int D, int R, int m, int64_t n_rows);
 cudaError_t tc_feature_map(const void* x, void* phi, int64_t n, const Params& P, cudaStream_t st);
+// Device address of the feature-map kernel's status word (set when a bounded wait ran out).
+const void* fmap_status_word();
 cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, float* den,
                         int B, int H, int L, const Params& P, float eps, bool causal, void* ws,
                         cudaStream_t st);

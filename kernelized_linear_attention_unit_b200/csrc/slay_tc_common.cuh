@@ -1,0 +1,92 @@
+// slay_tc_common.cuh -- pieces shared by the tensor-core kernels: bounded waits, the
+// per-row norm scale, shared-memory alignment and the tensor-map encoder.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "slay_tc_ptx.cuh"
+
+namespace slay {
+namespace tc {
+
+constexpr uint64_t kWaitNs = 2000000000ull;   // bound of every mbarrier wait (2 s)
+
+// A waiter that stops waiting (and reports) once any wait of this thread timed out.
+struct Waiter {
+    bool ok = true;
+    __device__ __forceinline__ void wait(uint64_t* bar, uint32_t& phase)
+    {
+        ok = mbar_wait(bar, phase, ok ? kWaitNs : 0) && ok;
+        phase ^= 1u;
+    }
+};
+
+// One arrival per warp (lane 0 after the warp has converged).
+__device__ __forceinline__ void warp_arrive(uint64_t* bar)
+{
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
+__device__ __forceinline__ void drain_after_failure(bool ok)
+{
+    if (ok) return;
+    const uint64_t t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < 20000000ull) {
+    }
+}
+
+// Sum of squares of one 64-element bf16 row (128 bytes; order does not matter, so the
+// swizzle is irrelevant) -> (1/|x|, 2 log2(1/|x|)) with the 1e-12 norm guard.
+__device__ __forceinline__ void row_scale(const unsigned char* row, float& inv, float& l2inv2)
+{
+    const uint4* p = reinterpret_cast<const uint4*>(row);
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // independent partial sums: short FMA chains
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const uint4 w = p[c];
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float lo = __uint_as_float(ws[e] << 16);
+            const float hi = __uint_as_float(ws[e] & 0xFFFF0000u);
+            acc[e] = fmaf(lo, lo, acc[e]);
+            acc[e] = fmaf(hi, hi, acc[e]);
+        }
+    }
+    const float s = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    const float n = fmaxf(sqrtf(s), 1e-12f);
+    inv = 1.0f / n;
+    l2inv2 = -2.0f * __log2f(n);
+}
+
+__device__ __forceinline__ unsigned char* aligned_smem(unsigned char* raw)
+{
+    return reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(raw) + 1023) &
+                                            ~uintptr_t(1023));
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+}  // namespace tc
+}  // namespace slay

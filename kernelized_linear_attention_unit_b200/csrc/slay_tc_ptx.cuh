@@ -75,8 +75,28 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t addr, uint32_t phas
     return done != 0;
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint32_t addr, uint32_t phase)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(addr), "r"(phase)
+        : "memory");
+    return done != 0;
+}
+
+#ifndef SLAY_WAIT_MODE
+#define SLAY_WAIT_MODE 0
+#endif
+
 // Bounded wait for the completion of `phase`.  Gives up after `limit_ns` of global time
 // and returns false (the caller records an error and leaves); never spins forever.
+// Mode 0 suspends the thread between polls (try_wait with a time hint), mode 1 polls with
+// try_wait (hardware-chosen suspension), mode 2 spins on test_wait.
+template <int kMode = SLAY_WAIT_MODE>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase,
                                           uint64_t limit_ns = 2000000000ull)
 {
@@ -84,7 +104,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase,
     if (mbar_try_wait(addr, phase)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 0; it < (1u << 30); ++it) {
-        if (mbar_try_wait_sleep(addr, phase, 100000u)) return true;
+        if (kMode == 0) {
+            if (mbar_try_wait_sleep(addr, phase, 100000u)) return true;
+        } else if (kMode == 1) {
+            if (mbar_try_wait(addr, phase)) return true;
+        } else {
+            if (mbar_test_wait(addr, phase)) return true;
+        }
         if (global_timer_ns() - t0 > limit_ns) return false;
     }
     return false;
@@ -109,6 +135,39 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
+}
+
+// Shared -> global tiled store (bulk async group of this thread); rows or columns outside
+// the tensor are not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int c0, int c1)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(smem_u32(src)), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Wait until at most N bulk groups of this thread still read their shared-memory source.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read()
+{
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// Wait until at most N bulk groups of this thread are incomplete (writes done).
+template <int N>
+__device__ __forceinline__ void bulk_wait()
+{
+    asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Barrier `id` (1..15) among `n` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t n)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map)

@@ -54,7 +54,10 @@ def small(dt, R, m, L, B=1, H=2, correlated=False, seed=21):
                                                  ("f32", "f32", 4, 64, 130),
                                                  ("bf16", "bf16", 4, 64, 1000),
                                                  ("bf16", "f32", 8, 64, 333),
-                                                 ("bf16", "bf16", 8, 64, 4097)])
+                                                 ("bf16", "bf16", 8, 64, 4097),
+                                                 ("bf16", "bf16", 2, 64, 40000),
+                                                 ("bf16", "bf16", 4, 32, 38001),
+                                                 ("bf16", "bf16", 3, 64, 777)])
 def test_feature_map(dt_in, dt_out, R, m, n):
     w = small(dt_in, R, m, n, B=1, H=1)
     q, _, _ = W.gen_qkv(w)
@@ -66,6 +69,7 @@ def test_feature_map(dt_in, dt_out, R, m, n):
     xt = dev(x, dt_in)
     phi = torch.empty((n, R * m), device="cuda", dtype=TDT[dt_out])
     bd.slay_feature_map(xt, phi, R, m, w.sketch_seed, _eps(w))
+    bd.slay_kernel_status(None)
     torch.cuda.synchronize()
     got = host(phi)
     tol = TOL["bf16"] if "bf16" in (dt_in, dt_out) else TOL["f32"]
