@@ -137,6 +137,7 @@ __device__ __forceinline__ Seg segment_of(int index, int nseg, int ntiles)
 
 struct KParams {
     int L, F, m, nseg, ntiles;
+    int all_segs;      // state kernel: 1 = every segment (bidirectional), 0 = all but the last
     float eps;
     float a2[kMaxR];
     float b2[kMaxR];
@@ -204,7 +205,8 @@ __device__ __forceinline__ void fill_ones(unsigned char* ones)
 
 
 // ------------------------------------------------------------ state kernel
-// grid = BH * (nseg - 1): segment seg of sequence bh writes
+// grid = BH * (nseg - 1) (causal: the last segment's sum is never needed) or BH * nseg
+// (bidirectional): segment seg of sequence bh writes
 //   ws_S[bh][seg][f][e] = sum_{t in seg} phi(k_t)_f v_t[e],  ws_z[bh][seg][f] = sum phi(k_t)_f
 // Projections are 64 features wide (N = 128: two packed 32-feature operands), double
 // buffered in TMEM; epilogue group g takes the projections n with n % 2 == g.  Tile i uses
@@ -223,7 +225,8 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int NT = kp.F / kSlice, halves = kp.F / 128;
     const uint32_t phik_bytes = NT * kTileBytes;
-    const Seg sg = segment_of(blockIdx.x + blockIdx.x / (kp.nseg - 1), kp.nseg, kp.ntiles);
+    const Seg sg = kp.all_segs ? segment_of(blockIdx.x, kp.nseg, kp.ntiles)
+                               : segment_of(blockIdx.x + blockIdx.x / (kp.nseg - 1), kp.nseg, kp.ntiles);
     constexpr uint32_t kColUS = 0;     // 2 x 128: projections
     constexpr uint32_t kColSS = 256;   // 2 x 80 : [S | z]
     // barrier roles here: QK_* hold the K tile; VF(b) / VE(b) the V buffers; TD(b) = the
@@ -813,6 +816,268 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
     if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
+// ------------------------------------------------------ bidirectional readout
+// out_i = phi(q_i)^T S / (phi(q_i)^T z + eps) with the state [S | z] of the whole sequence.
+// grid = BH * nseg; a CTA walks the tiles of one segment.  Warp 0 loads q tiles (two
+// buffers) and projection operands; warp 2 issues the q projections alternately into U0 /
+// U1; warps 4-7 and 8-11 turn them into phi(q) (group g writes the 32-feature half g of
+// each 64-feature slice); warp 1 issues the readout O = phiQ [S | z] (N = 80) slice by slice;
+// warps 12-15 first build the bf16 copy of the summed state, then write the outputs.
+struct SmemBidir {
+    uint32_t w, q, phiq, st, bar, tmem, total;
+};
+
+__host__ __device__ inline SmemBidir smem_bidir_layout(int F)
+{
+    SmemBidir s;
+    s.w = 0;
+    s.q = kWSlots * kWBytes;                // 2 buffers
+    s.phiq = s.q + 2 * kTileBytes;          // 2 slots of 64 features
+    s.st = s.phiq + 2 * kTileBytes;
+    s.bar = s.st + (F / kSlice) * kStBytes;
+    s.tmem = s.bar + NUM_BARS * 8;
+    s.total = s.tmem + 16;
+    return s;
+}
+
+// barrier roles here: QK_FULL / QK_EMPTY and V_FULL / V_EMPTY hold q buffers 0 / 1
+__global__ void __launch_bounds__(kOutThreads, 1)
+k_tc_bidir_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmw,
+               KParams kp, const float* __restrict__ wsS, const float* __restrict__ wsZ,
+               __nv_bfloat16* __restrict__ out, float* __restrict__ den, int* __restrict__ err)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* sm = aligned_smem(smem_raw);
+    const SmemBidir L = smem_bidir_layout(kp.F);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L.bar);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L.tmem);
+    const uint32_t sbase = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int NT = kp.F / kSlice, NS = kp.F / kSub, halves = kp.F / 128;
+    const Seg sg = segment_of(blockIdx.x, kp.nseg, kp.ntiles);
+    // q buffer b: full / empty barriers
+    auto QF = [bar](int b) { return &bar[b ? B_V_FULL : B_QK_FULL]; };
+    auto QE = [bar](int b) { return &bar[b ? B_V_EMPTY : B_QK_EMPTY]; };
+
+    if (warp == 1) {
+        tmem_alloc(tslot, 256);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bar[i], 1);
+        mbar_init(QE(0), 1 + 8);
+        mbar_init(QE(1), 1 + 8);
+        mbar_init(&bar[B_U_EMPTY0], 4);
+        mbar_init(&bar[B_U_EMPTY1], 4);
+        mbar_init(&bar[B_PQ_FULL0], 8);
+        mbar_init(&bar[B_PQ_FULL1], 8);
+        mbar_init(&bar[B_O_EMPTY], 4);
+        mbar_fence_init();
+        tma_prefetch_desc(&tmq);
+        tma_prefetch_desc(&tmw);
+    }
+    {   // the state copy: columns 65..79 stay zero
+        uint4* p = reinterpret_cast<uint4*>(sm + L.st);
+        for (int i = tid; i < NT * kStBytes / 16; i += kOutThreads) p[i] = make_uint4(0, 0, 0, 0);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+    if (warp >= 12) {   // [S | z] of the whole sequence: sum of all its segments
+        const int sp = warp & 3;
+        const uint32_t row = 32u * sp + lane;
+        for (int h = 0; h < halves; ++h) {
+            const int f = 128 * h + row;
+            float acc[64];
+#pragma unroll
+            for (int e = 0; e < 64; ++e) acc[e] = 0.0f;
+            float zf = 0.0f;
+            for (int s = 0; s < kp.nseg; ++s) {
+                const size_t segidx = static_cast<size_t>(sg.bh) * kp.nseg + s;
+                const float4* src = reinterpret_cast<const float4*>(wsS + (segidx * kp.F + f) * 64);
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const float4 x = src[q];
+                    acc[4 * q] += x.x; acc[4 * q + 1] += x.y; acc[4 * q + 2] += x.z; acc[4 * q + 3] += x.w;
+                }
+                zf += wsZ[segidx * kp.F + f];
+            }
+            write_state_row(sbase + L.st, kp.F, f, acc, zf);
+        }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    constexpr uint32_t kColO2 = 128;   // O after the two 64-column projection buffers
+    Waiter wt;
+    const int64_t rowbase = static_cast<int64_t>(sg.bh) * kp.L;
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t ph_qe = 0, ph_we = (1u << kWSlots) - 1u;
+            int n_glob = 0;
+            for (int tile = sg.t_begin, it = 0; tile < sg.t_end; ++tile, ++it) {
+                const int qb = it & 1;
+                if (it >= 2) {
+                    uint32_t ph = (ph_qe >> qb) & 1u;
+                    wt.wait(QE(qb), ph);
+                    ph_qe ^= 1u << qb;
+                }
+                mbar_arrive_expect_tx(QF(qb), kTileBytes);
+                tma_load_3d(sm + L.q + qb * kTileBytes, &tmq, QF(qb), 0, tile * kTile, sg.bh);
+                for (int n = 0; n < NS; ++n, ++n_glob) {
+                    const int slot = n_glob % kWSlots;
+                    uint32_t ph = (ph_we >> slot) & 1u;
+                    wt.wait(&bar[B_W_EMPTY0 + slot], ph);
+                    ph_we ^= (1u << slot);
+                    mbar_arrive_expect_tx(&bar[B_W_FULL0 + slot], kWBytes);
+                    tma_load_2d(sm + L.w + slot * kWBytes, &tmw, &bar[B_W_FULL0 + slot], 0, n * 64);
+                }
+            }
+        }
+    } else if (warp == 2) {
+        if (lane == 0) {
+            uint32_t ph_qf = 0, ph_wf = 0, ph_ue = 0x3u;
+            int n_glob = 0;
+            for (int tile = sg.t_begin, it = 0; tile < sg.t_end; ++tile, ++it) {
+                const int qb = it & 1;
+                uint32_t ph = (ph_qf >> qb) & 1u;
+                wt.wait(QF(qb), ph);
+                ph_qf ^= 1u << qb;
+                for (int n = 0; n < NS; ++n, ++n_glob) {
+                    const int slot = n_glob % kWSlots, g = n & 1;
+                    uint32_t pw = (ph_wf >> slot) & 1u;
+                    wt.wait(&bar[B_W_FULL0 + slot], pw);
+                    ph_wf ^= (1u << slot);
+                    uint32_t pu = (ph_ue >> g) & 1u;
+                    wt.wait(&bar[B_U_EMPTY0 + g], pu);
+                    ph_ue ^= 1u << g;
+                    tc_fence_after();
+                    issue_projection(tmem + 64 * g, sbase + L.q + qb * kTileBytes,
+                                     sbase + L.w + slot * kWBytes);
+                    umma_commit(&bar[B_U_FULL0 + g]);
+                    umma_commit(&bar[B_W_EMPTY0 + slot]);
+                }
+                umma_commit(QE(qb));
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            uint32_t ph_pqf = 0, ph_oe = 0;
+            constexpr uint32_t idO = idesc_bf16(128, 80, 0, 1);
+            const uint32_t st_sbo = static_cast<uint32_t>(kp.F) * 16;
+            for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+                for (int t = 0; t < NT; ++t) {
+                    const int pslot = t & 1;
+                    uint32_t ph = (ph_pqf >> pslot) & 1u;
+                    wt.wait(&bar[B_PQ_FULL0 + pslot], ph);
+                    ph_pqf ^= 1u << pslot;
+                    if (t == 0 && tile > sg.t_begin) wt.wait(&bar[B_O_EMPTY], ph_oe);
+                    tc_fence_after();
+                    const uint32_t aq = sbase + L.phiq + pslot * kTileBytes;
+                    const uint32_t bs = sbase + L.st + t * (kSlice / 8) * 128;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_bf16(tmem + kColO2, sdesc(aq + 32 * kk, 16, 1024, kLayoutSW128),
+                                  sdesc(bs + 256 * kk, 128, st_sbo, kLayoutNone), idO,
+                                  (t > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&bar[B_PQ_EMPTY0 + pslot]);
+                }
+                umma_commit(&bar[B_TILE_DONE]);
+            }
+        }
+    } else if (warp >= 4 && warp < 12) {
+        // phi(q): group g takes the projections n = 2t + g, i.e. half g of slice t
+        const int g = (warp >= 8) ? 1 : 0;
+        const int sp = warp & 3;
+        const uint32_t row = 32u * sp + lane;
+        const uint32_t trow = tmem + ((32u * sp) << 16);
+        uint32_t ph_qf = 0, ph_uf = 0, ph_pqe = 0;
+        int uses[2] = {0, 0};
+        for (int tile = sg.t_begin, it = 0; tile < sg.t_end; ++tile, ++it) {
+            const int qb = it & 1;
+            uint32_t ph = (ph_qf >> qb) & 1u;
+            wt.wait(QF(qb), ph);
+            ph_qf ^= 1u << qb;
+            float inv, l2i;
+            row_scale(sm + L.q + qb * kTileBytes + row * 128, inv, l2i);
+            warp_arrive(QE(qb));
+            for (int t = 0; t < NT; ++t) {
+                const int node = (t * kSlice) / kp.m;
+                const float a = kp.a2[node] * inv, b = kp.b2[node] + l2i;
+                const int pslot = t & 1;
+                wt.wait(&bar[B_U_FULL0 + g], ph_uf);
+                tc_fence_after();
+                uint32_t ur[32], pr[32];
+                tmem_ld32(trow + 64 * g, ur);
+                tmem_ld32(trow + 64 * g + 32, pr);
+                tmem_wait_ld();
+                reg_fence(ur);
+                reg_fence(pr);
+                tc_fence_before();
+                warp_arrive(&bar[B_U_EMPTY0 + g]);
+                if (uses[pslot] > 0) {   // both groups wait for the same completion
+                    uint32_t pe = (ph_pqe >> pslot) & 1u;
+                    wt.wait(&bar[B_PQ_EMPTY0 + pslot], pe);
+                    ph_pqe ^= 1u << pslot;
+                }
+                ++uses[pslot];
+                phi_sub_epilogue(ur, pr, a, b, sbase + L.phiq + pslot * kTileBytes, row, g, nullptr);
+                fence_async_smem();
+                warp_arrive(&bar[B_PQ_FULL0 + pslot]);
+            }
+        }
+    } else if (warp >= 12) {
+        // output: O[:, :64] / (O[:, 64] + eps)
+        const int sp = warp & 3;
+        const uint32_t row = 32u * sp + lane;
+        const uint32_t trow = tmem + ((32u * sp) << 16);
+        uint32_t ph_td = 0;
+        for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+            wt.wait(&bar[B_TILE_DONE], ph_td);
+            tc_fence_after();
+            uint32_t o0[32], o1[32], dr;
+            tmem_ld32(trow + kColO2, o0);
+            tmem_ld32(trow + kColO2 + 32, o1);
+            tmem_ld1(trow + kColO2 + 64, dr);
+            tmem_wait_ld();
+            reg_fence(o0);
+            reg_fence(o1);
+            reg_fence1(dr);
+            tc_fence_before();
+            warp_arrive(&bar[B_O_EMPTY]);
+            const float d = __uint_as_float(dr);
+            const float rz = 1.0f / (d + kp.eps);
+            const int grow = tile * kTile + static_cast<int>(row);
+            if (grow < kp.L) {
+                uint4* dst = reinterpret_cast<uint4*>(out + (rowbase + grow) * 64);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    dst[q] = make_uint4(
+                        pack_bf16(__uint_as_float(o0[8 * q]) * rz, __uint_as_float(o0[8 * q + 1]) * rz),
+                        pack_bf16(__uint_as_float(o0[8 * q + 2]) * rz, __uint_as_float(o0[8 * q + 3]) * rz),
+                        pack_bf16(__uint_as_float(o0[8 * q + 4]) * rz, __uint_as_float(o0[8 * q + 5]) * rz),
+                        pack_bf16(__uint_as_float(o0[8 * q + 6]) * rz, __uint_as_float(o0[8 * q + 7]) * rz));
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    dst[4 + q] = make_uint4(
+                        pack_bf16(__uint_as_float(o1[8 * q]) * rz, __uint_as_float(o1[8 * q + 1]) * rz),
+                        pack_bf16(__uint_as_float(o1[8 * q + 2]) * rz, __uint_as_float(o1[8 * q + 3]) * rz),
+                        pack_bf16(__uint_as_float(o1[8 * q + 4]) * rz, __uint_as_float(o1[8 * q + 5]) * rz),
+                        pack_bf16(__uint_as_float(o1[8 * q + 6]) * rz, __uint_as_float(o1[8 * q + 7]) * rz));
+                if (den) den[rowbase + grow] = d;
+            }
+        }
+    }
+    if (!wt.ok) atomicExch(err, 1);
+    drain_after_failure(wt.ok);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tmem, 256);
+}
+
 // ------------------------------------------------------------------ host side
 
 // [BH][L][64] bf16 viewed as a 3-D tensor, 128-token x 64 boxes, 128-byte swizzle;
@@ -859,7 +1124,7 @@ size_t smem_bytes_state(int F) { return smem_state_layout(F).total + 1024; }
 bool tc_supported(slay_op op, int B, int H, int L, int R, int m)
 {
     const int F = R * m;
-    if (op != SLAY_OP_CAUSAL_FWD) return false;
+    if (op != SLAY_OP_CAUSAL_FWD && op != SLAY_OP_BIDIR_FWD) return false;
     if (m % kSlice != 0 || F % 128 != 0 || F > 256) return false;
     if (static_cast<int64_t>(B) * H * L <= 0) return false;
     return smem_bytes_out(F) <= 232448;
@@ -867,7 +1132,7 @@ bool tc_supported(slay_op op, int B, int H, int L, int R, int m)
 
 size_t tc_workspace_bytes(slay_op op, int B, int H, int L, int R, int m)
 {
-    if (op != SLAY_OP_CAUSAL_FWD) return 0;
+    if (op != SLAY_OP_CAUSAL_FWD && op != SLAY_OP_BIDIR_FWD) return 0;
     const int F = R * m;
     const int BH = B * H;
     const int ntiles = (L + kTile - 1) / kTile;
@@ -899,7 +1164,7 @@ cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, 
                         int H, int L, const Params& P, float eps, bool causal, void* ws,
                         cudaStream_t st)
 {
-    if (!causal || !P.wB) return cudaErrorNotSupported;
+    if (!P.wB) return cudaErrorNotSupported;
     const int BH = B * H, F = P.F;
     const int ntiles = (L + kTile - 1) / kTile;
     const int nseg = choose_nseg(BH, ntiles);
@@ -909,6 +1174,7 @@ cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, 
         return cudaErrorInvalidValue;
     KParams kp;
     kp.L = L; kp.F = F; kp.m = P.m; kp.nseg = nseg; kp.ntiles = ntiles; kp.eps = eps;
+    kp.all_segs = causal ? 0 : 1;
     for (int r = 0; r < kMaxR; ++r) { kp.a2[r] = P.a2[r]; kp.b2[r] = P.b2[r]; }
     char* w = static_cast<char*>(ws);
     int* err = reinterpret_cast<int*>(w);
@@ -917,6 +1183,26 @@ cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, 
     float* wsZ = reinterpret_cast<float*>(w + kWsHeader + ((per * 64 * sizeof(float) + 255) & ~size_t(255)));
     cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), st);
     if (e != cudaSuccess) return e;
+    if (!causal) {
+        // every segment's sum, then the readout against their total
+        const size_t sms = smem_bytes_state(F);
+        e = cudaFuncSetAttribute(k_tc_causal_state, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(sms));
+        if (e != cudaSuccess) return e;
+        {
+            TraceScope trace_("tc_bidir_state", st);
+            k_tc_causal_state<<<BH * nseg, kThreads, sms, st>>>(mk, mv, mw, kp, wsS, wsZ, err);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+        const size_t smb = smem_bidir_layout(F).total + 1024;
+        e = cudaFuncSetAttribute(k_tc_bidir_out, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smb));
+        if (e != cudaSuccess) return e;
+        TraceScope trace_("tc_bidir_out", st);
+        k_tc_bidir_out<<<BH * nseg, kOutThreads, smb, st>>>(mq, mw, kp, wsS, wsZ,
+                                                           static_cast<__nv_bfloat16*>(out), den, err);
+        return cudaGetLastError();
+    }
     if (nseg > 1) {
         const size_t sm = smem_bytes_state(F);
         e = cudaFuncSetAttribute(k_tc_causal_state, cudaFuncAttributeMaxDynamicSharedMemorySize,
