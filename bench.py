@@ -225,6 +225,28 @@ def config_of(w, op):
 
 # ----------------------------------------------------------------- GPU leg
 
+def rank_workload(w, rank):
+    """The batch rank `rank` times: same shapes, data seed offset by 1000 * rank (weak
+    scaling, independent sequences per rank, no exchange)."""
+    return W.Workload(**{**w.__dict__, "data_seed": w.data_seed + 1000 * rank})
+
+
+def max_over_ranks(x, world, device="cpu"):
+    """Max of a per-rank float over all ranks (identity at world size 1)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, units_per_step, steps, max_total_ms):
+    """Whole-job units per second: every rank processed units_per_step per step."""
+    return world * units_per_step * steps / (max_total_ms / 1e3)
+
+
 def run_ours(args, w, op):
     import torch
     import torch.distributed as dist
@@ -252,7 +274,7 @@ def run_ours(args, w, op):
         return h
 
     # inputs: each rank draws its own batch (data seed offset by rank)
-    wr = W.Workload(**{**w.__dict__, "data_seed": w.data_seed + 1000 * rank})
+    wr = rank_workload(w, rank)
     if op == "decode":
         qn, kn, vn, Sn, zn = W.gen_decode(wr)
         q, k, v = to_dev(qn), to_dev(kn), to_dev(vn)
@@ -339,12 +361,8 @@ def run_ours(args, w, op):
     trace = bd.slay_trace_read()
     clocks = clk.stop()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    value = world * units_per_step * args.steps / (total_ms / 1e3)
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
+    value = job_throughput(world, units_per_step, args.steps, total_ms)
 
     # ---- end to end through the same public call: H2D of inputs, the call, D2H of result
     h2d = sum(x.numel() * x.element_size() for x in host_in)
@@ -363,12 +381,8 @@ def run_ours(args, w, op):
         e_ends[i].record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends))
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = world * units_per_step * args.steps / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)), world, dev)
+    e2e = job_throughput(world, units_per_step, args.steps, e2e_ms)
 
     # ---- roofline of the dominant kernel (largest total device time in the timed region)
     peaks, peak_src = load_peaks()

@@ -1,0 +1,84 @@
+"""Multi-rank host logic of bench.py on CPU: two gloo ranks (world size 2).
+
+The forward shards over independent (b, h) sequences, so the only cross-rank steps are the
+barriers around the timed region and the max over ranks of the device time; each rank
+draws its own batch.  These tests run those steps with real process groups (gloo over
+127.0.0.1), no GPU.
+"""
+import datetime
+import os
+import socket
+import sys
+import tempfile
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from kernelized_linear_attention_unit_b200 import workloads as W  # noqa: E402
+
+
+def _free_port():
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, outdir):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        local_ms = 10.0 + 5.0 * rank                      # rank 1 is the slow one
+        dist.barrier()
+        slowest = bench.max_over_ranks(local_ms, world)
+        value = bench.job_throughput(world, 16384, 4, slowest)
+        wr = bench.rank_workload(W.CAUSAL_2K, rank)
+        small = W.Workload(**{**wr.__dict__, "B": 1, "H": 2, "L": 16})
+        q, _, _ = W.gen_qkv(small)
+        np.save(os.path.join(outdir, "r%d.npy" % rank),
+                np.array([slowest, value, wr.data_seed, float(q.astype(np.float64).sum())]))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.fixture(scope="module")
+def two_ranks():
+    import torch.multiprocessing as mp
+    outdir = tempfile.mkdtemp(prefix="slay_gloo_")
+    mp.spawn(_rank_main, args=(2, _free_port(), outdir), nprocs=2, join=True)
+    return [np.load(os.path.join(outdir, "r%d.npy" % r)) for r in range(2)]
+
+
+def test_time_is_the_max_over_ranks(two_ranks):
+    for r in two_ranks:
+        assert r[0] == 15.0
+
+
+def test_value_counts_every_rank_over_the_slowest_time(two_ranks):
+    # 2 ranks x 16384 tokens x 4 steps in 15 ms
+    for r in two_ranks:
+        assert r[1] == pytest.approx(2 * 16384 * 4 / 0.015)
+
+
+def test_each_rank_draws_its_own_batch(two_ranks):
+    assert two_ranks[1][2] - two_ranks[0][2] == 1000
+    assert two_ranks[0][3] != two_ranks[1][3]
+
+
+def test_single_rank_is_identity():
+    assert bench.max_over_ranks(7.5, 1) == 7.5
+    assert bench.job_throughput(1, 100, 10, 1000.0) == pytest.approx(1000.0)
+
+
+def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
+    class Args:
+        gpus, steps, warmup = 2, 1, 1
+    monkeypatch.setenv("RANK", "1")
+    assert bench.run_reference(Args(), W.TINY, "causal") == 0
+    assert capsys.readouterr().out == ""
