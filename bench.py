@@ -65,6 +65,29 @@ def alu_peak_tflops(sm_mhz):
     return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
 
 
+def profiled_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summaries under profiles/
+    (lines "traffic: <kernel> <bytes> <sha256[:16] of its sources> <sources>"), or None
+    when no capture exists or the kernel's sources changed since it was taken."""
+    import glob
+    import hashlib
+    csrc = os.path.join(ROOT, "kernelized_linear_attention_unit_b200", "csrc")
+    for fn in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        for line in open(fn):
+            parts = line.split()
+            if len(parts) != 5 or parts[0] != "traffic:" or parts[1] != kernel:
+                continue
+            h = hashlib.sha256()
+            try:
+                for src in parts[4].split("+"):
+                    with open(os.path.join(csrc, src), "rb") as f:
+                        h.update(f.read())
+            except OSError:
+                return None
+            return int(parts[2]) if h.hexdigest()[:16] == parts[3] else None
+    return None
+
+
 def kernel_work(name, w, op):
     """Algorithmic work of one launch of kernel `name`: (amount, unit, bound).
 
@@ -407,7 +430,7 @@ def run_ours(args, w, op):
                 peak = alu_peak_tflops(peaks.get("sm_max_mhz", 1965.0))
                 u = "TFLOP/s"
             roofline = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak,
-                        "unit": u, "frac": achieved / peak, "traffic": None,
+                        "unit": u, "frac": achieved / peak, "traffic": profiled_traffic(dom),
                         "peak_source": peak_src + (" (fp32 FFMA: 148 SMs x 128 x 2 x max clock)"
                                                    if bound == "alu" else ""),
                         "algorithmic_%s_per_launch" % kind: amount,
