@@ -102,6 +102,12 @@ def kernel_work(name, w, op):
         return th * (8 * D * F + 4 * F * Dv + (C_CHUNK + 1) * (F + Dv)), "flop", "tensor"
     if name in ("tc_causal_state",):
         return th * (4 * D * F + 2 * F * Dv), "flop", "tensor"
+    # stored-phi(k) form: the state kernel maps k (its own segment sums are not algorithmic
+    # work), the output kernel does the rest of the causal forward
+    if name == "tc_kphi_state":
+        return th * (4 * D * F), "flop", "tensor"
+    if name == "tc_qphi_out":
+        return th * (4 * D * F + 4 * F * Dv + (C_CHUNK + 1) * (F + Dv)), "flop", "tensor"
     if name in ("tc_bidir_out",):
         return th * (4 * D * F + 2 * F * Dv), "flop", "tensor"
     if name in ("tc_bidir_state",):

@@ -30,7 +30,7 @@ class SlayError(RuntimeError):
         self.status = status
         msg = "%s: %s" % (where, lib().slay_status_string(status).decode())
         detail = lib().slay_last_error().decode()
-        if status == SLAY_ERR_CUDA and detail:
+        if status in (SLAY_ERR_CUDA, SLAY_ERR_TIMEOUT) and detail:
             msg += " (%s)" % detail
         super().__init__(msg)
 

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstdio>
 #include <cstdint>
 #include <cstring>
 #include <map>
@@ -27,6 +28,8 @@ slay_status cuda_fail(cudaError_t e)
     g_last_error = cudaGetErrorString(e);
     return SLAY_ERR_CUDA;
 }
+
+void set_last_error(const char* msg) { g_last_error = msg; }
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -309,7 +312,16 @@ slay_status slay_kernel_status(const void* workspace, void* stream)
             e = cudaMemcpyAsync(&flags[i], words[i], sizeof(int), cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_fail(e);
-    return (flags[0] || flags[1]) ? SLAY_ERR_TIMEOUT : SLAY_OK;
+    for (int i = 0; i < 2; ++i)
+        if (flags[i]) {
+            char msg[96];
+            std::snprintf(msg, sizeof msg,
+                          "a bounded wait ran out (barrier at shared-memory offset 0x%x)",
+                          static_cast<unsigned>(flags[i]) & 0xFFFFu);
+            set_last_error(msg);
+            return SLAY_ERR_TIMEOUT;
+        }
+    return SLAY_OK;
 }
 
 size_t slay_workspace_bytes(slay_op op, slay_dtype dt, int B, int H, int L, int D, int Dv, int R,

@@ -149,8 +149,11 @@ extern "C" slay_status slay_attn_causal_fwd_noalloc(const void* q, const void* k
     if (s != SLAY_OK) return s;
     if (static_cast<int64_t>(B) * H * L == 0) return SLAY_OK;
     if (den && (reinterpret_cast<uintptr_t>(den) % 4) != 0) return SLAY_ERR_INVALID_ARG;
-    if (attn_ws(SLAY_OP_CAUSAL_FWD, dt, B, H, L, Dv, R, m) > kScratchBytes)
-        return SLAY_ERR_UNSUPPORTED;
+    // the tensor-core path runs in its low-memory form here (phi(k) recomputed, not stored)
+    const bool tc = dt == SLAY_BF16 && tc_supported(SLAY_OP_CAUSAL_FWD, B, H, L, R, m);
+    const size_t need = tc ? tc_workspace_bytes(SLAY_OP_CAUSAL_FWD, B, H, L, R, m, true)
+                           : attn_ws(SLAY_OP_CAUSAL_FWD, dt, B, H, L, Dv, R, m);
+    if (need > kScratchBytes) return SLAY_ERR_UNSUPPORTED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     std::lock_guard<std::mutex> lock(g_mu);
     int dev = 0;
@@ -170,8 +173,8 @@ extern "C" slay_status slay_attn_causal_fwd_noalloc(const void* q, const void* k
         if ((s = load_params(&slot, D, R, m, seed, eps, st)) != SLAY_OK) return s;
     }
     cudaError_t e;
-    if (dt == SLAY_BF16 && tc_supported(SLAY_OP_CAUSAL_FWD, B, H, L, R, m))
-        e = tc_attn_fwd(q, k, v, out, den, B, H, L, slot.P, eps, true, slot.scratch, st);
+    if (tc)
+        e = tc_attn_fwd(q, k, v, out, den, B, H, L, slot.P, eps, true, slot.scratch, st, true);
     else if ((e = cudaMemsetAsync(slot.scratch, 0, sizeof(int), st)) == cudaSuccess)
         e = simt_attn_fwd(q, k, v, out, den, B, H, L, dt, slot.P, eps, true,
                           slot.scratch + kWsHeader, st);

@@ -211,10 +211,14 @@ __device__ __forceinline__ void fill_ones(unsigned char* ones)
 // Projections are 64 features wide (N = 128: two packed 32-feature operands), double
 // buffered in TMEM; epilogue group g takes the projections n with n % 2 == g.  Tile i uses
 // V and phi(k) buffer (i - first) % 2.
+// kStorePhi: also write phi(k) of every tile (bf16, [BH][L][F]) through TMA for the output
+// kernel that reads it instead of recomputing it; warp 10 issues those stores.
+template <bool kStorePhi>
 __global__ void __launch_bounds__(kThreads, 1)
 k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
-                  const __grid_constant__ CUtensorMap tmw, KParams kp, float* __restrict__ wsS,
-                  float* __restrict__ wsZ, int* __restrict__ err)
+                  const __grid_constant__ CUtensorMap tmw, const __grid_constant__ CUtensorMap tmpk,
+                  KParams kp, float* __restrict__ wsS, float* __restrict__ wsZ,
+                  int* __restrict__ err)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* sm = aligned_smem(smem_raw);
@@ -230,10 +234,13 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     constexpr uint32_t kColUS = 0;     // 2 x 128: projections
     constexpr uint32_t kColSS = 256;   // 2 x 80 : [S | z]
     // barrier roles here: QK_* hold the K tile; VF(b) / VE(b) the V buffers; TD(b) = the
-    // state update of a tile in buffer b is done; PK_FULL = all phiK of a tile written
+    // state update of a tile in buffer b is done; PKF(b) = all phiK of a tile in buffer b
+    // written (one barrier per buffer, so no waiter can fall two phases behind)
     uint64_t* VF = &bar[B_PQ_FULL0];
     uint64_t* VE = &bar[B_PQ_EMPTY0];
     uint64_t* TD = &bar[B_O_EMPTY];    // B_O_EMPTY, B_SBF_READY
+    uint64_t* ST = &bar[B_PK_FREE0];   // ST(b): the phi(k) store from buffer b has read it
+    auto PKF = [bar](int b) { return &bar[b ? B_PK_FULL1 : B_PK_FULL]; };
     if (warp == 1) {
         tmem_alloc(tslot, 512);
         tmem_relinquish();
@@ -244,10 +251,12 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         mbar_init(&bar[B_U_EMPTY0], 4);
         mbar_init(&bar[B_U_EMPTY1], 4);
         mbar_init(&bar[B_PK_FULL], 8);
+        mbar_init(&bar[B_PK_FULL1], 8);
         mbar_fence_init();
         tma_prefetch_desc(&tmk);
         tma_prefetch_desc(&tmv);
         tma_prefetch_desc(&tmw);
+        if (kStorePhi) tma_prefetch_desc(&tmpk);
     }
     fill_ones(sm + L.ones);
     fence_async_smem();
@@ -297,7 +306,7 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            uint32_t ph_kf = 0, ph_vf = 0, ph_wf = 0, ph_ue0 = 1, ph_ue1 = 1, ph_pk = 0;
+            uint32_t ph_kf = 0, ph_vf = 0, ph_wf = 0, ph_ue0 = 1, ph_ue1 = 1, ph_pk = 0;  // ph_pk: bit per buffer
             int n_glob = 0;
             constexpr uint32_t idU = idesc_bf16(128, 128, 0, 0);
             for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
@@ -321,7 +330,11 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                     umma_commit(&bar[B_W_EMPTY0 + slot]);
                 }
                 umma_commit(&bar[B_QK_EMPTY]);
-                wt.wait(&bar[B_PK_FULL], ph_pk);
+                {
+                    uint32_t pp = (ph_pk >> b) & 1u;
+                    wt.wait(PKF(b), pp);
+                    ph_pk ^= 1u << b;
+                }
                 uint32_t pv = (ph_vf >> b) & 1u;
                 wt.wait(&VF[b], pv);
                 ph_vf ^= (1u << b);
@@ -333,6 +346,25 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 umma_commit(&VE[b]);
                 umma_commit(&TD[b]);
             }
+        }
+    } else if (kStorePhi && warp == 10) {
+        if (lane == 0) {
+            uint32_t ph_pk = 0;
+            for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+                const int b = (tile - sg.t_begin) & 1;
+                {   // all of phi(k) of this tile written
+                    uint32_t pp = (ph_pk >> b) & 1u;
+                    wt.wait(PKF(b), pp);
+                    ph_pk ^= 1u << b;
+                }
+                for (int t = 0; t < NT; ++t)
+                    tma_store_3d(&tmpk, sm + L.phik + b * phik_bytes + t * kTileBytes, kSlice * t,
+                                 tile * kTile, sg.bh);
+                bulk_commit_group();
+                bulk_wait_read<0>();
+                mbar_arrive(&ST[b]);
+            }
+            bulk_wait<0>();
         }
     } else if (warp < 10) {
         const int grp = (warp >= 6) ? 1 : 0;
@@ -346,9 +378,10 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             float inv, l2i;
             row_scale(sm + L.k + row * 128, inv, l2i);
             warp_arrive(&bar[B_QK_EMPTY]);
-            if (li >= 2) {   // phiK buffer b free again (update of tile li-2 done)
-                uint32_t pt = (ph_td >> b) & 1u;
+            if (li >= 2) {   // phiK buffer b free again (update and store of tile li-2 done)
+                uint32_t pt = (ph_td >> b) & 1u, ps = pt;   // wait() flips its argument
                 wt.wait(&TD[b], pt);
+                if (kStorePhi) wt.wait(&ST[b], ps);
                 ph_td ^= (1u << b);
             }
             for (int n = grp; n < NT; n += 2) {
@@ -374,7 +407,7 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 phi_sub_epilogue(ub, pb, a, bb, tile_addr, row, 1, nullptr);
             }
             fence_async_smem();
-            warp_arrive(&bar[B_PK_FULL]);
+            warp_arrive(PKF(b));
         }
         // the segment's sums once the last update is done (it follows all earlier ones)
         {
@@ -406,7 +439,7 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             wsZ[segidx * kp.F + f] = __uint_as_float(zr);
         }
     }
-    if (!wt.ok) atomicExch(err, 1);
+    wt.report(err);
     drain_after_failure(wt.ok);
     tc_fence_before();
     __syncthreads();
@@ -615,7 +648,7 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 }
             }
         }
-        if (!wt.ok) atomicExch(err, 1);
+        wt.report(err);
         drain_after_failure(wt.ok);
     } else {
         regs_inc<136>();
@@ -808,7 +841,415 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 }
             }
         }
-        if (!wt.ok) atomicExch(err, 1);
+        wt.report(err);
+        drain_after_failure(wt.ok);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------- causal output reading stored phi(k)
+// As k_tc_causal_out, but phi(k) of every tile comes from HBM (written by the state kernel)
+// instead of being recomputed, which frees the k projections: warp 0 loads q tiles (two
+// buffers) and projection operands, warp 3 loads the phi(k) slices and v; warp 2 issues the
+// q projections alternately into U0 / U1; warps 4-7 and 8-11 turn them into phi(q) (group g
+// writes half g of each 64-feature slice); warp 1 and warps 12-15 as in k_tc_causal_out.
+struct SmemOutPk {
+    uint32_t w, q, v, ones, phik, phiq, st, bar, tmem, total;
+};
+
+__host__ __device__ inline SmemOutPk smem_outpk_layout(int F)
+{
+    SmemOutPk s;
+    s.w = 0;
+    s.q = kWSlots * kWBytes;                  // 2 buffers
+    s.v = s.q + 2 * kTileBytes;
+    s.ones = s.v + kTileBytes;                // right after V: fixed offset from it
+    s.phik = s.ones + kOnesBytes;
+    s.phiq = s.phik + (F / kSlice) * kTileBytes;
+    s.st = s.phiq + 2 * kTileBytes;
+    s.bar = s.st + (F / kSlice) * kStBytes;
+    s.tmem = s.bar + NUM_BARS * 8;
+    s.total = s.tmem + 16;
+    return s;
+}
+
+__global__ void __launch_bounds__(kOutThreads, 1)
+k_tc_causal_out_pk(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmpk,
+                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmw,
+                   KParams kp, const float* __restrict__ wsS, const float* __restrict__ wsZ,
+                   __nv_bfloat16* __restrict__ out, float* __restrict__ den, int* __restrict__ err)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* sm = aligned_smem(smem_raw);
+    const SmemOutPk L = smem_outpk_layout(kp.F);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L.bar);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L.tmem);
+    const uint32_t sbase = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int NT = kp.F / kSlice, NS = kp.F / kSub, halves = kp.F / 128;
+    const Seg sg = segment_of(blockIdx.x, kp.nseg, kp.ntiles);
+    // q buffer b: full / empty (the fourth W slot's barriers hold buffer 1)
+    auto QF = [bar](int b) { return &bar[b ? B_W_FULL3 : B_QK_FULL]; };
+    auto QE = [bar](int b) { return &bar[b ? B_W_EMPTY3 : B_QK_EMPTY]; };
+
+    if (warp == 1) {
+        tmem_alloc(tslot, 512);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bar[i], 1);
+        mbar_init(QE(0), 1 + 8);
+        mbar_init(QE(1), 1 + 8);
+        mbar_init(&bar[B_U_EMPTY0], 4);
+        mbar_init(&bar[B_U_EMPTY1], 4);
+        mbar_init(&bar[B_PQ_FULL0], 8);
+        mbar_init(&bar[B_PQ_FULL1], 8);
+        mbar_init(&bar[B_PSM_FULL], 4);
+        mbar_init(&bar[B_O_EMPTY], 4);
+        mbar_init(&bar[B_SBF_READY], 4);
+        mbar_fence_init();
+        tma_prefetch_desc(&tmq);
+        tma_prefetch_desc(&tmpk);
+        tma_prefetch_desc(&tmv);
+        tma_prefetch_desc(&tmw);
+    }
+    fill_ones(sm + L.ones);
+    {   // the state copy: columns 65..79 stay zero
+        uint4* p = reinterpret_cast<uint4*>(sm + L.st);
+        for (int i = tid; i < NT * kStBytes / 16; i += kOutThreads) p[i] = make_uint4(0, 0, 0, 0);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+    // registers: the single-thread issuers of warpgroup 0 give 32 of theirs to the three
+    // epilogue warpgroups (128*96 + 384*136 <= 65536); each role stays inside its branch
+    if (warp < 4) {
+        regs_dec<96>();
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        Waiter wt;
+        if (warp == 0) {
+            // ------------------------------------------------ TMA: q tiles, W sub-slices
+            if (lane == 0) {
+                uint32_t ph_qe = 0, ph_we = (1u << kWSlots) - 1u;
+                int n_glob = 0;
+                for (int tile = sg.t_begin, it = 0; tile < sg.t_end; ++tile, ++it) {
+                    const int qb = it & 1;
+                    if (it >= 2) {
+                        uint32_t ph = (ph_qe >> qb) & 1u;
+                        wt.wait(QE(qb), ph);
+                        ph_qe ^= 1u << qb;
+                    }
+                    mbar_arrive_expect_tx(QF(qb), kTileBytes);
+                    tma_load_3d(sm + L.q + qb * kTileBytes, &tmq, QF(qb), 0, tile * kTile, sg.bh);
+                    for (int n = 0; n < NS; ++n, ++n_glob) {
+                        const int slot = n_glob % kWSlots;
+                        uint32_t ph = (ph_we >> slot) & 1u;
+                        wt.wait(&bar[B_W_EMPTY0 + slot], ph);
+                        ph_we ^= (1u << slot);
+                        mbar_arrive_expect_tx(&bar[B_W_FULL0 + slot], kWBytes);
+                        tma_load_2d(sm + L.w + slot * kWBytes, &tmw, &bar[B_W_FULL0 + slot], 0, n * 64);
+                    }
+                }
+            }
+        } else if (warp == 3) {
+            // ----------------------------------------------- TMA: phi(k) slices and v
+            if (lane == 0) {
+                uint32_t ph_free = 0, ph_ve = 0;
+                for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+                    for (int t = 0; t < NT; ++t) {
+                        // a feature half is free once the previous tile's scores and state
+                        // update have read it
+                        if (tile > sg.t_begin && (t & 1) == 0) {
+                            uint32_t ph = (ph_free >> (t >> 1)) & 1u;
+                            wt.wait(&bar[B_PK_FREE0 + (t >> 1)], ph);
+                            ph_free ^= 1u << (t >> 1);
+                        }
+                        mbar_arrive_expect_tx(pk_full(bar, t), kTileBytes);
+                        tma_load_3d(sm + L.phik + t * kTileBytes, &tmpk, pk_full(bar, t), kSlice * t,
+                                    tile * kTile, sg.bh);
+                    }
+                    if (tile > sg.t_begin) wt.wait(&bar[B_V_EMPTY], ph_ve);
+                    mbar_arrive_expect_tx(&bar[B_V_FULL], kTileBytes);
+                    tma_load_3d(sm + L.v, &tmv, &bar[B_V_FULL], 0, tile * kTile, sg.bh);
+                }
+            }
+        } else if (warp == 2) {
+            // ------------------------------------------------- q projection issuer
+            if (lane == 0) {
+                uint32_t ph_qf = 0, ph_wf = 0, ph_ue = 0x3u;
+                int n_glob = 0;
+                for (int tile = sg.t_begin, it = 0; tile < sg.t_end; ++tile, ++it) {
+                    const int qb = it & 1;
+                    uint32_t ph = (ph_qf >> qb) & 1u;
+                    wt.wait(QF(qb), ph);
+                    ph_qf ^= 1u << qb;
+                    for (int n = 0; n < NS; ++n, ++n_glob) {
+                        const int slot = n_glob % kWSlots, g = n & 1;
+                        uint32_t pw = (ph_wf >> slot) & 1u;
+                        wt.wait(&bar[B_W_FULL0 + slot], pw);
+                        ph_wf ^= (1u << slot);
+                        uint32_t pu = (ph_ue >> g) & 1u;
+                        wt.wait(&bar[B_U_EMPTY0 + g], pu);
+                        ph_ue ^= 1u << g;
+                        tc_fence_after();
+                        issue_projection(tmem + (g ? kColU1 : kColU0), sbase + L.q + qb * kTileBytes,
+                                         sbase + L.w + slot * kWBytes);
+                        umma_commit(&bar[B_U_FULL0 + g]);
+                        umma_commit(&bar[B_W_EMPTY0 + slot]);
+                    }
+                    umma_commit(QE(qb));
+                }
+            }
+        } else {
+            // ------------------------------------------------------ main MMA issuer
+            if (lane == 0) {
+                uint32_t ph_vf = 0, ph_pqf = 0, ph_pkf = 0, ph_psm = 0, ph_oe = 0, ph_sbf = 0;
+                constexpr uint32_t idP = idesc_bf16(128, 128, 0, 0);
+                constexpr uint32_t idO = idesc_bf16(128, 80, 0, 1);
+                constexpr uint32_t idPV = idesc_bf16(128, 80, 0, 1);
+                const uint32_t st_sbo = static_cast<uint32_t>(kp.F) * 16;
+                for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+                    const bool last = tile + 1 == sg.t_end;
+                    for (int t = 0; t < NT; ++t) {
+                        const int pslot = t & 1;
+                        {
+                            uint32_t ph = (ph_pqf >> pslot) & 1u;
+                            wt.wait(&bar[B_PQ_FULL0 + pslot], ph);
+                            ph_pqf ^= 1u << pslot;
+                        }
+                        {
+                            uint32_t ph = (ph_pkf >> t) & 1u;
+                            wt.wait(pk_full(bar, t), ph);
+                            ph_pkf ^= 1u << t;
+                        }
+                        if (t == 0 && tile > sg.t_begin) {
+                            wt.wait(&bar[B_SBF_READY], ph_sbf);
+                            wt.wait(&bar[B_O_EMPTY], ph_oe);
+                        }
+                        tc_fence_after();
+                        const uint32_t aq = sbase + L.phiq + pslot * kTileBytes;
+                        const uint32_t bk = sbase + L.phik + t * kTileBytes;
+                        const uint32_t bs = sbase + L.st + t * (kSlice / 8) * 128;
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+                            const uint64_t ad = sdesc(aq + 32 * kk, 16, 1024, kLayoutSW128);
+                            umma_bf16(tmem + kColP, ad, sdesc(bk + 32 * kk, 16, 1024, kLayoutSW128), idP, acc);
+                            umma_bf16(tmem + kColO, ad, sdesc(bs + 256 * kk, 128, st_sbo, kLayoutNone), idO, acc);
+                        }
+                        umma_commit(&bar[B_PQ_EMPTY0 + pslot]);
+                        if ((t & 1) == 1) {
+                            if (!last) {
+                                if (t == 1) wt.wait(&bar[B_V_FULL], ph_vf);
+                                issue_state_half(tmem, kColS, sbase + L.phik, sbase + L.v,
+                                                 sbase + L.ones, t >> 1, false);
+                            }
+                            // the loader needs this half free again for the next tile
+                            if (!last) umma_commit(&bar[B_PK_FREE0 + (t >> 1)]);
+                        }
+                    }
+                    umma_commit(&bar[B_P_FULL]);
+                    if (last) wt.wait(&bar[B_V_FULL], ph_vf);
+                    wt.wait(&bar[B_PSM_FULL], ph_psm);
+                    tc_fence_after();
+                    const uint32_t lbo = L.ones - L.v;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_bf16_ts(tmem + kColO, tmem + kColP + 8 * kk,
+                                     sdesc(sbase + L.v + 2048 * kk, lbo, 1024, kLayoutSW128), idPV, 1u);
+                    umma_commit(&bar[B_TILE_DONE]);
+                    umma_commit(&bar[B_V_EMPTY]);
+                }
+            }
+        }
+        wt.report(err);
+        drain_after_failure(wt.ok);
+    } else {
+        regs_inc<136>();
+        if (warp >= 12) {   // state entering the segment (sum of the earlier segments)
+            const int sp = warp & 3;
+            const uint32_t row = 32u * sp + lane;
+            const uint32_t trow = tmem + ((32u * sp) << 16);
+            for (int h = 0; h < halves; ++h) {
+                const int f = 128 * h + row;
+                float acc[64];
+#pragma unroll
+                for (int e = 0; e < 64; ++e) acc[e] = 0.0f;
+                float zf = 0.0f;
+                for (int s = 0; s < sg.seg; ++s) {
+                    const size_t segidx = static_cast<size_t>(sg.bh) * kp.nseg + s;
+                    const float4* src = reinterpret_cast<const float4*>(wsS + (segidx * kp.F + f) * 64);
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const float4 x = src[q];
+                        acc[4 * q] += x.x; acc[4 * q + 1] += x.y; acc[4 * q + 2] += x.z; acc[4 * q + 3] += x.w;
+                    }
+                    zf += wsZ[segidx * kp.F + f];
+                }
+                uint32_t r[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(acc[e]);
+                tmem_st32(trow + kColS + 80 * h, r);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(acc[32 + e]);
+                tmem_st32(trow + kColS + 80 * h + 32, r);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(zf);
+                tmem_st32(trow + kColS + 80 * h + 64, r);
+                write_state_row(sbase + L.st, kp.F, f, acc, zf);
+            }
+            tmem_wait_st();
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        Waiter wt;
+        const int64_t rowbase = static_cast<int64_t>(sg.bh) * kp.L;
+        if (warp < 12) {
+            // ------------------------------------------ phi(q): group g, half g of slice t
+            const int g = (warp >= 8) ? 1 : 0;
+            const int sp = warp & 3;
+            const uint32_t row = 32u * sp + lane;
+            const uint32_t trow = tmem + ((32u * sp) << 16);
+            uint32_t ph_qf = 0, ph_uf = 0, ph_pqe = 0;
+            int uses0 = 0, uses1 = 0;
+            for (int tile = sg.t_begin, it = 0; tile < sg.t_end; ++tile, ++it) {
+                const int qb = it & 1;
+                uint32_t ph = (ph_qf >> qb) & 1u;
+                wt.wait(QF(qb), ph);
+                ph_qf ^= 1u << qb;
+                float inv, l2i;
+                row_scale(sm + L.q + qb * kTileBytes + row * 128, inv, l2i);
+                warp_arrive(QE(qb));
+                for (int t = 0; t < NT; ++t) {
+                    const int node = (t * kSlice) / kp.m;
+                    const float a = kp.a2[node] * inv, b = kp.b2[node] + l2i;
+                    const int pslot = t & 1;
+                    wt.wait(&bar[B_U_FULL0 + g], ph_uf);
+                    tc_fence_after();
+                    uint32_t ur[32], pr[32];
+                    const uint32_t col = g ? kColU1 : kColU0;
+                    tmem_ld32(trow + col, ur);
+                    tmem_ld32(trow + col + 32, pr);
+                    tmem_wait_ld();
+                    reg_fence(ur);
+                    reg_fence(pr);
+                    tc_fence_before();
+                    warp_arrive(&bar[B_U_EMPTY0 + g]);
+                    int& uses = pslot ? uses1 : uses0;
+                    if (uses > 0) {   // both groups wait for the same completion
+                        uint32_t pe = (ph_pqe >> pslot) & 1u;
+                        wt.wait(&bar[B_PQ_EMPTY0 + pslot], pe);
+                        ph_pqe ^= 1u << pslot;
+                    }
+                    ++uses;
+                    phi_sub_epilogue(ur, pr, a, b, sbase + L.phiq + pslot * kTileBytes, row, g, nullptr);
+                    fence_async_smem();
+                    warp_arrive(&bar[B_PQ_FULL0 + pslot]);
+                }
+            }
+        } else {
+            // ------------------------------------------------------------ tile tail
+            const int sp = warp & 3;
+            const uint32_t row = 32u * sp + lane;
+            const uint32_t trow = tmem + ((32u * sp) << 16);
+            uint32_t ph_pf = 0, ph_td = 0;
+            for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+                wt.wait(&bar[B_P_FULL], ph_pf);
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t pk[16];
+                    if (c <= sp) {
+                        uint32_t pv[32];
+                        tmem_ld32(trow + kColP + 32 * c, pv);
+                        tmem_wait_ld();
+                        reg_fence(pv);
+                        if (c < sp) {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                pk[j] = pack_bf16(__uint_as_float(pv[2 * j]), __uint_as_float(pv[2 * j + 1]));
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                pk[j] = pack_bf16((2 * j <= lane) ? __uint_as_float(pv[2 * j]) : 0.0f,
+                                                  (2 * j + 1 <= lane) ? __uint_as_float(pv[2 * j + 1]) : 0.0f);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) pk[j] = 0u;
+                    }
+                    tmem_st16(trow + kColP + 16 * c, pk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                warp_arrive(&bar[B_PSM_FULL]);
+                if (tile + 1 < sg.t_end) {
+                    for (int h = 0; h < halves; ++h) {
+                        const int f = 128 * h + row;
+                        uint32_t r0s[32], r1s[32], zr;
+                        tmem_ld32(trow + kColS + 80 * h, r0s);
+                        tmem_ld32(trow + kColS + 80 * h + 32, r1s);
+                        tmem_ld1(trow + kColS + 80 * h + 64, zr);
+                        tmem_wait_ld();
+                        reg_fence(r0s);
+                        reg_fence(r1s);
+                        reg_fence1(zr);
+                        float sv[64];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            sv[e] = __uint_as_float(r0s[e]);
+                            sv[32 + e] = __uint_as_float(r1s[e]);
+                        }
+                        write_state_row(sbase + L.st, kp.F, f, sv, __uint_as_float(zr));
+                    }
+                    fence_async_smem();
+                    tc_fence_before();
+                    warp_arrive(&bar[B_SBF_READY]);
+                }
+                wt.wait(&bar[B_TILE_DONE], ph_td);
+                tc_fence_after();
+                uint32_t o0[32], o1[32], dr;
+                tmem_ld32(trow + kColO, o0);
+                tmem_ld32(trow + kColO + 32, o1);
+                tmem_ld1(trow + kColO + 64, dr);
+                tmem_wait_ld();
+                reg_fence(o0);
+                reg_fence(o1);
+                reg_fence1(dr);
+                tc_fence_before();
+                warp_arrive(&bar[B_O_EMPTY]);
+                const float d = __uint_as_float(dr);
+                const float rz = 1.0f / (d + kp.eps);
+                const int grow = tile * kTile + static_cast<int>(row);
+                if (grow < kp.L) {
+                    uint4* dst = reinterpret_cast<uint4*>(out + (rowbase + grow) * 64);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        dst[q] = make_uint4(
+                            pack_bf16(__uint_as_float(o0[8 * q]) * rz, __uint_as_float(o0[8 * q + 1]) * rz),
+                            pack_bf16(__uint_as_float(o0[8 * q + 2]) * rz, __uint_as_float(o0[8 * q + 3]) * rz),
+                            pack_bf16(__uint_as_float(o0[8 * q + 4]) * rz, __uint_as_float(o0[8 * q + 5]) * rz),
+                            pack_bf16(__uint_as_float(o0[8 * q + 6]) * rz, __uint_as_float(o0[8 * q + 7]) * rz));
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        dst[4 + q] = make_uint4(
+                            pack_bf16(__uint_as_float(o1[8 * q]) * rz, __uint_as_float(o1[8 * q + 1]) * rz),
+                            pack_bf16(__uint_as_float(o1[8 * q + 2]) * rz, __uint_as_float(o1[8 * q + 3]) * rz),
+                            pack_bf16(__uint_as_float(o1[8 * q + 4]) * rz, __uint_as_float(o1[8 * q + 5]) * rz),
+                            pack_bf16(__uint_as_float(o1[8 * q + 6]) * rz, __uint_as_float(o1[8 * q + 7]) * rz));
+                    if (den) den[rowbase + grow] = d;
+                }
+            }
+        }
+        wt.report(err);
         drain_after_failure(wt.ok);
     }
     tc_fence_before();
@@ -995,7 +1436,7 @@ k_tc_bidir_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
         const uint32_t row = 32u * sp + lane;
         const uint32_t trow = tmem + ((32u * sp) << 16);
         uint32_t ph_qf = 0, ph_uf = 0, ph_pqe = 0;
-        int uses[2] = {0, 0};
+        int uses0 = 0, uses1 = 0;
         for (int tile = sg.t_begin, it = 0; tile < sg.t_end; ++tile, ++it) {
             const int qb = it & 1;
             uint32_t ph = (ph_qf >> qb) & 1u;
@@ -1018,12 +1459,13 @@ k_tc_bidir_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 reg_fence(pr);
                 tc_fence_before();
                 warp_arrive(&bar[B_U_EMPTY0 + g]);
-                if (uses[pslot] > 0) {   // both groups wait for the same completion
+                int& uses = pslot ? uses1 : uses0;
+                if (uses > 0) {   // both groups wait for the same completion
                     uint32_t pe = (ph_pqe >> pslot) & 1u;
                     wt.wait(&bar[B_PQ_EMPTY0 + pslot], pe);
                     ph_pqe ^= 1u << pslot;
                 }
-                ++uses[pslot];
+                ++uses;
                 phi_sub_epilogue(ur, pr, a, b, sbase + L.phiq + pslot * kTileBytes, row, g, nullptr);
                 fence_async_smem();
                 warp_arrive(&bar[B_PQ_FULL0 + pslot]);
@@ -1071,7 +1513,7 @@ k_tc_bidir_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             }
         }
     }
-    if (!wt.ok) atomicExch(err, 1);
+    wt.report(err);
     drain_after_failure(wt.ok);
     tc_fence_before();
     __syncthreads();
@@ -1130,15 +1572,33 @@ bool tc_supported(slay_op op, int B, int H, int L, int R, int m)
     return smem_bytes_out(F) <= 232448;
 }
 
-size_t tc_workspace_bytes(slay_op op, int B, int H, int L, int R, int m)
+namespace {
+
+// Workspace: header | per-segment S [BH][nseg][F][64] fp32 | z [BH][nseg][F] fp32 | and, for
+// the causal forward that stores phi(k), phi(k) [BH][L][F] bf16.
+struct WsLayout {
+    size_t s, z, phik, total;
+};
+
+WsLayout ws_layout(int BH, int L, int F, int nseg, bool with_phik)
+{
+    const size_t per = static_cast<size_t>(BH) * nseg * F;
+    WsLayout w;
+    w.s = kWsHeader;
+    w.z = w.s + ((per * 64 * sizeof(float) + 255) & ~size_t(255));
+    w.phik = w.z + ((per * sizeof(float) + 255) & ~size_t(255));
+    w.total = w.phik + (with_phik ? static_cast<size_t>(BH) * L * F * sizeof(uint16_t) : 0);
+    return w;
+}
+
+}  // namespace
+
+size_t tc_workspace_bytes(slay_op op, int B, int H, int L, int R, int m, bool lowmem)
 {
     if (op != SLAY_OP_CAUSAL_FWD && op != SLAY_OP_BIDIR_FWD) return 0;
-    const int F = R * m;
     const int BH = B * H;
-    const int ntiles = (L + kTile - 1) / kTile;
-    const int nseg = choose_nseg(BH, ntiles);
-    const size_t per = static_cast<size_t>(BH) * nseg * F;
-    return kWsHeader + ((per * 64 * sizeof(float) + 255) & ~size_t(255)) + per * sizeof(float);
+    const int nseg = choose_nseg(BH, (L + kTile - 1) / kTile);
+    return ws_layout(BH, L, R * m, nseg, op == SLAY_OP_CAUSAL_FWD && !lowmem).total;
 }
 
 size_t tc_wb_elems(int D, int R, int m)
@@ -1160,67 +1620,100 @@ void tc_pack_wb(int D, int R, int m, const uint16_t* om, const uint16_t* an, uin
         }
 }
 
+// [BH][L][F] bf16 phi(k) viewed as a 3-D tensor, 64-feature x 128-token boxes, 128-byte
+// swizzle (the layout the score and state MMAs read); rows past L read as zero, stores to
+// them are dropped.
+bool map_phik(CUtensorMap* m, const void* base, int F, int L, int BH)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(F), static_cast<cuuint64_t>(L),
+                                static_cast<cuuint64_t>(BH)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(F) * 2, static_cast<cuuint64_t>(L) * F * 2};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kTile), 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, size_t bytes)
+{
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(bytes));
+}
+
 cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, float* den, int B,
                         int H, int L, const Params& P, float eps, bool causal, void* ws,
-                        cudaStream_t st)
+                        cudaStream_t st, bool lowmem)
 {
     if (!P.wB) return cudaErrorNotSupported;
     const int BH = B * H, F = P.F;
     const int ntiles = (L + kTile - 1) / kTile;
     const int nseg = choose_nseg(BH, ntiles);
-    CUtensorMap mq, mk, mv, mw;
+    const bool store_phik = causal && !lowmem;
+    const WsLayout wl = ws_layout(BH, L, F, nseg, store_phik);
+    char* w = static_cast<char*>(ws);
+    CUtensorMap mq, mk, mv, mw, mpk;
     if (!map_rows(&mq, q, L, BH) || !map_rows(&mk, k, L, BH) || !map_rows(&mv, v, L, BH) ||
         !map_w(&mw, P.wB, F))
         return cudaErrorInvalidValue;
+    // without stored phi(k) the state kernel never touches this map: any valid one will do
+    if (!map_phik(&mpk, store_phik ? static_cast<const void*>(w + wl.phik) : P.wB, F,
+                  store_phik ? L : 1, store_phik ? BH : 1))
+        return cudaErrorInvalidValue;
     KParams kp;
     kp.L = L; kp.F = F; kp.m = P.m; kp.nseg = nseg; kp.ntiles = ntiles; kp.eps = eps;
-    kp.all_segs = causal ? 0 : 1;
+    kp.all_segs = (causal && lowmem) ? 0 : 1;
     for (int r = 0; r < kMaxR; ++r) { kp.a2[r] = P.a2[r]; kp.b2[r] = P.b2[r]; }
-    char* w = static_cast<char*>(ws);
     int* err = reinterpret_cast<int*>(w);
-    float* wsS = reinterpret_cast<float*>(w + kWsHeader);
-    const size_t per = static_cast<size_t>(BH) * nseg * F;
-    float* wsZ = reinterpret_cast<float*>(w + kWsHeader + ((per * 64 * sizeof(float) + 255) & ~size_t(255)));
+    float* wsS = reinterpret_cast<float*>(w + wl.s);
+    float* wsZ = reinterpret_cast<float*>(w + wl.z);
+    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
     cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), st);
     if (e != cudaSuccess) return e;
+    const size_t sms = smem_bytes_state(F);
     if (!causal) {
         // every segment's sum, then the readout against their total
-        const size_t sms = smem_bytes_state(F);
-        e = cudaFuncSetAttribute(k_tc_causal_state, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(sms));
-        if (e != cudaSuccess) return e;
+        if ((e = set_smem(k_tc_causal_state<false>, sms)) != cudaSuccess) return e;
         {
             TraceScope trace_("tc_bidir_state", st);
-            k_tc_causal_state<<<BH * nseg, kThreads, sms, st>>>(mk, mv, mw, kp, wsS, wsZ, err);
+            k_tc_causal_state<false><<<BH * nseg, kThreads, sms, st>>>(mk, mv, mw, mpk, kp, wsS, wsZ, err);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
         const size_t smb = smem_bidir_layout(F).total + 1024;
-        e = cudaFuncSetAttribute(k_tc_bidir_out, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smb));
-        if (e != cudaSuccess) return e;
+        if ((e = set_smem(k_tc_bidir_out, smb)) != cudaSuccess) return e;
         TraceScope trace_("tc_bidir_out", st);
-        k_tc_bidir_out<<<BH * nseg, kOutThreads, smb, st>>>(mq, mw, kp, wsS, wsZ,
-                                                           static_cast<__nv_bfloat16*>(out), den, err);
+        k_tc_bidir_out<<<BH * nseg, kOutThreads, smb, st>>>(mq, mw, kp, wsS, wsZ, o, den, err);
         return cudaGetLastError();
     }
-    if (nseg > 1) {
-        const size_t sm = smem_bytes_state(F);
-        e = cudaFuncSetAttribute(k_tc_causal_state, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(sm));
-        if (e != cudaSuccess) return e;
-        TraceScope trace_("tc_causal_state", st);
-        k_tc_causal_state<<<BH * (nseg - 1), kThreads, sm, st>>>(mk, mv, mw, kp, wsS, wsZ, err);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
+    if (store_phik) {
+        // phi(k) and every segment's sum once; the output kernel reads phi(k)
+        if ((e = set_smem(k_tc_causal_state<true>, sms)) != cudaSuccess) return e;
+        {
+            TraceScope trace_("tc_kphi_state", st);
+            k_tc_causal_state<true><<<BH * nseg, kThreads, sms, st>>>(mk, mv, mw, mpk, kp, wsS, wsZ, err);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+        const size_t smo = smem_outpk_layout(F).total + 1024;
+        if ((e = set_smem(k_tc_causal_out_pk, smo)) != cudaSuccess) return e;
+        TraceScope trace_("tc_qphi_out", st);
+        k_tc_causal_out_pk<<<BH * nseg, kOutThreads, smo, st>>>(mq, mpk, mv, mw, kp, wsS, wsZ, o, den, err);
+        return cudaGetLastError();
     }
-    const size_t sm = smem_bytes_out(F);
-    e = cudaFuncSetAttribute(k_tc_causal_out, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(sm));
-    if (e != cudaSuccess) return e;
+    // low-memory form (no phi(k) buffer): the output kernel recomputes phi(k)
+    if (nseg > 1) {
+        if ((e = set_smem(k_tc_causal_state<false>, sms)) != cudaSuccess) return e;
+        TraceScope trace_("tc_causal_state", st);
+        k_tc_causal_state<false><<<BH * (nseg - 1), kThreads, sms, st>>>(mk, mv, mw, mpk, kp, wsS, wsZ, err);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    const size_t smo = smem_bytes_out(F);
+    if ((e = set_smem(k_tc_causal_out, smo)) != cudaSuccess) return e;
     {
         TraceScope trace_("tc_causal_out", st);
-        k_tc_causal_out<<<BH * nseg, kOutThreads, sm, st>>>(mq, mk, mv, mw, kp, wsS, wsZ,
-                                                         static_cast<__nv_bfloat16*>(out), den, err);
+        k_tc_causal_out<<<BH * nseg, kOutThreads, smo, st>>>(mq, mk, mv, mw, kp, wsS, wsZ, o, den, err);
     }
     return cudaGetLastError();
 }

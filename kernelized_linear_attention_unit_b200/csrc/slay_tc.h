@@ -13,7 +13,9 @@ namespace slay {
 
 // Whether the tensor-core path takes this op at these sizes (bf16 mode only).
 bool tc_supported(slay_op op, int B, int H, int L, int R, int m);
-size_t tc_workspace_bytes(slay_op op, int B, int H, int L, int R, int m);
+// Workspace bytes of the tensor-core path.  The causal forward stores phi(k) ([BH][L][F]
+// bf16) unless `lowmem`, where the output kernel recomputes it instead.
+size_t tc_workspace_bytes(slay_op op, int B, int H, int L, int R, int m, bool lowmem = false);
 // Elements of the packed bf16 projection operand (0 when the path is not built).
 size_t tc_wb_elems(int D, int R, int m);
 // Pack bf16 omega / anchors ([F][D] row-major bit patterns) into the operand layout.
@@ -26,6 +28,6 @@ cudaError_t tc_feature_map(const void* x, void* phi, int64_t n, const Params& P,
 const void* fmap_status_word();
 cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, float* den,
                         int B, int H, int L, const Params& P, float eps, bool causal, void* ws,
-                        cudaStream_t st);
+                        cudaStream_t st, bool lowmem = false);
 
 }  // namespace slay

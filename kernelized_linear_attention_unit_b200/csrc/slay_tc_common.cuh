@@ -15,12 +15,22 @@ namespace tc {
 constexpr uint64_t kWaitNs = 2000000000ull;   // bound of every mbarrier wait (2 s)
 
 // A waiter that stops waiting (and reports) once any wait of this thread timed out.
+// `where` keeps the first barrier that ran out: 0x10000 | its shared-memory offset, the
+// value a kernel puts in the status word.
 struct Waiter {
     bool ok = true;
+    uint32_t where = 0;
     __device__ __forceinline__ void wait(uint64_t* bar, uint32_t& phase)
     {
-        ok = mbar_wait(bar, phase, ok ? kWaitNs : 0) && ok;
+        const bool done = mbar_wait(bar, phase, ok ? kWaitNs : 0);
+        if (!done && ok) where = 0x10000u | (smem_u32(bar) & 0xFFFFu);
+        ok = done && ok;
         phase ^= 1u;
+    }
+    // record the first failure in the status word (0 = every wait completed)
+    __device__ __forceinline__ void report(int* status) const
+    {
+        if (!ok) atomicCAS(status, 0, static_cast<int>(where));
     }
 };
 

@@ -256,7 +256,7 @@ k_tc_feature_map(const __grid_constant__ CUtensorMap tmx, const __grid_constant_
         }
         if (lane == 0) bulk_wait<0>();
     }
-    if (!wt.ok) atomicExch(&g_fmap_status, 1);
+    wt.report(&g_fmap_status);
     drain_after_failure(wt.ok);
     tc_fence_before();
     __syncthreads();
