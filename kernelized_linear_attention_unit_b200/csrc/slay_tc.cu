@@ -100,8 +100,9 @@ __host__ __device__ inline SmemOut smem_out_layout(int F)
     return s;
 }
 
-// State kernel: two 16 KiB projection operands (64 features each); V and phi(k) are double
-// buffered so that the phi(k) of tile i+1 is written while tile i's state update runs.
+// State kernel: two 16 KiB projection operands (64 features each); k tiles and phi(k) are
+// double buffered (the projections of tile i+1 and its phi(k) proceed while tile i's state
+// update runs); V, needed only by that update, has one buffer.
 constexpr int kWStateBytes = 2 * kWBytes;
 struct SmemState {
     uint32_t w, k, v, ones, phik, bar, tmem, total;
@@ -111,9 +112,9 @@ __host__ __device__ inline SmemState smem_state_layout(int F)
 {
     SmemState s;
     s.w = 0;
-    s.k = 2 * kWStateBytes;
-    s.v = s.k + kTileBytes;                 // 2 buffers
-    s.ones = s.v + 2 * kTileBytes;
+    s.k = 2 * kWStateBytes;                 // 2 buffers
+    s.v = s.k + 2 * kTileBytes;
+    s.ones = s.v + kTileBytes;              // right after V: fixed offset from it
     s.phik = s.ones + kOnesBytes;           // 2 buffers of F/64 tiles
     s.bar = s.phik + 2 * (F / kSlice) * kTileBytes;
     s.tmem = s.bar + NUM_BARS * 8;
@@ -210,7 +211,7 @@ __device__ __forceinline__ void fill_ones(unsigned char* ones)
 //   ws_S[bh][seg][f][e] = sum_{t in seg} phi(k_t)_f v_t[e],  ws_z[bh][seg][f] = sum phi(k_t)_f
 // Projections are 64 features wide (N = 128: two packed 32-feature operands), double
 // buffered in TMEM; epilogue group g takes the projections n with n % 2 == g.  Tile i uses
-// V and phi(k) buffer (i - first) % 2.
+// k and phi(k) buffer (i - first) % 2; warp 11 loads v.
 // kStorePhi: also write phi(k) of every tile (bf16, [BH][L][F]) through TMA for the output
 // kernel that reads it instead of recomputing it; warp 10 issues those stores.
 template <bool kStorePhi>
@@ -233,9 +234,11 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                                : segment_of(blockIdx.x + blockIdx.x / (kp.nseg - 1), kp.nseg, kp.ntiles);
     constexpr uint32_t kColUS = 0;     // 2 x 128: projections
     constexpr uint32_t kColSS = 256;   // 2 x 80 : [S | z]
-    // barrier roles here: QK_* hold the K tile; VF(b) / VE(b) the V buffers; TD(b) = the
-    // state update of a tile in buffer b is done; PKF(b) = all phiK of a tile in buffer b
-    // written (one barrier per buffer, so no waiter can fall two phases behind)
+    // barrier roles here: KF(b) / KE(b) the k buffers; VF / VE the V buffer; TD(b) = the
+    // state update of a tile in phi(k) buffer b is done; PKF(b) = all phiK of a tile in
+    // buffer b written (one barrier per buffer, so no waiter can fall two phases behind)
+    auto KF = [bar](int b) { return &bar[b ? B_V_FULL : B_QK_FULL]; };
+    auto KE = [bar](int b) { return &bar[b ? B_V_EMPTY : B_QK_EMPTY]; };
     uint64_t* VF = &bar[B_PQ_FULL0];
     uint64_t* VE = &bar[B_PQ_EMPTY0];
     uint64_t* TD = &bar[B_O_EMPTY];    // B_O_EMPTY, B_SBF_READY
@@ -247,7 +250,8 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     }
     if (tid == 0) {
         for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bar[i], 1);
-        mbar_init(&bar[B_QK_EMPTY], 1 + 8);
+        mbar_init(KE(0), 1 + 8);
+        mbar_init(KE(1), 1 + 8);
         mbar_init(&bar[B_U_EMPTY0], 4);
         mbar_init(&bar[B_U_EMPTY1], 4);
         mbar_init(&bar[B_PK_FULL], 8);
@@ -267,15 +271,16 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     Waiter wt;
 
     if (warp == 0) {
+        // k tiles (two buffers) and the projection operands
         if (lane == 0) {
-            uint32_t ph_ke = 0, ph_ve = 0, ph_we = 0x3u;  // both operand slots start free
+            uint32_t ph_ke = 0, ph_we = 0x3u;  // both operand slots start free
             int n_glob = 0;
-            mbar_arrive_expect_tx(&bar[B_QK_FULL], kTileBytes);
-            tma_load_3d(sm + L.k, &tmk, &bar[B_QK_FULL], 0, sg.t_begin * kTile, sg.bh);
-            mbar_arrive_expect_tx(&VF[0], kTileBytes);
-            tma_load_3d(sm + L.v, &tmv, &VF[0], 0, sg.t_begin * kTile, sg.bh);
+            for (int j = 0; j < 2 && sg.t_begin + j < sg.t_end; ++j) {
+                mbar_arrive_expect_tx(KF(j), kTileBytes);
+                tma_load_3d(sm + L.k + j * kTileBytes, &tmk, KF(j), 0, (sg.t_begin + j) * kTile, sg.bh);
+            }
             for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
-                const int nxt = tile + 1 - sg.t_begin;   // local index of the next tile
+                const int kb = (tile - sg.t_begin) & 1;
                 for (int n = 0; n < NT; ++n, ++n_glob) {
                     const int slot = n_glob & 1;
                     uint32_t ph = (ph_we >> slot) & 1u;
@@ -285,33 +290,40 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                     unsigned char* dst = sm + L.w + slot * kWStateBytes;
                     tma_load_2d(dst, &tmw, &bar[B_W_FULL0 + slot], 0, (2 * n) * 64);
                     tma_load_2d(dst + kWBytes, &tmw, &bar[B_W_FULL0 + slot], 0, (2 * n + 1) * 64);
-                    // V of the next tile into its buffer once that buffer's last update is done
-                    if (n == NT - 1 && tile + 1 < sg.t_end) {
-                        const int vb = nxt & 1;
-                        if (nxt >= 2) {
-                            uint32_t pv = (ph_ve >> vb) & 1u;
-                            wt.wait(&VE[vb], pv);
-                            ph_ve ^= (1u << vb);
-                        }
-                        mbar_arrive_expect_tx(&VF[vb], kTileBytes);
-                        tma_load_3d(sm + L.v + vb * kTileBytes, &tmv, &VF[vb], 0, (tile + 1) * kTile, sg.bh);
-                    }
                 }
-                if (tile + 1 < sg.t_end) {
-                    wt.wait(&bar[B_QK_EMPTY], ph_ke);
-                    mbar_arrive_expect_tx(&bar[B_QK_FULL], kTileBytes);
-                    tma_load_3d(sm + L.k, &tmk, &bar[B_QK_FULL], 0, (tile + 1) * kTile, sg.bh);
+                // k of tile + 2 into this tile's buffer once its projections and norms are done
+                if (tile + 2 < sg.t_end) {
+                    uint32_t pk = (ph_ke >> kb) & 1u;
+                    wt.wait(KE(kb), pk);
+                    ph_ke ^= 1u << kb;
+                    mbar_arrive_expect_tx(KF(kb), kTileBytes);
+                    tma_load_3d(sm + L.k + kb * kTileBytes, &tmk, KF(kb), 0, (tile + 2) * kTile, sg.bh);
                 }
+            }
+        }
+    } else if (warp == 11) {
+        // v tiles: one buffer, refilled once the previous tile's state update has read it
+        if (lane == 0) {
+            uint32_t ph_ve = 0;
+            for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+                if (tile > sg.t_begin) wt.wait(VE, ph_ve);
+                mbar_arrive_expect_tx(VF, kTileBytes);
+                tma_load_3d(sm + L.v, &tmv, VF, 0, tile * kTile, sg.bh);
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            uint32_t ph_kf = 0, ph_vf = 0, ph_wf = 0, ph_ue0 = 1, ph_ue1 = 1, ph_pk = 0;  // ph_pk: bit per buffer
+            uint32_t ph_kf = 0, ph_vf = 0, ph_wf = 0, ph_ue0 = 1, ph_ue1 = 1, ph_pk = 0;  // ph_kf, ph_pk: bit per buffer
             int n_glob = 0;
             constexpr uint32_t idU = idesc_bf16(128, 128, 0, 0);
             for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
                 const int b = (tile - sg.t_begin) & 1;
-                wt.wait(&bar[B_QK_FULL], ph_kf);
+                {
+                    uint32_t pk = (ph_kf >> b) & 1u;
+                    wt.wait(KF(b), pk);
+                    ph_kf ^= 1u << b;
+                }
+                const uint32_t kaddr = sbase + L.k + b * kTileBytes;
                 for (int n = 0; n < NT; ++n, ++n_glob) {
                     const int slot = n_glob & 1;
                     uint32_t ph = (ph_wf >> slot) & 1u;
@@ -324,26 +336,23 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         umma_bf16(tmem + kColUS + 128 * ub,
-                                  sdesc(sbase + L.k + 32 * kk, 16, 1024, kLayoutSW128),
+                                  sdesc(kaddr + 32 * kk, 16, 1024, kLayoutSW128),
                                   sdesc(w + 32 * kk, 16, 1024, kLayoutSW128), idU, kk > 0 ? 1u : 0u);
                     umma_commit(&bar[B_U_FULL0 + ub]);
                     umma_commit(&bar[B_W_EMPTY0 + slot]);
                 }
-                umma_commit(&bar[B_QK_EMPTY]);
+                umma_commit(KE(b));
                 {
                     uint32_t pp = (ph_pk >> b) & 1u;
                     wt.wait(PKF(b), pp);
                     ph_pk ^= 1u << b;
                 }
-                uint32_t pv = (ph_vf >> b) & 1u;
-                wt.wait(&VF[b], pv);
-                ph_vf ^= (1u << b);
+                wt.wait(VF, ph_vf);
                 tc_fence_after();
                 for (int h = 0; h < halves; ++h)
-                    issue_state_half(tmem, kColSS, sbase + L.phik + b * phik_bytes,
-                                     sbase + L.v + b * kTileBytes, sbase + L.ones, h,
-                                     tile == sg.t_begin);
-                umma_commit(&VE[b]);
+                    issue_state_half(tmem, kColSS, sbase + L.phik + b * phik_bytes, sbase + L.v,
+                                     sbase + L.ones, h, tile == sg.t_begin);
+                umma_commit(VE);
                 umma_commit(&TD[b]);
             }
         }
@@ -374,10 +383,14 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         uint32_t ph_kf = 0, ph_uf = 0, ph_td = 0;
         for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
             const int li = tile - sg.t_begin, b = li & 1;
-            wt.wait(&bar[B_QK_FULL], ph_kf);
+            {
+                uint32_t pk = (ph_kf >> b) & 1u;
+                wt.wait(KF(b), pk);
+                ph_kf ^= 1u << b;
+            }
             float inv, l2i;
-            row_scale(sm + L.k + row * 128, inv, l2i);
-            warp_arrive(&bar[B_QK_EMPTY]);
+            row_scale(sm + L.k + b * kTileBytes + row * 128, inv, l2i);
+            warp_arrive(KE(b));
             if (li >= 2) {   // phiK buffer b free again (update and store of tile li-2 done)
                 uint32_t pt = (ph_td >> b) & 1u, ps = pt;   // wait() flips its argument
                 wt.wait(&TD[b], pt);
