@@ -14,6 +14,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 
 #include "slay_internal.h"
@@ -696,9 +697,10 @@ __global__ void __launch_bounds__(NT) k_phi_bwd(const Tin* __restrict__ x,
 // One block per group of G sequences (b,h).  Phase 1: phi of q and k of the group.
 // Phase 2: stream S (read, add phi(k) v^T, write) and accumulate phi(q)^T S.
 constexpr int G = 4;
+constexpr int kDecodeBlocksPerSM = 5;   // register cap 51/thread: 5 resident blocks per SM
 
 template <typename T>
-__global__ void __launch_bounds__(NT) k_decode(const T* __restrict__ q, const T* __restrict__ k,
+__global__ void __launch_bounds__(NT, kDecodeBlocksPerSM) k_decode(const T* __restrict__ q, const T* __restrict__ k,
                                                const T* __restrict__ v, float* __restrict__ S,
                                                float* __restrict__ z, T* __restrict__ out, int N,
                                                Params P, float eps)
@@ -711,7 +713,8 @@ __global__ void __launch_bounds__(NT) k_decode(const T* __restrict__ q, const T*
     __shared__ float dred[NT / 32];
     const int tid = threadIdx.x;
     const int F = P.F;
-    const int n0 = blockIdx.x * G;
+    // persistent: block b serves groups b, b + gridDim.x, ... of G sequences each
+    for (int n0 = blockIdx.x * G; n0 < N; n0 += gridDim.x * G) {
     for (int idx = tid; idx < 2 * G * kD; idx += NT) {
         const int r = idx / kD, d = idx % kD;
         const int g = r % G, n = n0 + g;
@@ -788,6 +791,7 @@ __global__ void __launch_bounds__(NT) k_decode(const T* __restrict__ q, const T*
             st(out + static_cast<int64_t>(n) * kD + tid, num / (d + eps));
         }
         __syncthreads();
+    }
     }
 }
 
@@ -991,9 +995,16 @@ static cudaError_t decode_t(const void* q, const void* k, const void* v, float* 
                                     static_cast<int>(smem))) != cudaSuccess)
         return err;
     {
+        // one wave of resident blocks looping over the groups (no partial last wave)
+        int per_sm = 0, sms = 0, dev = 0;
+        if ((err = cudaGetDevice(&dev)) != cudaSuccess ||
+            (err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+            (err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode<T>, NT, smem)) != cudaSuccess)
+            return err;
+        const int groups = (N + G - 1) / G;
+        const int grid = std::max(1, std::min(groups, std::max(1, per_sm) * sms));
         TraceScope trace_("simt_decode", st);
-        k_decode<T><<<(N + G - 1) / G, NT, smem, st>>>(cp<T>(q), cp<T>(k), cp<T>(v), S, z, mp<T>(out),
-                                                       N, P, eps);
+        k_decode<T><<<grid, NT, smem, st>>>(cp<T>(q), cp<T>(k), cp<T>(v), S, z, mp<T>(out), N, P, eps);
     }
     return cudaGetLastError();
 }
