@@ -181,19 +181,34 @@ __global__ void k_scan(float* __restrict__ stt, float* __restrict__ tot, int BH,
     if (gid >= static_cast<int64_t>(BH) * FE) return;
     const int bh = static_cast<int>(gid / FE), idx = static_cast<int>(gid % FE);
     float* base = stt + static_cast<int64_t>(bh) * NC * FE + idx;
+    // chunks are read kBatch at a time (independent loads in flight), then summed in the
+    // same sequential order as a one-by-one walk
+    constexpr int kBatch = 16;
     float run = 0.0f;
-    if (mode == 2) {
-        for (int c = 0; c < NC; ++c) run += base[static_cast<int64_t>(c) * FE];
-        tot[static_cast<int64_t>(bh) * FE + idx] = run;
-        return;
+    for (int c0 = 0; c0 < NC; c0 += kBatch) {
+        float x[kBatch];
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+            const int cc = c0 + j;
+            const int c = (mode == 1) ? NC - 1 - cc : cc;
+            x[j] = (cc < NC) ? base[static_cast<int64_t>(c) * FE] : 0.0f;
+        }
+        if (mode == 2) {
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) run += x[j];
+            continue;
+        }
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+            const int cc = c0 + j;
+            if (cc < NC) {
+                const int c = (mode == 1) ? NC - 1 - cc : cc;
+                base[static_cast<int64_t>(c) * FE] = run;
+            }
+            run += x[j];
+        }
     }
-    for (int cc = 0; cc < NC; ++cc) {
-        const int c = (mode == 0) ? cc : NC - 1 - cc;
-        float* p = base + static_cast<int64_t>(c) * FE;
-        const float tmp = *p;
-        *p = run;
-        run += tmp;
-    }
+    if (mode == 2) tot[static_cast<int64_t>(bh) * FE + idx] = run;
 }
 
 // --------------------------------------------------------------- chunk output
