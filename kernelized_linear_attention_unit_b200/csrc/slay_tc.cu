@@ -172,31 +172,43 @@ __device__ __forceinline__ float phi_sub_epilogue(const uint32_t (&ur)[32], cons
     return dz;
 }
 
-// U (64 columns: 32 u then 32 p) = X [128 x 64] . W_n^T [64 x 64]
-__device__ __forceinline__ void issue_projection(uint32_t d_tmem, uint32_t x_addr, uint32_t w_addr)
+// Shared-memory descriptors are built once per operand buffer and stepped with plain adds:
+// the start-address field holds addr >> 4 in the low bits and every operand lies below
+// 256 KiB, so adding bytes >> 4 never carries into the next field.  (Rebuilding a
+// descriptor per MMA puts a chain of dependent integer ops in front of every issue and
+// halves the single issuing thread's MMA rate.)
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
+// K-major 128-byte-swizzled operand at `addr` (rows 128 bytes apart, 8-row groups 1 KiB apart)
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t addr) { return sdesc(addr, 16, 1024, kLayoutSW128); }
+
+// U (64 columns: 32 u then 32 p) = X [128 x 64] . W_n^T [64 x 64]; dx, dw: K-major descriptors
+__device__ __forceinline__ void issue_projection(uint32_t d_tmem, uint64_t dx, uint64_t dw)
 {
     constexpr uint32_t id = idesc_bf16(128, 64, 0, 0);
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-        umma_bf16(d_tmem, sdesc(x_addr + 32 * kk, 16, 1024, kLayoutSW128),
-                  sdesc(w_addr + 32 * kk, 16, 1024, kLayoutSW128), id, kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < 4; ++kk) umma_bf16(d_tmem, dx + 2 * kk, dw + 2 * kk, id, kk > 0 ? 1u : 0u);
 }
 
 // [S|z]_h (+)= phiK_h^T [V | 1] for feature half h: phiK as an MN-major A operand
 // (128 features = two 64-feature sub-tiles 16 KiB apart); B = V as an MN-major operand of
 // width 80 whose columns 64..79 come from the ones tile at LBO (= ones - V) bytes.
-__device__ __forceinline__ void issue_state_half(uint32_t tmem, uint32_t colS, uint32_t phik,
-                                                 uint32_t vaddr, uint32_t ones, int h, bool first)
+// dphik: desc_phik(phik base), dv: desc_v(v, ones) (see below)
+__device__ __forceinline__ void issue_state_half(uint32_t tmem, uint32_t colS, uint64_t dphik,
+                                                 uint64_t dv, int h, bool first)
 {
     constexpr uint32_t idS = idesc_bf16(128, 80, 1, 1);
-    const uint32_t a0 = phik + 2 * h * kTileBytes;
-    const uint32_t lbo = ones - vaddr;
+    const uint64_t da = desc_add(dphik, 2 * h * kTileBytes);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
-        umma_bf16(tmem + colS + 80 * h, sdesc(a0 + 2048 * kk, kTileBytes, 1024, kLayoutSW128),
-                  sdesc(vaddr + 2048 * kk, lbo, 1024, kLayoutSW128), idS,
+        umma_bf16(tmem + colS + 80 * h, da + 128 * kk, dv + 128 * kk, idS,
                   (first && kk == 0) ? 0u : 1u);
 }
+
+// phi(k) slices as the MN-major A operand of the state update (two 64-feature sub-tiles
+// 16 KiB apart), and [V | 1] as an MN-major B operand (the ones tile at LBO = ones - v)
+__device__ __forceinline__ uint64_t desc_phik(uint32_t phik) { return sdesc(phik, kTileBytes, 1024, kLayoutSW128); }
+__device__ __forceinline__ uint64_t desc_v(uint32_t v, uint32_t ones) { return sdesc(v, ones - v, 1024, kLayoutSW128); }
 
 __device__ __forceinline__ void fill_ones(unsigned char* ones)
 {
@@ -316,6 +328,8 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             uint32_t ph_kf = 0, ph_vf = 0, ph_wf = 0, ph_ue0 = 1, ph_ue1 = 1, ph_pk = 0;  // ph_kf, ph_pk: bit per buffer
             int n_glob = 0;
             constexpr uint32_t idU = idesc_bf16(128, 128, 0, 0);
+            const uint64_t dk0 = desc_kmajor(sbase + L.k), dw0 = desc_kmajor(sbase + L.w);
+            const uint64_t dph0 = desc_phik(sbase + L.phik), dv = desc_v(sbase + L.v, sbase + L.ones);
             for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
                 const int b = (tile - sg.t_begin) & 1;
                 {
@@ -323,7 +337,7 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                     wt.wait(KF(b), pk);
                     ph_kf ^= 1u << b;
                 }
-                const uint32_t kaddr = sbase + L.k + b * kTileBytes;
+                const uint64_t dk = desc_add(dk0, b * kTileBytes);
                 for (int n = 0; n < NT; ++n, ++n_glob) {
                     const int slot = n_glob & 1;
                     uint32_t ph = (ph_wf >> slot) & 1u;
@@ -332,12 +346,10 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                     const int ub = n & 1;
                     wt.wait(&bar[B_U_EMPTY0 + ub], ub ? ph_ue1 : ph_ue0);
                     tc_fence_after();
-                    const uint32_t w = sbase + L.w + slot * kWStateBytes;
+                    const uint64_t dw = desc_add(dw0, slot * kWStateBytes);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(tmem + kColUS + 128 * ub,
-                                  sdesc(kaddr + 32 * kk, 16, 1024, kLayoutSW128),
-                                  sdesc(w + 32 * kk, 16, 1024, kLayoutSW128), idU, kk > 0 ? 1u : 0u);
+                        umma_bf16(tmem + kColUS + 128 * ub, dk + 2 * kk, dw + 2 * kk, idU, kk > 0 ? 1u : 0u);
                     umma_commit(&bar[B_U_FULL0 + ub]);
                     umma_commit(&bar[B_W_EMPTY0 + slot]);
                 }
@@ -350,8 +362,8 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 wt.wait(VF, ph_vf);
                 tc_fence_after();
                 for (int h = 0; h < halves; ++h)
-                    issue_state_half(tmem, kColSS, sbase + L.phik + b * phik_bytes, sbase + L.v,
-                                     sbase + L.ones, h, tile == sg.t_begin);
+                    issue_state_half(tmem, kColSS, desc_add(dph0, b * phik_bytes), dv, h,
+                                     tile == sg.t_begin);
                 umma_commit(VE);
                 umma_commit(&TD[b]);
             }
@@ -588,6 +600,7 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 constexpr uint32_t idP = idesc_bf16(128, 128, 0, 0);
                 constexpr uint32_t idO = idesc_bf16(128, 80, 0, 1);
                 constexpr uint32_t idPV = idesc_bf16(128, 80, 0, 1);
+                const uint32_t st_sbo = static_cast<uint32_t>(kp.F) * 16;
                 for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
                     const bool last = tile + 1 == sg.t_end;
                     for (int t = 0; t < NT; ++t) {
@@ -603,24 +616,23 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                             wt.wait(&bar[B_O_EMPTY], ph_oe);
                         }
                         tc_fence_after();
-                        const uint32_t aq = sbase + L.phiq + pslot * kTileBytes;
-                        const uint32_t bk = sbase + L.phik + t * kTileBytes;
-                        const uint32_t bs = sbase + L.st + t * (kSlice / 8) * 128;
-                        const uint32_t st_sbo = static_cast<uint32_t>(kp.F) * 16;
-    #pragma unroll
+                        // descriptors once per slice, stepped by adds over its 4 K steps
+                        const uint64_t ad = desc_kmajor(sbase + L.phiq + pslot * kTileBytes);
+                        const uint64_t bk = desc_kmajor(sbase + L.phik + t * kTileBytes);
+                        const uint64_t bs = sdesc(sbase + L.st + t * (kSlice / 8) * 128, 128, st_sbo, kLayoutNone);
+#pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
                             const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-                            const uint64_t ad = sdesc(aq + 32 * kk, 16, 1024, kLayoutSW128);
-                            umma_bf16(tmem + kColP, ad, sdesc(bk + 32 * kk, 16, 1024, kLayoutSW128), idP, acc);
-                            umma_bf16(tmem + kColO, ad, sdesc(bs + 256 * kk, 128, st_sbo, kLayoutNone), idO, acc);
+                            umma_bf16(tmem + kColP, ad + 2 * kk, bk + 2 * kk, idP, acc);
+                            umma_bf16(tmem + kColO, ad + 2 * kk, bs + 16 * kk, idO, acc);
                         }
                         umma_commit(&bar[B_PQ_EMPTY0 + pslot]);
                         // state update of a feature half once its phiK slices are in place; the
                         // half's phiK slices are free for the next tile once it has been read
                         if (!last && (t & 1) == 1) {
                             if (t == 1) wt.wait(&bar[B_V_FULL], ph_vf);
-                            issue_state_half(tmem, kColS, sbase + L.phik, sbase + L.v, sbase + L.ones,
-                                             t >> 1, false);
+                            issue_state_half(tmem, kColS, desc_phik(sbase + L.phik),
+                                                 desc_v(sbase + L.v, sbase + L.ones), t >> 1, false);
                             umma_commit(&bar[B_PK_FREE0 + (t >> 1)]);
                         }
                     }
@@ -628,11 +640,10 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                     if (last) wt.wait(&bar[B_V_FULL], ph_vf);
                     wt.wait(&bar[B_PSM_FULL], ph_psm);
                     tc_fence_after();
-                    const uint32_t lbo = L.ones - L.v;
-    #pragma unroll
+                    const uint64_t dvv = desc_v(sbase + L.v, sbase + L.ones);
+#pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        umma_bf16_ts(tmem + kColO, tmem + kColP + 8 * kk,
-                                     sdesc(sbase + L.v + 2048 * kk, lbo, 1024, kLayoutSW128), idPV, 1u);
+                        umma_bf16_ts(tmem + kColO, tmem + kColP + 8 * kk, dvv + 128 * kk, idPV, 1u);
                     umma_commit(&bar[B_TILE_DONE]);
                     umma_commit(&bar[B_V_EMPTY]);
                 }
@@ -641,7 +652,7 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             // ------------------------------------------- projection issuers (q: 2, k: 3)
             if (lane == 0) {
                 const int g = warp - 2;
-                const uint32_t xaddr = sbase + (g ? L.k : L.q);
+                const uint64_t dx = desc_kmajor(sbase + (g ? L.k : L.q)), dw0 = desc_kmajor(sbase + L.w);
                 uint32_t ph_qkf = 0, ph_wf = 0, ph_ue = 1;
                 int n_glob = 0;
                 for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
@@ -653,7 +664,7 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                         ph_wf ^= (1u << slot);
                         wt.wait(&bar[B_U_EMPTY0 + g], ph_ue);
                         tc_fence_after();
-                        issue_projection(tmem + (g ? kColU1 : kColU0), xaddr, sbase + L.w + slot * kWBytes);
+                        issue_projection(tmem + (g ? kColU1 : kColU0), dx, desc_add(dw0, slot * kWBytes));
                         umma_commit(&bar[B_U_FULL0 + g]);
                         umma_commit(&bar[B_W_EMPTY0 + slot]);
                     }
@@ -996,6 +1007,7 @@ k_tc_causal_out_pk(const __grid_constant__ CUtensorMap tmq, const __grid_constan
             // ------------------------------------------------- q projection issuer
             if (lane == 0) {
                 uint32_t ph_qf = 0, ph_wf = 0, ph_ue = 0x3u;
+                const uint64_t dqx0 = desc_kmajor(sbase + L.q), dw0 = desc_kmajor(sbase + L.w);
                 int n_glob = 0;
                 for (int tile = sg.t_begin, it = 0; tile < sg.t_end; ++tile, ++it) {
                     const int qb = it & 1;
@@ -1011,8 +1023,8 @@ k_tc_causal_out_pk(const __grid_constant__ CUtensorMap tmq, const __grid_constan
                         wt.wait(&bar[B_U_EMPTY0 + g], pu);
                         ph_ue ^= 1u << g;
                         tc_fence_after();
-                        issue_projection(tmem + (g ? kColU1 : kColU0), sbase + L.q + qb * kTileBytes,
-                                         sbase + L.w + slot * kWBytes);
+                        issue_projection(tmem + (g ? kColU1 : kColU0), desc_add(dqx0, qb * kTileBytes),
+                                         desc_add(dw0, slot * kWBytes));
                         umma_commit(&bar[B_U_FULL0 + g]);
                         umma_commit(&bar[B_W_EMPTY0 + slot]);
                     }
@@ -1046,22 +1058,22 @@ k_tc_causal_out_pk(const __grid_constant__ CUtensorMap tmq, const __grid_constan
                             wt.wait(&bar[B_O_EMPTY], ph_oe);
                         }
                         tc_fence_after();
-                        const uint32_t aq = sbase + L.phiq + pslot * kTileBytes;
-                        const uint32_t bk = sbase + L.phik + t * kTileBytes;
-                        const uint32_t bs = sbase + L.st + t * (kSlice / 8) * 128;
+                        // descriptors once per slice, stepped by adds over its 4 K steps
+                        const uint64_t ad = desc_kmajor(sbase + L.phiq + pslot * kTileBytes);
+                        const uint64_t bk = desc_kmajor(sbase + L.phik + t * kTileBytes);
+                        const uint64_t bs = sdesc(sbase + L.st + t * (kSlice / 8) * 128, 128, st_sbo, kLayoutNone);
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
                             const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-                            const uint64_t ad = sdesc(aq + 32 * kk, 16, 1024, kLayoutSW128);
-                            umma_bf16(tmem + kColP, ad, sdesc(bk + 32 * kk, 16, 1024, kLayoutSW128), idP, acc);
-                            umma_bf16(tmem + kColO, ad, sdesc(bs + 256 * kk, 128, st_sbo, kLayoutNone), idO, acc);
+                            umma_bf16(tmem + kColP, ad + 2 * kk, bk + 2 * kk, idP, acc);
+                            umma_bf16(tmem + kColO, ad + 2 * kk, bs + 16 * kk, idO, acc);
                         }
                         umma_commit(&bar[B_PQ_EMPTY0 + pslot]);
                         if ((t & 1) == 1) {
                             if (!last) {
                                 if (t == 1) wt.wait(&bar[B_V_FULL], ph_vf);
-                                issue_state_half(tmem, kColS, sbase + L.phik, sbase + L.v,
-                                                 sbase + L.ones, t >> 1, false);
+                                issue_state_half(tmem, kColS, desc_phik(sbase + L.phik),
+                                                 desc_v(sbase + L.v, sbase + L.ones), t >> 1, false);
                             }
                             // the loader needs this half free again for the next tile
                             if (!last) umma_commit(&bar[B_PK_FREE0 + (t >> 1)]);
@@ -1071,11 +1083,10 @@ k_tc_causal_out_pk(const __grid_constant__ CUtensorMap tmq, const __grid_constan
                     if (last) wt.wait(&bar[B_V_FULL], ph_vf);
                     wt.wait(&bar[B_PSM_FULL], ph_psm);
                     tc_fence_after();
-                    const uint32_t lbo = L.ones - L.v;
+                    const uint64_t dvv = desc_v(sbase + L.v, sbase + L.ones);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        umma_bf16_ts(tmem + kColO, tmem + kColP + 8 * kk,
-                                     sdesc(sbase + L.v + 2048 * kk, lbo, 1024, kLayoutSW128), idPV, 1u);
+                        umma_bf16_ts(tmem + kColO, tmem + kColP + 8 * kk, dvv + 128 * kk, idPV, 1u);
                     umma_commit(&bar[B_TILE_DONE]);
                     umma_commit(&bar[B_V_EMPTY]);
                 }
@@ -1394,6 +1405,7 @@ k_tc_bidir_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
     } else if (warp == 2) {
         if (lane == 0) {
             uint32_t ph_qf = 0, ph_wf = 0, ph_ue = 0x3u;
+            const uint64_t dqx0 = desc_kmajor(sbase + L.q), dw0 = desc_kmajor(sbase + L.w);
             int n_glob = 0;
             for (int tile = sg.t_begin, it = 0; tile < sg.t_end; ++tile, ++it) {
                 const int qb = it & 1;
@@ -1409,8 +1421,7 @@ k_tc_bidir_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                     wt.wait(&bar[B_U_EMPTY0 + g], pu);
                     ph_ue ^= 1u << g;
                     tc_fence_after();
-                    issue_projection(tmem + 64 * g, sbase + L.q + qb * kTileBytes,
-                                     sbase + L.w + slot * kWBytes);
+                    issue_projection(tmem + 64 * g, desc_add(dqx0, qb * kTileBytes), desc_add(dw0, slot * kWBytes));
                     umma_commit(&bar[B_U_FULL0 + g]);
                     umma_commit(&bar[B_W_EMPTY0 + slot]);
                 }
@@ -1421,7 +1432,8 @@ k_tc_bidir_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
         if (lane == 0) {
             uint32_t ph_pqf = 0, ph_oe = 0;
             constexpr uint32_t idO = idesc_bf16(128, 80, 0, 1);
-            const uint32_t st_sbo = static_cast<uint32_t>(kp.F) * 16;
+            const uint64_t dq0 = desc_kmajor(sbase + L.phiq);
+            const uint64_t ds0 = sdesc(sbase + L.st, 128, static_cast<uint32_t>(kp.F) * 16, kLayoutNone);
             for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
                 for (int t = 0; t < NT; ++t) {
                     const int pslot = t & 1;
@@ -1430,13 +1442,11 @@ k_tc_bidir_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                     ph_pqf ^= 1u << pslot;
                     if (t == 0 && tile > sg.t_begin) wt.wait(&bar[B_O_EMPTY], ph_oe);
                     tc_fence_after();
-                    const uint32_t aq = sbase + L.phiq + pslot * kTileBytes;
-                    const uint32_t bs = sbase + L.st + t * (kSlice / 8) * 128;
+                    const uint64_t ad = desc_add(dq0, pslot * kTileBytes);
+                    const uint64_t bs = desc_add(ds0, t * (kSlice / 8) * 128);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(tmem + kColO2, sdesc(aq + 32 * kk, 16, 1024, kLayoutSW128),
-                                  sdesc(bs + 256 * kk, 128, st_sbo, kLayoutNone), idO,
-                                  (t > 0 || kk > 0) ? 1u : 0u);
+                        umma_bf16(tmem + kColO2, ad + 2 * kk, bs + 16 * kk, idO, (t > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&bar[B_PQ_EMPTY0 + pslot]);
                 }
                 umma_commit(&bar[B_TILE_DONE]);

@@ -141,13 +141,16 @@ k_tc_feature_map(const __grid_constant__ CUtensorMap tmx, const __grid_constant_
             uint32_t ph_w = 0, ph_xf = 0;
             wt.wait(&bar[FB_W], ph_w);
             constexpr uint32_t idU = idesc_bf16(128, 128, 0, 0);
+            // descriptors built once, stepped by adds (see the causal kernels)
+            const uint64_t dx0 = sdesc(sbase + L.x, 16, 1024, kLayoutSW128);
+            const uint64_t dw0 = sdesc(sbase + L.w, 16, 1024, kLayoutSW128);
             int it = 0, j = 0;
             for (int tile = blockIdx.x; tile < fp.ntiles; tile += gridDim.x, ++it) {
                 const int s = it % xbufs;
                 uint32_t ph = (ph_xf >> s) & 1u;
                 wt.wait(&bar[FB_XF + s], ph);
                 ph_xf ^= 1u << s;
-                const uint32_t xa = sbase + L.x + s * kBoxBytes;
+                const uint64_t dx = dx0 + ((s * kBoxBytes) >> 4);
                 for (int g = 0; g < ngroups; ++g, ++j) {
                     const int b = j % kUBufs;
                     if (j >= kUBufs) {
@@ -155,11 +158,10 @@ k_tc_feature_map(const __grid_constant__ CUtensorMap tmx, const __grid_constant_
                         wt.wait(&bar[FB_UE + b], pu);
                     }
                     tc_fence_after();
-                    const uint32_t wa = sbase + L.w + g * kGroupBytes;
+                    const uint64_t dw = dw0 + ((g * kGroupBytes) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(tmem + 128 * b, sdesc(xa + 32 * kk, 16, 1024, kLayoutSW128),
-                                  sdesc(wa + 32 * kk, 16, 1024, kLayoutSW128), idU, kk > 0 ? 1u : 0u);
+                        umma_bf16(tmem + 128 * b, dx + 2 * kk, dw + 2 * kk, idU, kk > 0 ? 1u : 0u);
                     umma_commit(&bar[FB_UF + b]);
                 }
                 umma_commit(&bar[FB_XE + s]);
