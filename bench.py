@@ -113,9 +113,11 @@ def kernel_work(name, w, op):
     if name in ("tc_bidir_state",):
         return th * (4 * D * F + 2 * F * Dv), "flop", "tensor"
     # the feature-map workload maps q and k rows (2 th rows, bf16 -> bf16) in one launch;
-    # the CUDA-core attention paths map q and k separately (th rows, fp32 features)
+    # the CUDA-core attention paths map q and k separately (th rows each; bf16 features in
+    # bf16 mode through the tensor-core map, fp32 features in fp32 mode)
     if name == "tc_feature_map":
-        return 2 * th * (D * 2 + F * 2), "byte", "hbm"
+        rows = 2 * th if op == "feature_map" else th
+        return rows * (D * 2 + F * 2), "byte", "hbm"
     if name == "simt_feature_map":
         if op == "feature_map":
             return 2 * th * (D * 2 + F * 2), "byte", "hbm"

@@ -15,9 +15,11 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <type_traits>
 #include <cstdint>
 
 #include "slay_internal.h"
+#include "slay_tc.h"
 
 namespace slay {
 namespace {
@@ -120,8 +122,8 @@ __global__ void __launch_bounds__(NT) k_feature_map(const Tin* __restrict__ x,
 // grid (ceil(F/64), NC, BH).  st[bh][c][f][e] = sum_{t in chunk c} phi[t][f] * Y[t][e],
 // e < 64 from Y, e = 64 the "ones" column (Y1 == nullptr) or Y's own column 64.
 // Y is either v (type T, 64 columns) or an fp32 [L][65] array.
-template <typename TY>
-__global__ void __launch_bounds__(NT) k_chunk_state(const float* __restrict__ phi,
+template <typename TY, typename TP>
+__global__ void __launch_bounds__(NT) k_chunk_state(const TP* __restrict__ phi,
                                                     const TY* __restrict__ Y, int ycols,
                                                     float* __restrict__ stt, int L, int F)
 {
@@ -131,11 +133,11 @@ __global__ void __launch_bounds__(NT) k_chunk_state(const float* __restrict__ ph
     const int f0 = blockIdx.x * C, c = blockIdx.y, bh = blockIdx.z;
     const int NC = gridDim.y;
     const int t0 = c * C;
-    const float* phb = phi + static_cast<int64_t>(bh) * L * F;
+    const TP* phb = phi + static_cast<int64_t>(bh) * L * F;
     const TY* yb = Y + static_cast<int64_t>(bh) * L * ycols;
     for (int idx = tid; idx < C * C; idx += NT) {
         const int t = idx >> 6, fl = idx & 63;
-        ph[t][fl] = (t0 + t < L && f0 + fl < F) ? phb[static_cast<int64_t>(t0 + t) * F + f0 + fl] : 0.0f;
+        ph[t][fl] = (t0 + t < L && f0 + fl < F) ? ld(phb + static_cast<int64_t>(t0 + t) * F + f0 + fl) : 0.0f;
     }
     for (int idx = tid; idx < C * E; idx += NT) {
         const int t = idx / E, e = idx % E;
@@ -223,8 +225,8 @@ struct OutSmem {
 };
 
 template <typename T>
-__global__ void __launch_bounds__(NT) k_chunk_out(const float* __restrict__ phq,
-                                                  const float* __restrict__ phk,
+__global__ void __launch_bounds__(NT) k_chunk_out(const T* __restrict__ phq,
+                                                  const T* __restrict__ phk,
                                                   const T* __restrict__ v,
                                                   const float* __restrict__ stt,
                                                   T* __restrict__ out, float* __restrict__ den,
@@ -235,8 +237,8 @@ __global__ void __launch_bounds__(NT) k_chunk_out(const float* __restrict__ phq,
     const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
     const int c = blockIdx.x, bh = blockIdx.y, NC = gridDim.x;
     const int i0 = c * C;
-    const float* qb = phq + static_cast<int64_t>(bh) * L * F;
-    const float* kb = phk + static_cast<int64_t>(bh) * L * F;
+    const T* qb = phq + static_cast<int64_t>(bh) * L * F;
+    const T* kb = phk + static_cast<int64_t>(bh) * L * F;
     const T* vb = v + static_cast<int64_t>(bh) * L * kD;
     // state entering this chunk (causal: exclusive prefix of chunk c; bidir: total)
     const float* sb = causal ? stt + (static_cast<int64_t>(bh) * NC + c) * F * E
@@ -257,8 +259,8 @@ __global__ void __launch_bounds__(NT) k_chunk_out(const float* __restrict__ phq,
                 const int t = idx >> 6, fl = idx & 63;
                 const bool ok = (i0 + t < L) && (f0 + fl < F);
                 const int64_t off = static_cast<int64_t>(i0 + t) * F + f0 + fl;
-                sm.qs[t][fl] = ok ? qb[off] : 0.0f;
-                sm.kt[t][fl] = ok ? kb[off] : 0.0f;
+                sm.qs[t][fl] = ok ? ld(qb + off) : 0.0f;
+                sm.kt[t][fl] = ok ? ld(kb + off) : 0.0f;
             }
             __syncthreads();
 #pragma unroll 4
@@ -301,7 +303,7 @@ __global__ void __launch_bounds__(NT) k_chunk_out(const float* __restrict__ phq,
         __syncthreads();
         for (int idx = tid; idx < C * C; idx += NT) {
             const int t = idx >> 6, fl = idx & 63;
-            sm.qs[t][fl] = (i0 + t < L && f0 + fl < F) ? qb[static_cast<int64_t>(i0 + t) * F + f0 + fl] : 0.0f;
+            sm.qs[t][fl] = (i0 + t < L && f0 + fl < F) ? ld(qb + static_cast<int64_t>(i0 + t) * F + f0 + fl) : 0.0f;
         }
         for (int idx = tid; idx < C * E; idx += NT) {
             const int fl = idx / E, e = idx % E;
@@ -376,8 +378,8 @@ struct BwdSmem {
 //   dphi(k_j) = sum_i c_ij phi(q_i) + G_c [v_j; 1]               (G_c = sum over later
 //   dv_j      = sum_i P_ij dn_i + G_c[:, :64]^T phi(k_j)           chunks of phi(q)[dn, delta]^T)
 template <typename T>
-__global__ void __launch_bounds__(NT) k_bwd_chunk(const float* __restrict__ phq,
-                                                  const float* __restrict__ phk,
+__global__ void __launch_bounds__(NT) k_bwd_chunk(const T* __restrict__ phq,
+                                                  const T* __restrict__ phk,
                                                   const T* __restrict__ v,
                                                   const float* __restrict__ dn,
                                                   const float* __restrict__ sfw,
@@ -392,8 +394,8 @@ __global__ void __launch_bounds__(NT) k_bwd_chunk(const float* __restrict__ phq,
     const int c = blockIdx.x, bh = blockIdx.y, NC = gridDim.x;
     const int i0 = c * C;
     const int64_t rb = static_cast<int64_t>(bh) * L;
-    const float* qb = phq + rb * F;
-    const float* kb = phk + rb * F;
+    const T* qb = phq + rb * F;
+    const T* kb = phk + rb * F;
     const float* S = sfw + (static_cast<int64_t>(bh) * NC + c) * F * E;
     const float* G = gbw + (static_cast<int64_t>(bh) * NC + c) * F * E;
 
@@ -411,8 +413,8 @@ __global__ void __launch_bounds__(NT) k_bwd_chunk(const float* __restrict__ phq,
             const int t = idx >> 6, fl = idx & 63;
             const bool ok = (i0 + t < L) && (f0 + fl < F);
             const int64_t off = static_cast<int64_t>(i0 + t) * F + f0 + fl;
-            sm.a[t][fl] = ok ? qb[off] : 0.0f;
-            sm.b[t][fl] = ok ? kb[off] : 0.0f;
+            sm.a[t][fl] = ok ? ld(qb + off) : 0.0f;
+            sm.b[t][fl] = ok ? ld(kb + off) : 0.0f;
         }
         __syncthreads();
         for (int fl = 0; fl < C; ++fl) {
@@ -469,8 +471,8 @@ __global__ void __launch_bounds__(NT) k_bwd_chunk(const float* __restrict__ phq,
             const int t = idx >> 6, fl = idx & 63;
             const bool ok = (i0 + t < L) && (f0 + fl < F);
             const int64_t off = static_cast<int64_t>(i0 + t) * F + f0 + fl;
-            sm.a[t][fl] = ok ? qb[off] : 0.0f;
-            sm.b[t][fl] = ok ? kb[off] : 0.0f;
+            sm.a[t][fl] = ok ? ld(qb + off) : 0.0f;
+            sm.b[t][fl] = ok ? ld(kb + off) : 0.0f;
         }
         for (int idx = tid; idx < C * E; idx += NT) {
             const int fl = idx / E, e = idx % E;
@@ -867,6 +869,15 @@ cudaError_t simt_feature_map(const void* x, void* phi, int64_t n, slay_dtype in_
     return fm_launch<__nv_bfloat16, float>(x, phi, n, P, st);
 }
 
+// phi of `rows` rows of x in the mode's dtype: tensor cores for bf16 where the shape allows
+template <typename T>
+static cudaError_t phi_map(const void* x, T* phi, int64_t rows, const Params& P, cudaStream_t st)
+{
+    if (std::is_same<T, __nv_bfloat16>::value && P.wB && tc_fmap_supported(P.D, P.R, P.m, rows))
+        return tc_feature_map(x, phi, rows, P, st);
+    return fm_launch<T, T>(x, phi, rows, P, st);
+}
+
 template <typename T>
 static cudaError_t attn_fwd_t(const void* q, const void* k, const void* v, void* out, float* den,
                               int B, int H, int L, const Params& P, float eps, bool causal,
@@ -875,17 +886,18 @@ static cudaError_t attn_fwd_t(const void* q, const void* k, const void* v, void*
     const int BH = B * H, F = P.F, NC = nchunks(L);
     const int64_t rows = static_cast<int64_t>(BH) * L;
     char* w = static_cast<char*>(ws);
-    float* phq = reinterpret_cast<float*>(w);
-    float* phk = reinterpret_cast<float*>(w + align256(rows * F * sizeof(float)));
+    // phi(q), phi(k) in the mode's dtype (the buffers are sized for fp32)
+    T* phq = reinterpret_cast<T*>(w);
+    T* phk = reinterpret_cast<T*>(w + align256(rows * F * sizeof(float)));
     float* stt = reinterpret_cast<float*>(w + 2 * align256(rows * F * sizeof(float)));
     float* tot = reinterpret_cast<float*>(w + 2 * align256(rows * F * sizeof(float)) +
                                           align256(static_cast<size_t>(BH) * NC * F * E * sizeof(float)));
     cudaError_t err;
-    if ((err = fm_launch<T, float>(q, phq, rows, P, st)) != cudaSuccess) return err;
-    if ((err = fm_launch<T, float>(k, phk, rows, P, st)) != cudaSuccess) return err;
+    if ((err = phi_map<T>(q, phq, rows, P, st)) != cudaSuccess) return err;
+    if ((err = phi_map<T>(k, phk, rows, P, st)) != cudaSuccess) return err;
     {
         TraceScope trace_("simt_chunk_state", st);
-        k_chunk_state<T><<<dim3((F + C - 1) / C, NC, BH), NT, 0, st>>>(phk, cp<T>(v), kD, stt, L, F);
+        k_chunk_state<T, T><<<dim3((F + C - 1) / C, NC, BH), NT, 0, st>>>(phk, cp<T>(v), kD, stt, L, F);
     }
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     const int FE = F * E;
@@ -926,16 +938,16 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
     const size_t phb = align256(rows * F * sizeof(float));
     const size_t stb = align256(static_cast<size_t>(BH) * NC * F * E * sizeof(float));
     char* w = static_cast<char*>(ws);
-    float* phq = reinterpret_cast<float*>(w);
-    float* phk = reinterpret_cast<float*>(w + phb);
+    T* phq = reinterpret_cast<T*>(w);   // phi in the mode's dtype (buffers sized for fp32)
+    T* phk = reinterpret_cast<T*>(w + phb);
     float* dphq = reinterpret_cast<float*>(w + 2 * phb);
     float* dphk = reinterpret_cast<float*>(w + 3 * phb);
     float* sfw = reinterpret_cast<float*>(w + 4 * phb);
     float* gbw = reinterpret_cast<float*>(w + 4 * phb + stb);
     float* dn = reinterpret_cast<float*>(w + 4 * phb + 2 * stb);
     cudaError_t err;
-    if ((err = fm_launch<T, float>(q, phq, rows, P, st)) != cudaSuccess) return err;
-    if ((err = fm_launch<T, float>(k, phk, rows, P, st)) != cudaSuccess) return err;
+    if ((err = phi_map<T>(q, phq, rows, P, st)) != cudaSuccess) return err;
+    if ((err = phi_map<T>(k, phk, rows, P, st)) != cudaSuccess) return err;
     {
         TraceScope trace_("simt_bwd_rowstats", st);
         k_bwd_rowstats<T><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
@@ -945,11 +957,11 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
     const dim3 sg((F + C - 1) / C, NC, BH);
     {
         TraceScope trace_("simt_chunk_state", st);
-        k_chunk_state<T><<<sg, NT, 0, st>>>(phk, cp<T>(v), kD, sfw, L, F);
+        k_chunk_state<T, T><<<sg, NT, 0, st>>>(phk, cp<T>(v), kD, sfw, L, F);
     }
     {
         TraceScope trace_("simt_chunk_state", st);
-        k_chunk_state<float><<<sg, NT, 0, st>>>(phq, dn, E, gbw, L, F);
+        k_chunk_state<float, T><<<sg, NT, 0, st>>>(phq, dn, E, gbw, L, F);
     }
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     const int FE = F * E;
