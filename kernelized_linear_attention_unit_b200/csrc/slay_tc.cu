@@ -330,42 +330,50 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             constexpr uint32_t idU = idesc_bf16(128, 128, 0, 0);
             const uint64_t dk0 = desc_kmajor(sbase + L.k), dw0 = desc_kmajor(sbase + L.w);
             const uint64_t dph0 = desc_phik(sbase + L.phik), dv = desc_v(sbase + L.v, sbase + L.ones);
-            for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+            // software-pipelined: the projections of tile i are issued before the state
+            // update of tile i-1, whose phi(k) (the other buffer) is complete by then, so the
+            // phi(k) warps never wait for the next tile's projections behind that update
+            for (int tile = sg.t_begin; tile <= sg.t_end; ++tile) {
                 const int b = (tile - sg.t_begin) & 1;
-                {
-                    uint32_t pk = (ph_kf >> b) & 1u;
-                    wt.wait(KF(b), pk);
-                    ph_kf ^= 1u << b;
-                }
-                const uint64_t dk = desc_add(dk0, b * kTileBytes);
-                for (int n = 0; n < NT; ++n, ++n_glob) {
-                    const int slot = n_glob & 1;
-                    uint32_t ph = (ph_wf >> slot) & 1u;
-                    wt.wait(&bar[B_W_FULL0 + slot], ph);
-                    ph_wf ^= (1u << slot);
-                    const int ub = n & 1;
-                    wt.wait(&bar[B_U_EMPTY0 + ub], ub ? ph_ue1 : ph_ue0);
-                    tc_fence_after();
-                    const uint64_t dw = desc_add(dw0, slot * kWStateBytes);
+                if (tile < sg.t_end) {
+                    {
+                        uint32_t pk = (ph_kf >> b) & 1u;
+                        wt.wait(KF(b), pk);
+                        ph_kf ^= 1u << b;
+                    }
+                    const uint64_t dk = desc_add(dk0, b * kTileBytes);
+                    for (int n = 0; n < NT; ++n, ++n_glob) {
+                        const int slot = n_glob & 1;
+                        uint32_t ph = (ph_wf >> slot) & 1u;
+                        wt.wait(&bar[B_W_FULL0 + slot], ph);
+                        ph_wf ^= (1u << slot);
+                        const int ub = n & 1;
+                        wt.wait(&bar[B_U_EMPTY0 + ub], ub ? ph_ue1 : ph_ue0);
+                        tc_fence_after();
+                        const uint64_t dw = desc_add(dw0, slot * kWStateBytes);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(tmem + kColUS + 128 * ub, dk + 2 * kk, dw + 2 * kk, idU, kk > 0 ? 1u : 0u);
-                    umma_commit(&bar[B_U_FULL0 + ub]);
-                    umma_commit(&bar[B_W_EMPTY0 + slot]);
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_bf16(tmem + kColUS + 128 * ub, dk + 2 * kk, dw + 2 * kk, idU, kk > 0 ? 1u : 0u);
+                        umma_commit(&bar[B_U_FULL0 + ub]);
+                        umma_commit(&bar[B_W_EMPTY0 + slot]);
+                    }
+                    umma_commit(KE(b));
                 }
-                umma_commit(KE(b));
-                {
-                    uint32_t pp = (ph_pk >> b) & 1u;
-                    wt.wait(PKF(b), pp);
-                    ph_pk ^= 1u << b;
+                if (tile > sg.t_begin) {   // state update of the previous tile
+                    const int pb = b ^ 1;
+                    {
+                        uint32_t pp = (ph_pk >> pb) & 1u;
+                        wt.wait(PKF(pb), pp);
+                        ph_pk ^= 1u << pb;
+                    }
+                    wt.wait(VF, ph_vf);
+                    tc_fence_after();
+                    for (int h = 0; h < halves; ++h)
+                        issue_state_half(tmem, kColSS, desc_add(dph0, pb * phik_bytes), dv, h,
+                                         tile - 1 == sg.t_begin);
+                    umma_commit(VE);
+                    umma_commit(&TD[pb]);
                 }
-                wt.wait(VF, ph_vf);
-                tc_fence_after();
-                for (int h = 0; h < halves; ++h)
-                    issue_state_half(tmem, kColSS, desc_add(dph0, b * phik_bytes), dv, h,
-                                     tile == sg.t_begin);
-                umma_commit(VE);
-                umma_commit(&TD[b]);
             }
         }
     } else if (kStorePhi && warp == 10) {
