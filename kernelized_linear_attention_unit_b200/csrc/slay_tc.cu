@@ -409,7 +409,7 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 ph_kf ^= 1u << b;
             }
             float inv, l2i;
-            row_scale(sm + L.k + b * kTileBytes + row * 128, inv, l2i);
+            row_scale(sm + L.k + b * kTileBytes + row * 128, row, inv, l2i);
             warp_arrive(KE(b));
             if (li >= 2) {   // phiK buffer b free again (update and store of tile li-2 done)
                 uint32_t pt = (ph_td >> b) & 1u, ps = pt;   // wait() flips its argument
@@ -736,7 +736,7 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
                 wt.wait(&bar[B_QK_FULL], ph_qkf);
                 float inv, l2i;
-                row_scale(sm + (grp ? L.k : L.q) + row * 128, inv, l2i);
+                row_scale(sm + (grp ? L.k : L.q) + row * 128, row, inv, l2i);
                 warp_arrive(&bar[B_QK_EMPTY]);
                 for (int t = 0; t < NT; ++t) {
                     const int node = (t * kSlice) / kp.m;
@@ -1158,7 +1158,7 @@ k_tc_causal_out_pk(const __grid_constant__ CUtensorMap tmq, const __grid_constan
                 wt.wait(QF(qb), ph);
                 ph_qf ^= 1u << qb;
                 float inv, l2i;
-                row_scale(sm + L.q + qb * kTileBytes + row * 128, inv, l2i);
+                row_scale(sm + L.q + qb * kTileBytes + row * 128, row, inv, l2i);
                 warp_arrive(QE(qb));
                 for (int t = 0; t < NT; ++t) {
                     const int node = (t * kSlice) / kp.m;
@@ -1474,7 +1474,7 @@ k_tc_bidir_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             wt.wait(QF(qb), ph);
             ph_qf ^= 1u << qb;
             float inv, l2i;
-            row_scale(sm + L.q + qb * kTileBytes + row * 128, inv, l2i);
+            row_scale(sm + L.q + qb * kTileBytes + row * 128, row, inv, l2i);
             warp_arrive(QE(qb));
             for (int t = 0; t < NT; ++t) {
                 const int node = (t * kSlice) / kp.m;

@@ -49,15 +49,19 @@ __device__ __forceinline__ void drain_after_failure(bool ok)
     }
 }
 
-// Sum of squares of one 64-element bf16 row (128 bytes; order does not matter, so the
-// swizzle is irrelevant) -> (1/|x|, 2 log2(1/|x|)) with the 1e-12 norm guard.
-__device__ __forceinline__ void row_scale(const unsigned char* row, float& inv, float& l2inv2)
+// Sum of squares of one 64-element bf16 row (128 bytes) -> (1/|x|, 2 log2(1/|x|)) with the
+// 1e-12 norm guard.  The order of the elements does not matter, so the row's 16-byte chunks
+// are read in the order of the 128-byte swizzle (chunk c ^ (row & 7) first): the lanes of
+// a warp, one row each, then hit distinct banks.
+__device__ __forceinline__ void row_scale(const unsigned char* row_ptr, uint32_t row, float& inv,
+                                          float& l2inv2)
 {
-    const uint4* p = reinterpret_cast<const uint4*>(row);
+    const uint4* p = reinterpret_cast<const uint4*>(row_ptr);
+    const uint32_t rot = row & 7u;
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // independent partial sums: short FMA chains
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-        const uint4 w = p[c];
+        const uint4 w = p[c ^ rot];
         const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {

@@ -8,16 +8,19 @@
 //
 // The map reads 128 bytes and writes 2F bytes per row, so it is bound by HBM bandwidth;
 // the tensor cores only take the projections off the CUDA cores.  Persistent kernel, one
-// CTA per SM, 128-row tiles dealt round-robin:
-//   warp 0      TMA: the packed projection operand once (resident), then row tiles into a
-//               ring of 4 (F <= 256) or 2 buffers
-//   warp 1      MMA: per tile and 64-feature group, U = X W_g^T with N = 128 (64 omega and
-//               64 anchor columns), four buffers in tensor memory (4 x 128 columns)
-//   warps 2-17  epilogue, four per SM sub-partition: warp w serves TMEM lanes 32*(w%4)
-//               and one 32-feature sub-slice of every other group; it writes its 32 x 32 block of
-//               phi to its own swizzled staging box and stores it by TMA (two boxes per
-//               warp, so a store overlaps the next group; no CTA-wide barrier)
-//   warp 18     the rows' norm scales, up to a ring of X tiles ahead of the epilogue
+// CTA per SM holding the packed projection operand W (resident) and two independent teams
+// of eight warps.  Each team owns 256 tensor-memory columns (two N = 128 buffers) and its
+// own ring of row tiles, and takes 128-row tiles round-robin.  Warp w of a team serves the
+// tensor-memory lanes 32 (w % 4) .. +31 (rows of the tile) and the 32-feature half w / 4 of
+// every 64-feature group.  Per tile and group g:
+//   - each warp waits for the projections U = X W_g^T of group g (an MMA issued two groups
+//     earlier by the team's first thread), reads its 32 rows x 64 columns into registers
+//     and signals the buffer's release barrier; once all eight warps have, the team's first
+//     warp issues the next MMA into that buffer;
+//   - each lane maps its row's 32 features and writes them into its warp's swizzled staging
+//     box, stored by TMA (32 rows x 32 features per box).
+// Each thread computes its own row's norm from the tile in shared memory.  Four warps per
+// SM sub-partition hide one another's latencies; the two teams share nothing but W.
 // Every wait is bounded; a timeout sets the library's feature-map status word.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -25,6 +28,7 @@
 
 #include <cstdint>
 
+#include "slay_exp2_poly.h"
 #include "slay_tc.h"
 #include "slay_tc_common.cuh"
 #include "slay_tc_ptx.cuh"
@@ -39,42 +43,40 @@ constexpr int kRows = 128;                     // rows per tile (MMA M)
 constexpr int kBoxBytes = kRows * 128;         // [128 rows][64 bf16] swizzled X tile = 16 KiB
 constexpr int kSubBytes = 64 * 128;            // packed operand of 32 features = 8 KiB
 constexpr int kGroupBytes = 2 * kSubBytes;     // 64 features (N = 128) = 16 KiB
-constexpr int kUBufs = 4;                      // projection buffers of 128 TMEM columns
-constexpr int kEpiWarps = 16;                  // 4 per SM sub-partition
-constexpr int kNormWarp = 2 + kEpiWarps;       // row-norm scales, ahead of the epilogue
-constexpr int kFmThreads = 32 * (3 + kEpiWarps);
-constexpr int kWarpBoxBytes = 32 * 64;         // one warp's [32 rows][32 bf16] output box
+constexpr int kTeams = 2;                      // independent teams of 8 warps per CTA
+constexpr int kTeamThreads = 256;
+constexpr int kIssuerWarp = 0;                 // MMA and TMA issue for both teams
+constexpr int kComputeWarps = kTeams * kTeamThreads / 32;
+constexpr int kFmThreads = kTeamThreads * kTeams + 32;
+constexpr int kStageBytes = 32 * 64;           // one warp's [32 rows][32 bf16] output box
 constexpr int kNumSMs = 148;
+constexpr int kMaxXBufs = 4;
 
 __device__ int g_fmap_status;                  // set to 1 by a kernel whose wait ran out
 
-enum { FB_W = 0, FB_XF = 1, FB_XE = 5, FB_RS = 9, FB_UF = 13, FB_UE = 17, FB_NUM = 21 };
+// barriers: W, then per team kMaxXBufs X-full, two U-full (MMA commit) and two U-empty
+// (one arrival per warp of the team)
+enum { FB_W = 0, FB_TEAM = 1, FB_XF = 0, FB_UF = kMaxXBufs, FB_UE = kMaxXBufs + 2,
+       FB_PER_TEAM = kMaxXBufs + 4, FB_NUM = 1 + kTeams * FB_PER_TEAM };
 
 struct FmLayout {
-    uint32_t w, x, rs, o, bar, tmem, total;
+    uint32_t w, x, o, bar, tmem, total;
     int xbufs, obufs;
 };
 
 __host__ __device__ inline FmLayout fm_layout(int F)
 {
     FmLayout l;
-    l.xbufs = F <= 256 ? 4 : 2;
-    l.obufs = F <= 256 ? 2 : 1;
-    l.w = 0;                                   // F/32 packed sub-slices, resident
+    l.xbufs = F <= 128 ? 4 : F <= 256 ? 3 : 2;   // X tiles in flight per team
+    l.obufs = F <= 384 ? 2 : 1;                  // staging boxes per warp
+    l.w = 0;                                     // F/32 packed sub-slices, resident
     l.x = (F / 32) * kSubBytes;
-    l.rs = l.x + l.xbufs * kBoxBytes;          // per X slot: (1/|x|, 2 log2(1/|x|)) per row
-    l.o = l.rs + l.xbufs * kRows * 8;          // epilogue warps x obufs staging boxes of 2 KiB
-    l.bar = l.o + kEpiWarps * l.obufs * kWarpBoxBytes;
+    l.o = l.x + kTeams * l.xbufs * kBoxBytes;
+    l.bar = l.o + kComputeWarps * l.obufs * kStageBytes;
     l.tmem = l.bar + FB_NUM * 8;
     l.total = l.tmem + 16;
     return l;
 }
-
-struct FmParams {
-    int F, m, ntiles;
-    float a2[kMaxR];
-    float b2[kMaxR];
-};
 
 // 64-byte swizzle of a [rows][64 B] box: 16-byte chunk c of row r sits at chunk
 // c ^ ((r >> 1) & 3), the pattern TMA applies for CU_TENSOR_MAP_SWIZZLE_64B.
@@ -82,6 +84,44 @@ __device__ __forceinline__ uint32_t sw64_off(uint32_t row, uint32_t chunk)
 {
     return row * 64u + ((chunk ^ ((row >> 1) & 3u)) << 4);
 }
+
+// Exponentials per pair of features taken by the polynomial below instead of the
+// special-function unit: 0 (none), 1 (one of every two pairs' second element) or 2 (every
+// pair's second element).  The special-function unit also does no conversions here: its
+// throughput is what bounds this kernel otherwise.
+#ifndef SLAY_FM_POLY
+#define SLAY_FM_POLY 1
+#endif
+
+// 2^x on the FMA pipe: j = round(x) by adding 1.5 * 2^23 (the sum's low mantissa bits hold
+// j), f = x - j in [-1/2, 1/2], 2^f from the degree-3 minimax polynomial of
+// slay_exp2_poly.h, and 2^j applied by adding j to the exponent field (the sum's bit
+// pattern times 2^23 is j << 23 modulo 2^32).  x is clamped to [-125, 126] so the exponent
+// field stays in range; the relative error is the polynomial's, below 1e-4.
+__device__ __forceinline__ float ex2_poly(float x)
+{
+    x = fminf(fmaxf(x, -125.0f), 126.0f);
+    const float t = __fadd_rn(x, 12582912.0f);
+    const float f = __fsub_rn(x, __fsub_rn(t, 12582912.0f));
+    float p = fmaf(SLAY_EXP2_C3, f, SLAY_EXP2_C2);
+    p = fmaf(p, f, SLAY_EXP2_C1);
+    p = fmaf(p, f, SLAY_EXP2_C0);
+    return __uint_as_float(__float_as_uint(t) * 8388608u + __float_as_uint(p));
+}
+
+// Two non-negative floats to a bf16 pair (lo in the low half), rounded to nearest with
+// ties away from zero: add half an ulp of bf16 to the bit pattern and keep the high halves.
+// Differs from round-to-nearest-even only on exact ties; no special-function-unit work.
+__device__ __forceinline__ uint32_t pack_bf16_ties_up(float lo, float hi)
+{
+    return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
+}
+
+struct FmParams {
+    int F, ntiles;
+    float a2[16];   // per 32-feature sub-slice (F <= 512): the scales of its node
+    float b2[16];
+};
 
 __global__ void __launch_bounds__(kFmThreads, 1)
 k_tc_feature_map(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
@@ -94,19 +134,21 @@ k_tc_feature_map(const __grid_constant__ CUtensorMap tmx, const __grid_constant_
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L.tmem);
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int ngroups = fp.F / 64;
+    // compute warp cw = warp - 1: team cw / 8; a warp reaches the TMEM lanes 32 (warp % 4)..,
+    // and the two warps of a team on the same lanes take the two 32-feature halves
+    const int cw = warp - 1, team = cw >> 3, tw = cw & 7;
+    const int q = warp & 3, half = tw >> 2;
+    const int ng = fp.F / 64;                    // 64-feature groups (>= 2)
     const int xbufs = L.xbufs;
 
-    if (warp == 1) {
+    if (warp == 0) {
         tmem_alloc(tslot, 512);
         tmem_relinquish();
     }
     if (tid == 0) {
         for (int i = 0; i < FB_NUM; ++i) mbar_init(&bar[i], 1);
-        for (int s = 0; s < 4; ++s) {
-            mbar_init(&bar[FB_XE + s], 2 + kEpiWarps);
-        }
-        for (int b = 0; b < kUBufs; ++b) mbar_init(&bar[FB_UE + b], kEpiWarps / 2);
+        for (int t = 0; t < kTeams; ++t)
+            for (int b = 0; b < 2; ++b) mbar_init(&bar[FB_TEAM + t * FB_PER_TEAM + FB_UE + b], 8);
         mbar_fence_init();
         tma_prefetch_desc(&tmx);
         tma_prefetch_desc(&tmw);
@@ -115,154 +157,194 @@ k_tc_feature_map(const __grid_constant__ CUtensorMap tmx, const __grid_constant_
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tslot;
+    const uint32_t tmem0 = *tslot;
     Waiter wt;
 
-    if (warp == 0) {
+    // tiles of team t: k-th = (k * gridDim.x + blockIdx.x) * kTeams + t
+    const int stride = gridDim.x * kTeams;
+    auto team_tiles = [&](int t) {
+        const int first = blockIdx.x * kTeams + t;
+        return first < fp.ntiles ? (fp.ntiles - 1 - first) / stride + 1 : 0;
+    };
+
+    if (warp == kIssuerWarp) {
+        // One thread issues for both teams.  Per team: job j = k * ng + g (tile k, group g)
+        // goes into buffer j & 1 once every warp of the team has read job j - 2 from it
+        // (UE) and tile k is in shared memory (XF); X slot k % xbufs is refilled with tile
+        // k + xbufs once the team has read the last group of tile k.  Polls never block, so
+        // one team's wait does not hold up the other; no progress for longer than the wait
+        // bound ends the loop with an error.
         if (lane == 0) {
-            mbar_arrive_expect_tx(&bar[FB_W], (fp.F / 32) * kSubBytes);
-            for (int n = 0; n < fp.F / 32; ++n)
-                tma_load_2d(sm + L.w + n * kSubBytes, &tmw, &bar[FB_W], 0, n * 64);
-            uint32_t ph_xe = 0;   // one phase bit per ring slot
-            int it = 0;
-            for (int tile = blockIdx.x; tile < fp.ntiles; tile += gridDim.x, ++it) {
-                const int s = it % xbufs;
-                if (it >= xbufs) {
-                    uint32_t ph = (ph_xe >> s) & 1u;
-                    wt.wait(&bar[FB_XE + s], ph);
-                    ph_xe ^= 1u << s;
-                }
-                mbar_arrive_expect_tx(&bar[FB_XF + s], kBoxBytes);
-                tma_load_2d(sm + L.x + s * kBoxBytes, &tmx, &bar[FB_XF + s], 0, tile * kRows);
-            }
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            uint32_t ph_w = 0, ph_xf = 0;
-            wt.wait(&bar[FB_W], ph_w);
-            constexpr uint32_t idU = idesc_bf16(128, 128, 0, 0);
-            // descriptors built once, stepped by adds (see the causal kernels)
-            const uint64_t dx0 = sdesc(sbase + L.x, 16, 1024, kLayoutSW128);
             const uint64_t dw0 = sdesc(sbase + L.w, 16, 1024, kLayoutSW128);
-            int it = 0, j = 0;
-            for (int tile = blockIdx.x; tile < fp.ntiles; tile += gridDim.x, ++it) {
-                const int s = it % xbufs;
-                uint32_t ph = (ph_xf >> s) & 1u;
-                wt.wait(&bar[FB_XF + s], ph);
-                ph_xf ^= 1u << s;
-                const uint64_t dx = dx0 + ((s * kBoxBytes) >> 4);
-                for (int g = 0; g < ngroups; ++g, ++j) {
-                    const int b = j % kUBufs;
-                    if (j >= kUBufs) {
-                        uint32_t pu = static_cast<uint32_t>((j / kUBufs - 1) & 1);
-                        wt.wait(&bar[FB_UE + b], pu);
+            constexpr uint32_t idU = idesc_bf16(128, 128, 0, 0);
+            // per team: next job jn = (tile kn, group gn), X slot of tile kn and its phase
+            int nt[kTeams], jn[kTeams], kn[kTeams], gn[kTeams], sn[kTeams], stage[kTeams];
+            uint32_t pn[kTeams];
+            uint64_t dx0[kTeams];
+            for (int t = 0; t < kTeams; ++t) {
+                nt[t] = team_tiles(t);
+                jn[t] = kn[t] = gn[t] = sn[t] = 0;
+                pn[t] = 0;
+                stage[t] = 1;                    // jobs 0 and 1 need no release
+                dx0[t] = sdesc(sbase + L.x + t * xbufs * kBoxBytes, 16, 1024, kLayoutSW128);
+            }
+            auto load_x = [&](int t, int k, int slot) {
+                uint64_t* xf = bar + FB_TEAM + t * FB_PER_TEAM + FB_XF + slot;
+                mbar_arrive_expect_tx(xf, kBoxBytes);
+                tma_load_2d(sm + L.x + (t * xbufs + slot) * kBoxBytes, &tmx, xf, 0,
+                            ((k * gridDim.x + blockIdx.x) * kTeams + t) * kRows);
+            };
+            if (nt[0] > 0) {
+                mbar_arrive_expect_tx(&bar[FB_W], (fp.F / 32) * kSubBytes);
+                for (int n = 0; n < fp.F / 32; ++n)
+                    tma_load_2d(sm + L.w + n * kSubBytes, &tmw, &bar[FB_W], 0, n * 64);
+            }
+            for (int t = 0; t < kTeams; ++t)
+                for (int k = 0; k < xbufs && k < nt[t]; ++k) load_x(t, k, k);
+            if (nt[0] > 0) {
+                uint32_t ph = 0;
+                wt.wait(&bar[FB_W], ph);
+            }
+            uint64_t t0 = global_timer_ns();
+            uint32_t polls = 0;
+            bool moved = false;
+            while (wt.ok) {
+                bool left = false;
+#pragma unroll
+                for (int t = 0; t < kTeams; ++t) {
+                    if (kn[t] >= nt[t]) continue;
+                    left = true;
+                    uint64_t* tb = bar + FB_TEAM + t * FB_PER_TEAM;
+                    const int j = jn[t];
+                    if (stage[t] == 0) {         // buffer j & 1 released by job j - 2?
+                        const int jp = j - 2;
+                        if (!mbar_test_wait(smem_u32(&tb[FB_UE + (jp & 1)]), (jp >> 1) & 1))
+                            continue;
+                        // job j - 2 was the last group of tile kn - 1 (gn == 1 for any
+                        // ng >= 2): its X slot takes tile kn - 1 + xbufs
+                        if (gn[t] == 1 && kn[t] - 1 + xbufs < nt[t])
+                            load_x(t, kn[t] - 1 + xbufs, sn[t] == 0 ? xbufs - 1 : sn[t] - 1);
+                        stage[t] = 1;
                     }
+                    if (gn[t] == 0 && !mbar_test_wait(smem_u32(&tb[FB_XF + sn[t]]), pn[t]))
+                        continue;                // tile kn not landed yet
                     tc_fence_after();
-                    const uint64_t dw = dw0 + ((g * kGroupBytes) >> 4);
+                    const uint64_t dx = dx0[t] + ((sn[t] * kBoxBytes) >> 4);
+                    const uint64_t dw = dw0 + ((gn[t] * kGroupBytes) >> 4);
+                    const uint32_t d = tmem0 + 256u * t + 128u * (j & 1);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(tmem + 128 * b, dx + 2 * kk, dw + 2 * kk, idU, kk > 0 ? 1u : 0u);
-                    umma_commit(&bar[FB_UF + b]);
+                        umma_bf16(d, dx + 2 * kk, dw + 2 * kk, idU, kk > 0 ? 1u : 0u);
+                    umma_commit(&tb[FB_UF + (j & 1)]);
+                    jn[t] = j + 1;
+                    stage[t] = j + 1 >= 2 ? 0 : 1;
+                    if (++gn[t] == ng) {
+                        gn[t] = 0;
+                        ++kn[t];
+                        if (++sn[t] == xbufs) {
+                            sn[t] = 0;
+                            pn[t] ^= 1u;
+                        }
+                    }
+                    moved = true;
                 }
-                umma_commit(&bar[FB_XE + s]);
+                if (!left) break;
+                if ((++polls & 255u) == 0) {
+                    const uint64_t now = global_timer_ns();
+                    if (moved) {
+                        t0 = now;
+                        moved = false;
+                    } else if (now - t0 > kWaitNs) {
+                        wt.ok = false;
+                        wt.where = 0x20000u;
+                    }
+                }
             }
         }
-    } else if (warp == kNormWarp) {
-        // (1/|x|, 2 log2(1/|x|)) of the 128 rows of each X tile, four rows per lane
-        uint32_t ph_xf = 0;
-        int it = 0;
-        for (int tile = blockIdx.x; tile < fp.ntiles; tile += gridDim.x, ++it) {
-            const int s = it % xbufs;
-            uint32_t ph = (ph_xf >> s) & 1u;
-            wt.wait(&bar[FB_XF + s], ph);
-            ph_xf ^= 1u << s;
-            float2* rs = reinterpret_cast<float2*>(sm + L.rs + s * kRows * 8);
+        __syncwarp();
+    }
+    else {   // the two teams' warps
+    uint64_t* tb = bar + FB_TEAM + team * FB_PER_TEAM;
+    uint64_t* XF = tb + FB_XF;
+    uint64_t* UF = tb + FB_UF;
+    uint64_t* UE = tb + FB_UE;
+    const unsigned char* xs = sm + L.x + team * xbufs * kBoxBytes;
+    const int first = blockIdx.x * kTeams + team;
+    const int nt = team_tiles(team);
+    const uint32_t row = 32u * q + lane;
+    const uint32_t tcol = tmem0 + 256u * team + ((32u * q) << 16) + 64u * half;
+    const int obufs = L.obufs;
+    const uint32_t obox = sbase + L.o + cw * obufs * kStageBytes;
+    int js = 0;                                  // staging boxes used by this warp
+    int s = 0;                                   // X slot of tile k and its phase
+    uint32_t xph = 0;
+    for (int k = 0; k < nt; ++k) {
+        {
+            uint32_t ph = xph;
+            wt.wait(&XF[s], ph);
+        }
+        float inv, l2i;
+        row_scale(xs + s * kBoxBytes + row * 128, row, inv, l2i);
+        const int row0 = (first + k * stride) * kRows + 32 * q;
+        for (int g = 0; g < ng; ++g, ++js) {
+            const int j = k * ng + g;
+            const uint32_t ph = static_cast<uint32_t>((j >> 1) & 1);
+            {
+                uint32_t p = ph;
+                wt.wait(&UF[j & 1], p);
+            }
+            tc_fence_after();
+            uint32_t ur[32], pr[32];
+            tmem_ld32(tcol + 128u * (j & 1), ur);
+            tmem_ld32(tcol + 128u * (j & 1) + 32, pr);
+            tmem_wait_ld();
+            reg_fence(ur);
+            reg_fence(pr);
+            tc_fence_before();
+            warp_arrive(&UE[j & 1]);             // this warp's rows of buffer j & 1 are read
+            const float a = fp.a2[2 * g + half] * inv, bb = fp.b2[2 * g + half] + l2i;
+            uint32_t pk[16];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int row = 32 * r + lane;
-                float inv, l2i;
-                row_scale(sm + L.x + s * kBoxBytes + row * 128, inv, l2i);
-                rs[row] = make_float2(inv, l2i);
+            for (int c = 0; c < 32; c += 2) {
+                const float x0 = __uint_as_float(pr[c]), x1 = __uint_as_float(pr[c + 1]);
+                const float e0 = ex2(fmaf(a, __uint_as_float(ur[c]), bb));
+                const float y1 = fmaf(a, __uint_as_float(ur[c + 1]), bb);
+                const bool poly = SLAY_FM_POLY == 2 || (SLAY_FM_POLY == 1 && (c & 2));
+                const float e1 = poly ? ex2_poly(y1) : ex2(y1);
+                pk[c >> 1] = pack_bf16_ties_up(e0 * x0 * x0, e1 * x1 * x1);
+            }
+            // the box was stored obufs groups ago: its reads must be done before it is rewritten
+            if (lane == 0) {
+                if (obufs == 2)
+                    bulk_wait_read<1>();
+                else
+                    bulk_wait_read<0>();
             }
             __syncwarp();
+            const uint32_t box = obox + (js & (obufs - 1)) * kStageBytes;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                st_shared_v4(box + sw64_off(lane, c), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
+                             pk[4 * c + 3]);
+            fence_async_smem();
+            __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&bar[FB_RS + s]);
-                mbar_arrive(&bar[FB_XE + s]);
+                tma_store_2d(&tmo, sm + (box - sbase), 64 * g + 32 * half, row0);
+                bulk_commit_group();
             }
         }
-    } else {
-        // epilogue warp ew: TMEM lanes 32*(warp%4) (rows of the tile); warps with pair = 0
-        // take the even 64-feature groups, pair = 1 the odd ones (the two pairs of a
-        // sub-partition work on different buffers, out of step); sub-slice `sub` of each
-        // group (u at columns 64 sub, p at 64 sub + 32 of the group's buffer)
-        const int ew = warp - 2, q = warp & 3, e = ew >> 2, pair = e >> 1, sub = e & 1;
-        const uint32_t row = 32u * q + lane;
-        const uint32_t trow = tmem + ((32u * q) << 16);
-        const int obufs = L.obufs;
-        uint32_t ph_rs = 0;
-        int it = 0, jw = 0;
-        for (int tile = blockIdx.x; tile < fp.ntiles; tile += gridDim.x, ++it) {
-            const int s = it % xbufs;
-            uint32_t ph = (ph_rs >> s) & 1u;
-            wt.wait(&bar[FB_RS + s], ph);
-            ph_rs ^= 1u << s;
-            const float2 v = reinterpret_cast<const float2*>(sm + L.rs + s * kRows * 8)[row];
-            const float inv = v.x, l2i = v.y;
-            warp_arrive(&bar[FB_XE + s]);
-            for (int g = pair; g < ngroups; g += 2, ++jw) {
-                const int j = it * ngroups + g;
-                const int b = j % kUBufs;
-                uint32_t pu = static_cast<uint32_t>((j / kUBufs) & 1);
-                wt.wait(&bar[FB_UF + b], pu);
-                tc_fence_after();
-                uint32_t ur[32], pr[32];
-                const uint32_t c0 = trow + 128 * b + 64 * sub;
-                tmem_ld32(c0, ur);
-                tmem_ld32(c0 + 32, pr);
-                tmem_wait_ld();
-                reg_fence(ur);
-                reg_fence(pr);
-                tc_fence_before();
-                warp_arrive(&bar[FB_UE + b]);
-                const int f0 = 64 * g + 32 * sub;
-                const int node = f0 / fp.m;
-                const float a = fp.a2[node] * inv, bb = fp.b2[node] + l2i;
-                uint32_t pk[16];
-#pragma unroll
-                for (int c = 0; c < 32; c += 2) {
-                    const float x0 = __uint_as_float(pr[c]), x1 = __uint_as_float(pr[c + 1]);
-                    pk[c >> 1] = pack_bf16(ex2(fmaf(a, __uint_as_float(ur[c]), bb)) * x0 * x0,
-                                           ex2(fmaf(a, __uint_as_float(ur[c + 1]), bb)) * x1 * x1);
-                }
-                // this warp's staging box was stored obufs groups ago: its reads must be done
-                if (lane == 0) {
-                    if (obufs == 2)
-                        bulk_wait_read<1>();
-                    else
-                        bulk_wait_read<0>();
-                }
-                __syncwarp();
-                const uint32_t box = sbase + L.o + (ew * obufs + jw % obufs) * kWarpBoxBytes;
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    st_shared_v4(box + sw64_off(lane, c), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
-                                 pk[4 * c + 3]);
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(&tmo, sm + L.o + (ew * obufs + jw % obufs) * kWarpBoxBytes, f0,
-                                 tile * kRows + 32 * q);
-                    bulk_commit_group();
-                }
-            }
+        if (++s == xbufs) {
+            s = 0;
+            xph ^= 1u;
         }
-        if (lane == 0) bulk_wait<0>();
+    }
+    if (lane == 0) bulk_wait<0>();
     }
     wt.report(&g_fmap_status);
     drain_after_failure(wt.ok);
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) tmem_dealloc(tmem, 512);
+    if (warp == 0) tmem_dealloc(tmem0, 512);
 }
 
 // [rows][cols] bf16, row stride cols*2 bytes, boxes of box_cols x box_rows; out-of-range
@@ -309,11 +391,11 @@ cudaError_t tc_feature_map(const void* x, void* phi, int64_t n, const Params& P,
         return cudaErrorInvalidValue;
     FmParams fp;
     fp.F = F;
-    fp.m = P.m;
     fp.ntiles = static_cast<int>((n + kRows - 1) / kRows);
-    for (int r = 0; r < kMaxR; ++r) {
-        fp.a2[r] = P.a2[r];
-        fp.b2[r] = P.b2[r];
+    for (int sub = 0; sub < 16; ++sub) {
+        const int node = sub < F / 32 ? sub * 32 / P.m : 0;
+        fp.a2[sub] = P.a2[node];
+        fp.b2[sub] = P.b2[node];
     }
     void* status = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&status, g_fmap_status);
@@ -323,7 +405,8 @@ cudaError_t tc_feature_map(const void* x, void* phi, int64_t n, const Params& P,
     e = cudaFuncSetAttribute(k_tc_feature_map, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    const int grid = fp.ntiles < kNumSMs ? fp.ntiles : kNumSMs;
+    const int pairs = (fp.ntiles + kTeams - 1) / kTeams;
+    const int grid = pairs < kNumSMs ? pairs : kNumSMs;
     TraceScope trace_("tc_feature_map", st);
     k_tc_feature_map<<<grid, kFmThreads, smem, st>>>(mx, mw, mo, fp);
     return cudaGetLastError();
