@@ -45,9 +45,8 @@ constexpr int kSubBytes = 64 * 128;            // packed operand of 32 features 
 constexpr int kGroupBytes = 2 * kSubBytes;     // 64 features (N = 128) = 16 KiB
 constexpr int kTeams = 2;                      // independent teams of 8 warps per CTA
 constexpr int kTeamThreads = 256;
-constexpr int kIssuerWarp = 0;                 // MMA and TMA issue for both teams
-constexpr int kComputeWarps = kTeams * kTeamThreads / 32;
-constexpr int kFmThreads = kTeamThreads * kTeams + 32;
+constexpr int kComputeWarps = kTeams * kTeamThreads / 32;   // warps kTeams.. of the CTA
+constexpr int kFmThreads = kTeamThreads * kTeams + 32 * kTeams;   // + one issuing warp per team
 constexpr int kStageBytes = 32 * 64;           // one warp's [32 rows][32 bf16] output box
 constexpr int kNumSMs = 148;
 constexpr int kMaxXBufs = 4;
@@ -87,8 +86,9 @@ __device__ __forceinline__ uint32_t sw64_off(uint32_t row, uint32_t chunk)
 
 // Exponentials per pair of features taken by the polynomial below instead of the
 // special-function unit: 0 (none), 1 (one of every two pairs' second element) or 2 (every
-// pair's second element).  The special-function unit also does no conversions here: its
-// throughput is what bounds this kernel otherwise.
+// pair's second element).  The special-function unit shares its issue queue with the
+// shared-memory and barrier operations that pace the pipeline, so a quarter of the
+// exponentials go to the FMA pipe (measured best: it costs about a dozen instructions each).
 #ifndef SLAY_FM_POLY
 #define SLAY_FM_POLY 1
 #endif
@@ -109,14 +109,6 @@ __device__ __forceinline__ float ex2_poly(float x)
     return __uint_as_float(__float_as_uint(t) * 8388608u + __float_as_uint(p));
 }
 
-// Two non-negative floats to a bf16 pair (lo in the low half), rounded to nearest with
-// ties away from zero: add half an ulp of bf16 to the bit pattern and keep the high halves.
-// Differs from round-to-nearest-even only on exact ties; no special-function-unit work.
-__device__ __forceinline__ uint32_t pack_bf16_ties_up(float lo, float hi)
-{
-    return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
-}
-
 struct FmParams {
     int F, ntiles;
     float a2[16];   // per 32-feature sub-slice (F <= 512): the scales of its node
@@ -134,9 +126,10 @@ k_tc_feature_map(const __grid_constant__ CUtensorMap tmx, const __grid_constant_
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L.tmem);
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // compute warp cw = warp - 1: team cw / 8; a warp reaches the TMEM lanes 32 (warp % 4)..,
-    // and the two warps of a team on the same lanes take the two 32-feature halves
-    const int cw = warp - 1, team = cw >> 3, tw = cw & 7;
+    // warp t < kTeams issues for team t; compute warp cw = warp - kTeams belongs to team
+    // cw / 8; a warp reaches the TMEM lanes 32 (warp % 4).., and the two warps of a team on
+    // the same lanes take the two 32-feature halves
+    const int cw = warp - kTeams, team = cw >> 3, tw = cw & 7;
     const int q = warp & 3, half = tw >> 2;
     const int ng = fp.F / 64;                    // 64-feature groups (>= 2)
     const int xbufs = L.xbufs;
@@ -167,97 +160,62 @@ k_tc_feature_map(const __grid_constant__ CUtensorMap tmx, const __grid_constant_
         return first < fp.ntiles ? (fp.ntiles - 1 - first) / stride + 1 : 0;
     };
 
-    if (warp == kIssuerWarp) {
-        // One thread issues for both teams.  Per team: job j = k * ng + g (tile k, group g)
-        // goes into buffer j & 1 once every warp of the team has read job j - 2 from it
-        // (UE) and tile k is in shared memory (XF); X slot k % xbufs is refilled with tile
-        // k + xbufs once the team has read the last group of tile k.  Polls never block, so
-        // one team's wait does not hold up the other; no progress for longer than the wait
-        // bound ends the loop with an error.
+    if (warp < kTeams) {
+        // Warp t issues for team t.  Job j = (tile k, group g) goes into buffer j & 1 once
+        // every warp of the team has read job j - 2 from it (UE) and tile k is in shared
+        // memory (XF); X slot k % xbufs takes tile k + xbufs once the team has read the last
+        // group of tile k.  One issuer per team keeps each team's chain short: an issuer
+        // waits only on its own team.
+        const int t = warp;
         if (lane == 0) {
+            const int nt = team_tiles(t);
+            uint64_t* tb = bar + FB_TEAM + t * FB_PER_TEAM;
             const uint64_t dw0 = sdesc(sbase + L.w, 16, 1024, kLayoutSW128);
+            const uint64_t dx0 = sdesc(sbase + L.x + t * xbufs * kBoxBytes, 16, 1024, kLayoutSW128);
             constexpr uint32_t idU = idesc_bf16(128, 128, 0, 0);
-            // per team: next job jn = (tile kn, group gn), X slot of tile kn and its phase
-            int nt[kTeams], jn[kTeams], kn[kTeams], gn[kTeams], sn[kTeams], stage[kTeams];
-            uint32_t pn[kTeams];
-            uint64_t dx0[kTeams];
-            for (int t = 0; t < kTeams; ++t) {
-                nt[t] = team_tiles(t);
-                jn[t] = kn[t] = gn[t] = sn[t] = 0;
-                pn[t] = 0;
-                stage[t] = 1;                    // jobs 0 and 1 need no release
-                dx0[t] = sdesc(sbase + L.x + t * xbufs * kBoxBytes, 16, 1024, kLayoutSW128);
-            }
-            auto load_x = [&](int t, int k, int slot) {
-                uint64_t* xf = bar + FB_TEAM + t * FB_PER_TEAM + FB_XF + slot;
-                mbar_arrive_expect_tx(xf, kBoxBytes);
-                tma_load_2d(sm + L.x + (t * xbufs + slot) * kBoxBytes, &tmx, xf, 0,
+            auto load_x = [&](int k, int slot) {
+                mbar_arrive_expect_tx(&tb[FB_XF + slot], kBoxBytes);
+                tma_load_2d(sm + L.x + (t * xbufs + slot) * kBoxBytes, &tmx, &tb[FB_XF + slot], 0,
                             ((k * gridDim.x + blockIdx.x) * kTeams + t) * kRows);
             };
-            if (nt[0] > 0) {
+            if (t == 0 && nt > 0) {
                 mbar_arrive_expect_tx(&bar[FB_W], (fp.F / 32) * kSubBytes);
                 for (int n = 0; n < fp.F / 32; ++n)
                     tma_load_2d(sm + L.w + n * kSubBytes, &tmw, &bar[FB_W], 0, n * 64);
             }
-            for (int t = 0; t < kTeams; ++t)
-                for (int k = 0; k < xbufs && k < nt[t]; ++k) load_x(t, k, k);
-            if (nt[0] > 0) {
+            for (int k = 0; k < xbufs && k < nt; ++k) load_x(k, k);
+            if (nt > 0) {
                 uint32_t ph = 0;
                 wt.wait(&bar[FB_W], ph);
             }
-            uint64_t t0 = global_timer_ns();
-            uint32_t polls = 0;
-            bool moved = false;
-            while (wt.ok) {
-                bool left = false;
-#pragma unroll
-                for (int t = 0; t < kTeams; ++t) {
-                    if (kn[t] >= nt[t]) continue;
-                    left = true;
-                    uint64_t* tb = bar + FB_TEAM + t * FB_PER_TEAM;
-                    const int j = jn[t];
-                    if (stage[t] == 0) {         // buffer j & 1 released by job j - 2?
-                        const int jp = j - 2;
-                        if (!mbar_test_wait(smem_u32(&tb[FB_UE + (jp & 1)]), (jp >> 1) & 1))
-                            continue;
-                        // job j - 2 was the last group of tile kn - 1 (gn == 1 for any
-                        // ng >= 2): its X slot takes tile kn - 1 + xbufs
-                        if (gn[t] == 1 && kn[t] - 1 + xbufs < nt[t])
-                            load_x(t, kn[t] - 1 + xbufs, sn[t] == 0 ? xbufs - 1 : sn[t] - 1);
-                        stage[t] = 1;
+            int j = 0, sn = 0;                   // job, X slot of its tile
+            uint32_t pn = 0;                     // that slot's phase
+            for (int k = 0; k < nt && wt.ok; ++k) {
+                {
+                    uint32_t ph = pn;
+                    wt.wait(&tb[FB_XF + sn], ph);
+                }
+                for (int g = 0; g < ng; ++g, ++j) {
+                    if (j >= 2) {                // buffer j & 1 released by job j - 2
+                        uint32_t ph = static_cast<uint32_t>(((j - 2) >> 1) & 1);
+                        wt.wait(&tb[FB_UE + (j & 1)], ph);
+                        // job j - 2 was the last group of tile k - 1 when g == 1 (ng >= 2):
+                        // its X slot takes tile k - 1 + xbufs
+                        if (g == 1 && k - 1 + xbufs < nt)
+                            load_x(k - 1 + xbufs, sn == 0 ? xbufs - 1 : sn - 1);
                     }
-                    if (gn[t] == 0 && !mbar_test_wait(smem_u32(&tb[FB_XF + sn[t]]), pn[t]))
-                        continue;                // tile kn not landed yet
                     tc_fence_after();
-                    const uint64_t dx = dx0[t] + ((sn[t] * kBoxBytes) >> 4);
-                    const uint64_t dw = dw0 + ((gn[t] * kGroupBytes) >> 4);
+                    const uint64_t dx = dx0 + ((sn * kBoxBytes) >> 4);
+                    const uint64_t dw = dw0 + ((g * kGroupBytes) >> 4);
                     const uint32_t d = tmem0 + 256u * t + 128u * (j & 1);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         umma_bf16(d, dx + 2 * kk, dw + 2 * kk, idU, kk > 0 ? 1u : 0u);
                     umma_commit(&tb[FB_UF + (j & 1)]);
-                    jn[t] = j + 1;
-                    stage[t] = j + 1 >= 2 ? 0 : 1;
-                    if (++gn[t] == ng) {
-                        gn[t] = 0;
-                        ++kn[t];
-                        if (++sn[t] == xbufs) {
-                            sn[t] = 0;
-                            pn[t] ^= 1u;
-                        }
-                    }
-                    moved = true;
                 }
-                if (!left) break;
-                if ((++polls & 255u) == 0) {
-                    const uint64_t now = global_timer_ns();
-                    if (moved) {
-                        t0 = now;
-                        moved = false;
-                    } else if (now - t0 > kWaitNs) {
-                        wt.ok = false;
-                        wt.where = 0x20000u;
-                    }
+                if (++sn == xbufs) {
+                    sn = 0;
+                    pn ^= 1u;
                 }
             }
         }
@@ -311,7 +269,7 @@ k_tc_feature_map(const __grid_constant__ CUtensorMap tmx, const __grid_constant_
                 const float y1 = fmaf(a, __uint_as_float(ur[c + 1]), bb);
                 const bool poly = SLAY_FM_POLY == 2 || (SLAY_FM_POLY == 1 && (c & 2));
                 const float e1 = poly ? ex2_poly(y1) : ex2(y1);
-                pk[c >> 1] = pack_bf16_ties_up(e0 * x0 * x0, e1 * x1 * x1);
+                pk[c >> 1] = pack_bf16(e0 * x0 * x0, e1 * x1 * x1);
             }
             // the box was stored obufs groups ago: its reads must be done before it is rewritten
             if (lane == 0) {
