@@ -136,18 +136,29 @@ __device__ __forceinline__ Seg segment_of(int index, int nseg, int ntiles)
     return s;
 }
 
+constexpr int kMaxSlices = 256 / kSlice;
+
 struct KParams {
-    int L, F, m, nseg, ntiles;
+    int L, F, nseg, ntiles;
     int all_segs;      // state kernel: 1 = every segment (bidirectional), 0 = all but the last
     float eps;
-    float a2[kMaxR];
-    float b2[kMaxR];
+    float a2[kMaxSlices];   // per 64-feature slice (m % 64 == 0): the scales of its node
+    float b2[kMaxSlices];
 };
+
+// v[t] for a slice index t < kMaxSlices, by selects (an indexed parameter array would be
+// copied to local memory)
+__device__ __forceinline__ float slice_val(const float (&v)[kMaxSlices], int t)
+{
+    static_assert(kMaxSlices == 4, "slice_val selects among four");
+    return t < 2 ? (t == 0 ? v[0] : v[1]) : (t == 2 ? v[2] : v[3]);
+}
 
 // phi of one 32-feature sub-slice from registers holding u (32) and p (32) of this row:
 // phi_j = exp2(a u_j + b) p_j^2, a = a2[r]/|x|, b = b2[r] + 2 log2(1/|x|).  Stores the 32
 // bf16 values as chunks [4*half, 4*half+4) of row `row` of the swizzled tile at tile_addr.
 // With zs != nullptr returns sum_j phi_j zs[j] (the inter-tile denominator term).
+template <bool kPoly = false>
 __device__ __forceinline__ float phi_sub_epilogue(const uint32_t (&ur)[32], const uint32_t (&pr)[32],
                                                   float a, float b, uint32_t tile_addr,
                                                   uint32_t row, int half, const float* zs)
@@ -157,8 +168,12 @@ __device__ __forceinline__ float phi_sub_epilogue(const uint32_t (&ur)[32], cons
 #pragma unroll
     for (int j = 0; j < 32; j += 2) {
         const float p0 = __uint_as_float(pr[j]), p1 = __uint_as_float(pr[j + 1]);
+        // with kPoly one exponential in four goes to the FMA pipe: the special-function
+        // unit's queue is shared with the shared-memory and barrier traffic that paces these
+        // kernels (the k side, which has the registers for it)
         const float f0 = ex2(fmaf(a, __uint_as_float(ur[j]), b)) * p0 * p0;
-        const float f1 = ex2(fmaf(a, __uint_as_float(ur[j + 1]), b)) * p1 * p1;
+        const float y1 = fmaf(a, __uint_as_float(ur[j + 1]), b);
+        const float f1 = ((kPoly && (j & 2)) ? ex2_poly(y1) : ex2(y1)) * p1 * p1;
         if (zs) {
             dz = fmaf(f0, zs[j], dz);
             dz = fmaf(f1, zs[j + 1], dz);
@@ -420,8 +435,7 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             for (int n = grp; n < NT; n += 2) {
                 wt.wait(&bar[B_U_FULL0 + grp], ph_uf);
                 tc_fence_after();
-                const int node = (n * kSlice) / kp.m;
-                const float a = kp.a2[node] * inv, bb = kp.b2[node] + l2i;
+                const float a = slice_val(kp.a2, n) * inv, bb = slice_val(kp.b2, n) + l2i;
                 const uint32_t col = kColUS + 128 * grp;
                 uint32_t ua[32], pa[32], ub[32], pb[32];
                 tmem_ld32(trow + col, ua);
@@ -436,8 +450,8 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 tc_fence_before();
                 warp_arrive(&bar[B_U_EMPTY0 + grp]);
                 const uint32_t tile_addr = sbase + L.phik + b * phik_bytes + n * kTileBytes;
-                phi_sub_epilogue(ua, pa, a, bb, tile_addr, row, 0, nullptr);
-                phi_sub_epilogue(ub, pb, a, bb, tile_addr, row, 1, nullptr);
+                phi_sub_epilogue<true>(ua, pa, a, bb, tile_addr, row, 0, nullptr);
+                phi_sub_epilogue<true>(ub, pb, a, bb, tile_addr, row, 1, nullptr);
             }
             fence_async_smem();
             warp_arrive(PKF(b));
@@ -739,8 +753,7 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 row_scale(sm + (grp ? L.k : L.q) + row * 128, row, inv, l2i);
                 warp_arrive(&bar[B_QK_EMPTY]);
                 for (int t = 0; t < NT; ++t) {
-                    const int node = (t * kSlice) / kp.m;
-                    const float a = kp.a2[node] * inv, b = kp.b2[node] + l2i;
+                    const float a = slice_val(kp.a2, t) * inv, b = slice_val(kp.b2, t) + l2i;
                     const int pslot = t & 1;
                     for (int half = 0; half < 2; ++half) {
                         wt.wait(&bar[B_U_FULL0 + grp], ph_uf);
@@ -1161,8 +1174,7 @@ k_tc_causal_out_pk(const __grid_constant__ CUtensorMap tmq, const __grid_constan
                 row_scale(sm + L.q + qb * kTileBytes + row * 128, row, inv, l2i);
                 warp_arrive(QE(qb));
                 for (int t = 0; t < NT; ++t) {
-                    const int node = (t * kSlice) / kp.m;
-                    const float a = kp.a2[node] * inv, b = kp.b2[node] + l2i;
+                    const float a = slice_val(kp.a2, t) * inv, b = slice_val(kp.b2, t) + l2i;
                     const int pslot = t & 1;
                     wt.wait(&bar[B_U_FULL0 + g], ph_uf);
                     tc_fence_after();
@@ -1477,8 +1489,7 @@ k_tc_bidir_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             row_scale(sm + L.q + qb * kTileBytes + row * 128, row, inv, l2i);
             warp_arrive(QE(qb));
             for (int t = 0; t < NT; ++t) {
-                const int node = (t * kSlice) / kp.m;
-                const float a = kp.a2[node] * inv, b = kp.b2[node] + l2i;
+                const float a = slice_val(kp.a2, t) * inv, b = slice_val(kp.b2, t) + l2i;
                 const int pslot = t & 1;
                 wt.wait(&bar[B_U_FULL0 + g], ph_uf);
                 tc_fence_after();
@@ -1695,9 +1706,13 @@ cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, 
                   store_phik ? L : 1, store_phik ? BH : 1))
         return cudaErrorInvalidValue;
     KParams kp;
-    kp.L = L; kp.F = F; kp.m = P.m; kp.nseg = nseg; kp.ntiles = ntiles; kp.eps = eps;
+    kp.L = L; kp.F = F; kp.nseg = nseg; kp.ntiles = ntiles; kp.eps = eps;
     kp.all_segs = (causal && lowmem) ? 0 : 1;
-    for (int r = 0; r < kMaxR; ++r) { kp.a2[r] = P.a2[r]; kp.b2[r] = P.b2[r]; }
+    for (int t = 0; t < kMaxSlices; ++t) {
+        const int node = t < F / kSlice ? t * kSlice / P.m : 0;
+        kp.a2[t] = P.a2[node];
+        kp.b2[t] = P.b2[node];
+    }
     int* err = reinterpret_cast<int*>(w);
     float* wsS = reinterpret_cast<float*>(w + wl.s);
     float* wsZ = reinterpret_cast<float*>(w + wl.z);

@@ -28,7 +28,6 @@
 
 #include <cstdint>
 
-#include "slay_exp2_poly.h"
 #include "slay_tc.h"
 #include "slay_tc_common.cuh"
 #include "slay_tc_ptx.cuh"
@@ -92,22 +91,6 @@ __device__ __forceinline__ uint32_t sw64_off(uint32_t row, uint32_t chunk)
 #ifndef SLAY_FM_POLY
 #define SLAY_FM_POLY 1
 #endif
-
-// 2^x on the FMA pipe: j = round(x) by adding 1.5 * 2^23 (the sum's low mantissa bits hold
-// j), f = x - j in [-1/2, 1/2], 2^f from the degree-3 minimax polynomial of
-// slay_exp2_poly.h, and 2^j applied by adding j to the exponent field (the sum's bit
-// pattern times 2^23 is j << 23 modulo 2^32).  x is clamped to [-125, 126] so the exponent
-// field stays in range; the relative error is the polynomial's, below 1e-4.
-__device__ __forceinline__ float ex2_poly(float x)
-{
-    x = fminf(fmaxf(x, -125.0f), 126.0f);
-    const float t = __fadd_rn(x, 12582912.0f);
-    const float f = __fsub_rn(x, __fsub_rn(t, 12582912.0f));
-    float p = fmaf(SLAY_EXP2_C3, f, SLAY_EXP2_C2);
-    p = fmaf(p, f, SLAY_EXP2_C1);
-    p = fmaf(p, f, SLAY_EXP2_C0);
-    return __uint_as_float(__float_as_uint(t) * 8388608u + __float_as_uint(p));
-}
 
 struct FmParams {
     int F, ntiles;
