@@ -98,16 +98,23 @@ def kernel_work(name, w, op):
     """
     D, Dv, F = w.D, w.Dv, w.F
     th = w.B * w.H * w.L                    # token-heads in the batch
-    if name in ("tc_causal_out",):
-        return th * (8 * D * F + 4 * F * Dv + (C_CHUNK + 1) * (F + Dv)), "flop", "tensor"
+    # The tensor-core kernels take at most 256 features per launch: a wider map runs as
+    # nch feature chunks (256 each, or 128 when F is not a multiple of 256), one launch of
+    # each kernel per chunk, whose sums meet before the division.  A launch gets its
+    # chunk's share; the masked P.V term (C+1) Dv, repeated per chunk, counts once.
+    nch = 1 if F <= 256 else (F // 256 if F % 256 == 0 else F // 128)
+    if name.startswith("tc_") and name != "tc_feature_map":
+        F = F // nch
+    if name in ("tc_causal_out", "tc_qphi_out"):
+        return (th * (4 * D * F + 4 * F * Dv + (C_CHUNK + 1) * F) +
+                th * (C_CHUNK + 1) * Dv // nch +
+                (th * 4 * D * F if name == "tc_causal_out" else 0)), "flop", "tensor"
     if name in ("tc_causal_state",):
         return th * (4 * D * F + 2 * F * Dv), "flop", "tensor"
     # stored-phi(k) form: the state kernel maps k (its own segment sums are not algorithmic
     # work), the output kernel does the rest of the causal forward
     if name == "tc_kphi_state":
         return th * (4 * D * F), "flop", "tensor"
-    if name == "tc_qphi_out":
-        return th * (4 * D * F + 4 * F * Dv + (C_CHUNK + 1) * (F + Dv)), "flop", "tensor"
     if name in ("tc_bidir_out",):
         return th * (4 * D * F + 2 * F * Dv), "flop", "tensor"
     if name in ("tc_bidir_state",):

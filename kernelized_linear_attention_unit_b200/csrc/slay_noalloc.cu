@@ -150,7 +150,7 @@ extern "C" slay_status slay_attn_causal_fwd_noalloc(const void* q, const void* k
     if (static_cast<int64_t>(B) * H * L == 0) return SLAY_OK;
     if (den && (reinterpret_cast<uintptr_t>(den) % 4) != 0) return SLAY_ERR_INVALID_ARG;
     // the tensor-core path runs in its low-memory form here (phi(k) recomputed, not stored)
-    const bool tc = dt == SLAY_BF16 && tc_supported(SLAY_OP_CAUSAL_FWD, B, H, L, R, m);
+    const bool tc = dt == SLAY_BF16 && tc_supported(SLAY_OP_CAUSAL_FWD, B, H, L, R, m, true);
     const size_t need = tc ? tc_workspace_bytes(SLAY_OP_CAUSAL_FWD, B, H, L, R, m, true)
                            : attn_ws(SLAY_OP_CAUSAL_FWD, dt, B, H, L, Dv, R, m);
     if (need > kScratchBytes) return SLAY_ERR_UNSUPPORTED;

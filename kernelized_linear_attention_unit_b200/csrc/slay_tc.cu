@@ -139,12 +139,65 @@ __device__ __forceinline__ Seg segment_of(int index, int nseg, int ntiles)
 constexpr int kMaxSlices = 256 / kSlice;
 
 struct KParams {
-    int L, F, nseg, ntiles;
+    int L, F, nseg, ntiles;   // F: the features of this launch (one chunk of at most 256)
     int all_segs;      // state kernel: 1 = every segment (bidirectional), 0 = all but the last
     float eps;
     float a2[kMaxSlices];   // per 64-feature slice (m % 64 == 0): the scales of its node
     float b2[kMaxSlices];
+    // Feature chunks.  Scores, readouts, numerators and denominators are sums over features,
+    // so a wider map runs as several chunks whose per-row numerators [rows][64] and
+    // denominators [rows] (fp32) meet in part_num / part_den: acc_in adds the earlier
+    // chunks' sums before the division, acc_out stores the sums there instead of the output.
+    int acc_in, acc_out;
+    float* part_num;
+    float* part_den;
 };
+
+// The output row `g` (global row index over [BH][L]) from its numerator o0|o1 (64 fp32 bit
+// patterns) and denominator d: out = num / (den + eps) in bf16 and den, or, with acc_out,
+// the chunk's running sums.
+__device__ __forceinline__ void finish_row(const KParams& kp, uint32_t (&o0)[32], uint32_t (&o1)[32],
+                                           float d, size_t g, __nv_bfloat16* out, float* den)
+{
+    if (kp.acc_in) {
+        const float4* src = reinterpret_cast<const float4*>(kp.part_num + g * 64);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            const float4 a = src[q];
+            uint32_t* o = q < 8 ? o0 : o1;
+            const int c = 4 * (q & 7);
+            o[c] = __float_as_uint(__uint_as_float(o[c]) + a.x);
+            o[c + 1] = __float_as_uint(__uint_as_float(o[c + 1]) + a.y);
+            o[c + 2] = __float_as_uint(__uint_as_float(o[c + 2]) + a.z);
+            o[c + 3] = __float_as_uint(__uint_as_float(o[c + 3]) + a.w);
+        }
+        d += kp.part_den[g];
+    }
+    if (kp.acc_out) {
+        float4* dst = reinterpret_cast<float4*>(kp.part_num + g * 64);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            const uint32_t* o = q < 8 ? o0 : o1;
+            const int c = 4 * (q & 7);
+            dst[q] = make_float4(__uint_as_float(o[c]), __uint_as_float(o[c + 1]),
+                                 __uint_as_float(o[c + 2]), __uint_as_float(o[c + 3]));
+        }
+        kp.part_den[g] = d;
+        return;
+    }
+    const float rz = 1.0f / (d + kp.eps);
+    uint4* dst = reinterpret_cast<uint4*>(out + g * 64);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const uint32_t* o = q < 4 ? o0 : o1;
+        const int c = 8 * (q & 3);
+        dst[q] = make_uint4(pack_bf16(__uint_as_float(o[c]) * rz, __uint_as_float(o[c + 1]) * rz),
+                            pack_bf16(__uint_as_float(o[c + 2]) * rz, __uint_as_float(o[c + 3]) * rz),
+                            pack_bf16(__uint_as_float(o[c + 4]) * rz, __uint_as_float(o[c + 5]) * rz),
+                            pack_bf16(__uint_as_float(o[c + 6]) * rz, __uint_as_float(o[c + 7]) * rz));
+    }
+    if (den) den[g] = d;
+}
 
 // v[t] for a slice index t < kMaxSlices, by selects (an indexed parameter array would be
 // copied to local memory)
@@ -863,27 +916,9 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 reg_fence1(dr);
                 tc_fence_before();
                 warp_arrive(&bar[B_O_EMPTY]);
-                const float d = __uint_as_float(dr);
-                const float rz = 1.0f / (d + kp.eps);
                 const int grow = tile * kTile + static_cast<int>(row);
-                if (grow < kp.L) {
-                    uint4* dst = reinterpret_cast<uint4*>(out + (rowbase + grow) * 64);
-    #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        dst[q] = make_uint4(
-                            pack_bf16(__uint_as_float(o0[8 * q]) * rz, __uint_as_float(o0[8 * q + 1]) * rz),
-                            pack_bf16(__uint_as_float(o0[8 * q + 2]) * rz, __uint_as_float(o0[8 * q + 3]) * rz),
-                            pack_bf16(__uint_as_float(o0[8 * q + 4]) * rz, __uint_as_float(o0[8 * q + 5]) * rz),
-                            pack_bf16(__uint_as_float(o0[8 * q + 6]) * rz, __uint_as_float(o0[8 * q + 7]) * rz));
-    #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        dst[4 + q] = make_uint4(
-                            pack_bf16(__uint_as_float(o1[8 * q]) * rz, __uint_as_float(o1[8 * q + 1]) * rz),
-                            pack_bf16(__uint_as_float(o1[8 * q + 2]) * rz, __uint_as_float(o1[8 * q + 3]) * rz),
-                            pack_bf16(__uint_as_float(o1[8 * q + 4]) * rz, __uint_as_float(o1[8 * q + 5]) * rz),
-                            pack_bf16(__uint_as_float(o1[8 * q + 6]) * rz, __uint_as_float(o1[8 * q + 7]) * rz));
-                    if (den) den[rowbase + grow] = d;
-                }
+                if (grow < kp.L)
+                    finish_row(kp, o0, o1, __uint_as_float(dr), rowbase + grow, out, den);
             }
         }
         wt.report(err);
@@ -1270,27 +1305,9 @@ k_tc_causal_out_pk(const __grid_constant__ CUtensorMap tmq, const __grid_constan
                 reg_fence1(dr);
                 tc_fence_before();
                 warp_arrive(&bar[B_O_EMPTY]);
-                const float d = __uint_as_float(dr);
-                const float rz = 1.0f / (d + kp.eps);
                 const int grow = tile * kTile + static_cast<int>(row);
-                if (grow < kp.L) {
-                    uint4* dst = reinterpret_cast<uint4*>(out + (rowbase + grow) * 64);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        dst[q] = make_uint4(
-                            pack_bf16(__uint_as_float(o0[8 * q]) * rz, __uint_as_float(o0[8 * q + 1]) * rz),
-                            pack_bf16(__uint_as_float(o0[8 * q + 2]) * rz, __uint_as_float(o0[8 * q + 3]) * rz),
-                            pack_bf16(__uint_as_float(o0[8 * q + 4]) * rz, __uint_as_float(o0[8 * q + 5]) * rz),
-                            pack_bf16(__uint_as_float(o0[8 * q + 6]) * rz, __uint_as_float(o0[8 * q + 7]) * rz));
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        dst[4 + q] = make_uint4(
-                            pack_bf16(__uint_as_float(o1[8 * q]) * rz, __uint_as_float(o1[8 * q + 1]) * rz),
-                            pack_bf16(__uint_as_float(o1[8 * q + 2]) * rz, __uint_as_float(o1[8 * q + 3]) * rz),
-                            pack_bf16(__uint_as_float(o1[8 * q + 4]) * rz, __uint_as_float(o1[8 * q + 5]) * rz),
-                            pack_bf16(__uint_as_float(o1[8 * q + 6]) * rz, __uint_as_float(o1[8 * q + 7]) * rz));
-                    if (den) den[rowbase + grow] = d;
-                }
+                if (grow < kp.L)
+                    finish_row(kp, o0, o1, __uint_as_float(dr), rowbase + grow, out, den);
             }
         }
         wt.report(err);
@@ -1532,27 +1549,8 @@ k_tc_bidir_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             reg_fence1(dr);
             tc_fence_before();
             warp_arrive(&bar[B_O_EMPTY]);
-            const float d = __uint_as_float(dr);
-            const float rz = 1.0f / (d + kp.eps);
             const int grow = tile * kTile + static_cast<int>(row);
-            if (grow < kp.L) {
-                uint4* dst = reinterpret_cast<uint4*>(out + (rowbase + grow) * 64);
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    dst[q] = make_uint4(
-                        pack_bf16(__uint_as_float(o0[8 * q]) * rz, __uint_as_float(o0[8 * q + 1]) * rz),
-                        pack_bf16(__uint_as_float(o0[8 * q + 2]) * rz, __uint_as_float(o0[8 * q + 3]) * rz),
-                        pack_bf16(__uint_as_float(o0[8 * q + 4]) * rz, __uint_as_float(o0[8 * q + 5]) * rz),
-                        pack_bf16(__uint_as_float(o0[8 * q + 6]) * rz, __uint_as_float(o0[8 * q + 7]) * rz));
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    dst[4 + q] = make_uint4(
-                        pack_bf16(__uint_as_float(o1[8 * q]) * rz, __uint_as_float(o1[8 * q + 1]) * rz),
-                        pack_bf16(__uint_as_float(o1[8 * q + 2]) * rz, __uint_as_float(o1[8 * q + 3]) * rz),
-                        pack_bf16(__uint_as_float(o1[8 * q + 4]) * rz, __uint_as_float(o1[8 * q + 5]) * rz),
-                        pack_bf16(__uint_as_float(o1[8 * q + 6]) * rz, __uint_as_float(o1[8 * q + 7]) * rz));
-                if (den) den[rowbase + grow] = d;
-            }
+            if (grow < kp.L) finish_row(kp, o0, o1, __uint_as_float(dr), rowbase + grow, out, den);
         }
     }
     wt.report(err);
@@ -1605,31 +1603,47 @@ size_t smem_bytes_state(int F) { return smem_state_layout(F).total + 1024; }
 
 }  // namespace
 
-bool tc_supported(slay_op op, int B, int H, int L, int R, int m)
+namespace {
+
+// Features per launch: the whole map up to 256, else chunks of 256 (or 128 when F is not a
+// multiple of 256) whose sums meet in the partial numerator / denominator buffers.
+int chunk_features(int F) { return F <= 256 ? F : (F % 256 == 0 ? 256 : 128); }
+
+}  // namespace
+
+bool tc_supported(slay_op op, int B, int H, int L, int R, int m, bool lowmem)
 {
     const int F = R * m;
     if (op != SLAY_OP_CAUSAL_FWD && op != SLAY_OP_BIDIR_FWD) return false;
-    if (m % kSlice != 0 || F % 128 != 0 || F > 256) return false;
+    if (m % kSlice != 0 || F % 128 != 0 || F > (lowmem ? 256 : 512)) return false;
     if (static_cast<int64_t>(B) * H * L <= 0) return false;
-    return smem_bytes_out(F) <= 232448;
+    return smem_bytes_out(chunk_features(F)) <= 232448;
 }
 
 namespace {
 
-// Workspace: header | per-segment S [BH][nseg][F][64] fp32 | z [BH][nseg][F] fp32 | and, for
-// the causal forward that stores phi(k), phi(k) [BH][L][F] bf16.
+// Workspace: header | per-segment S [BH][nseg][Fc][64] fp32 | z [BH][nseg][Fc] fp32 | for the
+// causal forward that stores phi(k): phi(k) [BH][L][Fc] bf16 | with more than one feature
+// chunk: partial numerators [BH][L][64] and denominators [BH][L] fp32.  Fc is the chunk
+// width; the chunks run one after another and reuse the per-chunk parts.
 struct WsLayout {
-    size_t s, z, phik, total;
+    size_t s, z, phik, num, den, total;
 };
 
 WsLayout ws_layout(int BH, int L, int F, int nseg, bool with_phik)
 {
-    const size_t per = static_cast<size_t>(BH) * nseg * F;
+    const int Fc = chunk_features(F);
+    const size_t per = static_cast<size_t>(BH) * nseg * Fc;
+    const size_t rows = static_cast<size_t>(BH) * L;
+    auto up = [](size_t b) { return (b + 255) & ~size_t(255); };
     WsLayout w;
     w.s = kWsHeader;
-    w.z = w.s + ((per * 64 * sizeof(float) + 255) & ~size_t(255));
-    w.phik = w.z + ((per * sizeof(float) + 255) & ~size_t(255));
-    w.total = w.phik + (with_phik ? static_cast<size_t>(BH) * L * F * sizeof(uint16_t) : 0);
+    w.z = w.s + up(per * 64 * sizeof(float));
+    w.phik = w.z + up(per * sizeof(float));
+    w.num = w.phik + up(with_phik ? rows * Fc * sizeof(uint16_t) : 0);
+    const bool chunked = Fc < F;
+    w.den = w.num + (chunked ? up(rows * 64 * sizeof(float)) : 0);
+    w.total = w.den + (chunked ? up(rows * sizeof(float)) : 0);
     return w;
 }
 
@@ -1691,77 +1705,90 @@ cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, 
                         cudaStream_t st, bool lowmem)
 {
     if (!P.wB) return cudaErrorNotSupported;
-    const int BH = B * H, F = P.F;
+    const int BH = B * H, F = P.F, Fc = chunk_features(F), nch = F / Fc;
+    if (lowmem && nch > 1) return cudaErrorNotSupported;
     const int ntiles = (L + kTile - 1) / kTile;
     const int nseg = choose_nseg(BH, ntiles);
     const bool store_phik = causal && !lowmem;
     const WsLayout wl = ws_layout(BH, L, F, nseg, store_phik);
     char* w = static_cast<char*>(ws);
-    CUtensorMap mq, mk, mv, mw, mpk;
-    if (!map_rows(&mq, q, L, BH) || !map_rows(&mk, k, L, BH) || !map_rows(&mv, v, L, BH) ||
-        !map_w(&mw, P.wB, F))
+    CUtensorMap mq, mk, mv, mpk;
+    if (!map_rows(&mq, q, L, BH) || !map_rows(&mk, k, L, BH) || !map_rows(&mv, v, L, BH))
         return cudaErrorInvalidValue;
     // without stored phi(k) the state kernel never touches this map: any valid one will do
-    if (!map_phik(&mpk, store_phik ? static_cast<const void*>(w + wl.phik) : P.wB, F,
+    if (!map_phik(&mpk, store_phik ? static_cast<const void*>(w + wl.phik) : P.wB, Fc,
                   store_phik ? L : 1, store_phik ? BH : 1))
         return cudaErrorInvalidValue;
-    KParams kp;
-    kp.L = L; kp.F = F; kp.nseg = nseg; kp.ntiles = ntiles; kp.eps = eps;
-    kp.all_segs = (causal && lowmem) ? 0 : 1;
-    for (int t = 0; t < kMaxSlices; ++t) {
-        const int node = t < F / kSlice ? t * kSlice / P.m : 0;
-        kp.a2[t] = P.a2[node];
-        kp.b2[t] = P.b2[node];
-    }
     int* err = reinterpret_cast<int*>(w);
     float* wsS = reinterpret_cast<float*>(w + wl.s);
     float* wsZ = reinterpret_cast<float*>(w + wl.z);
     __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
     cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), st);
     if (e != cudaSuccess) return e;
-    const size_t sms = smem_bytes_state(F);
-    if (!causal) {
-        // every segment's sum, then the readout against their total
-        if ((e = set_smem(k_tc_causal_state<false>, sms)) != cudaSuccess) return e;
-        {
-            TraceScope trace_("tc_bidir_state", st);
-            k_tc_causal_state<false><<<BH * nseg, kThreads, sms, st>>>(mk, mv, mw, mpk, kp, wsS, wsZ, err);
+    const size_t sms = smem_bytes_state(Fc);
+    for (int c = 0; c < nch; ++c) {
+        // chunk c: features [c Fc, (c+1) Fc), i.e. packed W sub-slices from c Fc / 32 on
+        CUtensorMap mw;
+        const uint16_t* wc = P.wB + static_cast<size_t>(c) * (Fc / kSub) * 64 * 64;
+        if (!map_w(&mw, wc, Fc)) return cudaErrorInvalidValue;
+        KParams kp;
+        kp.L = L; kp.F = Fc; kp.nseg = nseg; kp.ntiles = ntiles; kp.eps = eps;
+        kp.all_segs = (causal && lowmem) ? 0 : 1;
+        for (int t = 0; t < kMaxSlices; ++t) {
+            const int node = t < Fc / kSlice ? (c * Fc + t * kSlice) / P.m : 0;
+            kp.a2[t] = P.a2[node];
+            kp.b2[t] = P.b2[node];
+        }
+        kp.acc_in = c > 0;
+        kp.acc_out = c + 1 < nch;
+        kp.part_num = nch > 1 ? reinterpret_cast<float*>(w + wl.num) : nullptr;
+        kp.part_den = nch > 1 ? reinterpret_cast<float*>(w + wl.den) : nullptr;
+        if (!causal) {
+            // every segment's sum, then the readout against their total
+            if ((e = set_smem(k_tc_causal_state<false>, sms)) != cudaSuccess) return e;
+            {
+                TraceScope trace_("tc_bidir_state", st);
+                k_tc_causal_state<false><<<BH * nseg, kThreads, sms, st>>>(mk, mv, mw, mpk, kp, wsS, wsZ, err);
+                if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            }
+            const size_t smb = smem_bidir_layout(Fc).total + 1024;
+            if ((e = set_smem(k_tc_bidir_out, smb)) != cudaSuccess) return e;
+            TraceScope trace_("tc_bidir_out", st);
+            k_tc_bidir_out<<<BH * nseg, kOutThreads, smb, st>>>(mq, mw, kp, wsS, wsZ, o, den, err);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            continue;
+        }
+        if (store_phik) {
+            // phi(k) and every segment's sum once; the output kernel reads phi(k)
+            if ((e = set_smem(k_tc_causal_state<true>, sms)) != cudaSuccess) return e;
+            {
+                TraceScope trace_("tc_kphi_state", st);
+                k_tc_causal_state<true><<<BH * nseg, kThreads, sms, st>>>(mk, mv, mw, mpk, kp, wsS, wsZ, err);
+                if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            }
+            const size_t smo = smem_outpk_layout(Fc).total + 1024;
+            if ((e = set_smem(k_tc_causal_out_pk, smo)) != cudaSuccess) return e;
+            TraceScope trace_("tc_qphi_out", st);
+            k_tc_causal_out_pk<<<BH * nseg, kOutThreads, smo, st>>>(mq, mpk, mv, mw, kp, wsS, wsZ, o, den, err);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            continue;
+        }
+        // low-memory form (no phi(k) buffer): the output kernel recomputes phi(k)
+        if (nseg > 1) {
+            if ((e = set_smem(k_tc_causal_state<false>, sms)) != cudaSuccess) return e;
+            TraceScope trace_("tc_causal_state", st);
+            k_tc_causal_state<false><<<BH * (nseg - 1), kThreads, sms, st>>>(mk, mv, mw, mpk, kp, wsS, wsZ, err);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
-        const size_t smb = smem_bidir_layout(F).total + 1024;
-        if ((e = set_smem(k_tc_bidir_out, smb)) != cudaSuccess) return e;
-        TraceScope trace_("tc_bidir_out", st);
-        k_tc_bidir_out<<<BH * nseg, kOutThreads, smb, st>>>(mq, mw, kp, wsS, wsZ, o, den, err);
-        return cudaGetLastError();
-    }
-    if (store_phik) {
-        // phi(k) and every segment's sum once; the output kernel reads phi(k)
-        if ((e = set_smem(k_tc_causal_state<true>, sms)) != cudaSuccess) return e;
+        const size_t smo = smem_bytes_out(Fc);
+        if ((e = set_smem(k_tc_causal_out, smo)) != cudaSuccess) return e;
         {
-            TraceScope trace_("tc_kphi_state", st);
-            k_tc_causal_state<true><<<BH * nseg, kThreads, sms, st>>>(mk, mv, mw, mpk, kp, wsS, wsZ, err);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            TraceScope trace_("tc_causal_out", st);
+            k_tc_causal_out<<<BH * nseg, kOutThreads, smo, st>>>(mq, mk, mv, mw, kp, wsS, wsZ, o, den, err);
         }
-        const size_t smo = smem_outpk_layout(F).total + 1024;
-        if ((e = set_smem(k_tc_causal_out_pk, smo)) != cudaSuccess) return e;
-        TraceScope trace_("tc_qphi_out", st);
-        k_tc_causal_out_pk<<<BH * nseg, kOutThreads, smo, st>>>(mq, mpk, mv, mw, kp, wsS, wsZ, o, den, err);
-        return cudaGetLastError();
-    }
-    // low-memory form (no phi(k) buffer): the output kernel recomputes phi(k)
-    if (nseg > 1) {
-        if ((e = set_smem(k_tc_causal_state<false>, sms)) != cudaSuccess) return e;
-        TraceScope trace_("tc_causal_state", st);
-        k_tc_causal_state<false><<<BH * (nseg - 1), kThreads, sms, st>>>(mk, mv, mw, mpk, kp, wsS, wsZ, err);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    const size_t smo = smem_bytes_out(F);
-    if ((e = set_smem(k_tc_causal_out, smo)) != cudaSuccess) return e;
-    {
-        TraceScope trace_("tc_causal_out", st);
-        k_tc_causal_out<<<BH * nseg, kOutThreads, smo, st>>>(mq, mk, mv, mw, kp, wsS, wsZ, o, den, err);
-    }
-    return cudaGetLastError();
+    return cudaSuccess;
 }
 
 }  // namespace slay

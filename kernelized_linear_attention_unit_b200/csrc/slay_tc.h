@@ -11,8 +11,9 @@
 
 namespace slay {
 
-// Whether the tensor-core path takes this op at these sizes (bf16 mode only).
-bool tc_supported(slay_op op, int B, int H, int L, int R, int m);
+// Whether the tensor-core path takes this op at these sizes (bf16 mode only); F up to 512
+// (as feature chunks of at most 256), or up to 256 in the low-memory form (lowmem).
+bool tc_supported(slay_op op, int B, int H, int L, int R, int m, bool lowmem = false);
 // Workspace bytes of the tensor-core path.  The causal forward stores phi(k) ([BH][L][F]
 // bf16) unless `lowmem`, where the output kernel recomputes it instead.
 size_t tc_workspace_bytes(slay_op op, int B, int H, int L, int R, int m, bool lowmem = false);

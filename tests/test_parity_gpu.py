@@ -98,7 +98,8 @@ def _run_fwd(q, k, v, w, causal):
                                       ("bf16", 4, 64, 1), ("bf16", 8, 64, 257),
                                       ("bf16", 2, 16, 64), ("bf16", 2, 64, 129),
                                       ("bf16", 4, 64, 1000), ("bf16", 2, 64, 2049),
-                                      ("bf16", 4, 64, 128)])
+                                      ("bf16", 4, 64, 128), ("bf16", 6, 64, 300),
+                                      ("bf16", 8, 64, 1000)])
 def test_attn_fwd_small(dt, R, m, L, causal):
     w = small(dt, R, m, L)
     q, k, v = W.gen_qkv(w)
@@ -115,8 +116,10 @@ def test_attn_fwd_small(dt, R, m, L, causal):
 # Enough (b, h) slices that the sequence is cut into few segments, so one CTA walks
 # several 128-token tiles (state carried in tensor memory from tile to tile), with a
 # ragged last tile; and B*H >= 148, where a single segment covers the whole sequence.
+# F = 512 and 384 run as feature chunks (256 + 256, 3 x 128) summed before the division.
 @pytest.mark.parametrize("B,H,L,R,m", [(2, 37, 657, 4, 64), (1, 148, 300, 4, 64),
-                                       (2, 37, 520, 2, 64), (1, 50, 1111, 4, 64)])
+                                       (2, 37, 520, 2, 64), (1, 50, 1111, 4, 64),
+                                       (2, 37, 657, 8, 64), (1, 20, 700, 6, 64)])
 def test_attn_fwd_multi_tile_segments(B, H, L, R, m):
     w = W.Workload("multitile", B=B, H=H, L=L, R=R, m=m, dtype="bf16", data_seed=17)
     q, k, v = W.gen_qkv(w)
