@@ -138,6 +138,19 @@ def kernel_work(name, w, op):
     if name == "simt_scan":
         nc = (w.L + C_CHUNK - 1) // C_CHUNK
         return w.B * w.H * nc * F * (Dv + 1) * 4 * 2, "byte", "hbm"
+    # backward (CUDA cores): of the whole-backward count 16DF + 10F Dv + (C+1)(3F + 2Dv) per
+    # token-head, the phi backward takes 8DF per row (projections of x^ and their transpose,
+    # q and k launched separately), the two chunk-state launches 2F(Dv+1) each, the chunk
+    # kernel the rest; the row statistics read out, g, den and write [dn, delta] (bytes)
+    if name == "simt_phi_bwd":
+        return th * 8 * D * F, "flop", "alu"
+    # the tensor-core phi backward is bound by its reads: x (bf16), dphi (fp32), dx (fp32)
+    if name == "tc_phi_bwd":
+        return th * (2 * D + 4 * F + 4 * D), "byte", "hbm"
+    if name == "simt_bwd_chunk":
+        return th * (6 * F * Dv + (C_CHUNK + 1) * (3 * F + 2 * Dv)), "flop", "alu"
+    if name == "simt_bwd_rowstats":
+        return th * (2 * Dv * 2 + 4 + (Dv + 1) * 4), "byte", "hbm"
     if name == "simt_decode":
         per = F * Dv * 4 * 2 + F * 4 * 2 + (2 * D + 2 * Dv) * 2
         return w.B * w.H * per, "byte", "hbm"

@@ -15,8 +15,8 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
-#include <type_traits>
 #include <cstdint>
+#include <type_traits>
 
 #include "slay_internal.h"
 #include "slay_tc.h"
@@ -990,6 +990,11 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
     if ((err = cudaFuncSetAttribute(k_phi_bwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     static_cast<int>(psm))) != cudaSuccess)
         return err;
+    // bf16 inputs: the feature map's backward on tensor cores when it takes these sizes
+    if (std::is_same<T, __nv_bfloat16>::value && P.wB && tc_phi_bwd_supported(kD, P.R, P.m, rows)) {
+        if ((err = tc_phi_bwd(q, dphq, dq, rows, P, st)) != cudaSuccess) return err;
+        return tc_phi_bwd(k, dphk, dk, rows, P, st);
+    }
     const unsigned rg = static_cast<unsigned>((rows + C - 1) / C);
     {
         TraceScope trace_("simt_phi_bwd", st);

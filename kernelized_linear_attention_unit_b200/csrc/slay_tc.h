@@ -25,7 +25,13 @@ void tc_pack_wb(int D, int R, int m, const uint16_t* om, const uint16_t* an, uin
 // Feature map bf16 -> bf16 on tensor cores: D == 64, m % 32 == 0, F % 128 == 0, F <= 512.
 bool tc_fmap_supported(int D, int R, int m, int64_t n_rows);
 cudaError_t tc_feature_map(const void* x, void* phi, int64_t n, const Params& P, cudaStream_t st);
-// Device address of the feature-map kernel's status word (set when a bounded wait ran out).
+// Backward of the feature map on tensor cores (bf16 x, fp32 dphi [n][F] -> fp32 dx [n][64]):
+// same sizes as the forward map.
+bool tc_phi_bwd_supported(int D, int R, int m, int64_t n_rows);
+cudaError_t tc_phi_bwd(const void* x, const float* dphi, float* dx, int64_t n, const Params& P,
+                       cudaStream_t st);
+// Device address of the status word of the feature-map kernels, forward and backward (set
+// when a bounded wait ran out).
 const void* fmap_status_word();
 cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, float* den,
                         int B, int H, int L, const Params& P, float eps, bool causal, void* ws,

@@ -1,0 +1,400 @@
+// slay_tc_phibwd.cu -- tensor-core backward of the feature map: dx from dphi for bf16 rows.
+//
+// Method: "SLAY: Geometry-Aware Spherical Linearized Attention with Yat-Kernel" (nubint.ai
+// review, "Proposed method", steps 1, 3, 4, 5) defines, per row x and feature f = r*m + j,
+//   phi_f = c_r exp(sqrt(2 s_r) omega_f.x^ - s_r) (a_f.x^)^2,  x^ = x / |x|;
+// the pages give no backward, so it is the chain rule of that definition.  With u = omega_f.x
+// and p = a_f.x of the raw row, n = |x| and e = exp2(a2_r u/n + b2_r + 2 log2(1/n)) (so that
+// phi = e p^2 and c_r exp(..) = e n^2):
+//   dx^ = sum_f alpha_f omega_f + beta_f a_f,   t = dphi_f e p,
+//   alpha_f = t p sqrt(2 s_r),  beta_f = 2 n t,
+//   dx = (dx^ - x^ (x^ . dx^)) / n.
+// Both contractions run on tensor cores: per 128-row tile and 64-feature group g the
+// projections U = X W_g^T (N = 128: 64 omega and 64 anchor columns, as in the forward map),
+// then dX^ += [alpha | beta]_g [Omega_g ; A_g] (K = 128, N = 64) with the same resident W
+// tiles read as an MN-major operand.  The kernel reads x (bf16), dphi (fp32) and writes dx
+// (fp32): it is bound by the dphi reads (4F bytes per row).
+//
+// Persistent, one CTA per SM, 128-row tiles round-robin.  Warp 0 issues every TMA load and
+// MMA; warps 1-8 are the epilogue: warp w serves TMEM lanes 32 (w % 4).. (rows of the tile)
+// and the 32-feature half (w - 1) / 4 of every group.  Per group an epilogue warp reads its
+// projections, its rows' dphi (prefetched one group ahead) and writes its block of
+// [alpha | beta] into a K-major 128-byte-swizzled operand tile; per tile it turns dX^ into
+// dx.  Every wait is bounded; a timeout sets the library's feature-map status word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "slay_tc.h"
+#include "slay_tc_common.cuh"
+#include "slay_tc_ptx.cuh"
+
+namespace slay {
+
+using namespace tc;
+
+namespace {
+
+constexpr int kRows = 128;                  // rows per tile (MMA M)
+constexpr int kBoxBytes = kRows * 128;      // [128 rows][64 bf16] swizzled X tile = 16 KiB
+constexpr int kSubBytes = 64 * 128;         // packed W of 32 features = 8 KiB
+constexpr int kGroupBytes = 2 * kSubBytes;  // 64 features = 16 KiB
+constexpr int kABytes = 2 * kBoxBytes;      // [alpha | beta] of one group: two 16 KiB K-tiles
+constexpr int kEpiWarps = 8;
+constexpr int kPbThreads = 32 * (1 + kEpiWarps);
+constexpr int kNumSMs = 148;
+constexpr int kMaxXBufs = 4;
+constexpr uint32_t kColU = 0;               // two 128-column projection buffers
+constexpr uint32_t kColDX = 256;            // two 64-column dX^ accumulators
+
+enum {
+    PB_W = 0,
+    PB_XF = 1,                  // + slot
+    PB_XE = PB_XF + kMaxXBufs,  // + slot (8 warp arrivals: dx of the tile written)
+    PB_UF = PB_XE + kMaxXBufs,  // + buffer (projection MMA commit)
+    PB_AF = PB_UF + 2,          // + buffer (8 warp arrivals: [alpha | beta] written)
+    PB_AE = PB_AF + 2,          // + buffer (contraction MMA commit: operand free)
+    PB_DF = PB_AE + 2,          // + buffer (dX^ of a tile complete)
+    PB_DE = PB_DF + 2,          // + buffer (8 warp arrivals: dX^ read)
+    PB_NUM = PB_DE + 2
+};
+
+struct PbLayout {
+    uint32_t w, x, a, bar, tmem, total;
+    int xbufs;
+};
+
+__host__ __device__ inline PbLayout pb_layout(int F)
+{
+    PbLayout l;
+    l.xbufs = F <= 128 ? 4 : F <= 256 ? 3 : 2;
+    l.w = 0;
+    l.x = (F / 32) * kSubBytes;
+    l.a = l.x + l.xbufs * kBoxBytes;
+    l.bar = l.a + 2 * kABytes;
+    l.tmem = l.bar + PB_NUM * 8;
+    l.total = l.tmem + 16;
+    return l;
+}
+
+struct PbParams {
+    int F, ntiles;
+    float a2[16];   // per 32-feature sub-slice: the scales of its node (F <= 512)
+    float b2[16];
+    float sq[16];   // sqrt(2 s_r)
+};
+
+__global__ void __launch_bounds__(kPbThreads, 1)
+k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
+             const float* __restrict__ dphi, float* __restrict__ dx, int64_t n_rows, PbParams pp,
+             int* status)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* sm = aligned_smem(smem_raw);
+    const PbLayout L = pb_layout(pp.F);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L.bar);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L.tmem);
+    const uint32_t sbase = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int ng = pp.F / 64;
+    const int xbufs = L.xbufs;
+
+    if (warp == 0) {
+        tmem_alloc(tslot, 512);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        for (int i = 0; i < PB_NUM; ++i) mbar_init(&bar[i], 1);
+        for (int s = 0; s < kMaxXBufs; ++s) mbar_init(&bar[PB_XE + s], kEpiWarps);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bar[PB_AF + b], kEpiWarps);
+            mbar_init(&bar[PB_DE + b], kEpiWarps);
+        }
+        mbar_fence_init();
+        tma_prefetch_desc(&tmx);
+        tma_prefetch_desc(&tmw);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem0 = *tslot;
+    Waiter wt;
+    const int nt = static_cast<int>(blockIdx.x) < pp.ntiles
+                       ? (pp.ntiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                       : 0;
+    const int njobs = nt * ng;   // job j = tile k (k-th of this CTA), group g: j = k ng + g
+
+    if (warp == 0) {
+        if (lane == 0 && nt > 0) {
+            auto load_x = [&](int k) {
+                const int s = k % xbufs;
+                mbar_arrive_expect_tx(&bar[PB_XF + s], kBoxBytes);
+                tma_load_2d(sm + L.x + s * kBoxBytes, &tmx, &bar[PB_XF + s], 0,
+                            (k * static_cast<int>(gridDim.x) + static_cast<int>(blockIdx.x)) * kRows);
+            };
+            mbar_arrive_expect_tx(&bar[PB_W], (pp.F / 32) * kSubBytes);
+            for (int n = 0; n < pp.F / 32; ++n)
+                tma_load_2d(sm + L.w + n * kSubBytes, &tmw, &bar[PB_W], 0, n * 64);
+            for (int k = 0; k < xbufs && k < nt; ++k) load_x(k);
+            {
+                uint32_t ph = 0;
+                wt.wait(&bar[PB_W], ph);
+            }
+            constexpr uint32_t idU = idesc_bf16(128, 128, 0, 0);   // X (K-major) x W (K-major)
+            constexpr uint32_t idD = idesc_bf16(128, 64, 0, 1);    // [alpha|beta] x W (MN-major)
+            const uint64_t dx0 = sdesc(sbase + L.x, 16, 1024, kLayoutSW128);
+            const uint64_t dw0 = sdesc(sbase + L.w, 16, 1024, kLayoutSW128);
+            const uint64_t da0 = sdesc(sbase + L.a, 16, 1024, kLayoutSW128);
+            // projection job jp = (tile pk, group pg); X slot ps of tile pk and its phase
+            int jp = 0, pk = 0, pg = 0, ps = 0;
+            uint32_t pph = 0;
+            auto proj = [&]() {   // U[jp & 1] = X_pk W_pg^T, then advance to the next job
+                if (pg == 0) {
+                    uint32_t ph = pph;
+                    wt.wait(&bar[PB_XF + ps], ph);
+                }
+                tc_fence_after();
+                const uint64_t dx = dx0 + ((ps * kBoxBytes) >> 4);
+                const uint64_t dw = dw0 + ((pg * kGroupBytes) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_bf16(tmem0 + kColU + 128u * (jp & 1), dx + 2 * kk, dw + 2 * kk, idU,
+                              kk > 0 ? 1u : 0u);
+                umma_commit(&bar[PB_UF + (jp & 1)]);
+                ++jp;
+                if (++pg == ng) {
+                    pg = 0;
+                    ++pk;
+                    if (++ps == xbufs) {
+                        ps = 0;
+                        pph ^= 1u;
+                    }
+                }
+            };
+            proj();
+            if (njobs > 1) proj();
+            int k = 0, g = 0, xs_prev = xbufs - 1;   // contraction job j = (tile k, group g)
+            uint32_t xph_prev = 1;                    // phase of X slot of tile k - 1
+            for (int j = 0; j < njobs && wt.ok; ++j) {
+                {
+                    uint32_t ph = static_cast<uint32_t>((j >> 1) & 1);
+                    wt.wait(&bar[PB_AF + (j & 1)], ph);   // [alpha|beta]_j written, U_j read
+                }
+                if (g == 0 && k >= 1) {
+                    // every epilogue warp is past the dx of tile k - 1 (it wrote A of job j
+                    // after it): X slot (k - 1) % xbufs takes tile k - 1 + xbufs
+                    uint32_t ph = xph_prev;
+                    wt.wait(&bar[PB_XE + xs_prev], ph);
+                    if (k - 1 + xbufs < nt) load_x(k - 1 + xbufs);
+                }
+                if (g == 0 && k >= 2) {   // dX^ buffer k & 1 read by the dx of tile k - 2
+                    uint32_t ph = static_cast<uint32_t>(((k - 2) >> 1) & 1);
+                    wt.wait(&bar[PB_DE + (k & 1)], ph);
+                }
+                tc_fence_after();
+                // dX^_k += [alpha|beta]_j [Omega_g ; A_g]: K = 128 (two 64-wide K-tiles of
+                // the operand; the W rows of the group 2 KiB per 16-row K step)
+                const uint64_t da = da0 + (((j & 1) * kABytes) >> 4);
+                const uint64_t dwm = dw0 + ((g * kGroupBytes) >> 4);   // same tiles, MN-major
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_bf16(tmem0 + kColDX + 64u * (k & 1),
+                              da + (kk >> 2) * (kBoxBytes >> 4) + 2 * (kk & 3), dwm + 128 * kk, idD,
+                              (g > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(&bar[PB_AE + (j & 1)]);
+                if (g == ng - 1) umma_commit(&bar[PB_DF + (k & 1)]);
+                if (j + 2 < njobs) proj();   // job j + 2 into U[j & 1], read already (AF)
+                if (++g == ng) {
+                    g = 0;
+                    ++k;
+                    if (++xs_prev == xbufs) {
+                        xs_prev = 0;
+                        xph_prev ^= 1u;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else {
+        const int ew = warp - 1, q = warp & 3, half = ew >> 2;
+        const uint32_t row = 32u * q + lane;
+        const uint32_t trow = tmem0 + ((32u * q) << 16);
+        const uint32_t abase = sbase + L.a + half * kBoxBytes;
+        const int F = pp.F;
+        // dphi of (tile k, group g) for this lane's row: 32 fp32 (features 64g + 32 half ..)
+        auto dphi_ptr = [&](int k, int g) -> const float4* {
+            const int64_t r = static_cast<int64_t>(k * static_cast<int>(gridDim.x) +
+                                                   static_cast<int>(blockIdx.x)) * kRows + row;
+            const int64_t rr = r < n_rows ? r : n_rows - 1;   // rows past the end: any valid row
+            return reinterpret_cast<const float4*>(dphi + rr * F + 64 * g + 32 * half);
+        };
+        float4 dpn[8];
+        if (nt > 0) {
+            const float4* p = dphi_ptr(0, 0);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dpn[i] = __ldg(p + i);
+        }
+        for (int k = 0; k < nt; ++k) {
+            const int s = k % xbufs;
+            {
+                uint32_t ph = static_cast<uint32_t>((k / xbufs) & 1);
+                wt.wait(&bar[PB_XF + s], ph);
+            }
+            float inv, l2i;
+            const unsigned char* xrow = sm + L.x + s * kBoxBytes + row * 128;
+            row_scale(xrow, row, inv, l2i);
+            const float nrm = 1.0f / inv, two_n = 2.0f * nrm;
+            for (int g = 0; g < ng; ++g) {
+                const int j = k * ng + g;
+                float4 dp[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) dp[i] = dpn[i];
+                if (j + 1 < njobs) {   // prefetch the next group's dphi
+                    const float4* p = dphi_ptr(g + 1 < ng ? k : k + 1, g + 1 < ng ? g + 1 : 0);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) dpn[i] = __ldg(p + i);
+                }
+                {
+                    uint32_t ph = static_cast<uint32_t>((j >> 1) & 1);
+                    wt.wait(&bar[PB_UF + (j & 1)], ph);
+                }
+                tc_fence_after();
+                uint32_t ur[32], pr[32];
+                const uint32_t c0 = trow + kColU + 128u * (j & 1) + 64u * half;
+                tmem_ld32(c0, ur);
+                tmem_ld32(c0 + 32, pr);
+                tmem_wait_ld();
+                reg_fence(ur);
+                reg_fence(pr);
+                const int sub = 2 * g + half;
+                const float a = pp.a2[sub] * inv, bb = pp.b2[sub] + l2i, sq = pp.sq[sub];
+                uint32_t al[16], be[16];
+#pragma unroll
+                for (int c = 0; c < 32; c += 2) {
+                    const float4 d4 = dp[c >> 2];
+                    const float d0 = (c & 2) ? d4.z : d4.x, d1 = (c & 2) ? d4.w : d4.y;
+                    const float p0 = __uint_as_float(pr[c]), p1 = __uint_as_float(pr[c + 1]);
+                    const float t0 = d0 * ex2(fmaf(a, __uint_as_float(ur[c]), bb)) * p0;
+                    const float t1 = d1 * ex2(fmaf(a, __uint_as_float(ur[c + 1]), bb)) * p1;
+                    al[c >> 1] = pack_bf16(t0 * p0 * sq, t1 * p1 * sq);
+                    be[c >> 1] = pack_bf16(t0 * two_n, t1 * two_n);
+                }
+                if (j >= 2) {   // operand buffer j & 1 read by the contraction of job j - 2
+                    uint32_t ph = static_cast<uint32_t>(((j - 2) >> 1) & 1);
+                    wt.wait(&bar[PB_AE + (j & 1)], ph);
+                }
+                // K order of the operand: [alpha | beta] of sub-slice 2g in K-tile 0, of 2g+1
+                // in K-tile 1 -- the row order of the group's packed W (32 omega, 32 anchor)
+                const uint32_t arow = abase + (j & 1) * kABytes;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    st_shared_v4(arow + sw128_off(row, c), al[4 * c], al[4 * c + 1], al[4 * c + 2],
+                                 al[4 * c + 3]);
+                    st_shared_v4(arow + sw128_off(row, 4 + c), be[4 * c], be[4 * c + 1],
+                                 be[4 * c + 2], be[4 * c + 3]);
+                }
+                fence_async_smem();
+                tc_fence_before();
+                warp_arrive(&bar[PB_AF + (j & 1)]);
+            }
+            // dx of tile k: dX^ (64 columns) -> (dX^ - x^ (x^ . dX^)) / n, this warp's half
+            {
+                uint32_t ph = static_cast<uint32_t>((k >> 1) & 1);
+                wt.wait(&bar[PB_DF + (k & 1)], ph);
+            }
+            tc_fence_after();
+            uint32_t d0[32], d1[32];
+            tmem_ld32(trow + kColDX + 64u * (k & 1), d0);
+            tmem_ld32(trow + kColDX + 64u * (k & 1) + 32, d1);
+            tmem_wait_ld();
+            reg_fence(d0);
+            reg_fence(d1);
+            tc_fence_before();
+            warp_arrive(&bar[PB_DE + (k & 1)]);
+            // x^ of this row from the X tile (bf16, 128-byte swizzle): element e of chunk c
+            float xh[64];
+            const uint4* xr = reinterpret_cast<const uint4*>(xrow);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint4 w4 = xr[c ^ (row & 7)];
+                const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    xh[8 * c + 2 * e] = __uint_as_float(ws[e] << 16) * inv;
+                    xh[8 * c + 2 * e + 1] = __uint_as_float(ws[e] & 0xFFFF0000u) * inv;
+                }
+            }
+            warp_arrive(&bar[PB_XE + s]);   // this warp is done with X slot s
+            float dot[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                dot[c & 3] = fmaf(xh[c], __uint_as_float(d0[c]), dot[c & 3]);
+                dot[c & 3] = fmaf(xh[32 + c], __uint_as_float(d1[c]), dot[c & 3]);
+            }
+            const float xd = (dot[0] + dot[1]) + (dot[2] + dot[3]);
+            const int64_t r = static_cast<int64_t>(k * static_cast<int>(gridDim.x) +
+                                                   static_cast<int>(blockIdx.x)) * kRows + row;
+            if (r < n_rows) {
+                float4* dst = reinterpret_cast<float4*>(dx + r * 64 + 32 * half);
+                float o[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c)   // selects, not an indexed pointer (local memory)
+                    o[c] = ((half ? __uint_as_float(d1[c]) : __uint_as_float(d0[c])) -
+                            (half ? xh[32 + c] : xh[c]) * xd) * inv;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    dst[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+            }
+        }
+    }
+    wt.report(status);
+    drain_after_failure(wt.ok);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem0, 512);
+}
+
+}  // namespace
+
+bool tc_phi_bwd_supported(int D, int R, int m, int64_t n_rows)
+{
+    const int F = R * m;
+    return D == 64 && m % 32 == 0 && F % 128 == 0 && F <= 512 && n_rows > 0 &&
+           n_rows <= (int64_t(1) << 31) - kRows && pb_layout(F).total + 1024 <= 232448;
+}
+
+cudaError_t tc_phi_bwd(const void* x, const float* dphi, float* dx, int64_t n, const Params& P,
+                       cudaStream_t st)
+{
+    const int F = P.F;
+    if (!P.wB || !tc_phi_bwd_supported(64, P.R, P.m, n)) return cudaErrorNotSupported;
+    CUtensorMap mx, mw;
+    if (!map_2d(&mx, x, 64, static_cast<uint64_t>(n), 64, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map_2d(&mw, P.wB, 64, static_cast<uint64_t>(F / 32) * 64, 64, 64,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    PbParams pp;
+    pp.F = F;
+    pp.ntiles = static_cast<int>((n + kRows - 1) / kRows);
+    for (int sub = 0; sub < 16; ++sub) {
+        const int node = sub < F / 32 ? sub * 32 / P.m : 0;
+        pp.a2[sub] = P.a2[node];
+        pp.b2[sub] = P.b2[node];
+        pp.sq[sub] = P.sq[node];
+    }
+    int* status = static_cast<int*>(const_cast<void*>(fmap_status_word()));
+    if (!status) return cudaErrorInvalidValue;
+    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
+    if (e != cudaSuccess) return e;
+    const size_t smem = pb_layout(F).total + 1024;
+    e = cudaFuncSetAttribute(k_tc_phi_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const int grid = pp.ntiles < kNumSMs ? pp.ntiles : kNumSMs;
+    TraceScope trace_("tc_phi_bwd", st);
+    k_tc_phi_bwd<<<grid, kPbThreads, smem, st>>>(mx, mw, dphi, dx, n, pp, status);
+    return cudaGetLastError();
+}
+
+}  // namespace slay
