@@ -8,7 +8,7 @@
 // phi = e p^2 and c_r exp(..) = e n^2):
 //   dx^ = sum_f alpha_f omega_f + beta_f a_f,   t = dphi_f e p,
 //   alpha_f = t p sqrt(2 s_r),  beta_f = 2 n t,
-//   dx = (dx^ - x^ (x^ . dx^)) / n.
+//   dx = (dx^ - x^ (x^ . dx^)) / n   (dx^ / 1e-12 below the norm guard |x| < 1e-12).
 // Both contractions run on tensor cores: per 128-row tile and 64-feature group g the
 // projections U = X W_g^T (N = 128: 64 omega and 64 anchor columns, as in the forward map),
 // then dX^ += [alpha | beta]_g [Omega_g ; A_g] (K = 128, N = 64) with the same resident W
@@ -332,7 +332,9 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
                 dot[c & 3] = fmaf(xh[c], __uint_as_float(d0[c]), dot[c & 3]);
                 dot[c & 3] = fmaf(xh[32 + c], __uint_as_float(d1[c]), dot[c & 3]);
             }
-            const float xd = (dot[0] + dot[1]) + (dot[2] + dot[3]);
+            // below the 1e-12 norm guard x^ = x / 1e-12 is not a unit vector and its
+            // derivative is the identity / 1e-12: no tangential projection there
+            const float xd = nrm > 1e-12f ? (dot[0] + dot[1]) + (dot[2] + dot[3]) : 0.0f;
             const int64_t r = static_cast<int64_t>(k * static_cast<int>(gridDim.x) +
                                                    static_cast<int>(blockIdx.x)) * kRows + row;
             if (r < n_rows) {

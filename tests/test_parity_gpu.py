@@ -202,6 +202,24 @@ def test_attn_bwd_small(dt, R, m, L):
     assert rel_l2(gv, wv) <= TOL[dt]
 
 
+# Rows below the 1e-12 norm guard (x^ = x / 1e-12, not a unit vector) and a zero row take the
+# guarded derivative; the bf16 path runs the feature map's backward on tensor cores.
+@pytest.mark.parametrize("R,m,L", [(4, 64, 200), (8, 64, 130)])
+def test_attn_bwd_guarded_rows(R, m, L):
+    w = small("bf16", R, m, L)
+    q, k, v = W.gen_qkv(w)
+    q[0, 0, 3] = W.round_bf16(q[0, 0, 3] * 1e-14)   # inputs stay exact bf16 values
+    k[0, 1, 5] = W.round_bf16(k[0, 1, 5] * 1e-14)
+    k[0, 0, 7] = 0.0
+    g = W.gen_dout(w)
+    P = params(w)
+    wq, wk, wv = O.attn_causal_bwd(q, k, v, g, P)
+    gq, gk, gv = _run_bwd(q, k, v, g, w)
+    for got, want in ((gq, wq), (gk, wk), (gv, wv)):
+        assert np.isfinite(got).all()
+        assert rel_l2(got, want) <= TOL["bf16"]
+
+
 def test_attn_bwd_single_token():
     # L = 1: the only weight is a/(a+eps) ~ 1 - eps/a, so dq and dk are O(eps/a) and come
     # from the cancellation <v, dn> + delta with delta = -<g, out>/Z.  Rounding `out` to
