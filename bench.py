@@ -144,6 +144,12 @@ def kernel_work(name, w, op):
     # kernel the rest; the row statistics read out, g, den and write [dn, delta] (bytes)
     if name == "simt_phi_bwd":
         return th * 8 * D * F, "flop", "alu"
+    # the tensor-core chunk contraction of the backward moves, per token-head, phi(q), phi(k)
+    # (bf16), v, [dn, delta], dphi(q), dphi(k) (fp32), dv and its share of the two 128-token
+    # states it reads (2 F (Dv+1) fp32 per tile)
+    if name == "tc_bwd_tile":
+        return th * (2 * 2 * F + 2 * Dv + 4 * (Dv + 1) + 2 * 4 * F + 4 * Dv) + \
+            w.B * w.H * ((w.L + 127) // 128) * 2 * F * (Dv + 1) * 4, "byte", "hbm"
     # the tensor-core phi backward is bound by its reads: x (bf16), dphi (fp32), dx (fp32)
     if name == "tc_phi_bwd":
         return th * (2 * D + 4 * F + 4 * D), "byte", "hbm"

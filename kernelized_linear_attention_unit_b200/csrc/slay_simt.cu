@@ -976,16 +976,24 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
         k_scan<<<sgrid, 256, 0, st>>>(gbw, nullptr, BH, NC, FE, 1);
     }
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    const size_t smem = sizeof(BwdSmem);
-    if ((err = cudaFuncSetAttribute(k_bwd_chunk<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    static_cast<int>(smem))) != cudaSuccess)
-        return err;
-    {
-        TraceScope trace_("simt_bwd_chunk", st);
-        k_bwd_chunk<T><<<dim3(NC, BH), NT, smem, st>>>(phq, phk, cp<T>(v), dn, sfw, gbw, dphq, dphk,
-                                                       dv, L, F);
+    if (std::is_same<T, __nv_bfloat16>::value && tc_bwd_tile_supported(F, L)) {
+        // bf16 phi: the chunk contraction on tensor cores (status word = workspace header)
+        int* status = reinterpret_cast<int*>(w - kWsHeader);
+        if ((err = tc_bwd_tile(phq, phk, v, dn, sfw, gbw, dphq, dphk, dv, BH, L, F, status, st)) !=
+            cudaSuccess)
+            return err;
+    } else {
+        const size_t smem = sizeof(BwdSmem);
+        if ((err = cudaFuncSetAttribute(k_bwd_chunk<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(smem))) != cudaSuccess)
+            return err;
+        {
+            TraceScope trace_("simt_bwd_chunk", st);
+            k_bwd_chunk<T><<<dim3(NC, BH), NT, smem, st>>>(phq, phk, cp<T>(v), dn, sfw, gbw, dphq,
+                                                           dphk, dv, L, F);
+        }
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
     }
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
     const size_t psm = sizeof(PhiBwdSmem);
     if ((err = cudaFuncSetAttribute(k_phi_bwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     static_cast<int>(psm))) != cudaSuccess)

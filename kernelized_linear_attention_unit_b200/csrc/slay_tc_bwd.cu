@@ -1,0 +1,439 @@
+// slay_tc_bwd.cu -- tensor-core chunk contraction of the causal backward (bf16 mode).
+//
+// Method: "SLAY: Geometry-Aware Spherical Linearized Attention with Yat-Kernel" (nubint.ai
+// review, "Proposed method", step 6: the linear-attention contraction); the pages give no
+// backward, so this is the derivative of out_i = phi(q_i)^T S_i / (phi(q_i)^T z_i + eps).
+// With dn_i = g_i / Z_i, delta_i = -(g_i . out_i) / Z_i and, inside a 128-token tile,
+// P_ij = phi(q_i) . phi(k_j) and c_ij = v_j . dn_i + delta_i restricted to j <= i:
+//   dphi(q_i) = sum_j c_ij phi(k_j) + S_c[:, :64] dn_i + z_c delta_i
+//   dphi(k_j) = sum_i c_ij phi(q_i) + G_c[:, :64] v_j + zg_c
+//   dv_j      = sum_i P_ij dn_i + G_c[:, :64]^T phi(k_j)
+// where [S_c | z_c] = sum over earlier tokens of phi(k) [v, 1] (the state entering the tile)
+// and [G_c | zg_c] = sum over later tokens of phi(q) [dn, delta], both from the chunk-state
+// scans (64-token chunks: tile c starts at chunk 2c and ends with chunk 2c + 1).
+//
+// Per tile (M = 128 rows, all MMAs kind::f16, fp32 accumulators in tensor memory):
+//   phase A: P = sum_s phiQ_s phiK_s^T (64-feature slices s), C0 = dn V^T;
+//            the epilogue masks them (j <= i, inside L), adds delta_i to C0 and writes bf16
+//            P~ and C~ into shared memory;
+//   phase B: dV = P~^T dn, then per slice s: dphiQ_s = C~ phiK_s + dn S_s^T,
+//            dphiK_s = C~^T phiQ_s + V G_s^T, dV += phiK_s G_s; the epilogue adds the z terms
+//            and writes dphiQ, dphiK (fp32) per slice, dV per tile.
+// The ones / delta columns never enter an MMA (their terms are rank one, added in fp32),
+// so every contraction has K a multiple of 64.  The transposed products read the same
+// shared-memory tiles as MN-major operands.
+//
+// Persistent, one CTA per SM over the (b, h, tile) items.  Warp 0 issues the MMAs, warp 9
+// the TMA loads (V, and the phi slice pairs of both phases through a ring of two), warps 1-8
+// are the epilogue (lane quadrant w % 4, column half (w - 1) / 4).  Every wait is bounded; a
+// timeout sets the workspace status word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "slay_tc.h"
+#include "slay_tc_common.cuh"
+#include "slay_tc_ptx.cuh"
+
+namespace slay {
+
+using namespace tc;
+
+namespace {
+
+constexpr int kT = 128;                  // tokens per tile
+constexpr int kTile = kT * 128;          // [128][64] bf16, 128-byte swizzle = 16 KiB
+constexpr int kSG = 64 * 128;            // [64 f][64 e] bf16 = 8 KiB
+constexpr int kE = 65;                   // state / [dn | delta] columns in the scans' layout
+constexpr int kBwThreads = 32 * 10;
+constexpr int kNumSMs = 148;
+// tensor memory: phase A P [0,128) and C0 [128,256); phase B per-slice buffers b: dphiQ at
+// 128 b, dphiK at 128 b + 64; dV at 256
+constexpr uint32_t kColP = 0, kColC = 128, kColDV = 256;
+
+enum {
+    BW_VF = 0, BW_VE, BW_PF0, BW_PF1, BW_PE0, BW_PE1, BW_DNF, BW_DNE, BW_PCF, BW_PCTF, BW_PCTE,
+    BW_SGF0, BW_SGF1, BW_SGE0, BW_SGE1, BW_DQF0, BW_DQF1, BW_DQE0, BW_DQE1, BW_DVF, BW_DVE,
+    BW_NUM
+};
+
+struct BwLayout {
+    uint32_t phi, pt, ct, dn, v, sg, bar, tmem, total;
+};
+
+__host__ __device__ inline BwLayout bw_layout()
+{
+    BwLayout l;
+    l.phi = 0;                    // 2 slots x (phiQ slice, phiK slice)
+    l.pt = l.phi + 4 * kTile;     // P~ as two column halves [128 i][64 j]
+    l.ct = l.pt + 2 * kTile;      // C~ likewise
+    l.dn = l.ct + 2 * kTile;      // dn [128 i][64 e]
+    l.v = l.dn + kTile;           // V [128 j][64 e]
+    l.sg = l.v + kTile;           // 2 buffers x (S_s, G_s) [64 f][64 e]
+    l.bar = l.sg + 4 * kSG;
+    l.tmem = l.bar + BW_NUM * 8;
+    l.total = l.tmem + 16;
+    return l;
+}
+
+struct BwParams {
+    int L, F, ntiles, nitems, NC;
+};
+
+// 128-byte swizzled [rows][64 bf16] tile: 16-byte chunk c of row r at chunk c ^ (r & 7)
+__device__ __forceinline__ void st_row32(uint32_t tile, uint32_t row, int half, const uint32_t (&pk)[16])
+{
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+        st_shared_v4(tile + sw128_off(row, 4 * half + c), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
+                     pk[4 * c + 3]);
+}
+
+__global__ void __launch_bounds__(kBwThreads, 1)
+k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+              const __grid_constant__ CUtensorMap tmv, const float* __restrict__ dn,
+              const float* __restrict__ sfw, const float* __restrict__ gbw,
+              float* __restrict__ dphq, float* __restrict__ dphk, float* __restrict__ dv,
+              BwParams bp, int* err)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* sm = aligned_smem(smem_raw);
+    const BwLayout Lo = bw_layout();
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Lo.bar);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + Lo.tmem);
+    const uint32_t sbase = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int ns = bp.F / 64;
+
+    if (warp == 0) {
+        tmem_alloc(tslot, 512);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        for (int i = 0; i < BW_NUM; ++i) mbar_init(&bar[i], 1);
+        const int warp_counted[7] = {BW_DNF, BW_PCTF, BW_SGF0, BW_SGF1, BW_DQE0, BW_DQE1, BW_DVE};
+        for (int i = 0; i < 7; ++i) mbar_init(&bar[warp_counted[i]], 8);   // one arrival per epilogue warp
+        mbar_fence_init();
+        tma_prefetch_desc(&tmq);
+        tma_prefetch_desc(&tmk);
+        tma_prefetch_desc(&tmv);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+    Waiter wt;
+    // waits on the k-th completion (k >= 0) of a barrier
+    auto wait_k = [&](int b, int k) {
+        uint32_t ph = static_cast<uint32_t>(k & 1);
+        wt.wait(&bar[b], ph);
+    };
+
+    if (warp == 9) {
+        // ---------------------------------------------------------------- TMA loads
+        if (lane == 0) {
+            int use = 0, it = 0;   // phi slice-pair loads so far; items so far
+            for (int item = blockIdx.x; item < bp.nitems && wt.ok; item += gridDim.x, ++it) {
+                const int bh = item / bp.ntiles, t = item - bh * bp.ntiles;
+                if (it >= 1) wait_k(BW_VE, it - 1);
+                mbar_arrive_expect_tx(&bar[BW_VF], kTile);
+                tma_load_3d(sm + Lo.v, &tmv, &bar[BW_VF], 0, t * kT, bh);
+                for (int u = 0; u < 2 * ns; ++u, ++use) {   // phase A slices, then phase B
+                    const int s = u < ns ? u : u - ns, slot = use & 1;
+                    if (use >= 2) wait_k(BW_PE0 + slot, (use >> 1) - 1);
+                    mbar_arrive_expect_tx(&bar[BW_PF0 + slot], 2 * kTile);
+                    unsigned char* dst = sm + Lo.phi + slot * 2 * kTile;
+                    tma_load_3d(dst, &tmq, &bar[BW_PF0 + slot], 64 * s, t * kT, bh);
+                    tma_load_3d(dst + kTile, &tmk, &bar[BW_PF0 + slot], 64 * s, t * kT, bh);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 0) {
+        // ---------------------------------------------------------------- MMA issue
+        if (lane == 0) {
+            constexpr uint32_t idKK128 = idesc_bf16(128, 128, 0, 0);
+            constexpr uint32_t idKK64 = idesc_bf16(128, 64, 0, 0);
+            constexpr uint32_t idKM64 = idesc_bf16(128, 64, 0, 1);   // B MN-major
+            constexpr uint32_t idMM64 = idesc_bf16(128, 64, 1, 1);   // A and B MN-major
+            const uint64_t dphi0 = sdesc(sbase + Lo.phi, 16, 1024, kLayoutSW128);
+            const uint64_t dct_k = sdesc(sbase + Lo.ct, 16, 1024, kLayoutSW128);
+            const uint64_t dpt_m = sdesc(sbase + Lo.pt, kTile, 1024, kLayoutSW128);   // M = 128 over both halves
+            const uint64_t dct_m = sdesc(sbase + Lo.ct, kTile, 1024, kLayoutSW128);
+            const uint64_t ddn = sdesc(sbase + Lo.dn, 16, 1024, kLayoutSW128);
+            const uint64_t dvv = sdesc(sbase + Lo.v, 16, 1024, kLayoutSW128);
+            const uint64_t dsg0 = sdesc(sbase + Lo.sg, 16, 1024, kLayoutSW128);
+            int use = 0, gs = 0, it = 0;   // phi uses, slice-accumulator uses, items
+            for (int item = blockIdx.x; item < bp.nitems && wt.ok; item += gridDim.x, ++it) {
+                wait_k(BW_VF, it);
+                wait_k(BW_DNF, it);
+                // P / C0 overwrite the slice buffers of the previous item: both read
+                if (gs >= 1) wait_k(BW_DQE0 + ((gs - 1) & 1), (gs - 1) >> 1);
+                if (gs >= 2) wait_k(BW_DQE0 + ((gs - 2) & 1), (gs - 2) >> 1);
+                tc_fence_after();
+                // phase A
+                for (int s = 0; s < ns; ++s, ++use) {
+                    const int slot = use & 1;
+                    wait_k(BW_PF0 + slot, use >> 1);
+                    tc_fence_after();
+                    const uint64_t dq = dphi0 + ((slot * 2 * kTile) >> 4), dk = dq + (kTile >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_bf16(tmem + kColP, dq + 2 * kk, dk + 2 * kk, idKK128, (s > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&bar[BW_PE0 + slot]);
+                }
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_bf16(tmem + kColC, ddn + 2 * kk, dvv + 2 * kk, idKK128, kk > 0 ? 1u : 0u);
+                umma_commit(&bar[BW_PCF]);
+                // phase B
+                wait_k(BW_PCTF, it);
+                if (it >= 1) wait_k(BW_DVE, it - 1);
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)   // dV = P~^T dn (K = i)
+                    umma_bf16(tmem + kColDV, dpt_m + 128 * kk, ddn + 128 * kk, idMM64, kk > 0 ? 1u : 0u);
+                for (int s = 0; s < ns; ++s, ++use, ++gs) {
+                    // S/G buffer of slice k = it ns + s is k & 1 (gs == k: one per slice)
+                    const int slot = use & 1, b = gs & 1, sb = gs & 1;
+                    wait_k(BW_PF0 + slot, use >> 1);
+                    wait_k(BW_SGF0 + sb, gs >> 1);
+                    if (gs >= 2) wait_k(BW_DQE0 + b, (gs - 2) >> 1);
+                    tc_fence_after();
+                    const uint64_t dq = dphi0 + ((slot * 2 * kTile) >> 4), dk = dq + (kTile >> 4);
+                    const uint64_t ds = dsg0 + ((sb * 2 * kSG) >> 4), dg = ds + (kSG >> 4);
+                    const uint32_t cq = tmem + 128u * b, ck = cq + 64;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)   // dphiQ_s = C~ phiK_s (K = j)
+                        umma_bf16(cq, dct_k + (kk >> 2) * (kTile >> 4) + 2 * (kk & 3), dk + 128 * kk,
+                                  idKM64, kk > 0 ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)   // += dn S_s^T (K = e)
+                        umma_bf16(cq, ddn + 2 * kk, ds + 2 * kk, idKK64, 1u);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)   // dphiK_s = C~^T phiQ_s (K = i)
+                        umma_bf16(ck, dct_m + 128 * kk, dq + 128 * kk, idMM64, kk > 0 ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)   // += V G_s^T (K = e)
+                        umma_bf16(ck, dvv + 2 * kk, dg + 2 * kk, idKK64, 1u);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)   // dV += phiK_s G_s (K = f)
+                        umma_bf16(tmem + kColDV, dk + 2 * kk, dg + 128 * kk, idKM64, 1u);
+                    umma_commit(&bar[BW_DQF0 + b]);
+                    umma_commit(&bar[BW_SGE0 + sb]);
+                    umma_commit(&bar[BW_PE0 + slot]);
+                }
+                umma_commit(&bar[BW_DVF]);
+                umma_commit(&bar[BW_PCTE]);
+                umma_commit(&bar[BW_DNE]);
+                umma_commit(&bar[BW_VE]);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------------- epilogue
+        const int ew = warp - 1, q = warp & 3, half = ew >> 2, et = tid - 32;   // et 0..255
+        const uint32_t row = 32u * q + lane;
+        const uint32_t trow = tmem + ((32u * q) << 16);
+        int it = 0, gs = 0;
+        for (int item = blockIdx.x; item < bp.nitems && wt.ok; item += gridDim.x, ++it) {
+            const int bh = item / bp.ntiles, t = item - bh * bp.ntiles;
+            const int i_abs = t * kT + static_cast<int>(row);   // this thread's token
+            const bool valid = i_abs < bp.L;
+            const int64_t grow = static_cast<int64_t>(bh) * bp.L + i_abs;
+            const int c_in = 2 * t, c_out = 2 * t + 1 < bp.NC ? 2 * t + 1 : bp.NC - 1;
+            const float* Sb = sfw + (static_cast<int64_t>(bh) * bp.NC + c_in) * bp.F * kE;
+            const float* Gb = gbw + (static_cast<int64_t>(bh) * bp.NC + c_out) * bp.F * kE;
+            // dn (bf16 operand, this warp's 32 columns) and delta
+            if (it >= 1) wait_k(BW_DNE, it - 1);
+            float delta = 0.0f;
+            {
+                uint32_t pk[16];
+                const float* src = dn + grow * kE + 32 * half;
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    pk[c] = valid ? pack_bf16(src[2 * c], src[2 * c + 1]) : 0u;
+                if (valid) delta = dn[grow * kE + 64];
+                st_row32(sbase + Lo.dn, row, half, pk);
+            }
+            fence_async_smem();
+            warp_arrive(&bar[BW_DNF]);
+            // masked P~ and C~ (this warp's half of the columns j)
+            wait_k(BW_PCF, it);
+            tc_fence_after();
+            {
+                uint32_t pr[32], p2[32], cr[32], c2[32];
+                tmem_ld32(trow + kColP + 64 * half, pr);
+                tmem_ld32(trow + kColP + 64 * half + 32, p2);
+                tmem_ld32(trow + kColC + 64 * half, cr);
+                tmem_ld32(trow + kColC + 64 * half + 32, c2);
+                tmem_wait_ld();
+                reg_fence(pr);
+                reg_fence(p2);
+                reg_fence(cr);
+                reg_fence(c2);
+                if (it >= 1) wait_k(BW_PCTE, it - 1);
+                uint32_t pk[16], ck[16];
+                const int j0 = t * kT + 64 * half;   // absolute token of column 64 half
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const uint32_t* P = hh ? p2 : pr;
+                    const uint32_t* Cc = hh ? c2 : cr;
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const int jl = 64 * half + 32 * hh + 2 * c;     // column within the tile
+                        const bool k0 = valid && jl <= static_cast<int>(row) && j0 + 32 * hh + 2 * c < bp.L;
+                        const bool k1 = valid && jl + 1 <= static_cast<int>(row) && j0 + 32 * hh + 2 * c + 1 < bp.L;
+                        pk[c] = pack_bf16(k0 ? __uint_as_float(P[2 * c]) : 0.0f,
+                                          k1 ? __uint_as_float(P[2 * c + 1]) : 0.0f);
+                        ck[c] = pack_bf16(k0 ? __uint_as_float(Cc[2 * c]) + delta : 0.0f,
+                                          k1 ? __uint_as_float(Cc[2 * c + 1]) + delta : 0.0f);
+                    }
+                    // column chunk 4 hh .. of the half tile
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        st_shared_v4(sbase + Lo.pt + half * kTile + sw128_off(row, 4 * hh + c),
+                                     pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                        st_shared_v4(sbase + Lo.ct + half * kTile + sw128_off(row, 4 * hh + c),
+                                     ck[4 * c], ck[4 * c + 1], ck[4 * c + 2], ck[4 * c + 3]);
+                    }
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            warp_arrive(&bar[BW_PCTF]);
+            // per slice: S_s, G_s as bf16 operands (slice s), then the outputs of slice s - 1
+            auto write_slice = [&](int s, int b) {
+                wait_k(BW_DQF0 + b, gs >> 1);
+                tc_fence_after();
+                uint32_t qa[32], ka[32];
+                tmem_ld32(trow + 128u * b + 32 * half, qa);
+                tmem_ld32(trow + 128u * b + 64 + 32 * half, ka);
+                tmem_wait_ld();
+                reg_fence(qa);
+                reg_fence(ka);
+                tc_fence_before();
+                warp_arrive(&bar[BW_DQE0 + b]);
+                ++gs;
+                if (!valid) return;
+                const int f0 = 64 * s + 32 * half;
+                float4* oq = reinterpret_cast<float4*>(dphq + grow * bp.F + f0);
+                float4* ok = reinterpret_cast<float4*>(dphk + grow * bp.F + f0);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    float zq[4], zk[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        zq[e] = Sb[static_cast<int64_t>(f0 + 4 * c + e) * kE + 64];
+                        zk[e] = Gb[static_cast<int64_t>(f0 + 4 * c + e) * kE + 64];
+                    }
+                    oq[c] = make_float4(fmaf(delta, zq[0], __uint_as_float(qa[4 * c])),
+                                        fmaf(delta, zq[1], __uint_as_float(qa[4 * c + 1])),
+                                        fmaf(delta, zq[2], __uint_as_float(qa[4 * c + 2])),
+                                        fmaf(delta, zq[3], __uint_as_float(qa[4 * c + 3])));
+                    ok[c] = make_float4(__uint_as_float(ka[4 * c]) + zk[0], __uint_as_float(ka[4 * c + 1]) + zk[1],
+                                        __uint_as_float(ka[4 * c + 2]) + zk[2], __uint_as_float(ka[4 * c + 3]) + zk[3]);
+                }
+            };
+            for (int s = 0; s < ns; ++s) {
+                const int k = it * ns + s, sb = k & 1;
+                if (k >= 2) wait_k(BW_SGE0 + sb, (k >> 1) - 1);
+                {   // thread et converts 16 e of row f = et / 4 of S_s and of G_s
+                    const int f = et >> 2, e0 = 16 * (et & 3);
+                    const float* sr = Sb + static_cast<int64_t>(64 * s + f) * kE + e0;
+                    const float* gr = Gb + static_cast<int64_t>(64 * s + f) * kE + e0;
+                    uint32_t a8[8], g8[8];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        a8[c] = pack_bf16(sr[2 * c], sr[2 * c + 1]);
+                        g8[c] = pack_bf16(gr[2 * c], gr[2 * c + 1]);
+                    }
+                    const uint32_t ts = sbase + Lo.sg + sb * 2 * kSG, tg = ts + kSG;
+                    const int ch = 2 * (et & 3);
+                    st_shared_v4(ts + sw128_off(f, ch), a8[0], a8[1], a8[2], a8[3]);
+                    st_shared_v4(ts + sw128_off(f, ch + 1), a8[4], a8[5], a8[6], a8[7]);
+                    st_shared_v4(tg + sw128_off(f, ch), g8[0], g8[1], g8[2], g8[3]);
+                    st_shared_v4(tg + sw128_off(f, ch + 1), g8[4], g8[5], g8[6], g8[7]);
+                }
+                fence_async_smem();
+                warp_arrive(&bar[BW_SGF0 + sb]);
+                if (s >= 1) write_slice(s - 1, gs & 1);
+            }
+            write_slice(ns - 1, gs & 1);
+            // dV
+            wait_k(BW_DVF, it);
+            tc_fence_after();
+            {
+                uint32_t va[32];
+                tmem_ld32(trow + kColDV + 32 * half, va);
+                tmem_wait_ld();
+                reg_fence(va);
+                tc_fence_before();
+                warp_arrive(&bar[BW_DVE]);
+                if (valid) {
+                    float4* o = reinterpret_cast<float4*>(dv + grow * 64 + 32 * half);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        o[c] = make_float4(__uint_as_float(va[4 * c]), __uint_as_float(va[4 * c + 1]),
+                                           __uint_as_float(va[4 * c + 2]), __uint_as_float(va[4 * c + 3]));
+                }
+            }
+        }
+    }
+    wt.report(err);
+    drain_after_failure(wt.ok);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// [BH][L][cols] bf16 viewed as a 3-D tensor, boxes of 64 columns x 128 tokens, 128-byte
+// swizzle; rows past L read as zero.
+bool map_seq(CUtensorMap* m, const void* base, int cols, int L, int BH)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(L),
+                                static_cast<cuuint64_t>(BH)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 2,
+                                   static_cast<cuuint64_t>(L) * cols * 2};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kT), 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool tc_bwd_tile_supported(int F, int L)
+{
+    return F % 64 == 0 && F >= 64 && F <= 512 && L > 0 && bw_layout().total + 1024 <= 232448;
+}
+
+cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const float* dn,
+                        const float* sfw, const float* gbw, float* dphq, float* dphk, float* dv,
+                        int BH, int L, int F, int* err, cudaStream_t st)
+{
+    if (!tc_bwd_tile_supported(F, L)) return cudaErrorNotSupported;
+    CUtensorMap mq, mk, mv;
+    if (!map_seq(&mq, phq, F, L, BH) || !map_seq(&mk, phk, F, L, BH) || !map_seq(&mv, v, 64, L, BH))
+        return cudaErrorInvalidValue;
+    BwParams bp;
+    bp.L = L;
+    bp.F = F;
+    bp.ntiles = (L + kT - 1) / kT;
+    bp.nitems = BH * bp.ntiles;
+    bp.NC = (L + 63) / 64;
+    const size_t smem = bw_layout().total + 1024;
+    cudaError_t e = cudaFuncSetAttribute(k_tc_bwd_tile, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const int grid = bp.nitems < kNumSMs ? bp.nitems : kNumSMs;
+    TraceScope trace_("tc_bwd_tile", st);
+    k_tc_bwd_tile<<<grid, kBwThreads, smem, st>>>(mq, mk, mv, dn, sfw, gbw, dphq, dphk, dv, bp, err);
+    return cudaGetLastError();
+}
+
+}  // namespace slay

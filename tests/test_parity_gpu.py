@@ -189,7 +189,7 @@ def _run_bwd(q, k, v, g, w):
 
 @pytest.mark.parametrize("dt,R,m,L", [("f32", 2, 16, 100), ("f32", 4, 64, 130),
                                       ("bf16", 4, 64, 150), ("bf16", 8, 64, 64),
-                                      ("bf16", 2, 16, 65)])
+                                      ("bf16", 2, 16, 65), ("bf16", 3, 64, 300)])
 def test_attn_bwd_small(dt, R, m, L):
     w = small(dt, R, m, L)
     q, k, v = W.gen_qkv(w)
@@ -234,6 +234,19 @@ def test_attn_bwd_single_token():
     assert rel_l2(gv, wv) <= 1e-5
     assert rel_l2(gq, wq) <= 1e-3
     assert rel_l2(gk, wk) <= 1e-3
+
+
+def test_attn_bwd_many_items():
+    # 160 sequences of one tile each: on 148 SMs some CTAs take two (b, h, tile) items in turn
+    w = W.Workload("items", B=1, H=160, L=100, R=4, m=64, dtype="bf16", data_seed=23)
+    q, k, v = W.gen_qkv(w)
+    g = W.gen_dout(w)
+    P = params(w)
+    wq, wk, wv = O.attn_causal_bwd(q, k, v, g, P)
+    gq, gk, gv = _run_bwd(q, k, v, g, w)
+    assert rel_l2(gq, wq) <= TOL["bf16"]
+    assert rel_l2(gk, wk) <= TOL["bf16"]
+    assert rel_l2(gv, wv) <= TOL["bf16"]
 
 
 def test_attn_bwd_full_size_sampled():
