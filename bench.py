@@ -103,7 +103,8 @@ def kernel_work(name, w, op):
     # each kernel per chunk, whose sums meet before the division.  A launch gets its
     # chunk's share; the masked P.V term (C+1) Dv, repeated per chunk, counts once.
     nch = 1 if F <= 256 else (F // 256 if F % 256 == 0 else F // 128)
-    if name.startswith("tc_") and name != "tc_feature_map":
+    if name in ("tc_causal_out", "tc_qphi_out", "tc_causal_state", "tc_kphi_state",
+                "tc_bidir_out", "tc_bidir_state"):
         F = F // nch
     if name in ("tc_causal_out", "tc_qphi_out"):
         return (th * (4 * D * F + 4 * F * Dv + (C_CHUNK + 1) * F) +
@@ -147,6 +148,11 @@ def kernel_work(name, w, op):
     # the tensor-core chunk contraction of the backward moves, per token-head, phi(q), phi(k)
     # (bf16), v, [dn, delta], dphi(q), dphi(k) (fp32), dv and its share of the two 128-token
     # states it reads (2 F (Dv+1) fp32 per tile)
+    # the backward's per-tile sums read phi(q), phi(k), v, [dn, delta] and write two fp32
+    # [F][Dv+1] sums per 128-token tile
+    if name == "tc_bwd_states":
+        return th * (2 * 2 * F + 2 * Dv + 4 * (Dv + 1)) + \
+            w.B * w.H * ((w.L + 127) // 128) * 2 * F * (Dv + 1) * 4, "byte", "hbm"
     if name == "tc_bwd_tile":
         return th * (2 * 2 * F + 2 * Dv + 4 * (Dv + 1) + 2 * 4 * F + 4 * Dv) + \
             w.B * w.H * ((w.L + 127) // 128) * 2 * F * (Dv + 1) * 4, "byte", "hbm"

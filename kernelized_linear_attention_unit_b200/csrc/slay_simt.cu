@@ -954,31 +954,38 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
             cp<T>(out), den, cp<T>(dout), dn, rows, eps);
     }
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    const dim3 sg((F + C - 1) / C, NC, BH);
-    {
-        TraceScope trace_("simt_chunk_state", st);
-        k_chunk_state<T, T><<<sg, NT, 0, st>>>(phk, cp<T>(v), kD, sfw, L, F);
+    // bf16 phi: states, contraction on tensor cores over 128-token tiles; else 64-token chunks
+    const bool tcb = std::is_same<T, __nv_bfloat16>::value && tc_bwd_tile_supported(F, L);
+    const int NS = tcb ? (L + 127) / 128 : NC;   // state blocks per sequence
+    int* status = reinterpret_cast<int*>(w - kWsHeader);
+    if (tcb) {
+        if ((err = tc_bwd_states(phq, phk, v, dn, sfw, gbw, BH, L, F, status, st)) != cudaSuccess)
+            return err;
+    } else {
+        const dim3 sg((F + C - 1) / C, NC, BH);
+        {
+            TraceScope trace_("simt_chunk_state", st);
+            k_chunk_state<T, T><<<sg, NT, 0, st>>>(phk, cp<T>(v), kD, sfw, L, F);
+        }
+        {
+            TraceScope trace_("simt_chunk_state", st);
+            k_chunk_state<float, T><<<sg, NT, 0, st>>>(phq, dn, E, gbw, L, F);
+        }
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
     }
-    {
-        TraceScope trace_("simt_chunk_state", st);
-        k_chunk_state<float, T><<<sg, NT, 0, st>>>(phq, dn, E, gbw, L, F);
-    }
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
     const int FE = F * E;
     const int64_t nth = static_cast<int64_t>(BH) * FE;
     const unsigned sgrid = static_cast<unsigned>((nth + 255) / 256);
     {
         TraceScope trace_("simt_scan", st);
-        k_scan<<<sgrid, 256, 0, st>>>(sfw, nullptr, BH, NC, FE, 0);
+        k_scan<<<sgrid, 256, 0, st>>>(sfw, nullptr, BH, NS, FE, 0);
     }
     {
         TraceScope trace_("simt_scan", st);
-        k_scan<<<sgrid, 256, 0, st>>>(gbw, nullptr, BH, NC, FE, 1);
+        k_scan<<<sgrid, 256, 0, st>>>(gbw, nullptr, BH, NS, FE, 1);
     }
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    if (std::is_same<T, __nv_bfloat16>::value && tc_bwd_tile_supported(F, L)) {
-        // bf16 phi: the chunk contraction on tensor cores (status word = workspace header)
-        int* status = reinterpret_cast<int*>(w - kWsHeader);
+    if (tcb) {
         if ((err = tc_bwd_tile(phq, phk, v, dn, sfw, gbw, dphq, dphk, dv, BH, L, F, status, st)) !=
             cudaSuccess)
             return err;

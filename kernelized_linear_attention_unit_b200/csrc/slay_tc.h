@@ -30,9 +30,12 @@ cudaError_t tc_feature_map(const void* x, void* phi, int64_t n, const Params& P,
 bool tc_phi_bwd_supported(int D, int R, int m, int64_t n_rows);
 cudaError_t tc_phi_bwd(const void* x, const float* dphi, float* dx, int64_t n, const Params& P,
                        cudaStream_t st);
-// Chunk contraction of the causal backward on tensor cores (bf16 phi and v, fp32 [dn | delta]
-// rows and the chunk-state scans of 64-token chunks) -> fp32 dphi(q), dphi(k), dv.
+// Causal backward on tensor cores over 128-token tiles (bf16 phi and v, fp32 [dn | delta] rows):
+// the per-tile sums phi(k)^T [v, 1] and phi(q)^T [dn, delta] ([BH][tiles][F][65] fp32), and,
+// from their exclusive forward / reverse scans, the contraction -> fp32 dphi(q), dphi(k), dv.
 bool tc_bwd_tile_supported(int F, int L);
+cudaError_t tc_bwd_states(const void* phq, const void* phk, const void* v, const float* dn,
+                          float* st_s, float* st_g, int BH, int L, int F, int* err, cudaStream_t st);
 cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const float* dn,
                         const float* sfw, const float* gbw, float* dphq, float* dphk, float* dv,
                         int BH, int L, int F, int* err, cudaStream_t st);

@@ -9,8 +9,8 @@
 //   dphi(k_j) = sum_i c_ij phi(q_i) + G_c[:, :64] v_j + zg_c
 //   dv_j      = sum_i P_ij dn_i + G_c[:, :64]^T phi(k_j)
 // where [S_c | z_c] = sum over earlier tokens of phi(k) [v, 1] (the state entering the tile)
-// and [G_c | zg_c] = sum over later tokens of phi(q) [dn, delta], both from the chunk-state
-// scans (64-token chunks: tile c starts at chunk 2c and ends with chunk 2c + 1).
+// and [G_c | zg_c] = sum over later tokens of phi(q) [dn, delta]: the exclusive forward and
+// reverse scans of the per-tile sums that k_tc_bwd_states computes.
 //
 // Per tile (M = 128 rows, all MMAs kind::f16, fp32 accumulators in tensor memory):
 //   phase A: P = sum_s phiQ_s phiK_s^T (64-feature slices s), C0 = dn V^T;
@@ -78,7 +78,7 @@ __host__ __device__ inline BwLayout bw_layout()
 }
 
 struct BwParams {
-    int L, F, ntiles, nitems, NC;
+    int L, F, ntiles, nitems;
 };
 
 // 128-byte swizzled [rows][64 bf16] tile: 16-byte chunk c of row r at chunk c ^ (r & 7)
@@ -242,9 +242,8 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
             const int i_abs = t * kT + static_cast<int>(row);   // this thread's token
             const bool valid = i_abs < bp.L;
             const int64_t grow = static_cast<int64_t>(bh) * bp.L + i_abs;
-            const int c_in = 2 * t, c_out = 2 * t + 1 < bp.NC ? 2 * t + 1 : bp.NC - 1;
-            const float* Sb = sfw + (static_cast<int64_t>(bh) * bp.NC + c_in) * bp.F * kE;
-            const float* Gb = gbw + (static_cast<int64_t>(bh) * bp.NC + c_out) * bp.F * kE;
+            const float* Sb = sfw + (static_cast<int64_t>(bh) * bp.ntiles + t) * bp.F * kE;
+            const float* Gb = gbw + (static_cast<int64_t>(bh) * bp.ntiles + t) * bp.F * kE;
             // dn (bf16 operand, this warp's 32 columns) and delta
             if (it >= 1) wait_k(BW_DNE, it - 1);
             float delta = 0.0f;
@@ -320,13 +319,15 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
                 const int f0 = 64 * s + 32 * half;
                 float4* oq = reinterpret_cast<float4*>(dphq + grow * bp.F + f0);
                 float4* ok = reinterpret_cast<float4*>(dphk + grow * bp.F + f0);
+                const float* zs = Sb + 64 * static_cast<int64_t>(bp.F);   // [e = 64][f]
+                const float* zg = Gb + 64 * static_cast<int64_t>(bp.F);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     float zq[4], zk[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        zq[e] = Sb[static_cast<int64_t>(f0 + 4 * c + e) * kE + 64];
-                        zk[e] = Gb[static_cast<int64_t>(f0 + 4 * c + e) * kE + 64];
+                        zq[e] = zs[f0 + 4 * c + e];
+                        zk[e] = zg[f0 + 4 * c + e];
                     }
                     oq[c] = make_float4(fmaf(delta, zq[0], __uint_as_float(qa[4 * c])),
                                         fmaf(delta, zq[1], __uint_as_float(qa[4 * c + 1])),
@@ -339,18 +340,21 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
             for (int s = 0; s < ns; ++s) {
                 const int k = it * ns + s, sb = k & 1;
                 if (k >= 2) wait_k(BW_SGE0 + sb, (k >> 1) - 1);
-                {   // thread et converts 16 e of row f = et / 4 of S_s and of G_s
-                    const int f = et >> 2, e0 = 16 * (et & 3);
-                    const float* sr = Sb + static_cast<int64_t>(64 * s + f) * kE + e0;
-                    const float* gr = Gb + static_cast<int64_t>(64 * s + f) * kE + e0;
+                {   // thread et converts 16 e of feature f = et % 64 of S_s and of G_s (the
+                    // states are e-major: a warp's loads cover 32 consecutive features)
+                    const int f = et & 63, e0 = 16 * (et >> 6);
+                    const float* sr = Sb + static_cast<int64_t>(e0) * bp.F + 64 * s + f;
+                    const float* gr = Gb + static_cast<int64_t>(e0) * bp.F + 64 * s + f;
                     uint32_t a8[8], g8[8];
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
-                        a8[c] = pack_bf16(sr[2 * c], sr[2 * c + 1]);
-                        g8[c] = pack_bf16(gr[2 * c], gr[2 * c + 1]);
+                        a8[c] = pack_bf16(sr[(2 * c) * static_cast<int64_t>(bp.F)],
+                                          sr[(2 * c + 1) * static_cast<int64_t>(bp.F)]);
+                        g8[c] = pack_bf16(gr[(2 * c) * static_cast<int64_t>(bp.F)],
+                                          gr[(2 * c + 1) * static_cast<int64_t>(bp.F)]);
                     }
                     const uint32_t ts = sbase + Lo.sg + sb * 2 * kSG, tg = ts + kSG;
-                    const int ch = 2 * (et & 3);
+                    const int ch = 2 * (et >> 6);
                     st_shared_v4(ts + sw128_off(f, ch), a8[0], a8[1], a8[2], a8[3]);
                     st_shared_v4(ts + sw128_off(f, ch + 1), a8[4], a8[5], a8[6], a8[7]);
                     st_shared_v4(tg + sw128_off(f, ch), g8[0], g8[1], g8[2], g8[3]);
@@ -388,6 +392,207 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
+// ------------------------------------------------------------------ tile states
+// Per 128-token tile t of sequence bh: st_s[bh][t][e][f] = sum_{j in t} phi(k_j)_f [v_j, 1]_e
+// and st_g[bh][t][e][f] = sum_{i in t} phi(q_i)_f [dn_i, delta_i]_e (fp32, e = 64 the last
+// row; e-major so that a warp's 32 features store contiguously), the inputs of the
+// exclusive scans (element-wise over a tile's block) that give the contraction S_c and G_c.
+// Per item and 128-feature block mb: S = phiK_mb^T [V | 1] and G = phiQ_mb^T [dn | delta]
+// (M = 128 features, N = 80, K = 128 tokens), phi read as an MN-major A operand (two 64-
+// feature tiles), the extra column through a second 64-wide tile at the operand's leading
+// byte offset: constant ones for [V | 1], delta_i in every column for [dn | delta].
+// Warp 0 issues the MMAs, warp 9 the TMA loads, warps 1-8 convert [dn | delta] to bf16 and
+// write the sums (lane quadrant w % 4 = 32 features, half (w - 1) / 4 of the columns).
+constexpr int kStThreads = 32 * 10;
+
+enum {
+    ST_VF = 0, ST_VE, ST_PF0, ST_PF1, ST_PE0, ST_PE1, ST_YF, ST_YE, ST_DF0, ST_DF1, ST_DE0, ST_DE1,
+    ST_NUM
+};
+
+struct StLayout {
+    uint32_t phi, v, ones, dn, dl, bar, tmem, total;
+};
+
+__host__ __device__ inline StLayout st_layout()
+{
+    StLayout l;
+    l.phi = 0;                   // 2 slots x (phiQ 2 tiles, phiK 2 tiles) of one feature block
+    l.v = l.phi + 8 * kTile;
+    l.ones = l.v + kTile;        // right after V: [V | 1] at LBO = kTile
+    l.dn = l.ones + kTile;
+    l.dl = l.dn + kTile;         // right after dn: [dn | delta] at LBO = kTile
+    l.bar = l.dl + kTile;
+    l.tmem = l.bar + ST_NUM * 8;
+    l.total = l.tmem + 16;
+    return l;
+}
+
+__global__ void __launch_bounds__(kStThreads, 1)
+k_tc_bwd_states(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                const __grid_constant__ CUtensorMap tmv, const float* __restrict__ dn,
+                float* __restrict__ st_s, float* __restrict__ st_g, BwParams bp, int* err)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* sm = aligned_smem(smem_raw);
+    const StLayout Lo = st_layout();
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Lo.bar);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + Lo.tmem);
+    const uint32_t sbase = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nb = bp.F / 128;                  // 128-feature blocks (jobs per item)
+
+    if (warp == 0) {
+        tmem_alloc(tslot, 512);
+        tmem_relinquish();
+    }
+    {   // bf16 ones (the extra column of [V | 1], replicated over the tile)
+        uint32_t* p = reinterpret_cast<uint32_t*>(sm + Lo.ones);
+        for (int i = tid; i < kTile / 4; i += blockDim.x) p[i] = 0x3F803F80u;
+    }
+    if (tid == 0) {
+        for (int i = 0; i < ST_NUM; ++i) mbar_init(&bar[i], 1);
+        mbar_init(&bar[ST_YF], 8);
+        mbar_init(&bar[ST_DE0], 8);
+        mbar_init(&bar[ST_DE1], 8);
+        mbar_fence_init();
+        tma_prefetch_desc(&tmq);
+        tma_prefetch_desc(&tmk);
+        tma_prefetch_desc(&tmv);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+    Waiter wt;
+    auto wait_k = [&](int b, int k) {
+        uint32_t ph = static_cast<uint32_t>(k & 1);
+        wt.wait(&bar[b], ph);
+    };
+
+    if (warp == 9) {
+        if (lane == 0) {
+            int use = 0, it = 0;
+            for (int item = blockIdx.x; item < bp.nitems && wt.ok; item += gridDim.x, ++it) {
+                const int bh = item / bp.ntiles, t = item - bh * bp.ntiles;
+                if (it >= 1) wait_k(ST_VE, it - 1);
+                mbar_arrive_expect_tx(&bar[ST_VF], kTile);
+                tma_load_3d(sm + Lo.v, &tmv, &bar[ST_VF], 0, t * kT, bh);
+                for (int mb = 0; mb < nb; ++mb, ++use) {
+                    const int slot = use & 1;
+                    if (use >= 2) wait_k(ST_PE0 + slot, (use >> 1) - 1);
+                    mbar_arrive_expect_tx(&bar[ST_PF0 + slot], 4 * kTile);
+                    unsigned char* dst = sm + Lo.phi + slot * 4 * kTile;
+                    tma_load_3d(dst, &tmq, &bar[ST_PF0 + slot], 128 * mb, t * kT, bh);
+                    tma_load_3d(dst + kTile, &tmq, &bar[ST_PF0 + slot], 128 * mb + 64, t * kT, bh);
+                    tma_load_3d(dst + 2 * kTile, &tmk, &bar[ST_PF0 + slot], 128 * mb, t * kT, bh);
+                    tma_load_3d(dst + 3 * kTile, &tmk, &bar[ST_PF0 + slot], 128 * mb + 64, t * kT, bh);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 0) {
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16(128, 80, 1, 1);   // A, B MN-major
+            const uint64_t dphi0 = sdesc(sbase + Lo.phi, kTile, 1024, kLayoutSW128);
+            const uint64_t dvb = sdesc(sbase + Lo.v, Lo.ones - Lo.v, 1024, kLayoutSW128);
+            const uint64_t dyb = sdesc(sbase + Lo.dn, Lo.dl - Lo.dn, 1024, kLayoutSW128);
+            int use = 0, it = 0, job = 0;
+            for (int item = blockIdx.x; item < bp.nitems && wt.ok; item += gridDim.x, ++it) {
+                wait_k(ST_VF, it);
+                wait_k(ST_YF, it);
+                for (int mb = 0; mb < nb; ++mb, ++use, ++job) {
+                    const int slot = use & 1, b = job & 1;
+                    wait_k(ST_PF0 + slot, use >> 1);
+                    if (job >= 2) wait_k(ST_DE0 + b, (job >> 1) - 1);
+                    tc_fence_after();
+                    const uint64_t dq = dphi0 + ((slot * 4 * kTile) >> 4), dk = dq + ((2 * kTile) >> 4);
+                    const uint32_t cs = tmem + 160u * b, cg = cs + 80;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_bf16(cs, dk + 128 * kk, dvb + 128 * kk, idS, kk > 0 ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_bf16(cg, dq + 128 * kk, dyb + 128 * kk, idS, kk > 0 ? 1u : 0u);
+                    umma_commit(&bar[ST_DF0 + b]);
+                    umma_commit(&bar[ST_PE0 + slot]);
+                }
+                umma_commit(&bar[ST_VE]);
+                umma_commit(&bar[ST_YE]);
+            }
+        }
+        __syncwarp();
+    } else {
+        const int ew = warp - 1, q = warp & 3, half = ew >> 2;
+        const uint32_t row = 32u * q + lane;
+        const uint32_t trow = tmem + ((32u * q) << 16);
+        int it = 0, job = 0;
+        for (int item = blockIdx.x; item < bp.nitems && wt.ok; item += gridDim.x, ++it) {
+            const int bh = item / bp.ntiles, t = item - bh * bp.ntiles;
+            const int i_abs = t * kT + static_cast<int>(row);
+            const bool valid = i_abs < bp.L;
+            const int64_t grow = static_cast<int64_t>(bh) * bp.L + i_abs;
+            // [dn | delta] of this thread's token as bf16 operands (delta in every column of
+            // its row of the extension tile)
+            if (it >= 1) wait_k(ST_YE, it - 1);
+            {
+                uint32_t pk[16], dk[16];
+                const float* src = dn + grow * kE;
+                const float dl = valid ? src[64] : 0.0f;
+                const uint32_t dd = pack_bf16(dl, dl);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    pk[c] = valid ? pack_bf16(src[32 * half + 2 * c], src[32 * half + 2 * c + 1]) : 0u;
+                    dk[c] = dd;
+                }
+                st_row32(sbase + Lo.dn, row, half, pk);
+                st_row32(sbase + Lo.dl, row, half, dk);
+            }
+            fence_async_smem();
+            warp_arrive(&bar[ST_YF]);
+            for (int mb = 0; mb < nb; ++mb, ++job) {
+                const int b = job & 1;
+                wait_k(ST_DF0 + b, job >> 1);
+                tc_fence_after();
+                // feature f = 128 mb + row; this warp writes columns 32 half .. (+ e = 64 for half 1)
+                uint32_t sa[32], ga[32], sz = 0, gz = 0;
+                const uint32_t cs = trow + 160u * b, cg = cs + 80;
+                tmem_ld32(cs + 32 * half, sa);
+                tmem_ld32(cg + 32 * half, ga);
+                if (half) {
+                    tmem_ld1(cs + 64, sz);
+                    tmem_ld1(cg + 64, gz);
+                }
+                tmem_wait_ld();
+                reg_fence(sa);
+                reg_fence(ga);
+                reg_fence1(sz);
+                reg_fence1(gz);
+                tc_fence_before();
+                warp_arrive(&bar[ST_DE0 + b]);
+                const int f = 128 * mb + static_cast<int>(row);
+                const int64_t o = (static_cast<int64_t>(bh) * bp.ntiles + t) * bp.F * kE +
+                                  static_cast<int64_t>(32 * half) * bp.F + f;
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    st_s[o + static_cast<int64_t>(c) * bp.F] = __uint_as_float(sa[c]);
+                    st_g[o + static_cast<int64_t>(c) * bp.F] = __uint_as_float(ga[c]);
+                }
+                if (half) {
+                    st_s[o + 32 * static_cast<int64_t>(bp.F)] = __uint_as_float(sz);
+                    st_g[o + 32 * static_cast<int64_t>(bp.F)] = __uint_as_float(gz);
+                }
+            }
+        }
+    }
+    wt.report(err);
+    drain_after_failure(wt.ok);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
 // [BH][L][cols] bf16 viewed as a 3-D tensor, boxes of 64 columns x 128 tokens, 128-byte
 // swizzle; rows past L read as zero.
 bool map_seq(CUtensorMap* m, const void* base, int cols, int L, int BH)
@@ -409,7 +614,30 @@ bool map_seq(CUtensorMap* m, const void* base, int cols, int L, int BH)
 
 bool tc_bwd_tile_supported(int F, int L)
 {
-    return F % 64 == 0 && F >= 64 && F <= 512 && L > 0 && bw_layout().total + 1024 <= 232448;
+    return F % 128 == 0 && F >= 128 && F <= 512 && L > 0 && bw_layout().total + 1024 <= 232448 &&
+           st_layout().total + 1024 <= 232448;
+}
+
+cudaError_t tc_bwd_states(const void* phq, const void* phk, const void* v, const float* dn,
+                          float* st_s, float* st_g, int BH, int L, int F, int* err, cudaStream_t st)
+{
+    if (!tc_bwd_tile_supported(F, L)) return cudaErrorNotSupported;
+    CUtensorMap mq, mk, mv;
+    if (!map_seq(&mq, phq, F, L, BH) || !map_seq(&mk, phk, F, L, BH) || !map_seq(&mv, v, 64, L, BH))
+        return cudaErrorInvalidValue;
+    BwParams bp;
+    bp.L = L;
+    bp.F = F;
+    bp.ntiles = (L + kT - 1) / kT;
+    bp.nitems = BH * bp.ntiles;
+    const size_t smem = st_layout().total + 1024;
+    cudaError_t e = cudaFuncSetAttribute(k_tc_bwd_states, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const int grid = bp.nitems < kNumSMs ? bp.nitems : kNumSMs;
+    TraceScope trace_("tc_bwd_states", st);
+    k_tc_bwd_states<<<grid, kStThreads, smem, st>>>(mq, mk, mv, dn, st_s, st_g, bp, err);
+    return cudaGetLastError();
 }
 
 cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const float* dn,
@@ -425,7 +653,6 @@ cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const f
     bp.F = F;
     bp.ntiles = (L + kT - 1) / kT;
     bp.nitems = BH * bp.ntiles;
-    bp.NC = (L + 63) / 64;
     const size_t smem = bw_layout().total + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_tc_bwd_tile, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
