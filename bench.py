@@ -145,20 +145,20 @@ def kernel_work(name, w, op):
     # kernel the rest; the row statistics read out, g, den and write [dn, delta] (bytes)
     if name == "simt_phi_bwd":
         return th * 8 * D * F, "flop", "alu"
-    # the tensor-core chunk contraction of the backward moves, per token-head, phi(q), phi(k)
-    # (bf16), v, [dn, delta], dphi(q), dphi(k) (fp32), dv and its share of the two 128-token
-    # states it reads (2 F (Dv+1) fp32 per tile)
     # the backward's per-tile sums read phi(q), phi(k), v, [dn, delta] and write two fp32
     # [F][Dv+1] sums per 128-token tile
     if name == "tc_bwd_states":
         return th * (2 * 2 * F + 2 * Dv + 4 * (Dv + 1)) + \
             w.B * w.H * ((w.L + 127) // 128) * 2 * F * (Dv + 1) * 4, "byte", "hbm"
+    # the tensor-core chunk contraction of the backward moves, per token-head, phi(q), phi(k),
+    # v (bf16), [dn, delta] (fp32), dphi(q), dphi(k) (bf16: the tensor-core phi backward reads
+    # them), dv (fp32) and its share of the two 128-token states it reads (2 F (Dv+1) fp32)
     if name == "tc_bwd_tile":
-        return th * (2 * 2 * F + 2 * Dv + 4 * (Dv + 1) + 2 * 4 * F + 4 * Dv) + \
+        return th * (2 * 2 * F + 2 * Dv + 4 * (Dv + 1) + 2 * 2 * F + 4 * Dv) + \
             w.B * w.H * ((w.L + 127) // 128) * 2 * F * (Dv + 1) * 4, "byte", "hbm"
-    # the tensor-core phi backward is bound by its reads: x (bf16), dphi (fp32), dx (fp32)
+    # the tensor-core phi backward is bound by its reads: x (bf16), dphi (bf16), dx (fp32)
     if name == "tc_phi_bwd":
-        return th * (2 * D + 4 * F + 4 * D), "byte", "hbm"
+        return th * (2 * D + 2 * F + 4 * D), "byte", "hbm"
     if name == "simt_bwd_chunk":
         return th * (6 * F * Dv + (C_CHUNK + 1) * (3 * F + 2 * Dv)), "flop", "alu"
     if name == "simt_bwd_rowstats":

@@ -956,6 +956,10 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     // bf16 phi: states, contraction on tensor cores over 128-token tiles; else 64-token chunks
     const bool tcb = std::is_same<T, __nv_bfloat16>::value && tc_bwd_tile_supported(F, L);
+    // with the feature map's backward on tensor cores as well, dphi travels as bf16
+    const bool tcp = std::is_same<T, __nv_bfloat16>::value && P.wB &&
+                     tc_phi_bwd_supported(kD, P.R, P.m, rows);
+    const bool dphi16 = tcb && tcp;
     const int NS = tcb ? (L + 127) / 128 : NC;   // state blocks per sequence
     int* status = reinterpret_cast<int*>(w - kWsHeader);
     if (tcb) {
@@ -986,8 +990,8 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
     }
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     if (tcb) {
-        if ((err = tc_bwd_tile(phq, phk, v, dn, sfw, gbw, dphq, dphk, dv, BH, L, F, status, st)) !=
-            cudaSuccess)
+        if ((err = tc_bwd_tile(phq, phk, v, dn, sfw, gbw, dphq, dphk, dphi16, dv, BH, L, F, status,
+                               st)) != cudaSuccess)
             return err;
     } else {
         const size_t smem = sizeof(BwdSmem);
@@ -1006,7 +1010,7 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
                                     static_cast<int>(psm))) != cudaSuccess)
         return err;
     // bf16 inputs: the feature map's backward on tensor cores when it takes these sizes
-    if (std::is_same<T, __nv_bfloat16>::value && P.wB && tc_phi_bwd_supported(kD, P.R, P.m, rows)) {
+    if (dphi16) {
         if ((err = tc_phi_bwd(q, dphq, dq, rows, P, st)) != cudaSuccess) return err;
         return tc_phi_bwd(k, dphk, dk, rows, P, st);
     }

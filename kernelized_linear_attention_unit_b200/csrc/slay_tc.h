@@ -25,10 +25,11 @@ void tc_pack_wb(int D, int R, int m, const uint16_t* om, const uint16_t* an, uin
 // Feature map bf16 -> bf16 on tensor cores: D == 64, m % 32 == 0, F % 128 == 0, F <= 512.
 bool tc_fmap_supported(int D, int R, int m, int64_t n_rows);
 cudaError_t tc_feature_map(const void* x, void* phi, int64_t n, const Params& P, cudaStream_t st);
-// Backward of the feature map on tensor cores (bf16 x, fp32 dphi [n][F] -> fp32 dx [n][64]):
+// Backward of the feature map on tensor cores (bf16 x, bf16 dphi [n][F] -> fp32 dx [n][64]):
 // same sizes as the forward map.
 bool tc_phi_bwd_supported(int D, int R, int m, int64_t n_rows);
-cudaError_t tc_phi_bwd(const void* x, const float* dphi, float* dx, int64_t n, const Params& P,
+// dphi is [n][F] bf16 (as the tensor-core contraction stores it)
+cudaError_t tc_phi_bwd(const void* x, const void* dphi, float* dx, int64_t n, const Params& P,
                        cudaStream_t st);
 // Causal backward on tensor cores over 128-token tiles (bf16 phi and v, fp32 [dn | delta] rows):
 // the per-tile sums phi(k)^T [v, 1] and phi(q)^T [dn, delta] ([BH][tiles][F][65] fp32), and,
@@ -37,8 +38,8 @@ bool tc_bwd_tile_supported(int F, int L);
 cudaError_t tc_bwd_states(const void* phq, const void* phk, const void* v, const float* dn,
                           float* st_s, float* st_g, int BH, int L, int F, int* err, cudaStream_t st);
 cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const float* dn,
-                        const float* sfw, const float* gbw, float* dphq, float* dphk, float* dv,
-                        int BH, int L, int F, int* err, cudaStream_t st);
+                        const float* sfw, const float* gbw, void* dphq, void* dphk, bool dphi_bf16,
+                        float* dv, int BH, int L, int F, int* err, cudaStream_t st);
 // Device address of the status word of the feature-map kernels, forward and backward (set
 // when a bounded wait ran out).
 const void* fmap_status_word();

@@ -79,6 +79,7 @@ __host__ __device__ inline BwLayout bw_layout()
 
 struct BwParams {
     int L, F, ntiles, nitems;
+    int dphi_bf16;   // contraction: store dphi(q), dphi(k) as bf16 (else fp32)
 };
 
 // 128-byte swizzled [rows][64 bf16] tile: 16-byte chunk c of row r at chunk c ^ (r & 7)
@@ -94,7 +95,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
 k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
               const __grid_constant__ CUtensorMap tmv, const float* __restrict__ dn,
               const float* __restrict__ sfw, const float* __restrict__ gbw,
-              float* __restrict__ dphq, float* __restrict__ dphk, float* __restrict__ dv,
+              void* __restrict__ dphq, void* __restrict__ dphk, float* __restrict__ dv,
               BwParams bp, int* err)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -317,24 +318,32 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
                 ++gs;
                 if (!valid) return;
                 const int f0 = 64 * s + 32 * half;
-                float4* oq = reinterpret_cast<float4*>(dphq + grow * bp.F + f0);
-                float4* ok = reinterpret_cast<float4*>(dphk + grow * bp.F + f0);
                 const float* zs = Sb + 64 * static_cast<int64_t>(bp.F);   // [e = 64][f]
                 const float* zg = Gb + 64 * static_cast<int64_t>(bp.F);
+                float oq[32], ok[32];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    float zq[4], zk[4];
+                for (int c = 0; c < 32; ++c) {
+                    oq[c] = fmaf(delta, zs[f0 + c], __uint_as_float(qa[c]));
+                    ok[c] = __uint_as_float(ka[c]) + zg[f0 + c];
+                }
+                if (bp.dphi_bf16) {
+                    uint4* dq4 = reinterpret_cast<uint4*>(static_cast<uint16_t*>(dphq) + grow * bp.F + f0);
+                    uint4* dk4 = reinterpret_cast<uint4*>(static_cast<uint16_t*>(dphk) + grow * bp.F + f0);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        zq[e] = zs[f0 + 4 * c + e];
-                        zk[e] = zg[f0 + 4 * c + e];
+                    for (int c = 0; c < 4; ++c) {
+                        dq4[c] = make_uint4(pack_bf16(oq[8 * c], oq[8 * c + 1]), pack_bf16(oq[8 * c + 2], oq[8 * c + 3]),
+                                            pack_bf16(oq[8 * c + 4], oq[8 * c + 5]), pack_bf16(oq[8 * c + 6], oq[8 * c + 7]));
+                        dk4[c] = make_uint4(pack_bf16(ok[8 * c], ok[8 * c + 1]), pack_bf16(ok[8 * c + 2], ok[8 * c + 3]),
+                                            pack_bf16(ok[8 * c + 4], ok[8 * c + 5]), pack_bf16(ok[8 * c + 6], ok[8 * c + 7]));
                     }
-                    oq[c] = make_float4(fmaf(delta, zq[0], __uint_as_float(qa[4 * c])),
-                                        fmaf(delta, zq[1], __uint_as_float(qa[4 * c + 1])),
-                                        fmaf(delta, zq[2], __uint_as_float(qa[4 * c + 2])),
-                                        fmaf(delta, zq[3], __uint_as_float(qa[4 * c + 3])));
-                    ok[c] = make_float4(__uint_as_float(ka[4 * c]) + zk[0], __uint_as_float(ka[4 * c + 1]) + zk[1],
-                                        __uint_as_float(ka[4 * c + 2]) + zk[2], __uint_as_float(ka[4 * c + 3]) + zk[3]);
+                } else {
+                    float4* dq4 = reinterpret_cast<float4*>(static_cast<float*>(dphq) + grow * bp.F + f0);
+                    float4* dk4 = reinterpret_cast<float4*>(static_cast<float*>(dphk) + grow * bp.F + f0);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        dq4[c] = make_float4(oq[4 * c], oq[4 * c + 1], oq[4 * c + 2], oq[4 * c + 3]);
+                        dk4[c] = make_float4(ok[4 * c], ok[4 * c + 1], ok[4 * c + 2], ok[4 * c + 3]);
+                    }
                 }
             };
             for (int s = 0; s < ns; ++s) {
@@ -630,6 +639,7 @@ cudaError_t tc_bwd_states(const void* phq, const void* phk, const void* v, const
     bp.F = F;
     bp.ntiles = (L + kT - 1) / kT;
     bp.nitems = BH * bp.ntiles;
+    bp.dphi_bf16 = 0;
     const size_t smem = st_layout().total + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_tc_bwd_states, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
@@ -641,8 +651,8 @@ cudaError_t tc_bwd_states(const void* phq, const void* phk, const void* v, const
 }
 
 cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const float* dn,
-                        const float* sfw, const float* gbw, float* dphq, float* dphk, float* dv,
-                        int BH, int L, int F, int* err, cudaStream_t st)
+                        const float* sfw, const float* gbw, void* dphq, void* dphk, bool dphi_bf16,
+                        float* dv, int BH, int L, int F, int* err, cudaStream_t st)
 {
     if (!tc_bwd_tile_supported(F, L)) return cudaErrorNotSupported;
     CUtensorMap mq, mk, mv;
@@ -653,6 +663,7 @@ cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const f
     bp.F = F;
     bp.ntiles = (L + kT - 1) / kT;
     bp.nitems = BH * bp.ntiles;
+    bp.dphi_bf16 = dphi_bf16 ? 1 : 0;
     const size_t smem = bw_layout().total + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_tc_bwd_tile, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));

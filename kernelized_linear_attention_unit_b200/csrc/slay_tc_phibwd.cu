@@ -12,16 +12,18 @@
 // Both contractions run on tensor cores: per 128-row tile and 64-feature group g the
 // projections U = X W_g^T (N = 128: 64 omega and 64 anchor columns, as in the forward map),
 // then dX^ += [alpha | beta]_g [Omega_g ; A_g] (K = 128, N = 64) with the same resident W
-// tiles read as an MN-major operand.  The kernel reads x (bf16), dphi (fp32) and writes dx
-// (fp32): it is bound by the dphi reads (4F bytes per row).
+// tiles read as an MN-major operand.  The kernel reads x (bf16), dphi (bf16, as the
+// tensor-core contraction stores it) and writes dx (fp32): it is bound by the dphi reads
+// (2F bytes per row).
 //
 // Persistent, one CTA per SM, 128-row tiles round-robin.  Warp 0 issues every TMA load and
 // MMA; warps 1-8 are the epilogue: warp w serves TMEM lanes 32 (w % 4).. (rows of the tile)
 // and the 32-feature half (w - 1) / 4 of every group.  Per group an epilogue warp reads its
-// projections, its rows' dphi (prefetched one group ahead) and writes its block of
+// projections, its rows' dphi (bf16, prefetched one group ahead) and writes its block of
 // [alpha | beta] into a K-major 128-byte-swizzled operand tile; per tile it turns dX^ into
 // dx.  Every wait is bounded; a timeout sets the library's feature-map status word.
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -85,11 +87,21 @@ struct PbParams {
     float sq[16];   // sqrt(2 s_r)
 };
 
+// dphi value c = 0..31 of one row's 32-feature block held as four 16-byte words of bf16
+__device__ __forceinline__ float dphi_val(const uint4 (&d)[4], int c)
+{
+    const uint4 w = d[c >> 3];
+    const int k = (c >> 1) & 3;
+    const uint32_t u = k == 0 ? w.x : k == 1 ? w.y : k == 2 ? w.z : w.w;
+    return __uint_as_float((c & 1) ? (u & 0xFFFF0000u) : (u << 16));
+}
+
 __global__ void __launch_bounds__(kPbThreads, 1)
 k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
-             const float* __restrict__ dphi, float* __restrict__ dx, int64_t n_rows, PbParams pp,
-             int* status)
+             const __nv_bfloat16* __restrict__ dphi, float* __restrict__ dx, int64_t n_rows,
+             PbParams pp, int* status)
 {
+    constexpr int kW = 4;   // 16-byte words per 32 bf16 dphi values
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* sm = aligned_smem(smem_raw);
     const PbLayout L = pb_layout(pp.F);
@@ -222,18 +234,18 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
         const uint32_t trow = tmem0 + ((32u * q) << 16);
         const uint32_t abase = sbase + L.a + half * kBoxBytes;
         const int F = pp.F;
-        // dphi of (tile k, group g) for this lane's row: 32 fp32 (features 64g + 32 half ..)
-        auto dphi_ptr = [&](int k, int g) -> const float4* {
+        // dphi of (tile k, group g) for this lane's row: 32 values (features 64g + 32 half ..)
+        auto dphi_ptr = [&](int k, int g) -> const uint4* {
             const int64_t r = static_cast<int64_t>(k * static_cast<int>(gridDim.x) +
                                                    static_cast<int>(blockIdx.x)) * kRows + row;
             const int64_t rr = r < n_rows ? r : n_rows - 1;   // rows past the end: any valid row
-            return reinterpret_cast<const float4*>(dphi + rr * F + 64 * g + 32 * half);
+            return reinterpret_cast<const uint4*>(dphi + rr * F + 64 * g + 32 * half);
         };
-        float4 dpn[8];
+        uint4 dpn[kW];
         if (nt > 0) {
-            const float4* p = dphi_ptr(0, 0);
+            const uint4* p = dphi_ptr(0, 0);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) dpn[i] = __ldg(p + i);
+            for (int i = 0; i < kW; ++i) dpn[i] = __ldg(p + i);
         }
         for (int k = 0; k < nt; ++k) {
             const int s = k % xbufs;
@@ -247,13 +259,13 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
             const float nrm = 1.0f / inv, two_n = 2.0f * nrm;
             for (int g = 0; g < ng; ++g) {
                 const int j = k * ng + g;
-                float4 dp[8];
+                uint4 dp[kW];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) dp[i] = dpn[i];
+                for (int i = 0; i < kW; ++i) dp[i] = dpn[i];
                 if (j + 1 < njobs) {   // prefetch the next group's dphi
-                    const float4* p = dphi_ptr(g + 1 < ng ? k : k + 1, g + 1 < ng ? g + 1 : 0);
+                    const uint4* p = dphi_ptr(g + 1 < ng ? k : k + 1, g + 1 < ng ? g + 1 : 0);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) dpn[i] = __ldg(p + i);
+                    for (int i = 0; i < kW; ++i) dpn[i] = __ldg(p + i);
                 }
                 {
                     uint32_t ph = static_cast<uint32_t>((j >> 1) & 1);
@@ -272,8 +284,7 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
                 uint32_t al[16], be[16];
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
-                    const float4 d4 = dp[c >> 2];
-                    const float d0 = (c & 2) ? d4.z : d4.x, d1 = (c & 2) ? d4.w : d4.y;
+                    const float d0 = dphi_val(dp, c), d1 = dphi_val(dp, c + 1);
                     const float p0 = __uint_as_float(pr[c]), p1 = __uint_as_float(pr[c + 1]);
                     const float t0 = d0 * ex2(fmaf(a, __uint_as_float(ur[c]), bb)) * p0;
                     const float t1 = d1 * ex2(fmaf(a, __uint_as_float(ur[c + 1]), bb)) * p1;
@@ -366,7 +377,7 @@ bool tc_phi_bwd_supported(int D, int R, int m, int64_t n_rows)
            n_rows <= (int64_t(1) << 31) - kRows && pb_layout(F).total + 1024 <= 232448;
 }
 
-cudaError_t tc_phi_bwd(const void* x, const float* dphi, float* dx, int64_t n, const Params& P,
+cudaError_t tc_phi_bwd(const void* x, const void* dphi, float* dx, int64_t n, const Params& P,
                        cudaStream_t st)
 {
     const int F = P.F;
@@ -390,12 +401,13 @@ cudaError_t tc_phi_bwd(const void* x, const float* dphi, float* dx, int64_t n, c
     cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
     if (e != cudaSuccess) return e;
     const size_t smem = pb_layout(F).total + 1024;
+    const int grid = pp.ntiles < kNumSMs ? pp.ntiles : kNumSMs;
     e = cudaFuncSetAttribute(k_tc_phi_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    const int grid = pp.ntiles < kNumSMs ? pp.ntiles : kNumSMs;
     TraceScope trace_("tc_phi_bwd", st);
-    k_tc_phi_bwd<<<grid, kPbThreads, smem, st>>>(mx, mw, dphi, dx, n, pp, status);
+    k_tc_phi_bwd<<<grid, kPbThreads, smem, st>>>(mx, mw, static_cast<const __nv_bfloat16*>(dphi), dx,
+                                                 n, pp, status);
     return cudaGetLastError();
 }
 
