@@ -346,31 +346,41 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
                     }
                 }
             };
+            // thread et converts 16 e of feature f = et % 64 of S_s and of G_s (the sums are
+            // e-major: a warp's loads cover 32 consecutive features); the next slice's values
+            // are loaded while the previous slice's outputs are written
+            const int sf = et & 63, se0 = 16 * (et >> 6);
+            float sv[16], gv[16];
+            auto load_sg = [&](int s) {
+                const float* sr = Sb + static_cast<int64_t>(se0) * bp.F + 64 * s + sf;
+                const float* gr = Gb + static_cast<int64_t>(se0) * bp.F + 64 * s + sf;
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    sv[c] = sr[c * static_cast<int64_t>(bp.F)];
+                    gv[c] = gr[c * static_cast<int64_t>(bp.F)];
+                }
+            };
+            load_sg(0);
             for (int s = 0; s < ns; ++s) {
                 const int k = it * ns + s, sb = k & 1;
                 if (k >= 2) wait_k(BW_SGE0 + sb, (k >> 1) - 1);
-                {   // thread et converts 16 e of feature f = et % 64 of S_s and of G_s (the
-                    // states are e-major: a warp's loads cover 32 consecutive features)
-                    const int f = et & 63, e0 = 16 * (et >> 6);
-                    const float* sr = Sb + static_cast<int64_t>(e0) * bp.F + 64 * s + f;
-                    const float* gr = Gb + static_cast<int64_t>(e0) * bp.F + 64 * s + f;
+                {
                     uint32_t a8[8], g8[8];
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
-                        a8[c] = pack_bf16(sr[(2 * c) * static_cast<int64_t>(bp.F)],
-                                          sr[(2 * c + 1) * static_cast<int64_t>(bp.F)]);
-                        g8[c] = pack_bf16(gr[(2 * c) * static_cast<int64_t>(bp.F)],
-                                          gr[(2 * c + 1) * static_cast<int64_t>(bp.F)]);
+                        a8[c] = pack_bf16(sv[2 * c], sv[2 * c + 1]);
+                        g8[c] = pack_bf16(gv[2 * c], gv[2 * c + 1]);
                     }
                     const uint32_t ts = sbase + Lo.sg + sb * 2 * kSG, tg = ts + kSG;
                     const int ch = 2 * (et >> 6);
-                    st_shared_v4(ts + sw128_off(f, ch), a8[0], a8[1], a8[2], a8[3]);
-                    st_shared_v4(ts + sw128_off(f, ch + 1), a8[4], a8[5], a8[6], a8[7]);
-                    st_shared_v4(tg + sw128_off(f, ch), g8[0], g8[1], g8[2], g8[3]);
-                    st_shared_v4(tg + sw128_off(f, ch + 1), g8[4], g8[5], g8[6], g8[7]);
+                    st_shared_v4(ts + sw128_off(sf, ch), a8[0], a8[1], a8[2], a8[3]);
+                    st_shared_v4(ts + sw128_off(sf, ch + 1), a8[4], a8[5], a8[6], a8[7]);
+                    st_shared_v4(tg + sw128_off(sf, ch), g8[0], g8[1], g8[2], g8[3]);
+                    st_shared_v4(tg + sw128_off(sf, ch + 1), g8[4], g8[5], g8[6], g8[7]);
                 }
                 fence_async_smem();
                 warp_arrive(&bar[BW_SGF0 + sb]);
+                if (s + 1 < ns) load_sg(s + 1);
                 if (s >= 1) write_slice(s - 1, gs & 1);
             }
             write_slice(ns - 1, gs & 1);
