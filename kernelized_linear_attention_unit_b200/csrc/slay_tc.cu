@@ -224,9 +224,12 @@ __device__ __forceinline__ float phi_sub_epilogue(const uint32_t (&ur)[32], cons
         // with kPoly one exponential in four goes to the FMA pipe: the special-function
         // unit's queue is shared with the shared-memory and barrier traffic that paces these
         // kernels (the k side, which has the registers for it)
-        const float f0 = ex2(fmaf(a, __uint_as_float(ur[j]), b)) * p0 * p0;
-        const float y1 = fmaf(a, __uint_as_float(ur[j + 1]), b);
-        const float f1 = ((kPoly && (j & 2)) ? ex2_poly(y1) : ex2(y1)) * p1 * p1;
+        const float2 y = ffma2(make_float2(a, a), make_float2(__uint_as_float(ur[j]), __uint_as_float(ur[j + 1])),
+                               make_float2(b, b));
+        const float2 pp = make_float2(p0, p1);
+        const float2 e = make_float2(ex2(y.x), (kPoly && (j & 2)) ? ex2_poly(y.y) : ex2(y.y));
+        const float2 ff = fmul2(fmul2(e, pp), pp);   // packed two-wide fp32
+        const float f0 = ff.x, f1 = ff.y;
         if (zs) {
             dz = fmaf(f0, zs[j], dz);
             dz = fmaf(f1, zs[j + 1], dz);

@@ -86,8 +86,9 @@ __device__ __forceinline__ uint32_t sw64_off(uint32_t row, uint32_t chunk)
 // Exponentials per pair of features taken by the polynomial below instead of the
 // special-function unit: 0 (none), 1 (one of every two pairs' second element) or 2 (every
 // pair's second element).  The special-function unit shares its issue queue with the
-// shared-memory and barrier operations that pace the pipeline, so a quarter of the
-// exponentials go to the FMA pipe (measured best: it costs about a dozen instructions each).
+// shared-memory and barrier operations that pace the pipeline; with the packed two-wide
+// fp32 arithmetic below, 0 and 1 measure the same and 2 is slower (the polynomial costs
+// about a dozen instructions per value).
 #ifndef SLAY_FM_POLY
 #define SLAY_FM_POLY 1
 #endif
@@ -245,14 +246,16 @@ k_tc_feature_map(const __grid_constant__ CUtensorMap tmx, const __grid_constant_
             warp_arrive(&UE[j & 1]);             // this warp's rows of buffer j & 1 are read
             const float a = fp.a2[2 * g + half] * inv, bb = fp.b2[2 * g + half] + l2i;
             uint32_t pk[16];
+            const float2 a2 = make_float2(a, a), b2 = make_float2(bb, bb);
 #pragma unroll
             for (int c = 0; c < 32; c += 2) {
-                const float x0 = __uint_as_float(pr[c]), x1 = __uint_as_float(pr[c + 1]);
-                const float e0 = ex2(fmaf(a, __uint_as_float(ur[c]), bb));
-                const float y1 = fmaf(a, __uint_as_float(ur[c + 1]), bb);
+                // pairs of features through the packed two-wide fp32 instructions
+                const float2 x = make_float2(__uint_as_float(pr[c]), __uint_as_float(pr[c + 1]));
+                const float2 y = ffma2(a2, make_float2(__uint_as_float(ur[c]), __uint_as_float(ur[c + 1])), b2);
                 const bool poly = SLAY_FM_POLY == 2 || (SLAY_FM_POLY == 1 && (c & 2));
-                const float e1 = poly ? ex2_poly(y1) : ex2(y1);
-                pk[c >> 1] = pack_bf16(e0 * x0 * x0, e1 * x1 * x1);
+                const float2 e = make_float2(ex2(y.x), poly ? ex2_poly(y.y) : ex2(y.y));
+                const float2 f = fmul2(fmul2(e, x), x);
+                pk[c >> 1] = pack_bf16(f.x, f.y);
             }
             // the box was stored obufs groups ago: its reads must be done before it is rewritten
             if (lane == 0) {
