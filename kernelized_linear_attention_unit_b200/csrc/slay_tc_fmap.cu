@@ -204,85 +204,88 @@ k_tc_feature_map(const __grid_constant__ CUtensorMap tmx, const __grid_constant_
             }
         }
         __syncwarp();
-    }
-    else {   // the two teams' warps
-    uint64_t* tb = bar + FB_TEAM + team * FB_PER_TEAM;
-    uint64_t* XF = tb + FB_XF;
-    uint64_t* UF = tb + FB_UF;
-    uint64_t* UE = tb + FB_UE;
-    const unsigned char* xs = sm + L.x + team * xbufs * kBoxBytes;
-    const int first = blockIdx.x * kTeams + team;
-    const int nt = team_tiles(team);
-    const uint32_t row = 32u * q + lane;
-    const uint32_t tcol = tmem0 + 256u * team + ((32u * q) << 16) + 64u * half;
-    const int obufs = L.obufs;
-    const uint32_t obox = sbase + L.o + cw * obufs * kStageBytes;
-    int js = 0;                                  // staging boxes used by this warp
-    int s = 0;                                   // X slot of tile k and its phase
-    uint32_t xph = 0;
-    for (int k = 0; k < nt; ++k) {
-        {
-            uint32_t ph = xph;
-            wt.wait(&XF[s], ph);
-        }
-        float inv, l2i;
-        row_scale(xs + s * kBoxBytes + row * 128, row, inv, l2i);
-        const int row0 = (first + k * stride) * kRows + 32 * q;
-        for (int g = 0; g < ng; ++g, ++js) {
-            const int j = k * ng + g;
-            const uint32_t ph = static_cast<uint32_t>((j >> 1) & 1);
+    } else {   // the two teams' warps
+        uint64_t* tb = bar + FB_TEAM + team * FB_PER_TEAM;
+        uint64_t* XF = tb + FB_XF;
+        uint64_t* UF = tb + FB_UF;
+        uint64_t* UE = tb + FB_UE;
+        const unsigned char* xs = sm + L.x + team * xbufs * kBoxBytes;
+        const int first = blockIdx.x * kTeams + team;
+        const int nt = team_tiles(team);
+        const uint32_t row = 32u * q + lane;
+        const uint32_t tcol = tmem0 + 256u * team + ((32u * q) << 16) + 64u * half;
+        const int obufs = L.obufs;
+        const uint32_t obox = sbase + L.o + cw * obufs * kStageBytes;
+        int js = 0;                                  // staging boxes used by this warp
+        int s = 0;                                   // X slot of tile k and its phase
+        uint32_t xph = 0;
+        for (int k = 0; k < nt; ++k) {
             {
-                uint32_t p = ph;
-                wt.wait(&UF[j & 1], p);
+                uint32_t ph = xph;
+                wt.wait(&XF[s], ph);
             }
-            tc_fence_after();
-            uint32_t ur[32], pr[32];
-            tmem_ld32(tcol + 128u * (j & 1), ur);
-            tmem_ld32(tcol + 128u * (j & 1) + 32, pr);
-            tmem_wait_ld();
-            reg_fence(ur);
-            reg_fence(pr);
-            tc_fence_before();
-            warp_arrive(&UE[j & 1]);             // this warp's rows of buffer j & 1 are read
-            const float a = fp.a2[2 * g + half] * inv, bb = fp.b2[2 * g + half] + l2i;
-            uint32_t pk[16];
-            const float2 a2 = make_float2(a, a), b2 = make_float2(bb, bb);
+            float inv, l2i;
+            row_scale(xs + s * kBoxBytes + row * 128, row, inv, l2i);
+            const int row0 = (first + k * stride) * kRows + 32 * q;
+            for (int g = 0; g < ng; ++g, ++js) {
+                const int j = k * ng + g;
+                const uint32_t ph = static_cast<uint32_t>((j >> 1) & 1);
+                {
+                    uint32_t p = ph;
+                    wt.wait(&UF[j & 1], p);
+                }
+                tc_fence_after();
+                uint32_t ur[32], pr[32];
+                tmem_ld32(tcol + 128u * (j & 1), ur);
+                tmem_ld32(tcol + 128u * (j & 1) + 32, pr);
+                tmem_wait_ld();
+                reg_fence(ur);
+                reg_fence(pr);
+                tc_fence_before();
+                warp_arrive(&UE[j & 1]);             // this warp's rows of buffer j & 1 are read
+                const float a = fp.a2[2 * g + half] * inv, bb = fp.b2[2 * g + half] + l2i;
+                uint32_t pk[16];
+                const float2 a2 = make_float2(a, a), b2 = make_float2(bb, bb);
 #pragma unroll
-            for (int c = 0; c < 32; c += 2) {
-                // pairs of features through the packed two-wide fp32 instructions
-                const float2 x = make_float2(__uint_as_float(pr[c]), __uint_as_float(pr[c + 1]));
-                const float2 y = ffma2(a2, make_float2(__uint_as_float(ur[c]), __uint_as_float(ur[c + 1])), b2);
-                const bool poly = SLAY_FM_POLY == 2 || (SLAY_FM_POLY == 1 && (c & 2));
-                const float2 e = make_float2(ex2(y.x), poly ? ex2_poly(y.y) : ex2(y.y));
-                const float2 f = fmul2(fmul2(e, x), x);
-                pk[c >> 1] = pack_bf16(f.x, f.y);
-            }
-            // the box was stored obufs groups ago: its reads must be done before it is rewritten
-            if (lane == 0) {
-                if (obufs == 2)
-                    bulk_wait_read<1>();
-                else
-                    bulk_wait_read<0>();
-            }
-            __syncwarp();
-            const uint32_t box = obox + (js & (obufs - 1)) * kStageBytes;
+                for (int c = 0; c < 32; c += 2) {
+                    // pairs of features through the packed two-wide fp32 instructions
+                    const float2 x =
+                        make_float2(__uint_as_float(pr[c]), __uint_as_float(pr[c + 1]));
+                    const float2 u =
+                        make_float2(__uint_as_float(ur[c]), __uint_as_float(ur[c + 1]));
+                    const float2 y = ffma2(a2, u, b2);
+                    const bool poly = SLAY_FM_POLY == 2 || (SLAY_FM_POLY == 1 && (c & 2));
+                    const float2 e = make_float2(ex2(y.x), poly ? ex2_poly(y.y) : ex2(y.y));
+                    const float2 f = fmul2(fmul2(e, x), x);
+                    pk[c >> 1] = pack_bf16(f.x, f.y);
+                }
+                // the box was stored obufs groups ago: its reads must be done before it is
+                // rewritten
+                if (lane == 0) {
+                    if (obufs == 2)
+                        bulk_wait_read<1>();
+                    else
+                        bulk_wait_read<0>();
+                }
+                __syncwarp();
+                const uint32_t box = obox + (js & (obufs - 1)) * kStageBytes;
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-                st_shared_v4(box + sw64_off(lane, c), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
-                             pk[4 * c + 3]);
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                tma_store_2d(&tmo, sm + (box - sbase), 64 * g + 32 * half, row0);
-                bulk_commit_group();
+                for (int c = 0; c < 4; ++c)
+                    st_shared_v4(box + sw64_off(lane, c), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
+                                 pk[4 * c + 3]);
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmo, sm + (box - sbase), 64 * g + 32 * half, row0);
+                    bulk_commit_group();
+                }
+            }
+            if (++s == xbufs) {
+                s = 0;
+                xph ^= 1u;
             }
         }
-        if (++s == xbufs) {
-            s = 0;
-            xph ^= 1u;
-        }
-    }
-    if (lane == 0) bulk_wait<0>();
+        if (lane == 0) bulk_wait<0>();
     }
     wt.report(&g_fmap_status);
     drain_after_failure(wt.ok);
