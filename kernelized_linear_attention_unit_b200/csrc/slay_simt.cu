@@ -362,6 +362,25 @@ __global__ void k_bwd_rowstats(const T* __restrict__ out, const float* __restric
     if (lane == 0) dn[row * E + 64] = -s * rz;
 }
 
+// The same statistics for the tensor-core backward: dn as bf16 rows [row][64] (its MMA operand,
+// loaded by TMA) and delta as fp32 [row].
+template <typename T>
+__global__ void k_bwd_rowstats_tc(const T* __restrict__ out, const float* __restrict__ den,
+                                  const T* __restrict__ g, __nv_bfloat16* __restrict__ dn16,
+                                  float* __restrict__ delta, int64_t nrows, float eps)
+{
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= nrows) return;
+    const float rz = 1.0f / (den[row] + eps);
+    const float g0 = ld(g + row * kD + 2 * lane), g1 = ld(g + row * kD + 2 * lane + 1);
+    float s = g0 * ld(out + row * kD + 2 * lane) + g1 * ld(out + row * kD + 2 * lane + 1);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    reinterpret_cast<__nv_bfloat162*>(dn16 + row * kD)[lane] = __floats2bfloat162_rn(g0 * rz, g1 * rz);
+    if (lane == 0) delta[row] = -s * rz;
+}
+
 struct BwdSmem {
     float a[C][C + 1];    // phi(q) tile [i][fl]
     float b[C][C + 1];    // phi(k) tile [j][fl]
@@ -948,14 +967,21 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
     cudaError_t err;
     if ((err = phi_map<T>(q, phq, rows, P, st)) != cudaSuccess) return err;
     if ((err = phi_map<T>(k, phk, rows, P, st)) != cudaSuccess) return err;
-    {
-        TraceScope trace_("simt_bwd_rowstats", st);
-        k_bwd_rowstats<T><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
-            cp<T>(out), den, cp<T>(dout), dn, rows, eps);
-    }
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
     // bf16 phi: states, contraction on tensor cores over 128-token tiles; else 64-token chunks
     const bool tcb = std::is_same<T, __nv_bfloat16>::value && tc_bwd_tile_supported(F, L);
+    // tensor-core path: dn as bf16 rows and delta in the dn region (132 of its 260 bytes a row)
+    __nv_bfloat16* dn16 = reinterpret_cast<__nv_bfloat16*>(dn);
+    float* delta = reinterpret_cast<float*>(dn16 + rows * kD);
+    {
+        TraceScope trace_("simt_bwd_rowstats", st);
+        if (tcb)
+            k_bwd_rowstats_tc<T><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
+                cp<T>(out), den, cp<T>(dout), dn16, delta, rows, eps);
+        else
+            k_bwd_rowstats<T><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
+                cp<T>(out), den, cp<T>(dout), dn, rows, eps);
+    }
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
     // with the feature map's backward on tensor cores as well, dphi travels as bf16
     const bool tcp = std::is_same<T, __nv_bfloat16>::value && P.wB &&
                      tc_phi_bwd_supported(kD, P.R, P.m, rows);
@@ -963,7 +989,8 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
     const int NS = tcb ? (L + 127) / 128 : NC;   // state blocks per sequence
     int* status = reinterpret_cast<int*>(w - kWsHeader);
     if (tcb) {
-        if ((err = tc_bwd_states(phq, phk, v, dn, sfw, gbw, BH, L, F, status, st)) != cudaSuccess)
+        if ((err = tc_bwd_states(phq, phk, v, dn16, delta, sfw, gbw, BH, L, F, status, st)) !=
+            cudaSuccess)
             return err;
     } else {
         const dim3 sg((F + C - 1) / C, NC, BH);
@@ -990,8 +1017,8 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
     }
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     if (tcb) {
-        if ((err = tc_bwd_tile(phq, phk, v, dn, sfw, gbw, dphq, dphk, dphi16, dv, BH, L, F, status,
-                               st)) != cudaSuccess)
+        if ((err = tc_bwd_tile(phq, phk, v, dn16, delta, sfw, gbw, dphq, dphk, dphi16, dv, BH, L, F,
+                               status, st)) != cudaSuccess)
             return err;
     } else {
         const size_t smem = sizeof(BwdSmem);

@@ -31,15 +31,17 @@ bool tc_phi_bwd_supported(int D, int R, int m, int64_t n_rows);
 // dphi is [n][F] bf16 (as the tensor-core contraction stores it)
 cudaError_t tc_phi_bwd(const void* x, const void* dphi, float* dx, int64_t n, const Params& P,
                        cudaStream_t st);
-// Causal backward on tensor cores over 128-token tiles (bf16 phi and v, fp32 [dn | delta] rows):
-// the per-tile sums phi(k)^T [v, 1] and phi(q)^T [dn, delta] ([BH][tiles][F][65] fp32), and,
-// from their exclusive forward / reverse scans, the contraction -> fp32 dphi(q), dphi(k), dv.
+// Causal backward on tensor cores over 128-token tiles (bf16 phi, v and dn rows, fp32 delta):
+// the per-tile sums phi(k)^T [v, 1] and phi(q)^T [dn, delta] ([BH][tiles][65][F] fp32), and,
+// from their exclusive forward / reverse scans, the contraction -> dphi(q), dphi(k), dv.
 bool tc_bwd_tile_supported(int F, int L);
-cudaError_t tc_bwd_states(const void* phq, const void* phk, const void* v, const float* dn,
-                          float* st_s, float* st_g, int BH, int L, int F, int* err, cudaStream_t st);
-cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const float* dn,
-                        const float* sfw, const float* gbw, void* dphq, void* dphk, bool dphi_bf16,
-                        float* dv, int BH, int L, int F, int* err, cudaStream_t st);
+cudaError_t tc_bwd_states(const void* phq, const void* phk, const void* v, const void* dn16,
+                          const float* delta, float* st_s, float* st_g, int BH, int L, int F,
+                          int* err, cudaStream_t st);
+cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const void* dn16,
+                        const float* delta, const float* sfw, const float* gbw, void* dphq,
+                        void* dphk, bool dphi_bf16, float* dv, int BH, int L, int F, int* err,
+                        cudaStream_t st);
 // Device address of the status word of the feature-map kernels, forward and backward (set
 // when a bounded wait ran out).
 const void* fmap_status_word();

@@ -24,9 +24,9 @@
 // shared-memory tiles as MN-major operands.
 //
 // Persistent, one CTA per SM over the (b, h, tile) items.  Warp 0 issues the MMAs, warp 9
-// the TMA loads (V, and the phi slice pairs of both phases through a ring of two), warps 1-8
-// are the epilogue (lane quadrant w % 4, column half (w - 1) / 4).  Every wait is bounded; a
-// timeout sets the workspace status word.
+// the TMA loads (V and dn (bf16 rows), and the phi slice pairs of both phases through a ring
+// of two), warps 1-8 are the epilogue (lane quadrant w % 4, column half (w - 1) / 4; delta per
+// row from its fp32 array).  Every wait is bounded; a timeout sets the workspace status word.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -53,7 +53,7 @@ constexpr int kNumSMs = 148;
 constexpr uint32_t kColP = 0, kColC = 128, kColDV = 256;
 
 enum {
-    BW_VF = 0, BW_VE, BW_PF0, BW_PF1, BW_PE0, BW_PE1, BW_DNF, BW_DNE, BW_PCF, BW_PCTF, BW_PCTE,
+    BW_VF = 0, BW_VE, BW_PF0, BW_PF1, BW_PE0, BW_PE1, BW_PCF, BW_PCTF, BW_PCTE,
     BW_SGF0, BW_SGF1, BW_SGE0, BW_SGE1, BW_DQF0, BW_DQF1, BW_DQE0, BW_DQE1, BW_DVF, BW_DVE,
     BW_NUM
 };
@@ -68,7 +68,7 @@ __host__ __device__ inline BwLayout bw_layout()
     l.phi = 0;                    // 2 slots x (phiQ slice, phiK slice)
     l.pt = l.phi + 4 * kTile;     // P~ as two column halves [128 i][64 j]
     l.ct = l.pt + 2 * kTile;      // C~ likewise
-    l.dn = l.ct + 2 * kTile;      // dn [128 i][64 e]
+    l.dn = l.ct + 2 * kTile;      // dn [128 i][64 e] (TMA, with V)
     l.v = l.dn + kTile;           // V [128 j][64 e]
     l.sg = l.v + kTile;           // 2 buffers x (S_s, G_s) [64 f][64 e]
     l.bar = l.sg + 4 * kSG;
@@ -82,19 +82,11 @@ struct BwParams {
     int dphi_bf16;   // contraction: store dphi(q), dphi(k) as bf16 (else fp32)
 };
 
-// 128-byte swizzled [rows][64 bf16] tile: 16-byte chunk c of row r at chunk c ^ (r & 7)
-__device__ __forceinline__ void st_row32(uint32_t tile, uint32_t row, int half, const uint32_t (&pk)[16])
-{
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-        st_shared_v4(tile + sw128_off(row, 4 * half + c), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
-                     pk[4 * c + 3]);
-}
-
 __global__ void __launch_bounds__(kBwThreads, 1)
 k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-              const __grid_constant__ CUtensorMap tmv, const float* __restrict__ dn,
-              const float* __restrict__ sfw, const float* __restrict__ gbw,
+              const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdn,
+              const float* __restrict__ delta, const float* __restrict__ sfw,
+              const float* __restrict__ gbw,
               void* __restrict__ dphq, void* __restrict__ dphk, float* __restrict__ dv,
               BwParams bp, int* err)
 {
@@ -113,12 +105,13 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
     }
     if (tid == 0) {
         for (int i = 0; i < BW_NUM; ++i) mbar_init(&bar[i], 1);
-        const int warp_counted[7] = {BW_DNF, BW_PCTF, BW_SGF0, BW_SGF1, BW_DQE0, BW_DQE1, BW_DVE};
-        for (int i = 0; i < 7; ++i) mbar_init(&bar[warp_counted[i]], 8);   // one arrival per epilogue warp
+        const int warp_counted[6] = {BW_PCTF, BW_SGF0, BW_SGF1, BW_DQE0, BW_DQE1, BW_DVE};
+        for (int i = 0; i < 6; ++i) mbar_init(&bar[warp_counted[i]], 8);   // one arrival per epilogue warp
         mbar_fence_init();
         tma_prefetch_desc(&tmq);
         tma_prefetch_desc(&tmk);
         tma_prefetch_desc(&tmv);
+        tma_prefetch_desc(&tmdn);
     }
     tc_fence_before();
     __syncthreads();
@@ -138,8 +131,9 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
             for (int item = blockIdx.x; item < bp.nitems && wt.ok; item += gridDim.x, ++it) {
                 const int bh = item / bp.ntiles, t = item - bh * bp.ntiles;
                 if (it >= 1) wait_k(BW_VE, it - 1);
-                mbar_arrive_expect_tx(&bar[BW_VF], kTile);
+                mbar_arrive_expect_tx(&bar[BW_VF], 2 * kTile);   // V and dn
                 tma_load_3d(sm + Lo.v, &tmv, &bar[BW_VF], 0, t * kT, bh);
+                tma_load_3d(sm + Lo.dn, &tmdn, &bar[BW_VF], 0, t * kT, bh);
                 for (int u = 0; u < 2 * ns; ++u, ++use) {   // phase A slices, then phase B
                     const int s = u < ns ? u : u - ns, slot = use & 1;
                     if (use >= 2) wait_k(BW_PE0 + slot, (use >> 1) - 1);
@@ -168,7 +162,6 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
             int use = 0, gs = 0, it = 0;   // phi uses, slice-accumulator uses, items
             for (int item = blockIdx.x; item < bp.nitems && wt.ok; item += gridDim.x, ++it) {
                 wait_k(BW_VF, it);
-                wait_k(BW_DNF, it);
                 // P / C0 overwrite the slice buffers of the previous item: both read
                 if (gs >= 1) wait_k(BW_DQE0 + ((gs - 1) & 1), (gs - 1) >> 1);
                 if (gs >= 2) wait_k(BW_DQE0 + ((gs - 2) & 1), (gs - 2) >> 1);
@@ -227,8 +220,7 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
                 }
                 umma_commit(&bar[BW_DVF]);
                 umma_commit(&bar[BW_PCTE]);
-                umma_commit(&bar[BW_DNE]);
-                umma_commit(&bar[BW_VE]);
+                umma_commit(&bar[BW_VE]);   // V and dn free
             }
         }
         __syncwarp();
@@ -245,20 +237,7 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
             const int64_t grow = static_cast<int64_t>(bh) * bp.L + i_abs;
             const float* Sb = sfw + (static_cast<int64_t>(bh) * bp.ntiles + t) * bp.F * kE;
             const float* Gb = gbw + (static_cast<int64_t>(bh) * bp.ntiles + t) * bp.F * kE;
-            // dn (bf16 operand, this warp's 32 columns) and delta
-            if (it >= 1) wait_k(BW_DNE, it - 1);
-            float delta = 0.0f;
-            {
-                uint32_t pk[16];
-                const float* src = dn + grow * kE + 32 * half;
-#pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    pk[c] = valid ? pack_bf16(src[2 * c], src[2 * c + 1]) : 0u;
-                if (valid) delta = dn[grow * kE + 64];
-                st_row32(sbase + Lo.dn, row, half, pk);
-            }
-            fence_async_smem();
-            warp_arrive(&bar[BW_DNF]);
+            const float dl = valid ? delta[grow] : 0.0f;   // dn itself arrives by TMA with V
             // masked P~ and C~ (this warp's half of the columns j)
             wait_k(BW_PCF, it);
             tc_fence_after();
@@ -287,8 +266,8 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
                         const bool k1 = valid && jl + 1 <= static_cast<int>(row) && j0 + 32 * hh + 2 * c + 1 < bp.L;
                         pk[c] = pack_bf16(k0 ? __uint_as_float(P[2 * c]) : 0.0f,
                                           k1 ? __uint_as_float(P[2 * c + 1]) : 0.0f);
-                        ck[c] = pack_bf16(k0 ? __uint_as_float(Cc[2 * c]) + delta : 0.0f,
-                                          k1 ? __uint_as_float(Cc[2 * c + 1]) + delta : 0.0f);
+                        ck[c] = pack_bf16(k0 ? __uint_as_float(Cc[2 * c]) + dl : 0.0f,
+                                          k1 ? __uint_as_float(Cc[2 * c + 1]) + dl : 0.0f);
                     }
                     // column chunk 4 hh .. of the half tile
 #pragma unroll
@@ -323,7 +302,7 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
                 float oq[32], ok[32];
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
-                    oq[c] = fmaf(delta, zs[f0 + c], __uint_as_float(qa[c]));
+                    oq[c] = fmaf(dl, zs[f0 + c], __uint_as_float(qa[c]));
                     ok[c] = __uint_as_float(ka[c]) + zg[f0 + c];
                 }
                 if (bp.dphi_bf16) {
@@ -420,8 +399,9 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
 // (M = 128 features, N = 80, K = 128 tokens), phi read as an MN-major A operand (two 64-
 // feature tiles), the extra column through a second 64-wide tile at the operand's leading
 // byte offset: constant ones for [V | 1], delta_i in every column for [dn | delta].
-// Warp 0 issues the MMAs, warp 9 the TMA loads, warps 1-8 convert [dn | delta] to bf16 and
-// write the sums (lane quadrant w % 4 = 32 features, half (w - 1) / 4 of the columns).
+// Warp 0 issues the MMAs, warp 9 the TMA loads (V and the bf16 dn rows with them), warps 1-8
+// write delta into the extension tile and store the sums (lane quadrant w % 4 = 32
+// features, half (w - 1) / 4 of the columns).
 constexpr int kStThreads = 32 * 10;
 
 enum {
@@ -439,7 +419,7 @@ __host__ __device__ inline StLayout st_layout()
     l.phi = 0;                   // 2 slots x (phiQ 2 tiles, phiK 2 tiles) of one feature block
     l.v = l.phi + 8 * kTile;
     l.ones = l.v + kTile;        // right after V: [V | 1] at LBO = kTile
-    l.dn = l.ones + kTile;
+    l.dn = l.ones + kTile;       // dn (TMA, with V)
     l.dl = l.dn + kTile;         // right after dn: [dn | delta] at LBO = kTile
     l.bar = l.dl + kTile;
     l.tmem = l.bar + ST_NUM * 8;
@@ -449,8 +429,9 @@ __host__ __device__ inline StLayout st_layout()
 
 __global__ void __launch_bounds__(kStThreads, 1)
 k_tc_bwd_states(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                const __grid_constant__ CUtensorMap tmv, const float* __restrict__ dn,
-                float* __restrict__ st_s, float* __restrict__ st_g, BwParams bp, int* err)
+                const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdn,
+                const float* __restrict__ delta, float* __restrict__ st_s, float* __restrict__ st_g,
+                BwParams bp, int* err)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* sm = aligned_smem(smem_raw);
@@ -478,6 +459,7 @@ k_tc_bwd_states(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         tma_prefetch_desc(&tmq);
         tma_prefetch_desc(&tmk);
         tma_prefetch_desc(&tmv);
+        tma_prefetch_desc(&tmdn);
     }
     fence_async_smem();
     tc_fence_before();
@@ -496,8 +478,9 @@ k_tc_bwd_states(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             for (int item = blockIdx.x; item < bp.nitems && wt.ok; item += gridDim.x, ++it) {
                 const int bh = item / bp.ntiles, t = item - bh * bp.ntiles;
                 if (it >= 1) wait_k(ST_VE, it - 1);
-                mbar_arrive_expect_tx(&bar[ST_VF], kTile);
+                mbar_arrive_expect_tx(&bar[ST_VF], 2 * kTile);   // V and dn
                 tma_load_3d(sm + Lo.v, &tmv, &bar[ST_VF], 0, t * kT, bh);
+                tma_load_3d(sm + Lo.dn, &tmdn, &bar[ST_VF], 0, t * kT, bh);
                 for (int mb = 0; mb < nb; ++mb, ++use) {
                     const int slot = use & 1;
                     if (use >= 2) wait_k(ST_PE0 + slot, (use >> 1) - 1);
@@ -552,21 +535,13 @@ k_tc_bwd_states(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             const int i_abs = t * kT + static_cast<int>(row);
             const bool valid = i_abs < bp.L;
             const int64_t grow = static_cast<int64_t>(bh) * bp.L + i_abs;
-            // [dn | delta] of this thread's token as bf16 operands (delta in every column of
-            // its row of the extension tile)
+            // delta of this thread's token in the first 16 columns of its row of the extension
+            // tile (the columns the N = 80 operand reads; dn itself arrives by TMA with V)
             if (it >= 1) wait_k(ST_YE, it - 1);
             {
-                uint32_t pk[16], dk[16];
-                const float* src = dn + grow * kE;
-                const float dl = valid ? src[64] : 0.0f;
+                const float dl = valid ? delta[grow] : 0.0f;
                 const uint32_t dd = pack_bf16(dl, dl);
-#pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    pk[c] = valid ? pack_bf16(src[32 * half + 2 * c], src[32 * half + 2 * c + 1]) : 0u;
-                    dk[c] = dd;
-                }
-                st_row32(sbase + Lo.dn, row, half, pk);
-                st_row32(sbase + Lo.dl, row, half, dk);
+                st_shared_v4(sbase + Lo.dl + sw128_off(row, half), dd, dd, dd, dd);
             }
             fence_async_smem();
             warp_arrive(&bar[ST_YF]);
@@ -637,12 +612,14 @@ bool tc_bwd_tile_supported(int F, int L)
            st_layout().total + 1024 <= 232448;
 }
 
-cudaError_t tc_bwd_states(const void* phq, const void* phk, const void* v, const float* dn,
-                          float* st_s, float* st_g, int BH, int L, int F, int* err, cudaStream_t st)
+cudaError_t tc_bwd_states(const void* phq, const void* phk, const void* v, const void* dn16,
+                          const float* delta, float* st_s, float* st_g, int BH, int L, int F,
+                          int* err, cudaStream_t st)
 {
     if (!tc_bwd_tile_supported(F, L)) return cudaErrorNotSupported;
-    CUtensorMap mq, mk, mv;
-    if (!map_seq(&mq, phq, F, L, BH) || !map_seq(&mk, phk, F, L, BH) || !map_seq(&mv, v, 64, L, BH))
+    CUtensorMap mq, mk, mv, mdn;
+    if (!map_seq(&mq, phq, F, L, BH) || !map_seq(&mk, phk, F, L, BH) || !map_seq(&mv, v, 64, L, BH) ||
+        !map_seq(&mdn, dn16, 64, L, BH))
         return cudaErrorInvalidValue;
     BwParams bp;
     bp.L = L;
@@ -656,17 +633,19 @@ cudaError_t tc_bwd_states(const void* phq, const void* phk, const void* v, const
     if (e != cudaSuccess) return e;
     const int grid = bp.nitems < kNumSMs ? bp.nitems : kNumSMs;
     TraceScope trace_("tc_bwd_states", st);
-    k_tc_bwd_states<<<grid, kStThreads, smem, st>>>(mq, mk, mv, dn, st_s, st_g, bp, err);
+    k_tc_bwd_states<<<grid, kStThreads, smem, st>>>(mq, mk, mv, mdn, delta, st_s, st_g, bp, err);
     return cudaGetLastError();
 }
 
-cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const float* dn,
-                        const float* sfw, const float* gbw, void* dphq, void* dphk, bool dphi_bf16,
-                        float* dv, int BH, int L, int F, int* err, cudaStream_t st)
+cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const void* dn16,
+                        const float* delta, const float* sfw, const float* gbw, void* dphq,
+                        void* dphk, bool dphi_bf16, float* dv, int BH, int L, int F, int* err,
+                        cudaStream_t st)
 {
     if (!tc_bwd_tile_supported(F, L)) return cudaErrorNotSupported;
-    CUtensorMap mq, mk, mv;
-    if (!map_seq(&mq, phq, F, L, BH) || !map_seq(&mk, phk, F, L, BH) || !map_seq(&mv, v, 64, L, BH))
+    CUtensorMap mq, mk, mv, mdn;
+    if (!map_seq(&mq, phq, F, L, BH) || !map_seq(&mk, phk, F, L, BH) || !map_seq(&mv, v, 64, L, BH) ||
+        !map_seq(&mdn, dn16, 64, L, BH))
         return cudaErrorInvalidValue;
     BwParams bp;
     bp.L = L;
@@ -680,7 +659,8 @@ cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const f
     if (e != cudaSuccess) return e;
     const int grid = bp.nitems < kNumSMs ? bp.nitems : kNumSMs;
     TraceScope trace_("tc_bwd_tile", st);
-    k_tc_bwd_tile<<<grid, kBwThreads, smem, st>>>(mq, mk, mv, dn, sfw, gbw, dphq, dphk, dv, bp, err);
+    k_tc_bwd_tile<<<grid, kBwThreads, smem, st>>>(mq, mk, mv, mdn, delta, sfw, gbw, dphq, dphk, dv, bp,
+                                                  err);
     return cudaGetLastError();
 }
 
