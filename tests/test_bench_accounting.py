@@ -1,0 +1,69 @@
+"""bench.py's algorithmic work per launch (CPU): the launches of one step add up to the
+per-token-head counts of the method, also when the map is split into feature chunks.
+
+Per token-head, D = Dv = 64, C = 64: causal forward 8DF + 4F Dv + (C+1)(F+Dv) flop,
+bidirectional 8DF + 4F Dv flop; the feature map moves 2D + 2F bytes per row.
+"""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from kernelized_linear_attention_unit_b200 import workloads as W  # noqa: E402
+
+D = DV = 64
+C = 64
+
+
+def causal_flop(F):
+    return 8 * D * F + 4 * F * DV + (C + 1) * (F + DV)
+
+
+def chunks(F):
+    return 1 if F <= 256 else (F // 256 if F % 256 == 0 else F // 128)
+
+
+@pytest.mark.parametrize("R,m", [(4, 64), (8, 64), (6, 64), (2, 64)])
+def test_causal_launches_add_up(R, m):
+    w = W.Workload("acct", B=2, H=3, L=1000, R=R, m=m, dtype="bf16")
+    th = w.B * w.H * w.L
+    n = chunks(w.F)
+    per_step = n * (bench.kernel_work("tc_kphi_state", w, "causal")[0] +
+                    bench.kernel_work("tc_qphi_out", w, "causal")[0])
+    # the masked P.V term (C+1) Dv is counted once although every chunk computes it
+    assert per_step == pytest.approx(th * causal_flop(w.F), rel=1e-12, abs=n)
+
+
+@pytest.mark.parametrize("R,m", [(4, 64), (8, 64)])
+def test_bidir_launches_add_up(R, m):
+    w = W.Workload("acct", B=2, H=3, L=1000, R=R, m=m, dtype="bf16", causal=False)
+    th = w.B * w.H * w.L
+    n = chunks(w.F)
+    per_step = n * (bench.kernel_work("tc_bidir_state", w, "bidir")[0] +
+                    bench.kernel_work("tc_bidir_out", w, "bidir")[0])
+    assert per_step == th * (8 * D * w.F + 4 * w.F * DV)
+
+
+def test_feature_map_bytes():
+    w = W.CAUSAL_16K
+    th = w.B * w.H * w.L
+    amount, unit, bound = bench.kernel_work("tc_feature_map", w, "feature_map")
+    assert (unit, bound) == ("byte", "hbm")
+    assert amount == 2 * th * (2 * D + 2 * w.F)
+
+
+def test_backward_kernels_are_not_chunk_split():
+    # the backward's tensor-core kernels take the whole map: their counts use the full F
+    w = W.FWDBWD_8K
+    th = w.B * w.H * w.L
+    assert bench.kernel_work("tc_phi_bwd", w, "bwd")[0] == th * (2 * D + 2 * w.F + 4 * D)
+    tiles = w.B * w.H * ((w.L + 127) // 128)
+    states = tiles * 2 * w.F * (DV + 1) * 4
+    assert bench.kernel_work("tc_bwd_states", w, "bwd")[0] == \
+        th * (2 * 2 * w.F + 2 * DV + 4 * (DV + 1)) + states
+    assert bench.kernel_work("tc_bwd_tile", w, "bwd")[0] == \
+        th * (2 * 2 * w.F + 2 * DV + 4 * (DV + 1) + 2 * 2 * w.F + 4 * DV) + states
