@@ -31,8 +31,11 @@
  *   - dtype SLAY_F32: inputs/outputs fp32, all arithmetic fp32 on CUDA cores.
  *     dtype SLAY_BF16: q,k,v,out (and dout) bf16; arithmetic with fp32 accumulation,
  *     states S and z always fp32; gradients fp32.
- *   - Supported: D == Dv == 64, 1 <= R <= 16, 1 <= m, F = R*m <= 1024 (F % 16 == 0 on
- *     the bf16 tensor-core path; other F run on CUDA cores), eps > 0 and finite.
+ *   - Supported: D == Dv == 64, 1 <= R <= 16, 1 <= m, F = R*m <= 1024, eps > 0 and
+ *     finite.  The bf16 tensor-core kernels take F % 128 == 0 and F <= 512 (the attention
+ *     forward as feature chunks of at most 256 when F > 256), with m % 64 == 0 for the
+ *     attention forward and m % 32 == 0 for the feature map and its backward; other sizes
+ *     run on CUDA cores.
  *   - Errors are status codes, never exceptions or aborts.  On any error nothing is
  *     enqueued.  The library owns only its sketch-parameter cache: one small device
  *     buffer per (device, D, R, m, seed, eps), created on first use (synchronous
@@ -107,7 +110,11 @@ slay_status slay_attn_bidir_fwd(const void* q, const void* k, const void* v, voi
  * out, den : the forward's outputs for the same inputs (out in `dt`, den fp32).
  * dout     : device [B,H,L,Dv] in `dt`.
  * dq, dk   : device [B,H,L,D] fp32, dv : device [B,H,L,Dv] fp32, all written.
- * workspace: slay_workspace_bytes(SLAY_OP_CAUSAL_BWD, ...) bytes. */
+ * workspace: slay_workspace_bytes(SLAY_OP_CAUSAL_BWD, ...) bytes; its first int is the
+ *            status word of the tensor-core kernels (see slay_kernel_status).
+ * bf16 mode with tensor-core sizes: the per-128-token-tile sums, the contraction and the
+ * derivative through phi run on tensor cores with bf16 operands and fp32 accumulation;
+ * dphi(q), dphi(k) pass between the last two as bf16. */
 slay_status slay_attn_causal_bwd(const void* q, const void* k, const void* v,
                                  const void* out, const float* den, const void* dout,
                                  float* dq, float* dk, float* dv,
