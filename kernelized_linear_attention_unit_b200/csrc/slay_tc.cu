@@ -199,6 +199,52 @@ __device__ __forceinline__ void finish_row(const KParams& kp, uint32_t (&o0)[32]
     if (den) den[g] = d;
 }
 
+// finish_row with the chunk mode fixed at compile time (no code, and no registers, for the
+// modes a launch does not use)
+template <bool kIn, bool kOut>
+__device__ __forceinline__ void finish_row_t(const KParams& kp, uint32_t (&o0)[32], uint32_t (&o1)[32],
+                                             float d, size_t g, __nv_bfloat16* out, float* den)
+{
+    if (kIn) {
+        const float4* src = reinterpret_cast<const float4*>(kp.part_num + g * 64);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            const float4 a = src[q];
+            uint32_t* o = q < 8 ? o0 : o1;
+            const int c = 4 * (q & 7);
+            o[c] = __float_as_uint(__uint_as_float(o[c]) + a.x);
+            o[c + 1] = __float_as_uint(__uint_as_float(o[c + 1]) + a.y);
+            o[c + 2] = __float_as_uint(__uint_as_float(o[c + 2]) + a.z);
+            o[c + 3] = __float_as_uint(__uint_as_float(o[c + 3]) + a.w);
+        }
+        d += kp.part_den[g];
+    }
+    if (kOut) {
+        float4* dst = reinterpret_cast<float4*>(kp.part_num + g * 64);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            const uint32_t* o = q < 8 ? o0 : o1;
+            const int c = 4 * (q & 7);
+            dst[q] = make_float4(__uint_as_float(o[c]), __uint_as_float(o[c + 1]),
+                                 __uint_as_float(o[c + 2]), __uint_as_float(o[c + 3]));
+        }
+        kp.part_den[g] = d;
+        return;
+    }
+    const float rz = 1.0f / (d + kp.eps);
+    uint4* dst = reinterpret_cast<uint4*>(out + g * 64);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const uint32_t* o = q < 4 ? o0 : o1;
+        const int c = 8 * (q & 3);
+        dst[q] = make_uint4(pack_bf16(__uint_as_float(o[c]) * rz, __uint_as_float(o[c + 1]) * rz),
+                            pack_bf16(__uint_as_float(o[c + 2]) * rz, __uint_as_float(o[c + 3]) * rz),
+                            pack_bf16(__uint_as_float(o[c + 4]) * rz, __uint_as_float(o[c + 5]) * rz),
+                            pack_bf16(__uint_as_float(o[c + 6]) * rz, __uint_as_float(o[c + 7]) * rz));
+    }
+    if (den) den[g] = d;
+}
+
 // v[t] for a slice index t < kMaxSlices, by selects (an indexed parameter array would be
 // copied to local memory)
 __device__ __forceinline__ float slice_val(const float (&v)[kMaxSlices], int t)
@@ -933,72 +979,232 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
 }
 
 // ------------------------------------------- causal output reading stored phi(k)
-// As k_tc_causal_out, but phi(k) of every tile comes from HBM (written by the state kernel)
-// instead of being recomputed, which frees the k projections: warp 0 loads q tiles (two
-// buffers) and projection operands, warp 3 loads the phi(k) slices and v; warp 2 issues the
-// q projections alternately into U0 / U1; warps 4-7 and 8-11 turn them into phi(q) (group g
-// writes half g of each 64-feature slice); warp 1 and warps 12-15 as in k_tc_causal_out.
-struct SmemOutPk {
-    uint32_t w, q, v, ones, phik, phiq, st, bar, tmem, total;
+// grid = BH * nseg; one CTA walks the tiles of one segment with the state entering it, as
+// k_tc_causal_out does, but phi(k) of every tile comes from HBM (written by the state
+// kernel) instead of being recomputed, and phi(q) is written by its warps into tensor memory
+// (bf16 pairs), where the score and readout MMAs read it as their A operand: phi(q) never
+// passes through shared memory.  The projection operand W stays resident in shared memory
+// and each 64-feature slice is one N = 128 projection.  Tensor memory holds no z and no ones
+// column (to fit the phi(q) slot): the denominator is
+//   den_i = phi(q_i) . z_tile + sum_{j <= i in the tile} P_ij,
+// the first term from the readout against the state copy [S | z] (z_tile = z of the earlier
+// segments + the column sums of this segment's earlier phi(k) tiles, which the output warps
+// add up from the tiles in shared memory), the second summed in fp32 by the warps that mask
+// the scores.
+//
+// Warps: 0 TMA (W once; q tiles, two buffers; phi(k) slices; v), 1 the score / readout /
+// state / P.V MMAs, 2 the projections, 3 idle after setup; 4-11 phi(q) (group g = warp >= 8
+// takes features [32g, 32g+32) of every slice) and, between the first two slices of a tile,
+// the previous tile's masked bf16 scores; 12-15 the column sums of phi(k) (warp 12 + t sums
+// slice t), the state copy for the next readout and the outputs.
+constexpr uint32_t kTsU = 0;      // 128: projection of one 64-feature slice ([u | p] per 32)
+constexpr uint32_t kTsP = 128;    // 128: intra-tile scores, then bf16 P in place
+constexpr uint32_t kTsO = 256;    // 80 : numerator | phi(q) . z (column 64)
+constexpr uint32_t kTsS = 336;    // 2 x 64: state S of the feature halves
+constexpr uint32_t kTsQ = 464;    // 32 : phi(q) slice (64 features as 32 bf16 pairs)
+
+enum {
+    T_QF0 = 0, T_QF1, T_QE0, T_QE1, T_WF, T_UF, T_UE, T_PQF, T_PQE,
+    T_PKF0, T_PKF1, T_PKF2, T_PKF3, T_PKFREE0, T_PKFREE1,
+    T_VF, T_VE, T_PF, T_PSM, T_SD, T_TD, T_OE, T_SBF,
+    T_DF0, T_DF1, T_DE0, T_DE1, T_ZC0, T_ZC1,
+    NUM_TS_BARS
 };
 
-__host__ __device__ inline SmemOutPk smem_outpk_layout(int F)
+struct SmemOutTs {
+    uint32_t w, q, v, phik, st, zpre, ztile, den, bar, tmem, total;
+};
+
+__host__ __device__ inline SmemOutTs smem_outts_layout(int F)
 {
-    SmemOutPk s;
-    s.w = 0;
-    s.q = kWSlots * kWBytes;                  // 2 buffers
+    SmemOutTs s;
+    s.w = 0;                                     // F/32 sub-slices of 8 KiB, resident
+    s.q = s.w + (F / kSub) * kWBytes;            // 2 buffers
     s.v = s.q + 2 * kTileBytes;
-    s.ones = s.v + kTileBytes;                // right after V: fixed offset from it
-    s.phik = s.ones + kOnesBytes;
-    s.phiq = s.phik + (F / kSlice) * kTileBytes;
-    s.st = s.phiq + 2 * kTileBytes;
-    s.bar = s.st + (F / kSlice) * kStBytes;
-    s.tmem = s.bar + NUM_BARS * 8;
+    s.phik = s.v + kTileBytes;                   // F/64 slices
+    s.st = s.phik + (F / kSlice) * kTileBytes;   // [S | z] copy: F x 80 bf16 (write_state_row)
+    s.zpre = s.st + (F / kSlice) * kStBytes;     // fp32 [F]: z of the earlier segments
+    s.ztile = s.zpre + F * 4;                    // fp32 [2][F]: z entering the next tile
+    s.den = s.ztile + 2 * F * 4;                 // fp32 [2 tile parities][2 groups][128 rows]
+    s.bar = s.den + 2 * 2 * kTile * 4;
+    s.tmem = s.bar + NUM_TS_BARS * 8;
     s.total = s.tmem + 16;
     return s;
 }
 
+// Row f of the [S | z] copy (the layout of write_state_row) from the fp32 bit patterns of
+// S[f][0..32) (s0) and S[f][32..64) (s1).
+__device__ __forceinline__ void write_state_row_u(uint32_t st, int F, int f, const uint32_t (&s0)[32],
+                                                  const uint32_t (&s1)[32], float z)
+{
+    const uint32_t base = st + (f >> 3) * 128 + (f & 7) * 16;
+    const uint32_t sbo = static_cast<uint32_t>(F) * 16;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+        const uint32_t* s = g < 4 ? s0 : s1;
+        const int c = 8 * (g & 3);
+        st_shared_v4(base + g * sbo,
+                     pack_bf16(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                     pack_bf16(__uint_as_float(s[c + 2]), __uint_as_float(s[c + 3])),
+                     pack_bf16(__uint_as_float(s[c + 4]), __uint_as_float(s[c + 5])),
+                     pack_bf16(__uint_as_float(s[c + 6]), __uint_as_float(s[c + 7])));
+    }
+    st_shared_v4(base + 8 * sbo, pack_bf16(z, 0.0f), 0u, 0u, 0u);
+}
+
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+// Columns [32 part, 32 part + 32) of row f of the [S | z] copy (four of its 16-byte pieces)
+__device__ __forceinline__ void write_state_cols32(uint32_t st, int F, int f, int part, const uint32_t (&s)[32])
+{
+    const uint32_t sbo = static_cast<uint32_t>(F) * 16;
+    const uint32_t base = st + (f >> 3) * 128 + (f & 7) * 16 + 4 * part * sbo;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        st_shared_v4(base + q * sbo,
+                     pack_bf16(__uint_as_float(s[8 * q]), __uint_as_float(s[8 * q + 1])),
+                     pack_bf16(__uint_as_float(s[8 * q + 2]), __uint_as_float(s[8 * q + 3])),
+                     pack_bf16(__uint_as_float(s[8 * q + 4]), __uint_as_float(s[8 * q + 5])),
+                     pack_bf16(__uint_as_float(s[8 * q + 6]), __uint_as_float(s[8 * q + 7])));
+}
+
+// Column 64 (z) of row f of the [S | z] copy, with columns 65..71 zero
+__device__ __forceinline__ void write_state_z(uint32_t st, int F, int f, float z)
+{
+    st_shared_v4(st + (f >> 3) * 128 + (f & 7) * 16 + 8 * static_cast<uint32_t>(F) * 16, pack_bf16(z, 0.0f), 0u, 0u, 0u);
+}
+
+// phi of 32 features (u, p of this row) packed as 16 bf16 pairs
+__device__ __forceinline__ void phi_pack(const uint32_t (&ur)[32], const uint32_t (&pr)[32], float a, float b,
+                                         uint32_t (&pk)[16])
+{
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+        const float2 y = ffma2(make_float2(a, a), make_float2(__uint_as_float(ur[j]), __uint_as_float(ur[j + 1])),
+                               make_float2(b, b));
+        const float2 pp = make_float2(__uint_as_float(pr[j]), __uint_as_float(pr[j + 1]));
+        const float2 e = make_float2(ex2(y.x), ex2(y.y));
+        const float2 ff = fmul2(fmul2(e, pp), pp);
+        pk[j >> 1] = pack_bf16(ff.x, ff.y);
+    }
+}
+
+// [S]_h += phiK_h^T V for feature half h (N = 64: no ones column here)
+__device__ __forceinline__ void issue_state_half64(uint32_t tmem, uint64_t dphik, uint64_t dv, int h)
+{
+    constexpr uint32_t idS = idesc_bf16(128, 64, 1, 1);
+    const uint64_t da = desc_add(dphik, 2 * h * kTileBytes);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) umma_bf16(tmem + kTsS + 64 * h, da + 128 * kk, dv + 128 * kk, idS, 1u);
+}
+
+// The masked scores of tile `pit` of the segment as bf16 in place, by the phi(q) warp of
+// group g: the 32-column chunks c = g, g + 2 (chunks past the diagonal are zeros).  Chunk
+// c (fp32 columns [32c, 32c+32)) goes to bf16 columns 32g + 16(c/2): a group writes only the
+// columns of its own first chunk, after reading them, so the two groups of a quadrant never
+// overwrite what the other still reads.  The row's sum of its unmasked scores in these
+// chunks (fp32) goes to dens.
+__device__ __forceinline__ void ts_mask_scores(uint64_t* bar, Waiter& wt, uint32_t& ph_pf, uint32_t& ph_de,
+                                               uint32_t trow, uint32_t row, int lane, int sp, int g,
+                                               float* dens, int pit)
+{
+    wt.wait(&bar[T_PF], ph_pf);
+    tc_fence_after();
+    float dint = 0.0f;
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+        const int c = g + 2 * cc;
+        uint32_t pk[16];
+        uint32_t pv[32];
+        if (c <= sp) {
+            tmem_ld32(trow + kTsP + 32 * c, pv);
+            tmem_wait_ld();
+            reg_fence(pv);
+        }
+        if (c < sp) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float x0 = __uint_as_float(pv[2 * j]), x1 = __uint_as_float(pv[2 * j + 1]);
+                dint += x0 + x1;
+                pk[j] = pack_bf16(x0, x1);
+            }
+        } else if (c == sp) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float x0 = (2 * j <= lane) ? __uint_as_float(pv[2 * j]) : 0.0f;
+                const float x1 = (2 * j + 1 <= lane) ? __uint_as_float(pv[2 * j + 1]) : 0.0f;
+                dint += x0 + x1;
+                pk[j] = pack_bf16(x0, x1);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) pk[j] = 0u;
+        }
+        tmem_st16(trow + kTsP + 32 * g + 16 * cc, pk);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    warp_arrive(&bar[T_PSM]);
+    const int par = pit & 1;
+    if (pit >= 2) {
+        uint32_t pd = (ph_de >> par) & 1u;
+        wt.wait(&bar[T_DE0 + par], pd);
+        ph_de ^= 1u << par;
+    }
+    dens[(2 * par + g) * kTile + row] = dint;
+    warp_arrive(&bar[T_DF0 + par]);
+}
+
+template <int kAcc>   // bit 0: add the earlier chunks' sums; bit 1: store this chunk's sums
 __global__ void __launch_bounds__(kOutThreads, 1)
-k_tc_causal_out_pk(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmpk,
+k_tc_causal_out_ts(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmpk,
                    const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmw,
                    KParams kp, const float* __restrict__ wsS, const float* __restrict__ wsZ,
                    __nv_bfloat16* __restrict__ out, float* __restrict__ den, int* __restrict__ err)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* sm = aligned_smem(smem_raw);
-    const SmemOutPk L = smem_outpk_layout(kp.F);
+    const SmemOutTs L = smem_outts_layout(kp.F);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L.bar);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L.tmem);
+    float* zpre = reinterpret_cast<float*>(sm + L.zpre);
+    float* ztile = reinterpret_cast<float*>(sm + L.ztile);
+    float* dens = reinterpret_cast<float*>(sm + L.den);
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int NT = kp.F / kSlice, NS = kp.F / kSub, halves = kp.F / 128;
     const Seg sg = segment_of(blockIdx.x, kp.nseg, kp.ntiles);
-    // q buffer b: full / empty (the fourth W slot's barriers hold buffer 1)
-    auto QF = [bar](int b) { return &bar[b ? B_W_FULL3 : B_QK_FULL]; };
-    auto QE = [bar](int b) { return &bar[b ? B_W_EMPTY3 : B_QK_EMPTY]; };
 
     if (warp == 1) {
         tmem_alloc(tslot, 512);
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bar[i], 1);
-        mbar_init(QE(0), 1 + 8);
-        mbar_init(QE(1), 1 + 8);
-        mbar_init(&bar[B_U_EMPTY0], 4);
-        mbar_init(&bar[B_U_EMPTY1], 4);
-        mbar_init(&bar[B_PQ_FULL0], 8);
-        mbar_init(&bar[B_PQ_FULL1], 8);
-        mbar_init(&bar[B_PSM_FULL], 4);
-        mbar_init(&bar[B_O_EMPTY], 4);
-        mbar_init(&bar[B_SBF_READY], 4);
+        for (int i = 0; i < NUM_TS_BARS; ++i) mbar_init(&bar[i], 1);
+        mbar_init(&bar[T_QE0], 1 + 8);   // the projection issuer's commit + the phi(q) warps
+        mbar_init(&bar[T_QE1], 1 + 8);
+        mbar_init(&bar[T_UE], 8);
+        mbar_init(&bar[T_PQF], 8);
+        mbar_init(&bar[T_PSM], 8);
+        mbar_init(&bar[T_OE], 4);
+        mbar_init(&bar[T_SBF], 4);
+        mbar_init(&bar[T_DF0], 8);
+        mbar_init(&bar[T_DF1], 8);
+        mbar_init(&bar[T_DE0], 4);
+        mbar_init(&bar[T_DE1], 4);
+        mbar_init(&bar[T_ZC0], 2);       // column sums of the two slices of a feature half
+        mbar_init(&bar[T_ZC1], 2);
         mbar_fence_init();
         tma_prefetch_desc(&tmq);
         tma_prefetch_desc(&tmpk);
         tma_prefetch_desc(&tmv);
         tma_prefetch_desc(&tmw);
     }
-    fill_ones(sm + L.ones);
     {   // the state copy: columns 65..79 stay zero
         uint4* p = reinterpret_cast<uint4*>(sm + L.st);
         for (int i = tid; i < NT * kStBytes / 16; i += kOutThreads) p[i] = make_uint4(0, 0, 0, 0);
@@ -1007,8 +1213,6 @@ k_tc_causal_out_pk(const __grid_constant__ CUtensorMap tmq, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
-    // registers: the single-thread issuers of warpgroup 0 give 32 of theirs to the three
-    // epilogue warpgroups (128*96 + 384*136 <= 65536); each role stays inside its branch
     if (warp < 4) {
         regs_dec<96>();
         fence_async_smem();
@@ -1017,137 +1221,137 @@ k_tc_causal_out_pk(const __grid_constant__ CUtensorMap tmq, const __grid_constan
         tc_fence_after();
         Waiter wt;
         if (warp == 0) {
-            // ------------------------------------------------ TMA: q tiles, W sub-slices
+            // ---------------------------------------------------------------- TMA
+            // W once; then per tile the q tile (two buffers, needed a tile ahead by the
+            // projections), the phi(k) slices (each feature half once the previous tile's
+            // scores and state update have read it) and v (once the previous P.V is done)
             if (lane == 0) {
-                uint32_t ph_qe = 0, ph_we = (1u << kWSlots) - 1u;
-                int n_glob = 0;
-                for (int tile = sg.t_begin, it = 0; tile < sg.t_end; ++tile, ++it) {
+                mbar_arrive_expect_tx(&bar[T_WF], NS * kWBytes);
+                for (int n = 0; n < NS; ++n)
+                    tma_load_2d(sm + L.w + n * kWBytes, &tmw, &bar[T_WF], 0, n * 64);
+                uint32_t ph_qe = 0, ph_free = 0, ph_zc = 0, ph_ve = 0;
+                auto load_q = [&](int it) {
                     const int qb = it & 1;
                     if (it >= 2) {
                         uint32_t ph = (ph_qe >> qb) & 1u;
-                        wt.wait(QE(qb), ph);
+                        wt.wait(&bar[T_QE0 + qb], ph);
                         ph_qe ^= 1u << qb;
                     }
-                    mbar_arrive_expect_tx(QF(qb), kTileBytes);
-                    tma_load_3d(sm + L.q + qb * kTileBytes, &tmq, QF(qb), 0, tile * kTile, sg.bh);
-                    for (int n = 0; n < NS; ++n, ++n_glob) {
-                        const int slot = n_glob % kWSlots;
-                        uint32_t ph = (ph_we >> slot) & 1u;
-                        wt.wait(&bar[B_W_EMPTY0 + slot], ph);
-                        ph_we ^= (1u << slot);
-                        mbar_arrive_expect_tx(&bar[B_W_FULL0 + slot], kWBytes);
-                        tma_load_2d(sm + L.w + slot * kWBytes, &tmw, &bar[B_W_FULL0 + slot], 0, n * 64);
-                    }
-                }
-            }
-        } else if (warp == 3) {
-            // ----------------------------------------------- TMA: phi(k) slices and v
-            if (lane == 0) {
-                uint32_t ph_free = 0, ph_ve = 0;
-                for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+                    mbar_arrive_expect_tx(&bar[T_QF0 + qb], kTileBytes);
+                    tma_load_3d(sm + L.q + qb * kTileBytes, &tmq, &bar[T_QF0 + qb], 0,
+                                (sg.t_begin + it) * kTile, sg.bh);
+                };
+                const int n = sg.t_end - sg.t_begin;
+                load_q(0);
+                if (n > 1) load_q(1);
+                for (int tile = sg.t_begin, it = 0; tile < sg.t_end; ++tile, ++it) {
                     for (int t = 0; t < NT; ++t) {
-                        // a feature half is free once the previous tile's scores and state
-                        // update have read it
-                        if (tile > sg.t_begin && (t & 1) == 0) {
-                            uint32_t ph = (ph_free >> (t >> 1)) & 1u;
-                            wt.wait(&bar[B_PK_FREE0 + (t >> 1)], ph);
-                            ph_free ^= 1u << (t >> 1);
+                        if (it > 0 && (t & 1) == 0) {   // MMAs and column sums done with the half
+                            const int h = t >> 1;
+                            uint32_t ph = (ph_free >> h) & 1u;
+                            wt.wait(&bar[T_PKFREE0 + h], ph);
+                            ph_free ^= 1u << h;
+                            uint32_t pz = (ph_zc >> h) & 1u;
+                            wt.wait(&bar[T_ZC0 + h], pz);
+                            ph_zc ^= 1u << h;
                         }
-                        mbar_arrive_expect_tx(pk_full(bar, t), kTileBytes);
-                        tma_load_3d(sm + L.phik + t * kTileBytes, &tmpk, pk_full(bar, t), kSlice * t,
+                        mbar_arrive_expect_tx(&bar[T_PKF0 + t], kTileBytes);
+                        tma_load_3d(sm + L.phik + t * kTileBytes, &tmpk, &bar[T_PKF0 + t], kSlice * t,
                                     tile * kTile, sg.bh);
                     }
-                    if (tile > sg.t_begin) wt.wait(&bar[B_V_EMPTY], ph_ve);
-                    mbar_arrive_expect_tx(&bar[B_V_FULL], kTileBytes);
-                    tma_load_3d(sm + L.v, &tmv, &bar[B_V_FULL], 0, tile * kTile, sg.bh);
+                    if (it > 0) wt.wait(&bar[T_VE], ph_ve);
+                    mbar_arrive_expect_tx(&bar[T_VF], kTileBytes);
+                    tma_load_3d(sm + L.v, &tmv, &bar[T_VF], 0, tile * kTile, sg.bh);
+                    if (it + 2 < n) load_q(it + 2);
                 }
             }
         } else if (warp == 2) {
-            // ------------------------------------------------- q projection issuer
+            // ---------------------------------- q projections, one 64-feature slice each
             if (lane == 0) {
-                uint32_t ph_qf = 0, ph_wf = 0, ph_ue = 0x3u;
-                const uint64_t dqx0 = desc_kmajor(sbase + L.q), dw0 = desc_kmajor(sbase + L.w);
-                int n_glob = 0;
+                constexpr uint32_t idU = idesc_bf16(128, 128, 0, 0);
+                uint32_t ph_qf = 0, ph_ue = 1, ph_wf = 0;
+                const uint64_t dq0 = desc_kmajor(sbase + L.q), dw0 = desc_kmajor(sbase + L.w);
+                wt.wait(&bar[T_WF], ph_wf);
                 for (int tile = sg.t_begin, it = 0; tile < sg.t_end; ++tile, ++it) {
                     const int qb = it & 1;
                     uint32_t ph = (ph_qf >> qb) & 1u;
-                    wt.wait(QF(qb), ph);
+                    wt.wait(&bar[T_QF0 + qb], ph);
                     ph_qf ^= 1u << qb;
-                    for (int n = 0; n < NS; ++n, ++n_glob) {
-                        const int slot = n_glob % kWSlots, g = n & 1;
-                        uint32_t pw = (ph_wf >> slot) & 1u;
-                        wt.wait(&bar[B_W_FULL0 + slot], pw);
-                        ph_wf ^= (1u << slot);
-                        uint32_t pu = (ph_ue >> g) & 1u;
-                        wt.wait(&bar[B_U_EMPTY0 + g], pu);
-                        ph_ue ^= 1u << g;
+                    const uint64_t dq = desc_add(dq0, qb * kTileBytes);
+                    for (int t = 0; t < NT; ++t) {
+                        wt.wait(&bar[T_UE], ph_ue);
                         tc_fence_after();
-                        issue_projection(tmem + (g ? kColU1 : kColU0), desc_add(dqx0, qb * kTileBytes),
-                                         desc_add(dw0, slot * kWBytes));
-                        umma_commit(&bar[B_U_FULL0 + g]);
-                        umma_commit(&bar[B_W_EMPTY0 + slot]);
+                        const uint64_t dw = desc_add(dw0, t * 2 * kWBytes);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_bf16(tmem + kTsU, dq + 2 * kk, dw + 2 * kk, idU, kk > 0 ? 1u : 0u);
+                        umma_commit(&bar[T_UF]);
                     }
-                    umma_commit(QE(qb));
+                    umma_commit(&bar[T_QE0 + qb]);
                 }
             }
-        } else {
+        } else if (warp == 1) {
             // ------------------------------------------------------ main MMA issuer
             if (lane == 0) {
-                uint32_t ph_vf = 0, ph_pqf = 0, ph_pkf = 0, ph_psm = 0, ph_oe = 0, ph_sbf = 0;
+                uint32_t ph_pqf = 0, ph_pkf = 0, ph_vf = 0, ph_psm = 0, ph_oe = 0, ph_sbf = 0;
                 constexpr uint32_t idP = idesc_bf16(128, 128, 0, 0);
                 constexpr uint32_t idO = idesc_bf16(128, 80, 0, 1);
-                constexpr uint32_t idPV = idesc_bf16(128, 80, 0, 1);
+                constexpr uint32_t idPV = idesc_bf16(128, 64, 0, 1);
                 const uint32_t st_sbo = static_cast<uint32_t>(kp.F) * 16;
+                const uint64_t dph = desc_phik(sbase + L.phik);
+                const uint64_t dv = sdesc(sbase + L.v, kTileBytes, 1024, kLayoutSW128);
+                const uint32_t aq = tmem + kTsQ;
                 for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
                     const bool last = tile + 1 == sg.t_end;
+                    bool have_v = false;
                     for (int t = 0; t < NT; ++t) {
-                        const int pslot = t & 1;
-                        {
-                            uint32_t ph = (ph_pqf >> pslot) & 1u;
-                            wt.wait(&bar[B_PQ_FULL0 + pslot], ph);
-                            ph_pqf ^= 1u << pslot;
-                        }
+                        wt.wait(&bar[T_PQF], ph_pqf);
                         {
                             uint32_t ph = (ph_pkf >> t) & 1u;
-                            wt.wait(pk_full(bar, t), ph);
+                            wt.wait(&bar[T_PKF0 + t], ph);
                             ph_pkf ^= 1u << t;
                         }
                         if (t == 0 && tile > sg.t_begin) {
-                            wt.wait(&bar[B_SBF_READY], ph_sbf);
-                            wt.wait(&bar[B_O_EMPTY], ph_oe);
+                            wt.wait(&bar[T_SBF], ph_sbf);
+                            wt.wait(&bar[T_OE], ph_oe);
                         }
                         tc_fence_after();
-                        // descriptors once per slice, stepped by adds over its 4 K steps
-                        const uint64_t ad = desc_kmajor(sbase + L.phiq + pslot * kTileBytes);
                         const uint64_t bk = desc_kmajor(sbase + L.phik + t * kTileBytes);
                         const uint64_t bs = sdesc(sbase + L.st + t * (kSlice / 8) * 128, 128, st_sbo, kLayoutNone);
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
                             const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-                            umma_bf16(tmem + kColP, ad + 2 * kk, bk + 2 * kk, idP, acc);
-                            umma_bf16(tmem + kColO, ad + 2 * kk, bs + 16 * kk, idO, acc);
+                            umma_bf16_ts(tmem + kTsP, aq + 8 * kk, bk + 2 * kk, idP, acc);
+                            umma_bf16_ts(tmem + kTsO, aq + 8 * kk, bs + 16 * kk, idO, acc);
                         }
-                        umma_commit(&bar[B_PQ_EMPTY0 + pslot]);
-                        if ((t & 1) == 1) {
-                            if (!last) {
-                                if (t == 1) wt.wait(&bar[B_V_FULL], ph_vf);
-                                issue_state_half(tmem, kColS, desc_phik(sbase + L.phik),
-                                                 desc_v(sbase + L.v, sbase + L.ones), t >> 1, false);
-                            }
-                            // the loader needs this half free again for the next tile
-                            if (!last) umma_commit(&bar[B_PK_FREE0 + (t >> 1)]);
+                        umma_commit(&bar[T_PQE]);
+                        // every state half but the last right after its two slices; the last
+                        // one after the scores, where it overlaps the masking
+                        if ((t & 1) == 1 && !last && (t >> 1) + 1 < halves) {
+                            if (!have_v) { wt.wait(&bar[T_VF], ph_vf); have_v = true; }
+                            issue_state_half64(tmem, dph, dv, t >> 1);
+                            umma_commit(&bar[T_PKFREE0 + (t >> 1)]);
                         }
                     }
-                    umma_commit(&bar[B_P_FULL]);
-                    if (last) wt.wait(&bar[B_V_FULL], ph_vf);
-                    wt.wait(&bar[B_PSM_FULL], ph_psm);
+                    umma_commit(&bar[T_PF]);
+                    if (!have_v) { wt.wait(&bar[T_VF], ph_vf); have_v = true; }
+                    if (!last) {
+                        tc_fence_after();
+                        issue_state_half64(tmem, dph, dv, halves - 1);
+                        umma_commit(&bar[T_PKFREE0 + halves - 1]);
+                        umma_commit(&bar[T_SD]);
+                    }
+                    wt.wait(&bar[T_PSM], ph_psm);
                     tc_fence_after();
-                    const uint64_t dvv = desc_v(sbase + L.v, sbase + L.ones);
+                    // keys [16kk, 16kk+16): chunk c = kk/2 sits at bf16 columns 32(c%2) + 16(c/2)
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_bf16_ts(tmem + kColO, tmem + kColP + 8 * kk, dvv + 128 * kk, idPV, 1u);
-                    umma_commit(&bar[B_TILE_DONE]);
-                    umma_commit(&bar[B_V_EMPTY]);
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const int c = kk >> 1;
+                        const uint32_t acol = 32 * (c & 1) + 16 * (c >> 1) + 8 * (kk & 1);
+                        umma_bf16_ts(tmem + kTsO, tmem + kTsP + acol, dv + 128 * kk, idPV, 1u);
+                    }
+                    umma_commit(&bar[T_TD]);
+                    umma_commit(&bar[T_VE]);
                 }
             }
         }
@@ -1161,31 +1365,31 @@ k_tc_causal_out_pk(const __grid_constant__ CUtensorMap tmq, const __grid_constan
             const uint32_t trow = tmem + ((32u * sp) << 16);
             for (int h = 0; h < halves; ++h) {
                 const int f = 128 * h + row;
-                float acc[64];
-#pragma unroll
-                for (int e = 0; e < 64; ++e) acc[e] = 0.0f;
+                uint32_t r0[32], r1[32];
                 float zf = 0.0f;
-                for (int s = 0; s < sg.seg; ++s) {
-                    const size_t segidx = static_cast<size_t>(sg.bh) * kp.nseg + s;
-                    const float4* src = reinterpret_cast<const float4*>(wsS + (segidx * kp.F + f) * 64);
+                // the earlier segments' sums, one 32-column half at a time
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const float4 x = src[q];
-                        acc[4 * q] += x.x; acc[4 * q + 1] += x.y; acc[4 * q + 2] += x.z; acc[4 * q + 3] += x.w;
+                for (int part = 0; part < 2; ++part) {
+                    uint32_t (&r)[32] = part ? r1 : r0;
+                    float acc[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) acc[e] = 0.0f;
+                    for (int s = 0; s < sg.seg; ++s) {
+                        const size_t segidx = static_cast<size_t>(sg.bh) * kp.nseg + s;
+                        const float4* src = reinterpret_cast<const float4*>(wsS + (segidx * kp.F + f) * 64 + 32 * part);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 x = src[q];
+                            acc[4 * q] += x.x; acc[4 * q + 1] += x.y; acc[4 * q + 2] += x.z; acc[4 * q + 3] += x.w;
+                        }
+                        if (part == 0) zf += wsZ[segidx * kp.F + f];
                     }
-                    zf += wsZ[segidx * kp.F + f];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(acc[e]);
+                    tmem_st32(trow + kTsS + 64 * h + 32 * part, r);
                 }
-                uint32_t r[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(acc[e]);
-                tmem_st32(trow + kColS + 80 * h, r);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(acc[32 + e]);
-                tmem_st32(trow + kColS + 80 * h + 32, r);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(zf);
-                tmem_st32(trow + kColS + 80 * h + 64, r);
-                write_state_row(sbase + L.st, kp.F, f, acc, zf);
+                write_state_row_u(sbase + L.st, kp.F, f, r0, r1, zf);
+                zpre[f] = zf;
             }
             tmem_wait_st();
         }
@@ -1196,121 +1400,120 @@ k_tc_causal_out_pk(const __grid_constant__ CUtensorMap tmq, const __grid_constan
         Waiter wt;
         const int64_t rowbase = static_cast<int64_t>(sg.bh) * kp.L;
         if (warp < 12) {
-            // ------------------------------------------ phi(q): group g, half g of slice t
+            // ---------------------------------------- phi(q) and the masked scores
             const int g = (warp >= 8) ? 1 : 0;
             const int sp = warp & 3;
             const uint32_t row = 32u * sp + lane;
             const uint32_t trow = tmem + ((32u * sp) << 16);
-            uint32_t ph_qf = 0, ph_uf = 0, ph_pqe = 0;
-            int uses0 = 0, uses1 = 0;
+            uint32_t ph_qf = 0, ph_uf = 0, ph_pqe = 0, ph_de = 0, ph_pf = 0;
+            bool slot_used = false;
             for (int tile = sg.t_begin, it = 0; tile < sg.t_end; ++tile, ++it) {
                 const int qb = it & 1;
                 uint32_t ph = (ph_qf >> qb) & 1u;
-                wt.wait(QF(qb), ph);
+                wt.wait(&bar[T_QF0 + qb], ph);
                 ph_qf ^= 1u << qb;
                 float inv, l2i;
                 row_scale(sm + L.q + qb * kTileBytes + row * 128, row, inv, l2i);
-                warp_arrive(QE(qb));
+                warp_arrive(&bar[T_QE0 + qb]);
                 for (int t = 0; t < NT; ++t) {
                     const float a = slice_val(kp.a2, t) * inv, b = slice_val(kp.b2, t) + l2i;
-                    const int pslot = t & 1;
-                    wt.wait(&bar[B_U_FULL0 + g], ph_uf);
+                    wt.wait(&bar[T_UF], ph_uf);
                     tc_fence_after();
                     uint32_t ur[32], pr[32];
-                    const uint32_t col = g ? kColU1 : kColU0;
-                    tmem_ld32(trow + col, ur);
-                    tmem_ld32(trow + col + 32, pr);
+                    tmem_ld32(trow + kTsU + 64 * g, ur);
+                    tmem_ld32(trow + kTsU + 64 * g + 32, pr);
                     tmem_wait_ld();
                     reg_fence(ur);
                     reg_fence(pr);
                     tc_fence_before();
-                    warp_arrive(&bar[B_U_EMPTY0 + g]);
-                    int& uses = pslot ? uses1 : uses0;
-                    if (uses > 0) {   // both groups wait for the same completion
-                        uint32_t pe = (ph_pqe >> pslot) & 1u;
-                        wt.wait(&bar[B_PQ_EMPTY0 + pslot], pe);
-                        ph_pqe ^= 1u << pslot;
-                    }
-                    ++uses;
-                    phi_sub_epilogue(ur, pr, a, b, sbase + L.phiq + pslot * kTileBytes, row, g, nullptr);
-                    fence_async_smem();
-                    warp_arrive(&bar[B_PQ_FULL0 + pslot]);
+                    warp_arrive(&bar[T_UE]);
+                    uint32_t pk[16];
+                    phi_pack(ur, pr, a, b, pk);
+                    // the slot is free once the MMAs of the previous slice have read it
+                    if (slot_used) wt.wait(&bar[T_PQE], ph_pqe);
+                    slot_used = true;
+                    tmem_st16(trow + kTsQ + 16 * g, pk);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    warp_arrive(&bar[T_PQF]);
+                    // the previous tile's scores are complete once its last slice was read
+                    if (t == 0 && it > 0) ts_mask_scores(bar, wt, ph_pf, ph_de, trow, row, lane, sp, g, dens, it - 1);
                 }
             }
+            ts_mask_scores(bar, wt, ph_pf, ph_de, trow, row, lane, sp, g, dens, sg.t_end - 1 - sg.t_begin);
         } else {
-            // ------------------------------------------------------------ tile tail
-            const int sp = warp & 3;
+            // ------------------- column sums of phi(k), state copy for the next readout, outputs
+            const int sp = warp & 3, w = warp - 12;
             const uint32_t row = 32u * sp + lane;
             const uint32_t trow = tmem + ((32u * sp) << 16);
-            uint32_t ph_pf = 0, ph_td = 0;
-            for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
-                wt.wait(&bar[B_P_FULL], ph_pf);
-                tc_fence_after();
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t pk[16];
-                    if (c <= sp) {
-                        uint32_t pv[32];
-                        tmem_ld32(trow + kColP + 32 * c, pv);
-                        tmem_wait_ld();
-                        reg_fence(pv);
-                        if (c < sp) {
-#pragma unroll
-                            for (int j = 0; j < 16; ++j)
-                                pk[j] = pack_bf16(__uint_as_float(pv[2 * j]), __uint_as_float(pv[2 * j + 1]));
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 16; ++j)
-                                pk[j] = pack_bf16((2 * j <= lane) ? __uint_as_float(pv[2 * j]) : 0.0f,
-                                                  (2 * j + 1 <= lane) ? __uint_as_float(pv[2 * j + 1]) : 0.0f);
+            uint32_t ph_td = 0, ph_df = 0, ph_sd = 0, ph_pkf = 0;
+            // warp w < F/64: this segment's running sum of phi(k) over the tokens of its
+            // tiles so far, features 64w + 2 lane and 64w + 2 lane + 1
+            float zr0 = 0.0f, zr1 = 0.0f;
+            const int zf0 = kSlice * w + 2 * lane;
+            const uint32_t zbase = sbase + L.phik + w * kTileBytes + (lane & 3) * 4;
+            for (int tile = sg.t_begin, it = 0; tile < sg.t_end; ++tile, ++it) {
+                const bool last = tile + 1 == sg.t_end;
+                if (!last) {
+                    const int zb = it & 1;
+                    if (w < NT) {
+                        wt.wait(&bar[T_PKF0 + w], ph_pkf);
+                        float c0 = 0.0f, c1 = 0.0f;
+                        // row r, features 2 lane, 2 lane + 1: 16-byte chunk lane/4 of the
+                        // 128-byte swizzled row, at chunk (lane/4) ^ (r & 7)
+#pragma unroll 8
+                        for (int r = 0; r < kTile; ++r) {
+                            const uint32_t v2 = ld_shared_u32(zbase + r * 128 + (((lane >> 2) ^ (r & 7)) << 4));
+                            c0 += __uint_as_float(v2 << 16);
+                            c1 += __uint_as_float(v2 & 0xFFFF0000u);
                         }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) pk[j] = 0u;
+                        zr0 += c0;
+                        zr1 += c1;
+                        warp_arrive(&bar[T_ZC0 + (w >> 1)]);
+                        ztile[zb * kp.F + zf0] = zpre[zf0] + zr0;
+                        ztile[zb * kp.F + zf0 + 1] = zpre[zf0 + 1] + zr1;
                     }
-                    tmem_st16(trow + kColP + 16 * c, pk);
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                warp_arrive(&bar[B_PSM_FULL]);
-                if (tile + 1 < sg.t_end) {
+                    named_bar_sync(2, 128);
+                    wt.wait(&bar[T_SD], ph_sd);
+                    tc_fence_after();
                     for (int h = 0; h < halves; ++h) {
-                        const int f = 128 * h + row;
-                        uint32_t r0s[32], r1s[32], zr;
-                        tmem_ld32(trow + kColS + 80 * h, r0s);
-                        tmem_ld32(trow + kColS + 80 * h + 32, r1s);
-                        tmem_ld1(trow + kColS + 80 * h + 64, zr);
-                        tmem_wait_ld();
-                        reg_fence(r0s);
-                        reg_fence(r1s);
-                        reg_fence1(zr);
-                        float sv[64];
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            sv[e] = __uint_as_float(r0s[e]);
-                            sv[32 + e] = __uint_as_float(r1s[e]);
+                        const int f = 128 * h + static_cast<int>(row);
+#pragma unroll 1
+                        for (int part = 0; part < 2; ++part) {
+                            uint32_t sv[32];
+                            tmem_ld32(trow + kTsS + 64 * h + 32 * part, sv);
+                            tmem_wait_ld();
+                            reg_fence(sv);
+                            write_state_cols32(sbase + L.st, kp.F, f, part, sv);
                         }
-                        write_state_row(sbase + L.st, kp.F, f, sv, __uint_as_float(zr));
+                        write_state_z(sbase + L.st, kp.F, f, ztile[zb * kp.F + f]);
                     }
                     fence_async_smem();
                     tc_fence_before();
-                    warp_arrive(&bar[B_SBF_READY]);
+                    warp_arrive(&bar[T_SBF]);
                 }
-                wt.wait(&bar[B_TILE_DONE], ph_td);
+                wt.wait(&bar[T_TD], ph_td);
                 tc_fence_after();
                 uint32_t o0[32], o1[32], dr;
-                tmem_ld32(trow + kColO, o0);
-                tmem_ld32(trow + kColO + 32, o1);
-                tmem_ld1(trow + kColO + 64, dr);
+                tmem_ld32(trow + kTsO, o0);
+                tmem_ld32(trow + kTsO + 32, o1);
+                tmem_ld1(trow + kTsO + 64, dr);
                 tmem_wait_ld();
                 reg_fence(o0);
                 reg_fence(o1);
                 reg_fence1(dr);
                 tc_fence_before();
-                warp_arrive(&bar[B_O_EMPTY]);
+                warp_arrive(&bar[T_OE]);
+                const int par = it & 1;
+                {
+                    uint32_t pd = (ph_df >> par) & 1u;
+                    wt.wait(&bar[T_DF0 + par], pd);
+                    ph_df ^= 1u << par;
+                }
+                const float d = __uint_as_float(dr) + dens[(2 * par) * kTile + row] + dens[(2 * par + 1) * kTile + row];
+                warp_arrive(&bar[T_DE0 + par]);
                 const int grow = tile * kTile + static_cast<int>(row);
-                if (grow < kp.L)
-                    finish_row(kp, o0, o1, __uint_as_float(dr), rowbase + grow, out, den);
+                if (grow < kp.L) finish_row_t<(kAcc & 1) != 0, (kAcc & 2) != 0>(kp, o0, o1, d, rowbase + grow, out, den);
             }
         }
         wt.report(err);
@@ -1769,10 +1972,17 @@ cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, 
                 k_tc_causal_state<true><<<BH * nseg, kThreads, sms, st>>>(mk, mv, mw, mpk, kp, wsS, wsZ, err);
                 if ((e = cudaGetLastError()) != cudaSuccess) return e;
             }
-            const size_t smo = smem_outpk_layout(Fc).total + 1024;
-            if ((e = set_smem(k_tc_causal_out_pk, smo)) != cudaSuccess) return e;
+            const size_t smo = smem_outts_layout(Fc).total + 1024;
+            auto kern = k_tc_causal_out_ts<0>;
+            switch ((kp.acc_in ? 1 : 0) | (kp.acc_out ? 2 : 0)) {
+            case 1: kern = k_tc_causal_out_ts<1>; break;
+            case 2: kern = k_tc_causal_out_ts<2>; break;
+            case 3: kern = k_tc_causal_out_ts<3>; break;
+            default: break;
+            }
+            if ((e = set_smem(kern, smo)) != cudaSuccess) return e;
             TraceScope trace_("tc_qphi_out", st);
-            k_tc_causal_out_pk<<<BH * nseg, kOutThreads, smo, st>>>(mq, mpk, mv, mw, kp, wsS, wsZ, o, den, err);
+            kern<<<BH * nseg, kOutThreads, smo, st>>>(mq, mpk, mv, mw, kp, wsS, wsZ, o, den, err);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
             continue;
         }
