@@ -334,6 +334,23 @@ __device__ __forceinline__ void fill_ones(unsigned char* ones)
 }
 
 
+// State kernel projection order: the k-th projection of the li-th tile of a segment covers
+// the 64-feature slice state_slice(li, k) and reads its operand from slot k % 2.  With four
+// slices the odd tiles take them in the order 2, 3, 0, 1, so each slot's last slice of a tile
+// is its first of the next and only two of the four operands are reloaded per tile; with two
+// slices the slots never change.
+__device__ __forceinline__ int state_slice(int li, int k, int NT)
+{
+    return (NT == 4 && (li & 1)) ? (k ^ 2) : k;
+}
+// whether projection (li, k) needs its slot (re)loaded (the slot held another slice before)
+__device__ __forceinline__ bool state_reload(int li, int k, int NT)
+{
+    if (li == 0 && k < 2) return true;
+    const int pli = k >= 2 ? li : li - 1, pk = k >= 2 ? k - 2 : k + NT - 2;
+    return state_slice(pli, pk, NT) != state_slice(li, k, NT);
+}
+
 // ------------------------------------------------------------ state kernel
 // grid = BH * (nseg - 1) (causal: the last segment's sum is never needed) or BH * nseg
 // (bidirectional): segment seg of sequence bh writes
@@ -403,15 +420,15 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         // k tiles (two buffers) and the projection operands
         if (lane == 0) {
             uint32_t ph_ke = 0, ph_we = 0x3u;  // both operand slots start free
-            int n_glob = 0;
             for (int j = 0; j < 2 && sg.t_begin + j < sg.t_end; ++j) {
                 mbar_arrive_expect_tx(KF(j), kTileBytes);
                 tma_load_3d(sm + L.k + j * kTileBytes, &tmk, KF(j), 0, (sg.t_begin + j) * kTile, sg.bh);
             }
             for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
-                const int kb = (tile - sg.t_begin) & 1;
-                for (int n = 0; n < NT; ++n, ++n_glob) {
-                    const int slot = n_glob & 1;
+                const int li = tile - sg.t_begin, kb = li & 1;
+                for (int k = 0; k < NT; ++k) {
+                    if (!state_reload(li, k, NT)) continue;   // the slot already holds it
+                    const int slot = k & 1, n = state_slice(li, k, NT);
                     uint32_t ph = (ph_we >> slot) & 1u;
                     wt.wait(&bar[B_W_EMPTY0 + slot], ph);
                     ph_we ^= (1u << slot);
@@ -443,7 +460,6 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     } else if (warp == 1) {
         if (lane == 0) {
             uint32_t ph_kf = 0, ph_vf = 0, ph_wf = 0, ph_ue0 = 1, ph_ue1 = 1, ph_pk = 0;  // ph_kf, ph_pk: bit per buffer
-            int n_glob = 0;
             constexpr uint32_t idU = idesc_bf16(128, 128, 0, 0);
             const uint64_t dk0 = desc_kmajor(sbase + L.k), dw0 = desc_kmajor(sbase + L.w);
             const uint64_t dph0 = desc_phik(sbase + L.phik), dv = desc_v(sbase + L.v, sbase + L.ones);
@@ -459,12 +475,15 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                         ph_kf ^= 1u << b;
                     }
                     const uint64_t dk = desc_add(dk0, b * kTileBytes);
-                    for (int n = 0; n < NT; ++n, ++n_glob) {
-                        const int slot = n_glob & 1;
-                        uint32_t ph = (ph_wf >> slot) & 1u;
-                        wt.wait(&bar[B_W_FULL0 + slot], ph);
-                        ph_wf ^= (1u << slot);
-                        const int ub = n & 1;
+                    const int li = tile - sg.t_begin;
+                    for (int k = 0; k < NT; ++k) {
+                        const int slot = k & 1;
+                        if (state_reload(li, k, NT)) {
+                            uint32_t ph = (ph_wf >> slot) & 1u;
+                            wt.wait(&bar[B_W_FULL0 + slot], ph);
+                            ph_wf ^= (1u << slot);
+                        }
+                        const int ub = k & 1;
                         wt.wait(&bar[B_U_EMPTY0 + ub], ub ? ph_ue1 : ph_ue0);
                         tc_fence_after();
                         const uint64_t dw = desc_add(dw0, slot * kWStateBytes);
@@ -472,7 +491,9 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                         for (int kk = 0; kk < 4; ++kk)
                             umma_bf16(tmem + kColUS + 128 * ub, dk + 2 * kk, dw + 2 * kk, idU, kk > 0 ? 1u : 0u);
                         umma_commit(&bar[B_U_FULL0 + ub]);
-                        umma_commit(&bar[B_W_EMPTY0 + slot]);
+                        // the slot is released when its next use reloads it
+                        if (k + 2 < NT ? state_reload(li, k + 2, NT) : state_reload(li + 1, k + 2 - NT, NT))
+                            umma_commit(&bar[B_W_EMPTY0 + slot]);
                     }
                     umma_commit(KE(b));
                 }
@@ -534,7 +555,8 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 if (kStorePhi) wt.wait(&ST[b], ps);
                 ph_td ^= (1u << b);
             }
-            for (int n = grp; n < NT; n += 2) {
+            for (int k = grp; k < NT; k += 2) {
+                const int n = state_slice(li, k, NT);
                 wt.wait(&bar[B_U_FULL0 + grp], ph_uf);
                 tc_fence_after();
                 const float a = slice_val(kp.a2, n) * inv, bb = slice_val(kp.b2, n) + l2i;
@@ -1209,6 +1231,38 @@ k_tc_causal_out_ts(const __grid_constant__ CUtensorMap tmq, const __grid_constan
         uint4* p = reinterpret_cast<uint4*>(sm + L.st);
         for (int i = tid; i < NT * kStBytes / 16; i += kOutThreads) p[i] = make_uint4(0, 0, 0, 0);
     }
+    {
+        // The state entering the segment, the sum of the earlier segments' sums, by all
+        // threads with many loads in flight (one thread per 16-byte piece, segments two at a
+        // time), into the phi(k) slices' space, which no copy has reached yet: fp32 [F][64],
+        // the piece e4 of row f at piece position e4 ^ (f % 16) so that the tail warps, one
+        // row per lane, read it without bank conflicts; z into zpre.
+        float* sacc = reinterpret_cast<float*>(sm + L.phik);
+        const int J = kp.F / 32;   // pieces per thread: F * 16 / 512
+        float4 acc[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        float zsum = 0.0f;
+#pragma unroll 2
+        for (int s = 0; s < sg.seg; ++s) {
+            const size_t segidx = static_cast<size_t>(sg.bh) * kp.nseg + s;
+            const float4* src = reinterpret_cast<const float4*>(wsS + segidx * kp.F * 64);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (j < J) {
+                    const float4 x = src[tid + kOutThreads * j];
+                    acc[j].x += x.x; acc[j].y += x.y; acc[j].z += x.z; acc[j].w += x.w;
+                }
+            if (tid < kp.F) zsum += wsZ[segidx * kp.F + tid];
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (j < J) {
+                const int c = tid + kOutThreads * j, f = c >> 4, e4 = c & 15;
+                *reinterpret_cast<float4*>(sacc + f * 64 + ((e4 ^ (f & 15)) << 2)) = acc[j];
+            }
+        if (tid < kp.F) zpre[tid] = zsum;
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1363,33 +1417,21 @@ k_tc_causal_out_ts(const __grid_constant__ CUtensorMap tmq, const __grid_constan
             const int sp = warp & 3;
             const uint32_t row = 32u * sp + lane;
             const uint32_t trow = tmem + ((32u * sp) << 16);
+            const float* sacc = reinterpret_cast<const float*>(sm + L.phik);
             for (int h = 0; h < halves; ++h) {
                 const int f = 128 * h + row;
                 uint32_t r0[32], r1[32];
-                float zf = 0.0f;
-                // the earlier segments' sums, one 32-column half at a time
 #pragma unroll
-                for (int part = 0; part < 2; ++part) {
-                    uint32_t (&r)[32] = part ? r1 : r0;
-                    float acc[32];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) acc[e] = 0.0f;
-                    for (int s = 0; s < sg.seg; ++s) {
-                        const size_t segidx = static_cast<size_t>(sg.bh) * kp.nseg + s;
-                        const float4* src = reinterpret_cast<const float4*>(wsS + (segidx * kp.F + f) * 64 + 32 * part);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            const float4 x = src[q];
-                            acc[4 * q] += x.x; acc[4 * q + 1] += x.y; acc[4 * q + 2] += x.z; acc[4 * q + 3] += x.w;
-                        }
-                        if (part == 0) zf += wsZ[segidx * kp.F + f];
-                    }
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(acc[e]);
-                    tmem_st32(trow + kTsS + 64 * h + 32 * part, r);
+                for (int e4 = 0; e4 < 16; ++e4) {
+                    const float4 x = *reinterpret_cast<const float4*>(sacc + f * 64 + ((e4 ^ (f & 15)) << 2));
+                    uint32_t* r = e4 < 8 ? r0 : r1;
+                    const int c = 4 * (e4 & 7);
+                    r[c] = __float_as_uint(x.x); r[c + 1] = __float_as_uint(x.y);
+                    r[c + 2] = __float_as_uint(x.z); r[c + 3] = __float_as_uint(x.w);
                 }
-                write_state_row_u(sbase + L.st, kp.F, f, r0, r1, zf);
-                zpre[f] = zf;
+                tmem_st32(trow + kTsS + 64 * h, r0);
+                tmem_st32(trow + kTsS + 64 * h + 32, r1);
+                write_state_row_u(sbase + L.st, kp.F, f, r0, r1, zpre[f]);
             }
             tmem_wait_st();
         }
