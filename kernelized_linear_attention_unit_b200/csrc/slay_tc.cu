@@ -632,6 +632,81 @@ __device__ __forceinline__ void write_state_row(uint32_t st, int F, int f, const
     st_shared_v4(base + 8 * sbo, pack_bf16(z, 0.0f), 0u, 0u, 0u);
 }
 
+// Row f of the [S | z] copy (the layout of write_state_row) from the fp32 bit patterns of
+// S[f][0..32) (s0) and S[f][32..64) (s1).
+__device__ __forceinline__ void write_state_row_u(uint32_t st, int F, int f, const uint32_t (&s0)[32],
+                                                  const uint32_t (&s1)[32], float z)
+{
+    const uint32_t base = st + (f >> 3) * 128 + (f & 7) * 16;
+    const uint32_t sbo = static_cast<uint32_t>(F) * 16;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+        const uint32_t* s = g < 4 ? s0 : s1;
+        const int c = 8 * (g & 3);
+        st_shared_v4(base + g * sbo,
+                     pack_bf16(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                     pack_bf16(__uint_as_float(s[c + 2]), __uint_as_float(s[c + 3])),
+                     pack_bf16(__uint_as_float(s[c + 4]), __uint_as_float(s[c + 5])),
+                     pack_bf16(__uint_as_float(s[c + 6]), __uint_as_float(s[c + 7])));
+    }
+    st_shared_v4(base + 8 * sbo, pack_bf16(z, 0.0f), 0u, 0u, 0u);
+}
+
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+// The sum over segments [0, nseg) of sequence bh of the per-segment sums S [BH][nseg][F][64]
+// and z [BH][nseg][F], by all kOutThreads threads with 16-byte coalesced loads (one thread
+// per piece, segments two at a time): S into sacc as fp32 [F][64] with the piece e4 of row f
+// at piece position e4 ^ (f % 16) (read back one row per lane without bank conflicts, see
+// read_state_sum), z into zacc.  The caller synchronises the block before reading them.
+__device__ __forceinline__ void sum_segments(const float* __restrict__ wsS, const float* __restrict__ wsZ,
+                                             int bh, int nseg, int nsum, int F, float* sacc, float* zacc)
+{
+    const int tid = threadIdx.x;
+    const int J = F / 32;   // pieces per thread: F * 16 / kOutThreads
+    float4 acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    float zsum = 0.0f;
+#pragma unroll 2
+    for (int s = 0; s < nsum; ++s) {
+        const size_t segidx = static_cast<size_t>(bh) * nseg + s;
+        const float4* src = reinterpret_cast<const float4*>(wsS + segidx * F * 64);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (j < J) {
+                const float4 x = src[tid + kOutThreads * j];
+                acc[j].x += x.x; acc[j].y += x.y; acc[j].z += x.z; acc[j].w += x.w;
+            }
+        if (tid < F) zsum += wsZ[segidx * F + tid];
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        if (j < J) {
+            const int c = tid + kOutThreads * j, f = c >> 4, e4 = c & 15;
+            *reinterpret_cast<float4*>(sacc + f * 64 + ((e4 ^ (f & 15)) << 2)) = acc[j];
+        }
+    if (tid < F) zacc[tid] = zsum;
+}
+
+// Row f of a sum_segments result as fp32 bit patterns: columns [0, 32) into r0, [32, 64) r1
+__device__ __forceinline__ void read_state_sum(const float* sacc, int f, uint32_t (&r0)[32], uint32_t (&r1)[32])
+{
+#pragma unroll
+    for (int e4 = 0; e4 < 16; ++e4) {
+        const float4 x = *reinterpret_cast<const float4*>(sacc + f * 64 + ((e4 ^ (f & 15)) << 2));
+        uint32_t* r = e4 < 8 ? r0 : r1;
+        const int c = 4 * (e4 & 7);
+        r[c] = __float_as_uint(x.x); r[c + 1] = __float_as_uint(x.y);
+        r[c + 2] = __float_as_uint(x.z); r[c + 3] = __float_as_uint(x.w);
+    }
+}
+
 // Output kernel: phi(k) slice t (of at most 4) is signalled on its own barrier, so the
 // phi(k) warps, which may run a tile ahead, never complete a phase the MMA warp has not
 // yet waited for.
@@ -690,6 +765,10 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         uint4* p = reinterpret_cast<uint4*>(sm + L.st);
         for (int i = tid; i < NT * kStBytes / 16; i += kOutThreads) p[i] = make_uint4(0, 0, 0, 0);
     }
+    // the state entering the segment (sum of the earlier segments' sums) into the phi(k)
+    // space, z into the phi(q) space (neither is written before the next block barrier)
+    sum_segments(wsS, wsZ, sg.bh, kp.nseg, sg.seg, kp.F, reinterpret_cast<float*>(sm + L.phik),
+                 reinterpret_cast<float*>(sm + L.phiq));
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -829,31 +908,15 @@ k_tc_causal_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             const uint32_t trow = tmem + ((32u * sp) << 16);
             for (int h = 0; h < halves; ++h) {
                 const int f = 128 * h + row;
-                float acc[64];
-    #pragma unroll
-                for (int e = 0; e < 64; ++e) acc[e] = 0.0f;
-                float zf = 0.0f;
-                for (int s = 0; s < sg.seg; ++s) {
-                    const size_t segidx = static_cast<size_t>(sg.bh) * kp.nseg + s;
-                    const float4* src = reinterpret_cast<const float4*>(wsS + (segidx * kp.F + f) * 64);
-    #pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const float4 x = src[q];
-                        acc[4 * q] += x.x; acc[4 * q + 1] += x.y; acc[4 * q + 2] += x.z; acc[4 * q + 3] += x.w;
-                    }
-                    zf += wsZ[segidx * kp.F + f];
-                }
-                uint32_t r[32];
-    #pragma unroll
-                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(acc[e]);
-                tmem_st32(trow + kColS + 80 * h, r);
-    #pragma unroll
-                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(acc[32 + e]);
-                tmem_st32(trow + kColS + 80 * h + 32, r);
-    #pragma unroll
-                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(zf);
-                tmem_st32(trow + kColS + 80 * h + 64, r);  // z columns (a later half rewrites its own)
-                write_state_row(sbase + L.st, kp.F, f, acc, zf);
+                uint32_t r0[32], r1[32];
+                read_state_sum(reinterpret_cast<const float*>(sm + L.phik), f, r0, r1);
+                const float zf = reinterpret_cast<const float*>(sm + L.phiq)[f];
+                tmem_st32(trow + kColS + 80 * h, r0);
+                tmem_st32(trow + kColS + 80 * h + 32, r1);
+                write_state_row_u(sbase + L.st, kp.F, f, r0, r1, zf);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) r0[e] = __float_as_uint(zf);
+                tmem_st32(trow + kColS + 80 * h + 64, r0);  // z columns (a later half rewrites its own)
             }
             tmem_wait_st();
         }
@@ -1054,33 +1117,6 @@ __host__ __device__ inline SmemOutTs smem_outts_layout(int F)
     return s;
 }
 
-// Row f of the [S | z] copy (the layout of write_state_row) from the fp32 bit patterns of
-// S[f][0..32) (s0) and S[f][32..64) (s1).
-__device__ __forceinline__ void write_state_row_u(uint32_t st, int F, int f, const uint32_t (&s0)[32],
-                                                  const uint32_t (&s1)[32], float z)
-{
-    const uint32_t base = st + (f >> 3) * 128 + (f & 7) * 16;
-    const uint32_t sbo = static_cast<uint32_t>(F) * 16;
-#pragma unroll
-    for (int g = 0; g < 8; ++g) {
-        const uint32_t* s = g < 4 ? s0 : s1;
-        const int c = 8 * (g & 3);
-        st_shared_v4(base + g * sbo,
-                     pack_bf16(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
-                     pack_bf16(__uint_as_float(s[c + 2]), __uint_as_float(s[c + 3])),
-                     pack_bf16(__uint_as_float(s[c + 4]), __uint_as_float(s[c + 5])),
-                     pack_bf16(__uint_as_float(s[c + 6]), __uint_as_float(s[c + 7])));
-    }
-    st_shared_v4(base + 8 * sbo, pack_bf16(z, 0.0f), 0u, 0u, 0u);
-}
-
-__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr)
-{
-    uint32_t v;
-    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-    return v;
-}
-
 // Columns [32 part, 32 part + 32) of row f of the [S | z] copy (four of its 16-byte pieces)
 __device__ __forceinline__ void write_state_cols32(uint32_t st, int F, int f, int part, const uint32_t (&s)[32])
 {
@@ -1231,38 +1267,9 @@ k_tc_causal_out_ts(const __grid_constant__ CUtensorMap tmq, const __grid_constan
         uint4* p = reinterpret_cast<uint4*>(sm + L.st);
         for (int i = tid; i < NT * kStBytes / 16; i += kOutThreads) p[i] = make_uint4(0, 0, 0, 0);
     }
-    {
-        // The state entering the segment, the sum of the earlier segments' sums, by all
-        // threads with many loads in flight (one thread per 16-byte piece, segments two at a
-        // time), into the phi(k) slices' space, which no copy has reached yet: fp32 [F][64],
-        // the piece e4 of row f at piece position e4 ^ (f % 16) so that the tail warps, one
-        // row per lane, read it without bank conflicts; z into zpre.
-        float* sacc = reinterpret_cast<float*>(sm + L.phik);
-        const int J = kp.F / 32;   // pieces per thread: F * 16 / 512
-        float4 acc[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        float zsum = 0.0f;
-#pragma unroll 2
-        for (int s = 0; s < sg.seg; ++s) {
-            const size_t segidx = static_cast<size_t>(sg.bh) * kp.nseg + s;
-            const float4* src = reinterpret_cast<const float4*>(wsS + segidx * kp.F * 64);
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                if (j < J) {
-                    const float4 x = src[tid + kOutThreads * j];
-                    acc[j].x += x.x; acc[j].y += x.y; acc[j].z += x.z; acc[j].w += x.w;
-                }
-            if (tid < kp.F) zsum += wsZ[segidx * kp.F + tid];
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            if (j < J) {
-                const int c = tid + kOutThreads * j, f = c >> 4, e4 = c & 15;
-                *reinterpret_cast<float4*>(sacc + f * 64 + ((e4 ^ (f & 15)) << 2)) = acc[j];
-            }
-        if (tid < kp.F) zpre[tid] = zsum;
-    }
+    // The state entering the segment, the sum of the earlier segments' sums, into the phi(k)
+    // slices' space (no copy has reached it yet), z into zpre
+    sum_segments(wsS, wsZ, sg.bh, kp.nseg, sg.seg, kp.F, reinterpret_cast<float*>(sm + L.phik), zpre);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1417,18 +1424,10 @@ k_tc_causal_out_ts(const __grid_constant__ CUtensorMap tmq, const __grid_constan
             const int sp = warp & 3;
             const uint32_t row = 32u * sp + lane;
             const uint32_t trow = tmem + ((32u * sp) << 16);
-            const float* sacc = reinterpret_cast<const float*>(sm + L.phik);
             for (int h = 0; h < halves; ++h) {
                 const int f = 128 * h + row;
                 uint32_t r0[32], r1[32];
-#pragma unroll
-                for (int e4 = 0; e4 < 16; ++e4) {
-                    const float4 x = *reinterpret_cast<const float4*>(sacc + f * 64 + ((e4 ^ (f & 15)) << 2));
-                    uint32_t* r = e4 < 8 ? r0 : r1;
-                    const int c = 4 * (e4 & 7);
-                    r[c] = __float_as_uint(x.x); r[c + 1] = __float_as_uint(x.y);
-                    r[c + 2] = __float_as_uint(x.z); r[c + 3] = __float_as_uint(x.w);
-                }
+                read_state_sum(reinterpret_cast<const float*>(sm + L.phik), f, r0, r1);
                 tmem_st32(trow + kTsS + 64 * h, r0);
                 tmem_st32(trow + kTsS + 64 * h + 32, r1);
                 write_state_row_u(sbase + L.st, kp.F, f, r0, r1, zpre[f]);
@@ -1574,7 +1573,7 @@ k_tc_causal_out_ts(const __grid_constant__ CUtensorMap tmq, const __grid_constan
 // each 64-feature slice); warp 1 issues the readout O = phiQ [S | z] (N = 80) slice by slice;
 // warps 12-15 first build the bf16 copy of the summed state, then write the outputs.
 struct SmemBidir {
-    uint32_t w, q, phiq, st, bar, tmem, total;
+    uint32_t w, q, phiq, st, scr, zt, bar, tmem, total;
 };
 
 __host__ __device__ inline SmemBidir smem_bidir_layout(int F)
@@ -1584,7 +1583,9 @@ __host__ __device__ inline SmemBidir smem_bidir_layout(int F)
     s.q = kWSlots * kWBytes;                // 2 buffers
     s.phiq = s.q + 2 * kTileBytes;          // 2 slots of 64 features
     s.st = s.phiq + 2 * kTileBytes;
-    s.bar = s.st + (F / kSlice) * kStBytes;
+    s.scr = s.st + (F / kSlice) * kStBytes;   // fp32 [F][64]: the summed state, once
+    s.zt = s.scr + F * 256;                   // fp32 [F]: the summed z
+    s.bar = s.zt + F * 4;
     s.tmem = s.bar + NUM_BARS * 8;
     s.total = s.tmem + 16;
     return s;
@@ -1630,30 +1631,21 @@ k_tc_bidir_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
         uint4* p = reinterpret_cast<uint4*>(sm + L.st);
         for (int i = tid; i < NT * kStBytes / 16; i += kOutThreads) p[i] = make_uint4(0, 0, 0, 0);
     }
+    // [S | z] of the whole sequence: the sum of all its segments
+    sum_segments(wsS, wsZ, sg.bh, kp.nseg, kp.nseg, kp.F, reinterpret_cast<float*>(sm + L.scr),
+                 reinterpret_cast<float*>(sm + L.zt));
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
-    if (warp >= 12) {   // [S | z] of the whole sequence: sum of all its segments
+    if (warp >= 12) {
         const int sp = warp & 3;
         const uint32_t row = 32u * sp + lane;
         for (int h = 0; h < halves; ++h) {
             const int f = 128 * h + row;
-            float acc[64];
-#pragma unroll
-            for (int e = 0; e < 64; ++e) acc[e] = 0.0f;
-            float zf = 0.0f;
-            for (int s = 0; s < kp.nseg; ++s) {
-                const size_t segidx = static_cast<size_t>(sg.bh) * kp.nseg + s;
-                const float4* src = reinterpret_cast<const float4*>(wsS + (segidx * kp.F + f) * 64);
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const float4 x = src[q];
-                    acc[4 * q] += x.x; acc[4 * q + 1] += x.y; acc[4 * q + 2] += x.z; acc[4 * q + 3] += x.w;
-                }
-                zf += wsZ[segidx * kp.F + f];
-            }
-            write_state_row(sbase + L.st, kp.F, f, acc, zf);
+            uint32_t r0[32], r1[32];
+            read_state_sum(reinterpret_cast<const float*>(sm + L.scr), f, r0, r1);
+            write_state_row_u(sbase + L.st, kp.F, f, r0, r1, reinterpret_cast<const float*>(sm + L.zt)[f]);
         }
     }
     fence_async_smem();
