@@ -356,8 +356,9 @@ __device__ __forceinline__ bool state_reload(int li, int k, int NT)
 // (bidirectional): segment seg of sequence bh writes
 //   ws_S[bh][seg][f][e] = sum_{t in seg} phi(k_t)_f v_t[e],  ws_z[bh][seg][f] = sum phi(k_t)_f
 // Projections are 64 features wide (N = 128: two packed 32-feature operands), double
-// buffered in TMEM; epilogue group g takes the projections n with n % 2 == g.  Tile i uses
-// k and phi(k) buffer (i - first) % 2; warp 11 loads v.
+// buffered in TMEM (warp 1 issues them); epilogue group g takes the projections k with
+// k % 2 == g.  Tile i uses k and phi(k) buffer (i - first) % 2; warp 11 loads v and issues
+// the state updates.
 // kStorePhi: also write phi(k) of every tile (bf16, [BH][L][F]) through TMA for the output
 // kernel that reads it instead of recomputing it; warp 10 issues those stores.
 template <bool kStorePhi>
@@ -448,27 +449,39 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             }
         }
     } else if (warp == 11) {
-        // v tiles: one buffer, refilled once the previous tile's state update has read it
+        // v tiles (one buffer, refilled once the previous tile's state update has read it)
+        // and the state updates, issued here so that they never hold up the projections
         if (lane == 0) {
-            uint32_t ph_ve = 0;
+            uint32_t ph_ve = 0, ph_vf = 0, ph_pk = 0;   // ph_pk: bit per phi(k) buffer
+            const uint64_t dph0 = desc_phik(sbase + L.phik), dv = desc_v(sbase + L.v, sbase + L.ones);
             for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
+                const int b = (tile - sg.t_begin) & 1;
                 if (tile > sg.t_begin) wt.wait(VE, ph_ve);
                 mbar_arrive_expect_tx(VF, kTileBytes);
                 tma_load_3d(sm + L.v, &tmv, VF, 0, tile * kTile, sg.bh);
+                {
+                    uint32_t pp = (ph_pk >> b) & 1u;
+                    wt.wait(PKF(b), pp);
+                    ph_pk ^= 1u << b;
+                }
+                wt.wait(VF, ph_vf);
+                tc_fence_after();
+                for (int h = 0; h < halves; ++h)
+                    issue_state_half(tmem, kColSS, desc_add(dph0, b * phik_bytes), dv, h, tile == sg.t_begin);
+                umma_commit(VE);
+                umma_commit(&TD[b]);
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            uint32_t ph_kf = 0, ph_vf = 0, ph_wf = 0, ph_ue0 = 1, ph_ue1 = 1, ph_pk = 0;  // ph_kf, ph_pk: bit per buffer
+            uint32_t ph_kf = 0, ph_wf = 0, ph_ue0 = 1, ph_ue1 = 1;  // ph_kf: bit per buffer
             constexpr uint32_t idU = idesc_bf16(128, 128, 0, 0);
             const uint64_t dk0 = desc_kmajor(sbase + L.k), dw0 = desc_kmajor(sbase + L.w);
-            const uint64_t dph0 = desc_phik(sbase + L.phik), dv = desc_v(sbase + L.v, sbase + L.ones);
-            // software-pipelined: the projections of tile i are issued before the state
-            // update of tile i-1, whose phi(k) (the other buffer) is complete by then, so the
-            // phi(k) warps never wait for the next tile's projections behind that update
-            for (int tile = sg.t_begin; tile <= sg.t_end; ++tile) {
+            // the projections only (warp 11 issues the state updates): the phi(k) warps never
+            // wait for a projection behind an update
+            for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
                 const int b = (tile - sg.t_begin) & 1;
-                if (tile < sg.t_end) {
+                {
                     {
                         uint32_t pk = (ph_kf >> b) & 1u;
                         wt.wait(KF(b), pk);
@@ -496,21 +509,6 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                             umma_commit(&bar[B_W_EMPTY0 + slot]);
                     }
                     umma_commit(KE(b));
-                }
-                if (tile > sg.t_begin) {   // state update of the previous tile
-                    const int pb = b ^ 1;
-                    {
-                        uint32_t pp = (ph_pk >> pb) & 1u;
-                        wt.wait(PKF(pb), pp);
-                        ph_pk ^= 1u << pb;
-                    }
-                    wt.wait(VF, ph_vf);
-                    tc_fence_after();
-                    for (int h = 0; h < halves; ++h)
-                        issue_state_half(tmem, kColSS, desc_add(dph0, pb * phik_bytes), dv, h,
-                                         tile - 1 == sg.t_begin);
-                    umma_commit(VE);
-                    umma_commit(&TD[pb]);
                 }
             }
         }
