@@ -126,13 +126,17 @@ struct Seg {
     int bh, seg, t_begin, t_end;
 };
 
+// Segment `seg` of sequence bh: ntiles / nseg tiles each, the first ntiles % nseg segments one
+// more.  The longer segments come first because a later segment's output CTA also sums the
+// state of all earlier segments before its first tile.
 __device__ __forceinline__ Seg segment_of(int index, int nseg, int ntiles)
 {
     Seg s;
     s.bh = index / nseg;
     s.seg = index % nseg;
-    s.t_begin = static_cast<int>((static_cast<int64_t>(s.seg) * ntiles) / nseg);
-    s.t_end = static_cast<int>((static_cast<int64_t>(s.seg + 1) * ntiles) / nseg);
+    const int q = ntiles / nseg, r = ntiles % nseg;
+    s.t_begin = s.seg * q + (s.seg < r ? s.seg : r);
+    s.t_end = s.t_begin + q + (s.seg < r ? 1 : 0);
     return s;
 }
 
