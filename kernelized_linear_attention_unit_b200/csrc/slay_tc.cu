@@ -338,6 +338,12 @@ __device__ __forceinline__ void fill_ones(unsigned char* ones)
 }
 
 
+// Programmatic dependent launch: a grid launched with programmatic stream serialization may
+// start before the grid ahead of it in the stream has finished; griddep_wait blocks until that
+// grid has completed and its memory operations are visible (at once when there is none).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+
 // State kernel projection order: the k-th projection of the li-th tile of a segment covers
 // the 64-feature slice state_slice(li, k) and reads its operand from slot k % 2.  With four
 // slices the odd tiles take them in the order 2, 3, 0, 1, so each slot's last slice of a tile
@@ -383,6 +389,9 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     const uint32_t phik_bytes = NT * kTileBytes;
     const Seg sg = kp.all_segs ? segment_of(blockIdx.x, kp.nseg, kp.ntiles)
                                : segment_of(blockIdx.x + blockIdx.x / (kp.nseg - 1), kp.nseg, kp.ntiles);
+    // the readout kernel that follows may be scheduled now (onto SMs this grid leaves free,
+    // then onto those its CTAs release); it waits for this grid's results before reading them
+    griddep_launch_dependents();
     constexpr uint32_t kColUS = 0;     // 2 x 128: projections
     constexpr uint32_t kColSS = 256;   // 2 x 80 : [S | z]
     // barrier roles here: KF(b) / KE(b) the k buffers; VF / VE the V buffer; TD(b) = the
@@ -1264,6 +1273,14 @@ k_tc_causal_out_ts(const __grid_constant__ CUtensorMap tmq, const __grid_constan
         tma_prefetch_desc(&tmpk);
         tma_prefetch_desc(&tmv);
         tma_prefetch_desc(&tmw);
+        // W and the first two q tiles (regions the prologue below does not touch) load while
+        // the state entering the segment is summed
+        mbar_arrive_expect_tx(&bar[T_WF], NS * kWBytes);
+        for (int n = 0; n < NS; ++n) tma_load_2d(sm + L.w + n * kWBytes, &tmw, &bar[T_WF], 0, n * 64);
+        for (int j = 0; j < 2 && sg.t_begin + j < sg.t_end; ++j) {
+            mbar_arrive_expect_tx(&bar[T_QF0 + j], kTileBytes);
+            tma_load_3d(sm + L.q + j * kTileBytes, &tmq, &bar[T_QF0 + j], 0, (sg.t_begin + j) * kTile, sg.bh);
+        }
     }
     {   // the state copy: columns 65..79 stay zero
         uint4* p = reinterpret_cast<uint4*>(sm + L.st);
@@ -1271,6 +1288,7 @@ k_tc_causal_out_ts(const __grid_constant__ CUtensorMap tmq, const __grid_constan
     }
     // The state entering the segment, the sum of the earlier segments' sums, into the phi(k)
     // slices' space (no copy has reached it yet), z into zpre
+    griddep_wait();   // the state kernel's sums and phi(k) (launched as its dependent)
     sum_segments(wsS, wsZ, sg.bh, kp.nseg, sg.seg, kp.F, reinterpret_cast<float*>(sm + L.phik), zpre);
     tc_fence_before();
     __syncthreads();
@@ -1285,13 +1303,11 @@ k_tc_causal_out_ts(const __grid_constant__ CUtensorMap tmq, const __grid_constan
         Waiter wt;
         if (warp == 0) {
             // ---------------------------------------------------------------- TMA
-            // W once; then per tile the q tile (two buffers, needed a tile ahead by the
-            // projections), the phi(k) slices (each feature half once the previous tile's
-            // scores and state update have read it) and v (once the previous P.V is done)
+            // per tile (W and the first two q tiles are loading since the start) the q tile two
+            // ahead (two buffers, needed a tile ahead by the projections), the phi(k) slices
+            // (each feature half once the previous tile's scores, state update and column sums
+            // are done with it) and v (once the previous P.V is done)
             if (lane == 0) {
-                mbar_arrive_expect_tx(&bar[T_WF], NS * kWBytes);
-                for (int n = 0; n < NS; ++n)
-                    tma_load_2d(sm + L.w + n * kWBytes, &tmw, &bar[T_WF], 0, n * 64);
                 uint32_t ph_qe = 0, ph_free = 0, ph_zc = 0, ph_ve = 0;
                 auto load_q = [&](int it) {
                     const int qb = it & 1;
@@ -1305,8 +1321,6 @@ k_tc_causal_out_ts(const __grid_constant__ CUtensorMap tmq, const __grid_constan
                                 (sg.t_begin + it) * kTile, sg.bh);
                 };
                 const int n = sg.t_end - sg.t_begin;
-                load_q(0);
-                if (n > 1) load_q(1);
                 for (int tile = sg.t_begin, it = 0; tile < sg.t_end; ++tile, ++it) {
                     for (int t = 0; t < NT; ++t) {
                         if (it > 0 && (t & 1) == 0) {   // MMAs and column sums done with the half
@@ -1634,6 +1648,7 @@ k_tc_bidir_out(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
         for (int i = tid; i < NT * kStBytes / 16; i += kOutThreads) p[i] = make_uint4(0, 0, 0, 0);
     }
     // [S | z] of the whole sequence: the sum of all its segments
+    griddep_wait();   // the state kernel's sums (launched as its dependent)
     sum_segments(wsS, wsZ, sg.bh, kp.nseg, kp.nseg, kp.F, reinterpret_cast<float*>(sm + L.scr),
                  reinterpret_cast<float*>(sm + L.zt));
     tc_fence_before();
@@ -1935,6 +1950,25 @@ bool map_phik(CUtensorMap* m, const void* base, int F, int L, int BH)
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Launch `kernel` as the programmatic dependent of the kernel before it on `st` (it may start
+// while that one finishes and waits for its results with griddep_wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), int grid, int block, size_t smem, cudaStream_t st,
+                             Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 template <typename K>
 cudaError_t set_smem(K kernel, size_t bytes)
 {
@@ -1996,7 +2030,8 @@ cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, 
             const size_t smb = smem_bidir_layout(Fc).total + 1024;
             if ((e = set_smem(k_tc_bidir_out, smb)) != cudaSuccess) return e;
             TraceScope trace_("tc_bidir_out", st);
-            k_tc_bidir_out<<<BH * nseg, kOutThreads, smb, st>>>(mq, mw, kp, wsS, wsZ, o, den, err);
+            e = launch_dependent(k_tc_bidir_out, BH * nseg, kOutThreads, smb, st, mq, mw, kp, wsS, wsZ, o, den, err);
+            if (e != cudaSuccess) return e;
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
             continue;
         }
@@ -2018,7 +2053,8 @@ cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, 
             }
             if ((e = set_smem(kern, smo)) != cudaSuccess) return e;
             TraceScope trace_("tc_qphi_out", st);
-            kern<<<BH * nseg, kOutThreads, smo, st>>>(mq, mpk, mv, mw, kp, wsS, wsZ, o, den, err);
+            e = launch_dependent(kern, BH * nseg, kOutThreads, smo, st, mq, mpk, mv, mw, kp, wsS, wsZ, o, den, err);
+            if (e != cudaSuccess) return e;
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
             continue;
         }
