@@ -529,11 +529,20 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         if (lane == 0) {
             uint32_t ph_pk = 0;
             for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
-                const int b = (tile - sg.t_begin) & 1;
+                const int b = (tile - sg.t_begin) & 1, li = tile - sg.t_begin;
                 {   // all of phi(k) of this tile written
                     uint32_t pp = (ph_pk >> b) & 1u;
                     wt.wait(PKF(b), pp);
                     ph_pk ^= 1u << b;
+                }
+                // the next tile's operand reloads go first through this CTA's copy engine:
+                // the projections wait for them, while this store has a tile of slack
+                if (NT == 4 && tile + 1 < sg.t_end) {
+                    // reload of slot s in tile j >= 1 is that slot's completion j + 1
+                    for (int sl = 0; sl < 2; ++sl) {
+                        uint32_t pw = static_cast<uint32_t>(li + 2) & 1u;
+                        wt.wait(&bar[B_W_FULL0 + sl], pw);
+                    }
                 }
                 for (int t = 0; t < NT; ++t)
                     tma_store_3d(&tmpk, sm + L.phik + b * phik_bytes + t * kTileBytes, kSlice * t,
