@@ -385,7 +385,7 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L.tmem);
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int NT = kp.F / kSlice, halves = kp.F / 128;
+    const int NT = kp.F / kSlice;
     const uint32_t phik_bytes = NT * kTileBytes;
     const Seg sg = kp.all_segs ? segment_of(blockIdx.x, kp.nseg, kp.ntiles)
                                : segment_of(blockIdx.x + blockIdx.x / (kp.nseg - 1), kp.nseg, kp.ntiles);
@@ -393,7 +393,7 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     // then onto those its CTAs release); it waits for this grid's results before reading them
     griddep_launch_dependents();
     constexpr uint32_t kColUS = 0;     // 2 x 128: projections
-    constexpr uint32_t kColSS = 256;   // 2 x 80 : [S | z]
+    constexpr uint32_t kColST = 256;   // F: the transposed state, lanes 0-63 S^T, 64-127 z
     // barrier roles here: KF(b) / KE(b) the k buffers; VF / VE the V buffer; TD(b) = the
     // state update of a tile in phi(k) buffer b is done; PKF(b) = all phiK of a tile in
     // buffer b written (one barrier per buffer, so no waiter can fall two phases behind)
@@ -466,6 +466,9 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         // and the state updates, issued here so that they never hold up the projections
         if (lane == 0) {
             uint32_t ph_ve = 0, ph_vf = 0, ph_pk = 0;   // ph_pk: bit per phi(k) buffer
+            // [S | z]^T += [V | 1]^T phi(k): M = 128 (v columns, then the ones tile at LBO),
+            // N = F (all of phi(k) at once: its 64-feature tiles 16 KiB apart), K = 128 tokens
+            const uint32_t idT = idesc_bf16(128, static_cast<uint32_t>(kp.F), 1, 1);
             const uint64_t dph0 = desc_phik(sbase + L.phik), dv = desc_v(sbase + L.v, sbase + L.ones);
             for (int tile = sg.t_begin; tile < sg.t_end; ++tile) {
                 const int b = (tile - sg.t_begin) & 1;
@@ -479,8 +482,11 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 }
                 wt.wait(VF, ph_vf);
                 tc_fence_after();
-                for (int h = 0; h < halves; ++h)
-                    issue_state_half(tmem, kColSS, desc_add(dph0, b * phik_bytes), dv, h, tile == sg.t_begin);
+                const uint64_t dph = desc_add(dph0, b * phik_bytes);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_bf16(tmem + kColST, dv + 128 * kk, dph + 128 * kk, idT,
+                              (tile == sg.t_begin && kk == 0) ? 0u : 1u);
                 umma_commit(VE);
                 umma_commit(&TD[b]);
             }
@@ -608,26 +614,33 @@ k_tc_causal_state(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         }
         tc_fence_after();
         const size_t segidx = static_cast<size_t>(sg.bh) * kp.nseg + sg.seg;
-        for (int h = grp; h < halves; h += 2) {
-            const int f = 128 * h + row;
-            uint32_t r0[32], r1[32], zr;
-            tmem_ld32(trow + kColSS + 80 * h, r0);
-            tmem_ld32(trow + kColSS + 80 * h + 32, r1);
-            tmem_ld1(trow + kColSS + 80 * h + 64, zr);
-            tmem_wait_ld();
-            reg_fence(r0);
-            reg_fence(r1);
-            reg_fence1(zr);
-            float4* dst = reinterpret_cast<float4*>(wsS + (segidx * kp.F + f) * 64);
+        if (sp < 2) {
+            // S[f][e] = S^T[e][f]: lane e of quadrants 0, 1; group g takes features
+            // [g F/2, (g+1) F/2), 32 at a time (a warp's stores: 32 consecutive e of one f)
+            const int fh = kp.F / 2;
+            for (int f0 = grp * fh; f0 < (grp + 1) * fh; f0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(trow + kColST + f0, r);
+                tmem_wait_ld();
+                reg_fence(r);
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-                dst[q] = make_float4(__uint_as_float(r0[4 * q]), __uint_as_float(r0[4 * q + 1]),
-                                     __uint_as_float(r0[4 * q + 2]), __uint_as_float(r0[4 * q + 3]));
+                for (int j = 0; j < 32; ++j) wsS[(segidx * kp.F + f0 + j) * 64 + row] = __uint_as_float(r[j]);
+            }
+        } else if (sp == 2 && grp == 0) {
+            // z: every lane of quadrant 2 holds it (the ones rows); lane 0 writes it
+            for (int f0 = 0; f0 < kp.F; f0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(trow + kColST + f0, r);
+                tmem_wait_ld();
+                reg_fence(r);
+                if (lane == 0) {
+                    float4* dst = reinterpret_cast<float4*>(wsZ + segidx * kp.F + f0);
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-                dst[8 + q] = make_float4(__uint_as_float(r1[4 * q]), __uint_as_float(r1[4 * q + 1]),
-                                         __uint_as_float(r1[4 * q + 2]), __uint_as_float(r1[4 * q + 3]));
-            wsZ[segidx * kp.F + f] = __uint_as_float(zr);
+                    for (int q = 0; q < 8; ++q)
+                        dst[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                                             __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+                }
+            }
         }
     }
     wt.report(err);
