@@ -1508,6 +1508,9 @@ k_tc_causal_out_ts(const __grid_constant__ CUtensorMap tmq, const __grid_constan
                     warp_arrive(&bar[T_UE]);
                     uint32_t pk[16];
                     phi_pack(ur, pr, a, b, pk);
+                    // the previous tile's scores, complete with its last slice, are masked first:
+                    // this slice's MMAs also wait for the readout of those scores' outputs
+                    if (t == 0 && it > 0) ts_mask_scores(bar, wt, ph_pf, ph_de, trow, row, lane, sp, g, dens, it - 1);
                     // the slot is free once the MMAs of the previous slice have read it
                     if (slot_used) wt.wait(&bar[T_PQE], ph_pqe);
                     slot_used = true;
@@ -1515,8 +1518,6 @@ k_tc_causal_out_ts(const __grid_constant__ CUtensorMap tmq, const __grid_constan
                     tmem_wait_st();
                     tc_fence_before();
                     warp_arrive(&bar[T_PQF]);
-                    // the previous tile's scores are complete once its last slice was read
-                    if (t == 0 && it > 0) ts_mask_scores(bar, wt, ph_pf, ph_de, trow, row, lane, sp, g, dens, it - 1);
                 }
             }
             ts_mask_scores(bar, wt, ph_pf, ph_de, trow, row, lane, sp, g, dens, sg.t_end - 1 - sg.t_begin);
