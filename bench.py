@@ -4,6 +4,9 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload causal_16k|causal_2k|bidir_vision|fwd_8k|bwd_8k|decode|feature_map]
 
+With --gpus N > 1 outside torchrun, bench.py starts the N ranks itself (torch.distributed.run
+on 127.0.0.1); under torchrun, --gpus must equal WORLD_SIZE.
+
 One step = one pass of the whole forward path (feature map of q and k, causal contraction,
 normalisation) over one batch of synthetic inputs already resident in HBM.  Default
 workload: B=1, H=16, L=16384, D=Dv=64, R=4 nodes, m=64 features per node (F=256), bf16
@@ -525,7 +528,61 @@ def run_ours(args, w, op):
     return 0
 
 
-def main():
+# ------------------------------------------------------------ rank launch
+
+def free_port():
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def relaunch_ranks(n, argv):
+    """Run this same command line as n ranks under torch.distributed.run on this node
+    (rendezvous on 127.0.0.1); returns the launcher's exit status."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           "--nproc-per-node", str(n), "--master-addr", "127.0.0.1",
+           "--master-port", str(free_port()), os.path.abspath(__file__)] + list(argv)
+    return subprocess.call(cmd)
+
+
+def check_launch(args):
+    """--check-launch: start the process group exactly as the benchmark does (NCCL with a
+    GPU per rank, gloo without one), run its barrier and max-over-ranks steps on a fixed
+    per-rank number, and have rank 0 print which ranks took part.  Times nothing."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    device = "cpu"
+    backend = "gloo"
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
+        device, backend = torch.device("cuda", local), "nccl"
+    if world > 1:
+        kw = {"device_id": device} if backend == "nccl" else {}
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60), **kw)
+        dist.barrier()
+    slowest = max_over_ranks(float(rank), world, device)
+    ranks = [rank]
+    if world > 1:
+        got = [None] * world
+        dist.all_gather_object(got, rank)
+        ranks = got
+        dist.barrier()
+    if rank == 0:
+        print(json.dumps({"launch_check": True, "n_gpus": world, "ranks": ranks,
+                          "backend": backend if world > 1 else None,
+                          "max_over_ranks": slowest}), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    argv = sys.argv[1:] if argv is None else argv
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
@@ -533,9 +590,21 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="causal_16k", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    args = ap.parse_args()
+    ap.add_argument("--check-launch", action="store_true",
+                    help="start the ranks and the process group, report them, time nothing")
+    args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
+    world_env = os.environ.get("WORLD_SIZE")
+    if world_env is None and args.gpus > 1:
+        # not started by torchrun: start the N ranks here, one process per GPU
+        return relaunch_ranks(args.gpus, argv)
+    if world_env is not None and int(world_env) != args.gpus:
+        ap.error("--gpus %d does not match WORLD_SIZE=%s" % (args.gpus, world_env))
+    if args.check_launch:
+        return check_launch(args)
     w, op = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w, op)

@@ -152,7 +152,10 @@ slay_status slay_decode_step(const void* q, const void* k, const void* v,
  * Sharing: all calls on a device share both arrays, which keep the last call's contents
  *   (no part of them needs to start at zero).  Calls that overlap on the GPU -- on
  *   different streams, or from different host threads -- race on them; calls in order on
- *   one stream do not. */
+ *   one stream do not.  The parameter upload of a call with a new key is ordered only on
+ *   that call's stream: a later call with the same key on another stream must be ordered
+ *   after it (an event, or a synchronisation), or it may read the slot before the copy
+ *   has landed. */
 slay_status slay_attn_causal_fwd_noalloc(const void* q, const void* k, const void* v,
                                          void* out, float* den, int B, int H, int L, int D,
                                          int Dv, slay_dtype dt, int R, int m, uint64_t seed,
@@ -170,6 +173,17 @@ slay_status slay_attn_causal_fwd_noalloc(const void* q, const void* k, const voi
  * SLAY_ERR_INVALID_ARG for a workspace that is not 256-byte aligned, SLAY_ERR_CUDA if the
  * copy fails.  The status of a call is only defined once it has been enqueued. */
 slay_status slay_kernel_status(const void* workspace, void* stream);
+
+/* Test hook for the failure path of the bounded waits (the pages have no counterpart;
+ * off by default, for tests only).  With on != 0, the next slay_feature_map call that runs
+ * the tensor-core kernel bounds every wait of that launch at 1 ms and has one warp
+ * withhold one release of a projection buffer (a barrier that guards no copy or MMA in
+ * flight), so that the issuing thread waits for a phase that never completes: the wait
+ * runs out, the kernel stops early (its phi output is then incomplete), drains, frees its
+ * tensor memory and sets the feature-map status word, which slay_kernel_status(NULL, ...)
+ * reports as SLAY_ERR_TIMEOUT.  The hook disarms itself at that launch; on == 0 disarms
+ * it earlier.  No GPU fault is involved and the context stays usable.  Returns SLAY_OK. */
+slay_status slay_debug_expire_wait(int on);
 
 /* Workspace bytes an entry point needs for these sizes (0 if none; SIZE_MAX if the
  * sizes are unsupported).  Feature map and decode need none. */

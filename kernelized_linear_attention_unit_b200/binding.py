@@ -22,7 +22,8 @@ OP_FEATURE_MAP, OP_CAUSAL_FWD, OP_BIDIR_FWD, OP_CAUSAL_BWD, OP_DECODE = range(5)
 EXPORTS = ["slay_feature_map", "slay_attn_causal_fwd", "slay_attn_bidir_fwd",
            "slay_attn_causal_bwd", "slay_decode_step", "slay_workspace_bytes", "slay_prepare",
            "slay_sketch_params", "slay_status_string", "slay_last_error", "slay_trace_enable",
-           "slay_trace_read", "slay_attn_causal_fwd_noalloc", "slay_kernel_status"]
+           "slay_trace_read", "slay_attn_causal_fwd_noalloc", "slay_kernel_status",
+           "slay_debug_expire_wait"]
 
 
 class SlayError(RuntimeError):
@@ -68,6 +69,8 @@ def lib():
     L.slay_last_error.restype = C.c_char_p
     L.slay_kernel_status.argtypes = [vp, vp]
     L.slay_kernel_status.restype = i32
+    L.slay_debug_expire_wait.argtypes = [i32]
+    L.slay_debug_expire_wait.restype = i32
     L.slay_trace_enable.argtypes = [i32]
     L.slay_trace_enable.restype = i32
     L.slay_trace_read.argtypes = [C.POINTER(C.c_char_p), C.POINTER(C.c_float), i32]

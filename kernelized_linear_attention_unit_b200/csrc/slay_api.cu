@@ -357,6 +357,12 @@ slay_status slay_sketch_params(int D, int R, int m, uint64_t seed, float eps, fl
     return SLAY_OK;
 }
 
+slay_status slay_debug_expire_wait(int on)
+{
+    fmap_arm_wait_fault(on);
+    return SLAY_OK;
+}
+
 const char* slay_status_string(slay_status st)
 {
     switch (st) {

@@ -151,8 +151,11 @@ extern "C" slay_status slay_attn_causal_fwd_noalloc(const void* q, const void* k
     if (den && (reinterpret_cast<uintptr_t>(den) % 4) != 0) return SLAY_ERR_INVALID_ARG;
     // the tensor-core path runs in its low-memory form here (phi(k) recomputed, not stored)
     const bool tc = dt == SLAY_BF16 && tc_supported(SLAY_OP_CAUSAL_FWD, B, H, L, R, m, true);
+    // the size of the path that runs: bf16 sizes outside the low-memory tensor-core form
+    // (F > 256 among them) take the CUDA-core kernels, whose scratch is far larger than
+    // the regular tensor-core workspace for the same sizes
     const size_t need = tc ? tc_workspace_bytes(SLAY_OP_CAUSAL_FWD, B, H, L, R, m, true)
-                           : attn_ws(SLAY_OP_CAUSAL_FWD, dt, B, H, L, Dv, R, m);
+                           : kWsHeader + simt_ws_causal(B, H, L, Dv, R * m);
     if (need > kScratchBytes) return SLAY_ERR_UNSUPPORTED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     std::lock_guard<std::mutex> lock(g_mu);

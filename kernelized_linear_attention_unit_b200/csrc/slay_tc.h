@@ -42,6 +42,9 @@ cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const v
                         const float* delta, const float* sfw, const float* gbw, void* dphq,
                         void* dphk, bool dphi_bf16, float* dv, int BH, int L, int F, int* err,
                         cudaStream_t st);
+// Test hook: the next tensor-core feature-map launch withholds one barrier arrival and
+// bounds its waits at 1 ms, so that a wait runs out (on != 0 arms it, 0 disarms it).
+void fmap_arm_wait_fault(int on);
 // Device address of the status word of the feature-map kernels, forward and backward (set
 // when a bounded wait ran out).
 const void* fmap_status_word();

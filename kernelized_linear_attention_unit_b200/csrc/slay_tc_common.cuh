@@ -21,9 +21,10 @@ constexpr uint64_t kWaitNs = 2000000000ull;   // bound of every mbarrier wait (2
 struct Waiter {
     bool ok = true;
     uint32_t where = 0;
+    uint64_t limit = kWaitNs;   // bound of each wait (only a test hook shortens it)
     __device__ __forceinline__ void wait(uint64_t* bar, uint32_t& phase)
     {
-        const bool done = mbar_wait(bar, phase, ok ? kWaitNs : 0);
+        const bool done = mbar_wait(bar, phase, ok ? limit : 0);
         if (!done && ok) where = 0x10000u | (smem_u32(bar) & 0xFFFFu);
         ok = done && ok;
         phase ^= 1u;

@@ -26,6 +26,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "slay_tc.h"
@@ -97,7 +98,16 @@ struct FmParams {
     int F, ntiles;
     float a2[16];   // per 32-feature sub-slice (F <= 512): the scales of its node
     float b2[16];
+    // Test hook of the failure path (0 in every normal call): the first compute warp of
+    // CTA 0 withholds its release of projection buffer 0 after the tile's first group, so
+    // team 0's issuer waits for a phase that never completes; every wait of the launch is
+    // bounded by wait_ns.
+    int withhold;
+    unsigned long long wait_ns;
 };
+
+// Armed by slay_debug_expire_wait, consumed by the next tensor-core feature-map launch.
+std::atomic<int> g_fmap_fault{0};
 
 __global__ void __launch_bounds__(kFmThreads, 1)
 k_tc_feature_map(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
@@ -136,6 +146,7 @@ k_tc_feature_map(const __grid_constant__ CUtensorMap tmx, const __grid_constant_
     tc_fence_after();
     const uint32_t tmem0 = *tslot;
     Waiter wt;
+    wt.limit = fp.wait_ns;
 
     // tiles of team t: k-th = (k * gridDim.x + blockIdx.x) * kTeams + t
     const int stride = gridDim.x * kTeams;
@@ -242,7 +253,10 @@ k_tc_feature_map(const __grid_constant__ CUtensorMap tmx, const __grid_constant_
                 reg_fence(ur);
                 reg_fence(pr);
                 tc_fence_before();
-                warp_arrive(&UE[j & 1]);             // this warp's rows of buffer j & 1 are read
+                // this warp's rows of buffer j & 1 are read (the test hook withholds one
+                // release: it guards only the next MMA into the buffer, none in flight)
+                if (!(fp.withhold && blockIdx.x == 0 && cw == 0 && j == 0))
+                    warp_arrive(&UE[j & 1]);
                 const float a = fp.a2[2 * g + half] * inv, bb = fp.b2[2 * g + half] + l2i;
                 uint32_t pk[16];
                 const float2 a2 = make_float2(a, a), b2 = make_float2(bb, bb);
@@ -323,6 +337,8 @@ cudaError_t tc_feature_map(const void* x, void* phi, int64_t n, const Params& P,
     FmParams fp;
     fp.F = F;
     fp.ntiles = static_cast<int>((n + kRows - 1) / kRows);
+    fp.withhold = g_fmap_fault.exchange(0);
+    fp.wait_ns = fp.withhold ? 1000000ull : kWaitNs;   // 1 ms under the test hook
     for (int sub = 0; sub < 16; ++sub) {
         const int node = sub < F / 32 ? sub * 32 / P.m : 0;
         fp.a2[sub] = P.a2[node];
@@ -342,5 +358,7 @@ cudaError_t tc_feature_map(const void* x, void* phi, int64_t n, const Params& P,
     k_tc_feature_map<<<grid, kFmThreads, smem, st>>>(mx, mw, mo, fp);
     return cudaGetLastError();
 }
+
+void fmap_arm_wait_fault(int on) { g_fmap_fault.store(on ? 1 : 0); }
 
 }  // namespace slay

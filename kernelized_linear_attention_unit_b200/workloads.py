@@ -20,7 +20,8 @@ import numpy as np
 SKETCH_SEED = 1234
 EPS = 1e-6
 
-_STREAM = {"q": 0, "k": 1, "v": 2, "dout": 3, "mu": 4, "S": 5, "z": 6}
+_STREAM = {"q": 0, "k": 1, "v": 2, "dout": 3, "mu": 4, "S": 5, "z": 6,
+           "scale_q": 7, "scale_k": 8}
 
 
 @dataclass(frozen=True)
@@ -134,6 +135,37 @@ def gen_decode(w: Workload, Bt=None, H=None):
     z = (1.0 + _rng(w.data_seed, "z").random((Bt, H, w.F), dtype=np.float32)).astype(np.float32)
     return (to_dtype(q, w.dtype), to_dtype(k, w.dtype), to_dtype(v, w.dtype),
             np.ascontiguousarray(S), np.ascontiguousarray(z))
+
+
+def row_scales(w: Workload, shape, tensor: str, extremes=(6.0, -6.0, 10.0, -10.0)):
+    """Per-row factors 10^e for a tensor whose rows are indexed by `shape` (all but the
+    last axis): e ~ U(-3, 3), and the first len(extremes) rows of a seeded permutation get
+    e = extremes[i] exactly (rows far from unit length, inside the range the library
+    states it supports)."""
+    rng = _rng(w.data_seed, "scale_" + tensor)
+    e = rng.uniform(-3.0, 3.0, size=shape)
+    flat = e.reshape(-1)
+    pick = rng.permutation(flat.size)[:len(extremes)]
+    for i, r in enumerate(pick):
+        flat[r] = extremes[i]
+    return np.power(10.0, e)
+
+
+def scale_rows(w: Workload, x: np.ndarray, tensor: str, extremes=(6.0, -6.0, 10.0, -10.0)):
+    """x with every row multiplied by row_scales(...), rounded to w.dtype: the same values
+    feed the library and the oracle, so only the library's normalisation is exercised."""
+    f = row_scales(w, x.shape[:-1], tensor, extremes)
+    return to_dtype(np.asarray(x, np.float64) * f[..., None], w.dtype)
+
+
+def tile_border_rows(L: int, tile: int = 128):
+    """Sorted row indices: the first and the last row of every `tile`-row block (every
+    segment the tensor-core kernels cut a sequence into starts and ends on such rows)."""
+    s = set()
+    for t0 in range(0, L, tile):
+        s.add(t0)
+        s.add(min(t0 + tile, L) - 1)
+    return np.array(sorted(s), dtype=np.int64)
 
 
 def sample_rows(L: int, n: int, seed: int = 7, chunk: int = 64):

@@ -126,3 +126,19 @@ def test_sketch_params_rejects_bad_args():
     assert L.slay_sketch_params(64, 0, 4, 1, 1e-6, None, None, None, None) == bd.SLAY_ERR_INVALID_ARG
     assert L.slay_sketch_params(64, 4, 4, 1, -1.0, None, None, None, None) == bd.SLAY_ERR_INVALID_ARG
     assert L.slay_sketch_params(64, 4, 4, 1, 1e-6, None, None, None, None) == bd.SLAY_OK
+
+
+def test_noalloc_sizes_the_path_that_runs():
+    # bf16 with F = 512 takes the CUDA-core kernels inside the no-allocation entry point
+    # (its tensor-core form needs F <= 256); their scratch at B1 H1 L8192 (about 49 MiB)
+    # exceeds the 32 MiB array, so the call must be rejected before anything is enqueued,
+    # while the regular tensor-core workspace for the same sizes would have fitted.
+    L = bd.lib()
+    f = L.slay_attn_causal_fwd_noalloc
+    tc_ws = bd.slay_workspace_bytes(bd.OP_CAUSAL_FWD, bd.SLAY_BF16, 1, 1, 8192, 64, 64, 8, 64)
+    assert tc_ws < (32 << 20)
+    for Ln in (8192, 6144):
+        assert f(_fake(), _fake(), _fake(), _fake(), None, 1, 1, Ln, 64, 64, bd.SLAY_BF16, 8, 64,
+                 1234, 1e-6, None) == bd.SLAY_ERR_UNSUPPORTED
+    assert f(_fake(), _fake(), _fake(), _fake(), None, 1, 16, 16384, 64, 64, bd.SLAY_F32, 4, 64,
+             1234, 1e-6, None) == bd.SLAY_ERR_UNSUPPORTED

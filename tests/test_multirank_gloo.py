@@ -82,3 +82,30 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     monkeypatch.setenv("RANK", "1")
     assert bench.run_reference(Args(), W.TINY, "causal") == 0
     assert capsys.readouterr().out == ""
+
+
+def _json_lines(out):
+    import json
+    return [json.loads(l) for l in out.splitlines() if l.startswith("{")]
+
+
+def test_gpus_flag_starts_that_many_ranks():
+    # `python bench.py --gpus 2` outside torchrun starts two ranks itself; without a GPU they
+    # form a gloo group, and rank 0 reports both
+    import subprocess
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                        "--check-launch"], capture_output=True, text=True, env=env, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = _json_lines(r.stdout)
+    assert len(lines) == 1, r.stdout
+    assert lines[0]["n_gpus"] == 2
+    assert sorted(lines[0]["ranks"]) == [0, 1]
+    assert lines[0]["max_over_ranks"] == 1.0
+
+
+def test_gpus_flag_must_match_the_launcher(monkeypatch):
+    monkeypatch.setenv("WORLD_SIZE", "4")
+    with pytest.raises(SystemExit):
+        bench.main(["--gpus", "2", "--check-launch"])

@@ -2,10 +2,18 @@
 
 Inputs come from the shared seeded recipe (kernelized_linear_attention_unit_b200.workloads)
 and are rounded to the mode's dtype before either side sees them, so both compute on the
-same values.  Tolerances (relative L2 error, whole tensor): 1e-5 in fp32 mode and 1.5e-2 in
-bf16-input / fp32-accumulate mode.  Small cases are compared element by element over every
-row; the full-size workloads are compared on sampled rows (ends, chunk and tile borders,
-random rows), in the launch configuration the benchmark times.
+same values.  Bars (relative L2 error): 1e-5 in fp32 mode and 1.5e-2 in bf16-input /
+fp32-accumulate mode for the whole tensor, ten times that for every single row
+(tests/parity_check.py).  Small cases are compared over every row; the full-size workloads
+on the first and last row of every 128-token tile (every segment the tensor-core kernels
+cut a sequence into starts and ends on one) plus random rows, in the launch configuration
+the benchmark times.
+
+"Scaled" cases multiply every q and k row by 10^U(-3,3), with a few rows at 10^{+-6} and
+10^{+-10}, before rounding: the workloads' own rows are unit length, so without these the
+kernels' normalisation (the sphere projection of the review's "Proposed method", step 1)
+and, in the backward, the projection of the gradient onto the sphere's tangent space
+would go unchecked.
 """
 import numpy as np
 import pytest
@@ -14,6 +22,7 @@ import torch
 import oracle as O
 from kernelized_linear_attention_unit_b200 import binding as bd
 from kernelized_linear_attention_unit_b200 import workloads as W
+from parity_check import check, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -33,12 +42,6 @@ def host(t):
     return t.float().cpu().numpy().astype(np.float64)
 
 
-def rel_l2(a, b):
-    a = np.asarray(a, np.float64)
-    b = np.asarray(b, np.float64)
-    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
-
-
 def params(w):
     return O.sketch_params(w.D, w.R, w.m, w.sketch_seed, _eps(w))
 
@@ -48,8 +51,22 @@ def small(dt, R, m, L, B=1, H=2, correlated=False, seed=21):
                       data_seed=seed)
 
 
+def qkv(w, scaled=False):
+    q, k, v = W.gen_qkv(w)
+    if scaled:
+        q = W.scale_rows(w, q, "q")
+        k = W.scale_rows(w, k, "k")
+    return q, k, v
+
+
+def tag(w, what, scaled=False):
+    return "%s %s B%dH%dL%d R%d m%d%s" % (what, w.dtype, w.B, w.H, w.L, w.R, w.m,
+                                           " scaled" if scaled else "")
+
+
 # ------------------------------------------------------------- feature map
 
+@pytest.mark.parametrize("scaled", [False, True])
 @pytest.mark.parametrize("dt_in,dt_out,R,m,n", [("f32", "f32", 2, 16, 1000),
                                                  ("f32", "f32", 4, 64, 130),
                                                  ("bf16", "bf16", 4, 64, 1000),
@@ -58,12 +75,12 @@ def small(dt, R, m, L, B=1, H=2, correlated=False, seed=21):
                                                  ("bf16", "bf16", 2, 64, 40000),
                                                  ("bf16", "bf16", 4, 32, 38001),
                                                  ("bf16", "bf16", 3, 64, 777)])
-def test_feature_map(dt_in, dt_out, R, m, n):
+def test_feature_map(dt_in, dt_out, R, m, n, scaled):
     w = small(dt_in, R, m, n, B=1, H=1)
-    q, _, _ = W.gen_qkv(w)
+    q, _, _ = qkv(w, scaled)
     x = q.reshape(n, 64).copy()
     x[3] = 0.0                       # degenerate zero row -> phi = 0
-    x[5] *= 37.0                     # rescaled row -> same phi
+    x[5] = W.to_dtype(x[5] * 37.0, dt_in)   # rescaled row -> same phi
     P = params(w)
     want = O.feature_map(x, P)
     xt = dev(x, dt_in)
@@ -73,7 +90,8 @@ def test_feature_map(dt_in, dt_out, R, m, n):
     torch.cuda.synchronize()
     got = host(phi)
     tol = TOL["bf16"] if "bf16" in (dt_in, dt_out) else TOL["f32"]
-    assert rel_l2(got, want) <= tol
+    check("phi %s->%s n%d R%d m%d%s" % (dt_in, dt_out, n, R, m, " scaled" if scaled else ""),
+          got, want, tol)
     assert (got[3] == 0).all()
     assert (np.delete(got, 3, axis=0) >= 0).all()
 
@@ -92,14 +110,22 @@ def _run_fwd(q, k, v, w, causal):
     return host(out), host(den)
 
 
+def _check_fwd(name, got, gden, want, wden, tol):
+    check(name + " out", got, want, tol)
+    check(name + " den", gden, wden, tol, per_element=True)
+
+
+FWD_SMALL = [("f32", 2, 16, 256), ("f32", 2, 16, 1), ("f32", 4, 64, 200),
+             ("f32", 3, 16, 129), ("bf16", 4, 64, 300),
+             ("bf16", 4, 64, 1), ("bf16", 8, 64, 257),
+             ("bf16", 2, 16, 64), ("bf16", 2, 64, 129),
+             ("bf16", 4, 64, 1000), ("bf16", 2, 64, 2049),
+             ("bf16", 4, 64, 128), ("bf16", 6, 64, 300),
+             ("bf16", 8, 64, 1000)]
+
+
 @pytest.mark.parametrize("causal", [True, False])
-@pytest.mark.parametrize("dt,R,m,L", [("f32", 2, 16, 256), ("f32", 2, 16, 1), ("f32", 4, 64, 200),
-                                      ("f32", 3, 16, 129), ("bf16", 4, 64, 300),
-                                      ("bf16", 4, 64, 1), ("bf16", 8, 64, 257),
-                                      ("bf16", 2, 16, 64), ("bf16", 2, 64, 129),
-                                      ("bf16", 4, 64, 1000), ("bf16", 2, 64, 2049),
-                                      ("bf16", 4, 64, 128), ("bf16", 6, 64, 300),
-                                      ("bf16", 8, 64, 1000)])
+@pytest.mark.parametrize("dt,R,m,L", FWD_SMALL)
 def test_attn_fwd_small(dt, R, m, L, causal):
     w = small(dt, R, m, L)
     q, k, v = W.gen_qkv(w)
@@ -107,28 +133,42 @@ def test_attn_fwd_small(dt, R, m, L, causal):
     P = params(w)
     want, wden = O.attn_quadratic(q, k, v, P, causal)
     got, gden = _run_fwd(q, k, v, w, causal)
-    assert rel_l2(got, want) <= TOL[dt]
-    assert rel_l2(gden, wden) <= TOL[dt]
-    assert np.isfinite(got).all()
+    _check_fwd(tag(w, "causal" if causal else "bidir"), got, gden, want, wden, TOL[dt])
     assert (got[0, 1, min(2, L - 1)] == 0).all()
+
+
+# q and k rows far from unit length, on every path: fp32 (CUDA cores), bf16 sizes the
+# tensor cores take (one feature chunk, two chunks, three 128-feature chunks) and bf16 sizes
+# they do not (m % 64 != 0).
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("dt,R,m,L", [("f32", 2, 16, 256), ("f32", 4, 64, 200),
+                                      ("bf16", 4, 64, 300), ("bf16", 8, 64, 257),
+                                      ("bf16", 2, 16, 129), ("bf16", 4, 64, 1000),
+                                      ("bf16", 6, 64, 300)])
+def test_attn_fwd_scaled_rows(dt, R, m, L, causal):
+    w = small(dt, R, m, L, seed=22)
+    q, k, v = qkv(w, scaled=True)
+    P = params(w)
+    want, wden = O.attn_quadratic(q, k, v, P, causal)
+    got, gden = _run_fwd(q, k, v, w, causal)
+    _check_fwd(tag(w, "causal" if causal else "bidir", True), got, gden, want, wden, TOL[dt])
 
 
 # Enough (b, h) slices that the sequence is cut into few segments, so one CTA walks
 # several 128-token tiles (state carried in tensor memory from tile to tile), with a
 # ragged last tile; and B*H >= 148, where a single segment covers the whole sequence.
 # F = 512 and 384 run as feature chunks (256 + 256, 3 x 128) summed before the division.
+@pytest.mark.parametrize("scaled", [False, True])
 @pytest.mark.parametrize("B,H,L,R,m", [(2, 37, 657, 4, 64), (1, 148, 300, 4, 64),
                                        (2, 37, 520, 2, 64), (1, 50, 1111, 4, 64),
                                        (2, 37, 657, 8, 64), (1, 20, 700, 6, 64)])
-def test_attn_fwd_multi_tile_segments(B, H, L, R, m):
+def test_attn_fwd_multi_tile_segments(B, H, L, R, m, scaled):
     w = W.Workload("multitile", B=B, H=H, L=L, R=R, m=m, dtype="bf16", data_seed=17)
-    q, k, v = W.gen_qkv(w)
+    q, k, v = qkv(w, scaled)
     P = params(w)
     want, wden = O.attn_quadratic(q, k, v, P, True)
     got, gden = _run_fwd(q, k, v, w, True)
-    assert np.isfinite(got).all()
-    assert rel_l2(got, want) <= TOL["bf16"]
-    assert rel_l2(gden, wden) <= TOL["bf16"]
+    _check_fwd(tag(w, "causal", scaled), got, gden, want, wden, TOL["bf16"])
 
 
 def test_tiny_workload_both_modes():
@@ -138,35 +178,54 @@ def test_tiny_workload_both_modes():
     for causal in (True, False):
         want, wden = O.attn_quadratic(q, k, v, P, causal)
         got, gden = _run_fwd(q, k, v, w, causal)
-        assert rel_l2(got, want) <= TOL["f32"]
-        assert rel_l2(gden, wden) <= TOL["f32"]
+        _check_fwd(tag(w, "tiny causal" if causal else "tiny bidir"), got, gden, want, wden,
+                   TOL["f32"])
 
 
-FULL = [W.CAUSAL_2K, W.CAUSAL_16K, W.BIDIR_VISION, W.FWDBWD_8K]
+# (workload, (b, h) slices checked): every slice of the causal workloads, at the first and
+# last row of every tile plus random rows; a spread of slices of the wide vision batch.
+FULL = [(W.CAUSAL_2K, None), (W.CAUSAL_16K, None), (W.BIDIR_VISION, (4, 3)),
+        (W.FWDBWD_8K, None)]
 
 
-@pytest.mark.parametrize("w", FULL, ids=[x.name for x in FULL])
-def test_attn_fwd_full_size_sampled(w):
+@pytest.mark.parametrize("w,sl", FULL, ids=[x[0].name for x in FULL])
+def test_attn_fwd_full_size_sampled(w, sl):
     q, k, v = W.gen_qkv(w)
     got, gden = _run_fwd(q, k, v, w, w.causal)
     assert np.isfinite(got).all() and (gden > 0).all()
-    rows = W.sample_rows(w.L, 24)
-    # oracle on a subset of (b, h) slices at full length
-    bsel, hsel = slice(0, min(w.B, 2)), slice(0, min(w.H, 4))
+    rows = np.union1d(W.tile_border_rows(w.L), W.sample_rows(w.L, 24))
+    if sl is None:
+        bsel, hsel = slice(0, w.B), slice(0, w.H)
+    else:
+        bsel = slice(0, w.B, max(1, w.B // sl[0]))
+        hsel = slice(0, w.H, max(1, w.H // sl[1]))
     P = params(w)
     want, wden = O.attn_quadratic_rows(q[bsel, hsel], k[bsel, hsel], v[bsel, hsel], P,
                                        w.causal, rows)
-    assert rel_l2(got[bsel, hsel][:, :, rows], want) <= TOL[w.dtype]
-    assert rel_l2(gden[bsel, hsel][:, :, rows], wden) <= TOL[w.dtype]
+    _check_fwd("full " + w.name, got[bsel, hsel][:, :, rows], gden[bsel, hsel][:, :, rows],
+               want, wden, TOL[w.dtype])
 
 
-def test_bidir_correlated_small():
-    w = small("bf16", 4, 64, 160, B=2, H=3, correlated=True)
-    q, k, v = W.gen_qkv(w)
+def test_attn_fwd_full_size_scaled_rows():
+    # the headline shape with rows far from unit length (all heads, every tile border)
+    w = W.CAUSAL_16K
+    q, k, v = qkv(w, scaled=True)
+    got, gden = _run_fwd(q, k, v, w, True)
+    rows = W.tile_border_rows(w.L)
     P = params(w)
-    want, _ = O.attn_quadratic(q, k, v, P, False)
-    got, _ = _run_fwd(q, k, v, w, False)
-    assert rel_l2(got, want) <= TOL["bf16"]
+    want, wden = O.attn_quadratic_rows(q, k, v, P, True, rows)
+    _check_fwd("full scaled " + w.name, got[:, :, rows], gden[:, :, rows], want, wden,
+               TOL["bf16"])
+
+
+@pytest.mark.parametrize("scaled", [False, True])
+def test_bidir_correlated_small(scaled):
+    w = small("bf16", 4, 64, 160, B=2, H=3, correlated=True)
+    q, k, v = qkv(w, scaled)
+    P = params(w)
+    want, wden = O.attn_quadratic(q, k, v, P, False)
+    got, gden = _run_fwd(q, k, v, w, False)
+    _check_fwd(tag(w, "bidir corr", scaled), got, gden, want, wden, TOL["bf16"])
 
 
 # ------------------------------------------------------------ backward
@@ -187,23 +246,29 @@ def _run_bwd(q, k, v, g, w):
     return host(dq), host(dk), host(dv)
 
 
+def _check_bwd(name, got, want, tol):
+    for nm, g, wv in zip(("dq", "dk", "dv"), got, want):
+        check("%s %s" % (name, nm), g, wv, tol)
+
+
+@pytest.mark.parametrize("scaled", [False, True])
 @pytest.mark.parametrize("dt,R,m,L", [("f32", 2, 16, 100), ("f32", 4, 64, 130),
                                       ("bf16", 4, 64, 150), ("bf16", 8, 64, 64),
                                       ("bf16", 2, 16, 65), ("bf16", 3, 64, 300)])
-def test_attn_bwd_small(dt, R, m, L):
+def test_attn_bwd_small(dt, R, m, L, scaled):
     w = small(dt, R, m, L)
-    q, k, v = W.gen_qkv(w)
+    q, k, v = qkv(w, scaled)
     g = W.gen_dout(w)
     P = params(w)
-    wq, wk, wv = O.attn_causal_bwd(q, k, v, g, P)
-    gq, gk, gv = _run_bwd(q, k, v, g, w)
-    assert rel_l2(gq, wq) <= TOL[dt]
-    assert rel_l2(gk, wk) <= TOL[dt]
-    assert rel_l2(gv, wv) <= TOL[dt]
+    want = O.attn_causal_bwd(q, k, v, g, P)
+    got = _run_bwd(q, k, v, g, w)
+    _check_bwd(tag(w, "bwd", scaled), got, want, TOL[dt])
 
 
 # Rows below the 1e-12 norm guard (x^ = x / 1e-12, not a unit vector) and a zero row take the
-# guarded derivative; the bf16 path runs the feature map's backward on tensor cores.
+# guarded derivative; the bf16 path runs the feature map's backward on tensor cores.  The
+# guarded rows' gradients are about 1e12 times the others', so they are checked apart: the
+# guarded rows on their own, and every other row without them.
 @pytest.mark.parametrize("R,m,L", [(4, 64, 200), (8, 64, 130)])
 def test_attn_bwd_guarded_rows(R, m, L):
     w = small("bf16", R, m, L)
@@ -215,9 +280,18 @@ def test_attn_bwd_guarded_rows(R, m, L):
     P = params(w)
     wq, wk, wv = O.attn_causal_bwd(q, k, v, g, P)
     gq, gk, gv = _run_bwd(q, k, v, g, w)
-    for got, want in ((gq, wq), (gk, wk), (gv, wv)):
-        assert np.isfinite(got).all()
-        assert rel_l2(got, want) <= TOL["bf16"]
+    name = tag(w, "bwd guarded")
+    tol = TOL["bf16"]
+    check(name + " dq guarded row", gq[0, 0, 3][None], wq[0, 0, 3][None], tol)
+    check(name + " dk guarded row", gk[0, 1, 5][None], wk[0, 1, 5][None], tol)
+    assert (gk[0, 0, 7] == 0).all() and (wk[0, 0, 7] == 0).all()   # zero key: no gradient
+    mq = np.ones(gq.shape[:-1], bool)
+    mq[0, 0, 3] = False
+    mk = np.ones(gk.shape[:-1], bool)
+    mk[0, 1, 5] = False
+    check(name + " dq other rows", gq[mq], wq[mq], tol)
+    check(name + " dk other rows", gk[mk], wk[mk], tol)
+    check(name + " dv", gv, wv, tol)
 
 
 def test_attn_bwd_single_token():
@@ -231,9 +305,9 @@ def test_attn_bwd_single_token():
     P = params(w)
     wq, wk, wv = O.attn_causal_bwd(q, k, v, g, P)
     gq, gk, gv = _run_bwd(q, k, v, g, w)
-    assert rel_l2(gv, wv) <= 1e-5
-    assert rel_l2(gq, wq) <= 1e-3
-    assert rel_l2(gk, wk) <= 1e-3
+    check("bwd L1 f32 dv", gv, wv, 1e-5)
+    check("bwd L1 f32 dq", gq, wq, 1e-3)
+    check("bwd L1 f32 dk", gk, wk, 1e-3)
 
 
 def test_attn_bwd_many_items():
@@ -242,27 +316,27 @@ def test_attn_bwd_many_items():
     q, k, v = W.gen_qkv(w)
     g = W.gen_dout(w)
     P = params(w)
-    wq, wk, wv = O.attn_causal_bwd(q, k, v, g, P)
-    gq, gk, gv = _run_bwd(q, k, v, g, w)
-    assert rel_l2(gq, wq) <= TOL["bf16"]
-    assert rel_l2(gk, wk) <= TOL["bf16"]
-    assert rel_l2(gv, wv) <= TOL["bf16"]
+    want = O.attn_causal_bwd(q, k, v, g, P)
+    got = _run_bwd(q, k, v, g, w)
+    _check_bwd(tag(w, "bwd items"), got, want, TOL["bf16"])
 
 
-def test_attn_bwd_full_size_sampled():
+@pytest.mark.parametrize("scaled", [False, True])
+def test_attn_bwd_full_size_sampled(scaled):
+    # eight (b, h) slices, the first and last row of every 128-token tile and random rows
     w = W.FWDBWD_8K
-    q, k, v = W.gen_qkv(w)
+    q, k, v = qkv(w, scaled)
     g = W.gen_dout(w)
     gq, gk, gv = _run_bwd(q, k, v, g, w)
     assert np.isfinite(gq).all() and np.isfinite(gk).all() and np.isfinite(gv).all()
-    rows = W.sample_rows(w.L, 12)
-    bsel, hsel = slice(0, 1), slice(0, 2)
+    rows = np.union1d(W.tile_border_rows(w.L), W.sample_rows(w.L, 12))
+    bsel, hsel = slice(0, 2), slice(0, 16, 4)
     P = params(w)
-    wq, wk, wv = O.attn_causal_bwd_rows(q[bsel, hsel], k[bsel, hsel], v[bsel, hsel],
-                                        g[bsel, hsel], P, rows)
-    assert rel_l2(gq[bsel, hsel][:, :, rows], wq) <= TOL["bf16"]
-    assert rel_l2(gk[bsel, hsel][:, :, rows], wk) <= TOL["bf16"]
-    assert rel_l2(gv[bsel, hsel][:, :, rows], wv) <= TOL["bf16"]
+    want = O.attn_causal_bwd_rows(q[bsel, hsel], k[bsel, hsel], v[bsel, hsel],
+                                  g[bsel, hsel], P, rows)
+    got = tuple(x[bsel, hsel][:, :, rows] for x in (gq, gk, gv))
+    _check_bwd(("full scaled " if scaled else "full ") + w.name + " bwd", got, want,
+               TOL["bf16"])
 
 
 # -------------------------------------------------------------- decode
@@ -277,35 +351,48 @@ def _run_decode(q, k, v, S, z, w):
     return host(out), St.cpu().numpy().astype(np.float64), zt.cpu().numpy().astype(np.float64)
 
 
+def _check_decode(name, got, want, S, z, dt):
+    (go, gS, gz), (wo, wS, wz) = got, want
+    tol = TOL[dt]
+    check(name + " out", go, wo, tol)
+    check(name + " S", gS, wS, 1e-5 if dt == "f32" else tol)
+    check(name + " z", gz, wz, 1e-5 if dt == "f32" else tol)
+    if dt == "bf16":
+        # the increments phi(k) v^T and phi(k) are small next to the states, so they are
+        # checked on their own too (whole tensor only: where an increment is far below the
+        # state, the fp32 rounding of the stored state decides its row's error); in fp32
+        # mode that rounding is of the order of the bar itself, so only S and z are checked
+        S0 = S.astype(np.float64)
+        z0 = z.astype(np.float64)
+        check(name + " dS", gS - S0, wS - S0, tol, row_factor=np.inf)
+        check(name + " dz", gz - z0, wz - z0, tol, row_factor=np.inf)
+
+
+@pytest.mark.parametrize("scaled", [False, True])
 @pytest.mark.parametrize("dt,R,m,Bt,H", [("f32", 2, 16, 3, 2), ("f32", 8, 64, 5, 3),
                                          ("bf16", 4, 64, 7, 2), ("bf16", 8, 64, 9, 16)])
-def test_decode_small(dt, R, m, Bt, H):
+def test_decode_small(dt, R, m, Bt, H, scaled):
     w = W.Workload("dec", B=Bt, H=H, L=1, R=R, m=m, dtype=dt, data_seed=31)
     q, k, v, S, z = W.gen_decode(w)
+    if scaled:
+        q = W.scale_rows(w, q, "q")
+        k = W.scale_rows(w, k, "k")
     P = params(w)
-    wo, wS, wz = O.decode_step(q, k, v, S, z, P)
-    go, gS, gz = _run_decode(q, k, v, S, z, w)
-    tol = TOL[dt]
-    assert rel_l2(go, wo) <= tol
-    assert rel_l2(gS, wS) <= 1e-5 if dt == "f32" else rel_l2(gS, wS) <= tol
-    assert rel_l2(gz, wz) <= 1e-5 if dt == "f32" else rel_l2(gz, wz) <= tol
+    want = O.decode_step(q, k, v, S, z, P)
+    got = _run_decode(q, k, v, S, z, w)
+    _check_decode("decode %s Bt%dH%d R%d m%d%s" % (dt, Bt, H, R, m, " scaled" if scaled else ""),
+                  got, want, S, z, dt)
 
 
 def test_decode_full_size():
     w = W.DECODE
     q, k, v, S, z = W.gen_decode(w)
     go, gS, gz = _run_decode(q, k, v, S, z, w)
-    sel = slice(0, 32)
+    sel = slice(0, w.B, 8)     # 32 of the 256 sequences, all heads
     P = params(w)
-    wo, wS, wz = O.decode_step(q[sel], k[sel], v[sel], S[sel], z[sel], P)
-    assert rel_l2(go[sel], wo) <= TOL["bf16"]
-    assert rel_l2(gS[sel], wS) <= TOL["bf16"]
-    assert rel_l2(gz[sel], wz) <= TOL["bf16"]
-    # the state update itself is fp32: the increment phi(k) v^T is tiny next to S ~ N(0,1),
-    # so check the increment separately
-    dS = gS[sel] - S[sel].astype(np.float64)
-    wdS = wS - S[sel].astype(np.float64)
-    assert rel_l2(dS, wdS) <= TOL["bf16"]
+    want = O.decode_step(q[sel], k[sel], v[sel], S[sel], z[sel], P)
+    _check_decode("decode full " + w.name, (go[sel], gS[sel], gz[sel]), want, S[sel], z[sel],
+                  "bf16")
 
 
 def test_decode_chain_matches_causal():
@@ -324,4 +411,4 @@ def test_decode_chain_matches_causal():
         bd.slay_decode_step(qi, ki, vi, St, zt, o, w.R, w.m, w.sketch_seed, _eps(w))
         outs.append(o)
     got = torch.stack(outs, dim=2).cpu().numpy()
-    assert rel_l2(got, want) <= TOL["f32"]
+    check("decode chain f32", got, want, TOL["f32"])
