@@ -53,6 +53,12 @@ def lib():
         L.orc_attn_causal_bwd_rows.argtypes = ([dp, dp, dp, dp] + shp + par +
                                                [C.c_double, i64p, C.c_int, dp, dp, dp])
         L.orc_attn_causal_bwd_rows.restype = None
+        L.orc_attn_causal_bwd_given.argtypes = ([dp, dp, dp, dp, dp, dp] + shp + par +
+                                                [C.c_double, dp, dp, dp])
+        L.orc_attn_causal_bwd_given.restype = None
+        L.orc_attn_causal_bwd_given_rows.argtypes = ([dp, dp, dp, dp, dp, dp] + shp + par +
+                                                     [C.c_double, i64p, C.c_int, dp, dp, dp])
+        L.orc_attn_causal_bwd_given_rows.restype = None
         L.orc_num_threads.argtypes = []
         L.orc_num_threads.restype = C.c_int
         _lib = L
@@ -204,6 +210,35 @@ def attn_causal_bwd_rows(q, k, v, dout, P: Params, rows):
     return dq, dk, dv
 
 
+def attn_causal_bwd_given(q, k, v, out, den, dout, P: Params):
+    """Gradients at a given forward output (out [B,H,L,Dv], den [B,H,L]), the inputs the
+    library's backward takes; equals attn_causal_bwd when out, den are the exact ones."""
+    q, k, v, o, dn, g = _d(q), _d(k), _d(v), _d(out), _d(den), _d(dout)
+    B, H, L, D, Dv = _shape4(q, v)
+    dq = np.zeros(q.shape)
+    dk = np.zeros(k.shape)
+    dv = np.zeros(v.shape)
+    lib().orc_attn_causal_bwd_given(_p(q), _p(k), _p(v), _p(o), _p(dn), _p(g), B, H, L, D, Dv,
+                                    P.R, P.m, *P.args(), P.eps, _p(dq), _p(dk), _p(dv))
+    return dq, dk, dv
+
+
+def attn_causal_bwd_given_rows(q, k, v, out, den, dout, P: Params, rows):
+    q, k, v, o, dn, g = _d(q), _d(k), _d(v), _d(out), _d(den), _d(dout)
+    B, H, L, D, Dv = _shape4(q, v)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    nr = rows.size
+    dq = np.zeros((B, H, nr, D))
+    dk = np.zeros((B, H, nr, D))
+    dv = np.zeros((B, H, nr, Dv))
+    lib().orc_attn_causal_bwd_given_rows(_p(q), _p(k), _p(v), _p(o), _p(dn), _p(g), B, H, L,
+                                         D, Dv, P.R, P.m, *P.args(), P.eps,
+                                         rows.ctypes.data_as(C.POINTER(C.c_int64)), nr,
+                                         _p(dq), _p(dk), _p(dv))
+    return dq, dk, dv
+
+
 __all__ = ["lib", "num_threads", "philox4x32_10", "gauss_laguerre", "Params", "sketch_params",
            "yat_kernel", "quad_kernel", "feature_map", "attn_quadratic", "attn_quadratic_rows",
-           "attn_recurrent", "decode_step", "attn_causal_bwd", "attn_causal_bwd_rows"]
+           "attn_recurrent", "decode_step", "attn_causal_bwd", "attn_causal_bwd_rows",
+           "attn_causal_bwd_given", "attn_causal_bwd_given_rows"]

@@ -107,6 +107,22 @@ void orc_attn_causal_bwd(const double* q, const double* k, const double* v,
 /* The same gradients at rows[0..nrows) only (dq at query rows, dk/dv at key rows);
  * out/den of every row come from the O(L) form above.
  * dq_rows, dk_rows [B,H,nrows,D], dv_rows [B,H,nrows,Dv]. */
+/* The backward at a given forward output (out, den are inputs, as to the library's
+ * backward): see slay_oracle.c. */
+void orc_attn_causal_bwd_given(const double* q, const double* k, const double* v,
+                               const double* out, const double* den, const double* dout,
+                               int B, int H, int L, int D, int Dv, int R, int m,
+                               const double* omega, const double* anchors,
+                               const double* s, const double* wt, double eps,
+                               double* dq, double* dk, double* dv);
+void orc_attn_causal_bwd_given_rows(const double* q, const double* k, const double* v,
+                                    const double* out, const double* den,
+                                    const double* dout,
+                                    int B, int H, int L, int D, int Dv, int R, int m,
+                                    const double* omega, const double* anchors,
+                                    const double* s, const double* wt, double eps,
+                                    const int64_t* rows, int nrows,
+                                    double* dq_rows, double* dk_rows, double* dv_rows);
 void orc_attn_causal_bwd_rows(const double* q, const double* k, const double* v,
                               const double* dout,
                               int B, int H, int L, int D, int Dv, int R, int m,

@@ -339,3 +339,35 @@ def test_backward_rows_variant_equals_full():
     np.testing.assert_allclose(rq, dq[:, :, rows], rtol=1e-10, atol=1e-14)
     np.testing.assert_allclose(rk, dk[:, :, rows], rtol=1e-10, atol=1e-14)
     np.testing.assert_allclose(rv, dv[:, :, rows], rtol=1e-10, atol=1e-14)
+
+
+def test_backward_given_output_reduces_to_the_pinned_backward():
+    # at the exact forward output the "given" form is the finite-difference-pinned backward
+    q, k, v = _small(18, B=1, H=2, L=23, D=8, Dv=4)
+    g = np.random.default_rng(19).standard_normal(v.shape)
+    P = O.sketch_params(D=8, R=2, m=5, seed=9, eps=1e-6)
+    out, den = O.attn_quadratic(q, k, v, P, True)
+    want = O.attn_causal_bwd(q, k, v, g, P)
+    got = O.attn_causal_bwd_given(q, k, v, out, den, g, P)
+    for a, b in zip(got, want):
+        np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-13)
+    rows = np.array([0, 7, 22])
+    for a, b in zip(O.attn_causal_bwd_given_rows(q, k, v, out, den, g, P, rows), got):
+        np.testing.assert_allclose(a, b[:, :, rows], rtol=1e-10, atol=1e-14)
+
+
+def test_backward_given_output_depends_on_out_only_through_delta():
+    # out enters only through delta_i = -<g_i, out_i>/(den_i + eps): dv does not depend on
+    # it, and dq, dk are affine in it (a perturbation's effect doubles when it doubles)
+    q, k, v = _small(20, B=1, H=1, L=17, D=8, Dv=4)
+    g = np.random.default_rng(21).standard_normal(v.shape)
+    P = O.sketch_params(D=8, R=2, m=5, seed=9, eps=1e-6)
+    out, den = O.attn_quadratic(q, k, v, P, True)
+    u = np.random.default_rng(22).standard_normal(out.shape) * 1e-3
+    base = O.attn_causal_bwd_given(q, k, v, out, den, g, P)
+    one = O.attn_causal_bwd_given(q, k, v, out + u, den, g, P)
+    two = O.attn_causal_bwd_given(q, k, v, out + 2 * u, den, g, P)
+    np.testing.assert_allclose(one[2], base[2], rtol=1e-13, atol=1e-15)
+    for b, o1, o2 in zip(base[:2], one[:2], two[:2]):
+        assert np.linalg.norm(o1 - b) > 0
+        np.testing.assert_allclose(o2 - b, 2 * (o1 - b), rtol=1e-6, atol=1e-12)

@@ -22,7 +22,7 @@ import torch
 import oracle as O
 from kernelized_linear_attention_unit_b200 import binding as bd
 from kernelized_linear_attention_unit_b200 import workloads as W
-from parity_check import check, rel_l2
+from parity_check import check, gradient_row_scale, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -246,9 +246,39 @@ def _run_bwd(q, k, v, g, w):
     return host(dq), host(dk), host(dv)
 
 
-def _check_bwd(name, got, want, tol):
-    for nm, g, wv in zip(("dq", "dk", "dv"), got, want):
-        check("%s %s" % (name, nm), g, wv, tol)
+def _bwd_reference(q, k, v, g, P, dt, rows=None):
+    """The oracle's gradients (at every row, or at `rows`) and their per-row scales: the
+    same gradients at the oracle's own forward output rounded to dt (the dtype in which the
+    backward receives `out`) measure how strongly each row cancels."""
+    out, den = O.attn_recurrent(q, k, v, P, True)
+    ro, rd = W.to_dtype(out, dt), W.to_dtype(den, "f32")
+    if rows is None:
+        want = O.attn_causal_bwd(q, k, v, g, P)
+        pert = O.attn_causal_bwd_given(q, k, v, ro, rd, g, P)
+    else:
+        want = O.attn_causal_bwd_rows(q, k, v, g, P, rows)
+        pert = O.attn_causal_bwd_given_rows(q, k, v, ro, rd, g, P, rows)
+    return want, [gradient_row_scale(a, b, dt) for a, b in zip(want, pert)]
+
+
+def _check_bwd(name, got, ref, tol, xnorm=None):
+    """dq, dk, dv against the oracle.  xnorm: row norms of (q, k) when the rows are far from
+    unit length: dq and dk scale as 1/|x|, so rows are weighted by |x| (on both sides) and
+    the whole-tensor error is not decided by the smallest rows alone."""
+    want, scales = ref
+    for i, (nm, g, wv, sc) in enumerate(zip(("dq", "dk", "dv"), got, want, scales)):
+        if xnorm is not None and i < 2:
+            f = xnorm[i]
+            g, wv, sc = g * f[..., None], wv * f[..., None], sc * f
+        check("%s %s" % (name, nm), g, wv, tol, row_scale=sc)
+
+
+def _xnorm(q, k, rows=None):
+    nq = np.linalg.norm(np.asarray(q, np.float64), axis=-1)
+    nk = np.linalg.norm(np.asarray(k, np.float64), axis=-1)
+    if rows is not None:
+        nq, nk = nq[..., rows], nk[..., rows]
+    return nq, nk
 
 
 @pytest.mark.parametrize("scaled", [False, True])
@@ -260,9 +290,9 @@ def test_attn_bwd_small(dt, R, m, L, scaled):
     q, k, v = qkv(w, scaled)
     g = W.gen_dout(w)
     P = params(w)
-    want = O.attn_causal_bwd(q, k, v, g, P)
+    ref = _bwd_reference(q, k, v, g, P, dt)
     got = _run_bwd(q, k, v, g, w)
-    _check_bwd(tag(w, "bwd", scaled), got, want, TOL[dt])
+    _check_bwd(tag(w, "bwd", scaled), got, ref, TOL[dt], _xnorm(q, k) if scaled else None)
 
 
 # Rows below the 1e-12 norm guard (x^ = x / 1e-12, not a unit vector) and a zero row take the
@@ -278,20 +308,22 @@ def test_attn_bwd_guarded_rows(R, m, L):
     k[0, 0, 7] = 0.0
     g = W.gen_dout(w)
     P = params(w)
-    wq, wk, wv = O.attn_causal_bwd(q, k, v, g, P)
+    (wq, wk, wv), (sq, sk, sv) = _bwd_reference(q, k, v, g, P, "bf16")
     gq, gk, gv = _run_bwd(q, k, v, g, w)
     name = tag(w, "bwd guarded")
     tol = TOL["bf16"]
-    check(name + " dq guarded row", gq[0, 0, 3][None], wq[0, 0, 3][None], tol)
-    check(name + " dk guarded row", gk[0, 1, 5][None], wk[0, 1, 5][None], tol)
+    check(name + " dq guarded row", gq[0, 0, 3][None], wq[0, 0, 3][None], tol,
+          row_scale=sq[0, 0, 3][None])
+    check(name + " dk guarded row", gk[0, 1, 5][None], wk[0, 1, 5][None], tol,
+          row_scale=sk[0, 1, 5][None])
     assert (gk[0, 0, 7] == 0).all() and (wk[0, 0, 7] == 0).all()   # zero key: no gradient
     mq = np.ones(gq.shape[:-1], bool)
     mq[0, 0, 3] = False
     mk = np.ones(gk.shape[:-1], bool)
     mk[0, 1, 5] = False
-    check(name + " dq other rows", gq[mq], wq[mq], tol)
-    check(name + " dk other rows", gk[mk], wk[mk], tol)
-    check(name + " dv", gv, wv, tol)
+    check(name + " dq other rows", gq[mq], wq[mq], tol, row_scale=sq[mq])
+    check(name + " dk other rows", gk[mk], wk[mk], tol, row_scale=sk[mk])
+    check(name + " dv", gv, wv, tol, row_scale=sv)
 
 
 def test_attn_bwd_single_token():
@@ -316,9 +348,9 @@ def test_attn_bwd_many_items():
     q, k, v = W.gen_qkv(w)
     g = W.gen_dout(w)
     P = params(w)
-    want = O.attn_causal_bwd(q, k, v, g, P)
+    ref = _bwd_reference(q, k, v, g, P, "bf16")
     got = _run_bwd(q, k, v, g, w)
-    _check_bwd(tag(w, "bwd items"), got, want, TOL["bf16"])
+    _check_bwd(tag(w, "bwd items"), got, ref, TOL["bf16"])
 
 
 @pytest.mark.parametrize("scaled", [False, True])
@@ -332,11 +364,11 @@ def test_attn_bwd_full_size_sampled(scaled):
     rows = np.union1d(W.tile_border_rows(w.L), W.sample_rows(w.L, 12))
     bsel, hsel = slice(0, 2), slice(0, 16, 4)
     P = params(w)
-    want = O.attn_causal_bwd_rows(q[bsel, hsel], k[bsel, hsel], v[bsel, hsel],
-                                  g[bsel, hsel], P, rows)
+    qs, ks = q[bsel, hsel], k[bsel, hsel]
+    ref = _bwd_reference(qs, ks, v[bsel, hsel], g[bsel, hsel], P, "bf16", rows)
     got = tuple(x[bsel, hsel][:, :, rows] for x in (gq, gk, gv))
-    _check_bwd(("full scaled " if scaled else "full ") + w.name + " bwd", got, want,
-               TOL["bf16"])
+    _check_bwd(("full scaled " if scaled else "full ") + w.name + " bwd", got, ref,
+               TOL["bf16"], _xnorm(qs, ks, rows) if scaled else None)
 
 
 # -------------------------------------------------------------- decode
