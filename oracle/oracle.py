@@ -59,6 +59,10 @@ def lib():
         L.orc_attn_causal_bwd_given_rows.argtypes = ([dp, dp, dp, dp, dp, dp] + shp + par +
                                                      [C.c_double, i64p, C.c_int, dp, dp, dp])
         L.orc_attn_causal_bwd_given_rows.restype = None
+        L.orc_feature_map_bwd.argtypes = [dp, dp, C.c_int64, C.c_int, C.c_int, C.c_int] + par + [dp]
+        L.orc_feature_map_bwd.restype = None
+        L.orc_attn_bidir_bwd.argtypes = [dp, dp, dp, dp] + shp + par + [C.c_double, dp, dp, dp]
+        L.orc_attn_bidir_bwd.restype = None
         L.orc_num_threads.argtypes = []
         L.orc_num_threads.restype = C.c_int
         _lib = L
@@ -238,7 +242,29 @@ def attn_causal_bwd_given_rows(q, k, v, out, den, dout, P: Params, rows):
     return dq, dk, dv
 
 
+def feature_map_bwd(x, dphi, P: Params):
+    """dx [..., D] of sum(dphi * phi(x)) (the derivative of feature_map)."""
+    x, g = _d(x), _d(dphi)
+    n = x.size // P.D
+    dx = np.zeros((n, P.D))
+    lib().orc_feature_map_bwd(_p(x), _p(g), n, P.D, P.R, P.m, *P.args(), _p(dx))
+    return dx.reshape(x.shape)
+
+
+def attn_bidir_bwd(q, k, v, dout, P: Params):
+    """Gradients of sum(dout * out) for the bidirectional forward."""
+    q, k, v, g = _d(q), _d(k), _d(v), _d(dout)
+    B, H, L, D, Dv = _shape4(q, v)
+    dq = np.zeros(q.shape)
+    dk = np.zeros(k.shape)
+    dv = np.zeros(v.shape)
+    lib().orc_attn_bidir_bwd(_p(q), _p(k), _p(v), _p(g), B, H, L, D, Dv, P.R, P.m, *P.args(),
+                             P.eps, _p(dq), _p(dk), _p(dv))
+    return dq, dk, dv
+
+
 __all__ = ["lib", "num_threads", "philox4x32_10", "gauss_laguerre", "Params", "sketch_params",
            "yat_kernel", "quad_kernel", "feature_map", "attn_quadratic", "attn_quadratic_rows",
            "attn_recurrent", "decode_step", "attn_causal_bwd", "attn_causal_bwd_rows",
-           "attn_causal_bwd_given", "attn_causal_bwd_given_rows"]
+           "attn_causal_bwd_given", "attn_causal_bwd_given_rows", "feature_map_bwd",
+           "attn_bidir_bwd"]

@@ -643,6 +643,78 @@ void orc_attn_causal_bwd_rows(const double* q, const double* k, const double* v,
     }
 }
 
+/* The feature map's backward on its own: dx[n][D] from dphi[n][F] row by row through
+ * phi_backward_row (the derivative of phi, steps 1, 3 and 5 of the review's "Proposed
+ * method"; the pages give no backward). */
+void orc_feature_map_bwd(const double* x, const double* dphi, int64_t n, int D, int R, int m,
+                         const double* omega, const double* anchors, const double* s,
+                         const double* wt, double* dx)
+{
+    const int64_t F = (int64_t)R * m;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i)
+        phi_backward_row(x + i * D, dphi + i * F, D, R, m, omega, anchors, s, wt, dx + i * D);
+}
+
+/* Backward of the bidirectional forward: out_i = num_i / Z_i with num_i = sum_j a_ij v_j and
+ * Z_i = sum_j a_ij + eps over ALL keys j, a_ij = <phi(q_i), phi(k_j)>.  As in the causal
+ * case (dn_i = g_i/Z_i, delta_i = -<g_i, out_i>/Z_i, c_ij = <v_j, dn_i> + delta_i), without
+ * the mask:
+ *   dphi(q_i) = sum_j c_ij phi(k_j),  dphi(k_j) = sum_i c_ij phi(q_i),  dv_j = sum_i a_ij dn_i. */
+void orc_attn_bidir_bwd(const double* q, const double* k, const double* v, const double* dout,
+                        int B, int H, int L, int D, int Dv, int R, int m,
+                        const double* omega, const double* anchors,
+                        const double* s, const double* wt, double eps,
+                        double* dq, double* dk, double* dv)
+{
+    const int64_t F = (int64_t)R * m;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bh = 0; bh < B * H; ++bh) {
+        const double* qs = q + (int64_t)bh * L * D;
+        const double* ks = k + (int64_t)bh * L * D;
+        const double* vs = v + (int64_t)bh * L * Dv;
+        const double* gs = dout + (int64_t)bh * L * Dv;
+        double* pq = phi_slice(qs, L, D, R, m, omega, anchors, s, wt);
+        double* pk = phi_slice(ks, L, D, R, m, omega, anchors, s, wt);
+        double* outv = (double*)malloc(sizeof(double) * (size_t)L * Dv);
+        double* den = (double*)malloc(sizeof(double) * (size_t)L);
+        for (int i = 0; i < L; ++i)
+            quad_row(pq + (int64_t)i * F, pk, vs, L, Dv, F, eps, 0, i,
+                     outv + (int64_t)i * Dv, den + i);
+        double* dn = (double*)malloc(sizeof(double) * (size_t)L * Dv);
+        double* delta = (double*)malloc(sizeof(double) * (size_t)L);
+        for (int i = 0; i < L; ++i) {
+            double Z = den[i] + eps;
+            for (int e = 0; e < Dv; ++e) dn[(int64_t)i * Dv + e] = gs[(int64_t)i * Dv + e] / Z;
+            delta[i] = -dot(gs + (int64_t)i * Dv, outv + (int64_t)i * Dv, Dv) / Z;
+        }
+        double* dpq = (double*)calloc((size_t)L * F, sizeof(double));
+        double* dpk = (double*)calloc((size_t)L * F, sizeof(double));
+        double* dvs = dv + (int64_t)bh * L * Dv;
+        for (int64_t t = 0; t < (int64_t)L * Dv; ++t) dvs[t] = 0.0;
+        for (int i = 0; i < L; ++i) {
+            for (int j = 0; j < L; ++j) {
+                double c = dot(vs + (int64_t)j * Dv, dn + (int64_t)i * Dv, Dv) + delta[i];
+                double a = dot(pq + (int64_t)i * F, pk + (int64_t)j * F, F);
+                for (int64_t f = 0; f < F; ++f) {
+                    dpq[(int64_t)i * F + f] += c * pk[(int64_t)j * F + f];
+                    dpk[(int64_t)j * F + f] += c * pq[(int64_t)i * F + f];
+                }
+                for (int e = 0; e < Dv; ++e)
+                    dvs[(int64_t)j * Dv + e] += a * dn[(int64_t)i * Dv + e];
+            }
+        }
+        for (int i = 0; i < L; ++i) {
+            phi_backward_row(qs + (int64_t)i * D, dpq + (int64_t)i * F, D, R, m,
+                             omega, anchors, s, wt, dq + ((int64_t)bh * L + i) * D);
+            phi_backward_row(ks + (int64_t)i * D, dpk + (int64_t)i * F, D, R, m,
+                             omega, anchors, s, wt, dk + ((int64_t)bh * L + i) * D);
+        }
+        free(pq); free(pk); free(outv); free(den); free(dn); free(delta);
+        free(dpq); free(dpk);
+    }
+}
+
 int orc_num_threads(void)
 {
 #ifdef _OPENMP

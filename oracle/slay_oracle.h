@@ -132,6 +132,16 @@ void orc_attn_causal_bwd_rows(const double* q, const double* k, const double* v,
                               double* dq_rows, double* dk_rows, double* dv_rows);
 
 /* Number of OpenMP threads the oracle uses (1 when built without OpenMP). */
+/* Feature-map backward (dx from dphi, row by row) and the bidirectional backward: see
+ * slay_oracle.c. */
+void orc_feature_map_bwd(const double* x, const double* dphi, int64_t n, int D, int R, int m,
+                         const double* omega, const double* anchors, const double* s,
+                         const double* wt, double* dx);
+void orc_attn_bidir_bwd(const double* q, const double* k, const double* v, const double* dout,
+                        int B, int H, int L, int D, int Dv, int R, int m,
+                        const double* omega, const double* anchors,
+                        const double* s, const double* wt, double eps,
+                        double* dq, double* dk, double* dv);
 int orc_num_threads(void);
 
 #ifdef __cplusplus

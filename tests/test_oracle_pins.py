@@ -371,3 +371,80 @@ def test_backward_given_output_depends_on_out_only_through_delta():
     for b, o1, o2 in zip(base[:2], one[:2], two[:2]):
         assert np.linalg.norm(o1 - b) > 0
         np.testing.assert_allclose(o2 - b, 2 * (o1 - b), rtol=1e-6, atol=1e-12)
+
+
+def _fd_grad(loss, arrays, h=1e-6):
+    """Central finite differences of loss(**arrays) with respect to every array."""
+    out = {}
+    for name, x in arrays.items():
+        fd = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp = x.copy(); xp[idx] += h
+            xm = x.copy(); xm[idx] -= h
+            fd[idx] = (loss(**{**arrays, name: xp}) - loss(**{**arrays, name: xm})) / (2 * h)
+        out[name] = fd
+    return out
+
+
+def test_bidir_backward_matches_finite_differences():
+    B, H, L, D, Dv = 1, 1, 7, 6, 4
+    rng = np.random.default_rng(25)
+    q = rng.standard_normal((B, H, L, D))
+    k = rng.standard_normal((B, H, L, D))
+    v = rng.standard_normal((B, H, L, Dv))
+    g = rng.standard_normal((B, H, L, Dv))
+    P = O.sketch_params(D=D, R=2, m=3, seed=8, eps=1e-3)
+
+    def loss(q, k, v):
+        out, _ = O.attn_quadratic(q, k, v, P, False)
+        return float(np.sum(out * g))
+
+    fd = _fd_grad(loss, {"q": q, "k": k, "v": v})
+    dq, dk, dv = O.attn_bidir_bwd(q, k, v, g, P)
+    for name, grad in (("q", dq), ("k", dk), ("v", dv)):
+        err = np.linalg.norm(fd[name] - grad) / np.linalg.norm(fd[name])
+        assert err < 1e-7, (name, err)
+
+
+def test_bidir_backward_differs_from_causal_except_where_it_must_agree():
+    # the last query sees every key in both forms, and the bidirectional gradient with
+    # respect to v is the causal one plus the contributions of earlier queries to later keys
+    # (non-zero), so a dropped or kept mask shows
+    q, k, v = _small(26, B=1, H=1, L=9, D=8, Dv=4)
+    g = np.zeros(v.shape)
+    g[..., -1, :] = np.random.default_rng(27).standard_normal(4)   # loss on the last row only
+    P = O.sketch_params(D=8, R=2, m=5, seed=9, eps=1e-6)
+    cb = O.attn_causal_bwd(q, k, v, g, P)
+    bb = O.attn_bidir_bwd(q, k, v, g, P)
+    for a, b in zip(cb, bb):
+        np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-13)
+    g2 = np.random.default_rng(28).standard_normal(v.shape)
+    cb = O.attn_causal_bwd(q, k, v, g2, P)
+    bb = O.attn_bidir_bwd(q, k, v, g2, P)
+    assert np.linalg.norm(cb[2] - bb[2]) > 1e-3 * np.linalg.norm(bb[2])
+
+
+def test_feature_map_backward_matches_finite_differences():
+    rng = np.random.default_rng(29)
+    D = 6
+    x = rng.standard_normal((5, D))
+    x[2] *= 1e-14                      # a row under the norm guard
+    x[3] *= 7.0                        # a rescaled row
+    P = O.sketch_params(D=D, R=2, m=4, seed=10, eps=1e-3)
+    G = rng.standard_normal((5, P.F))
+
+    def loss(x):
+        return float(np.sum(O.feature_map(x, P) * G))
+
+    fd = _fd_grad(loss, {"x": x}, h=1e-7)["x"]
+    got = O.feature_map_bwd(x, G, P)
+    for r in (0, 1, 3, 4):             # finite differences are meaningless at 1e-14 scale
+        err = np.linalg.norm(fd[r] - got[r]) / np.linalg.norm(fd[r])
+        assert err < 1e-6, (r, err)
+    # the guarded row (|x| ~ 1e-14): differences with a step scaled to its size
+    fd2 = _fd_grad(lambda x: float(np.sum(O.feature_map(x, P) * G[2:3])), {"x": x[2:3].copy()},
+                   h=1e-20)["x"][0]
+    err = np.linalg.norm(fd2 - got[2]) / np.linalg.norm(fd2)
+    assert err < 1e-6, err
