@@ -2,7 +2,8 @@
 """Benchmark of the SLAY causal forward (spherical Yat-kernel linear attention) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload causal_16k|causal_2k|bidir_vision|fwd_8k|bwd_8k|decode|feature_map]
+                    [--workload causal_16k|causal_2k|bidir_vision|fwd_8k|bwd_8k|bidir_bwd|decode|
+                                feature_map|feature_map_bwd]
 
 With --gpus N > 1 outside torchrun, bench.py starts the N ranks itself (torch.distributed.run
 on 127.0.0.1); under torchrun, --gpus must equal WORLD_SIZE.
@@ -41,6 +42,8 @@ WORKLOADS = {
     "bidir_vision": (W.BIDIR_VISION, "bidir"),
     "fwd_8k": (W.FWDBWD_8K, "causal"),
     "bwd_8k": (W.FWDBWD_8K, "bwd"),
+    "bidir_bwd": (W.BIDIR_VISION, "bidir_bwd"),
+    "feature_map_bwd": (W.CAUSAL_16K, "feature_map_bwd"),
     "decode": (W.DECODE, "decode"),
     "feature_map": (W.CAUSAL_16K, "feature_map"),
 }
@@ -153,16 +156,19 @@ def kernel_work(name, w, op):
     if name == "tc_bwd_states":
         return th * (2 * 2 * F + 2 * Dv + 4 * (Dv + 1)) + \
             w.B * w.H * ((w.L + 127) // 128) * 2 * F * (Dv + 1) * 4, "byte", "hbm"
-    # the tensor-core chunk contraction of the backward moves, per token-head, phi(q), phi(k),
-    # v (bf16), [dn, delta] (fp32), dphi(q), dphi(k) (bf16: the tensor-core phi backward reads
-    # them), dv (fp32) and its share of the two 128-token states it reads (2 F (Dv+1) fp32)
+    # the tensor-core chunk contraction of the backward, by its algorithmic flops per
+    # token-head: the three products with the scanned sums (dphi(q) = S dn, dphi(k) = G v,
+    # dv = G^T phi(k): 2 F Dv each) and the masked intra-tile terms (scores and c_ij, the
+    # dphi(q), dphi(k) and dv contractions over the C+1 keys of a causal chunk row on average)
     if name == "tc_bwd_tile":
-        return th * (2 * 2 * F + 2 * Dv + 4 * (Dv + 1) + 2 * 2 * F + 4 * Dv) + \
-            w.B * w.H * ((w.L + 127) // 128) * 2 * F * (Dv + 1) * 4, "byte", "hbm"
-    # the tensor-core phi backward is bound by its reads: x (bf16), dphi (bf16), dx (fp32)
+        return th * (6 * F * Dv + (C_CHUNK + 1) * (3 * F + 2 * Dv)), "flop", "tensor"
+    # the tensor-core phi backward is bound by its reads: x (bf16), dphi (bf16), dx (fp32);
+    # the feature-map backward workload maps q and k rows (2 th rows) in one launch each
     if name == "tc_phi_bwd":
         return th * (2 * D + 2 * F + 4 * D), "byte", "hbm"
     if name == "simt_bwd_chunk":
+        if op == "bidir_bwd":   # S [dn; delta], G [v; 1], G^T phi(k): no masked term
+            return th * (2 * F * (Dv + 1) * 2 + 2 * F * Dv), "flop", "alu"
         return th * (6 * F * Dv + (C_CHUNK + 1) * (3 * F + 2 * Dv)), "flop", "alu"
     if name == "simt_bwd_rowstats":
         return th * (2 * Dv * 2 + 4 + (Dv + 1) * 4), "byte", "hbm"
@@ -244,16 +250,35 @@ def oracle_sample(w, op, max_heads):
         return dt, n, threads, "%d of %d (b,h) decode states" % (n, w.B * w.H)
     h = max(1, min(w.H, max_heads))
     q, k, v = W.gen_qkv(w, B=1, H=h)
-    t0 = time.perf_counter()
-    if op == "feature_map":
-        O.feature_map(q, P)
-        O.feature_map(k, P)
-    else:
-        O.attn_recurrent(q, k, v, P, op != "bidir")
-    dt = time.perf_counter() - t0
+    form = "O(L) fp64 form"
     tokens = h / w.H * w.L          # token-equivalents (a token carries H heads)
-    return dt, tokens, threads, "%d of %d heads of one sequence at L=%d, O(L) fp64 form" % (
-        h, w.H, w.L)
+    if op == "bwd":
+        # the causal backward has no O(L) oracle form: its per-row form on a seeded sample of
+        # 32 rows of each head (each row sums over all later queries and earlier keys)
+        g = W.gen_dout(w, B=1, H=h)
+        rows = np.sort(np.random.default_rng(11).choice(w.L, 32, replace=False))
+        t0 = time.perf_counter()
+        O.attn_causal_bwd_rows(q, k, v, g, P, rows)
+        dt = time.perf_counter() - t0
+        tokens = h / w.H * len(rows)
+        form = "per-row fp64 backward at 32 rows"
+    else:
+        t0 = time.perf_counter()
+        if op == "feature_map":
+            O.feature_map(q, P)
+            O.feature_map(k, P)
+        elif op == "feature_map_bwd":
+            gq = W.gen_dphi(w, w.L * h)
+            O.feature_map_bwd(q.reshape(-1, w.D), gq, P)
+            O.feature_map_bwd(k.reshape(-1, w.D), gq, P)
+            form = "fp64 feature-map backward"
+        elif op == "bidir_bwd":
+            O.attn_bidir_bwd(q, k, v, W.gen_dout(w, B=1, H=h), P)
+            form = "quadratic fp64 backward"
+        else:
+            O.attn_recurrent(q, k, v, P, op != "bidir")
+        dt = time.perf_counter() - t0
+    return dt, tokens, threads, "%d of %d heads of one sequence at L=%d, %s" % (h, w.H, w.L, form)
 
 
 def oracle_baseline(w, op, cores, target_s=10.0, max_reps=30):
@@ -378,17 +403,33 @@ def run_ours(args, w, op):
             bd.slay_feature_map(x, out, w.R, w.m, w.sketch_seed, eps)
         units_per_step = w.B * w.L
         unit = "tokens/s"
+    elif op == "feature_map_bwd":
+        qn, kn, _ = W.gen_qkv(wr)
+        x = to_dev(np.concatenate([qn.reshape(-1, w.D), kn.reshape(-1, w.D)]))
+        gphi = to_dev(W.gen_dphi(wr, x.shape[0]))
+        out = torch.empty((x.shape[0], w.D), device=dev, dtype=torch.float32)
+        host_in, dev_in = [pinned(x.cpu()), pinned(gphi.cpu())], [x, gphi]
+
+        def step():
+            bd.slay_feature_map_bwd(x, gphi, out, w.R, w.m, w.sketch_seed, eps)
+        units_per_step = w.B * w.L
+        unit = "tokens/s"
     else:
         qn, kn, vn = W.gen_qkv(wr)
         q, k, v = to_dev(qn), to_dev(kn), to_dev(vn)
         out = torch.empty(v.shape, device=dev, dtype=tdt)
         den = torch.empty(v.shape[:-1], device=dev, dtype=torch.float32)
         host_in, dev_in = [pinned(x.cpu()) for x in (q, k, v)], [q, k, v]
-        if op == "bwd":
+        if op in ("bwd", "bidir_bwd"):
+            causal = op == "bwd"
             g = to_dev(W.gen_dout(wr))
-            ws = bd.alloc_workspace(bd.OP_CAUSAL_BWD, tdt, w.B, w.H, w.L, w.D, w.Dv, w.R, w.m, dev)
-            wsf = bd.alloc_workspace(bd.OP_CAUSAL_FWD, tdt, w.B, w.H, w.L, w.D, w.Dv, w.R, w.m, dev)
-            bd.slay_attn_causal_fwd(q, k, v, out, den, w.R, w.m, w.sketch_seed, eps, wsf)
+            opb = bd.OP_CAUSAL_BWD if causal else bd.OP_BIDIR_BWD
+            opf = bd.OP_CAUSAL_FWD if causal else bd.OP_BIDIR_FWD
+            ws = bd.alloc_workspace(opb, tdt, w.B, w.H, w.L, w.D, w.Dv, w.R, w.m, dev)
+            wsf = bd.alloc_workspace(opf, tdt, w.B, w.H, w.L, w.D, w.Dv, w.R, w.m, dev)
+            fwd = bd.slay_attn_causal_fwd if causal else bd.slay_attn_bidir_fwd
+            bwd = bd.slay_attn_causal_bwd if causal else bd.slay_attn_bidir_bwd
+            fwd(q, k, v, out, den, w.R, w.m, w.sketch_seed, eps, wsf)
             dq = torch.empty(q.shape, device=dev, dtype=torch.float32)
             dk = torch.empty_like(dq)
             dv = torch.empty(v.shape, device=dev, dtype=torch.float32)
@@ -396,8 +437,7 @@ def run_ours(args, w, op):
             dev_in.append(g)
 
             def step():
-                bd.slay_attn_causal_bwd(q, k, v, out, den, g, dq, dk, dv, w.R, w.m,
-                                        w.sketch_seed, eps, ws)
+                bwd(q, k, v, out, den, g, dq, dk, dv, w.R, w.m, w.sketch_seed, eps, ws)
         else:
             opc = bd.OP_BIDIR_FWD if op == "bidir" else bd.OP_CAUSAL_FWD
             ws = bd.alloc_workspace(opc, tdt, w.B, w.H, w.L, w.D, w.Dv, w.R, w.m, dev)
@@ -407,7 +447,7 @@ def run_ours(args, w, op):
                 fn(q, k, v, out, den, w.R, w.m, w.sketch_seed, eps, ws)
         units_per_step = w.B * w.L
         unit = "tokens/s"
-    result = dq if op == "bwd" else out
+    result = dq if op in ("bwd", "bidir_bwd") else out
     host_out = torch.empty(result.shape, dtype=result.dtype, pin_memory=True)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     bd.slay_prepare(w.D, w.R, w.m, w.sketch_seed, eps)
@@ -504,6 +544,19 @@ def run_ours(args, w, op):
                                   "second timed pass (%.4f ms per step with them)"
                                   % (sum(traced_ms) / args.steps)}
 
+    # the backward workloads also by the whole step's algorithmic flops (per token-head, D =
+    # Dv = 64, C = 64): causal 16 D F + 10 F Dv + (C+1)(3F + 2Dv); bidirectional
+    # 16 D F + 10 F Dv (no masked term)
+    step_roofline = None
+    if op in ("bwd", "bidir_bwd"):
+        D_, Dv_, F_ = w.D, w.Dv, w.F
+        per = 16 * D_ * F_ + 10 * F_ * Dv_ + ((C_CHUNK + 1) * (3 * F_ + 2 * Dv_) if op == "bwd" else 0)
+        flop = per * w.B * w.H * w.L
+        tflops = flop / (total_ms / args.steps / 1e3) / 1e12
+        step_roofline = {"bound": "tensor", "algorithmic_flop_per_step": flop,
+                         "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": tflops / peaks["bf16_tflops"], "peak_source": peak_src}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         cores = os.cpu_count() or 1
@@ -521,6 +574,7 @@ def run_ours(args, w, op):
                         "d2h_bytes_per_step": d2h},
                 "gpu_launches": len(trace),
                 "roofline": roofline, "kernels": kernels, "clocks": clocks,
+                "step_roofline": step_roofline,
                 "cpu_baseline": cpu}
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -69,7 +69,8 @@ typedef enum {
     SLAY_OP_CAUSAL_FWD = 1,
     SLAY_OP_BIDIR_FWD = 2,
     SLAY_OP_CAUSAL_BWD = 3,
-    SLAY_OP_DECODE = 4
+    SLAY_OP_DECODE = 4,
+    SLAY_OP_BIDIR_BWD = 5
 } slay_op;
 
 /* Feature map phi (review, "Proposed method", steps 1, 3, 4, 5).
@@ -121,6 +122,40 @@ slay_status slay_attn_causal_bwd(const void* q, const void* k, const void* v,
                                  int B, int H, int L, int D, int Dv,
                                  slay_dtype dt, int R, int m, uint64_t seed, float eps,
                                  void* workspace, size_t ws_bytes, void* stream);
+
+/* Backward of the bidirectional forward: gradients of sum_i <dout_i, out_i> with respect
+ * to q, k, v (the pages give no backward; it is the derivative of slay_attn_bidir_fwd).
+ * With Z_i = den_i + eps, dn_i = dout_i / Z_i, delta_i = -<dout_i, out_i> / Z_i and the
+ * whole-sequence sums S = sum_j phi(k_j) v_j^T, z = sum_j phi(k_j),
+ * G = sum_i phi(q_i) dn_i^T, zg = sum_i phi(q_i) delta_i:
+ *   dphi(q_i) = S dn_i + z delta_i,  dphi(k_j) = G v_j + zg,  dv_j = G^T phi(k_j),
+ * then through phi and the sphere projection as in slay_attn_causal_bwd.
+ * Arguments, layouts and dtypes: as slay_attn_causal_bwd (out, den: the bidirectional
+ * forward's outputs for the same inputs); workspace:
+ * slay_workspace_bytes(SLAY_OP_BIDIR_BWD, ...) bytes, its first int the kernel status word.
+ * The sums and the per-row products run on CUDA cores in fp32; in bf16 mode phi and the
+ * derivative through phi run on tensor cores where the sizes allow (as in the forward), with
+ * dphi passed between them as bf16. */
+slay_status slay_attn_bidir_bwd(const void* q, const void* k, const void* v,
+                                const void* out, const float* den, const void* dout,
+                                float* dq, float* dk, float* dv,
+                                int B, int H, int L, int D, int Dv,
+                                slay_dtype dt, int R, int m, uint64_t seed, float eps,
+                                void* workspace, size_t ws_bytes, void* stream);
+
+/* Backward of the feature map alone (review, "Proposed method", steps 1, 3, 4, 5; the
+ * pages give no backward): dx = (d phi / d x)^T dphi for every row, through the sphere
+ * projection (dx = (dx^ - x^ <x^, dx^>) / |x|, or dx^ / 1e-12 under the norm guard).
+ * x    : device [n_rows, D] in x_dt (F32 or BF16), the rows slay_feature_map was given.
+ * dphi : device [n_rows, R*m] in dphi_dt (F32 or BF16).
+ * dx   : device [n_rows, D] fp32, written.  No workspace.
+ * bf16 x and bf16 dphi with m % 32 == 0, F % 128 == 0, F <= 512 take the tensor-core kernel
+ * (projection and its transpose on tcgen05, bf16 operands, fp32 accumulation; its bounded
+ * waits report through slay_kernel_status(NULL, ...)); other combinations run on CUDA cores
+ * in fp32. */
+slay_status slay_feature_map_bwd(const void* x, const void* dphi, float* dx, int64_t n_rows,
+                                 int D, slay_dtype x_dt, slay_dtype dphi_dt, int R, int m,
+                                 uint64_t seed, float eps, void* stream);
 
 /* One recurrent decode step for Bt*H independent sequences (abstract: linear time
  * and memory; the O(1)-per-token form of the causal contraction), inclusive:
@@ -186,7 +221,7 @@ slay_status slay_kernel_status(const void* workspace, void* stream);
 slay_status slay_debug_expire_wait(int on);
 
 /* Workspace bytes an entry point needs for these sizes (0 if none; SIZE_MAX if the
- * sizes are unsupported).  Feature map and decode need none. */
+ * sizes are unsupported).  Feature map, its backward and decode need none. */
 size_t slay_workspace_bytes(slay_op op, slay_dtype dt, int B, int H, int L, int D, int Dv,
                             int R, int m);
 

@@ -17,13 +17,13 @@ LIB_PATH = os.path.join(_HERE, "libslay.so")
 SLAY_OK, SLAY_ERR_INVALID_ARG, SLAY_ERR_UNSUPPORTED, SLAY_ERR_CUDA, SLAY_ERR_TIMEOUT, \
     SLAY_ERR_NO_MEMORY = range(6)
 SLAY_F32, SLAY_BF16 = 0, 1
-OP_FEATURE_MAP, OP_CAUSAL_FWD, OP_BIDIR_FWD, OP_CAUSAL_BWD, OP_DECODE = range(5)
+OP_FEATURE_MAP, OP_CAUSAL_FWD, OP_BIDIR_FWD, OP_CAUSAL_BWD, OP_DECODE, OP_BIDIR_BWD = range(6)
 
 EXPORTS = ["slay_feature_map", "slay_attn_causal_fwd", "slay_attn_bidir_fwd",
            "slay_attn_causal_bwd", "slay_decode_step", "slay_workspace_bytes", "slay_prepare",
            "slay_sketch_params", "slay_status_string", "slay_last_error", "slay_trace_enable",
            "slay_trace_read", "slay_attn_causal_fwd_noalloc", "slay_kernel_status",
-           "slay_debug_expire_wait"]
+           "slay_debug_expire_wait", "slay_attn_bidir_bwd", "slay_feature_map_bwd"]
 
 
 class SlayError(RuntimeError):
@@ -57,6 +57,8 @@ def lib():
                                                i32, i32, u64, f32, vp]
     L.slay_attn_causal_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
                                        i32, i32, i32, i32, u64, f32, vp, sz, vp]
+    L.slay_attn_bidir_bwd.argtypes = L.slay_attn_causal_bwd.argtypes
+    L.slay_feature_map_bwd.argtypes = [vp, vp, vp, i64, i32, i32, i32, i32, i32, u64, f32, vp]
     L.slay_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                    u64, f32, vp]
     L.slay_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32]
@@ -77,6 +79,7 @@ def lib():
     L.slay_trace_read.restype = i32
     for name in ("slay_feature_map", "slay_attn_causal_fwd", "slay_attn_bidir_fwd",
                  "slay_attn_causal_bwd", "slay_decode_step", "slay_prepare",
+                 "slay_attn_bidir_bwd", "slay_feature_map_bwd",
                  "slay_attn_causal_fwd_noalloc",
                  "slay_sketch_params"):
         getattr(L, name).restype = i32
@@ -223,8 +226,8 @@ def slay_attn_causal_fwd_noalloc(q, k, v, out, den, R, m, seed, eps, stream=None
                                               _stream(stream)), "slay_attn_causal_fwd_noalloc")
 
 
-def slay_attn_causal_bwd(q, k, v, out, den, dout, dq, dk, dv, R, m, seed, eps, workspace=None,
-                         stream=None):
+def _attn_bwd(fn, name, op, q, k, v, out, den, dout, dq, dk, dv, R, m, seed, eps, workspace,
+              stream):
     _check(q, "q")
     B, H, L, D = q.shape
     Dv = v.shape[-1]
@@ -237,17 +240,43 @@ def slay_attn_causal_bwd(q, k, v, out, den, dout, dq, dk, dv, R, m, seed, eps, w
     _check(dk, "dk", torch.float32, (B, H, L, D))
     _check(dv, "dv", torch.float32, (B, H, L, Dv))
     dt = _dt(q)
-    need = slay_workspace_bytes(OP_CAUSAL_BWD, dt, B, H, L, D, Dv, R, m)
+    need = slay_workspace_bytes(op, dt, B, H, L, D, Dv, R, m)
     if workspace is None:
-        workspace = alloc_workspace(OP_CAUSAL_BWD, dt, B, H, L, D, Dv, R, m, q.device)
+        workspace = alloc_workspace(op, dt, B, H, L, D, Dv, R, m, q.device)
     wbytes = workspace.numel() * workspace.element_size()
     if wbytes < need:
         raise ValueError("workspace has %d bytes, %d needed" % (wbytes, need))
-    _raise(lib().slay_attn_causal_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(den), _ptr(dout),
-                                      _ptr(dq), _ptr(dk), _ptr(dv), B, H, L, D, Dv, dt, R, m,
-                                      seed, eps, _ptr(workspace), wbytes, _stream(stream)),
-           "slay_attn_causal_bwd")
+    _raise(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(den), _ptr(dout), _ptr(dq), _ptr(dk),
+              _ptr(dv), B, H, L, D, Dv, dt, R, m, seed, eps, _ptr(workspace), wbytes,
+              _stream(stream)), name)
     return workspace
+
+
+def slay_attn_causal_bwd(q, k, v, out, den, dout, dq, dk, dv, R, m, seed, eps, workspace=None,
+                         stream=None):
+    """Enqueue the causal backward; returns the workspace it used."""
+    return _attn_bwd(lib().slay_attn_causal_bwd, "slay_attn_causal_bwd", OP_CAUSAL_BWD, q, k, v,
+                     out, den, dout, dq, dk, dv, R, m, seed, eps, workspace, stream)
+
+
+def slay_attn_bidir_bwd(q, k, v, out, den, dout, dq, dk, dv, R, m, seed, eps, workspace=None,
+                        stream=None):
+    """Enqueue the bidirectional backward; returns the workspace it used."""
+    return _attn_bwd(lib().slay_attn_bidir_bwd, "slay_attn_bidir_bwd", OP_BIDIR_BWD, q, k, v,
+                     out, den, dout, dq, dk, dv, R, m, seed, eps, workspace, stream)
+
+
+def slay_feature_map_bwd(x, dphi, dx, R, m, seed, eps, stream=None):
+    """dx[n, D] (fp32) = (d phi / d x)^T dphi for x[n, D] (f32 or bf16), dphi[n, R*m]."""
+    _check(x, "x")
+    _check(dphi, "dphi")
+    D = x.shape[-1]
+    n = x.numel() // D if D else 0
+    if dphi.numel() != n * R * m or dphi.shape[-1] != R * m:
+        raise ValueError("dphi must have %d rows of %d features" % (n, R * m))
+    _check(dx, "dx", torch.float32, tuple(x.shape))
+    _raise(lib().slay_feature_map_bwd(_ptr(x), _ptr(dphi), _ptr(dx), n, D, _dt(x), _dt(dphi), R,
+                                      m, seed, eps, _stream(stream)), "slay_feature_map_bwd")
 
 
 def slay_kernel_status(workspace=None, stream=None):

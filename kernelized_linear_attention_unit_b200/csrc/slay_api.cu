@@ -167,6 +167,7 @@ size_t attn_ws(slay_op op, slay_dtype dt, int B, int H, int L, int Dv, int R, in
         case SLAY_OP_CAUSAL_FWD: return kWsHeader + simt_ws_causal(B, H, L, Dv, F);
         case SLAY_OP_BIDIR_FWD: return kWsHeader + simt_ws_bidir(B, H, L, Dv, F);
         case SLAY_OP_CAUSAL_BWD: return kWsHeader + simt_ws_bwd(B, H, L, Dv, F);
+        case SLAY_OP_BIDIR_BWD: return kWsHeader + simt_ws_bidir_bwd(B, H, L, Dv, F);
         default: return 0;
     }
 }
@@ -247,11 +248,15 @@ slay_status slay_attn_bidir_fwd(const void* q, const void* k, const void* v, voi
                     stream, false);
 }
 
-slay_status slay_attn_causal_bwd(const void* q, const void* k, const void* v, const void* out,
-                                 const float* den, const void* dout, float* dq, float* dk,
-                                 float* dv, int B, int H, int L, int D, int Dv, slay_dtype dt,
-                                 int R, int m, uint64_t seed, float eps, void* workspace,
-                                 size_t ws_bytes, void* stream)
+}  // extern "C"
+
+namespace slay {
+namespace {
+
+slay_status attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                     const float* den, const void* dout, float* dq, float* dk, float* dv, int B,
+                     int H, int L, int D, int Dv, slay_dtype dt, int R, int m, uint64_t seed,
+                     float eps, void* workspace, size_t ws_bytes, void* stream, bool causal)
 {
     slay_status s = check_attn(q, k, v, out, B, H, L, D, Dv, dt, R, m, eps);
     if (s != SLAY_OK) return s;
@@ -260,16 +265,64 @@ slay_status slay_attn_causal_bwd(const void* q, const void* k, const void* v, co
     if (!aligned(den, 4) || !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) ||
         !aligned(dv, 16))
         return SLAY_ERR_INVALID_ARG;
-    const size_t need = attn_ws(SLAY_OP_CAUSAL_BWD, dt, B, H, L, Dv, R, m);
+    const size_t need = attn_ws(causal ? SLAY_OP_CAUSAL_BWD : SLAY_OP_BIDIR_BWD, dt, B, H, L, Dv,
+                                R, m);
     if (need > 0 && (!workspace || ws_bytes < need || !aligned(workspace, 256)))
         return SLAY_ERR_INVALID_ARG;
     Params P;
     if ((s = get_params(D, R, m, seed, eps, &P)) != SLAY_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
+    char* w = static_cast<char*>(workspace) + kWsHeader;
     if (e == cudaSuccess)
-        e = simt_attn_causal_bwd(q, k, v, out, den, dout, dq, dk, dv, B, H, L, dt, P, eps,
-                                 static_cast<char*>(workspace) + kWsHeader, st);
+        e = causal ? simt_attn_causal_bwd(q, k, v, out, den, dout, dq, dk, dv, B, H, L, dt, P, eps,
+                                          w, st)
+                   : simt_attn_bidir_bwd(q, k, v, out, den, dout, dq, dk, dv, B, H, L, dt, P, eps,
+                                         w, st);
+    return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
+}
+
+}  // namespace
+}  // namespace slay
+
+extern "C" {
+
+slay_status slay_attn_causal_bwd(const void* q, const void* k, const void* v, const void* out,
+                                 const float* den, const void* dout, float* dq, float* dk,
+                                 float* dv, int B, int H, int L, int D, int Dv, slay_dtype dt,
+                                 int R, int m, uint64_t seed, float eps, void* workspace,
+                                 size_t ws_bytes, void* stream)
+{
+    return attn_bwd(q, k, v, out, den, dout, dq, dk, dv, B, H, L, D, Dv, dt, R, m, seed, eps,
+                    workspace, ws_bytes, stream, true);
+}
+
+slay_status slay_attn_bidir_bwd(const void* q, const void* k, const void* v, const void* out,
+                                const float* den, const void* dout, float* dq, float* dk,
+                                float* dv, int B, int H, int L, int D, int Dv, slay_dtype dt,
+                                int R, int m, uint64_t seed, float eps, void* workspace,
+                                size_t ws_bytes, void* stream)
+{
+    return attn_bwd(q, k, v, out, den, dout, dq, dk, dv, B, H, L, D, Dv, dt, R, m, seed, eps,
+                    workspace, ws_bytes, stream, false);
+}
+
+slay_status slay_feature_map_bwd(const void* x, const void* dphi, float* dx, int64_t n_rows,
+                                 int D, slay_dtype x_dt, slay_dtype dphi_dt, int R, int m,
+                                 uint64_t seed, float eps, void* stream)
+{
+    if (n_rows < 0) return SLAY_ERR_INVALID_ARG;
+    slay_status s = check_shape(D, kD, R, m);
+    if (s != SLAY_OK) return s;
+    if (!dtype_ok(x_dt) || !dtype_ok(dphi_dt) || !eps_ok(eps)) return SLAY_ERR_INVALID_ARG;
+    if (n_rows == 0) return SLAY_OK;
+    if (!x || !dphi || !dx || !aligned(x, 16) || !aligned(dphi, 16) || !aligned(dx, 16))
+        return SLAY_ERR_INVALID_ARG;
+    if (n_rows > (int64_t(1) << 36)) return SLAY_ERR_UNSUPPORTED;
+    Params P;
+    if ((s = get_params(D, R, m, seed, eps, &P)) != SLAY_OK) return s;
+    cudaError_t e = simt_feature_map_bwd(x, dphi, dx, n_rows, x_dt, dphi_dt, P,
+                                         static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
 }
 
@@ -330,7 +383,8 @@ size_t slay_workspace_bytes(slay_op op, slay_dtype dt, int B, int H, int L, int 
     if (B < 0 || H < 0 || L < 0 || !dtype_ok(dt)) return SIZE_MAX;
     if (check_shape(D, Dv, R, m) != SLAY_OK) return SIZE_MAX;
     if (op == SLAY_OP_FEATURE_MAP || op == SLAY_OP_DECODE) return 0;
-    if (op != SLAY_OP_CAUSAL_FWD && op != SLAY_OP_BIDIR_FWD && op != SLAY_OP_CAUSAL_BWD)
+    if (op != SLAY_OP_CAUSAL_FWD && op != SLAY_OP_BIDIR_FWD && op != SLAY_OP_CAUSAL_BWD &&
+        op != SLAY_OP_BIDIR_BWD)
         return SIZE_MAX;
     if (static_cast<int64_t>(B) * H * L == 0) return 0;
     return attn_ws(op, dt, B, H, L, Dv, R, m);

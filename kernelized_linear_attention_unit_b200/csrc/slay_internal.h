@@ -74,6 +74,7 @@ const void* noalloc_status_word();
 size_t simt_ws_causal(int B, int H, int L, int Dv, int F);
 size_t simt_ws_bidir(int B, int H, int L, int Dv, int F);
 size_t simt_ws_bwd(int B, int H, int L, int Dv, int F);
+size_t simt_ws_bidir_bwd(int B, int H, int L, int Dv, int F);
 
 cudaError_t simt_feature_map(const void* x, void* phi, int64_t n, slay_dtype in_dt,
                              slay_dtype out_dt, const Params& P, cudaStream_t st);
@@ -84,6 +85,14 @@ cudaError_t simt_attn_causal_bwd(const void* q, const void* k, const void* v,
                                  const void* out, const float* den, const void* dout,
                                  float* dq, float* dk, float* dv, int B, int H, int L,
                                  slay_dtype dt, const Params& P, float eps, void* ws,
+                                 cudaStream_t st);
+cudaError_t simt_attn_bidir_bwd(const void* q, const void* k, const void* v,
+                                const void* out, const float* den, const void* dout,
+                                float* dq, float* dk, float* dv, int B, int H, int L,
+                                slay_dtype dt, const Params& P, float eps, void* ws,
+                                cudaStream_t st);
+cudaError_t simt_feature_map_bwd(const void* x, const void* dphi, float* dx, int64_t n,
+                                 slay_dtype x_dt, slay_dtype dphi_dt, const Params& P,
                                  cudaStream_t st);
 cudaError_t simt_decode_step(const void* q, const void* k, const void* v, float* S, float* z,
                              void* out, int N, slay_dtype dt, const Params& P, float eps,

@@ -396,15 +396,19 @@ struct BwdSmem {
 //   dphi(q_i) = sum_j c_ij phi(k_j) + S_c [dn_i; delta_i]        (S_c = [S | z] entering)
 //   dphi(k_j) = sum_i c_ij phi(q_i) + G_c [v_j; 1]               (G_c = sum over later
 //   dv_j      = sum_i P_ij dn_i + G_c[:, :64]^T phi(k_j)           chunks of phi(q)[dn, delta]^T)
-template <typename T>
+// kBidir: the bidirectional form, where every query sees every key: no masked intra-chunk
+// terms, and S, G are the whole sequence's sums ([BH][F][E], one per sequence):
+//   dphi(q_i) = S [dn_i; delta_i],  dphi(k_j) = G [v_j; 1],  dv_j = G[:, :64]^T phi(k_j).
+// dphi is written in TD (fp32, or bf16 for the tensor-core feature-map backward).
+template <typename T, bool kBidir, typename TD>
 __global__ void __launch_bounds__(NT) k_bwd_chunk(const T* __restrict__ phq,
                                                   const T* __restrict__ phk,
                                                   const T* __restrict__ v,
                                                   const float* __restrict__ dn,
                                                   const float* __restrict__ sfw,
                                                   const float* __restrict__ gbw,
-                                                  float* __restrict__ dphq,
-                                                  float* __restrict__ dphk,
+                                                  TD* __restrict__ dphq,
+                                                  TD* __restrict__ dphk,
                                                   float* __restrict__ dv, int L, int F)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -415,8 +419,9 @@ __global__ void __launch_bounds__(NT) k_bwd_chunk(const T* __restrict__ phq,
     const int64_t rb = static_cast<int64_t>(bh) * L;
     const T* qb = phq + rb * F;
     const T* kb = phk + rb * F;
-    const float* S = sfw + (static_cast<int64_t>(bh) * NC + c) * F * E;
-    const float* G = gbw + (static_cast<int64_t>(bh) * NC + c) * F * E;
+    const int64_t sidx = kBidir ? static_cast<int64_t>(bh) : static_cast<int64_t>(bh) * NC + c;
+    const float* S = sfw + sidx * F * E;
+    const float* G = gbw + sidx * F * E;
 
     for (int idx = tid; idx < C * E; idx += NT) {
         const int t = idx / E, e = idx % E;
@@ -424,6 +429,8 @@ __global__ void __launch_bounds__(NT) k_bwd_chunk(const T* __restrict__ phq,
         sm.vs[t][e] = ok ? ((e < kD) ? ld(v + (rb + i0 + t) * kD + e) : 1.0f) : 0.0f;
         sm.dn[t][e] = ok ? dn[(rb + i0 + t) * E + e] : 0.0f;
     }
+    float dva[4][4] = {};   // dv rows j = ty + 16 i, cols e = tx + 16 jj
+    if (!kBidir) {
     // P over all feature tiles
     float pa[4][4] = {};
     for (int f0 = 0; f0 < F; f0 += C) {
@@ -470,8 +477,7 @@ __global__ void __launch_bounds__(NT) k_bwd_chunk(const T* __restrict__ phq,
             sm.pm[r][cc] = keep ? pa[i][j] : 0.0f;
             sm.cm[r][cc] = keep ? ca[i][j] + sm.dn[r][64] : 0.0f;
         }
-    // dv accumulators (rows j = ty + 16 i, cols e = tx + 16 jj): sum_i P_ij dn_i
-    float dva[4][4] = {};
+    // dv: sum_i P_ij dn_i
     __syncthreads();
     for (int i = 0; i < C; ++i) {
         float a[4], b[4];
@@ -484,6 +490,7 @@ __global__ void __launch_bounds__(NT) k_bwd_chunk(const T* __restrict__ phq,
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) dva[jr][jj] = fmaf(a[jr], b[jj], dva[jr][jj]);
     }
+    }   // !kBidir
     for (int f0 = 0; f0 < F; f0 += C) {
         __syncthreads();
         for (int idx = tid; idx < C * C; idx += NT) {
@@ -501,6 +508,7 @@ __global__ void __launch_bounds__(NT) k_bwd_chunk(const T* __restrict__ phq,
         // dphi(q)[i][fl] (rows i = ty+16a, features fl = tx+16b)
         {
             float acc[4][4] = {};
+            if (!kBidir)
             for (int j = 0; j < C; ++j) {
                 float a[4], b[4];
 #pragma unroll
@@ -530,7 +538,7 @@ __global__ void __launch_bounds__(NT) k_bwd_chunk(const T* __restrict__ phq,
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
                     const int f = f0 + tx + 16 * jj;
-                    if (f < F) dphq[(rb + i0 + r) * F + f] = acc[i][jj];
+                    if (f < F) st(dphq + (rb + i0 + r) * F + f, acc[i][jj]);
                 }
             }
         }
@@ -543,6 +551,7 @@ __global__ void __launch_bounds__(NT) k_bwd_chunk(const T* __restrict__ phq,
         // dphi(k)[j][fl]
         {
             float acc[4][4] = {};
+            if (!kBidir)
             for (int i = 0; i < C; ++i) {
                 float a[4], b[4];
 #pragma unroll
@@ -572,7 +581,7 @@ __global__ void __launch_bounds__(NT) k_bwd_chunk(const T* __restrict__ phq,
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
                     const int f = f0 + tx + 16 * jj;
-                    if (f < F) dphk[(rb + i0 + r) * F + f] = acc[jr][jj];
+                    if (f < F) st(dphk + (rb + i0 + r) * F + f, acc[jr][jj]);
                 }
             }
         }
@@ -611,9 +620,9 @@ struct PhiBwdSmem {
     float nrm[C];
 };
 
-template <typename Tin>
+template <typename Tin, typename TG>
 __global__ void __launch_bounds__(NT) k_phi_bwd(const Tin* __restrict__ x,
-                                                const float* __restrict__ dphi,
+                                                const TG* __restrict__ dphi,
                                                 float* __restrict__ dx, int64_t n, Params P)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -676,7 +685,7 @@ __global__ void __launch_bounds__(NT) k_phi_bwd(const Tin* __restrict__ x,
                 if (f < F && row0 + r < n) {
                     const int node = f / P.m;
                     const float cE = exp2f(fmaf(P.a2[node], u[i][j], P.b2[node]));
-                    const float g = dphi[(row0 + r) * F + f];
+                    const float g = ld(dphi + (row0 + r) * F + f);
                     gov = g * cE * p[i][j] * p[i][j] * P.sq[node];
                     gav = 2.0f * g * cE * p[i][j];
                 }
@@ -863,6 +872,13 @@ size_t simt_ws_bwd(int B, int H, int L, int /*Dv*/, int F)
     return 4 * phi + 2 * stt + dn;
 }
 
+// the causal backward's carve-outs plus the two whole-sequence sums [BH][F][E]
+size_t simt_ws_bidir_bwd(int B, int H, int L, int Dv, int F)
+{
+    const size_t BH = static_cast<size_t>(B) * H;
+    return simt_ws_bwd(B, H, L, Dv, F) + 2 * align256(BH * F * E * sizeof(float));
+}
+
 template <typename Tin, typename Tout>
 static cudaError_t fm_launch(const void* x, void* phi, int64_t n, const Params& P, cudaStream_t st)
 {
@@ -950,7 +966,7 @@ template <typename T>
 static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const void* out,
                               const float* den, const void* dout, float* dq, float* dk,
                               float* dv, int B, int H, int L, const Params& P, float eps,
-                              void* ws, cudaStream_t st)
+                              void* ws, cudaStream_t st, bool bidir)
 {
     const int BH = B * H, F = P.F, NC = nchunks(L);
     const int64_t rows = static_cast<int64_t>(BH) * L;
@@ -968,7 +984,8 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
     if ((err = phi_map<T>(q, phq, rows, P, st)) != cudaSuccess) return err;
     if ((err = phi_map<T>(k, phk, rows, P, st)) != cudaSuccess) return err;
     // bf16 phi: states, contraction on tensor cores over 128-token tiles; else 64-token chunks
-    const bool tcb = std::is_same<T, __nv_bfloat16>::value && tc_bwd_tile_supported(F, L);
+    // (the bidirectional form always takes the chunk kernels: no masked term, whole sums)
+    const bool tcb = !bidir && std::is_same<T, __nv_bfloat16>::value && tc_bwd_tile_supported(F, L);
     // tensor-core path: dn as bf16 rows and delta in the dn region (132 of its 260 bytes a row)
     __nv_bfloat16* dn16 = reinterpret_cast<__nv_bfloat16*>(dn);
     float* delta = reinterpret_cast<float*>(dn16 + rows * kD);
@@ -985,7 +1002,7 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
     // with the feature map's backward on tensor cores as well, dphi travels as bf16
     const bool tcp = std::is_same<T, __nv_bfloat16>::value && P.wB &&
                      tc_phi_bwd_supported(kD, P.R, P.m, rows);
-    const bool dphi16 = tcb && tcp;
+    const bool dphi16 = (tcb || bidir) && tcp;
     const int NS = tcb ? (L + 127) / 128 : NC;   // state blocks per sequence
     int* status = reinterpret_cast<int*>(w - kWsHeader);
     if (tcb) {
@@ -1007,33 +1024,60 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
     const int FE = F * E;
     const int64_t nth = static_cast<int64_t>(BH) * FE;
     const unsigned sgrid = static_cast<unsigned>((nth + 255) / 256);
+    // bidirectional: the whole-sequence sums, after the causal carve-outs
+    float* stot = reinterpret_cast<float*>(w + simt_ws_bwd(B, H, L, kD, F));
+    float* gtot = stot + align256(static_cast<size_t>(BH) * FE * sizeof(float)) / sizeof(float);
     {
         TraceScope trace_("simt_scan", st);
-        k_scan<<<sgrid, 256, 0, st>>>(sfw, nullptr, BH, NS, FE, 0);
+        k_scan<<<sgrid, 256, 0, st>>>(sfw, stot, BH, NS, FE, bidir ? 2 : 0);
     }
     {
         TraceScope trace_("simt_scan", st);
-        k_scan<<<sgrid, 256, 0, st>>>(gbw, nullptr, BH, NS, FE, 1);
+        k_scan<<<sgrid, 256, 0, st>>>(gbw, gtot, BH, NS, FE, bidir ? 2 : 1);
     }
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    if (tcb) {
+    if (bidir) {
+        // dphi as bf16 when the tensor-core feature-map backward takes it, else fp32
+        if (dphi16) {
+            auto kern = k_bwd_chunk<T, true, __nv_bfloat16>;
+            const size_t smem = sizeof(BwdSmem);
+            if ((err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            static_cast<int>(smem))) != cudaSuccess)
+                return err;
+            TraceScope trace_("simt_bwd_chunk", st);
+            kern<<<dim3(NC, BH), NT, smem, st>>>(phq, phk, cp<T>(v), dn, stot, gtot,
+                                                 reinterpret_cast<__nv_bfloat16*>(dphq),
+                                                 reinterpret_cast<__nv_bfloat16*>(dphk), dv, L, F);
+        } else {
+            auto kern = k_bwd_chunk<T, true, float>;
+            const size_t smem = sizeof(BwdSmem);
+            if ((err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            static_cast<int>(smem))) != cudaSuccess)
+                return err;
+            TraceScope trace_("simt_bwd_chunk", st);
+            kern<<<dim3(NC, BH), NT, smem, st>>>(phq, phk, cp<T>(v), dn, stot, gtot, dphq, dphk,
+                                                 dv, L, F);
+        }
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    } else if (tcb) {
         if ((err = tc_bwd_tile(phq, phk, v, dn16, delta, sfw, gbw, dphq, dphk, dphi16, dv, BH, L, F,
                                status, st)) != cudaSuccess)
             return err;
     } else {
         const size_t smem = sizeof(BwdSmem);
-        if ((err = cudaFuncSetAttribute(k_bwd_chunk<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        auto kern = k_bwd_chunk<T, false, float>;
+        if ((err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         static_cast<int>(smem))) != cudaSuccess)
             return err;
         {
             TraceScope trace_("simt_bwd_chunk", st);
-            k_bwd_chunk<T><<<dim3(NC, BH), NT, smem, st>>>(phq, phk, cp<T>(v), dn, sfw, gbw, dphq,
-                                                           dphk, dv, L, F);
+            kern<<<dim3(NC, BH), NT, smem, st>>>(phq, phk, cp<T>(v), dn, sfw, gbw, dphq, dphk, dv,
+                                                 L, F);
         }
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
     }
     const size_t psm = sizeof(PhiBwdSmem);
-    if ((err = cudaFuncSetAttribute(k_phi_bwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if ((err = cudaFuncSetAttribute(k_phi_bwd<T, float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     static_cast<int>(psm))) != cudaSuccess)
         return err;
     // bf16 inputs: the feature map's backward on tensor cores when it takes these sizes
@@ -1044,11 +1088,11 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
     const unsigned rg = static_cast<unsigned>((rows + C - 1) / C);
     {
         TraceScope trace_("simt_phi_bwd", st);
-        k_phi_bwd<T><<<rg, NT, psm, st>>>(cp<T>(q), dphq, dq, rows, P);
+        k_phi_bwd<T, float><<<rg, NT, psm, st>>>(cp<T>(q), dphq, dq, rows, P);
     }
     {
         TraceScope trace_("simt_phi_bwd", st);
-        k_phi_bwd<T><<<rg, NT, psm, st>>>(cp<T>(k), dphk, dk, rows, P);
+        k_phi_bwd<T, float><<<rg, NT, psm, st>>>(cp<T>(k), dphk, dk, rows, P);
     }
     return cudaGetLastError();
 }
@@ -1059,8 +1103,49 @@ cudaError_t simt_attn_causal_bwd(const void* q, const void* k, const void* v, co
                                  float eps, void* ws, cudaStream_t st)
 {
     if (dt == SLAY_F32)
-        return attn_bwd_t<float>(q, k, v, out, den, dout, dq, dk, dv, B, H, L, P, eps, ws, st);
-    return attn_bwd_t<__nv_bfloat16>(q, k, v, out, den, dout, dq, dk, dv, B, H, L, P, eps, ws, st);
+        return attn_bwd_t<float>(q, k, v, out, den, dout, dq, dk, dv, B, H, L, P, eps, ws, st, false);
+    return attn_bwd_t<__nv_bfloat16>(q, k, v, out, den, dout, dq, dk, dv, B, H, L, P, eps, ws, st,
+                                     false);
+}
+
+cudaError_t simt_attn_bidir_bwd(const void* q, const void* k, const void* v, const void* out,
+                                const float* den, const void* dout, float* dq, float* dk,
+                                float* dv, int B, int H, int L, slay_dtype dt, const Params& P,
+                                float eps, void* ws, cudaStream_t st)
+{
+    if (dt == SLAY_F32)
+        return attn_bwd_t<float>(q, k, v, out, den, dout, dq, dk, dv, B, H, L, P, eps, ws, st, true);
+    return attn_bwd_t<__nv_bfloat16>(q, k, v, out, den, dout, dq, dk, dv, B, H, L, P, eps, ws, st,
+                                     true);
+}
+
+template <typename Tin, typename TG>
+static cudaError_t phi_bwd_launch(const void* x, const void* dphi, float* dx, int64_t n,
+                                  const Params& P, cudaStream_t st)
+{
+    const size_t psm = sizeof(PhiBwdSmem);
+    cudaError_t err = cudaFuncSetAttribute(k_phi_bwd<Tin, TG>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(psm));
+    if (err != cudaSuccess) return err;
+    TraceScope trace_("simt_phi_bwd", st);
+    k_phi_bwd<Tin, TG><<<static_cast<unsigned>((n + C - 1) / C), NT, psm, st>>>(
+        cp<Tin>(x), cp<TG>(dphi), dx, n, P);
+    return cudaGetLastError();
+}
+
+cudaError_t simt_feature_map_bwd(const void* x, const void* dphi, float* dx, int64_t n,
+                                 slay_dtype x_dt, slay_dtype dphi_dt, const Params& P,
+                                 cudaStream_t st)
+{
+    // bf16 rows and bf16 dphi: the tensor-core kernel where it takes the sizes
+    if (x_dt == SLAY_BF16 && dphi_dt == SLAY_BF16 && P.wB && tc_phi_bwd_supported(kD, P.R, P.m, n))
+        return tc_phi_bwd(x, dphi, dx, n, P, st);
+    if (x_dt == SLAY_F32)
+        return dphi_dt == SLAY_F32 ? phi_bwd_launch<float, float>(x, dphi, dx, n, P, st)
+                                   : phi_bwd_launch<float, __nv_bfloat16>(x, dphi, dx, n, P, st);
+    return dphi_dt == SLAY_F32 ? phi_bwd_launch<__nv_bfloat16, float>(x, dphi, dx, n, P, st)
+                               : phi_bwd_launch<__nv_bfloat16, __nv_bfloat16>(x, dphi, dx, n, P, st);
 }
 
 template <typename T>

@@ -21,7 +21,7 @@ SKETCH_SEED = 1234
 EPS = 1e-6
 
 _STREAM = {"q": 0, "k": 1, "v": 2, "dout": 3, "mu": 4, "S": 5, "z": 6,
-           "scale_q": 7, "scale_k": 8}
+           "scale_q": 7, "scale_k": 8, "dphi": 9}
 
 
 @dataclass(frozen=True)
@@ -118,6 +118,12 @@ def gen_dout(w: Workload, B=None, H=None, L=None):
     H = w.H if H is None else H
     L = w.L if L is None else L
     g = _rng(w.data_seed, "dout").standard_normal((B, H, L, w.Dv))
+    return to_dtype(g, w.dtype)
+
+
+def gen_dphi(w: Workload, n: int):
+    """An upstream gradient for n rows of features: [n, F] iid N(0, 1), in w.dtype's values."""
+    g = _rng(w.data_seed, "dphi").standard_normal((n, w.F))
     return to_dtype(g, w.dtype)
 
 

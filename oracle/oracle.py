@@ -63,6 +63,9 @@ def lib():
         L.orc_feature_map_bwd.restype = None
         L.orc_attn_bidir_bwd.argtypes = [dp, dp, dp, dp] + shp + par + [C.c_double, dp, dp, dp]
         L.orc_attn_bidir_bwd.restype = None
+        L.orc_attn_bidir_bwd_given.argtypes = ([dp, dp, dp, dp, dp, dp] + shp + par +
+                                              [C.c_double, dp, dp, dp])
+        L.orc_attn_bidir_bwd_given.restype = None
         L.orc_num_threads.argtypes = []
         L.orc_num_threads.restype = C.c_int
         _lib = L
@@ -263,8 +266,20 @@ def attn_bidir_bwd(q, k, v, dout, P: Params):
     return dq, dk, dv
 
 
+def attn_bidir_bwd_given(q, k, v, out, den, dout, P: Params):
+    """Bidirectional gradients at a given forward output (out, den as inputs)."""
+    q, k, v, o, dn, g = _d(q), _d(k), _d(v), _d(out), _d(den), _d(dout)
+    B, H, L, D, Dv = _shape4(q, v)
+    dq = np.zeros(q.shape)
+    dk = np.zeros(k.shape)
+    dv = np.zeros(v.shape)
+    lib().orc_attn_bidir_bwd_given(_p(q), _p(k), _p(v), _p(o), _p(dn), _p(g), B, H, L, D, Dv,
+                                   P.R, P.m, *P.args(), P.eps, _p(dq), _p(dk), _p(dv))
+    return dq, dk, dv
+
+
 __all__ = ["lib", "num_threads", "philox4x32_10", "gauss_laguerre", "Params", "sketch_params",
            "yat_kernel", "quad_kernel", "feature_map", "attn_quadratic", "attn_quadratic_rows",
            "attn_recurrent", "decode_step", "attn_causal_bwd", "attn_causal_bwd_rows",
            "attn_causal_bwd_given", "attn_causal_bwd_given_rows", "feature_map_bwd",
-           "attn_bidir_bwd"]
+           "attn_bidir_bwd", "attn_bidir_bwd_given"]

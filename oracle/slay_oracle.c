@@ -715,6 +715,59 @@ void orc_attn_bidir_bwd(const double* q, const double* k, const double* v, const
     }
 }
 
+/* orc_attn_bidir_bwd at a GIVEN forward output (out [B,H,L,Dv], den [B,H,L] as inputs, as
+ * the library's backward receives them); with the exact output it is orc_attn_bidir_bwd. */
+void orc_attn_bidir_bwd_given(const double* q, const double* k, const double* v,
+                              const double* out, const double* den_in, const double* dout,
+                              int B, int H, int L, int D, int Dv, int R, int m,
+                              const double* omega, const double* anchors,
+                              const double* s, const double* wt, double eps,
+                              double* dq, double* dk, double* dv)
+{
+    const int64_t F = (int64_t)R * m;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bh = 0; bh < B * H; ++bh) {
+        const double* qs = q + (int64_t)bh * L * D;
+        const double* ks = k + (int64_t)bh * L * D;
+        const double* vs = v + (int64_t)bh * L * Dv;
+        const double* os = out + (int64_t)bh * L * Dv;
+        const double* ds = den_in + (int64_t)bh * L;
+        const double* gs = dout + (int64_t)bh * L * Dv;
+        double* pq = phi_slice(qs, L, D, R, m, omega, anchors, s, wt);
+        double* pk = phi_slice(ks, L, D, R, m, omega, anchors, s, wt);
+        double* dn = (double*)malloc(sizeof(double) * (size_t)L * Dv);
+        double* delta = (double*)malloc(sizeof(double) * (size_t)L);
+        for (int i = 0; i < L; ++i) {
+            double Z = ds[i] + eps;
+            for (int e = 0; e < Dv; ++e) dn[(int64_t)i * Dv + e] = gs[(int64_t)i * Dv + e] / Z;
+            delta[i] = -dot(gs + (int64_t)i * Dv, os + (int64_t)i * Dv, Dv) / Z;
+        }
+        double* dpq = (double*)calloc((size_t)L * F, sizeof(double));
+        double* dpk = (double*)calloc((size_t)L * F, sizeof(double));
+        double* dvs = dv + (int64_t)bh * L * Dv;
+        for (int64_t t = 0; t < (int64_t)L * Dv; ++t) dvs[t] = 0.0;
+        for (int i = 0; i < L; ++i) {
+            for (int j = 0; j < L; ++j) {
+                double c = dot(vs + (int64_t)j * Dv, dn + (int64_t)i * Dv, Dv) + delta[i];
+                double a = dot(pq + (int64_t)i * F, pk + (int64_t)j * F, F);
+                for (int64_t f = 0; f < F; ++f) {
+                    dpq[(int64_t)i * F + f] += c * pk[(int64_t)j * F + f];
+                    dpk[(int64_t)j * F + f] += c * pq[(int64_t)i * F + f];
+                }
+                for (int e = 0; e < Dv; ++e)
+                    dvs[(int64_t)j * Dv + e] += a * dn[(int64_t)i * Dv + e];
+            }
+        }
+        for (int i = 0; i < L; ++i) {
+            phi_backward_row(qs + (int64_t)i * D, dpq + (int64_t)i * F, D, R, m,
+                             omega, anchors, s, wt, dq + ((int64_t)bh * L + i) * D);
+            phi_backward_row(ks + (int64_t)i * D, dpk + (int64_t)i * F, D, R, m,
+                             omega, anchors, s, wt, dk + ((int64_t)bh * L + i) * D);
+        }
+        free(pq); free(pk); free(dn); free(delta); free(dpq); free(dpk);
+    }
+}
+
 int orc_num_threads(void)
 {
 #ifdef _OPENMP

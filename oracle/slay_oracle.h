@@ -142,6 +142,12 @@ void orc_attn_bidir_bwd(const double* q, const double* k, const double* v, const
                         const double* omega, const double* anchors,
                         const double* s, const double* wt, double eps,
                         double* dq, double* dk, double* dv);
+void orc_attn_bidir_bwd_given(const double* q, const double* k, const double* v,
+                              const double* out, const double* den, const double* dout,
+                              int B, int H, int L, int D, int Dv, int R, int m,
+                              const double* omega, const double* anchors,
+                              const double* s, const double* wt, double eps,
+                              double* dq, double* dk, double* dv);
 int orc_num_threads(void);
 
 #ifdef __cplusplus

@@ -65,5 +65,16 @@ def test_backward_kernels_are_not_chunk_split():
     states = tiles * 2 * w.F * (DV + 1) * 4
     assert bench.kernel_work("tc_bwd_states", w, "bwd")[0] == \
         th * (2 * 2 * w.F + 2 * DV + 4 * (DV + 1)) + states
-    assert bench.kernel_work("tc_bwd_tile", w, "bwd")[0] == \
-        th * (2 * 2 * w.F + 2 * DV + 4 * (DV + 1) + 2 * 2 * w.F + 4 * DV) + states
+    # the contraction by its flops: three products with the scanned sums (2 F Dv each) and
+    # the masked intra-tile terms over the C + 1 keys of a causal chunk row on average
+    amount, unit, bound = bench.kernel_work("tc_bwd_tile", w, "bwd")
+    assert (unit, bound) == ("flop", "tensor")
+    assert amount == th * (6 * w.F * DV + 65 * (3 * w.F + 2 * DV))
+
+
+def test_backward_step_flops_are_the_per_token_head_count():
+    # 16 D F + 10 F Dv + (C+1)(3F + 2Dv) per token-head = 960,128 at F = 512: 2.52e11 per step
+    w = W.FWDBWD_8K
+    per = 16 * D * w.F + 10 * w.F * DV + 65 * (3 * w.F + 2 * DV)
+    assert per == 960128
+    assert abs(per * w.B * w.H * w.L - 2.517e11) < 1e9

@@ -448,3 +448,20 @@ def test_feature_map_backward_matches_finite_differences():
                    h=1e-20)["x"][0]
     err = np.linalg.norm(fd2 - got[2]) / np.linalg.norm(fd2)
     assert err < 1e-6, err
+
+
+def test_bidir_backward_given_output_reduces_and_is_affine_in_out():
+    q, k, v = _small(30, B=1, H=2, L=13, D=8, Dv=4)
+    g = np.random.default_rng(31).standard_normal(v.shape)
+    P = O.sketch_params(D=8, R=2, m=5, seed=9, eps=1e-6)
+    out, den = O.attn_quadratic(q, k, v, P, False)
+    want = O.attn_bidir_bwd(q, k, v, g, P)
+    base = O.attn_bidir_bwd_given(q, k, v, out, den, g, P)
+    for a, b in zip(base, want):
+        np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-13)
+    u = np.random.default_rng(32).standard_normal(out.shape) * 1e-3
+    one = O.attn_bidir_bwd_given(q, k, v, out + u, den, g, P)
+    two = O.attn_bidir_bwd_given(q, k, v, out + 2 * u, den, g, P)
+    np.testing.assert_allclose(one[2], base[2], rtol=1e-13, atol=1e-15)
+    for b, o1, o2 in zip(base[:2], one[:2], two[:2]):
+        np.testing.assert_allclose(o2 - b, 2 * (o1 - b), rtol=1e-6, atol=1e-12)

@@ -444,3 +444,102 @@ def test_decode_chain_matches_causal():
         outs.append(o)
     got = torch.stack(outs, dim=2).cpu().numpy()
     check("decode chain f32", got, want, TOL["f32"])
+
+
+# ------------------------------------------------- bidirectional backward
+
+def _run_bidir_bwd(q, k, v, g, w):
+    B, H, L, _ = q.shape
+    qt, kt, vt, gt = dev(q, w.dtype), dev(k, w.dtype), dev(v, w.dtype), dev(g, w.dtype)
+    out = torch.empty((B, H, L, w.Dv), device="cuda", dtype=TDT[w.dtype])
+    den = torch.empty((B, H, L), device="cuda", dtype=torch.float32)
+    bd.slay_attn_bidir_fwd(qt, kt, vt, out, den, w.R, w.m, w.sketch_seed, _eps(w))
+    dq = torch.empty((B, H, L, w.D), device="cuda", dtype=torch.float32)
+    dk = torch.empty_like(dq)
+    dv = torch.empty((B, H, L, w.Dv), device="cuda", dtype=torch.float32)
+    ws = bd.slay_attn_bidir_bwd(qt, kt, vt, out, den, gt, dq, dk, dv, w.R, w.m, w.sketch_seed,
+                                _eps(w))
+    bd.slay_kernel_status(ws)
+    bd.slay_kernel_status(None)
+    torch.cuda.synchronize()
+    return host(dq), host(dk), host(dv)
+
+
+def _bidir_reference(q, k, v, g, P, dt):
+    """The oracle's bidirectional gradients and their per-row cancellation scales (the same
+    gradients at the oracle's own forward output rounded to dt; see gradient_row_scale)."""
+    out, den = O.attn_quadratic(q, k, v, P, False)
+    want = O.attn_bidir_bwd(q, k, v, g, P)
+    pert = O.attn_bidir_bwd_given(q, k, v, W.to_dtype(out, dt), W.to_dtype(den, "f32"), g, P)
+    return want, [gradient_row_scale(a, b, dt) for a, b in zip(want, pert)]
+
+
+@pytest.mark.parametrize("scaled", [False, True])
+@pytest.mark.parametrize("dt,R,m,L,B,H,corr", [("f32", 2, 16, 100, 1, 2, False),
+                                              ("f32", 4, 64, 130, 1, 2, False),
+                                              ("bf16", 4, 64, 150, 1, 2, False),
+                                              ("bf16", 8, 64, 64, 1, 2, False),
+                                              ("bf16", 2, 16, 65, 1, 2, False),
+                                              ("bf16", 4, 64, 257, 2, 3, True),
+                                              ("bf16", 3, 64, 300, 1, 2, False)])
+def test_attn_bidir_bwd_small(dt, R, m, L, B, H, corr, scaled):
+    w = small(dt, R, m, L, B=B, H=H, correlated=corr)
+    q, k, v = qkv(w, scaled)
+    g = W.gen_dout(w)
+    P = params(w)
+    ref = _bidir_reference(q, k, v, g, P, dt)
+    got = _run_bidir_bwd(q, k, v, g, w)
+    _check_bwd(tag(w, "bidir bwd" + (" corr" if corr else ""), scaled), got, ref, TOL[dt],
+               _xnorm(q, k) if scaled else None)
+
+
+def test_attn_bidir_bwd_vision_shape_sampled():
+    # the vision-shaped workload (32 x 12 sequences of 32 x 32 patches, correlated angles):
+    # the whole batch runs, the oracle checks a spread of eight (b, h) sequences in full
+    w = W.BIDIR_VISION
+    q, k, v = W.gen_qkv(w)
+    g = W.gen_dout(w)
+    gq, gk, gv = _run_bidir_bwd(q, k, v, g, w)
+    assert np.isfinite(gq).all() and np.isfinite(gk).all() and np.isfinite(gv).all()
+    bsel, hsel = slice(0, w.B, w.B // 4), slice(0, w.H, w.H // 2)
+    P = params(w)
+    ref = _bidir_reference(q[bsel, hsel], k[bsel, hsel], v[bsel, hsel], g[bsel, hsel], P, "bf16")
+    got = tuple(x[bsel, hsel] for x in (gq, gk, gv))
+    _check_bwd("full " + w.name + " bidir bwd", got, ref, TOL["bf16"])
+
+
+# ------------------------------------------------- feature-map backward
+
+@pytest.mark.parametrize("scaled", [False, True])
+@pytest.mark.parametrize("dt_x,dt_g,R,m,n", [("f32", "f32", 2, 16, 1000),
+                                             ("f32", "f32", 4, 64, 130),
+                                             ("bf16", "bf16", 4, 64, 1000),
+                                             ("bf16", "bf16", 8, 64, 4097),
+                                             ("bf16", "f32", 4, 64, 333),
+                                             ("bf16", "bf16", 2, 16, 777),
+                                             ("bf16", "bf16", 4, 32, 38001)])
+def test_feature_map_bwd(dt_x, dt_g, R, m, n, scaled):
+    w = small(dt_x, R, m, n, B=1, H=1)
+    q, _, _ = qkv(w, scaled)
+    x = q.reshape(n, 64).copy()
+    x[3] = 0.0                                     # zero row: guarded derivative
+    x[7] = W.to_dtype(x[7] * 1e-14, dt_x)          # under the 1e-12 norm guard
+    gw = W.Workload("g", B=1, H=1, L=n, R=R, m=m, dtype=dt_g, data_seed=w.data_seed)
+    G = W.gen_dphi(gw, n)
+    P = params(w)
+    want = O.feature_map_bwd(x, G, P)
+    xt, gt = dev(x, dt_x), dev(G, dt_g)
+    dx = torch.empty((n, 64), device="cuda", dtype=torch.float32)
+    bd.slay_feature_map_bwd(xt, gt, dx, R, m, w.sketch_seed, _eps(w))
+    bd.slay_kernel_status(None)
+    torch.cuda.synchronize()
+    got = host(dx)
+    tol = TOL["bf16"] if "bf16" in (dt_x, dt_g) else TOL["f32"]
+    name = "phi bwd %s,%s n%d R%d m%d%s" % (dt_x, dt_g, n, R, m, " scaled" if scaled else "")
+    # rows far from unit length have gradients scaled by 1/|x|: weighted by |x| on both sides
+    nx = np.linalg.norm(x.astype(np.float64), axis=-1)
+    keep = np.ones(n, bool)
+    keep[[3, 7]] = False
+    check(name, got[keep] * nx[keep, None], want[keep] * nx[keep, None], tol)
+    check(name + " guarded row", got[7][None], want[7][None], tol)
+    assert np.isfinite(got).all()
