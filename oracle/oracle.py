@@ -66,6 +66,15 @@ def lib():
         L.orc_attn_bidir_bwd_given.argtypes = ([dp, dp, dp, dp, dp, dp] + shp + par +
                                               [C.c_double, dp, dp, dp])
         L.orc_attn_bidir_bwd_given.restype = None
+        L.orc_sketch_params_kind.argtypes = [C.c_int, C.c_int, C.c_int, C.c_uint64, C.c_double,
+                                             C.c_int, C.c_int, dp, dp, dp, dp, dp]
+        L.orc_sketch_params_kind.restype = C.c_int
+        L.orc_feature_map_kind.argtypes = [dp, C.c_int64, C.c_int, C.c_int, C.c_int, dp, dp, dp,
+                                           dp, dp, C.c_int, dp]
+        L.orc_feature_map_kind.restype = None
+        L.orc_attn_from_phi.argtypes = [dp, dp, dp] + [C.c_int] * 5 + [C.c_double, C.c_int,
+                                                                      dp, dp]
+        L.orc_attn_from_phi.restype = None
         L.orc_num_threads.argtypes = []
         L.orc_num_threads.restype = C.c_int
         _lib = L
@@ -278,8 +287,58 @@ def attn_bidir_bwd_given(q, k, v, out, den, dout, P: Params):
     return dq, dk, dv
 
 
+PHI_ANCHOR, PHI_ORTHOGONAL, PHI_SIGNED, PHI_PER_HEAD, PHI_PERFORMER = range(5)
+
+
+class KindParams:
+    """Sketch parameters of one variant (kind) and head: omega, anchors, anchors_b [F, D],
+    s, wt [R]; drawn by the oracle's own Philox and Gram-Schmidt."""
+
+    def __init__(self, D, R, m, seed, eps, kind, head=0):
+        F = R * m
+        self.D, self.R, self.m, self.seed, self.eps, self.F = D, R, m, seed, eps, F
+        self.kind, self.head = kind, head
+        self.omega = np.zeros((F, D))
+        self.anchors = np.zeros((F, D))
+        self.anchors_b = np.zeros((F, D))
+        self.s = np.zeros(R)
+        self.wt = np.zeros(R)
+        rc = lib().orc_sketch_params_kind(D, R, m, C.c_uint64(seed), eps, kind, head,
+                                          _p(self.omega), _p(self.anchors), _p(self.anchors_b),
+                                          _p(self.s), _p(self.wt))
+        if rc != 0:
+            raise ValueError("sketch_params_kind failed")
+
+
+def sketch_params_kind(D, R, m, seed, eps, kind, head=0) -> KindParams:
+    return KindParams(D, R, m, seed, eps, kind, head)
+
+
+def feature_map_kind(x, P: KindParams):
+    x = _d(x)
+    n = x.size // P.D
+    phi = np.zeros((n, P.F))
+    lib().orc_feature_map_kind(_p(x), n, P.D, P.R, P.m, _p(P.omega), _p(P.anchors),
+                               _p(P.anchors_b), _p(P.s), _p(P.wt), P.kind, _p(phi))
+    return phi.reshape(x.shape[:-1] + (P.F,))
+
+
+def attn_from_phi(pq, pk, v, eps, causal):
+    """The masked-sum contraction on given features pq, pk [B,H,L,F] and v [B,H,L,Dv]."""
+    pq, pk, v = _d(pq), _d(pk), _d(v)
+    B, H, L, F = pq.shape
+    Dv = v.shape[-1]
+    out = np.zeros((B, H, L, Dv))
+    den = np.zeros((B, H, L))
+    lib().orc_attn_from_phi(_p(pq), _p(pk), _p(v), B, H, L, F, Dv, float(eps), int(causal),
+                            _p(out), _p(den))
+    return out, den
+
+
 __all__ = ["lib", "num_threads", "philox4x32_10", "gauss_laguerre", "Params", "sketch_params",
            "yat_kernel", "quad_kernel", "feature_map", "attn_quadratic", "attn_quadratic_rows",
            "attn_recurrent", "decode_step", "attn_causal_bwd", "attn_causal_bwd_rows",
            "attn_causal_bwd_given", "attn_causal_bwd_given_rows", "feature_map_bwd",
-           "attn_bidir_bwd", "attn_bidir_bwd_given"]
+           "attn_bidir_bwd", "attn_bidir_bwd_given", "KindParams", "sketch_params_kind",
+           "feature_map_kind", "attn_from_phi", "PHI_ANCHOR", "PHI_ORTHOGONAL", "PHI_SIGNED",
+           "PHI_PER_HEAD", "PHI_PERFORMER"]

@@ -71,6 +71,20 @@ static double orc_normal(uint64_t seed, uint32_t idx, uint32_t tag)
     return sqrt(-2.0 * log(u1)) * cos(two_pi * u2);
 }
 
+/* The same normal from the counter (idx, tag, head, 0): the per-head draw of a sketch
+ * variant (head 0 is the counter above). */
+static double orc_normal_h(uint64_t seed, uint32_t idx, uint32_t tag, uint32_t head)
+{
+    uint32_t ctr[4] = { idx, tag, head, 0u };
+    uint32_t key[2] = { (uint32_t)(seed & 0xffffffffu), (uint32_t)(seed >> 32) };
+    uint32_t o[4];
+    orc_philox4x32_10(ctr, key, o);
+    const double two_pi = 6.283185307179586476925286766559;
+    double u1 = ((double)o[0] + 0.5) * (1.0 / 4294967296.0);
+    double u2 = ((double)o[1] + 0.5) * (1.0 / 4294967296.0);
+    return sqrt(-2.0 * log(u1)) * cos(two_pi * u2);
+}
+
 /* --------------------------------------------------------- Gauss-Laguerre */
 
 /* L_n(t) and L_{n-1}(t) by the three-term recurrence
@@ -213,6 +227,111 @@ static double dot(const double* a, const double* b, int64_t n)
 }
 
 /* phi of every row of one (b,h) slice: returns a malloc'd [L, F] array. */
+/* Sketch variants (the pages leave the anchor form and the feature bank open: review,
+ * "Proposed method", steps 3 and 5; orthogonal banks appear as prior art on the LinSimp
+ * page).  kind:
+ *   0 positive anchor (the default above): iid omega, phi = c e^{...} (a.x^)^2;
+ *   1 orthogonal: omega rows orthogonalised in blocks of D consecutive rows of a node by
+ *     Gram-Schmidt in draw order, each row keeping the length of its own Gaussian draw
+ *     (so every row is still N(0, I) marginally); anchors as kind 0;
+ *   2 signed anchor: phi = c e^{...} (a.x^)(b.x^) with a second anchor set b (tag 2),
+ *     unbiased for x^2 / D^2 but not positive;
+ *   3 per head: kind 0 drawn per head h with the counter (f D + d, tag, h, 0);
+ *   4 Performer FAVOR+: phi_f = exp(omega_f.x^ - 1/2) / sqrt(F), omega orthogonal as kind 1
+ *     (no quadrature, no anchor; the estimator of exp(q^.k^)).
+ * Values are rounded to float as in orc_sketch_params.  anchors_b is written for kind 2. */
+int orc_sketch_params_kind(int D, int R, int m, uint64_t seed, double eps, int kind, int head,
+                           double* omega, double* anchors, double* anchors_b, double* s,
+                           double* wt)
+{
+    double tn[64], wn[64];
+    if (kind < 0 || kind > 4 || head < 0 || D > 1024) return -1;
+    if (orc_gauss_laguerre(R, tn, wn) != 0) return -1;
+    for (int r = 0; r < R; ++r) {
+        s[r] = tn[r] / (2.0 + eps);
+        wt[r] = wn[r] / (2.0 + eps);
+    }
+    const int64_t F = (int64_t)R * m;
+    const uint32_t h = kind == 3 ? (uint32_t)head : 0u;
+    double* g = (double*)malloc(sizeof(double) * (size_t)F * D);
+    for (int64_t f = 0; f < F; ++f)
+        for (int d = 0; d < D; ++d) {
+            uint32_t idx = (uint32_t)(f * D + d);
+            g[f * D + d] = orc_normal_h(seed, idx, 0u, h);
+            anchors[f * D + d] = (double)(float)(orc_normal_h(seed, idx, 1u, h) / sqrt((double)D));
+            if (kind == 2)
+                anchors_b[f * D + d] = (double)(float)(orc_normal_h(seed, idx, 2u, h) / sqrt((double)D));
+        }
+    if (kind == 1 || kind == 4) {
+        /* classical Gram-Schmidt on each block: q_j = g_j - sum_{i<j} (g_j . e_i) e_i,
+         * e_j = q_j / |q_j|, row j = e_j |g_j| */
+        double* e = (double*)malloc(sizeof(double) * (size_t)D * D);
+        for (int r = 0; r < R; ++r)
+            for (int b0 = 0; b0 < m; b0 += D) {
+                int nb = m - b0 < D ? m - b0 : D;
+                for (int j = 0; j < nb; ++j) {
+                    const double* gj = g + ((int64_t)r * m + b0 + j) * D;
+                    double* ej = e + (int64_t)j * D;
+                    for (int d = 0; d < D; ++d) ej[d] = gj[d];
+                    for (int i = 0; i < j; ++i) {
+                        double c = dot(gj, e + (int64_t)i * D, D);
+                        for (int d = 0; d < D; ++d) ej[d] -= c * e[(int64_t)i * D + d];
+                    }
+                    double n = sqrt(dot(ej, ej, D));
+                    for (int d = 0; d < D; ++d) ej[d] /= n;
+                }
+                for (int j = 0; j < nb; ++j) {
+                    double* gj = g + ((int64_t)r * m + b0 + j) * D;
+                    double len = sqrt(dot(gj, gj, D));
+                    for (int d = 0; d < D; ++d) gj[d] = e[(int64_t)j * D + d] * len;
+                }
+            }
+        free(e);
+    }
+    for (int64_t t = 0; t < F * D; ++t) omega[t] = (double)(float)g[t];
+    free(g);
+    return 0;
+}
+
+/* phi of one row for a sketch variant (kinds 0-3 share the quadrature; kind 4 is FAVOR+) */
+static void phi_row_kind(const double* x, int D, int R, int m, const double* omega,
+                         const double* anchors, const double* anchors_b, const double* s,
+                         const double* wt, int kind, double* phi)
+{
+    double nrm = 0.0;
+    for (int d = 0; d < D; ++d) nrm += x[d] * x[d];
+    nrm = sqrt(nrm);
+    if (nrm < 1e-12) nrm = 1e-12;
+    double xh[1024];
+    for (int d = 0; d < D; ++d) xh[d] = x[d] / nrm;
+    const int64_t F = (int64_t)R * m;
+    for (int r = 0; r < R; ++r) {
+        double sq = sqrt(2.0 * s[r]);
+        double scale = sqrt(wt[r] / m);
+        for (int j = 0; j < m; ++j) {
+            int64_t f = (int64_t)r * m + j;
+            double u = dot(omega + f * D, xh, D);
+            if (kind == 4) {
+                phi[f] = exp(u - 0.5) / sqrt((double)F);
+                continue;
+            }
+            double p = dot(anchors + f * D, xh, D);
+            double pb = kind == 2 ? dot(anchors_b + f * D, xh, D) : p;
+            phi[f] = scale * exp(sq * u - s[r]) * p * pb;
+        }
+    }
+}
+
+void orc_feature_map_kind(const double* x, int64_t n, int D, int R, int m,
+                          const double* omega, const double* anchors, const double* anchors_b,
+                          const double* s, const double* wt, int kind, double* phi)
+{
+    const int64_t F = (int64_t)R * m;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i)
+        phi_row_kind(x + i * D, D, R, m, omega, anchors, anchors_b, s, wt, kind, phi + i * F);
+}
+
 static double* phi_slice(const double* x, int L, int D, int R, int m,
                          const double* omega, const double* anchors,
                          const double* s, const double* wt)
@@ -765,6 +884,24 @@ void orc_attn_bidir_bwd_given(const double* q, const double* k, const double* v,
                              omega, anchors, s, wt, dk + ((int64_t)bh * L + i) * D);
         }
         free(pq); free(pk); free(dn); free(delta); free(dpq); free(dpk);
+    }
+}
+
+/* The linear-attention contraction on given features (review, "Proposed method", step 6,
+ * as its plain masked sum): out_i = sum_{j in J(i)} (pq_i . pk_j) v_j / (sum_{j in J(i)}
+ * pq_i . pk_j + eps), J(i) = {j <= i} (causal) or all j.  pq, pk: [B,H,L,F]. */
+void orc_attn_from_phi(const double* pq, const double* pk, const double* v,
+                       int B, int H, int L, int F, int Dv, double eps, int causal,
+                       double* out, double* den)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bh = 0; bh < B * H; ++bh) {
+        const double* qs = pq + (int64_t)bh * L * F;
+        const double* ks = pk + (int64_t)bh * L * F;
+        const double* vs = v + (int64_t)bh * L * Dv;
+        for (int i = 0; i < L; ++i)
+            quad_row(qs + (int64_t)i * F, ks, vs, L, Dv, F, eps, causal, i,
+                     out + ((int64_t)bh * L + i) * Dv, den + (int64_t)bh * L + i);
     }
 }
 

@@ -148,6 +148,15 @@ void orc_attn_bidir_bwd_given(const double* q, const double* k, const double* v,
                               const double* omega, const double* anchors,
                               const double* s, const double* wt, double eps,
                               double* dq, double* dk, double* dv);
+int orc_sketch_params_kind(int D, int R, int m, uint64_t seed, double eps, int kind, int head,
+                           double* omega, double* anchors, double* anchors_b, double* s,
+                           double* wt);
+void orc_feature_map_kind(const double* x, int64_t n, int D, int R, int m,
+                          const double* omega, const double* anchors, const double* anchors_b,
+                          const double* s, const double* wt, int kind, double* phi);
+void orc_attn_from_phi(const double* pq, const double* pk, const double* v,
+                       int B, int H, int L, int F, int Dv, double eps, int causal,
+                       double* out, double* den);
 int orc_num_threads(void);
 
 #ifdef __cplusplus

@@ -465,3 +465,109 @@ def test_bidir_backward_given_output_reduces_and_is_affine_in_out():
     np.testing.assert_allclose(one[2], base[2], rtol=1e-13, atol=1e-15)
     for b, o1, o2 in zip(base[:2], one[:2], two[:2]):
         np.testing.assert_allclose(o2 - b, 2 * (o1 - b), rtol=1e-6, atol=1e-12)
+
+
+# ----------------------------------------------------------- sketch variants
+
+def test_kind_zero_is_the_default_map():
+    P0 = O.sketch_params(D=16, R=3, m=8, seed=5, eps=1e-6)
+    Pk = O.sketch_params_kind(16, 3, 8, 5, 1e-6, O.PHI_ANCHOR)
+    assert np.array_equal(P0.omega, Pk.omega) and np.array_equal(P0.anchors, Pk.anchors)
+    x = np.random.default_rng(40).standard_normal((7, 16))
+    assert np.array_equal(O.feature_map(x, P0), O.feature_map_kind(x, Pk))
+
+
+def test_orthogonal_bank_blocks():
+    D, R, m = 8, 2, 20                     # blocks of 8, 8 and 4 rows in each node
+    P0 = O.sketch_params(D=D, R=R, m=m, seed=6, eps=1e-6)
+    P = O.sketch_params_kind(D, R, m, 6, 1e-6, O.PHI_ORTHOGONAL)
+    assert np.array_equal(P.anchors, P0.anchors)
+    # every row keeps the length of its Gaussian draw; the first row of a block is unchanged
+    np.testing.assert_allclose(np.linalg.norm(P.omega, axis=1), np.linalg.norm(P0.omega, axis=1),
+                               rtol=1e-6)
+    for r in range(R):
+        for b0 in (0, 8, 16):
+            f0 = r * m + b0
+            nb = min(8, m - b0)
+            assert np.array_equal(P.omega[f0], P0.omega[f0])
+            blk = P.omega[f0:f0 + nb]
+            G = blk @ blk.T
+            nrm = np.sqrt(np.diag(G))
+            cos = G / np.outer(nrm, nrm)
+            assert np.abs(cos - np.eye(nb)).max() < 1e-6
+    # rows of different blocks are not made orthogonal
+    cross = P.omega[0] @ P.omega[8] / (np.linalg.norm(P.omega[0]) * np.linalg.norm(P.omega[8]))
+    assert abs(cross) > 1e-3
+
+
+def _mc_product(P, x, D, R, m, kind_map):
+    q = np.zeros(D); q[0] = 1.0
+    k = np.zeros(D); k[0] = x; k[1] = math.sqrt(1 - x * x)
+    pq = kind_map(q[None], P)[0]
+    pk = kind_map(k[None], P)[0]
+    return (pq * pk).reshape(R, m) * m
+
+
+@pytest.mark.parametrize("x", [0.35, -0.4])
+def test_orthogonal_bank_keeps_the_estimator_unbiased(x):
+    # every omega row is N(0, I) marginally, so the per-node mean is kind 0's closed form.
+    # The top node is left out: its weight exp(sqrt(2 s) w.(q + k) - 2 s) is log-normal with
+    # sigma near 4 there, too heavy-tailed for a bound from the sample spread; the lower
+    # nodes already fail if the rows lost their Gaussian lengths (unit rows change the mgf).
+    D, R, m = 4, 3, 200000
+    P = O.sketch_params_kind(D, R, m, 12, 1e-6, O.PHI_ORTHOGONAL)
+    prod = _mc_product(P, x, D, R, m, O.feature_map_kind)
+    for r in range(R - 1):
+        want = P.wt[r] * math.exp(2 * P.s[r] * x) * (1 + 2 * x * x) / D ** 2
+        sem = prod[r].std() / math.sqrt(m)
+        assert abs(prod[r].mean() - want) < 4.5 * sem, (r, prod[r].mean(), want, sem)
+
+
+@pytest.mark.parametrize("x", [0.35, -0.4])
+def test_signed_anchor_is_unbiased_for_the_square(x):
+    # E[(a.q)(b.q)(a.k)(b.k)] = E[(a.q)(a.k)] E[(b.q)(b.k)] = (x / D)^2 for independent a, b
+    D, R, m = 4, 3, 200000
+    P = O.sketch_params_kind(D, R, m, 13, 1e-6, O.PHI_SIGNED)
+    assert not np.array_equal(P.anchors, P.anchors_b)
+    prod = _mc_product(P, x, D, R, m, O.feature_map_kind)
+    for r in range(R):
+        want = P.wt[r] * math.exp(2 * P.s[r] * x) * x * x / D ** 2
+        sem = prod[r].std() / math.sqrt(m)
+        assert abs(prod[r].mean() - want) < 4.5 * sem, (r, prod[r].mean(), want, sem)
+    phi = O.feature_map_kind(np.random.default_rng(41).standard_normal((50, D)), P)
+    assert (phi < 0).any() and (phi > 0).any()      # signed: not a positive feature map
+
+
+def test_per_head_draws():
+    P0 = O.sketch_params(D=16, R=2, m=8, seed=7, eps=1e-6)
+    h0 = O.sketch_params_kind(16, 2, 8, 7, 1e-6, O.PHI_PER_HEAD, head=0)
+    h3 = O.sketch_params_kind(16, 2, 8, 7, 1e-6, O.PHI_PER_HEAD, head=3)
+    assert np.array_equal(h0.omega, P0.omega) and np.array_equal(h0.anchors, P0.anchors)
+    assert not np.array_equal(h3.omega, h0.omega)
+    big = O.sketch_params_kind(64, 4, 256, 7, 1e-6, O.PHI_PER_HEAD, head=5)
+    assert abs(big.omega.mean()) < 0.01 and abs(big.omega.var() - 1) < 0.02
+    assert abs(big.anchors.var() * 64 - 1) < 0.02
+
+
+@pytest.mark.parametrize("x", [0.35, -0.4])
+def test_performer_features_estimate_exp(x):
+    # FAVOR+: E[exp(w.q - 1/2) exp(w.k - 1/2)] = exp(|q + k|^2 / 2 - 1) = exp(q.k) on the
+    # sphere, so F * mean_f phi_f(q) phi_f(k) -> exp(x)
+    D, R, m = 4, 1, 200000
+    P = O.sketch_params_kind(D, R, m, 14, 1e-6, O.PHI_PERFORMER)
+    prod = _mc_product(P, x, D, R, m, O.feature_map_kind)[0]
+    sem = prod.std() / math.sqrt(m)
+    assert abs(prod.mean() - math.exp(x)) < 4.5 * sem, (prod.mean(), math.exp(x), sem)
+    assert sem < 0.02 * math.exp(x)
+    phi = O.feature_map_kind(np.random.default_rng(42).standard_normal((20, D)), P)
+    assert (phi > 0).all()
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_contraction_on_given_features_is_the_quadratic_form(causal):
+    q, k, v = _small(43, B=1, H=2, L=29, D=16, Dv=8)
+    P = O.sketch_params(D=16, R=3, m=8, seed=5, eps=1e-6)
+    want, wden = O.attn_quadratic(q, k, v, P, causal)
+    got, gden = O.attn_from_phi(O.feature_map(q, P), O.feature_map(k, P), v, P.eps, causal)
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(gden, wden, rtol=1e-12)
