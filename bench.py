@@ -3,7 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload causal_16k|causal_2k|bidir_vision|fwd_8k|bwd_8k|bidir_bwd|decode|
-                                feature_map|feature_map_bwd]
+                                feature_map|feature_map_bwd|matched_budget]
 
 With --gpus N > 1 outside torchrun, bench.py starts the N ranks itself (torch.distributed.run
 on 127.0.0.1); under torchrun, --gpus must equal WORLD_SIZE.
@@ -44,6 +44,7 @@ WORKLOADS = {
     "bwd_8k": (W.FWDBWD_8K, "bwd"),
     "bidir_bwd": (W.BIDIR_VISION, "bidir_bwd"),
     "feature_map_bwd": (W.CAUSAL_16K, "feature_map_bwd"),
+    "matched_budget": (W.CAUSAL_16K, "matched_budget"),
     "decode": (W.DECODE, "decode"),
     "feature_map": (W.CAUSAL_16K, "feature_map"),
 }
@@ -582,6 +583,92 @@ def run_ours(args, w, op):
     return 0
 
 
+# ------------------------------------------------- matched-feature-budget comparison
+
+def run_comparison(args, w):
+    """Latency of the causal forward at one feature budget F = R*m with different feature
+    maps on the same kernels: the SLAY map (positive anchor) and the Performer FAVOR+ map,
+    both by the CUDA-core variant kernel, each followed by the same contraction on the given
+    features; the SLAY map on tensor cores followed by that contraction; and the fused
+    tensor-core SLAY forward.  Inputs resident in HBM, L2 flushed between steps, CUDA events
+    on the launching stream; rank 0 prints one JSON line (a comparison, not the headline)."""
+    import torch
+    from kernelized_linear_attention_unit_b200 import binding as bd
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    eps = float(np.float32(w.eps))
+    qn, kn, vn = W.gen_qkv(w)
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dev).to(torch.bfloat16)
+    q, k, v = to(qn), to(kn), to(vn)
+    B, H, L, F = w.B, w.H, w.L, w.F
+    pq = torch.empty((B, H, L, F), device=dev, dtype=torch.bfloat16)
+    pk = torch.empty_like(pq)
+    out = torch.empty_like(v)
+    den = torch.empty((B, H, L), device=dev, dtype=torch.float32)
+    wl = bd.alloc_workspace(bd.OP_LINEAR_ATTN, bd.SLAY_BF16, B, H, L, 64, 64, 1, F, dev)
+    wf = bd.alloc_workspace(bd.OP_CAUSAL_FWD, bd.SLAY_BF16, B, H, L, 64, 64, w.R, w.m, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def maps(kind):
+        if kind is None:          # the library's default map (tensor cores for these sizes)
+            bd.slay_feature_map(q, pq, w.R, w.m, w.sketch_seed, eps)
+            bd.slay_feature_map(k, pk, w.R, w.m, w.sketch_seed, eps)
+        else:                     # the CUDA-core variant kernel (per head with one head = SLAY)
+            bd.slay_feature_map_ex(q, pq, w.R, w.m, w.sketch_seed, eps, kind, 1, L)
+            bd.slay_feature_map_ex(k, pk, w.R, w.m, w.sketch_seed, eps, kind, 1, L)
+
+    def contract():
+        bd.slay_linear_attn_fwd(pq, pk, v, out, den, eps, True, wl)
+
+    arms = {
+        "slay_anchor_cuda_cores": (lambda: maps(bd.PHI_PER_HEAD), contract),
+        "performer_favor_cuda_cores": (lambda: maps(bd.PHI_PERFORMER), contract),
+        "slay_anchor_tensor_cores": (lambda: maps(None), contract),
+        "slay_fused_tensor_cores": (None, lambda: bd.slay_attn_causal_fwd(
+            q, k, v, out, den, w.R, w.m, w.sketch_seed, eps, wf)),
+    }
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for a, b in ev:
+            flush.zero_()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in ev) / args.steps
+
+    res = {}
+    for name, (mp_, ct) in arms.items():
+        step = (lambda m=mp_, c=ct: (m(), c())) if mp_ else ct
+        ms = timed(step)
+        entry = {"ms_per_step": ms, "tokens_per_s": B * L / (ms / 1e3)}
+        if mp_:
+            entry["map_ms"] = timed(mp_)
+        res[name] = entry
+    base = res["slay_anchor_cuda_cores"]
+    perf = res["performer_favor_cuda_cores"]
+    if rank == 0:
+        line = {"metric": "causal fwd latency at a matched feature budget (F=%d)" % F,
+                "value": base["tokens_per_s"], "unit": "tokens/s", "n_gpus": 1,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": base["ms_per_step"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": {**config_of(w, "causal"), "workload": "matched_budget_" + w.name},
+                "comparison": res,
+                "map_ratio_performer_over_slay": perf["map_ms"] / base["map_ms"],
+                "step_ratio_performer_over_slay": perf["ms_per_step"] / base["ms_per_step"]}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 # ------------------------------------------------------------ rank launch
 
 def free_port():
@@ -662,6 +749,8 @@ def main(argv=None):
     w, op = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w, op)
+    if op == "matched_budget":
+        return run_comparison(args, w)
     return run_ours(args, w, op)
 
 

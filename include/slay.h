@@ -70,8 +70,25 @@ typedef enum {
     SLAY_OP_BIDIR_FWD = 2,
     SLAY_OP_CAUSAL_BWD = 3,
     SLAY_OP_DECODE = 4,
-    SLAY_OP_BIDIR_BWD = 5
+    SLAY_OP_BIDIR_BWD = 5,
+    SLAY_OP_LINEAR_ATTN = 6     /* slay_linear_attn_fwd: R * m = the number of features */
 } slay_op;
+
+/* Feature-map variants (slay_feature_map_ex).  The pages leave the form of the anchor
+ * feature and of the random-feature bank open (review, "Proposed method", steps 3 and 5);
+ * orthogonal banks and FAVOR+ features are prior art on the other pages and the abstract
+ * compares SLAY with Performers.  Sketch draws follow the Philox spec above; "orthogonal"
+ * rows are made orthonormal in blocks of D consecutive rows of a node (Gram-Schmidt in draw
+ * order), each row keeping the length of its own Gaussian draw. */
+typedef enum {
+    SLAY_PHI_ANCHOR = 0,       /* SLAY: iid omega, positive anchor (a.x^)^2 (the default) */
+    SLAY_PHI_ORTHOGONAL = 1,   /* SLAY with an orthogonal omega bank */
+    SLAY_PHI_SIGNED = 2,       /* SLAY with (a.x^)(b.x^), b a second anchor set (counter tag 2):
+                                  unbiased for (q^.k^)^2 / D^2, not positive */
+    SLAY_PHI_PER_HEAD = 3,     /* SLAY with omega, a drawn per head h (counter (f*D+d, tag, h, 0)) */
+    SLAY_PHI_PERFORMER = 4     /* Performer FAVOR+: exp(omega_f.x^ - 1/2) / sqrt(F), orthogonal
+                                  omega, F = R*m features; estimates exp(q^.k^) */
+} slay_phi_kind;
 
 /* Feature map phi (review, "Proposed method", steps 1, 3, 4, 5).
  * x   : device [n_rows, D] in `in_dt` (rows need not be unit length; they are
@@ -142,6 +159,39 @@ slay_status slay_attn_bidir_bwd(const void* q, const void* k, const void* v,
                                 int B, int H, int L, int D, int Dv,
                                 slay_dtype dt, int R, int m, uint64_t seed, float eps,
                                 void* workspace, size_t ws_bytes, void* stream);
+
+/* Feature map of a variant kind (slay_phi_kind), for the matched-feature-budget comparisons
+ * and the sketch variants; arguments as slay_feature_map plus:
+ *   kind          : the variant; SLAY_PHI_ANCHOR is slay_feature_map itself.
+ *   heads, rows_per_head : for SLAY_PHI_PER_HEAD, the rows are sequences of rows_per_head
+ *                   rows ([B,H,L,D] with rows_per_head = L) and sequence z uses head z % heads'
+ *                   parameters (n_rows must be a multiple of rows_per_head); ignored otherwise.
+ * Variants other than SLAY_PHI_ANCHOR run on CUDA cores in fp32; the library caches their
+ * parameters per (device, D, R, m, seed, eps, kind, heads) like the default ones. */
+slay_status slay_feature_map_ex(const void* x, void* phi, int64_t n_rows, int D,
+                               slay_dtype in_dt, slay_dtype out_dt, int R, int m, uint64_t seed,
+                               float eps, int kind, int heads, int64_t rows_per_head,
+                               void* stream);
+
+/* Host copy of a variant's sketch parameters (for tests): omega, anchors, anchors_b
+ * [R*m, D] float (anchors_b only for SLAY_PHI_SIGNED; each may be NULL), s, w [R] double, for
+ * head `head` (SLAY_PHI_PER_HEAD; other kinds ignore it).  Host only. */
+slay_status slay_sketch_params_ex(int D, int R, int m, uint64_t seed, float eps, int kind,
+                                  int head, float* omega_host, float* anchors_host,
+                                  float* anchors_b_host, double* s_host, double* w_host);
+
+/* The linear-attention contraction on given features (review, "Proposed method", step 6):
+ *   out_i = sum_{j in J(i)} (phq_i . phk_j) v_j / (sum_{j in J(i)} phq_i . phk_j + eps)
+ * computed in O(L) by 64-token chunks with fp32 states, J(i) = {j <= i} (causal != 0) or
+ * all j.  Any feature map composes with it: slay_feature_map(_ex) for q and k, then this.
+ * phq, phk : device [B,H,L,F] in dt;  v : device [B,H,L,Dv] in dt;  out : [B,H,L,Dv] in dt;
+ * den      : device [B,H,L] fp32 or NULL (den_i without eps).  F <= 1024, Dv == 64.
+ * workspace: slay_workspace_bytes(SLAY_OP_LINEAR_ATTN, dt, B, H, L, 64, Dv, 1, F) bytes.
+ * CUDA cores, fp32 arithmetic (bf16 operands are widened on load). */
+slay_status slay_linear_attn_fwd(const void* phq, const void* phk, const void* v, void* out,
+                                 float* den, int B, int H, int L, int F, int Dv, slay_dtype dt,
+                                 float eps, int causal, void* workspace, size_t ws_bytes,
+                                 void* stream);
 
 /* Backward of the feature map alone (review, "Proposed method", steps 1, 3, 4, 5; the
  * pages give no backward): dx = (d phi / d x)^T dphi for every row, through the sphere

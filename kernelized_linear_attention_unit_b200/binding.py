@@ -17,13 +17,16 @@ LIB_PATH = os.path.join(_HERE, "libslay.so")
 SLAY_OK, SLAY_ERR_INVALID_ARG, SLAY_ERR_UNSUPPORTED, SLAY_ERR_CUDA, SLAY_ERR_TIMEOUT, \
     SLAY_ERR_NO_MEMORY = range(6)
 SLAY_F32, SLAY_BF16 = 0, 1
-OP_FEATURE_MAP, OP_CAUSAL_FWD, OP_BIDIR_FWD, OP_CAUSAL_BWD, OP_DECODE, OP_BIDIR_BWD = range(6)
+OP_FEATURE_MAP, OP_CAUSAL_FWD, OP_BIDIR_FWD, OP_CAUSAL_BWD, OP_DECODE, OP_BIDIR_BWD, \
+    OP_LINEAR_ATTN = range(7)
+PHI_ANCHOR, PHI_ORTHOGONAL, PHI_SIGNED, PHI_PER_HEAD, PHI_PERFORMER = range(5)
 
 EXPORTS = ["slay_feature_map", "slay_attn_causal_fwd", "slay_attn_bidir_fwd",
            "slay_attn_causal_bwd", "slay_decode_step", "slay_workspace_bytes", "slay_prepare",
            "slay_sketch_params", "slay_status_string", "slay_last_error", "slay_trace_enable",
            "slay_trace_read", "slay_attn_causal_fwd_noalloc", "slay_kernel_status",
-           "slay_debug_expire_wait", "slay_attn_bidir_bwd", "slay_feature_map_bwd"]
+           "slay_debug_expire_wait", "slay_attn_bidir_bwd", "slay_feature_map_bwd",
+           "slay_feature_map_ex", "slay_sketch_params_ex", "slay_linear_attn_fwd"]
 
 
 class SlayError(RuntimeError):
@@ -59,6 +62,11 @@ def lib():
                                        i32, i32, i32, i32, u64, f32, vp, sz, vp]
     L.slay_attn_bidir_bwd.argtypes = L.slay_attn_causal_bwd.argtypes
     L.slay_feature_map_bwd.argtypes = [vp, vp, vp, i64, i32, i32, i32, i32, i32, u64, f32, vp]
+    L.slay_feature_map_ex.argtypes = [vp, vp, i64, i32, i32, i32, i32, i32, u64, f32, i32, i32,
+                                      i64, vp]
+    L.slay_sketch_params_ex.argtypes = [i32, i32, i32, u64, f32, i32, i32, vp, vp, vp, vp, vp]
+    L.slay_linear_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32,
+                                       i32, vp, sz, vp]
     L.slay_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                    u64, f32, vp]
     L.slay_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32]
@@ -79,7 +87,8 @@ def lib():
     L.slay_trace_read.restype = i32
     for name in ("slay_feature_map", "slay_attn_causal_fwd", "slay_attn_bidir_fwd",
                  "slay_attn_causal_bwd", "slay_decode_step", "slay_prepare",
-                 "slay_attn_bidir_bwd", "slay_feature_map_bwd",
+                 "slay_attn_bidir_bwd", "slay_feature_map_bwd", "slay_feature_map_ex",
+                 "slay_sketch_params_ex", "slay_linear_attn_fwd",
                  "slay_attn_causal_fwd_noalloc",
                  "slay_sketch_params"):
         getattr(L, name).restype = i32
@@ -264,6 +273,54 @@ def slay_attn_bidir_bwd(q, k, v, out, den, dout, dq, dk, dv, R, m, seed, eps, wo
     """Enqueue the bidirectional backward; returns the workspace it used."""
     return _attn_bwd(lib().slay_attn_bidir_bwd, "slay_attn_bidir_bwd", OP_BIDIR_BWD, q, k, v,
                      out, den, dout, dq, dk, dv, R, m, seed, eps, workspace, stream)
+
+
+def slay_feature_map_ex(x, phi, R, m, seed, eps, kind, heads=1, rows_per_head=0, stream=None):
+    """phi of a variant kind (PHI_*); per-head rows are sequences of rows_per_head rows."""
+    _check(x, "x")
+    _check(phi, "phi")
+    D = x.shape[-1]
+    n = x.numel() // D if D else 0
+    if phi.numel() != n * R * m or phi.shape[-1] != R * m:
+        raise ValueError("phi must have %d rows of %d features" % (n, R * m))
+    _raise(lib().slay_feature_map_ex(_ptr(x), _ptr(phi), n, D, _dt(x), _dt(phi), R, m, seed,
+                                     eps, kind, heads, rows_per_head, _stream(stream)),
+           "slay_feature_map_ex")
+
+
+def slay_sketch_params_ex(D, R, m, seed, eps, kind, head=0):
+    """Host copy of a variant's (omega, anchors, anchors_b [F,D] f32, s, wt [R] f64)."""
+    import numpy as np
+    F = R * m
+    om = np.zeros((F, D), np.float32)
+    an = np.zeros((F, D), np.float32)
+    anb = np.zeros((F, D), np.float32)
+    s = np.zeros(R, np.float64)
+    w = np.zeros(R, np.float64)
+    _raise(lib().slay_sketch_params_ex(D, R, m, seed, eps, kind, head, om.ctypes.data,
+                                       an.ctypes.data, anb.ctypes.data, s.ctypes.data,
+                                       w.ctypes.data), "slay_sketch_params_ex")
+    return om, an, anb, s, w
+
+
+def slay_linear_attn_fwd(phq, phk, v, out, den, eps, causal, workspace=None, stream=None):
+    """The contraction on given features phq, phk [B,H,L,F] (causal or bidirectional)."""
+    _check(phq, "phq")
+    B, H, L, F = phq.shape
+    Dv = v.shape[-1]
+    _check(phk, "phk", phq.dtype, (B, H, L, F))
+    _check(v, "v", phq.dtype, (B, H, L, Dv))
+    _check(out, "out", phq.dtype, (B, H, L, Dv))
+    if den is not None:
+        _check(den, "den", torch.float32, (B, H, L))
+    dt = _dt(phq)
+    if workspace is None:
+        workspace = alloc_workspace(OP_LINEAR_ATTN, dt, B, H, L, 64, Dv, 1, F, phq.device)
+    wbytes = workspace.numel() * workspace.element_size()
+    _raise(lib().slay_linear_attn_fwd(_ptr(phq), _ptr(phk), _ptr(v), _ptr(out), _ptr(den), B, H,
+                                      L, F, Dv, dt, eps, 1 if causal else 0, _ptr(workspace),
+                                      wbytes, _stream(stream)), "slay_linear_attn_fwd")
+    return workspace
 
 
 def slay_feature_map_bwd(x, dphi, dx, R, m, seed, eps, stream=None):

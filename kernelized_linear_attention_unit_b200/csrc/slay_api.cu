@@ -128,6 +128,77 @@ slay_status get_params(int D, int R, int m, uint64_t seed, float eps, Params* ou
     return SLAY_OK;
 }
 
+// ---- sketch variants: one cache entry per (device, D, R, m, seed, eps, kind, heads)
+using VKey = std::tuple<int, int, int, int, uint64_t, uint32_t, int, int>;
+
+struct VEntry {
+    void* dev = nullptr;
+    VarParams P{};
+};
+
+std::map<VKey, VEntry>& vcache()
+{
+    static std::map<VKey, VEntry>* c = new std::map<VKey, VEntry>();  // held until exit
+    return *c;
+}
+
+slay_status get_var_params(int D, int R, int m, uint64_t seed, float eps, int kind, int H,
+                           VarParams* out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    const VKey key{dev, D, R, m, seed, float_bits(eps), kind, H};
+    std::lock_guard<std::mutex> lock(g_mu);
+    auto it = vcache().find(key);
+    if (it != vcache().end()) { *out = it->second.P; return SLAY_OK; }
+    const int F = R * m;
+    const size_t nF = static_cast<size_t>(F) * D;
+    std::vector<float> om(nF), an(nF), anb(nF);
+    // [3][H][D][F]: omega^T, anchors^T, second anchors^T
+    std::vector<float> host(3 * static_cast<size_t>(H) * nF, 0.0f);
+    double sr[kMaxR], wt[kMaxR];
+    for (int h = 0; h < H; ++h) {
+        if (!draw_sketch_kind(D, R, m, seed, static_cast<double>(eps), kind, h, om.data(),
+                              an.data(), anb.data(), sr, wt))
+            return SLAY_ERR_INVALID_ARG;
+        for (int f = 0; f < F; ++f)
+            for (int d = 0; d < D; ++d) {
+                const size_t src = static_cast<size_t>(f) * D + d;
+                const size_t dst = static_cast<size_t>(h) * nF + static_cast<size_t>(d) * F + f;
+                host[dst] = om[src];
+                host[static_cast<size_t>(H) * nF + dst] = an[src];
+                host[2 * static_cast<size_t>(H) * nF + dst] = kind == 2 ? anb[src] : 0.0f;
+            }
+    }
+    VEntry ent;
+    const size_t bytes = host.size() * sizeof(float);
+    e = cudaMalloc(&ent.dev, bytes);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaMemcpy(ent.dev, host.data(), bytes, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) { cudaFree(ent.dev); return cuda_fail(e); }
+    float* d = static_cast<float*>(ent.dev);
+    VarParams& P = ent.P;
+    P.omT = d;
+    P.anT = d + static_cast<size_t>(H) * nF;
+    P.anbT = d + 2 * static_cast<size_t>(H) * nF;
+    P.F = F; P.m = m; P.R = R; P.H = H; P.kind = kind;
+    const double log2e = 1.4426950408889634073599246810019;
+    for (int r = 0; r < kMaxR; ++r) {
+        if (r >= R) { P.a2[r] = P.b2[r] = 0.0f; continue; }
+        if (kind == 4) {   // FAVOR+: exp(u - 1/2) / sqrt(F) = exp2(log2e u - (log2e + log2 F) / 2)
+            P.a2[r] = static_cast<float>(log2e);
+            P.b2[r] = static_cast<float>(-0.5 * (log2e + std::log2(static_cast<double>(F))));
+        } else {
+            P.a2[r] = static_cast<float>(std::sqrt(2.0 * sr[r]) * log2e);
+            P.b2[r] = static_cast<float>(std::log2(std::sqrt(wt[r] / m)) - sr[r] * log2e);
+        }
+    }
+    vcache()[key] = ent;
+    *out = P;
+    return SLAY_OK;
+}
+
 }  // namespace
 
 bool eps_ok(float eps) { return std::isfinite(eps) && eps > 0.0f; }
@@ -168,6 +239,7 @@ size_t attn_ws(slay_op op, slay_dtype dt, int B, int H, int L, int Dv, int R, in
         case SLAY_OP_BIDIR_FWD: return kWsHeader + simt_ws_bidir(B, H, L, Dv, F);
         case SLAY_OP_CAUSAL_BWD: return kWsHeader + simt_ws_bwd(B, H, L, Dv, F);
         case SLAY_OP_BIDIR_BWD: return kWsHeader + simt_ws_bidir_bwd(B, H, L, Dv, F);
+        case SLAY_OP_LINEAR_ATTN: return kWsHeader + simt_ws_linear(B, H, L, F);
         default: return 0;
     }
 }
@@ -307,6 +379,77 @@ slay_status slay_attn_bidir_bwd(const void* q, const void* k, const void* v, con
                     workspace, ws_bytes, stream, false);
 }
 
+slay_status slay_feature_map_ex(const void* x, void* phi, int64_t n_rows, int D,
+                               slay_dtype in_dt, slay_dtype out_dt, int R, int m, uint64_t seed,
+                               float eps, int kind, int heads, int64_t rows_per_head,
+                               void* stream)
+{
+    if (kind < SLAY_PHI_ANCHOR || kind > SLAY_PHI_PERFORMER) return SLAY_ERR_INVALID_ARG;
+    if (kind == SLAY_PHI_ANCHOR)
+        return slay_feature_map(x, phi, n_rows, D, in_dt, out_dt, R, m, seed, eps, stream);
+    if (n_rows < 0) return SLAY_ERR_INVALID_ARG;
+    slay_status s = check_shape(D, kD, R, m);
+    if (s != SLAY_OK) return s;
+    if (!dtype_ok(in_dt) || !dtype_ok(out_dt) || !eps_ok(eps)) return SLAY_ERR_INVALID_ARG;
+    if (in_dt == SLAY_F32 && out_dt == SLAY_BF16) return SLAY_ERR_UNSUPPORTED;
+    int H = 1;
+    int64_t Lh = n_rows;
+    if (kind == SLAY_PHI_PER_HEAD) {
+        if (heads <= 0 || heads > 1024 || rows_per_head <= 0) return SLAY_ERR_INVALID_ARG;
+        if (n_rows % rows_per_head != 0) return SLAY_ERR_INVALID_ARG;
+        H = heads;
+        Lh = rows_per_head;
+    }
+    if (n_rows == 0) return SLAY_OK;
+    if (!x || !phi || !aligned(x, 16) || !aligned(phi, 16)) return SLAY_ERR_INVALID_ARG;
+    if ((Lh + 63) / 64 > (int64_t(1) << 31) - 1 || n_rows / Lh > 65535) return SLAY_ERR_UNSUPPORTED;
+    VarParams P;
+    if ((s = get_var_params(D, R, m, seed, eps, kind, H, &P)) != SLAY_OK) return s;
+    cudaError_t e = simt_feature_map_kind(x, phi, n_rows, Lh, in_dt, out_dt, P,
+                                          static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
+}
+
+slay_status slay_sketch_params_ex(int D, int R, int m, uint64_t seed, float eps, int kind,
+                                  int head, float* omega_host, float* anchors_host,
+                                  float* anchors_b_host, double* s_host, double* w_host)
+{
+    if (D <= 0 || D > 4096 || R <= 0 || R > kMaxR || m <= 0 || !eps_ok(eps) || head < 0)
+        return SLAY_ERR_INVALID_ARG;
+    if (kind < SLAY_PHI_ANCHOR || kind > SLAY_PHI_PERFORMER) return SLAY_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(R) * m * D > (int64_t(1) << 31)) return SLAY_ERR_UNSUPPORTED;
+    if (!draw_sketch_kind(D, R, m, seed, static_cast<double>(eps), kind, head, omega_host,
+                          anchors_host, anchors_b_host, s_host, w_host))
+        return SLAY_ERR_INVALID_ARG;
+    return SLAY_OK;
+}
+
+slay_status slay_linear_attn_fwd(const void* phq, const void* phk, const void* v, void* out,
+                                 float* den, int B, int H, int L, int F, int Dv, slay_dtype dt,
+                                 float eps, int causal, void* workspace, size_t ws_bytes,
+                                 void* stream)
+{
+    if (B < 0 || H < 0 || L < 0 || F <= 0 || Dv <= 0) return SLAY_ERR_INVALID_ARG;
+    if (Dv != kD) return SLAY_ERR_UNSUPPORTED;
+    if (F > kMaxF) return SLAY_ERR_UNSUPPORTED;
+    if (!dtype_ok(dt) || !eps_ok(eps)) return SLAY_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(B) * H * L == 0) return SLAY_OK;
+    if (!phq || !phk || !v || !out) return SLAY_ERR_INVALID_ARG;
+    if (!aligned(phq, 16) || !aligned(phk, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        (den && !aligned(den, 4)))
+        return SLAY_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(B) * H > 65535 || (static_cast<int64_t>(L) + 63) / 64 > 65535)
+        return SLAY_ERR_UNSUPPORTED;
+    const size_t need = kWsHeader + simt_ws_linear(B, H, L, F);
+    if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return SLAY_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
+    if (e == cudaSuccess)
+        e = simt_linear_attn(phq, phk, v, out, den, B, H, L, F, dt, eps, causal != 0,
+                             static_cast<char*>(workspace) + kWsHeader, st);
+    return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
+}
+
 slay_status slay_feature_map_bwd(const void* x, const void* dphi, float* dx, int64_t n_rows,
                                  int D, slay_dtype x_dt, slay_dtype dphi_dt, int R, int m,
                                  uint64_t seed, float eps, void* stream)
@@ -384,8 +527,12 @@ size_t slay_workspace_bytes(slay_op op, slay_dtype dt, int B, int H, int L, int 
     if (check_shape(D, Dv, R, m) != SLAY_OK) return SIZE_MAX;
     if (op == SLAY_OP_FEATURE_MAP || op == SLAY_OP_DECODE) return 0;
     if (op != SLAY_OP_CAUSAL_FWD && op != SLAY_OP_BIDIR_FWD && op != SLAY_OP_CAUSAL_BWD &&
-        op != SLAY_OP_BIDIR_BWD)
+        op != SLAY_OP_BIDIR_BWD && op != SLAY_OP_LINEAR_ATTN)
         return SIZE_MAX;
+    if (op == SLAY_OP_LINEAR_ATTN) {   // the contraction alone: F = R * m features given
+        if (static_cast<int64_t>(B) * H * L == 0) return 0;
+        return kWsHeader + simt_ws_linear(B, H, L, R * m);
+    }
     if (static_cast<int64_t>(B) * H * L == 0) return 0;
     return attn_ws(op, dt, B, H, L, Dv, R, m);
 }

@@ -32,6 +32,18 @@ struct Params {
     float c[kMaxR];
 };
 
+// Device view of a sketch variant's parameters (slay_phi_kind): omega^T, anchors^T and, for
+// the signed kind, the second anchors^T, each [H][D][F] (H heads for the per-head kind, else
+// 1); phi_f = exp2(a2[r] u + b2[r]) times the anchor factor of the kind.
+struct VarParams {
+    const float* omT;
+    const float* anT;
+    const float* anbT;
+    int F, m, R, H, kind;
+    float a2[kMaxR];
+    float b2[kMaxR];
+};
+
 // ---- per-launch timing (slay_trace.cpp) ----
 // Brackets the kernel launched inside its scope with CUDA events while tracing is on.
 class TraceScope {
@@ -53,6 +65,9 @@ bool gauss_laguerre(int R, double* t, double* w);
 // omega, anchors: [F*D] float, s, wt: [R] double.  false on failure.
 bool draw_sketch(int D, int R, int m, uint64_t seed, double eps, float* omega,
                  float* anchors, double* s, double* wt);
+// A sketch variant (kind 0-4, see slay_phi_kind) for one head; anchors_b only for kind 2.
+bool draw_sketch_kind(int D, int R, int m, uint64_t seed, double eps, int kind, int head,
+                      float* omega, float* anchors, float* anchors_b, double* s, double* wt);
 
 // ---- argument checks and workspace sizing shared by the entry points (slay_api.cu) ----
 bool eps_ok(float eps);
@@ -94,6 +109,13 @@ cudaError_t simt_attn_bidir_bwd(const void* q, const void* k, const void* v,
 cudaError_t simt_feature_map_bwd(const void* x, const void* dphi, float* dx, int64_t n,
                                  slay_dtype x_dt, slay_dtype dphi_dt, const Params& P,
                                  cudaStream_t st);
+cudaError_t simt_feature_map_kind(const void* x, void* phi, int64_t n, int64_t Lh,
+                                  slay_dtype in_dt, slay_dtype out_dt, const VarParams& P,
+                                  cudaStream_t st);
+size_t simt_ws_linear(int B, int H, int L, int F);
+cudaError_t simt_linear_attn(const void* phq, const void* phk, const void* v, void* out,
+                             float* den, int B, int H, int L, int F, slay_dtype dt, float eps,
+                             bool causal, void* ws, cudaStream_t st);
 cudaError_t simt_decode_step(const void* q, const void* k, const void* v, float* S, float* z,
                              void* out, int N, slay_dtype dt, const Params& P, float eps,
                              cudaStream_t st);

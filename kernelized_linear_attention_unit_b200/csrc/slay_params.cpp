@@ -11,7 +11,9 @@
 // (diagonal 2k+1, off-diagonal k), isolated by Sturm-sequence bisection, and the
 // weights come from the Christoffel function w = 1 / sum_k L_k(t)^2 (the Laguerre
 // polynomials are orthonormal for e^{-t}).
+#include <algorithm>
 #include <cmath>
+#include <vector>
 #include <cstdint>
 
 #include "slay_internal.h"
@@ -79,11 +81,11 @@ bool gauss_laguerre(int R, double* t, double* w)
     return true;
 }
 
-// Standard normal from one Philox block: counter (idx, tag, 0, 0), Box-Muller on the
+// Standard normal from one Philox block: counter (idx, tag, head, 0), Box-Muller on the
 // first two words, each mapped to (0,1) as (word + 1/2) * 2^-32.
-static double philox_normal(uint64_t seed, uint32_t idx, uint32_t tag)
+static double philox_normal(uint64_t seed, uint32_t idx, uint32_t tag, uint32_t head = 0)
 {
-    const uint32_t ctr[4] = {idx, tag, 0u, 0u};
+    const uint32_t ctr[4] = {idx, tag, head, 0u};
     const uint32_t key[2] = {static_cast<uint32_t>(seed & 0xffffffffu),
                              static_cast<uint32_t>(seed >> 32)};
     uint32_t o[4];
@@ -111,6 +113,62 @@ bool draw_sketch(int D, int R, int m, uint64_t seed, double eps, float* omega,
             if (omega) omega[f * D + d] = static_cast<float>(philox_normal(seed, idx, 0u));
             if (anchors) anchors[f * D + d] = static_cast<float>(philox_normal(seed, idx, 1u) / rs);
         }
+    return true;
+}
+
+bool draw_sketch_kind(int D, int R, int m, uint64_t seed, double eps, int kind, int head,
+                      float* omega, float* anchors, float* anchors_b, double* s, double* wt)
+{
+    if (kind < 0 || kind > 4 || head < 0 || D <= 0) return false;
+    double t[kMaxR], w[kMaxR];
+    if (!gauss_laguerre(R, t, w)) return false;
+    for (int r = 0; r < R; ++r) {
+        if (s) s[r] = t[r] / (2.0 + eps);
+        if (wt) wt[r] = w[r] / (2.0 + eps);
+    }
+    const int64_t F = static_cast<int64_t>(R) * m;
+    const uint32_t h = kind == 3 ? static_cast<uint32_t>(head) : 0u;
+    const double rs = std::sqrt(static_cast<double>(D));
+    std::vector<double> g(static_cast<size_t>(F) * D);
+    for (int64_t f = 0; f < F; ++f)
+        for (int d = 0; d < D; ++d) {
+            const uint32_t idx = static_cast<uint32_t>(f * D + d);
+            g[f * D + d] = philox_normal(seed, idx, 0u, h);
+            if (anchors) anchors[f * D + d] = static_cast<float>(philox_normal(seed, idx, 1u, h) / rs);
+            if (anchors_b && kind == 2)
+                anchors_b[f * D + d] = static_cast<float>(philox_normal(seed, idx, 2u, h) / rs);
+        }
+    if (kind == 1 || kind == 4) {
+        // Blocks of D consecutive rows of a node made orthonormal by modified Gram-Schmidt
+        // (each row is reduced against the finished ones one at a time), then each row
+        // scaled back to the length of its own Gaussian draw.
+        std::vector<double> len(static_cast<size_t>(D));
+        for (int r = 0; r < R; ++r)
+            for (int b0 = 0; b0 < m; b0 += D) {
+                const int nb = std::min(D, m - b0);
+                double* blk = g.data() + (static_cast<int64_t>(r) * m + b0) * D;
+                for (int j = 0; j < nb; ++j) {
+                    double* row = blk + static_cast<int64_t>(j) * D;
+                    double l2 = 0.0;
+                    for (int d = 0; d < D; ++d) l2 += row[d] * row[d];
+                    len[j] = std::sqrt(l2);
+                    for (int i = 0; i < j; ++i) {
+                        const double* e = blk + static_cast<int64_t>(i) * D;
+                        double c = 0.0;
+                        for (int d = 0; d < D; ++d) c += row[d] * e[d];
+                        for (int d = 0; d < D; ++d) row[d] -= c * e[d];
+                    }
+                    double n2 = 0.0;
+                    for (int d = 0; d < D; ++d) n2 += row[d] * row[d];
+                    const double inv = 1.0 / std::sqrt(n2);
+                    for (int d = 0; d < D; ++d) row[d] *= inv;
+                }
+                for (int j = 0; j < nb; ++j)
+                    for (int d = 0; d < D; ++d) blk[static_cast<int64_t>(j) * D + d] *= len[j];
+            }
+    }
+    if (omega)
+        for (int64_t i = 0; i < F * D; ++i) omega[i] = static_cast<float>(g[i]);
     return true;
 }
 

@@ -118,7 +118,92 @@ __global__ void __launch_bounds__(NT) k_feature_map(const Tin* __restrict__ x,
     }
 }
 
-// ------------------------------------------------------------- chunk states
+// --------------------------------------------------- feature map, sketch variants
+// The CUDA-core feature map for a sketch variant (slay_phi_kind): grid (ceil(Lh/64),
+// ceil(F/64), n/Lh) over rows grouped Lh to a sequence; sequence z uses head z % H's
+// parameters (heads are H = 1 except for the per-head kind).  kSigned: the polynomial factor
+// (a.x^)(b.x^) with the second anchor set; kPerformer: phi = exp2(a2 u + b2) with no anchor
+// (the node constants then hold log2 e and -(log2 e + log2 F)/2).
+struct FmKindSmem {
+    float xs[C][65];
+    float wo[C][C + 1];
+    float wa[C][C + 1];
+    float wb[C][C + 1];
+    float inv[C];
+};
+
+template <typename Tin, typename Tout, bool kSigned, bool kPerformer>
+__global__ void __launch_bounds__(NT) k_feature_map_kind(const Tin* __restrict__ x,
+                                                         Tout* __restrict__ phi, int64_t Lh,
+                                                         VarParams P)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    FmKindSmem& sm = *reinterpret_cast<FmKindSmem*>(smem_raw);
+    const int tid = threadIdx.x;
+    const int64_t seq = blockIdx.z;
+    const int head = static_cast<int>(seq % P.H);
+    const int64_t r0 = static_cast<int64_t>(blockIdx.x) * C;   // row within the sequence
+    const int64_t base = seq * Lh;                               // first row of the sequence
+    const int f0 = blockIdx.y * C;
+    const int F = P.F;
+    const size_t hoff = static_cast<size_t>(head) * kD * F;
+    const float* omT = P.omT + hoff;
+    const float* anT = P.anT + hoff;
+    const float* anbT = kSigned ? P.anbT + hoff : nullptr;
+    for (int idx = tid; idx < C * C; idx += NT) {
+        const int r = idx >> 6, d = idx & 63;
+        sm.xs[r][d] = (r0 + r < Lh) ? ld(x + (base + r0 + r) * kD + d) : 0.0f;
+        const int f = f0 + (idx & 63), dd = idx >> 6;
+        sm.wo[dd][idx & 63] = (f < F) ? omT[dd * F + f] : 0.0f;
+        if (!kPerformer) sm.wa[dd][idx & 63] = (f < F) ? anT[dd * F + f] : 0.0f;
+        if (kSigned) sm.wb[dd][idx & 63] = (f < F) ? anbT[dd * F + f] : 0.0f;
+    }
+    __syncthreads();
+    tile_inv_norms(sm.xs, sm.inv);
+    __syncthreads();
+    const int ty = tid >> 4, tx = tid & 15;
+    float au[4][4] = {}, ap[4][4] = {}, bp[4][4] = {};
+#pragma unroll 4
+    for (int d = 0; d < C; ++d) {
+        float xv[4], o[4], a[4], b[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xv[i] = sm.xs[ty + 16 * i][d];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            o[j] = sm.wo[d][tx + 16 * j];
+            a[j] = kPerformer ? 0.0f : sm.wa[d][tx + 16 * j];
+            b[j] = kSigned ? sm.wb[d][tx + 16 * j] : 0.0f;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                au[i][j] = fmaf(xv[i], o[j], au[i][j]);
+                if (!kPerformer) ap[i][j] = fmaf(xv[i], a[j], ap[i][j]);
+                if (kSigned) bp[i][j] = fmaf(xv[i], b[j], bp[i][j]);
+            }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = ty + 16 * i;
+        if (r0 + r >= Lh) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int f = f0 + tx + 16 * j;
+            if (f >= F) continue;
+            const int node = f / P.m;
+            const float u = au[i][j] * sm.inv[r];
+            float val = exp2f(fmaf(P.a2[node], u, P.b2[node]));
+            if (!kPerformer) {
+                const float p = ap[i][j] * sm.inv[r];
+                val *= kSigned ? p * (bp[i][j] * sm.inv[r]) : p * p;
+            }
+            st(phi + (base + r0 + r) * F + f, val);
+        }
+    }
+}
+
+// ------------------------------------------------------------- chunk states// ------------------------------------------------------------- chunk states
 // grid (ceil(F/64), NC, BH).  st[bh][c][f][e] = sum_{t in chunk c} phi[t][f] * Y[t][e],
 // e < 64 from Y, e = 64 the "ones" column (Y1 == nullptr) or Y's own column 64.
 // Y is either v (type T, 64 columns) or an fp32 [L][65] array.
@@ -960,6 +1045,94 @@ cudaError_t simt_attn_fwd(const void* q, const void* k, const void* v, void* out
 {
     if (dt == SLAY_F32) return attn_fwd_t<float>(q, k, v, out, den, B, H, L, P, eps, causal, ws, st);
     return attn_fwd_t<__nv_bfloat16>(q, k, v, out, den, B, H, L, P, eps, causal, ws, st);
+}
+
+template <typename Tin, typename Tout, bool kSigned, bool kPerformer>
+static cudaError_t fm_kind_launch(const void* x, void* phi, int64_t n, int64_t Lh,
+                                  const VarParams& P, cudaStream_t st)
+{
+    auto kern = k_feature_map_kind<Tin, Tout, kSigned, kPerformer>;
+    const size_t smem = sizeof(FmKindSmem);
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    const dim3 grid(static_cast<unsigned>((Lh + C - 1) / C), (P.F + C - 1) / C,
+                    static_cast<unsigned>(n / Lh));
+    TraceScope trace_("simt_feature_map_kind", st);
+    kern<<<grid, NT, smem, st>>>(cp<Tin>(x), mp<Tout>(phi), Lh, P);
+    return cudaGetLastError();
+}
+
+template <typename Tin, typename Tout>
+static cudaError_t fm_kind_t(const void* x, void* phi, int64_t n, int64_t Lh, const VarParams& P,
+                             cudaStream_t st)
+{
+    if (P.kind == 2) return fm_kind_launch<Tin, Tout, true, false>(x, phi, n, Lh, P, st);
+    if (P.kind == 4) return fm_kind_launch<Tin, Tout, false, true>(x, phi, n, Lh, P, st);
+    return fm_kind_launch<Tin, Tout, false, false>(x, phi, n, Lh, P, st);
+}
+
+cudaError_t simt_feature_map_kind(const void* x, void* phi, int64_t n, int64_t Lh,
+                                  slay_dtype in_dt, slay_dtype out_dt, const VarParams& P,
+                                  cudaStream_t st)
+{
+    if (in_dt == SLAY_F32 && out_dt == SLAY_F32) return fm_kind_t<float, float>(x, phi, n, Lh, P, st);
+    if (in_dt == SLAY_BF16 && out_dt == SLAY_BF16)
+        return fm_kind_t<__nv_bfloat16, __nv_bfloat16>(x, phi, n, Lh, P, st);
+    return fm_kind_t<__nv_bfloat16, float>(x, phi, n, Lh, P, st);
+}
+
+// The contraction on given features phi(q), phi(k) [BH][L][F] (in the mode's dtype): chunk
+// states, the scan over chunks (causal prefix or whole-sequence total) and the chunk output.
+size_t simt_ws_linear(int B, int H, int L, int F)
+{
+    const size_t BH = static_cast<size_t>(B) * H;
+    return align256(BH * nchunks(L) * static_cast<size_t>(F) * E * sizeof(float)) +
+           align256(BH * static_cast<size_t>(F) * E * sizeof(float));
+}
+
+template <typename T>
+static cudaError_t linear_attn_t(const void* phq_, const void* phk_, const void* v, void* out,
+                                 float* den, int B, int H, int L, int F, float eps, bool causal,
+                                 void* ws, cudaStream_t st)
+{
+    const int BH = B * H, NC = nchunks(L);
+    const T* phq = cp<T>(phq_);
+    const T* phk = cp<T>(phk_);
+    char* w = static_cast<char*>(ws);
+    float* stt = reinterpret_cast<float*>(w);
+    float* tot = reinterpret_cast<float*>(w + align256(static_cast<size_t>(BH) * NC * F * E * sizeof(float)));
+    cudaError_t err;
+    {
+        TraceScope trace_("simt_chunk_state", st);
+        k_chunk_state<T, T><<<dim3((F + C - 1) / C, NC, BH), NT, 0, st>>>(phk, cp<T>(v), kD, stt, L, F);
+    }
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    const int64_t nth = static_cast<int64_t>(BH) * F * E;
+    {
+        TraceScope trace_("simt_scan", st);
+        k_scan<<<static_cast<unsigned>((nth + 255) / 256), 256, 0, st>>>(stt, tot, BH, NC, F * E,
+                                                                         causal ? 0 : 2);
+    }
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    const size_t smem = sizeof(OutSmem);
+    if ((err = cudaFuncSetAttribute(k_chunk_out<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(smem))) != cudaSuccess)
+        return err;
+    {
+        TraceScope trace_("simt_chunk_out", st);
+        k_chunk_out<T><<<dim3(NC, BH), NT, smem, st>>>(phq, phk, cp<T>(v), causal ? stt : tot,
+                                                       mp<T>(out), den, L, F, eps, causal ? 1 : 0);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t simt_linear_attn(const void* phq, const void* phk, const void* v, void* out,
+                             float* den, int B, int H, int L, int F, slay_dtype dt, float eps,
+                             bool causal, void* ws, cudaStream_t st)
+{
+    if (dt == SLAY_F32) return linear_attn_t<float>(phq, phk, v, out, den, B, H, L, F, eps, causal, ws, st);
+    return linear_attn_t<__nv_bfloat16>(phq, phk, v, out, den, B, H, L, F, eps, causal, ws, st);
 }
 
 template <typename T>

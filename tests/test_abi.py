@@ -142,3 +142,41 @@ def test_noalloc_sizes_the_path_that_runs():
                  1234, 1e-6, None) == bd.SLAY_ERR_UNSUPPORTED
     assert f(_fake(), _fake(), _fake(), _fake(), None, 1, 16, 16384, 64, 64, bd.SLAY_F32, 4, 64,
              1234, 1e-6, None) == bd.SLAY_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("kind", [0, 1, 2, 3, 4])
+def test_variant_sketch_params_match_oracle(kind):
+    # the library's draws (its own Philox, modified Gram-Schmidt) against the oracle's (its own
+    # Philox, classical Gram-Schmidt): bit for bit where nothing is orthogonalised, to fp32
+    # rounding where the two Gram-Schmidt orders round differently
+    D, R, m, seed = 16, 3, 20, 91
+    eps = float(np.float32(1e-6))
+    for head in ((0, 2) if kind == 3 else (0,)):
+        om, an, anb, s, w = bd.slay_sketch_params_ex(D, R, m, seed, eps, kind, head)
+        P = O.sketch_params_kind(D, R, m, seed, eps, kind, head)
+        assert np.array_equal(an.astype(np.float64), P.anchors)
+        if kind == 2:
+            assert np.array_equal(anb.astype(np.float64), P.anchors_b)
+        if kind in (1, 4):
+            np.testing.assert_allclose(om.astype(np.float64), P.omega, rtol=2e-6, atol=2e-6)
+        else:
+            assert np.array_equal(om.astype(np.float64), P.omega)
+        np.testing.assert_allclose(s, P.s, rtol=1e-13)
+        np.testing.assert_allclose(w, P.wt, rtol=1e-11)
+
+
+def test_variant_and_contraction_argument_errors():
+    L = bd.lib()
+    fx = L.slay_feature_map_ex
+    assert fx(_fake(), _fake(), 10, 64, bd.SLAY_F32, bd.SLAY_F32, 4, 64, 1, 1e-6, 9, 1, 0, None) \
+        == bd.SLAY_ERR_INVALID_ARG                                          # unknown kind
+    assert fx(_fake(), _fake(), 10, 64, bd.SLAY_F32, bd.SLAY_F32, 4, 64, 1, 1e-6,
+              bd.PHI_PER_HEAD, 2, 3, None) == bd.SLAY_ERR_INVALID_ARG        # 10 % 3 != 0
+    assert fx(None, None, 0, 64, bd.SLAY_F32, bd.SLAY_F32, 4, 64, 1, 1e-6, bd.PHI_PERFORMER, 1,
+              0, None) == bd.SLAY_OK
+    la = L.slay_linear_attn_fwd
+    assert la(_fake(), _fake(), _fake(), _fake(), None, 1, 1, 64, 2048, 64, bd.SLAY_F32, 1e-6, 1,
+              _fake(0x20000), 1 << 40, None) == bd.SLAY_ERR_UNSUPPORTED     # F > 1024
+    assert la(_fake(), _fake(), _fake(), _fake(), None, 1, 1, 64, 256, 64, bd.SLAY_F32, 1e-6, 1,
+              None, 0, None) == bd.SLAY_ERR_INVALID_ARG                     # no workspace
+    assert bd.slay_workspace_bytes(bd.OP_LINEAR_ATTN, bd.SLAY_F32, 1, 2, 100, 64, 64, 1, 256) > 0

@@ -543,3 +543,73 @@ def test_feature_map_bwd(dt_x, dt_g, R, m, n, scaled):
     check(name, got[keep] * nx[keep, None], want[keep] * nx[keep, None], tol)
     check(name + " guarded row", got[7][None], want[7][None], tol)
     assert np.isfinite(got).all()
+
+
+# ------------------------------------------ feature-map variants and the contraction
+
+KINDS = {"orthogonal": 1, "signed": 2, "per_head": 3, "performer": 4}
+
+
+@pytest.mark.parametrize("scaled", [False, True])
+@pytest.mark.parametrize("kind", sorted(KINDS))
+@pytest.mark.parametrize("dt_in,dt_out,R,m,B,H,L", [("f32", "f32", 2, 16, 1, 3, 100),
+                                                   ("bf16", "bf16", 4, 64, 2, 3, 130),
+                                                   ("bf16", "f32", 8, 64, 1, 2, 70)])
+def test_feature_map_variants(kind, dt_in, dt_out, R, m, B, H, L, scaled):
+    w = small(dt_in, R, m, L, B=B, H=H)
+    q, _, _ = qkv(w, scaled)
+    kd = KINDS[kind]
+    F = w.F
+    eps = _eps(w)
+    if kd == 3:   # per head: the rows of head h use head h's draw
+        want = np.concatenate([O.feature_map_kind(q[:, h:h + 1], O.sketch_params_kind(
+            64, R, m, w.sketch_seed, eps, kd, h)) for h in range(H)], axis=1)
+    else:
+        want = O.feature_map_kind(q, O.sketch_params_kind(64, R, m, w.sketch_seed, eps, kd))
+    xt = dev(q, dt_in)
+    phi = torch.empty((B, H, L, F), device="cuda", dtype=TDT[dt_out])
+    bd.slay_feature_map_ex(xt, phi, R, m, w.sketch_seed, eps, kd, heads=H, rows_per_head=L)
+    torch.cuda.synchronize()
+    tol = TOL["bf16"] if "bf16" in (dt_in, dt_out) else TOL["f32"]
+    check("phi %s %s->%s R%d m%d%s" % (kind, dt_in, dt_out, R, m, " scaled" if scaled else ""),
+          host(phi), want, tol)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("dt,F,L", [("f32", 32, 100), ("f32", 256, 129), ("bf16", 256, 300),
+                                    ("bf16", 512, 257), ("bf16", 384, 1)])
+def test_linear_attn_on_given_features(dt, F, L, causal):
+    # the oracle's features (rounded to the mode's dtype) feed both sides
+    w = small(dt, 4, F // 4, L, B=2, H=2)
+    q, k, v = W.gen_qkv(w)
+    P = O.sketch_params(64, 4, F // 4, w.sketch_seed, _eps(w))
+    pq = W.to_dtype(O.feature_map(q, P), dt)
+    pk = W.to_dtype(O.feature_map(k, P), dt)
+    want, wden = O.attn_from_phi(pq, pk, v, P.eps, causal)
+    out = torch.empty(v.shape, device="cuda", dtype=TDT[dt])
+    den = torch.empty(v.shape[:-1], device="cuda", dtype=torch.float32)
+    ws = bd.slay_linear_attn_fwd(dev(pq, dt), dev(pk, dt), dev(v, dt), out, den, _eps(w), causal)
+    bd.slay_kernel_status(ws)
+    torch.cuda.synchronize()
+    _check_fwd("linear attn %s F%d L%d %s" % (dt, F, L, "causal" if causal else "bidir"),
+               host(out), host(den), want, wden, TOL[dt])
+
+
+@pytest.mark.parametrize("kind", ["performer", "orthogonal"])
+def test_variant_attention_composed(kind):
+    # a variant's map for q and k, then the contraction, against the oracle's composition
+    w = small("bf16", 4, 64, 200, B=1, H=2, seed=24)
+    q, k, v = W.gen_qkv(w)
+    kd = KINDS[kind]
+    P = O.sketch_params_kind(64, 4, 64, w.sketch_seed, _eps(w), kd)
+    want, wden = O.attn_from_phi(O.feature_map_kind(q, P), O.feature_map_kind(k, P), v, P.eps,
+                                 True)
+    pq = torch.empty((1, 2, 200, 256), device="cuda", dtype=torch.bfloat16)
+    pk = torch.empty_like(pq)
+    bd.slay_feature_map_ex(dev(q, "bf16"), pq, 4, 64, w.sketch_seed, _eps(w), kd)
+    bd.slay_feature_map_ex(dev(k, "bf16"), pk, 4, 64, w.sketch_seed, _eps(w), kd)
+    out = torch.empty((1, 2, 200, 64), device="cuda", dtype=torch.bfloat16)
+    den = torch.empty((1, 2, 200), device="cuda", dtype=torch.float32)
+    bd.slay_linear_attn_fwd(pq, pk, dev(v, "bf16"), out, den, _eps(w), True)
+    torch.cuda.synchronize()
+    _check_fwd("composed %s causal" % kind, host(out), host(den), want, wden, TOL["bf16"])
