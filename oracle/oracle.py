@@ -75,6 +75,9 @@ def lib():
         L.orc_attn_from_phi.argtypes = [dp, dp, dp] + [C.c_int] * 5 + [C.c_double, C.c_int,
                                                                       dp, dp]
         L.orc_attn_from_phi.restype = None
+        L.orc_attn_causal_state.argtypes = [dp, dp, dp, dp, dp] + shp + par + [C.c_double,
+                                                                             dp, dp, dp, dp]
+        L.orc_attn_causal_state.restype = None
         L.orc_num_threads.argtypes = []
         L.orc_num_threads.restype = C.c_int
         _lib = L
@@ -335,10 +338,28 @@ def attn_from_phi(pq, pk, v, eps, causal):
     return out, den
 
 
+def attn_causal_state(q, k, v, P: Params, S0=None, z0=None):
+    """Causal forward continued from state (S0 [B,H,F,Dv], z0 [B,H,F]; None = zero);
+    returns (out, den, S1, z1) with the state after the last token."""
+    q, k, v = _d(q), _d(k), _d(v)
+    B, H, L, D, Dv = _shape4(q, v)
+    F = P.F
+    out = np.zeros((B, H, L, Dv))
+    den = np.zeros((B, H, L))
+    S1 = np.zeros((B, H, F, Dv))
+    z1 = np.zeros((B, H, F))
+    s0 = None if S0 is None else _d(S0)
+    zz0 = None if z0 is None else _d(z0)
+    lib().orc_attn_causal_state(_p(q), _p(k), _p(v), None if s0 is None else _p(s0),
+                                None if zz0 is None else _p(zz0), B, H, L, D, Dv, P.R, P.m,
+                                *P.args(), P.eps, _p(out), _p(den), _p(S1), _p(z1))
+    return out, den, S1, z1
+
+
 __all__ = ["lib", "num_threads", "philox4x32_10", "gauss_laguerre", "Params", "sketch_params",
            "yat_kernel", "quad_kernel", "feature_map", "attn_quadratic", "attn_quadratic_rows",
            "attn_recurrent", "decode_step", "attn_causal_bwd", "attn_causal_bwd_rows",
            "attn_causal_bwd_given", "attn_causal_bwd_given_rows", "feature_map_bwd",
            "attn_bidir_bwd", "attn_bidir_bwd_given", "KindParams", "sketch_params_kind",
            "feature_map_kind", "attn_from_phi", "PHI_ANCHOR", "PHI_ORTHOGONAL", "PHI_SIGNED",
-           "PHI_PER_HEAD", "PHI_PERFORMER"]
+           "PHI_PER_HEAD", "PHI_PERFORMER", "attn_causal_state"]

@@ -905,6 +905,49 @@ void orc_attn_from_phi(const double* pq, const double* pk, const double* v,
     }
 }
 
+/* The causal recurrence continued from a given state (review, "Proposed method", step 6:
+ * the prefix state carries everything the earlier tokens contribute; abstract: O(L) time and
+ * memory).  Per (b,h): S = S0, z = z0; for each token i: S += phi(k_i) v_i^T, z += phi(k_i),
+ * out_i = phi(q_i)^T S / (phi(q_i)^T z + eps); S1, z1 = the state after the last token.
+ * S0, z0: [B,H,F,Dv], [B,H,F] (NULL = zero); S1, z1 may be NULL. */
+void orc_attn_causal_state(const double* q, const double* k, const double* v,
+                           const double* S0, const double* z0,
+                           int B, int H, int L, int D, int Dv, int R, int m,
+                           const double* omega, const double* anchors,
+                           const double* s, const double* wt, double eps,
+                           double* out, double* den, double* S1, double* z1)
+{
+    const int64_t F = (int64_t)R * m;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bh = 0; bh < B * H; ++bh) {
+        double* pq = phi_slice(q + (int64_t)bh * L * D, L, D, R, m, omega, anchors, s, wt);
+        double* pk = phi_slice(k + (int64_t)bh * L * D, L, D, R, m, omega, anchors, s, wt);
+        const double* vs = v + (int64_t)bh * L * Dv;
+        double* S = (double*)calloc((size_t)F * (size_t)Dv, sizeof(double));
+        double* z = (double*)calloc((size_t)F, sizeof(double));
+        if (S0) for (int64_t t = 0; t < F * Dv; ++t) S[t] = S0[(int64_t)bh * F * Dv + t];
+        if (z0) for (int64_t f = 0; f < F; ++f) z[f] = z0[(int64_t)bh * F + f];
+        for (int i = 0; i < L; ++i) {
+            for (int64_t f = 0; f < F; ++f) {
+                double a = pk[(int64_t)i * F + f];
+                z[f] += a;
+                for (int e = 0; e < Dv; ++e) S[f * Dv + e] += a * vs[(int64_t)i * Dv + e];
+            }
+            const double* p = pq + (int64_t)i * F;
+            double d = dot(p, z, F);
+            for (int e = 0; e < Dv; ++e) {
+                double acc = 0.0;
+                for (int64_t f = 0; f < F; ++f) acc += p[f] * S[f * Dv + e];
+                out[((int64_t)bh * L + i) * Dv + e] = acc / (d + eps);
+            }
+            if (den) den[(int64_t)bh * L + i] = d;
+        }
+        if (S1) for (int64_t t = 0; t < F * Dv; ++t) S1[(int64_t)bh * F * Dv + t] = S[t];
+        if (z1) for (int64_t f = 0; f < F; ++f) z1[(int64_t)bh * F + f] = z[f];
+        free(pq); free(pk); free(S); free(z);
+    }
+}
+
 int orc_num_threads(void)
 {
 #ifdef _OPENMP

@@ -157,6 +157,12 @@ void orc_feature_map_kind(const double* x, int64_t n, int D, int R, int m,
 void orc_attn_from_phi(const double* pq, const double* pk, const double* v,
                        int B, int H, int L, int F, int Dv, double eps, int causal,
                        double* out, double* den);
+void orc_attn_causal_state(const double* q, const double* k, const double* v,
+                           const double* S0, const double* z0,
+                           int B, int H, int L, int D, int Dv, int R, int m,
+                           const double* omega, const double* anchors,
+                           const double* s, const double* wt, double eps,
+                           double* out, double* den, double* S1, double* z1);
 int orc_num_threads(void);
 
 #ifdef __cplusplus

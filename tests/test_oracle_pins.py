@@ -571,3 +571,49 @@ def test_contraction_on_given_features_is_the_quadratic_form(causal):
     got, gden = O.attn_from_phi(O.feature_map(q, P), O.feature_map(k, P), v, P.eps, causal)
     np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-14)
     np.testing.assert_allclose(gden, wden, rtol=1e-12)
+
+
+# ------------------------------------------------------- state continuation
+
+def test_causal_state_from_zero_is_the_causal_form():
+    q, k, v = _small(50, B=1, H=2, L=23, D=8, Dv=4)
+    P = O.sketch_params(D=8, R=2, m=5, seed=9, eps=1e-6)
+    want, wden = O.attn_quadratic(q, k, v, P, True)
+    out, den, S1, z1 = O.attn_causal_state(q, k, v, P)
+    np.testing.assert_allclose(out, want, rtol=1e-11, atol=1e-14)
+    np.testing.assert_allclose(den, wden, rtol=1e-11)
+    # the final state is the total sum phi(k)[v, 1]^T
+    pk = O.feature_map(k, P)
+    np.testing.assert_allclose(S1, np.einsum("bhlf,bhle->bhfe", pk, v), rtol=1e-11, atol=1e-15)
+    np.testing.assert_allclose(z1, pk.sum(axis=2), rtol=1e-11)
+
+
+@pytest.mark.parametrize("cuts", [(9,), (4, 11, 17), (1, 2, 22)])
+def test_causal_state_chains_over_a_split_sequence(cuts):
+    # sequence parallelism: each part continues from the state the earlier parts end in
+    q, k, v = _small(51, B=2, H=1, L=23, D=8, Dv=4)
+    P = O.sketch_params(D=8, R=2, m=5, seed=9, eps=1e-6)
+    want, wden = O.attn_quadratic(q, k, v, P, True)
+    S, z, outs, dens = None, None, [], []
+    bounds = (0,) + tuple(cuts) + (23,)
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        o, d, S, z = O.attn_causal_state(q[:, :, a:b], k[:, :, a:b], v[:, :, a:b], P, S, z)
+        outs.append(o)
+        dens.append(d)
+    np.testing.assert_allclose(np.concatenate(outs, axis=2), want, rtol=1e-11, atol=1e-14)
+    np.testing.assert_allclose(np.concatenate(dens, axis=2), wden, rtol=1e-11)
+
+
+def test_causal_state_is_the_decode_recurrence():
+    q, k, v = _small(52, B=1, H=2, L=6, D=8, Dv=4)
+    P = O.sketch_params(D=8, R=2, m=5, seed=9, eps=1e-6)
+    rng = np.random.default_rng(53)
+    S0 = rng.standard_normal((1, 2, P.F, 4)) * 1e-3
+    z0 = rng.random((1, 2, P.F)) * 1e-3
+    out, den, S1, z1 = O.attn_causal_state(q, k, v, P, S0, z0)
+    S, z = S0.copy(), z0.copy()
+    for i in range(6):
+        o, S, z = O.decode_step(q[:, :, i], k[:, :, i], v[:, :, i], S, z, P)
+        np.testing.assert_allclose(out[:, :, i], o, rtol=1e-11, atol=1e-14)
+    np.testing.assert_allclose(S1, S, rtol=1e-12, atol=1e-16)
+    np.testing.assert_allclose(z1, z, rtol=1e-12)
