@@ -3,7 +3,10 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload causal_16k|causal_2k|bidir_vision|fwd_8k|bwd_8k|bidir_bwd|decode|
-                                feature_map|feature_map_bwd|matched_budget]
+                                feature_map|feature_map_bwd|matched_budget|seqpar_16k]
+
+seqpar_16k splits the headline sequence over the N ranks (strong scaling, one all-gather of
+the pieces' states per step); every other workload gives each rank its own batch (weak).
 
 With --gpus N > 1 outside torchrun, bench.py starts the N ranks itself (torch.distributed.run
 on 127.0.0.1); under torchrun, --gpus must equal WORLD_SIZE.
@@ -45,6 +48,7 @@ WORKLOADS = {
     "bidir_bwd": (W.BIDIR_VISION, "bidir_bwd"),
     "feature_map_bwd": (W.CAUSAL_16K, "feature_map_bwd"),
     "matched_budget": (W.CAUSAL_16K, "matched_budget"),
+    "seqpar_16k": (W.CAUSAL_16K, "seqpar"),
     "decode": (W.DECODE, "decode"),
     "feature_map": (W.CAUSAL_16K, "feature_map"),
 }
@@ -117,7 +121,7 @@ def kernel_work(name, w, op):
         return (th * (4 * D * F + 4 * F * Dv + (C_CHUNK + 1) * F) +
                 th * (C_CHUNK + 1) * Dv // nch +
                 (th * 4 * D * F if name == "tc_causal_out" else 0)), "flop", "tensor"
-    if name in ("tc_causal_state",):
+    if name in ("tc_causal_state", "tc_state_sums"):
         return th * (4 * D * F + 2 * F * Dv), "flop", "tensor"
     # stored-phi(k) form: the state kernel maps k (its own segment sums are not algorithmic
     # work), the output kernel does the rest of the causal forward
@@ -323,7 +327,7 @@ def run_reference(args, w, op):
 
 
 def config_of(w, op):
-    return {"workload": w.name if op not in ("bwd", "feature_map") else "%s_%s" % (w.name, op),
+    return {"workload": w.name if op in ("causal", "bidir", "decode") else "%s_%s" % (w.name, op),
             "B": w.B, "H": w.H, "L": w.L, "D": w.D, "Dv": w.Dv, "R": w.R, "m": w.m, "F": w.F,
             "op": op, "eps": w.eps, "sketch_seed": w.sketch_seed,
             "l2": "flushed between timed steps (256 MiB write outside the timed events)"}
@@ -379,8 +383,9 @@ def run_ours(args, w, op):
         h.copy_(t)
         return h
 
-    # inputs: each rank draws its own batch (data seed offset by rank)
-    wr = rank_workload(w, rank)
+    # inputs: each rank draws its own batch (data seed offset by rank); the sequence-parallel
+    # workload shares one sequence
+    wr = w if op == "seqpar" else rank_workload(w, rank)
     if op == "decode":
         qn, kn, vn, Sn, zn = W.gen_decode(wr)
         q, k, v = to_dev(qn), to_dev(kn), to_dev(vn)
@@ -403,6 +408,23 @@ def run_ours(args, w, op):
         def step():
             bd.slay_feature_map(x, out, w.R, w.m, w.sketch_seed, eps)
         units_per_step = w.B * w.L
+        unit = "tokens/s"
+    elif op == "seqpar":
+        from kernelized_linear_attention_unit_b200 import seqpar
+        # this rank's contiguous piece of the one long sequence (every rank draws the whole
+        # sequence from the same seed and keeps its piece)
+        qn, kn, vn = W.gen_qkv(w)
+        a, b = rank * w.L // world, (rank + 1) * w.L // world
+        q, k, v = (to_dev(np.ascontiguousarray(x[:, :, a:b])) for x in (qn, kn, vn))
+        out = torch.empty(v.shape, device=dev, dtype=tdt)
+        den = torch.empty(v.shape[:-1], device=dev, dtype=torch.float32)
+        host_in, dev_in = [pinned(x.cpu()) for x in (q, k, v)], [q, k, v]
+        ops = seqpar.LibraryOps(w.R, w.m, w.sketch_seed, eps)
+        scratch = {}
+
+        def step():
+            seqpar.causal_fwd_seqpar(q, k, v, out, den, w.F, ops, scratch=scratch)
+        units_per_step = w.B * (b - a)
         unit = "tokens/s"
     elif op == "feature_map_bwd":
         qn, kn, _ = W.gen_qkv(wr)
@@ -569,7 +591,8 @@ def run_ours(args, w, op):
         line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+                "scaling": "strong" if op == "seqpar" else "weak", "vs_baseline": None,
+                "dtype": w.dtype, "data": "synthetic",
                 "config": config_of(w, op),
                 "e2e": {"value": e2e, "unit": unit, "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},

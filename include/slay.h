@@ -71,7 +71,8 @@ typedef enum {
     SLAY_OP_CAUSAL_BWD = 3,
     SLAY_OP_DECODE = 4,
     SLAY_OP_BIDIR_BWD = 5,
-    SLAY_OP_LINEAR_ATTN = 6     /* slay_linear_attn_fwd: R * m = the number of features */
+    SLAY_OP_LINEAR_ATTN = 6,    /* slay_linear_attn_fwd: R * m = the number of features */
+    SLAY_OP_CAUSAL_STATE = 7    /* slay_causal_state */
 } slay_op;
 
 /* Feature-map variants (slay_feature_map_ex).  The pages leave the form of the anchor
@@ -112,6 +113,41 @@ slay_status slay_attn_causal_fwd(const void* q, const void* k, const void* v, vo
                                  float* den, int B, int H, int L, int D, int Dv,
                                  slay_dtype dt, int R, int m, uint64_t seed, float eps,
                                  void* workspace, size_t ws_bytes, void* stream);
+
+/* The causal forward continued from a state (review, "Proposed method", step 6: the
+ * prefix state S_i = S_0 + sum_{j<=i} phi(k_j) v_j^T, z_i likewise, carries all earlier
+ * tokens; abstract: O(L) time and memory).  With it a sequence can be processed in pieces --
+ * prefill after a cached prefix, or one piece per GPU (sequence parallelism: each rank
+ * takes the sum of the earlier ranks' slay_causal_state results, see slay_state_prefix).
+ * Arguments as slay_attn_causal_fwd (same workspace size), plus:
+ * S_in, z_in   : device [B,H,R*m,Dv] and [B,H,R*m] fp32, the state before the first token of
+ *                this piece, or both NULL for a zero state (then the call equals
+ *                slay_attn_causal_fwd);
+ * S_out, z_out : device, same shapes, written with the state after the last token, or both
+ *                NULL.  16-byte aligned.  They must not alias S_in, z_in. */
+slay_status slay_attn_causal_fwd_state(const void* q, const void* k, const void* v, void* out,
+                                       float* den, const float* S_in, const float* z_in,
+                                       float* S_out, float* z_out, int B, int H, int L, int D,
+                                       int Dv, slay_dtype dt, int R, int m, uint64_t seed,
+                                       float eps, void* workspace, size_t ws_bytes, void* stream);
+
+/* The causal state of a piece of a sequence without its outputs:
+ *   S_out = S_in + sum_j phi(k_j) v_j^T,  z_out = z_in + sum_j phi(k_j)
+ * over the L tokens of each (b,h) (S_in, z_in NULL: zero).  Layouts as
+ * slay_attn_causal_fwd_state; workspace slay_workspace_bytes(SLAY_OP_CAUSAL_STATE, ...).
+ * bf16 at tensor-core sizes: the state kernel of the causal forward over every segment
+ * (phi(k) and the sums on tensor cores), then the total; otherwise CUDA cores. */
+slay_status slay_causal_state(const void* k, const void* v, const float* S_in, const float* z_in,
+                              float* S_out, float* z_out, int B, int H, int L, int D, int Dv,
+                              slay_dtype dt, int R, int m, uint64_t seed, float eps,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+/* Exclusive prefix over ranks of all-gathered piece states (sequence parallelism):
+ *   S_in = sum_{r < rank} S_all[r],  z_in = sum_{r < rank} z_all[r]
+ * S_all: device [nranks][BH][F][Dv] fp32, z_all: [nranks][BH][F]; S_in [BH][F][Dv],
+ * z_in [BH][F] written (zero for rank 0).  F = R*m <= 1024, Dv == 64. */
+slay_status slay_state_prefix(const float* S_all, const float* z_all, int nranks, int rank,
+                              float* S_in, float* z_in, int BH, int F, int Dv, void* stream);
 
 /* Bidirectional SLAY attention forward: as above with S, z summed over all keys
  * (review, "Proposed method", step 6, non-causal form).  Same arguments; workspace

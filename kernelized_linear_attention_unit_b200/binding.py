@@ -18,7 +18,7 @@ SLAY_OK, SLAY_ERR_INVALID_ARG, SLAY_ERR_UNSUPPORTED, SLAY_ERR_CUDA, SLAY_ERR_TIM
     SLAY_ERR_NO_MEMORY = range(6)
 SLAY_F32, SLAY_BF16 = 0, 1
 OP_FEATURE_MAP, OP_CAUSAL_FWD, OP_BIDIR_FWD, OP_CAUSAL_BWD, OP_DECODE, OP_BIDIR_BWD, \
-    OP_LINEAR_ATTN = range(7)
+    OP_LINEAR_ATTN, OP_CAUSAL_STATE = range(8)
 PHI_ANCHOR, PHI_ORTHOGONAL, PHI_SIGNED, PHI_PER_HEAD, PHI_PERFORMER = range(5)
 
 EXPORTS = ["slay_feature_map", "slay_attn_causal_fwd", "slay_attn_bidir_fwd",
@@ -26,7 +26,8 @@ EXPORTS = ["slay_feature_map", "slay_attn_causal_fwd", "slay_attn_bidir_fwd",
            "slay_sketch_params", "slay_status_string", "slay_last_error", "slay_trace_enable",
            "slay_trace_read", "slay_attn_causal_fwd_noalloc", "slay_kernel_status",
            "slay_debug_expire_wait", "slay_attn_bidir_bwd", "slay_feature_map_bwd",
-           "slay_feature_map_ex", "slay_sketch_params_ex", "slay_linear_attn_fwd"]
+           "slay_feature_map_ex", "slay_sketch_params_ex", "slay_linear_attn_fwd",
+           "slay_attn_causal_fwd_state", "slay_causal_state", "slay_state_prefix"]
 
 
 class SlayError(RuntimeError):
@@ -67,6 +68,11 @@ def lib():
     L.slay_sketch_params_ex.argtypes = [i32, i32, i32, u64, f32, i32, i32, vp, vp, vp, vp, vp]
     L.slay_linear_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32,
                                        i32, vp, sz, vp]
+    L.slay_attn_causal_fwd_state.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32,
+                                             i32, i32, i32, i32, i32, u64, f32, vp, sz, vp]
+    L.slay_causal_state.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
+                                    u64, f32, vp, sz, vp]
+    L.slay_state_prefix.argtypes = [vp, vp, i32, i32, vp, vp, i32, i32, i32, vp]
     L.slay_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                    u64, f32, vp]
     L.slay_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32]
@@ -88,7 +94,8 @@ def lib():
     for name in ("slay_feature_map", "slay_attn_causal_fwd", "slay_attn_bidir_fwd",
                  "slay_attn_causal_bwd", "slay_decode_step", "slay_prepare",
                  "slay_attn_bidir_bwd", "slay_feature_map_bwd", "slay_feature_map_ex",
-                 "slay_sketch_params_ex", "slay_linear_attn_fwd",
+                 "slay_sketch_params_ex", "slay_linear_attn_fwd", "slay_attn_causal_fwd_state",
+                 "slay_causal_state", "slay_state_prefix",
                  "slay_attn_causal_fwd_noalloc",
                  "slay_sketch_params"):
         getattr(L, name).restype = i32
@@ -321,6 +328,71 @@ def slay_linear_attn_fwd(phq, phk, v, out, den, eps, causal, workspace=None, str
                                       L, F, Dv, dt, eps, 1 if causal else 0, _ptr(workspace),
                                       wbytes, _stream(stream)), "slay_linear_attn_fwd")
     return workspace
+
+
+def _state_ptrs(S, z, BH_shape, F, name):
+    if S is None and z is None:
+        return None, None
+    _check(S, name + " S", torch.float32, BH_shape + (F, 64))
+    _check(z, name + " z", torch.float32, BH_shape + (F,))
+    return _ptr(S), _ptr(z)
+
+
+def slay_attn_causal_fwd_state(q, k, v, out, den, R, m, seed, eps, S_in=None, z_in=None,
+                               S_out=None, z_out=None, workspace=None, stream=None):
+    """Causal forward from state (S_in, z_in) [B,H,F,64], [B,H,F] (None: zero), writing the
+    final state into S_out, z_out if given; returns the workspace it used."""
+    _check(q, "q")
+    B, H, L, D = q.shape
+    Dv = v.shape[-1]
+    _check(k, "k", q.dtype, (B, H, L, D))
+    _check(v, "v", q.dtype, (B, H, L, Dv))
+    _check(out, "out", q.dtype, (B, H, L, Dv))
+    if den is not None:
+        _check(den, "den", torch.float32, (B, H, L))
+    F = R * m
+    si, zi = _state_ptrs(S_in, z_in, (B, H), F, "state in")
+    so, zo = _state_ptrs(S_out, z_out, (B, H), F, "state out")
+    dt = _dt(q)
+    if workspace is None:
+        workspace = alloc_workspace(OP_CAUSAL_FWD, dt, B, H, L, D, Dv, R, m, q.device)
+    wbytes = workspace.numel() * workspace.element_size()
+    _raise(lib().slay_attn_causal_fwd_state(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(den), si, zi,
+                                            so, zo, B, H, L, D, Dv, dt, R, m, seed, eps,
+                                            _ptr(workspace), wbytes, _stream(stream)),
+           "slay_attn_causal_fwd_state")
+    return workspace
+
+
+def slay_causal_state(k, v, S_out, z_out, R, m, seed, eps, S_in=None, z_in=None, workspace=None,
+                      stream=None):
+    """S_out = S_in + sum phi(k) v^T, z_out = z_in + sum phi(k) over the tokens of k, v."""
+    _check(k, "k")
+    B, H, L, D = k.shape
+    Dv = v.shape[-1]
+    _check(v, "v", k.dtype, (B, H, L, Dv))
+    F = R * m
+    si, zi = _state_ptrs(S_in, z_in, (B, H), F, "state in")
+    so, zo = _state_ptrs(S_out, z_out, (B, H), F, "state out")
+    dt = _dt(k)
+    if workspace is None:
+        workspace = alloc_workspace(OP_CAUSAL_STATE, dt, B, H, L, D, Dv, R, m, k.device)
+    wbytes = workspace.numel() * workspace.element_size()
+    _raise(lib().slay_causal_state(_ptr(k), _ptr(v), si, zi, so, zo, B, H, L, D, Dv, dt, R, m,
+                                   seed, eps, _ptr(workspace), wbytes, _stream(stream)),
+           "slay_causal_state")
+    return workspace
+
+
+def slay_state_prefix(S_all, z_all, rank, S_in, z_in, stream=None):
+    """S_in = sum of S_all[r] for r < rank (S_all [N,B,H,F,64], z_all [N,B,H,F])."""
+    _check(S_all, "S_all", torch.float32)
+    N, B, H, F, Dv = S_all.shape
+    _check(z_all, "z_all", torch.float32, (N, B, H, F))
+    _check(S_in, "S_in", torch.float32, (B, H, F, Dv))
+    _check(z_in, "z_in", torch.float32, (B, H, F))
+    _raise(lib().slay_state_prefix(_ptr(S_all), _ptr(z_all), N, rank, _ptr(S_in), _ptr(z_in),
+                                   B * H, F, Dv, _stream(stream)), "slay_state_prefix")
 
 
 def slay_feature_map_bwd(x, dphi, dx, R, m, seed, eps, stream=None):

@@ -232,14 +232,19 @@ slay_status check_attn(const void* q, const void* k, const void* v, const void* 
 size_t attn_ws(slay_op op, slay_dtype dt, int B, int H, int L, int Dv, int R, int m)
 {
     const int F = R * m;
-    if (dt == SLAY_BF16 && tc_supported(op, B, H, L, R, m))
+    if (op == SLAY_OP_CAUSAL_STATE) {
+        if (dt == SLAY_BF16 && tc_supported(SLAY_OP_CAUSAL_FWD, B, H, L, R, m))
+            return tc_state_workspace_bytes(B, H, L, R, m);
+    } else if (dt == SLAY_BF16 && tc_supported(op, B, H, L, R, m)) {
         return tc_workspace_bytes(op, B, H, L, R, m);
+    }
     switch (op) {
         case SLAY_OP_CAUSAL_FWD: return kWsHeader + simt_ws_causal(B, H, L, Dv, F);
         case SLAY_OP_BIDIR_FWD: return kWsHeader + simt_ws_bidir(B, H, L, Dv, F);
         case SLAY_OP_CAUSAL_BWD: return kWsHeader + simt_ws_bwd(B, H, L, Dv, F);
         case SLAY_OP_BIDIR_BWD: return kWsHeader + simt_ws_bidir_bwd(B, H, L, Dv, F);
         case SLAY_OP_LINEAR_ATTN: return kWsHeader + simt_ws_linear(B, H, L, F);
+        case SLAY_OP_CAUSAL_STATE: return kWsHeader + simt_ws_state(B, H, L, F);
         default: return 0;
     }
 }
@@ -450,6 +455,104 @@ slay_status slay_linear_attn_fwd(const void* phq, const void* phk, const void* v
     return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
 }
 
+namespace slay {
+namespace {
+
+// the state arguments of the state-continuation entry points: both of a pair or neither
+slay_status check_state_ptrs(const float* s, const float* z)
+{
+    if ((s == nullptr) != (z == nullptr)) return SLAY_ERR_INVALID_ARG;
+    if (s && (!aligned(s, 16) || !aligned(z, 16))) return SLAY_ERR_INVALID_ARG;
+    return SLAY_OK;
+}
+
+}  // namespace
+}  // namespace slay
+
+slay_status slay_attn_causal_fwd_state(const void* q, const void* k, const void* v, void* out,
+                                       float* den, const float* S_in, const float* z_in,
+                                       float* S_out, float* z_out, int B, int H, int L, int D,
+                                       int Dv, slay_dtype dt, int R, int m, uint64_t seed,
+                                       float eps, void* workspace, size_t ws_bytes, void* stream)
+{
+    slay_status s = check_attn(q, k, v, out, B, H, L, D, Dv, dt, R, m, eps);
+    if (s != SLAY_OK) return s;
+    if ((s = check_state_ptrs(S_in, z_in)) != SLAY_OK) return s;
+    if ((s = check_state_ptrs(S_out, z_out)) != SLAY_OK) return s;
+    if (static_cast<int64_t>(B) * H * L == 0) return SLAY_OK;
+    if (den && !aligned(den, 4)) return SLAY_ERR_INVALID_ARG;
+    const size_t need = attn_ws(SLAY_OP_CAUSAL_FWD, dt, B, H, L, Dv, R, m);
+    if (need > 0 && (!workspace || ws_bytes < need || !aligned(workspace, 256)))
+        return SLAY_ERR_INVALID_ARG;
+    Params P;
+    if ((s = get_params(D, R, m, seed, eps, &P)) != SLAY_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const StateIO sio{S_in, z_in, S_out, z_out};
+    cudaError_t e;
+    if (dt == SLAY_BF16 && tc_supported(SLAY_OP_CAUSAL_FWD, B, H, L, R, m)) {
+        e = tc_attn_fwd(q, k, v, out, den, B, H, L, P, eps, true, workspace, st, false, &sio);
+    } else {
+        e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
+        if (e == cudaSuccess)
+            e = simt_attn_fwd(q, k, v, out, den, B, H, L, dt, P, eps, true,
+                              static_cast<char*>(workspace) + kWsHeader, st, &sio);
+    }
+    return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
+}
+
+slay_status slay_causal_state(const void* k, const void* v, const float* S_in, const float* z_in,
+                              float* S_out, float* z_out, int B, int H, int L, int D, int Dv,
+                              slay_dtype dt, int R, int m, uint64_t seed, float eps,
+                              void* workspace, size_t ws_bytes, void* stream)
+{
+    slay_status s = check_attn(k, k, v, v, B, H, L, D, Dv, dt, R, m, eps);
+    if (s != SLAY_OK) return s;
+    if ((s = check_state_ptrs(S_in, z_in)) != SLAY_OK) return s;
+    if (!S_out || !z_out) return SLAY_ERR_INVALID_ARG;
+    if ((s = check_state_ptrs(S_out, z_out)) != SLAY_OK) return s;
+    if (static_cast<int64_t>(B) * H == 0) return SLAY_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (L == 0) {   // an empty chunk: the state passes through unchanged
+        const size_t bs = static_cast<size_t>(B) * H * R * m * Dv * sizeof(float);
+        const size_t bz = static_cast<size_t>(B) * H * R * m * sizeof(float);
+        cudaError_t e = S_in ? cudaMemcpyAsync(S_out, S_in, bs, cudaMemcpyDeviceToDevice, st)
+                             : cudaMemsetAsync(S_out, 0, bs, st);
+        if (e == cudaSuccess)
+            e = S_in ? cudaMemcpyAsync(z_out, z_in, bz, cudaMemcpyDeviceToDevice, st)
+                     : cudaMemsetAsync(z_out, 0, bz, st);
+        return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
+    }
+    const size_t need = attn_ws(SLAY_OP_CAUSAL_STATE, dt, B, H, L, Dv, R, m);
+    if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return SLAY_ERR_INVALID_ARG;
+    Params P;
+    if ((s = get_params(D, R, m, seed, eps, &P)) != SLAY_OK) return s;
+    const StateIO sio{S_in, z_in, S_out, z_out};
+    cudaError_t e;
+    if (dt == SLAY_BF16 && tc_supported(SLAY_OP_CAUSAL_FWD, B, H, L, R, m)) {
+        e = tc_causal_state(k, v, B, H, L, P, workspace, st, sio);
+    } else {
+        e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
+        if (e == cudaSuccess)
+            e = simt_causal_state(k, v, B, H, L, dt, P, static_cast<char*>(workspace) + kWsHeader,
+                                  st, sio);
+    }
+    return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
+}
+
+slay_status slay_state_prefix(const float* S_all, const float* z_all, int nranks, int rank,
+                              float* S_in, float* z_in, int BH, int F, int Dv, void* stream)
+{
+    if (nranks <= 0 || rank < 0 || rank >= nranks || BH < 0 || F <= 0 || Dv <= 0)
+        return SLAY_ERR_INVALID_ARG;
+    if (Dv != kD || F > kMaxF) return SLAY_ERR_UNSUPPORTED;
+    if (BH == 0) return SLAY_OK;
+    if (!S_all || !z_all || !S_in || !z_in) return SLAY_ERR_INVALID_ARG;
+    const int64_t ns = static_cast<int64_t>(BH) * F * Dv, nz = static_cast<int64_t>(BH) * F;
+    cudaError_t e = simt_state_prefix(S_all, z_all, nranks, rank, ns, nz, S_in, z_in,
+                                      static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
+}
+
 slay_status slay_feature_map_bwd(const void* x, const void* dphi, float* dx, int64_t n_rows,
                                  int D, slay_dtype x_dt, slay_dtype dphi_dt, int R, int m,
                                  uint64_t seed, float eps, void* stream)
@@ -527,7 +630,7 @@ size_t slay_workspace_bytes(slay_op op, slay_dtype dt, int B, int H, int L, int 
     if (check_shape(D, Dv, R, m) != SLAY_OK) return SIZE_MAX;
     if (op == SLAY_OP_FEATURE_MAP || op == SLAY_OP_DECODE) return 0;
     if (op != SLAY_OP_CAUSAL_FWD && op != SLAY_OP_BIDIR_FWD && op != SLAY_OP_CAUSAL_BWD &&
-        op != SLAY_OP_BIDIR_BWD && op != SLAY_OP_LINEAR_ATTN)
+        op != SLAY_OP_BIDIR_BWD && op != SLAY_OP_LINEAR_ATTN && op != SLAY_OP_CAUSAL_STATE)
         return SIZE_MAX;
     if (op == SLAY_OP_LINEAR_ATTN) {   // the contraction alone: F = R * m features given
         if (static_cast<int64_t>(B) * H * L == 0) return 0;

@@ -93,9 +93,15 @@ size_t simt_ws_bidir_bwd(int B, int H, int L, int Dv, int F);
 
 cudaError_t simt_feature_map(const void* x, void* phi, int64_t n, slay_dtype in_dt,
                              slay_dtype out_dt, const Params& P, cudaStream_t st);
+struct StateIO;
 cudaError_t simt_attn_fwd(const void* q, const void* k, const void* v, void* out, float* den,
                           int B, int H, int L, slay_dtype dt, const Params& P, float eps,
-                          bool causal, void* ws, cudaStream_t st);
+                          bool causal, void* ws, cudaStream_t st, const StateIO* sio = nullptr);
+size_t simt_ws_state(int B, int H, int L, int F);
+cudaError_t simt_causal_state(const void* k, const void* v, int B, int H, int L, slay_dtype dt,
+                              const Params& P, void* ws, cudaStream_t st, const StateIO& sio);
+cudaError_t simt_state_prefix(const float* s_all, const float* z_all, int nranks, int rank,
+                              int64_t ns, int64_t nz, float* s_in, float* z_in, cudaStream_t st);
 cudaError_t simt_attn_causal_bwd(const void* q, const void* k, const void* v,
                                  const void* out, const float* den, const void* dout,
                                  float* dq, float* dk, float* dv, int B, int H, int L,

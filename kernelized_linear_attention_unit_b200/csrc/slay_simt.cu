@@ -298,6 +298,33 @@ __global__ void k_scan(float* __restrict__ stt, float* __restrict__ tot, int BH,
     if (mode == 2) tot[static_cast<int64_t>(bh) * FE + idx] = run;
 }
 
+// Exclusive forward prefix over chunks of st[bh][c][f][65] starting from a given state
+// (s_in [bh][f][64], z_in [bh][f]; null = zero), with the state after the last chunk written
+// to s_out / z_out (each may be null).  One thread per (bh, f, e).
+__global__ void k_scan_state(float* __restrict__ stt, int BH, int NC, int F,
+                             const float* __restrict__ s_in, const float* __restrict__ z_in,
+                             float* __restrict__ s_out, float* __restrict__ z_out)
+{
+    const int FE = F * E;
+    const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (gid >= static_cast<int64_t>(BH) * FE) return;
+    const int bh = static_cast<int>(gid / FE), idx = static_cast<int>(gid % FE);
+    const int f = idx / E, e = idx % E;
+    float run = 0.0f;
+    if (s_in) run = e < kD ? s_in[(static_cast<int64_t>(bh) * F + f) * kD + e] : z_in[static_cast<int64_t>(bh) * F + f];
+    float* base = stt + static_cast<int64_t>(bh) * NC * FE + idx;
+    for (int c = 0; c < NC; ++c) {
+        const float x = base[static_cast<int64_t>(c) * FE];
+        base[static_cast<int64_t>(c) * FE] = run;
+        run += x;
+    }
+    if (e < kD) {
+        if (s_out) s_out[(static_cast<int64_t>(bh) * F + f) * kD + e] = run;
+    } else if (z_out) {
+        z_out[static_cast<int64_t>(bh) * F + f] = run;
+    }
+}
+
 // --------------------------------------------------------------- chunk output
 // grid (NC, BH), dynamic smem.  Causal: intra-chunk masked term + prefix state.
 // Bidirectional: total state only.
@@ -1001,7 +1028,7 @@ static cudaError_t phi_map(const void* x, T* phi, int64_t rows, const Params& P,
 template <typename T>
 static cudaError_t attn_fwd_t(const void* q, const void* k, const void* v, void* out, float* den,
                               int B, int H, int L, const Params& P, float eps, bool causal,
-                              void* ws, cudaStream_t st)
+                              void* ws, cudaStream_t st, const StateIO* sio)
 {
     const int BH = B * H, F = P.F, NC = nchunks(L);
     const int64_t rows = static_cast<int64_t>(BH) * L;
@@ -1024,7 +1051,11 @@ static cudaError_t attn_fwd_t(const void* q, const void* k, const void* v, void*
     const int64_t nth = static_cast<int64_t>(BH) * FE;
     {
         TraceScope trace_("simt_scan", st);
-        k_scan<<<static_cast<unsigned>((nth + 255) / 256), 256, 0, st>>>(stt, tot, BH, NC, FE, causal ? 0 : 2);
+        if (causal && sio)
+            k_scan_state<<<static_cast<unsigned>((nth + 255) / 256), 256, 0, st>>>(
+                stt, BH, NC, F, sio->s_in, sio->z_in, sio->s_out, sio->z_out);
+        else
+            k_scan<<<static_cast<unsigned>((nth + 255) / 256), 256, 0, st>>>(stt, tot, BH, NC, FE, causal ? 0 : 2);
     }
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     const size_t smem = sizeof(OutSmem);
@@ -1039,12 +1070,79 @@ static cudaError_t attn_fwd_t(const void* q, const void* k, const void* v, void*
     return cudaGetLastError();
 }
 
+// The causal state of a whole sequence chunk, sum_j phi(k_j) [v_j, 1]^T -> S [bh][f][64],
+// z [bh][f] (plus an optional initial state): phi(k), the chunk states, their total.
+template <typename T>
+static cudaError_t causal_state_t(const void* k, const void* v, int B, int H, int L,
+                                  const Params& P, void* ws, cudaStream_t st, const StateIO& sio)
+{
+    const int BH = B * H, F = P.F, NC = nchunks(L);
+    const int64_t rows = static_cast<int64_t>(BH) * L;
+    char* w = static_cast<char*>(ws);
+    T* phk = reinterpret_cast<T*>(w);
+    float* stt = reinterpret_cast<float*>(w + align256(rows * F * sizeof(float)));
+    cudaError_t err;
+    if ((err = phi_map<T>(k, phk, rows, P, st)) != cudaSuccess) return err;
+    {
+        TraceScope trace_("simt_chunk_state", st);
+        k_chunk_state<T, T><<<dim3((F + C - 1) / C, NC, BH), NT, 0, st>>>(phk, cp<T>(v), kD, stt, L, F);
+    }
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    const int64_t nth = static_cast<int64_t>(BH) * F * E;
+    TraceScope trace_("simt_scan", st);
+    k_scan_state<<<static_cast<unsigned>((nth + 255) / 256), 256, 0, st>>>(stt, BH, NC, F, sio.s_in,
+                                                                           sio.z_in, sio.s_out, sio.z_out);
+    return cudaGetLastError();
+}
+
+size_t simt_ws_state(int B, int H, int L, int F)
+{
+    const size_t BH = static_cast<size_t>(B) * H;
+    return align256(BH * L * F * sizeof(float)) +
+           align256(BH * nchunks(L) * static_cast<size_t>(F) * E * sizeof(float));
+}
+
+cudaError_t simt_causal_state(const void* k, const void* v, int B, int H, int L, slay_dtype dt,
+                              const Params& P, void* ws, cudaStream_t st, const StateIO& sio)
+{
+    if (dt == SLAY_F32) return causal_state_t<float>(k, v, B, H, L, P, ws, st, sio);
+    return causal_state_t<__nv_bfloat16>(k, v, B, H, L, P, ws, st, sio);
+}
+
+// S_in = sum of the per-rank states of the ranks before `rank` (an exclusive prefix over the
+// all-gathered [nranks][BH][F][64] states and [nranks][BH][F] z), one thread per element
+__global__ void k_state_prefix(const float* __restrict__ s_all, const float* __restrict__ z_all,
+                               int nranks, int rank, int64_t ns, int64_t nz,
+                               float* __restrict__ s_in, float* __restrict__ z_in)
+{
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < ns;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        float a = 0.0f;
+        for (int r = 0; r < rank && r < nranks; ++r) a += s_all[static_cast<int64_t>(r) * ns + i];
+        s_in[i] = a;
+        if (i < nz) {
+            float b = 0.0f;
+            for (int r = 0; r < rank && r < nranks; ++r) b += z_all[static_cast<int64_t>(r) * nz + i];
+            z_in[i] = b;
+        }
+    }
+}
+
+cudaError_t simt_state_prefix(const float* s_all, const float* z_all, int nranks, int rank,
+                              int64_t ns, int64_t nz, float* s_in, float* z_in, cudaStream_t st)
+{
+    const int grid = static_cast<int>(std::min<int64_t>((ns + 255) / 256, 1184));
+    TraceScope trace_("simt_state_prefix", st);
+    k_state_prefix<<<grid, 256, 0, st>>>(s_all, z_all, nranks, rank, ns, nz, s_in, z_in);
+    return cudaGetLastError();
+}
+
 cudaError_t simt_attn_fwd(const void* q, const void* k, const void* v, void* out, float* den,
                           int B, int H, int L, slay_dtype dt, const Params& P, float eps,
-                          bool causal, void* ws, cudaStream_t st)
+                          bool causal, void* ws, cudaStream_t st, const StateIO* sio)
 {
-    if (dt == SLAY_F32) return attn_fwd_t<float>(q, k, v, out, den, B, H, L, P, eps, causal, ws, st);
-    return attn_fwd_t<__nv_bfloat16>(q, k, v, out, den, B, H, L, P, eps, causal, ws, st);
+    if (dt == SLAY_F32) return attn_fwd_t<float>(q, k, v, out, den, B, H, L, P, eps, causal, ws, st, sio);
+    return attn_fwd_t<__nv_bfloat16>(q, k, v, out, den, B, H, L, P, eps, causal, ws, st, sio);
 }
 
 template <typename Tin, typename Tout, bool kSigned, bool kPerformer>

@@ -155,6 +155,12 @@ struct KParams {
     int acc_in, acc_out;
     float* part_num;
     float* part_den;
+    // The state entering the sequence (causal forward continued from a state): S [bh][f][64]
+    // and z [bh][f] of this launch's feature chunk, bh strides s_stride / z_stride floats;
+    // null for a zero state.
+    const float* s_in;
+    const float* z_in;
+    int s_stride, z_stride;
 };
 
 // The output row `g` (global row index over [BH][L]) from its numerator o0|o1 (64 fp32 bit
@@ -698,7 +704,8 @@ __device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr)
 // at piece position e4 ^ (f % 16) (read back one row per lane without bank conflicts, see
 // read_state_sum), z into zacc.  The caller synchronises the block before reading them.
 __device__ __forceinline__ void sum_segments(const float* __restrict__ wsS, const float* __restrict__ wsZ,
-                                             int bh, int nseg, int nsum, int F, float* sacc, float* zacc)
+                                             int bh, int nseg, int nsum, int F, float* sacc, float* zacc,
+                                             const KParams* kp = nullptr)
 {
     const int tid = threadIdx.x;
     const int J = F / 32;   // pieces per thread: F * 16 / kOutThreads
@@ -706,6 +713,13 @@ __device__ __forceinline__ void sum_segments(const float* __restrict__ wsS, cons
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[j] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     float zsum = 0.0f;
+    if (kp && kp->s_in) {   // the state the sequence starts from (same [F][64] piece order)
+        const float4* src = reinterpret_cast<const float4*>(kp->s_in + static_cast<size_t>(bh) * kp->s_stride);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (j < J) acc[j] = src[tid + kOutThreads * j];
+        if (tid < F) zsum = kp->z_in[static_cast<size_t>(bh) * kp->z_stride + tid];
+    }
 #pragma unroll 2
     for (int s = 0; s < nsum; ++s) {
         const size_t segidx = static_cast<size_t>(bh) * nseg + s;
@@ -1311,7 +1325,7 @@ k_tc_causal_out_ts(const __grid_constant__ CUtensorMap tmq, const __grid_constan
     // The state entering the segment, the sum of the earlier segments' sums, into the phi(k)
     // slices' space (no copy has reached it yet), z into zpre
     griddep_wait();   // the state kernel's sums and phi(k) (launched as its dependent)
-    sum_segments(wsS, wsZ, sg.bh, kp.nseg, sg.seg, kp.F, reinterpret_cast<float*>(sm + L.phik), zpre);
+    sum_segments(wsS, wsZ, sg.bh, kp.nseg, sg.seg, kp.F, reinterpret_cast<float*>(sm + L.phik), zpre, &kp);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1999,9 +2013,89 @@ cudaError_t set_smem(K kernel, size_t bytes)
                                 static_cast<int>(bytes));
 }
 
+// The state after the whole sequence for one feature chunk: S_out[bh][c0 + f][e] = S_in +
+// sum over the nseg per-segment sums (every segment's sum is in the workspace when the state
+// kernel ran over all of them), z likewise.  One thread per (bh, f, e) or (bh, f).
+__global__ void k_state_total(const float* __restrict__ wsS, const float* __restrict__ wsZ, int BH,
+                              int nseg, int Fc, int Ftot, int c0, const float* __restrict__ s_in,
+                              const float* __restrict__ z_in, float* __restrict__ s_out,
+                              float* __restrict__ z_out)
+{
+    const int64_t n = static_cast<int64_t>(BH) * Fc * 64;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int bh = static_cast<int>(i / (static_cast<int64_t>(Fc) * 64));
+        const int fe = static_cast<int>(i % (static_cast<int64_t>(Fc) * 64));
+        const size_t dst = static_cast<size_t>(bh) * Ftot * 64 + static_cast<size_t>(c0) * 64 + fe;
+        float acc = s_in ? s_in[dst] : 0.0f;
+        for (int sgi = 0; sgi < nseg; ++sgi)
+            acc += wsS[(static_cast<size_t>(bh) * nseg + sgi) * Fc * 64 + fe];
+        s_out[dst] = acc;
+        if ((fe & 63) == 0) {
+            const int f = fe >> 6;
+            const size_t dz = static_cast<size_t>(bh) * Ftot + c0 + f;
+            float az = z_in ? z_in[dz] : 0.0f;
+            for (int sgi = 0; sgi < nseg; ++sgi) az += wsZ[(static_cast<size_t>(bh) * nseg + sgi) * Fc + f];
+            z_out[dz] = az;
+        }
+    }
+}
+
+size_t tc_state_workspace_bytes(int B, int H, int L, int R, int m)
+{
+    const int BH = B * H;
+    return ws_layout(BH, L, R * m, choose_nseg(BH, (L + kTile - 1) / kTile), false).total;
+}
+
+cudaError_t tc_causal_state(const void* k, const void* v, int B, int H, int L, const Params& P,
+                            void* ws, cudaStream_t st, const StateIO& sio)
+{
+    if (!P.wB) return cudaErrorNotSupported;
+    const int BH = B * H, F = P.F, Fc = chunk_features(F), nch = F / Fc;
+    const int ntiles = (L + kTile - 1) / kTile;
+    const int nseg = choose_nseg(BH, ntiles);
+    const WsLayout wl = ws_layout(BH, L, F, nseg, false);
+    char* w = static_cast<char*>(ws);
+    CUtensorMap mk, mv, mpk;
+    if (!map_rows(&mk, k, L, BH) || !map_rows(&mv, v, L, BH) || !map_phik(&mpk, P.wB, Fc, 1, 1))
+        return cudaErrorInvalidValue;
+    int* err = reinterpret_cast<int*>(w);
+    float* wsS = reinterpret_cast<float*>(w + wl.s);
+    float* wsZ = reinterpret_cast<float*>(w + wl.z);
+    cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), st);
+    if (e != cudaSuccess) return e;
+    const size_t sms = smem_bytes_state(Fc);
+    if ((e = set_smem(k_tc_causal_state<false>, sms)) != cudaSuccess) return e;
+    for (int c = 0; c < nch; ++c) {
+        CUtensorMap mw;
+        const uint16_t* wc = P.wB + static_cast<size_t>(c) * (Fc / kSub) * 64 * 64;
+        if (!map_w(&mw, wc, Fc)) return cudaErrorInvalidValue;
+        KParams kp{};
+        kp.L = L; kp.F = Fc; kp.nseg = nseg; kp.ntiles = ntiles;
+        kp.all_segs = 1;
+        for (int t = 0; t < kMaxSlices; ++t) {
+            const int node = t < Fc / kSlice ? (c * Fc + t * kSlice) / P.m : 0;
+            kp.a2[t] = P.a2[node];
+            kp.b2[t] = P.b2[node];
+        }
+        {
+            TraceScope trace_("tc_state_sums", st);
+            k_tc_causal_state<false><<<BH * nseg, kThreads, sms, st>>>(mk, mv, mw, mpk, kp, wsS, wsZ, err);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+        TraceScope trace_("tc_state_total", st);
+        const int64_t n = static_cast<int64_t>(BH) * Fc * 64;
+        const int grid = static_cast<int>(std::min<int64_t>((n + 255) / 256, 4 * kNumSMs));
+        k_state_total<<<grid, 256, 0, st>>>(wsS, wsZ, BH, nseg, Fc, F, c * Fc, sio.s_in, sio.z_in,
+                                            sio.s_out, sio.z_out);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
 cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, float* den, int B,
                         int H, int L, const Params& P, float eps, bool causal, void* ws,
-                        cudaStream_t st, bool lowmem)
+                        cudaStream_t st, bool lowmem, const StateIO* sio)
 {
     if (!P.wB) return cudaErrorNotSupported;
     const int BH = B * H, F = P.F, Fc = chunk_features(F), nch = F / Fc;
@@ -2042,6 +2136,10 @@ cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, 
         kp.acc_out = c + 1 < nch;
         kp.part_num = nch > 1 ? reinterpret_cast<float*>(w + wl.num) : nullptr;
         kp.part_den = nch > 1 ? reinterpret_cast<float*>(w + wl.den) : nullptr;
+        kp.s_in = (sio && sio->s_in) ? sio->s_in + static_cast<size_t>(c) * Fc * 64 : nullptr;
+        kp.z_in = (sio && sio->s_in) ? sio->z_in + static_cast<size_t>(c) * Fc : nullptr;
+        kp.s_stride = F * 64;
+        kp.z_stride = F;
         if (!causal) {
             // every segment's sum, then the readout against their total
             if ((e = set_smem(k_tc_causal_state<false>, sms)) != cudaSuccess) return e;
@@ -2075,10 +2173,20 @@ cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, 
             default: break;
             }
             if ((e = set_smem(kern, smo)) != cudaSuccess) return e;
-            TraceScope trace_("tc_qphi_out", st);
-            e = launch_dependent(kern, BH * nseg, kOutThreads, smo, st, mq, mpk, mv, mw, kp, wsS, wsZ, o, den, err);
-            if (e != cudaSuccess) return e;
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            {
+                TraceScope trace_("tc_qphi_out", st);
+                e = launch_dependent(kern, BH * nseg, kOutThreads, smo, st, mq, mpk, mv, mw, kp, wsS, wsZ, o, den, err);
+                if (e != cudaSuccess) return e;
+                if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            }
+            if (sio && sio->s_out) {   // the state after the sequence, this chunk's features
+                TraceScope trace_("tc_state_total", st);
+                const int64_t n = static_cast<int64_t>(BH) * Fc * 64;
+                const int grid = static_cast<int>(std::min<int64_t>((n + 255) / 256, 4 * kNumSMs));
+                k_state_total<<<grid, 256, 0, st>>>(wsS, wsZ, BH, nseg, Fc, F, c * Fc, kp.s_in ? sio->s_in : nullptr,
+                                                    kp.s_in ? sio->z_in : nullptr, sio->s_out, sio->z_out);
+                if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            }
             continue;
         }
         // low-memory form (no phi(k) buffer): the output kernel recomputes phi(k)

@@ -48,8 +48,22 @@ void fmap_arm_wait_fault(int on);
 // Device address of the status word of the feature-map kernels, forward and backward (set
 // when a bounded wait ran out).
 const void* fmap_status_word();
+// A causal forward continued from a state and / or returning the final one: S [BH][F][64],
+// z [BH][F] fp32 (s_in null: zero state; s_out null: not written).
+struct StateIO {
+    const float* s_in;
+    const float* z_in;
+    float* s_out;
+    float* z_out;
+};
 cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, float* den,
                         int B, int H, int L, const Params& P, float eps, bool causal, void* ws,
-                        cudaStream_t st, bool lowmem = false);
+                        cudaStream_t st, bool lowmem = false, const StateIO* sio = nullptr);
+
+// The state of a whole sequence on tensor cores (k projections, phi(k) and per-segment sums
+// by the state kernel over every segment, then their total plus sio.s_in into sio.s_out).
+size_t tc_state_workspace_bytes(int B, int H, int L, int R, int m);
+cudaError_t tc_causal_state(const void* k, const void* v, int B, int H, int L, const Params& P,
+                            void* ws, cudaStream_t st, const StateIO& sio);
 
 }  // namespace slay

@@ -1,0 +1,76 @@
+"""Sequence-parallel causal SLAY forward over the ranks of a process group.
+
+The causal contraction's prefix state carries everything earlier tokens contribute
+(review, "Proposed method", step 6), so a long sequence split into contiguous pieces, one
+per rank in rank order, needs one exchange: each rank sums its own piece's state
+(slay_causal_state: sum of phi(k) [v, 1]^T), the ranks all-gather those states (F x (Dv+1)
+fp32 per (b, h)), each rank adds up the states of the ranks before it (slay_state_prefix)
+and runs its piece's causal forward from that state (slay_attn_causal_fwd_state).  The
+collective is NCCL's all-gather over NVLink on GPUs (any backend works: the states are
+ordinary tensors); no kernel waits on another rank's memory.
+
+Every step of the path runs in the library's kernels; this module orders them and calls the
+collective.  The three steps are passed in as an object with methods state, prefix and
+forward (LibraryOps by default), so the same orchestration runs in tests on CPU ranks.
+"""
+from typing import Optional
+
+import torch
+import torch.distributed as dist
+
+from . import binding as bd
+
+
+class LibraryOps:
+    """The three steps through libslay.so (device tensors)."""
+
+    def __init__(self, R, m, seed, eps):
+        self.R, self.m, self.seed, self.eps = R, m, seed, eps
+
+    def state(self, k, v, S_out, z_out):
+        bd.slay_causal_state(k, v, S_out, z_out, self.R, self.m, self.seed, self.eps)
+
+    def prefix(self, S_all, z_all, rank, S_in, z_in):
+        bd.slay_state_prefix(S_all, z_all, rank, S_in, z_in)
+
+    def forward(self, q, k, v, out, den, S_in, z_in):
+        bd.slay_attn_causal_fwd_state(q, k, v, out, den, self.R, self.m, self.seed, self.eps,
+                                      S_in=S_in, z_in=z_in)
+
+
+def gather_states(S_loc: torch.Tensor, z_loc: torch.Tensor, group=None):
+    """All ranks' piece states stacked in rank order: [N, B, H, F, Dv] and [N, B, H, F]."""
+    world = dist.get_world_size(group) if dist.is_initialized() else 1
+    if world == 1:
+        return S_loc.unsqueeze(0), z_loc.unsqueeze(0)
+    S_list = [torch.empty_like(S_loc) for _ in range(world)]
+    z_list = [torch.empty_like(z_loc) for _ in range(world)]
+    dist.all_gather(S_list, S_loc.contiguous(), group=group)
+    dist.all_gather(z_list, z_loc.contiguous(), group=group)
+    return torch.stack(S_list), torch.stack(z_list)
+
+
+def causal_fwd_seqpar(q, k, v, out, den, F: int, ops, group=None,
+                      scratch: Optional[dict] = None):
+    """This rank's piece [B, H, Lr, D] of a sequence split over the group in rank order:
+    out (and den, if given) of the causal forward of the whole sequence at this piece's rows.
+
+    F = R * m features; ops: LibraryOps (or an object with the same three methods);
+    scratch: optional dict reused across calls for the state buffers."""
+    rank = dist.get_rank(group) if dist.is_initialized() else 0
+    B, H = q.shape[0], q.shape[1]
+    Dv = v.shape[-1]
+    sc = scratch if scratch is not None else {}
+    shape_s, shape_z = (B, H, F, Dv), (B, H, F)
+    if sc.get("shape") != (shape_s, q.device):
+        sc.clear()
+        sc["shape"] = (shape_s, q.device)
+        for name in ("S_loc", "S_in"):
+            sc[name] = torch.empty(shape_s, dtype=torch.float32, device=q.device)
+        for name in ("z_loc", "z_in"):
+            sc[name] = torch.empty(shape_z, dtype=torch.float32, device=q.device)
+    ops.state(k, v, sc["S_loc"], sc["z_loc"])
+    S_all, z_all = gather_states(sc["S_loc"], sc["z_loc"], group)
+    ops.prefix(S_all, z_all, rank, sc["S_in"], sc["z_in"])
+    ops.forward(q, k, v, out, den, sc["S_in"], sc["z_in"])
+    return out

@@ -109,3 +109,77 @@ def test_gpus_flag_must_match_the_launcher(monkeypatch):
     monkeypatch.setenv("WORLD_SIZE", "4")
     with pytest.raises(SystemExit):
         bench.main(["--gpus", "2", "--check-launch"])
+
+
+class _OracleOps:
+    """The three sequence-parallel steps computed by the fp64 oracle on CPU tensors (a
+    stand-in for the library on ranks without a GPU; the orchestration under test is the
+    package's own)."""
+
+    def __init__(self, P):
+        self.P = P
+
+    def state(self, k, v, S_out, z_out):
+        import oracle as O
+        _, _, S, z = O.attn_causal_state(k.numpy(), k.numpy(), v.numpy(), self.P)
+        S_out.copy_(torch_from(S))
+        z_out.copy_(torch_from(z))
+
+    def prefix(self, S_all, z_all, rank, S_in, z_in):
+        S_in.copy_(S_all[:rank].sum(0) if rank else torch_zeros_like(S_in))
+        z_in.copy_(z_all[:rank].sum(0) if rank else torch_zeros_like(z_in))
+
+    def forward(self, q, k, v, out, den, S_in, z_in):
+        import oracle as O
+        o, d, _, _ = O.attn_causal_state(q.numpy(), k.numpy(), v.numpy(), self.P,
+                                         S_in.double().numpy(), z_in.double().numpy())
+        out.copy_(torch_from(o))
+        den.copy_(torch_from(d))
+
+
+def torch_from(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a)).float()
+
+
+def torch_zeros_like(t):
+    import torch
+    return torch.zeros_like(t)
+
+
+def _seqpar_rank(rank, world, port, outdir):
+    import torch
+    import torch.distributed as dist
+    import oracle as O
+    from kernelized_linear_attention_unit_b200 import seqpar
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        w = W.Workload("sp", B=1, H=2, L=90, R=2, m=8, dtype="f32", data_seed=61)
+        q, k, v = W.gen_qkv(w)
+        P = O.sketch_params(w.D, w.R, w.m, w.sketch_seed, float(np.float32(w.eps)))
+        a, b = rank * w.L // world, (rank + 1) * w.L // world
+        piece = [torch.from_numpy(np.ascontiguousarray(x[:, :, a:b])).double() for x in (q, k, v)]
+        out = torch.empty((1, 2, b - a, 64))
+        den = torch.empty((1, 2, b - a))
+        seqpar.causal_fwd_seqpar(*piece, out, den, w.F, _OracleOps(P))
+        np.save(os.path.join(outdir, "sp%d.npy" % rank), out.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sequence_parallel_orchestration_two_ranks():
+    # two gloo ranks each hold half of a sequence; the package's orchestration (piece state,
+    # all-gather, prefix over earlier ranks, forward from it) reproduces the whole sequence
+    import torch.multiprocessing as mp
+    import oracle as O
+    outdir = tempfile.mkdtemp(prefix="slay_sp_")
+    mp.spawn(_seqpar_rank, args=(2, _free_port(), outdir), nprocs=2, join=True)
+    got = np.concatenate([np.load(os.path.join(outdir, "sp%d.npy" % r)) for r in range(2)], axis=2)
+    w = W.Workload("sp", B=1, H=2, L=90, R=2, m=8, dtype="f32", data_seed=61)
+    q, k, v = W.gen_qkv(w)
+    P = O.sketch_params(w.D, w.R, w.m, w.sketch_seed, float(np.float32(w.eps)))
+    want, _ = O.attn_quadratic(q, k, v, P, True)
+    assert np.abs(got - want).max() < 1e-5 * np.abs(want).max()

@@ -613,3 +613,60 @@ def test_variant_attention_composed(kind):
     bd.slay_linear_attn_fwd(pq, pk, dev(v, "bf16"), out, den, _eps(w), True)
     torch.cuda.synchronize()
     _check_fwd("composed %s causal" % kind, host(out), host(den), want, wden, TOL["bf16"])
+
+
+# ------------------------------------------- state continuation, sequence parallelism
+
+@pytest.mark.parametrize("dt,R,m,L,cuts", [("bf16", 4, 64, 1000, (300, 700)),
+                                           ("bf16", 8, 64, 700, (128, 512)),
+                                           ("f32", 2, 16, 300, (1, 150)),
+                                           ("bf16", 2, 16, 257, (64, 65))])
+def test_sequence_pieces_emulating_ranks(dt, R, m, L, cuts):
+    # the sequence-parallel decomposition on one GPU: every piece's state, the exclusive
+    # prefix over pieces, each piece's forward from that prefix; the pieces' outputs and the
+    # last piece's final state against the oracle's whole-sequence forward
+    w = small(dt, R, m, L, B=1, H=3, seed=25)
+    q, k, v = W.gen_qkv(w)
+    P = params(w)
+    want, wden, wS, wz = O.attn_causal_state(q, k, v, P)
+    bounds = (0,) + tuple(cuts) + (L,)
+    pieces = [(a, b) for a, b in zip(bounds[:-1], bounds[1:])]
+    F = w.F
+    eps = _eps(w)
+    Ss, zs = [], []
+    for a, b in pieces:
+        S = torch.empty((1, 3, F, 64), device="cuda")
+        z = torch.empty((1, 3, F), device="cuda")
+        ws = bd.slay_causal_state(dev(k[:, :, a:b], dt), dev(v[:, :, a:b], dt), S, z, R, m,
+                                  w.sketch_seed, eps)
+        bd.slay_kernel_status(ws)
+        Ss.append(S)
+        zs.append(z)
+    S_all, z_all = torch.stack(Ss), torch.stack(zs)
+    outs, dens = [], []
+    S_fin = torch.empty((1, 3, F, 64), device="cuda")
+    z_fin = torch.empty((1, 3, F), device="cuda")
+    for r, (a, b) in enumerate(pieces):
+        S_in = torch.empty((1, 3, F, 64), device="cuda")
+        z_in = torch.empty((1, 3, F), device="cuda")
+        bd.slay_state_prefix(S_all, z_all, r, S_in, z_in)
+        out = torch.empty((1, 3, b - a, 64), device="cuda", dtype=TDT[dt])
+        den = torch.empty((1, 3, b - a), device="cuda")
+        last = r == len(pieces) - 1
+        ws = bd.slay_attn_causal_fwd_state(dev(q[:, :, a:b], dt), dev(k[:, :, a:b], dt),
+                                           dev(v[:, :, a:b], dt), out, den, R, m, w.sketch_seed,
+                                           eps, S_in=S_in, z_in=z_in,
+                                           S_out=S_fin if last else None,
+                                           z_out=z_fin if last else None)
+        bd.slay_kernel_status(ws)
+        outs.append(host(out))
+        dens.append(host(den))
+    torch.cuda.synchronize()
+    name = "pieces %s R%d m%d L%d %s" % (dt, R, m, L, cuts)
+    _check_fwd(name, np.concatenate(outs, axis=2), np.concatenate(dens, axis=2), want, wden,
+               TOL[dt])
+    # the states are fp32 sums on both sides; in bf16 mode phi(k) is rounded to bf16 first
+    check(name + " final S", host(S_fin), wS, TOL[dt])
+    check(name + " final z", host(z_fin), wz, TOL[dt])
+    check(name + " piece-0 S", host(Ss[0]), O.attn_causal_state(
+        q[:, :, :cuts[0]], k[:, :, :cuts[0]], v[:, :, :cuts[0]], P)[2], TOL[dt])
