@@ -1255,8 +1255,8 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
     if ((err = phi_map<T>(q, phq, rows, P, st)) != cudaSuccess) return err;
     if ((err = phi_map<T>(k, phk, rows, P, st)) != cudaSuccess) return err;
     // bf16 phi: states, contraction on tensor cores over 128-token tiles; else 64-token chunks
-    // (the bidirectional form always takes the chunk kernels: no masked term, whole sums)
-    const bool tcb = !bidir && std::is_same<T, __nv_bfloat16>::value && tc_bwd_tile_supported(F, L);
+    // (the bidirectional form: the same kernels with whole-sequence sums and no masked term)
+    const bool tcb = std::is_same<T, __nv_bfloat16>::value && tc_bwd_tile_supported(F, L);
     // tensor-core path: dn as bf16 rows and delta in the dn region (132 of its 260 bytes a row)
     __nv_bfloat16* dn16 = reinterpret_cast<__nv_bfloat16*>(dn);
     float* delta = reinterpret_cast<float*>(dn16 + rows * kD);
@@ -1307,7 +1307,11 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
         k_scan<<<sgrid, 256, 0, st>>>(gbw, gtot, BH, NS, FE, bidir ? 2 : 1);
     }
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    if (bidir) {
+    if (tcb) {
+        if ((err = tc_bwd_tile(phq, phk, v, dn16, delta, bidir ? stot : sfw, bidir ? gtot : gbw,
+                               dphq, dphk, dphi16, dv, BH, L, F, status, st, bidir)) != cudaSuccess)
+            return err;
+    } else if (bidir) {
         // dphi as bf16 when the tensor-core feature-map backward takes it, else fp32
         if (dphi16) {
             auto kern = k_bwd_chunk<T, true, __nv_bfloat16>;
@@ -1330,10 +1334,6 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
                                                  dv, L, F);
         }
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    } else if (tcb) {
-        if ((err = tc_bwd_tile(phq, phk, v, dn16, delta, sfw, gbw, dphq, dphk, dphi16, dv, BH, L, F,
-                               status, st)) != cudaSuccess)
-            return err;
     } else {
         const size_t smem = sizeof(BwdSmem);
         auto kern = k_bwd_chunk<T, false, float>;

@@ -38,10 +38,11 @@ bool tc_bwd_tile_supported(int F, int L);
 cudaError_t tc_bwd_states(const void* phq, const void* phk, const void* v, const void* dn16,
                           const float* delta, float* st_s, float* st_g, int BH, int L, int F,
                           int* err, cudaStream_t st);
+// bidir: the bidirectional form (no masked term; sfw, gbw are each sequence's whole sums).
 cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const void* dn16,
                         const float* delta, const float* sfw, const float* gbw, void* dphq,
                         void* dphk, bool dphi_bf16, float* dv, int BH, int L, int F, int* err,
-                        cudaStream_t st);
+                        cudaStream_t st, bool bidir = false);
 // Test hook: the next tensor-core feature-map launch withholds one barrier arrival and
 // bounds its waits at 1 ms, so that a wait runs out (on != 0 arms it, 0 disarms it).
 void fmap_arm_wait_fault(int on);

@@ -80,6 +80,8 @@ __host__ __device__ inline BwLayout bw_layout()
 struct BwParams {
     int L, F, ntiles, nitems;
     int dphi_bf16;   // contraction: store dphi(q), dphi(k) as bf16 (else fp32)
+    int bidir;       // contraction: the bidirectional form (no masked intra-tile term; sfw,
+                     // gbw hold each sequence's whole sums [BH][65][F], not per-tile scans)
 };
 
 __global__ void __launch_bounds__(kBwThreads, 1)
@@ -235,8 +237,10 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
             const int i_abs = t * kT + static_cast<int>(row);   // this thread's token
             const bool valid = i_abs < bp.L;
             const int64_t grow = static_cast<int64_t>(bh) * bp.L + i_abs;
-            const float* Sb = sfw + (static_cast<int64_t>(bh) * bp.ntiles + t) * bp.F * kE;
-            const float* Gb = gbw + (static_cast<int64_t>(bh) * bp.ntiles + t) * bp.F * kE;
+            const int64_t sidx = bp.bidir ? static_cast<int64_t>(bh) : static_cast<int64_t>(bh) * bp.ntiles + t;
+            const float* Sb = sfw + sidx * bp.F * kE;
+            const float* Gb = gbw + sidx * bp.F * kE;
+            const bool intra = valid && !bp.bidir;   // the masked term exists only when causal
             const float dl = valid ? delta[grow] : 0.0f;   // dn itself arrives by TMA with V
             // masked P~ and C~ (this warp's half of the columns j)
             wait_k(BW_PCF, it);
@@ -262,8 +266,8 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
                         const int jl = 64 * half + 32 * hh + 2 * c;     // column within the tile
-                        const bool k0 = valid && jl <= static_cast<int>(row) && j0 + 32 * hh + 2 * c < bp.L;
-                        const bool k1 = valid && jl + 1 <= static_cast<int>(row) && j0 + 32 * hh + 2 * c + 1 < bp.L;
+                        const bool k0 = intra && jl <= static_cast<int>(row) && j0 + 32 * hh + 2 * c < bp.L;
+                        const bool k1 = intra && jl + 1 <= static_cast<int>(row) && j0 + 32 * hh + 2 * c + 1 < bp.L;
                         pk[c] = pack_bf16(k0 ? __uint_as_float(P[2 * c]) : 0.0f,
                                           k1 ? __uint_as_float(P[2 * c + 1]) : 0.0f);
                         ck[c] = pack_bf16(k0 ? __uint_as_float(Cc[2 * c]) + dl : 0.0f,
@@ -627,6 +631,7 @@ cudaError_t tc_bwd_states(const void* phq, const void* phk, const void* v, const
     bp.ntiles = (L + kT - 1) / kT;
     bp.nitems = BH * bp.ntiles;
     bp.dphi_bf16 = 0;
+    bp.bidir = 0;
     const size_t smem = st_layout().total + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_tc_bwd_states, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
@@ -640,7 +645,7 @@ cudaError_t tc_bwd_states(const void* phq, const void* phk, const void* v, const
 cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const void* dn16,
                         const float* delta, const float* sfw, const float* gbw, void* dphq,
                         void* dphk, bool dphi_bf16, float* dv, int BH, int L, int F, int* err,
-                        cudaStream_t st)
+                        cudaStream_t st, bool bidir)
 {
     if (!tc_bwd_tile_supported(F, L)) return cudaErrorNotSupported;
     CUtensorMap mq, mk, mv, mdn;
@@ -653,6 +658,7 @@ cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const v
     bp.ntiles = (L + kT - 1) / kT;
     bp.nitems = BH * bp.ntiles;
     bp.dphi_bf16 = dphi_bf16 ? 1 : 0;
+    bp.bidir = bidir ? 1 : 0;
     const size_t smem = bw_layout().total + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_tc_bwd_tile, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
