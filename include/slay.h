@@ -36,6 +36,14 @@
  *     forward as feature chunks of at most 256 when F > 256), with m % 64 == 0 for the
  *     attention forward and m % 32 == 0 for the feature map and its backward; other sizes
  *     run on CUDA cores.
+ *   - q and k rows (and the feature map's x rows) need not be unit length: every kernel
+ *     projects them onto the sphere.  Supported row norms: up to 1e15.  Rows below 1e-12
+ *     take the norm guard (x^ = x / 1e-12, a zero row maps to phi = 0).  The fp32 kernels
+ *     divide by the norm before the projections.  The bf16 tensor-core kernels project the
+ *     raw row and fold 1/|x|^2 into phi's exponent, so that exponent must stay inside
+ *     fp32's range for every feature: at |x| = 2^50 (about 1e15) the row error is still
+ *     fp32 rounding for R <= 16; from about 2^55 the smallest features are flushed or
+ *     clamped and the error grows; at 1.8e19 the fp32 sum of squares overflows.
  *   - Errors are status codes, never exceptions or aborts.  On any error nothing is
  *     enqueued.  The library owns only its sketch-parameter cache: one small device
  *     buffer per (device, D, R, m, seed, eps), created on first use (synchronous

@@ -10,10 +10,11 @@ cut a sequence into starts and ends on one) plus random rows, in the launch conf
 the benchmark times.
 
 "Scaled" cases multiply every q and k row by 10^U(-3,3), with a few rows at 10^{+-6} and
-10^{+-10}, before rounding: the workloads' own rows are unit length, so without these the
-kernels' normalisation (the sphere projection of the review's "Proposed method", step 1)
-and, in the backward, the projection of the gradient onto the sphere's tangent space
-would go unchecked.
+10^{+-10}, before rounding (and the "norm range" cases put rows at both ends of the
+range the library supports, 1e-12 .. 1e15): the workloads' own rows are unit length, so
+without these the kernels' normalisation (the sphere projection of the review's "Proposed
+method", step 1) and, in the backward, the projection of the gradient onto the sphere's
+tangent space would go unchecked.
 """
 import numpy as np
 import pytest
@@ -94,6 +95,40 @@ def test_feature_map(dt_in, dt_out, R, m, n, scaled):
           got, want, tol)
     assert (got[3] == 0).all()
     assert (np.delete(got, 3, axis=0) >= 0).all()
+
+
+# The ends of the row-norm range the library states it supports (1e-12 .. 1e15): the
+# bf16 tensor-core kernels fold 1/|x|^2 into the exponent of phi, which must stay inside
+# fp32's exponent range for every feature; the fp32 kernels normalise first.
+NORM_ENDS = (15.0, 15.0, 14.0, 13.5, 12.0, -11.0, -11.9, -11.9)
+
+
+@pytest.mark.parametrize("dt,R,m", [("bf16", 4, 64), ("bf16", 8, 64), ("bf16", 16, 32),
+                                    ("f32", 8, 64)])
+def test_feature_map_norm_range(dt, R, m):
+    w = small(dt, R, m, 2000, B=1, H=1, seed=23)
+    q, _, _ = W.gen_qkv(w)
+    x = W.scale_rows(w, q.reshape(2000, 64), "q", extremes=NORM_ENDS)
+    P = params(w)
+    want = O.feature_map(x, P)
+    phi = torch.empty((2000, R * m), device="cuda", dtype=TDT[dt])
+    bd.slay_feature_map(dev(x, dt), phi, R, m, w.sketch_seed, _eps(w))
+    bd.slay_kernel_status(None)
+    torch.cuda.synchronize()
+    check("phi norm range %s R%d m%d" % (dt, R, m), host(phi), want, TOL[dt])
+
+
+@pytest.mark.parametrize("dt,R,m,L", [("bf16", 4, 64, 700), ("bf16", 8, 64, 300),
+                                      ("f32", 4, 64, 300)])
+def test_attn_fwd_norm_range(dt, R, m, L):
+    w = small(dt, R, m, L, seed=24)
+    q, k, v = W.gen_qkv(w)
+    q = W.scale_rows(w, q, "q", extremes=NORM_ENDS)
+    k = W.scale_rows(w, k, "k", extremes=NORM_ENDS)
+    P = params(w)
+    want, wden = O.attn_quadratic(q, k, v, P, True)
+    got, gden = _run_fwd(q, k, v, w, True)
+    _check_fwd(tag(w, "causal norm range"), got, gden, want, wden, TOL[dt])
 
 
 # ------------------------------------------------------------ forward
