@@ -170,7 +170,8 @@ def kernel_work(name, w, op):
     # the tensor-core phi backward is bound by its reads: x (bf16), dphi (bf16), dx (fp32);
     # the feature-map backward workload maps q and k rows (2 th rows) in one launch each
     if name == "tc_phi_bwd":
-        return th * (2 * D + 2 * F + 4 * D), "byte", "hbm"
+        rows = 2 * th if op == "feature_map_bwd" else th
+        return rows * (2 * D + 2 * F + 4 * D), "byte", "hbm"
     if name == "simt_bwd_chunk":
         if op == "bidir_bwd":   # S [dn; delta], G [v; 1], G^T phi(k): no masked term
             return th * (2 * F * (Dv + 1) * 2 + 2 * F * Dv), "flop", "alu"

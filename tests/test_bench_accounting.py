@@ -61,6 +61,9 @@ def test_backward_kernels_are_not_chunk_split():
     w = W.FWDBWD_8K
     th = w.B * w.H * w.L
     assert bench.kernel_work("tc_phi_bwd", w, "bwd")[0] == th * (2 * D + 2 * w.F + 4 * D)
+    # the feature-map backward workload maps the q and the k rows in one launch
+    assert bench.kernel_work("tc_phi_bwd", w, "feature_map_bwd")[0] == \
+        2 * th * (2 * D + 2 * w.F + 4 * D)
     tiles = w.B * w.H * ((w.L + 127) // 128)
     states = tiles * 2 * w.F * (DV + 1) * 4
     assert bench.kernel_work("tc_bwd_states", w, "bwd")[0] == \
