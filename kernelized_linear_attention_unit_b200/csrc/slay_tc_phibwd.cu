@@ -19,7 +19,7 @@
 // Persistent, one CTA per SM, 128-row tiles round-robin.  Warp 0 issues every TMA load and
 // MMA; warps 1-8 are the epilogue: warp w serves TMEM lanes 32 (w % 4).. (rows of the tile)
 // and the 32-feature half (w - 1) / 4 of every group.  Per group an epilogue warp reads its
-// projections, its rows' dphi (bf16, prefetched one group ahead) and writes its block of
+// projections, its rows' dphi (bf16, loaded three groups ahead) and writes its block of
 // [alpha | beta] into a K-major 128-byte-swizzled operand tile; per tile it turns dX^ into
 // dx.  Every wait is bounded; a timeout sets the library's feature-map status word.
 #include <cuda.h>
@@ -101,7 +101,8 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
              const __nv_bfloat16* __restrict__ dphi, float* __restrict__ dx, int64_t n_rows,
              PbParams pp, int* status)
 {
-    constexpr int kW = 4;   // 16-byte words per 32 bf16 dphi values
+    constexpr int kW = 4;     // 16-byte words per 32 bf16 dphi values
+    constexpr int kPre = 3;   // dphi groups loaded ahead
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* sm = aligned_smem(smem_raw);
     const PbLayout L = pb_layout(pp.F);
@@ -241,12 +242,25 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
             const int64_t rr = r < n_rows ? r : n_rows - 1;   // rows past the end: any valid row
             return reinterpret_cast<const uint4*>(dphi + rr * F + 64 * g + 32 * half);
         };
-        uint4 dpn[kW];
-        if (nt > 0) {
-            const uint4* p = dphi_ptr(0, 0);
+        // dphi ring: kPre groups in flight ahead of the one being consumed (a warp's 32
+        // rows x 64 bytes per group; at one group ahead the loads' DRAM latency, not the
+        // bandwidth, set the pace).  (fk, fg) is the next job to fetch.
+        uint4 pf[kPre][kW];
+        int fk = 0, fg = 0, fetched = 0;
+        auto fetch = [&](uint4 (&dst)[kW]) {
+            if (fetched < njobs) {
+                const uint4* p = dphi_ptr(fk, fg);
 #pragma unroll
-            for (int i = 0; i < kW; ++i) dpn[i] = __ldg(p + i);
-        }
+                for (int i = 0; i < kW; ++i) dst[i] = __ldg(p + i);
+                if (++fg == ng) {
+                    fg = 0;
+                    ++fk;
+                }
+                ++fetched;
+            }
+        };
+#pragma unroll
+        for (int d = 0; d < kPre; ++d) fetch(pf[d]);
         for (int k = 0; k < nt; ++k) {
             const int s = k % xbufs;
             {
@@ -261,12 +275,12 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
                 const int j = k * ng + g;
                 uint4 dp[kW];
 #pragma unroll
-                for (int i = 0; i < kW; ++i) dp[i] = dpn[i];
-                if (j + 1 < njobs) {   // prefetch the next group's dphi
-                    const uint4* p = dphi_ptr(g + 1 < ng ? k : k + 1, g + 1 < ng ? g + 1 : 0);
+                for (int i = 0; i < kW; ++i) dp[i] = pf[0][i];
 #pragma unroll
-                    for (int i = 0; i < kW; ++i) dpn[i] = __ldg(p + i);
-                }
+                for (int d = 0; d + 1 < kPre; ++d)
+#pragma unroll
+                    for (int i = 0; i < kW; ++i) pf[d][i] = pf[d + 1][i];
+                fetch(pf[kPre - 1]);   // job j + kPre
                 {
                     uint32_t ph = static_cast<uint32_t>((j >> 1) & 1);
                     wt.wait(&bar[PB_UF + (j & 1)], ph);
@@ -323,42 +337,51 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
             reg_fence(d1);
             tc_fence_before();
             warp_arrive(&bar[PB_DE + (k & 1)]);
-            // x^ of this row from the X tile (bf16, 128-byte swizzle): element e of chunk c
-            float xh[64];
+            // x^ of this row from the X tile (bf16, 128-byte swizzle: 16-byte chunk c of the
+            // row at c ^ (row & 7)), read where it is used so that it holds no registers
             const uint4* xr = reinterpret_cast<const uint4*>(xrow);
+            float dot[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 const uint4 w4 = xr[c ^ (row & 7)];
                 const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    xh[8 * c + 2 * e] = __uint_as_float(ws[e] << 16) * inv;
-                    xh[8 * c + 2 * e + 1] = __uint_as_float(ws[e] & 0xFFFF0000u) * inv;
+                    const int i = 8 * c + 2 * e;   // element index 0..63
+                    const float lo = __uint_as_float(ws[e] << 16);
+                    const float hi = __uint_as_float(ws[e] & 0xFFFF0000u);
+                    const float dlo = i < 32 ? __uint_as_float(d0[i]) : __uint_as_float(d1[i - 32]);
+                    const float dhi = i < 32 ? __uint_as_float(d0[i + 1]) : __uint_as_float(d1[i - 31]);
+                    dot[e] = fmaf(lo, dlo, dot[e]);
+                    dot[e] = fmaf(hi, dhi, dot[e]);
                 }
-            }
-            warp_arrive(&bar[PB_XE + s]);   // this warp is done with X slot s
-            float dot[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                dot[c & 3] = fmaf(xh[c], __uint_as_float(d0[c]), dot[c & 3]);
-                dot[c & 3] = fmaf(xh[32 + c], __uint_as_float(d1[c]), dot[c & 3]);
             }
             // below the 1e-12 norm guard x^ = x / 1e-12 is not a unit vector and its
             // derivative is the identity / 1e-12: no tangential projection there
-            const float xd = nrm > 1e-12f ? (dot[0] + dot[1]) + (dot[2] + dot[3]) : 0.0f;
+            const float xd = nrm > 1e-12f ? ((dot[0] + dot[1]) + (dot[2] + dot[3])) * inv : 0.0f;
             const int64_t r = static_cast<int64_t>(k * static_cast<int>(gridDim.x) +
                                                    static_cast<int>(blockIdx.x)) * kRows + row;
             if (r < n_rows) {
                 float4* dst = reinterpret_cast<float4*>(dx + r * 64 + 32 * half);
-                float o[32];
 #pragma unroll
-                for (int c = 0; c < 32; ++c)   // selects, not an indexed pointer (local memory)
-                    o[c] = ((half ? __uint_as_float(d1[c]) : __uint_as_float(d0[c])) -
-                            (half ? xh[32 + c] : xh[c]) * xd) * inv;
+                for (int c = 0; c < 4; ++c) {   // this warp's 32 columns: chunks 4 half .. + 3
+                    const uint4 w4 = xr[(4 * half + c) ^ (row & 7)];
+                    const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
+                    float o[8];
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    dst[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = 8 * c + 2 * e;   // column within the half
+                        // selects, not an indexed pointer (local memory)
+                        const float dlo = half ? __uint_as_float(d1[i]) : __uint_as_float(d0[i]);
+                        const float dhi = half ? __uint_as_float(d1[i + 1]) : __uint_as_float(d0[i + 1]);
+                        o[2 * e] = (dlo - __uint_as_float(ws[e] << 16) * inv * xd) * inv;
+                        o[2 * e + 1] = (dhi - __uint_as_float(ws[e] & 0xFFFF0000u) * inv * xd) * inv;
+                    }
+                    dst[2 * c] = make_float4(o[0], o[1], o[2], o[3]);
+                    dst[2 * c + 1] = make_float4(o[4], o[5], o[6], o[7]);
+                }
             }
+            warp_arrive(&bar[PB_XE + s]);   // this warp is done with X slot s
         }
     }
     wt.report(status);
