@@ -286,8 +286,16 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
             fence_async_smem();
             tc_fence_before();
             warp_arrive(&bar[BW_PCTF]);
-            // per slice: S_s, G_s as bf16 operands (slice s), then the outputs of slice s - 1
-            auto write_slice = [&](int s, int b) {
+            // per slice: S_s, G_s as bf16 operands (slice s), then the outputs of slice s - 1.
+            // The rank-one terms' z_c and zg_c of the warp's 32 features: lane c loads feature
+            // f0 + c (issued ahead of the wait, see load_z) and the warp broadcasts them.
+            const float* zs = Sb + 64 * static_cast<int64_t>(bp.F);   // [e = 64][f]
+            const float* zg = Gb + 64 * static_cast<int64_t>(bp.F);
+            auto load_z = [&](int s, float& zsl, float& zgl) {
+                zsl = zs[64 * s + 32 * half + lane];
+                zgl = zg[64 * s + 32 * half + lane];
+            };
+            auto write_slice = [&](int s, int b, float zsl, float zgl) {
                 wait_k(BW_DQF0 + b, gs >> 1);
                 tc_fence_after();
                 uint32_t qa[32], ka[32];
@@ -299,16 +307,14 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
                 tc_fence_before();
                 warp_arrive(&bar[BW_DQE0 + b]);
                 ++gs;
-                if (!valid) return;
                 const int f0 = 64 * s + 32 * half;
-                const float* zs = Sb + 64 * static_cast<int64_t>(bp.F);   // [e = 64][f]
-                const float* zg = Gb + 64 * static_cast<int64_t>(bp.F);
                 float oq[32], ok[32];
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    oq[c] = fmaf(dl, zs[f0 + c], __uint_as_float(qa[c]));
-                    ok[c] = __uint_as_float(ka[c]) + zg[f0 + c];
+                for (int c = 0; c < 32; ++c) {   // every lane takes part in the broadcasts
+                    oq[c] = fmaf(dl, __shfl_sync(0xffffffffu, zsl, c), __uint_as_float(qa[c]));
+                    ok[c] = __uint_as_float(ka[c]) + __shfl_sync(0xffffffffu, zgl, c);
                 }
+                if (!valid) return;
                 if (bp.dphi_bf16) {
                     uint4* dq4 = reinterpret_cast<uint4*>(static_cast<uint16_t*>(dphq) + grow * bp.F + f0);
                     uint4* dk4 = reinterpret_cast<uint4*>(static_cast<uint16_t*>(dphk) + grow * bp.F + f0);
@@ -344,8 +350,10 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
                 }
             };
             load_sg(0);
+            float zsl = 0.0f, zgl = 0.0f;   // z terms of the slice written next
             for (int s = 0; s < ns; ++s) {
                 const int k = it * ns + s, sb = k & 1;
+                if (s >= 1) load_z(s - 1, zsl, zgl);
                 if (k >= 2) wait_k(BW_SGE0 + sb, (k >> 1) - 1);
                 {
                     uint32_t a8[8], g8[8];
@@ -364,9 +372,10 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
                 fence_async_smem();
                 warp_arrive(&bar[BW_SGF0 + sb]);
                 if (s + 1 < ns) load_sg(s + 1);
-                if (s >= 1) write_slice(s - 1, gs & 1);
+                if (s >= 1) write_slice(s - 1, gs & 1, zsl, zgl);
             }
-            write_slice(ns - 1, gs & 1);
+            load_z(ns - 1, zsl, zgl);
+            write_slice(ns - 1, gs & 1, zsl, zgl);
             // dV
             wait_k(BW_DVF, it);
             tc_fence_after();
