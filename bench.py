@@ -147,6 +147,14 @@ def kernel_work(name, w, op):
         if op == "bidir":
             return th * 2 * F * (Dv + 1), "flop", "alu"
         return th * ((C_CHUNK + 1) * (F + Dv + 1) + 2 * F * (Dv + 1)), "flop", "alu"
+    # the tensor-core backward's scans: both sums' per-tile fp32 slabs read; the causal form
+    # writes each tile's operand (bf16 [F][64]) and z (fp32 [F]) back, the bidirectional form
+    # only the whole-sequence sums
+    if name == "tc_bwd_scan":
+        tiles = w.B * w.H * ((w.L + 127) // 128)
+        rd = 2 * tiles * F * (Dv + 1) * 4
+        wr = 2 * (w.B * w.H if op == "bidir_bwd" else tiles) * F * (Dv * 2 + 4)
+        return rd + wr, "byte", "hbm"
     if name == "simt_scan":
         nc = (w.L + C_CHUNK - 1) // C_CHUNK
         return w.B * w.H * nc * F * (Dv + 1) * 4 * 2, "byte", "hbm"

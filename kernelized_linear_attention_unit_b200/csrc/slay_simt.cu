@@ -1298,15 +1298,19 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
     // bidirectional: the whole-sequence sums, after the causal carve-outs
     float* stot = reinterpret_cast<float*>(w + simt_ws_bwd(B, H, L, kD, F));
     float* gtot = stot + align256(static_cast<size_t>(BH) * FE * sizeof(float)) / sizeof(float);
-    {
-        TraceScope trace_("simt_scan", st);
-        k_scan<<<sgrid, 256, 0, st>>>(sfw, stot, BH, NS, FE, bidir ? 2 : 0);
+    if (tcb) {   // the tile sums scanned into the contraction's bf16 operands (in place)
+        if ((err = tc_bwd_scan(sfw, gbw, stot, gtot, BH, L, F, bidir, st)) != cudaSuccess) return err;
+    } else {
+        {
+            TraceScope trace_("simt_scan", st);
+            k_scan<<<sgrid, 256, 0, st>>>(sfw, stot, BH, NS, FE, bidir ? 2 : 0);
+        }
+        {
+            TraceScope trace_("simt_scan", st);
+            k_scan<<<sgrid, 256, 0, st>>>(gbw, gtot, BH, NS, FE, bidir ? 2 : 1);
+        }
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
     }
-    {
-        TraceScope trace_("simt_scan", st);
-        k_scan<<<sgrid, 256, 0, st>>>(gbw, gtot, BH, NS, FE, bidir ? 2 : 1);
-    }
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
     if (tcb) {
         if ((err = tc_bwd_tile(phq, phk, v, dn16, delta, bidir ? stot : sfw, bidir ? gtot : gbw,
                                dphq, dphk, dphi16, dv, BH, L, F, status, st, bidir)) != cudaSuccess)

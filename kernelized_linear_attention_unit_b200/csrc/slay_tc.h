@@ -38,7 +38,13 @@ bool tc_bwd_tile_supported(int F, int L);
 cudaError_t tc_bwd_states(const void* phq, const void* phk, const void* v, const void* dn16,
                           const float* delta, float* st_s, float* st_g, int BH, int L, int F,
                           int* err, cudaStream_t st);
+// The per-tile sums of tc_bwd_states scanned over each sequence's tiles (S forward, G
+// backward, exclusive) and rewritten in place as the contraction's bf16 operands and fp32 z;
+// bidir: the whole-sequence sums into tot_s, tot_g instead (BH x F x 65 floats each).
+cudaError_t tc_bwd_scan(float* st_s, float* st_g, float* tot_s, float* tot_g, int BH, int L, int F,
+                        bool bidir, cudaStream_t st);
 // bidir: the bidirectional form (no masked term; sfw, gbw are each sequence's whole sums).
+// sfw, gbw hold tc_bwd_scan's operands.
 cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const void* dn16,
                         const float* delta, const float* sfw, const float* gbw, void* dphq,
                         void* dphk, bool dphi_bf16, float* dv, int BH, int L, int F, int* err,

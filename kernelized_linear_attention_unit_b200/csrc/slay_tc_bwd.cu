@@ -46,6 +46,11 @@ constexpr int kT = 128;                  // tokens per tile
 constexpr int kTile = kT * 128;          // [128][64] bf16, 128-byte swizzle = 16 KiB
 constexpr int kSG = 64 * 128;            // [64 f][64 e] bf16 = 8 KiB
 constexpr int kE = 65;                   // state / [dn | delta] columns in the scans' layout
+// The per-tile sums are stored per 64-feature slab: [65 e][64 f] fp32 (kSlabF floats).  The
+// scan rewrites each slab in place as the contraction's operand: [64 f][64 e] bf16 (8 KiB,
+// loaded by TMA) followed by z (e = 64) as fp32 [64 f] at float offset kZOff.
+constexpr int kSlabF = 64 * kE;
+constexpr int kZOff = 64 * 64 / 2;
 constexpr int kBwThreads = 32 * 10;
 constexpr int kNumSMs = 148;
 // tensor memory: phase A P [0,128) and C0 [128,256); phase B per-slice buffers b: dphiQ at
@@ -87,6 +92,7 @@ struct BwParams {
 __global__ void __launch_bounds__(kBwThreads, 1)
 k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
               const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdn,
+              const __grid_constant__ CUtensorMap tms, const __grid_constant__ CUtensorMap tmg,
               const float* __restrict__ delta, const float* __restrict__ sfw,
               const float* __restrict__ gbw,
               void* __restrict__ dphq, void* __restrict__ dphk, float* __restrict__ dv,
@@ -107,13 +113,15 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
     }
     if (tid == 0) {
         for (int i = 0; i < BW_NUM; ++i) mbar_init(&bar[i], 1);
-        const int warp_counted[6] = {BW_PCTF, BW_SGF0, BW_SGF1, BW_DQE0, BW_DQE1, BW_DVE};
-        for (int i = 0; i < 6; ++i) mbar_init(&bar[warp_counted[i]], 8);   // one arrival per epilogue warp
+        const int warp_counted[4] = {BW_PCTF, BW_DQE0, BW_DQE1, BW_DVE};
+        for (int i = 0; i < 4; ++i) mbar_init(&bar[warp_counted[i]], 8);   // one arrival per epilogue warp
         mbar_fence_init();
         tma_prefetch_desc(&tmq);
         tma_prefetch_desc(&tmk);
         tma_prefetch_desc(&tmv);
         tma_prefetch_desc(&tmdn);
+        tma_prefetch_desc(&tms);
+        tma_prefetch_desc(&tmg);
     }
     tc_fence_before();
     __syncthreads();
@@ -136,8 +144,18 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
                 mbar_arrive_expect_tx(&bar[BW_VF], 2 * kTile);   // V and dn
                 tma_load_3d(sm + Lo.v, &tmv, &bar[BW_VF], 0, t * kT, bh);
                 tma_load_3d(sm + Lo.dn, &tmdn, &bar[BW_VF], 0, t * kT, bh);
+                // operand slab of slice s: tile t's (bidirectional: the sequence's) slab s
+                const int64_t slab0 = (bp.bidir ? static_cast<int64_t>(bh) : static_cast<int64_t>(bh) * bp.ntiles + t) * ns;
                 for (int u = 0; u < 2 * ns; ++u, ++use) {   // phase A slices, then phase B
                     const int s = u < ns ? u : u - ns, slot = use & 1;
+                    if (u >= ns) {   // S_s and G_s for phase B (buffer of slice k = it ns + s)
+                        const int k = it * ns + s, sb = k & 1;
+                        if (k >= 2) wait_k(BW_SGE0 + sb, (k >> 1) - 1);
+                        mbar_arrive_expect_tx(&bar[BW_SGF0 + sb], 2 * kSG);
+                        unsigned char* sgd = sm + Lo.sg + sb * 2 * kSG;
+                        tma_load_3d(sgd, &tms, &bar[BW_SGF0 + sb], 0, 0, static_cast<int>(slab0 + s));
+                        tma_load_3d(sgd + kSG, &tmg, &bar[BW_SGF0 + sb], 0, 0, static_cast<int>(slab0 + s));
+                    }
                     if (use >= 2) wait_k(BW_PE0 + slot, (use >> 1) - 1);
                     mbar_arrive_expect_tx(&bar[BW_PF0 + slot], 2 * kTile);
                     unsigned char* dst = sm + Lo.phi + slot * 2 * kTile;
@@ -228,7 +246,7 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
         __syncwarp();
     } else {
         // ---------------------------------------------------------------- epilogue
-        const int ew = warp - 1, q = warp & 3, half = ew >> 2, et = tid - 32;   // et 0..255
+        const int ew = warp - 1, q = warp & 3, half = ew >> 2;
         const uint32_t row = 32u * q + lane;
         const uint32_t trow = tmem + ((32u * q) << 16);
         int it = 0, gs = 0;
@@ -286,14 +304,12 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
             fence_async_smem();
             tc_fence_before();
             warp_arrive(&bar[BW_PCTF]);
-            // per slice: S_s, G_s as bf16 operands (slice s), then the outputs of slice s - 1.
-            // The rank-one terms' z_c and zg_c of the warp's 32 features: lane c loads feature
-            // f0 + c (issued ahead of the wait, see load_z) and the warp broadcasts them.
-            const float* zs = Sb + 64 * static_cast<int64_t>(bp.F);   // [e = 64][f]
-            const float* zg = Gb + 64 * static_cast<int64_t>(bp.F);
+            // per slice the outputs (S_s and G_s reach the MMAs by TMA, already bf16).  The
+            // rank-one terms' z_c and zg_c of the warp's 32 features: lane c loads feature
+            // f0 + c from the slab's fp32 z (a slice ahead) and the warp broadcasts them.
             auto load_z = [&](int s, float& zsl, float& zgl) {
-                zsl = zs[64 * s + 32 * half + lane];
-                zgl = zg[64 * s + 32 * half + lane];
+                zsl = Sb[static_cast<int64_t>(s) * kSlabF + kZOff + 32 * half + lane];
+                zgl = Gb[static_cast<int64_t>(s) * kSlabF + kZOff + 32 * half + lane];
             };
             auto write_slice = [&](int s, int b, float zsl, float zgl) {
                 wait_k(BW_DQF0 + b, gs >> 1);
@@ -335,47 +351,14 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
                     }
                 }
             };
-            // thread et converts 16 e of feature f = et % 64 of S_s and of G_s (the sums are
-            // e-major: a warp's loads cover 32 consecutive features); the next slice's values
-            // are loaded while the previous slice's outputs are written
-            const int sf = et & 63, se0 = 16 * (et >> 6);
-            float sv[16], gv[16];
-            auto load_sg = [&](int s) {
-                const float* sr = Sb + static_cast<int64_t>(se0) * bp.F + 64 * s + sf;
-                const float* gr = Gb + static_cast<int64_t>(se0) * bp.F + 64 * s + sf;
-#pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    sv[c] = sr[c * static_cast<int64_t>(bp.F)];
-                    gv[c] = gr[c * static_cast<int64_t>(bp.F)];
-                }
-            };
-            load_sg(0);
-            float zsl = 0.0f, zgl = 0.0f;   // z terms of the slice written next
+            float zsl, zgl, zsn = 0.0f, zgn = 0.0f;
+            load_z(0, zsl, zgl);
             for (int s = 0; s < ns; ++s) {
-                const int k = it * ns + s, sb = k & 1;
-                if (s >= 1) load_z(s - 1, zsl, zgl);
-                if (k >= 2) wait_k(BW_SGE0 + sb, (k >> 1) - 1);
-                {
-                    uint32_t a8[8], g8[8];
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        a8[c] = pack_bf16(sv[2 * c], sv[2 * c + 1]);
-                        g8[c] = pack_bf16(gv[2 * c], gv[2 * c + 1]);
-                    }
-                    const uint32_t ts = sbase + Lo.sg + sb * 2 * kSG, tg = ts + kSG;
-                    const int ch = 2 * (et >> 6);
-                    st_shared_v4(ts + sw128_off(sf, ch), a8[0], a8[1], a8[2], a8[3]);
-                    st_shared_v4(ts + sw128_off(sf, ch + 1), a8[4], a8[5], a8[6], a8[7]);
-                    st_shared_v4(tg + sw128_off(sf, ch), g8[0], g8[1], g8[2], g8[3]);
-                    st_shared_v4(tg + sw128_off(sf, ch + 1), g8[4], g8[5], g8[6], g8[7]);
-                }
-                fence_async_smem();
-                warp_arrive(&bar[BW_SGF0 + sb]);
-                if (s + 1 < ns) load_sg(s + 1);
-                if (s >= 1) write_slice(s - 1, gs & 1, zsl, zgl);
+                if (s + 1 < ns) load_z(s + 1, zsn, zgn);
+                write_slice(s, gs & 1, zsl, zgl);
+                zsl = zsn;
+                zgl = zgn;
             }
-            load_z(ns - 1, zsl, zgl);
-            write_slice(ns - 1, gs & 1, zsl, zgl);
             // dV
             wait_k(BW_DVF, it);
             tc_fence_after();
@@ -404,10 +387,11 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
 }
 
 // ------------------------------------------------------------------ tile states
-// Per 128-token tile t of sequence bh: st_s[bh][t][e][f] = sum_{j in t} phi(k_j)_f [v_j, 1]_e
-// and st_g[bh][t][e][f] = sum_{i in t} phi(q_i)_f [dn_i, delta_i]_e (fp32, e = 64 the last
-// row; e-major so that a warp's 32 features store contiguously), the inputs of the
-// exclusive scans (element-wise over a tile's block) that give the contraction S_c and G_c.
+// Per 128-token tile t of sequence bh: st_s[bh][t][slab][e][f] = sum_{j in t} phi(k_j)_f
+// [v_j, 1]_e and st_g[bh][t][slab][e][f] = sum_{i in t} phi(q_i)_f [dn_i, delta_i]_e (fp32,
+// 64-feature slabs, e = 64 the last row; e-major inside a slab so that a warp's 32 features
+// store contiguously), the inputs of the scans (k_scan_slabs) that give the contraction S_c
+// and G_c.
 // Per item and 128-feature block mb: S = phiK_mb^T [V | 1] and G = phiQ_mb^T [dn | delta]
 // (M = 128 features, N = 80, K = 128 tokens), phi read as an MN-major A operand (two 64-
 // feature tiles), the extra column through a second 64-wide tile at the operand's leading
@@ -578,17 +562,19 @@ k_tc_bwd_states(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 reg_fence1(gz);
                 tc_fence_before();
                 warp_arrive(&bar[ST_DE0 + b]);
+                // slab f / 64, element (e, f % 64) at e * 64 + f % 64: for each e a warp's 32
+                // consecutive features store 128 contiguous bytes
                 const int f = 128 * mb + static_cast<int>(row);
                 const int64_t o = (static_cast<int64_t>(bh) * bp.ntiles + t) * bp.F * kE +
-                                  static_cast<int64_t>(32 * half) * bp.F + f;
+                                  static_cast<int64_t>(f >> 6) * kSlabF + 64 * (32 * half) + (f & 63);
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
-                    st_s[o + static_cast<int64_t>(c) * bp.F] = __uint_as_float(sa[c]);
-                    st_g[o + static_cast<int64_t>(c) * bp.F] = __uint_as_float(ga[c]);
+                    st_s[o + 64 * c] = __uint_as_float(sa[c]);
+                    st_g[o + 64 * c] = __uint_as_float(ga[c]);
                 }
                 if (half) {
-                    st_s[o + 32 * static_cast<int64_t>(bp.F)] = __uint_as_float(sz);
-                    st_g[o + 32 * static_cast<int64_t>(bp.F)] = __uint_as_float(gz);
+                    st_s[o + 64 * 32] = __uint_as_float(sz);
+                    st_g[o + 64 * 32] = __uint_as_float(gz);
                 }
             }
         }
@@ -598,6 +584,80 @@ k_tc_bwd_states(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------------ scans over tiles
+// One CTA per (sequence bh, 64-feature slab) and sum (blockIdx.y: 0 = S, 1 = G): walks the
+// sequence's tiles in order (S: forward; G: backward) keeping fp32 running sums and writes,
+// over each tile's slab, the sum over the tiles before it (S_c) or after it (G_c) -- the
+// exclusive prefix / suffix -- as the contraction's operand: [64 f][64 e] bf16 and z fp32.
+// total != 0 (the bidirectional form): the whole-sequence sums instead, written once to
+// tot_s / tot_g ([BH][slabs] slabs of the same form); the per-tile sums are left as they are.
+// Thread: feature fl = tid % 64 and the 16 e of group eg = tid / 64 (group 3 also e = 64),
+// so its operand row piece is 32 contiguous bytes.  A tile's sums are all in registers (and
+// added) before the barrier after which its slab is overwritten.
+constexpr int kScanThreads = 256;
+
+__global__ void __launch_bounds__(kScanThreads)
+k_scan_slabs(float* __restrict__ st_s, float* __restrict__ st_g, float* __restrict__ tot_s,
+             float* __restrict__ tot_g, int NS, int nsl, int total)
+{
+    const int which = blockIdx.y;
+    const int bh = static_cast<int>(blockIdx.x) / nsl, slab = static_cast<int>(blockIdx.x) - bh * nsl;
+    float* base = (which ? st_g : st_s) + (static_cast<int64_t>(bh) * NS * nsl + slab) * kSlabF;
+    const int64_t tstride = static_cast<int64_t>(nsl) * kSlabF;   // floats from tile to tile
+    const int fl = threadIdx.x & 63, eg = threadIdx.x >> 6;
+    const bool hasz = eg == 3;
+    const bool rev = !total && which == 1;
+    float run[17], x[17];
+#pragma unroll
+    for (int c = 0; c < 17; ++c) run[c] = 0.0f;
+    auto load = [&](int t) {
+        const float* p = base + t * tstride + (16 * eg) * 64 + fl;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) x[c] = p[64 * c];
+        x[16] = hasz ? base[t * tstride + 64 * 64 + fl] : 0.0f;
+    };
+    auto store = [&](float* slab_base, const float (&val)[17]) {
+        uint4* op = reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(slab_base) + fl * 128 + 32 * eg);
+        op[0] = make_uint4(pack_bf16(val[0], val[1]), pack_bf16(val[2], val[3]),
+                           pack_bf16(val[4], val[5]), pack_bf16(val[6], val[7]));
+        op[1] = make_uint4(pack_bf16(val[8], val[9]), pack_bf16(val[10], val[11]),
+                           pack_bf16(val[12], val[13]), pack_bf16(val[14], val[15]));
+        if (hasz) slab_base[kZOff + fl] = val[16];
+    };
+    const int t0 = rev ? NS - 1 : 0, step = rev ? -1 : 1;
+    load(t0);
+    for (int i = 0; i < NS; ++i) {
+        const int t = t0 + i * step;
+        float out[17];
+#pragma unroll
+        for (int c = 0; c < 17; ++c) {
+            out[c] = run[c];
+            run[c] += x[c];
+        }
+        if (i + 1 < NS) load(t + step);   // the next tile's sums, in flight during the stores
+        if (!total) {
+            __syncthreads();   // every thread has added tile t's sums: its slab may be overwritten
+            store(base + t * tstride, out);
+        }
+    }
+    if (total) store((which ? tot_g : tot_s) + (static_cast<int64_t>(bh) * nsl + slab) * kSlabF, run);
+}
+
+// Operand slabs ([nslabs] x [64 f][64 e] bf16, kSlabF floats apart) viewed as a 3-D tensor,
+// one [64][64] box per slab, 128-byte swizzle.
+bool map_slabs(CUtensorMap* m, const float* base, int64_t nslabs)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {64, 64, static_cast<cuuint64_t>(nslabs)};
+    const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(kSlabF) * 4};
+    const cuuint32_t box[3] = {64, 64, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<float*>(base), dims, strides, box,
+              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // [BH][L][cols] bf16 viewed as a 3-D tensor, boxes of 64 columns x 128 tokens, 128-byte
@@ -668,14 +728,29 @@ cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const v
     bp.nitems = BH * bp.ntiles;
     bp.dphi_bf16 = dphi_bf16 ? 1 : 0;
     bp.bidir = bidir ? 1 : 0;
+    // the operand slabs the scans wrote: per tile (causal) or per sequence (bidirectional)
+    const int64_t nslabs = static_cast<int64_t>(BH) * (bidir ? 1 : bp.ntiles) * (F / 64);
+    CUtensorMap ms, mg;
+    if (!map_slabs(&ms, sfw, nslabs) || !map_slabs(&mg, gbw, nslabs)) return cudaErrorInvalidValue;
     const size_t smem = bw_layout().total + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_tc_bwd_tile, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     const int grid = bp.nitems < kNumSMs ? bp.nitems : kNumSMs;
     TraceScope trace_("tc_bwd_tile", st);
-    k_tc_bwd_tile<<<grid, kBwThreads, smem, st>>>(mq, mk, mv, mdn, delta, sfw, gbw, dphq, dphk, dv, bp,
-                                                  err);
+    k_tc_bwd_tile<<<grid, kBwThreads, smem, st>>>(mq, mk, mv, mdn, ms, mg, delta, sfw, gbw, dphq, dphk,
+                                                  dv, bp, err);
+    return cudaGetLastError();
+}
+
+cudaError_t tc_bwd_scan(float* st_s, float* st_g, float* tot_s, float* tot_g, int BH, int L, int F,
+                        bool bidir, cudaStream_t st)
+{
+    if (!tc_bwd_tile_supported(F, L)) return cudaErrorNotSupported;
+    const int NS = (L + kT - 1) / kT, nsl = F / 64;
+    TraceScope trace_("tc_bwd_scan", st);
+    k_scan_slabs<<<dim3(static_cast<unsigned>(BH * nsl), 2), kScanThreads, 0, st>>>(
+        st_s, st_g, tot_s, tot_g, NS, nsl, bidir ? 1 : 0);
     return cudaGetLastError();
 }
 

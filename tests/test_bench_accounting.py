@@ -66,6 +66,8 @@ def test_backward_kernels_are_not_chunk_split():
         2 * th * (2 * D + 2 * w.F + 4 * D)
     tiles = w.B * w.H * ((w.L + 127) // 128)
     states = tiles * 2 * w.F * (DV + 1) * 4
+    # the scans read both sums' fp32 slabs and write the bf16 operands and fp32 z
+    assert bench.kernel_work("tc_bwd_scan", w, "bwd")[0] == states + tiles * 2 * w.F * (DV * 2 + 4)
     assert bench.kernel_work("tc_bwd_states", w, "bwd")[0] == \
         th * (2 * 2 * w.F + 2 * DV + 4 * (DV + 1)) + states
     # the contraction by its flops: three products with the scanned sums (2 F Dv each) and
