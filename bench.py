@@ -147,12 +147,12 @@ def kernel_work(name, w, op):
         if op == "bidir":
             return th * 2 * F * (Dv + 1), "flop", "alu"
         return th * ((C_CHUNK + 1) * (F + Dv + 1) + 2 * F * (Dv + 1)), "flop", "alu"
-    # the tensor-core backward's scans: both sums' per-tile fp32 slabs read; the causal form
-    # writes each tile's operand (bf16 [F][64]) and z (fp32 [F]) back, the bidirectional form
-    # only the whole-sequence sums
-    if name == "tc_bwd_scan":
+    # the tensor-core backward's running sums: phi(q), phi(k) (bf16) and v, dn read once; the
+    # causal form writes every tile's operands (bf16 [F][64] and fp32 z, for S and for G), the
+    # bidirectional form the whole-sequence sums only
+    if name == "tc_bwd_sums":
         tiles = w.B * w.H * ((w.L + 127) // 128)
-        rd = 2 * tiles * F * (Dv + 1) * 4
+        rd = th * (2 * F * 2 + 2 * Dv * 2)
         wr = 2 * (w.B * w.H if op == "bidir_bwd" else tiles) * F * (Dv * 2 + 4)
         return rd + wr, "byte", "hbm"
     if name == "simt_scan":
@@ -164,11 +164,6 @@ def kernel_work(name, w, op):
     # kernel the rest; the row statistics read out, g, den and write [dn, delta] (bytes)
     if name == "simt_phi_bwd":
         return th * 8 * D * F, "flop", "alu"
-    # the backward's per-tile sums read phi(q), phi(k), v, [dn, delta] and write two fp32
-    # [F][Dv+1] sums per 128-token tile
-    if name == "tc_bwd_states":
-        return th * (2 * 2 * F + 2 * Dv + 4 * (Dv + 1)) + \
-            w.B * w.H * ((w.L + 127) // 128) * 2 * F * (Dv + 1) * 4, "byte", "hbm"
     # the tensor-core chunk contraction of the backward, by its algorithmic flops per
     # token-head: the three products with the scanned sums (dphi(q) = S dn, dphi(k) = G v,
     # dv = G^T phi(k): 2 F Dv each) and the masked intra-tile terms (scores and c_ij, the

@@ -1276,11 +1276,7 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
     const bool dphi16 = (tcb || bidir) && tcp;
     const int NS = tcb ? (L + 127) / 128 : NC;   // state blocks per sequence
     int* status = reinterpret_cast<int*>(w - kWsHeader);
-    if (tcb) {
-        if ((err = tc_bwd_states(phq, phk, v, dn16, delta, sfw, gbw, BH, L, F, status, st)) !=
-            cudaSuccess)
-            return err;
-    } else {
+    if (!tcb) {   // (tensor-core path: the running sums below, after the total buffers)
         const dim3 sg((F + C - 1) / C, NC, BH);
         {
             TraceScope trace_("simt_chunk_state", st);
@@ -1298,8 +1294,10 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
     // bidirectional: the whole-sequence sums, after the causal carve-outs
     float* stot = reinterpret_cast<float*>(w + simt_ws_bwd(B, H, L, kD, F));
     float* gtot = stot + align256(static_cast<size_t>(BH) * FE * sizeof(float)) / sizeof(float);
-    if (tcb) {   // the tile sums scanned into the contraction's bf16 operands (in place)
-        if ((err = tc_bwd_scan(sfw, gbw, stot, gtot, BH, L, F, bidir, st)) != cudaSuccess) return err;
+    if (tcb) {   // running sums over the tiles, written as the contraction's bf16 operands
+        if ((err = tc_bwd_sums(phq, phk, v, dn16, delta, sfw, gbw, stot, gtot, BH, L, F, bidir,
+                               status, st)) != cudaSuccess)
+            return err;
     } else {
         {
             TraceScope trace_("simt_scan", st);

@@ -32,19 +32,18 @@ bool tc_phi_bwd_supported(int D, int R, int m, int64_t n_rows);
 cudaError_t tc_phi_bwd(const void* x, const void* dphi, float* dx, int64_t n, const Params& P,
                        cudaStream_t st);
 // Causal backward on tensor cores over 128-token tiles (bf16 phi, v and dn rows, fp32 delta):
-// the per-tile sums phi(k)^T [v, 1] and phi(q)^T [dn, delta] ([BH][tiles][65][F] fp32), and,
-// from their exclusive forward / reverse scans, the contraction -> dphi(q), dphi(k), dv.
+// the sums of phi(k) [v, 1] over the tokens before each tile and of phi(q) [dn, delta] over
+// the tokens after it, then the contraction -> dphi(q), dphi(k), dv.
 bool tc_bwd_tile_supported(int F, int L);
-cudaError_t tc_bwd_states(const void* phq, const void* phk, const void* v, const void* dn16,
-                          const float* delta, float* st_s, float* st_g, int BH, int L, int F,
-                          int* err, cudaStream_t st);
-// The per-tile sums of tc_bwd_states scanned over each sequence's tiles (S forward, G
-// backward, exclusive) and rewritten in place as the contraction's bf16 operands and fp32 z;
-// bidir: the whole-sequence sums into tot_s, tot_g instead (BH x F x 65 floats each).
-cudaError_t tc_bwd_scan(float* st_s, float* st_g, float* tot_s, float* tot_g, int BH, int L, int F,
-                        bool bidir, cudaStream_t st);
+// The contraction's S_c and G_c in one launch: per (sequence, 128-feature block, sum) the
+// tiles walked in order with the running sums on chip, written per tile as the contraction's
+// operand slabs: [64 f][64 e] bf16 and z fp32 per 64 features, 65 x 64 floats apart (bidir:
+// the whole-sequence sums into tot_s, tot_g).
+cudaError_t tc_bwd_sums(const void* phq, const void* phk, const void* v, const void* dn16,
+                        const float* delta, float* st_s, float* st_g, float* tot_s, float* tot_g,
+                        int BH, int L, int F, bool bidir, int* err, cudaStream_t st);
 // bidir: the bidirectional form (no masked term; sfw, gbw are each sequence's whole sums).
-// sfw, gbw hold tc_bwd_scan's operands.
+// sfw, gbw hold tc_bwd_sums' operands.
 cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const void* dn16,
                         const float* delta, const float* sfw, const float* gbw, void* dphq,
                         void* dphk, bool dphi_bf16, float* dv, int BH, int L, int F, int* err,

@@ -9,8 +9,8 @@
 //   dphi(k_j) = sum_i c_ij phi(q_i) + G_c[:, :64] v_j + zg_c
 //   dv_j      = sum_i P_ij dn_i + G_c[:, :64]^T phi(k_j)
 // where [S_c | z_c] = sum over earlier tokens of phi(k) [v, 1] (the state entering the tile)
-// and [G_c | zg_c] = sum over later tokens of phi(q) [dn, delta]: the exclusive forward and
-// reverse scans of the per-tile sums that k_tc_bwd_states computes.
+// and [G_c | zg_c] = sum over later tokens of phi(q) [dn, delta], which k_tc_bwd_sums writes
+// per tile as bf16 operands (and z in fp32).
 //
 // Per tile (M = 128 rows, all MMAs kind::f16, fp32 accumulators in tensor memory):
 //   phase A: P = sum_s phiQ_s phiK_s^T (64-feature slices s), C0 = dn V^T;
@@ -45,10 +45,10 @@ namespace {
 constexpr int kT = 128;                  // tokens per tile
 constexpr int kTile = kT * 128;          // [128][64] bf16, 128-byte swizzle = 16 KiB
 constexpr int kSG = 64 * 128;            // [64 f][64 e] bf16 = 8 KiB
-constexpr int kE = 65;                   // state / [dn | delta] columns in the scans' layout
-// The per-tile sums are stored per 64-feature slab: [65 e][64 f] fp32 (kSlabF floats).  The
-// scan rewrites each slab in place as the contraction's operand: [64 f][64 e] bf16 (8 KiB,
-// loaded by TMA) followed by z (e = 64) as fp32 [64 f] at float offset kZOff.
+constexpr int kE = 65;                   // [S | z] / [G | zg] columns
+// The sums reach the contraction per 64-feature slab, kSlabF floats apart (the workspace is
+// sized for fp32 [65][64] slabs): [64 f][64 e] bf16 (8 KiB, loaded by TMA) followed by z
+// (e = 64) as fp32 [64 f] at float offset kZOff.
 constexpr int kSlabF = 64 * kE;
 constexpr int kZOff = 64 * 64 / 2;
 constexpr int kBwThreads = 32 * 10;
@@ -86,7 +86,7 @@ struct BwParams {
     int L, F, ntiles, nitems;
     int dphi_bf16;   // contraction: store dphi(q), dphi(k) as bf16 (else fp32)
     int bidir;       // contraction: the bidirectional form (no masked intra-tile term; sfw,
-                     // gbw hold each sequence's whole sums [BH][65][F], not per-tile scans)
+                     // gbw hold each sequence's whole sums, not each tile's)
 };
 
 __global__ void __launch_bounds__(kBwThreads, 1)
@@ -386,77 +386,78 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-// ------------------------------------------------------------------ tile states
-// Per 128-token tile t of sequence bh: st_s[bh][t][slab][e][f] = sum_{j in t} phi(k_j)_f
-// [v_j, 1]_e and st_g[bh][t][slab][e][f] = sum_{i in t} phi(q_i)_f [dn_i, delta_i]_e (fp32,
-// 64-feature slabs, e = 64 the last row; e-major inside a slab so that a warp's 32 features
-// store contiguously), the inputs of the scans (k_scan_slabs) that give the contraction S_c
-// and G_c.
-// Per item and 128-feature block mb: S = phiK_mb^T [V | 1] and G = phiQ_mb^T [dn | delta]
-// (M = 128 features, N = 80, K = 128 tokens), phi read as an MN-major A operand (two 64-
-// feature tiles), the extra column through a second 64-wide tile at the operand's leading
-// byte offset: constant ones for [V | 1], delta_i in every column for [dn | delta].
-// Warp 0 issues the MMAs, warp 9 the TMA loads (V and the bf16 dn rows with them), warps 1-8
-// write delta into the extension tile and store the sums (lane quadrant w % 4 = 32
-// features, half (w - 1) / 4 of the columns).
-constexpr int kStThreads = 32 * 10;
+// ------------------------------------------------------------ running sums over tiles
+// The contraction's S_c and G_c directly: one CTA per (sequence bh, 128-feature block mb,
+// sum: blockIdx.x & 1 == 0 S, 1 G) walks the sequence's tiles (S forward, G backward),
+// accumulates each tile's sum -- S_t = phiK_mb^T [V | 1], G_t = phiQ_mb^T [dn | delta] (M = 128
+// features, N = 80, K = 128 tokens, phi read as an MN-major A operand, the extra column
+// through a second tile at the B operand's leading-byte offset: constant ones, or delta in
+// every column) -- into fp32 running sums held by the epilogue threads, and writes, per tile,
+// the sum over the tiles before it (S) or after it (G) as an operand slab: [64 f][64 e] bf16
+// and z fp32 (the form k_tc_bwd_tile loads by TMA).  total != 0 (bidirectional): only the
+// whole-sequence sums, into tot_s / tot_g.  Tiles stream through two slots (phi block, V or
+// dn, the extension tile) and two accumulators, so tile i + 1's MMAs run while tile i's sums
+// are read.  Warp 0 issues the MMAs, warp 9 the TMA loads, warps 1-8 are the epilogue (lane
+// quadrant w % 4 = 32 features, e half (w - 1) / 4; half 1 also e = 64) and, for G, write
+// delta into the extension tile (row = token).
+constexpr int kSumThreads = 32 * 10;
 
-enum {
-    ST_VF = 0, ST_VE, ST_PF0, ST_PF1, ST_PE0, ST_PE1, ST_YF, ST_YE, ST_DF0, ST_DF1, ST_DE0, ST_DE1,
-    ST_NUM
+enum { SU_PF0 = 0, SU_PF1, SU_PE0, SU_PE1, SU_XF0, SU_XF1, SU_DF0, SU_DF1, SU_DE0, SU_DE1, SU_NUM };
+
+struct SuLayout {
+    uint32_t phi, y, bar, tmem, total;
 };
 
-struct StLayout {
-    uint32_t phi, v, ones, dn, dl, bar, tmem, total;
-};
-
-__host__ __device__ inline StLayout st_layout()
+__host__ __device__ inline SuLayout su_layout()
 {
-    StLayout l;
-    l.phi = 0;                   // 2 slots x (phiQ 2 tiles, phiK 2 tiles) of one feature block
-    l.v = l.phi + 8 * kTile;
-    l.ones = l.v + kTile;        // right after V: [V | 1] at LBO = kTile
-    l.dn = l.ones + kTile;       // dn (TMA, with V)
-    l.dl = l.dn + kTile;         // right after dn: [dn | delta] at LBO = kTile
-    l.bar = l.dl + kTile;
-    l.tmem = l.bar + ST_NUM * 8;
+    SuLayout l;
+    l.phi = 0;                    // 2 slots x (two 64-feature tiles of the block)
+    l.y = l.phi + 4 * kTile;      // 2 slots x (V or dn tile, then its extension tile at LBO)
+    l.bar = l.y + 4 * kTile;
+    l.tmem = l.bar + SU_NUM * 8;
     l.total = l.tmem + 16;
     return l;
 }
 
-__global__ void __launch_bounds__(kStThreads, 1)
-k_tc_bwd_states(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdn,
-                const float* __restrict__ delta, float* __restrict__ st_s, float* __restrict__ st_g,
-                BwParams bp, int* err)
+__global__ void __launch_bounds__(kSumThreads, 1)
+k_tc_bwd_sums(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+              const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdn,
+              const float* __restrict__ delta, float* __restrict__ st_s, float* __restrict__ st_g,
+              float* __restrict__ tot_s, float* __restrict__ tot_g, BwParams bp, int* err)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* sm = aligned_smem(smem_raw);
-    const StLayout Lo = st_layout();
+    const SuLayout Lo = su_layout();
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Lo.bar);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + Lo.tmem);
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int nb = bp.F / 128;                  // 128-feature blocks (jobs per item)
+    const int nb = bp.F / 128, NS = bp.ntiles, nsl = bp.F / 64;
+    const int g = static_cast<int>(blockIdx.x) & 1;   // 0: S (keys, forward), 1: G (queries, backward)
+    const int job = static_cast<int>(blockIdx.x) >> 1;
+    const int bh = job / nb, mb = job - bh * nb;
+    const bool total = bp.bidir != 0;
+    auto tile_of = [&](int i) { return (g && !total) ? NS - 1 - i : i; };
 
     if (warp == 0) {
-        tmem_alloc(tslot, 512);
+        tmem_alloc(tslot, 256);
         tmem_relinquish();
     }
-    {   // bf16 ones (the extra column of [V | 1], replicated over the tile)
-        uint32_t* p = reinterpret_cast<uint32_t*>(sm + Lo.ones);
-        for (int i = tid; i < kTile / 4; i += blockDim.x) p[i] = 0x3F803F80u;
+    if (!g) {   // S: the extension tiles are constant bf16 ones
+        for (int b = 0; b < 2; ++b) {
+            uint32_t* p = reinterpret_cast<uint32_t*>(sm + Lo.y + (2 * b + 1) * kTile);
+            for (int i = tid; i < kTile / 4; i += blockDim.x) p[i] = 0x3F803F80u;
+        }
     }
     if (tid == 0) {
-        for (int i = 0; i < ST_NUM; ++i) mbar_init(&bar[i], 1);
-        mbar_init(&bar[ST_YF], 8);
-        mbar_init(&bar[ST_DE0], 8);
-        mbar_init(&bar[ST_DE1], 8);
+        for (int i = 0; i < SU_NUM; ++i) mbar_init(&bar[i], 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bar[SU_XF0 + b], 8);
+            mbar_init(&bar[SU_DE0 + b], 8);
+        }
         mbar_fence_init();
-        tma_prefetch_desc(&tmq);
-        tma_prefetch_desc(&tmk);
-        tma_prefetch_desc(&tmv);
-        tma_prefetch_desc(&tmdn);
+        tma_prefetch_desc(g ? &tmq : &tmk);
+        tma_prefetch_desc(g ? &tmdn : &tmv);
     }
     fence_async_smem();
     tc_fence_before();
@@ -471,23 +472,16 @@ k_tc_bwd_states(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
 
     if (warp == 9) {
         if (lane == 0) {
-            int use = 0, it = 0;
-            for (int item = blockIdx.x; item < bp.nitems && wt.ok; item += gridDim.x, ++it) {
-                const int bh = item / bp.ntiles, t = item - bh * bp.ntiles;
-                if (it >= 1) wait_k(ST_VE, it - 1);
-                mbar_arrive_expect_tx(&bar[ST_VF], 2 * kTile);   // V and dn
-                tma_load_3d(sm + Lo.v, &tmv, &bar[ST_VF], 0, t * kT, bh);
-                tma_load_3d(sm + Lo.dn, &tmdn, &bar[ST_VF], 0, t * kT, bh);
-                for (int mb = 0; mb < nb; ++mb, ++use) {
-                    const int slot = use & 1;
-                    if (use >= 2) wait_k(ST_PE0 + slot, (use >> 1) - 1);
-                    mbar_arrive_expect_tx(&bar[ST_PF0 + slot], 4 * kTile);
-                    unsigned char* dst = sm + Lo.phi + slot * 4 * kTile;
-                    tma_load_3d(dst, &tmq, &bar[ST_PF0 + slot], 128 * mb, t * kT, bh);
-                    tma_load_3d(dst + kTile, &tmq, &bar[ST_PF0 + slot], 128 * mb + 64, t * kT, bh);
-                    tma_load_3d(dst + 2 * kTile, &tmk, &bar[ST_PF0 + slot], 128 * mb, t * kT, bh);
-                    tma_load_3d(dst + 3 * kTile, &tmk, &bar[ST_PF0 + slot], 128 * mb + 64, t * kT, bh);
-                }
+            const CUtensorMap* mphi = g ? &tmq : &tmk;
+            const CUtensorMap* my = g ? &tmdn : &tmv;
+            for (int i = 0; i < NS && wt.ok; ++i) {
+                const int b = i & 1, t = tile_of(i);
+                if (i >= 2) wait_k(SU_PE0 + b, (i >> 1) - 1);
+                mbar_arrive_expect_tx(&bar[SU_PF0 + b], 3 * kTile);
+                unsigned char* dp = sm + Lo.phi + b * 2 * kTile;
+                tma_load_3d(dp, mphi, &bar[SU_PF0 + b], 128 * mb, t * kT, bh);
+                tma_load_3d(dp + kTile, mphi, &bar[SU_PF0 + b], 128 * mb + 64, t * kT, bh);
+                tma_load_3d(sm + Lo.y + 2 * b * kTile, my, &bar[SU_PF0 + b], 0, t * kT, bh);
             }
         }
         __syncwarp();
@@ -495,154 +489,82 @@ k_tc_bwd_states(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         if (lane == 0) {
             constexpr uint32_t idS = idesc_bf16(128, 80, 1, 1);   // A, B MN-major
             const uint64_t dphi0 = sdesc(sbase + Lo.phi, kTile, 1024, kLayoutSW128);
-            const uint64_t dvb = sdesc(sbase + Lo.v, Lo.ones - Lo.v, 1024, kLayoutSW128);
-            const uint64_t dyb = sdesc(sbase + Lo.dn, Lo.dl - Lo.dn, 1024, kLayoutSW128);
-            int use = 0, it = 0, job = 0;
-            for (int item = blockIdx.x; item < bp.nitems && wt.ok; item += gridDim.x, ++it) {
-                wait_k(ST_VF, it);
-                wait_k(ST_YF, it);
-                for (int mb = 0; mb < nb; ++mb, ++use, ++job) {
-                    const int slot = use & 1, b = job & 1;
-                    wait_k(ST_PF0 + slot, use >> 1);
-                    if (job >= 2) wait_k(ST_DE0 + b, (job >> 1) - 1);
-                    tc_fence_after();
-                    const uint64_t dq = dphi0 + ((slot * 4 * kTile) >> 4), dk = dq + ((2 * kTile) >> 4);
-                    const uint32_t cs = tmem + 160u * b, cg = cs + 80;
+            const uint64_t dy0 = sdesc(sbase + Lo.y, kTile, 1024, kLayoutSW128);
+            for (int i = 0; i < NS && wt.ok; ++i) {
+                const int b = i & 1;
+                wait_k(SU_PF0 + b, i >> 1);
+                if (g) wait_k(SU_XF0 + b, i >> 1);
+                if (i >= 2) wait_k(SU_DE0 + b, (i >> 1) - 1);
+                tc_fence_after();
+                const uint64_t da = dphi0 + ((b * 2 * kTile) >> 4), dbb = dy0 + ((b * 2 * kTile) >> 4);
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_bf16(cs, dk + 128 * kk, dvb + 128 * kk, idS, kk > 0 ? 1u : 0u);
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_bf16(cg, dq + 128 * kk, dyb + 128 * kk, idS, kk > 0 ? 1u : 0u);
-                    umma_commit(&bar[ST_DF0 + b]);
-                    umma_commit(&bar[ST_PE0 + slot]);
-                }
-                umma_commit(&bar[ST_VE]);
-                umma_commit(&bar[ST_YE]);
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_bf16(tmem + 128u * b, da + 128 * kk, dbb + 128 * kk, idS, kk > 0 ? 1u : 0u);
+                umma_commit(&bar[SU_PE0 + b]);
+                umma_commit(&bar[SU_DF0 + b]);
             }
         }
         __syncwarp();
     } else {
         const int ew = warp - 1, q = warp & 3, half = ew >> 2;
-        const uint32_t row = 32u * q + lane;
+        const uint32_t row = 32u * q + lane;   // TMEM lane: feature 128 mb + row; token row of delta
         const uint32_t trow = tmem + ((32u * q) << 16);
-        int it = 0, job = 0;
-        for (int item = blockIdx.x; item < bp.nitems && wt.ok; item += gridDim.x, ++it) {
-            const int bh = item / bp.ntiles, t = item - bh * bp.ntiles;
-            const int i_abs = t * kT + static_cast<int>(row);
-            const bool valid = i_abs < bp.L;
-            const int64_t grow = static_cast<int64_t>(bh) * bp.L + i_abs;
-            // delta of this thread's token in the first 16 columns of its row of the extension
-            // tile (the columns the N = 80 operand reads; dn itself arrives by TMA with V)
-            if (it >= 1) wait_k(ST_YE, it - 1);
-            {
-                const float dl = valid ? delta[grow] : 0.0f;
-                const uint32_t dd = pack_bf16(dl, dl);
-                st_shared_v4(sbase + Lo.dl + sw128_off(row, half), dd, dd, dd, dd);
-            }
-            fence_async_smem();
-            warp_arrive(&bar[ST_YF]);
-            for (int mb = 0; mb < nb; ++mb, ++job) {
-                const int b = job & 1;
-                wait_k(ST_DF0 + b, job >> 1);
-                tc_fence_after();
-                // feature f = 128 mb + row; this warp writes columns 32 half .. (+ e = 64 for half 1)
-                uint32_t sa[32], ga[32], sz = 0, gz = 0;
-                const uint32_t cs = trow + 160u * b, cg = cs + 80;
-                tmem_ld32(cs + 32 * half, sa);
-                tmem_ld32(cg + 32 * half, ga);
-                if (half) {
-                    tmem_ld1(cs + 64, sz);
-                    tmem_ld1(cg + 64, gz);
-                }
-                tmem_wait_ld();
-                reg_fence(sa);
-                reg_fence(ga);
-                reg_fence1(sz);
-                reg_fence1(gz);
-                tc_fence_before();
-                warp_arrive(&bar[ST_DE0 + b]);
-                // slab f / 64, element (e, f % 64) at e * 64 + f % 64: for each e a warp's 32
-                // consecutive features store 128 contiguous bytes
-                const int f = 128 * mb + static_cast<int>(row);
-                const int64_t o = (static_cast<int64_t>(bh) * bp.ntiles + t) * bp.F * kE +
-                                  static_cast<int64_t>(f >> 6) * kSlabF + 64 * (32 * half) + (f & 63);
+        const int f = 128 * mb + static_cast<int>(row);
+        float run[33];
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    st_s[o + 64 * c] = __uint_as_float(sa[c]);
-                    st_g[o + 64 * c] = __uint_as_float(ga[c]);
-                }
-                if (half) {
-                    st_s[o + 64 * 32] = __uint_as_float(sz);
-                    st_g[o + 64 * 32] = __uint_as_float(gz);
-                }
-            }
+        for (int c = 0; c < 33; ++c) run[c] = 0.0f;
+        // delta of this thread's token in its 16-byte chunk `half` of the extension row (the
+        // 16 columns the N = 80 operand reads), for walk step i
+        auto write_delta = [&](int i) {
+            const int b = i & 1, t = tile_of(i);
+            if (i >= 2) wait_k(SU_PE0 + b, (i >> 1) - 1);   // the MMAs of step i - 2 read it
+            const int i_abs = t * kT + static_cast<int>(row);
+            const float dl = i_abs < bp.L ? delta[static_cast<int64_t>(bh) * bp.L + i_abs] : 0.0f;
+            const uint32_t dd = pack_bf16(dl, dl);
+            st_shared_v4(sbase + Lo.y + (2 * b + 1) * kTile + sw128_off(row, half), dd, dd, dd, dd);
+            fence_async_smem();
+            warp_arrive(&bar[SU_XF0 + b]);
+        };
+        // the operand slab form of feature f's running sums: row f % 64 of slab f / 64, this
+        // warp's 32 e (64 bytes), and z for half 1
+        auto store = [&](float* slab_base) {
+            uint4* op = reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(slab_base) +
+                                                 (f & 63) * 128 + 64 * half);
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                op[c] = make_uint4(pack_bf16(run[8 * c], run[8 * c + 1]), pack_bf16(run[8 * c + 2], run[8 * c + 3]),
+                                   pack_bf16(run[8 * c + 4], run[8 * c + 5]), pack_bf16(run[8 * c + 6], run[8 * c + 7]));
+            if (half) slab_base[kZOff + (f & 63)] = run[32];
+        };
+        float* sums = g ? st_g : st_s;
+        if (g && NS > 0) write_delta(0);
+        for (int i = 0; i < NS && wt.ok; ++i) {
+            const int b = i & 1, t = tile_of(i);
+            if (g && i + 1 < NS) write_delta(i + 1);
+            // the sum over the tiles walked so far, before tile t: its operand (causal)
+            if (!total)
+                store(sums + ((static_cast<int64_t>(bh) * NS + t) * nsl + (f >> 6)) * kSlabF);
+            wait_k(SU_DF0 + b, i >> 1);
+            tc_fence_after();
+            uint32_t a[32], z = 0;
+            tmem_ld32(trow + 128u * b + 32 * half, a);
+            if (half) tmem_ld1(trow + 128u * b + 64, z);
+            tmem_wait_ld();
+            reg_fence(a);
+            reg_fence1(z);
+            tc_fence_before();
+            warp_arrive(&bar[SU_DE0 + b]);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) run[c] += __uint_as_float(a[c]);
+            run[32] += __uint_as_float(z);
         }
+        if (total) store((g ? tot_g : tot_s) + (static_cast<int64_t>(bh) * nsl + (f >> 6)) * kSlabF);
     }
     wt.report(err);
     drain_after_failure(wt.ok);
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 512);
-}
-
-// ------------------------------------------------------------------ scans over tiles
-// One CTA per (sequence bh, 64-feature slab) and sum (blockIdx.y: 0 = S, 1 = G): walks the
-// sequence's tiles in order (S: forward; G: backward) keeping fp32 running sums and writes,
-// over each tile's slab, the sum over the tiles before it (S_c) or after it (G_c) -- the
-// exclusive prefix / suffix -- as the contraction's operand: [64 f][64 e] bf16 and z fp32.
-// total != 0 (the bidirectional form): the whole-sequence sums instead, written once to
-// tot_s / tot_g ([BH][slabs] slabs of the same form); the per-tile sums are left as they are.
-// Thread: feature fl = tid % 64 and the 16 e of group eg = tid / 64 (group 3 also e = 64),
-// so its operand row piece is 32 contiguous bytes.  A tile's sums are all in registers (and
-// added) before the barrier after which its slab is overwritten.
-constexpr int kScanThreads = 256;
-
-__global__ void __launch_bounds__(kScanThreads)
-k_scan_slabs(float* __restrict__ st_s, float* __restrict__ st_g, float* __restrict__ tot_s,
-             float* __restrict__ tot_g, int NS, int nsl, int total)
-{
-    const int which = blockIdx.y;
-    const int bh = static_cast<int>(blockIdx.x) / nsl, slab = static_cast<int>(blockIdx.x) - bh * nsl;
-    float* base = (which ? st_g : st_s) + (static_cast<int64_t>(bh) * NS * nsl + slab) * kSlabF;
-    const int64_t tstride = static_cast<int64_t>(nsl) * kSlabF;   // floats from tile to tile
-    const int fl = threadIdx.x & 63, eg = threadIdx.x >> 6;
-    const bool hasz = eg == 3;
-    const bool rev = !total && which == 1;
-    float run[17], x[17];
-#pragma unroll
-    for (int c = 0; c < 17; ++c) run[c] = 0.0f;
-    auto load = [&](int t) {
-        const float* p = base + t * tstride + (16 * eg) * 64 + fl;
-#pragma unroll
-        for (int c = 0; c < 16; ++c) x[c] = p[64 * c];
-        x[16] = hasz ? base[t * tstride + 64 * 64 + fl] : 0.0f;
-    };
-    auto store = [&](float* slab_base, const float (&val)[17]) {
-        uint4* op = reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(slab_base) + fl * 128 + 32 * eg);
-        op[0] = make_uint4(pack_bf16(val[0], val[1]), pack_bf16(val[2], val[3]),
-                           pack_bf16(val[4], val[5]), pack_bf16(val[6], val[7]));
-        op[1] = make_uint4(pack_bf16(val[8], val[9]), pack_bf16(val[10], val[11]),
-                           pack_bf16(val[12], val[13]), pack_bf16(val[14], val[15]));
-        if (hasz) slab_base[kZOff + fl] = val[16];
-    };
-    const int t0 = rev ? NS - 1 : 0, step = rev ? -1 : 1;
-    load(t0);
-    for (int i = 0; i < NS; ++i) {
-        const int t = t0 + i * step;
-        float out[17];
-#pragma unroll
-        for (int c = 0; c < 17; ++c) {
-            out[c] = run[c];
-            run[c] += x[c];
-        }
-        if (i + 1 < NS) load(t + step);   // the next tile's sums, in flight during the stores
-        if (!total) {
-            __syncthreads();   // every thread has added tile t's sums: its slab may be overwritten
-            store(base + t * tstride, out);
-        }
-    }
-    if (total) store((which ? tot_g : tot_s) + (static_cast<int64_t>(bh) * nsl + slab) * kSlabF, run);
+    if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
 // Operand slabs ([nslabs] x [64 f][64 e] bf16, kSlabF floats apart) viewed as a 3-D tensor,
@@ -682,33 +604,7 @@ bool map_seq(CUtensorMap* m, const void* base, int cols, int L, int BH)
 bool tc_bwd_tile_supported(int F, int L)
 {
     return F % 128 == 0 && F >= 128 && F <= 512 && L > 0 && bw_layout().total + 1024 <= 232448 &&
-           st_layout().total + 1024 <= 232448;
-}
-
-cudaError_t tc_bwd_states(const void* phq, const void* phk, const void* v, const void* dn16,
-                          const float* delta, float* st_s, float* st_g, int BH, int L, int F,
-                          int* err, cudaStream_t st)
-{
-    if (!tc_bwd_tile_supported(F, L)) return cudaErrorNotSupported;
-    CUtensorMap mq, mk, mv, mdn;
-    if (!map_seq(&mq, phq, F, L, BH) || !map_seq(&mk, phk, F, L, BH) || !map_seq(&mv, v, 64, L, BH) ||
-        !map_seq(&mdn, dn16, 64, L, BH))
-        return cudaErrorInvalidValue;
-    BwParams bp;
-    bp.L = L;
-    bp.F = F;
-    bp.ntiles = (L + kT - 1) / kT;
-    bp.nitems = BH * bp.ntiles;
-    bp.dphi_bf16 = 0;
-    bp.bidir = 0;
-    const size_t smem = st_layout().total + 1024;
-    cudaError_t e = cudaFuncSetAttribute(k_tc_bwd_states, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    const int grid = bp.nitems < kNumSMs ? bp.nitems : kNumSMs;
-    TraceScope trace_("tc_bwd_states", st);
-    k_tc_bwd_states<<<grid, kStThreads, smem, st>>>(mq, mk, mv, mdn, delta, st_s, st_g, bp, err);
-    return cudaGetLastError();
+           su_layout().total + 1024 <= 232448;
 }
 
 cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const void* dn16,
@@ -728,7 +624,7 @@ cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const v
     bp.nitems = BH * bp.ntiles;
     bp.dphi_bf16 = dphi_bf16 ? 1 : 0;
     bp.bidir = bidir ? 1 : 0;
-    // the operand slabs the scans wrote: per tile (causal) or per sequence (bidirectional)
+    // the operand slabs k_tc_bwd_sums wrote: per tile (causal) or per sequence (bidirectional)
     const int64_t nslabs = static_cast<int64_t>(BH) * (bidir ? 1 : bp.ntiles) * (F / 64);
     CUtensorMap ms, mg;
     if (!map_slabs(&ms, sfw, nslabs) || !map_slabs(&mg, gbw, nslabs)) return cudaErrorInvalidValue;
@@ -743,15 +639,31 @@ cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const v
     return cudaGetLastError();
 }
 
-cudaError_t tc_bwd_scan(float* st_s, float* st_g, float* tot_s, float* tot_g, int BH, int L, int F,
-                        bool bidir, cudaStream_t st)
+cudaError_t tc_bwd_sums(const void* phq, const void* phk, const void* v, const void* dn16,
+                        const float* delta, float* st_s, float* st_g, float* tot_s, float* tot_g,
+                        int BH, int L, int F, bool bidir, int* err, cudaStream_t st)
 {
     if (!tc_bwd_tile_supported(F, L)) return cudaErrorNotSupported;
-    const int NS = (L + kT - 1) / kT, nsl = F / 64;
-    TraceScope trace_("tc_bwd_scan", st);
-    k_scan_slabs<<<dim3(static_cast<unsigned>(BH * nsl), 2), kScanThreads, 0, st>>>(
-        st_s, st_g, tot_s, tot_g, NS, nsl, bidir ? 1 : 0);
+    CUtensorMap mq, mk, mv, mdn;
+    if (!map_seq(&mq, phq, F, L, BH) || !map_seq(&mk, phk, F, L, BH) || !map_seq(&mv, v, 64, L, BH) ||
+        !map_seq(&mdn, dn16, 64, L, BH))
+        return cudaErrorInvalidValue;
+    BwParams bp;
+    bp.L = L;
+    bp.F = F;
+    bp.ntiles = (L + kT - 1) / kT;
+    bp.nitems = BH * bp.ntiles;
+    bp.dphi_bf16 = 0;
+    bp.bidir = bidir ? 1 : 0;
+    const size_t smem = su_layout().total + 1024;
+    cudaError_t e = cudaFuncSetAttribute(k_tc_bwd_sums, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    TraceScope trace_("tc_bwd_sums", st);
+    k_tc_bwd_sums<<<BH * (F / 128) * 2, kSumThreads, smem, st>>>(mq, mk, mv, mdn, delta, st_s, st_g,
+                                                                 tot_s, tot_g, bp, err);
     return cudaGetLastError();
 }
+
 
 }  // namespace slay

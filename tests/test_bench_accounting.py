@@ -65,11 +65,9 @@ def test_backward_kernels_are_not_chunk_split():
     assert bench.kernel_work("tc_phi_bwd", w, "feature_map_bwd")[0] == \
         2 * th * (2 * D + 2 * w.F + 4 * D)
     tiles = w.B * w.H * ((w.L + 127) // 128)
-    states = tiles * 2 * w.F * (DV + 1) * 4
-    # the scans read both sums' fp32 slabs and write the bf16 operands and fp32 z
-    assert bench.kernel_work("tc_bwd_scan", w, "bwd")[0] == states + tiles * 2 * w.F * (DV * 2 + 4)
-    assert bench.kernel_work("tc_bwd_states", w, "bwd")[0] == \
-        th * (2 * 2 * w.F + 2 * DV + 4 * (DV + 1)) + states
+    # the running sums read phi(q), phi(k), v, dn once and write every tile's operands
+    assert bench.kernel_work("tc_bwd_sums", w, "bwd")[0] == \
+        th * (4 * w.F + 4 * DV) + tiles * 2 * w.F * (DV * 2 + 4)
     # the contraction by its flops: three products with the scanned sums (2 F Dv each) and
     # the masked intra-tile terms over the C + 1 keys of a causal chunk row on average
     amount, unit, bound = bench.kernel_work("tc_bwd_tile", w, "bwd")
