@@ -64,8 +64,9 @@ enum {
 };
 
 struct BwLayout {
-    uint32_t phi, pt, ct, dn, v, sg, bar, tmem, total;
+    uint32_t phi, pt, ct, dn, v, sg, stg, bar, tmem, total;
 };
+constexpr int kStgBytes = 2 * 32 * 64;   // per epilogue warp: dphiQ, dphiK boxes [32 rows][32 bf16]
 
 __host__ __device__ inline BwLayout bw_layout()
 {
@@ -76,7 +77,8 @@ __host__ __device__ inline BwLayout bw_layout()
     l.dn = l.ct + 2 * kTile;      // dn [128 i][64 e] (TMA, with V)
     l.v = l.dn + kTile;           // V [128 j][64 e]
     l.sg = l.v + kTile;           // 2 buffers x (S_s, G_s) [64 f][64 e]
-    l.bar = l.sg + 4 * kSG;
+    l.stg = l.sg + 4 * kSG;       // 8 epilogue warps x kStgBytes: bf16 dphi staged for TMA stores
+    l.bar = l.stg + 8 * kStgBytes;
     l.tmem = l.bar + BW_NUM * 8;
     l.total = l.tmem + 16;
     return l;
@@ -93,6 +95,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
 k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
               const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdn,
               const __grid_constant__ CUtensorMap tms, const __grid_constant__ CUtensorMap tmg,
+              const __grid_constant__ CUtensorMap tmdq, const __grid_constant__ CUtensorMap tmdk,
               const float* __restrict__ delta, const float* __restrict__ sfw,
               const float* __restrict__ gbw,
               void* __restrict__ dphq, void* __restrict__ dphk, float* __restrict__ dv,
@@ -330,18 +333,33 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
                     oq[c] = fmaf(dl, __shfl_sync(0xffffffffu, zsl, c), __uint_as_float(qa[c]));
                     ok[c] = __uint_as_float(ka[c]) + __shfl_sync(0xffffffffu, zgl, c);
                 }
-                if (!valid) return;
                 if (bp.dphi_bf16) {
-                    uint4* dq4 = reinterpret_cast<uint4*>(static_cast<uint16_t*>(dphq) + grow * bp.F + f0);
-                    uint4* dk4 = reinterpret_cast<uint4*>(static_cast<uint16_t*>(dphk) + grow * bp.F + f0);
+                    // this warp's 32 rows x 32 features of dphiQ and dphiK through its staging
+                    // boxes (64-byte swizzle: chunk c of row r at c ^ ((r >> 1) & 3), so a
+                    // warp's 16-byte writes spread over 8 bank groups) and two TMA stores;
+                    // rows past L are clipped by the tensor map
+                    const uint32_t qbuf = sbase + Lo.stg + ew * kStgBytes, kbuf = qbuf + 32 * 64;
+                    if (lane == 0) bulk_wait_read<0>();   // the previous slice's stores read them
+                    __syncwarp();
+                    const uint32_t rsw = (static_cast<uint32_t>(lane) >> 1) & 3u;
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
-                        dq4[c] = make_uint4(pack_bf16(oq[8 * c], oq[8 * c + 1]), pack_bf16(oq[8 * c + 2], oq[8 * c + 3]),
-                                            pack_bf16(oq[8 * c + 4], oq[8 * c + 5]), pack_bf16(oq[8 * c + 6], oq[8 * c + 7]));
-                        dk4[c] = make_uint4(pack_bf16(ok[8 * c], ok[8 * c + 1]), pack_bf16(ok[8 * c + 2], ok[8 * c + 3]),
-                                            pack_bf16(ok[8 * c + 4], ok[8 * c + 5]), pack_bf16(ok[8 * c + 6], ok[8 * c + 7]));
+                        const uint32_t off = lane * 64u + ((static_cast<uint32_t>(c) ^ rsw) << 4);
+                        st_shared_v4(qbuf + off, pack_bf16(oq[8 * c], oq[8 * c + 1]), pack_bf16(oq[8 * c + 2], oq[8 * c + 3]),
+                                     pack_bf16(oq[8 * c + 4], oq[8 * c + 5]), pack_bf16(oq[8 * c + 6], oq[8 * c + 7]));
+                        st_shared_v4(kbuf + off, pack_bf16(ok[8 * c], ok[8 * c + 1]), pack_bf16(ok[8 * c + 2], ok[8 * c + 3]),
+                                     pack_bf16(ok[8 * c + 4], ok[8 * c + 5]), pack_bf16(ok[8 * c + 6], ok[8 * c + 7]));
+                    }
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        const int r0 = t * kT + 32 * q;
+                        tma_store_3d(&tmdq, sm + Lo.stg + ew * kStgBytes, f0, r0, bh);
+                        tma_store_3d(&tmdk, sm + Lo.stg + ew * kStgBytes + 32 * 64, f0, r0, bh);
+                        bulk_commit_group();
                     }
                 } else {
+                    if (!valid) return;
                     float4* dq4 = reinterpret_cast<float4*>(static_cast<float*>(dphq) + grow * bp.F + f0);
                     float4* dk4 = reinterpret_cast<float4*>(static_cast<float*>(dphk) + grow * bp.F + f0);
 #pragma unroll
@@ -378,6 +396,7 @@ k_tc_bwd_tile(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
                 }
             }
         }
+        if (lane == 0) bulk_wait<0>();   // this warp's dphi stores have landed
     }
     wt.report(err);
     drain_after_failure(wt.ok);
@@ -567,6 +586,22 @@ k_tc_bwd_sums(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
     if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
+// bf16 dphi [BH][L][F] viewed as a 3-D tensor for the contraction's TMA stores: boxes of 32
+// features x 32 tokens, 64-byte swizzle; rows past L are not written.
+bool map_dphi(CUtensorMap* m, void* base, int F, int L, int BH)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(F), static_cast<cuuint64_t>(L),
+                                static_cast<cuuint64_t>(BH)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(F) * 2, static_cast<cuuint64_t>(L) * F * 2};
+    const cuuint32_t box[3] = {32, 32, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Operand slabs ([nslabs] x [64 f][64 e] bf16, kSlabF floats apart) viewed as a 3-D tensor,
 // one [64][64] box per slab, 128-byte swizzle.
 bool map_slabs(CUtensorMap* m, const float* base, int64_t nslabs)
@@ -626,16 +661,18 @@ cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const v
     bp.bidir = bidir ? 1 : 0;
     // the operand slabs k_tc_bwd_sums wrote: per tile (causal) or per sequence (bidirectional)
     const int64_t nslabs = static_cast<int64_t>(BH) * (bidir ? 1 : bp.ntiles) * (F / 64);
-    CUtensorMap ms, mg;
+    CUtensorMap ms, mg, mdq = mq, mdk = mk;   // (mdq, mdk unused when dphi is fp32)
     if (!map_slabs(&ms, sfw, nslabs) || !map_slabs(&mg, gbw, nslabs)) return cudaErrorInvalidValue;
+    if (dphi_bf16 && (!map_dphi(&mdq, dphq, F, L, BH) || !map_dphi(&mdk, dphk, F, L, BH)))
+        return cudaErrorInvalidValue;
     const size_t smem = bw_layout().total + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_tc_bwd_tile, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     const int grid = bp.nitems < kNumSMs ? bp.nitems : kNumSMs;
     TraceScope trace_("tc_bwd_tile", st);
-    k_tc_bwd_tile<<<grid, kBwThreads, smem, st>>>(mq, mk, mv, mdn, ms, mg, delta, sfw, gbw, dphq, dphk,
-                                                  dv, bp, err);
+    k_tc_bwd_tile<<<grid, kBwThreads, smem, st>>>(mq, mk, mv, mdn, ms, mg, mdq, mdk, delta, sfw, gbw,
+                                                  dphq, dphk, dv, bp, err);
     return cudaGetLastError();
 }
 
