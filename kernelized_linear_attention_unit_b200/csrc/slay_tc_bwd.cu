@@ -424,7 +424,7 @@ constexpr int kSumThreads = 32 * 10;
 enum { SU_PF0 = 0, SU_PF1, SU_PE0, SU_PE1, SU_XF0, SU_XF1, SU_DF0, SU_DF1, SU_DE0, SU_DE1, SU_NUM };
 
 struct SuLayout {
-    uint32_t phi, y, bar, tmem, total;
+    uint32_t phi, y, stg, bar, tmem, total;
 };
 
 __host__ __device__ inline SuLayout su_layout()
@@ -432,7 +432,8 @@ __host__ __device__ inline SuLayout su_layout()
     SuLayout l;
     l.phi = 0;                    // 2 slots x (two 64-feature tiles of the block)
     l.y = l.phi + 4 * kTile;      // 2 slots x (V or dn tile, then its extension tile at LBO)
-    l.bar = l.y + 4 * kTile;
+    l.stg = l.y + 4 * kTile;      // 8 epilogue warps x [32 f][32 e] bf16 staged for TMA stores
+    l.bar = l.stg + 8 * 32 * 64;
     l.tmem = l.bar + SU_NUM * 8;
     l.total = l.tmem + 16;
     return l;
@@ -441,6 +442,7 @@ __host__ __device__ inline SuLayout su_layout()
 __global__ void __launch_bounds__(kSumThreads, 1)
 k_tc_bwd_sums(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
               const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdn,
+              const __grid_constant__ CUtensorMap tmso, const __grid_constant__ CUtensorMap tmgo,
               const float* __restrict__ delta, float* __restrict__ st_s, float* __restrict__ st_g,
               float* __restrict__ tot_s, float* __restrict__ tot_g, BwParams bp, int* err)
 {
@@ -545,15 +547,26 @@ k_tc_bwd_sums(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
             warp_arrive(&bar[SU_XF0 + b]);
         };
         // the operand slab form of feature f's running sums: row f % 64 of slab f / 64, this
-        // warp's 32 e (64 bytes), and z for half 1
-        auto store = [&](float* slab_base) {
-            uint4* op = reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(slab_base) +
-                                                 (f & 63) * 128 + 64 * half);
+        // warp's 32 e (64 bytes) through its staging box (64-byte swizzle: chunk c of row r
+        // at c ^ ((r >> 1) & 3)) and a TMA store of [32 f][32 e]; z (half 1) stored directly
+        const CUtensorMap* mout = g ? &tmgo : &tmso;
+        const uint32_t sbox = sbase + Lo.stg + ew * 32 * 64;
+        auto store = [&](int64_t slab, float* zdst) {
+            if (lane == 0) bulk_wait_read<0>();   // the box's previous store has read it
+            __syncwarp();
+            const uint32_t rsw = (static_cast<uint32_t>(lane) >> 1) & 3u;
 #pragma unroll
             for (int c = 0; c < 4; ++c)
-                op[c] = make_uint4(pack_bf16(run[8 * c], run[8 * c + 1]), pack_bf16(run[8 * c + 2], run[8 * c + 3]),
-                                   pack_bf16(run[8 * c + 4], run[8 * c + 5]), pack_bf16(run[8 * c + 6], run[8 * c + 7]));
-            if (half) slab_base[kZOff + (f & 63)] = run[32];
+                st_shared_v4(sbox + lane * 64u + ((static_cast<uint32_t>(c) ^ rsw) << 4),
+                             pack_bf16(run[8 * c], run[8 * c + 1]), pack_bf16(run[8 * c + 2], run[8 * c + 3]),
+                             pack_bf16(run[8 * c + 4], run[8 * c + 5]), pack_bf16(run[8 * c + 6], run[8 * c + 7]));
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_3d(mout, sm + Lo.stg + ew * 32 * 64, 32 * half, 32 * (q & 1), static_cast<int>(slab));
+                bulk_commit_group();
+            }
+            if (half) zdst[kZOff + (f & 63)] = run[32];
         };
         float* sums = g ? st_g : st_s;
         if (g && NS > 0) write_delta(0);
@@ -561,8 +574,10 @@ k_tc_bwd_sums(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
             const int b = i & 1, t = tile_of(i);
             if (g && i + 1 < NS) write_delta(i + 1);
             // the sum over the tiles walked so far, before tile t: its operand (causal)
-            if (!total)
-                store(sums + ((static_cast<int64_t>(bh) * NS + t) * nsl + (f >> 6)) * kSlabF);
+            if (!total) {
+                const int64_t slab = (static_cast<int64_t>(bh) * NS + t) * nsl + (f >> 6);
+                store(slab, sums + slab * kSlabF);
+            }
             wait_k(SU_DF0 + b, i >> 1);
             tc_fence_after();
             uint32_t a[32], z = 0;
@@ -577,7 +592,11 @@ k_tc_bwd_sums(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
             for (int c = 0; c < 32; ++c) run[c] += __uint_as_float(a[c]);
             run[32] += __uint_as_float(z);
         }
-        if (total) store((g ? tot_g : tot_s) + (static_cast<int64_t>(bh) * nsl + (f >> 6)) * kSlabF);
+        if (total) {
+            const int64_t slab = static_cast<int64_t>(bh) * nsl + (f >> 6);
+            store(slab, (g ? tot_g : tot_s) + slab * kSlabF);
+        }
+        if (lane == 0) bulk_wait<0>();   // this warp's stores have landed
     }
     wt.report(err);
     drain_after_failure(wt.ok);
@@ -615,6 +634,20 @@ bool map_slabs(CUtensorMap* m, const float* base, int64_t nslabs)
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<float*>(base), dims, strides, box,
               es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The same slabs for k_tc_bwd_sums' TMA stores: boxes of 32 e x 32 f, 64-byte swizzle.
+bool map_slabs_out(CUtensorMap* m, float* base, int64_t nslabs)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {64, 64, static_cast<cuuint64_t>(nslabs)};
+    const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(kSlabF) * 4};
+    const cuuint32_t box[3] = {32, 32, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // [BH][L][cols] bf16 viewed as a 3-D tensor, boxes of 64 columns x 128 tokens, 128-byte
@@ -692,13 +725,18 @@ cudaError_t tc_bwd_sums(const void* phq, const void* phk, const void* v, const v
     bp.nitems = BH * bp.ntiles;
     bp.dphi_bf16 = 0;
     bp.bidir = bidir ? 1 : 0;
+    // outputs: every tile's slabs (causal) or every sequence's (bidirectional)
+    const int64_t nslabs = static_cast<int64_t>(BH) * (bidir ? 1 : bp.ntiles) * (F / 64);
+    CUtensorMap mso, mgo;
+    if (!map_slabs_out(&mso, bidir ? tot_s : st_s, nslabs) || !map_slabs_out(&mgo, bidir ? tot_g : st_g, nslabs))
+        return cudaErrorInvalidValue;
     const size_t smem = su_layout().total + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_tc_bwd_sums, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     TraceScope trace_("tc_bwd_sums", st);
-    k_tc_bwd_sums<<<BH * (F / 128) * 2, kSumThreads, smem, st>>>(mq, mk, mv, mdn, delta, st_s, st_g,
-                                                                 tot_s, tot_g, bp, err);
+    k_tc_bwd_sums<<<BH * (F / 128) * 2, kSumThreads, smem, st>>>(mq, mk, mv, mdn, mso, mgo, delta, st_s,
+                                                                 st_g, tot_s, tot_g, bp, err);
     return cudaGetLastError();
 }
 

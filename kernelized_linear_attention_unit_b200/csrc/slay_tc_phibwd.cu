@@ -295,15 +295,21 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
                 reg_fence(pr);
                 const int sub = 2 * g + half;
                 const float a = pp.a2[sub] * inv, bb = pp.b2[sub] + l2i, sq = pp.sq[sub];
+                const float2 a2 = make_float2(a, a), b2 = make_float2(bb, bb);
+                const float2 sq2 = make_float2(sq, sq), tn2 = make_float2(two_n, two_n);
                 uint32_t al[16], be[16];
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
-                    const float d0 = dphi_val(dp, c), d1 = dphi_val(dp, c + 1);
-                    const float p0 = __uint_as_float(pr[c]), p1 = __uint_as_float(pr[c + 1]);
-                    const float t0 = d0 * ex2(fmaf(a, __uint_as_float(ur[c]), bb)) * p0;
-                    const float t1 = d1 * ex2(fmaf(a, __uint_as_float(ur[c + 1]), bb)) * p1;
-                    al[c >> 1] = pack_bf16(t0 * p0 * sq, t1 * p1 * sq);
-                    be[c >> 1] = pack_bf16(t0 * two_n, t1 * two_n);
+                    // pairs of features through the packed two-wide fp32 instructions (each
+                    // lane rounds like the scalar form, in the same order)
+                    const float2 d = make_float2(dphi_val(dp, c), dphi_val(dp, c + 1));
+                    const float2 p = make_float2(__uint_as_float(pr[c]), __uint_as_float(pr[c + 1]));
+                    const float2 y = ffma2(a2, make_float2(__uint_as_float(ur[c]), __uint_as_float(ur[c + 1])), b2);
+                    const float2 t = fmul2(fmul2(d, make_float2(ex2(y.x), ex2(y.y))), p);
+                    const float2 af = fmul2(fmul2(t, p), sq2);
+                    const float2 bf = fmul2(t, tn2);
+                    al[c >> 1] = pack_bf16(af.x, af.y);
+                    be[c >> 1] = pack_bf16(bf.x, bf.y);
                 }
                 if (j >= 2) {   // operand buffer j & 1 read by the contraction of job j - 2
                     uint32_t ph = static_cast<uint32_t>(((j - 2) >> 1) & 1);
