@@ -475,22 +475,35 @@ __global__ void k_bwd_rowstats(const T* __restrict__ out, const float* __restric
 }
 
 // The same statistics for the tensor-core backward: dn as bf16 rows [row][64] (its MMA operand,
-// loaded by TMA) and delta as fp32 [row].
-template <typename T>
-__global__ void k_bwd_rowstats_tc(const T* __restrict__ out, const float* __restrict__ den,
-                                  const T* __restrict__ g, __nv_bfloat16* __restrict__ dn16,
+// loaded by TMA) and delta as fp32 [row].  bf16 rows only: eight lanes per row, each with 16
+// bytes (eight values) of out, g and dn, so a warp serves four rows with full-width accesses.
+__global__ void k_bwd_rowstats_tc(const __nv_bfloat16* __restrict__ out, const float* __restrict__ den,
+                                  const __nv_bfloat16* __restrict__ g, __nv_bfloat16* __restrict__ dn16,
                                   float* __restrict__ delta, int64_t nrows, float eps)
 {
-    const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (row >= nrows) return;
-    const float rz = 1.0f / (den[row] + eps);
-    const float g0 = ld(g + row * kD + 2 * lane), g1 = ld(g + row * kD + 2 * lane + 1);
-    float s = g0 * ld(out + row * kD + 2 * lane) + g1 * ld(out + row * kD + 2 * lane + 1);
+    const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 3;
+    const int part = threadIdx.x & 7;   // values 8 part .. 8 part + 7 of the row
+    const bool ok = row < nrows;
+    const int64_t r = ok ? row : nrows - 1;   // (the shuffles below need every lane)
+    const uint4 gv = reinterpret_cast<const uint4*>(g + r * kD)[part];
+    const uint4 ov = reinterpret_cast<const uint4*>(out + r * kD)[part];
+    const float rz = 1.0f / (den[r] + eps);
+    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w}, ow[4] = {ov.x, ov.y, ov.z, ov.w};
+    float s = 0.0f;
+    uint32_t dw[4];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    reinterpret_cast<__nv_bfloat162*>(dn16 + row * kD)[lane] = __floats2bfloat162_rn(g0 * rz, g1 * rz);
-    if (lane == 0) delta[row] = -s * rz;
+    for (int i = 0; i < 4; ++i) {
+        const float g0 = __uint_as_float(gw[i] << 16), g1 = __uint_as_float(gw[i] & 0xFFFF0000u);
+        s = fmaf(g0, __uint_as_float(ow[i] << 16), s);
+        s = fmaf(g1, __uint_as_float(ow[i] & 0xFFFF0000u), s);
+        const __nv_bfloat162 d = __floats2bfloat162_rn(g0 * rz, g1 * rz);
+        dw[i] = *reinterpret_cast<const uint32_t*>(&d);
+    }
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (!ok) return;
+    reinterpret_cast<uint4*>(dn16 + row * kD)[part] = make_uint4(dw[0], dw[1], dw[2], dw[3]);
+    if (part == 0) delta[row] = -s * rz;
 }
 
 struct BwdSmem {
@@ -1263,8 +1276,9 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
     {
         TraceScope trace_("simt_bwd_rowstats", st);
         if (tcb)
-            k_bwd_rowstats_tc<T><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
-                cp<T>(out), den, cp<T>(dout), dn16, delta, rows, eps);
+            k_bwd_rowstats_tc<<<static_cast<unsigned>((rows + 31) / 32), 256, 0, st>>>(
+                reinterpret_cast<const __nv_bfloat16*>(out), den,
+                reinterpret_cast<const __nv_bfloat16*>(dout), dn16, delta, rows, eps);
         else
             k_bwd_rowstats<T><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
                 cp<T>(out), den, cp<T>(dout), dn, rows, eps);
