@@ -19,7 +19,7 @@
 // Persistent, one CTA per SM, 128-row tiles round-robin.  Warp 0 issues every TMA load and
 // MMA; warps 1-8 are the epilogue: warp w serves TMEM lanes 32 (w % 4).. (rows of the tile)
 // and the 32-feature half (w - 1) / 4 of every group.  Per group an epilogue warp reads its
-// projections, its rows' dphi (bf16, loaded three groups ahead) and writes its block of
+// projections, its rows' dphi (bf16, loaded two groups ahead) and writes its block of
 // [alpha | beta] into a K-major 128-byte-swizzled operand tile; per tile it turns dX^ into
 // dx.  Every wait is bounded; a timeout sets the library's feature-map status word.
 #include <cuda.h>
@@ -44,17 +44,21 @@ constexpr int kSubBytes = 64 * 128;         // packed W of 32 features = 8 KiB
 constexpr int kGroupBytes = 2 * kSubBytes;  // 64 features = 16 KiB
 constexpr int kABytes = 2 * kBoxBytes;      // [alpha | beta] of one group: two 16 KiB K-tiles
 constexpr int kEpiWarps = 8;
-constexpr int kPbThreads = 32 * (1 + kEpiWarps);
+constexpr int kPbThreads = 32 * (2 + kEpiWarps);   // MMA warp, 8 epilogue warps, TMA warp
 constexpr int kNumSMs = 148;
-constexpr int kMaxXBufs = 4;
+constexpr int kXBufs = 3;                   // X tiles in flight
+constexpr int kRing = 3;                    // W groups and dphi tiles in flight (slot = job % 3)
 constexpr uint32_t kColU = 0;               // two 128-column projection buffers
 constexpr uint32_t kColDX = 256;            // two 64-column dX^ accumulators
 
 enum {
-    PB_W = 0,
-    PB_XF = 1,                  // + slot
-    PB_XE = PB_XF + kMaxXBufs,  // + slot (8 warp arrivals: dx of the tile written)
-    PB_UF = PB_XE + kMaxXBufs,  // + buffer (projection MMA commit)
+    PB_XF = 0,                  // + slot (TMA: X tile)
+    PB_XE = PB_XF + kXBufs,     // + slot (8 warp arrivals: dx of the tile written)
+    PB_WF = PB_XE + kXBufs,     // + slot (TMA: W group)
+    PB_WE = PB_WF + kRing,      // + slot (contraction MMA commit: the group's W free)
+    PB_GF = PB_WE + kRing,      // + slot (TMA: dphi tile)
+    PB_GE = PB_GF + kRing,      // + slot (8 warp arrivals: dphi read)
+    PB_UF = PB_GE + kRing,      // + buffer (projection MMA commit)
     PB_AF = PB_UF + 2,          // + buffer (8 warp arrivals: [alpha | beta] written)
     PB_AE = PB_AF + 2,          // + buffer (contraction MMA commit: operand free)
     PB_DF = PB_AE + 2,          // + buffer (dX^ of a tile complete)
@@ -63,18 +67,17 @@ enum {
 };
 
 struct PbLayout {
-    uint32_t w, x, a, bar, tmem, total;
-    int xbufs;
+    uint32_t w, x, a, d, bar, tmem, total;
 };
 
-__host__ __device__ inline PbLayout pb_layout(int F)
+__host__ __device__ inline PbLayout pb_layout(int /*F*/)
 {
     PbLayout l;
-    l.xbufs = F <= 128 ? 4 : F <= 256 ? 3 : 2;
-    l.w = 0;
-    l.x = (F / 32) * kSubBytes;
-    l.a = l.x + l.xbufs * kBoxBytes;
-    l.bar = l.a + 2 * kABytes;
+    l.w = 0;                                // kRing W groups (16 KiB each)
+    l.x = l.w + kRing * kGroupBytes;        // kXBufs X tiles
+    l.a = l.x + kXBufs * kBoxBytes;         // 2 [alpha | beta] operands
+    l.d = l.a + 2 * kABytes;                // kRing dphi tiles [128 rows][64 features]
+    l.bar = l.d + kRing * kBoxBytes;
     l.tmem = l.bar + PB_NUM * 8;
     l.total = l.tmem + 16;
     return l;
@@ -96,13 +99,26 @@ __device__ __forceinline__ float dphi_val(const uint4 (&d)[4], int c)
     return __uint_as_float((c & 1) ? (u & 0xFFFF0000u) : (u << 16));
 }
 
+// Slot and use count of a ring walked in order: the u-th use of slot s waits for phase u & 1
+// of its full barrier and (u >= 1) phase (u - 1) & 1 of its empty barrier.
+struct Ring {
+    int slot = 0, use = 0, n;
+    __device__ explicit Ring(int n_) : n(n_) {}
+    __device__ void next()
+    {
+        if (++slot == n) {
+            slot = 0;
+            ++use;
+        }
+    }
+};
+
 __global__ void __launch_bounds__(kPbThreads, 1)
 k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
-             const __nv_bfloat16* __restrict__ dphi, float* __restrict__ dx, int64_t n_rows,
+             const __grid_constant__ CUtensorMap tmd, float* __restrict__ dx, int64_t n_rows,
              PbParams pp, int* status)
 {
     constexpr int kW = 4;     // 16-byte words per 32 bf16 dphi values
-    constexpr int kPre = 3;   // dphi groups loaded ahead
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* sm = aligned_smem(smem_raw);
     const PbLayout L = pb_layout(pp.F);
@@ -111,7 +127,6 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ng = pp.F / 64;
-    const int xbufs = L.xbufs;
 
     if (warp == 0) {
         tmem_alloc(tslot, 512);
@@ -119,7 +134,8 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
     }
     if (tid == 0) {
         for (int i = 0; i < PB_NUM; ++i) mbar_init(&bar[i], 1);
-        for (int s = 0; s < kMaxXBufs; ++s) mbar_init(&bar[PB_XE + s], kEpiWarps);
+        for (int s = 0; s < kXBufs; ++s) mbar_init(&bar[PB_XE + s], kEpiWarps);
+        for (int s = 0; s < kRing; ++s) mbar_init(&bar[PB_GE + s], kEpiWarps);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bar[PB_AF + b], kEpiWarps);
             mbar_init(&bar[PB_DE + b], kEpiWarps);
@@ -127,6 +143,7 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
         mbar_fence_init();
         tma_prefetch_desc(&tmx);
         tma_prefetch_desc(&tmw);
+        tma_prefetch_desc(&tmd);
     }
     tc_fence_before();
     __syncthreads();
@@ -137,69 +154,90 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
                        ? (pp.ntiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
                        : 0;
     const int njobs = nt * ng;   // job j = tile k (k-th of this CTA), group g: j = k ng + g
+    auto row0_of = [&](int k) {
+        return (k * static_cast<int>(gridDim.x) + static_cast<int>(blockIdx.x)) * kRows;
+    };
 
-    if (warp == 0) {
-        if (lane == 0 && nt > 0) {
-            auto load_x = [&](int k) {
-                const int s = k % xbufs;
-                mbar_arrive_expect_tx(&bar[PB_XF + s], kBoxBytes);
-                tma_load_2d(sm + L.x + s * kBoxBytes, &tmx, &bar[PB_XF + s], 0,
-                            (k * static_cast<int>(gridDim.x) + static_cast<int>(blockIdx.x)) * kRows);
-            };
-            mbar_arrive_expect_tx(&bar[PB_W], (pp.F / 32) * kSubBytes);
-            for (int n = 0; n < pp.F / 32; ++n)
-                tma_load_2d(sm + L.w + n * kSubBytes, &tmw, &bar[PB_W], 0, n * 64);
-            for (int k = 0; k < xbufs && k < nt; ++k) load_x(k);
-            {
-                uint32_t ph = 0;
-                wt.wait(&bar[PB_W], ph);
+    if (warp == 9) {
+        // ---------------------------------------------------------------- TMA loads, in
+        // job order: the X tile at each tile's first group, then per job its W group and its
+        // dphi tile, each into a slot freed by the job kRing (X: kXBufs tiles) before
+        if (lane == 0) {
+            Ring xr(kXBufs), rr(kRing);
+            for (int j = 0, k = 0, g = 0; j < njobs && wt.ok; ++j) {
+                if (g == 0) {
+                    if (xr.use >= 1) {
+                        uint32_t ph = static_cast<uint32_t>((xr.use - 1) & 1);
+                        wt.wait(&bar[PB_XE + xr.slot], ph);
+                    }
+                    mbar_arrive_expect_tx(&bar[PB_XF + xr.slot], kBoxBytes);
+                    tma_load_2d(sm + L.x + xr.slot * kBoxBytes, &tmx, &bar[PB_XF + xr.slot], 0, row0_of(k));
+                    xr.next();
+                }
+                if (rr.use >= 1) {
+                    uint32_t ph = static_cast<uint32_t>((rr.use - 1) & 1);
+                    wt.wait(&bar[PB_WE + rr.slot], ph);
+                }
+                mbar_arrive_expect_tx(&bar[PB_WF + rr.slot], kGroupBytes);
+                unsigned char* wd = sm + L.w + rr.slot * kGroupBytes;
+                tma_load_2d(wd, &tmw, &bar[PB_WF + rr.slot], 0, (2 * g) * 64);
+                tma_load_2d(wd + kSubBytes, &tmw, &bar[PB_WF + rr.slot], 0, (2 * g + 1) * 64);
+                if (rr.use >= 1) {
+                    uint32_t ph = static_cast<uint32_t>((rr.use - 1) & 1);
+                    wt.wait(&bar[PB_GE + rr.slot], ph);
+                }
+                mbar_arrive_expect_tx(&bar[PB_GF + rr.slot], kBoxBytes);
+                tma_load_2d(sm + L.d + rr.slot * kBoxBytes, &tmd, &bar[PB_GF + rr.slot], 64 * g, row0_of(k));
+                rr.next();
+                if (++g == ng) {
+                    g = 0;
+                    ++k;
+                }
             }
+        }
+        __syncwarp();
+    } else if (warp == 0) {
+        // ---------------------------------------------------------------- MMA issue
+        if (lane == 0 && nt > 0) {
             constexpr uint32_t idU = idesc_bf16(128, 128, 0, 0);   // X (K-major) x W (K-major)
             constexpr uint32_t idD = idesc_bf16(128, 64, 0, 1);    // [alpha|beta] x W (MN-major)
             const uint64_t dx0 = sdesc(sbase + L.x, 16, 1024, kLayoutSW128);
             const uint64_t dw0 = sdesc(sbase + L.w, 16, 1024, kLayoutSW128);
             const uint64_t da0 = sdesc(sbase + L.a, 16, 1024, kLayoutSW128);
-            // projection job jp = (tile pk, group pg); X slot ps of tile pk and its phase
-            int jp = 0, pk = 0, pg = 0, ps = 0;
-            uint32_t pph = 0;
+            // projection job jp = (tile pk, group pg) from X slot px and W slot pw
+            int jp = 0, pg = 0;
+            Ring px(kXBufs), pw(kRing);
             auto proj = [&]() {   // U[jp & 1] = X_pk W_pg^T, then advance to the next job
                 if (pg == 0) {
-                    uint32_t ph = pph;
-                    wt.wait(&bar[PB_XF + ps], ph);
+                    uint32_t ph = static_cast<uint32_t>(px.use & 1);
+                    wt.wait(&bar[PB_XF + px.slot], ph);
+                }
+                {
+                    uint32_t ph = static_cast<uint32_t>(pw.use & 1);
+                    wt.wait(&bar[PB_WF + pw.slot], ph);
                 }
                 tc_fence_after();
-                const uint64_t dx = dx0 + ((ps * kBoxBytes) >> 4);
-                const uint64_t dw = dw0 + ((pg * kGroupBytes) >> 4);
+                const uint64_t dx = dx0 + ((px.slot * kBoxBytes) >> 4);
+                const uint64_t dw = dw0 + ((pw.slot * kGroupBytes) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     umma_bf16(tmem0 + kColU + 128u * (jp & 1), dx + 2 * kk, dw + 2 * kk, idU,
                               kk > 0 ? 1u : 0u);
                 umma_commit(&bar[PB_UF + (jp & 1)]);
                 ++jp;
+                pw.next();
                 if (++pg == ng) {
                     pg = 0;
-                    ++pk;
-                    if (++ps == xbufs) {
-                        ps = 0;
-                        pph ^= 1u;
-                    }
+                    px.next();
                 }
             };
             proj();
             if (njobs > 1) proj();
-            int k = 0, g = 0, xs_prev = xbufs - 1;   // contraction job j = (tile k, group g)
-            uint32_t xph_prev = 1;                    // phase of X slot of tile k - 1
-            for (int j = 0; j < njobs && wt.ok; ++j) {
+            Ring cw(kRing);   // W slot of contraction job j
+            for (int j = 0, k = 0, g = 0; j < njobs && wt.ok; ++j) {
                 {
                     uint32_t ph = static_cast<uint32_t>((j >> 1) & 1);
                     wt.wait(&bar[PB_AF + (j & 1)], ph);   // [alpha|beta]_j written, U_j read
-                }
-                if (g == 0 && k >= 1) {
-                    // every epilogue warp is past the dx of tile k - 1 (it wrote A of job j
-                    // after it): X slot (k - 1) % xbufs takes tile k - 1 + xbufs
-                    uint32_t ph = xph_prev;
-                    wt.wait(&bar[PB_XE + xs_prev], ph);
-                    if (k - 1 + xbufs < nt) load_x(k - 1 + xbufs);
                 }
                 if (g == 0 && k >= 2) {   // dX^ buffer k & 1 read by the dx of tile k - 2
                     uint32_t ph = static_cast<uint32_t>(((k - 2) >> 1) & 1);
@@ -209,22 +247,20 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
                 // dX^_k += [alpha|beta]_j [Omega_g ; A_g]: K = 128 (two 64-wide K-tiles of
                 // the operand; the W rows of the group 2 KiB per 16-row K step)
                 const uint64_t da = da0 + (((j & 1) * kABytes) >> 4);
-                const uint64_t dwm = dw0 + ((g * kGroupBytes) >> 4);   // same tiles, MN-major
+                const uint64_t dwm = dw0 + ((cw.slot * kGroupBytes) >> 4);   // same tiles, MN-major
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     umma_bf16(tmem0 + kColDX + 64u * (k & 1),
                               da + (kk >> 2) * (kBoxBytes >> 4) + 2 * (kk & 3), dwm + 128 * kk, idD,
                               (g > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(&bar[PB_AE + (j & 1)]);
+                umma_commit(&bar[PB_WE + cw.slot]);   // the group's W (projection and contraction) done
                 if (g == ng - 1) umma_commit(&bar[PB_DF + (k & 1)]);
+                cw.next();
                 if (j + 2 < njobs) proj();   // job j + 2 into U[j & 1], read already (AF)
                 if (++g == ng) {
                     g = 0;
                     ++k;
-                    if (++xs_prev == xbufs) {
-                        xs_prev = 0;
-                        xph_prev ^= 1u;
-                    }
                 }
             }
         }
@@ -234,37 +270,11 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
         const uint32_t row = 32u * q + lane;
         const uint32_t trow = tmem0 + ((32u * q) << 16);
         const uint32_t abase = sbase + L.a + half * kBoxBytes;
-        const int F = pp.F;
-        // dphi of (tile k, group g) for this lane's row: 32 values (features 64g + 32 half ..)
-        auto dphi_ptr = [&](int k, int g) -> const uint4* {
-            const int64_t r = static_cast<int64_t>(k * static_cast<int>(gridDim.x) +
-                                                   static_cast<int>(blockIdx.x)) * kRows + row;
-            const int64_t rr = r < n_rows ? r : n_rows - 1;   // rows past the end: any valid row
-            return reinterpret_cast<const uint4*>(dphi + rr * F + 64 * g + 32 * half);
-        };
-        // dphi ring: kPre groups in flight ahead of the one being consumed (a warp's 32
-        // rows x 64 bytes per group; at one group ahead the loads' DRAM latency, not the
-        // bandwidth, set the pace).  (fk, fg) is the next job to fetch.
-        uint4 pf[kPre][kW];
-        int fk = 0, fg = 0, fetched = 0;
-        auto fetch = [&](uint4 (&dst)[kW]) {
-            if (fetched < njobs) {
-                const uint4* p = dphi_ptr(fk, fg);
-#pragma unroll
-                for (int i = 0; i < kW; ++i) dst[i] = __ldg(p + i);
-                if (++fg == ng) {
-                    fg = 0;
-                    ++fk;
-                }
-                ++fetched;
-            }
-        };
-#pragma unroll
-        for (int d = 0; d < kPre; ++d) fetch(pf[d]);
+        Ring xring(kXBufs), dr(kRing);
         for (int k = 0; k < nt; ++k) {
-            const int s = k % xbufs;
+            const int s = xring.slot;
             {
-                uint32_t ph = static_cast<uint32_t>((k / xbufs) & 1);
+                uint32_t ph = static_cast<uint32_t>(xring.use & 1);
                 wt.wait(&bar[PB_XF + s], ph);
             }
             float inv, l2i;
@@ -273,14 +283,18 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
             const float nrm = 1.0f / inv, two_n = 2.0f * nrm;
             for (int g = 0; g < ng; ++g) {
                 const int j = k * ng + g;
+                // this row's 32 dphi of the group from the TMA tile (128-byte swizzle: 16-byte
+                // chunk c of row r at c ^ (r & 7)); the slot is released at once
                 uint4 dp[kW];
+                {
+                    uint32_t ph = static_cast<uint32_t>(dr.use & 1);
+                    wt.wait(&bar[PB_GF + dr.slot], ph);
+                }
+                const uint4* drow = reinterpret_cast<const uint4*>(sm + L.d + dr.slot * kBoxBytes + row * 128);
 #pragma unroll
-                for (int i = 0; i < kW; ++i) dp[i] = pf[0][i];
-#pragma unroll
-                for (int d = 0; d + 1 < kPre; ++d)
-#pragma unroll
-                    for (int i = 0; i < kW; ++i) pf[d][i] = pf[d + 1][i];
-                fetch(pf[kPre - 1]);   // job j + kPre
+                for (int i = 0; i < kW; ++i) dp[i] = drow[(4 * half + i) ^ (row & 7)];
+                warp_arrive(&bar[PB_GE + dr.slot]);
+                dr.next();
                 {
                     uint32_t ph = static_cast<uint32_t>((j >> 1) & 1);
                     wt.wait(&bar[PB_UF + (j & 1)], ph);
@@ -388,6 +402,7 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
                 }
             }
             warp_arrive(&bar[PB_XE + s]);   // this warp is done with X slot s
+            xring.next();
         }
     }
     wt.report(status);
@@ -411,10 +426,11 @@ cudaError_t tc_phi_bwd(const void* x, const void* dphi, float* dx, int64_t n, co
 {
     const int F = P.F;
     if (!P.wB || !tc_phi_bwd_supported(64, P.R, P.m, n)) return cudaErrorNotSupported;
-    CUtensorMap mx, mw;
+    CUtensorMap mx, mw, md;
     if (!map_2d(&mx, x, 64, static_cast<uint64_t>(n), 64, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map_2d(&mw, P.wB, 64, static_cast<uint64_t>(F / 32) * 64, 64, 64,
-                CU_TENSOR_MAP_SWIZZLE_128B))
+                CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map_2d(&md, dphi, F, static_cast<uint64_t>(n), 64, kRows, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     PbParams pp;
     pp.F = F;
@@ -435,8 +451,7 @@ cudaError_t tc_phi_bwd(const void* x, const void* dphi, float* dx, int64_t n, co
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     TraceScope trace_("tc_phi_bwd", st);
-    k_tc_phi_bwd<<<grid, kPbThreads, smem, st>>>(mx, mw, static_cast<const __nv_bfloat16*>(dphi), dx,
-                                                 n, pp, status);
+    k_tc_phi_bwd<<<grid, kPbThreads, smem, st>>>(mx, mw, md, dx, n, pp, status);
     return cudaGetLastError();
 }
 
