@@ -270,7 +270,74 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
         const uint32_t row = 32u * q + lane;
         const uint32_t trow = tmem0 + ((32u * q) << 16);
         const uint32_t abase = sbase + L.a + half * kBoxBytes;
+        // dx of tile k (X slot s, its rows' 1/|x| and |x|): dX^ (64 columns) -> (dX^ - x^
+        // (x^ . dX^)) / n, this warp's half.  It runs after the next tile's jobs, so the wait
+        // for the tile's last contraction is hidden behind them (dX^ is double buffered; the
+        // X slot is released here, with kXBufs tiles in flight).
+        auto dx_tile = [&](int k, int s, float inv, float nrm) {
+            const unsigned char* xrow = sm + L.x + s * kBoxBytes + row * 128;
+            {
+                uint32_t ph = static_cast<uint32_t>((k >> 1) & 1);
+                wt.wait(&bar[PB_DF + (k & 1)], ph);
+            }
+            tc_fence_after();
+            uint32_t d0[32], d1[32];
+            tmem_ld32(trow + kColDX + 64u * (k & 1), d0);
+            tmem_ld32(trow + kColDX + 64u * (k & 1) + 32, d1);
+            tmem_wait_ld();
+            reg_fence(d0);
+            reg_fence(d1);
+            tc_fence_before();
+            warp_arrive(&bar[PB_DE + (k & 1)]);
+            // x^ of this row from the X tile (bf16, 128-byte swizzle: 16-byte chunk c of the
+            // row at c ^ (row & 7)), read where it is used so that it holds no registers
+            const uint4* xr = reinterpret_cast<const uint4*>(xrow);
+            float dot[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint4 w4 = xr[c ^ (row & 7)];
+                const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = 8 * c + 2 * e;   // element index 0..63
+                    const float lo = __uint_as_float(ws[e] << 16);
+                    const float hi = __uint_as_float(ws[e] & 0xFFFF0000u);
+                    const float dlo = i < 32 ? __uint_as_float(d0[i]) : __uint_as_float(d1[i - 32]);
+                    const float dhi = i < 32 ? __uint_as_float(d0[i + 1]) : __uint_as_float(d1[i - 31]);
+                    dot[e] = fmaf(lo, dlo, dot[e]);
+                    dot[e] = fmaf(hi, dhi, dot[e]);
+                }
+            }
+            // below the 1e-12 norm guard x^ = x / 1e-12 is not a unit vector and its
+            // derivative is the identity / 1e-12: no tangential projection there
+            const float xd = nrm > 1e-12f ? ((dot[0] + dot[1]) + (dot[2] + dot[3])) * inv : 0.0f;
+            const int64_t r = static_cast<int64_t>(k * static_cast<int>(gridDim.x) +
+                                                   static_cast<int>(blockIdx.x)) * kRows + row;
+            if (r < n_rows) {
+                float4* dst = reinterpret_cast<float4*>(dx + r * 64 + 32 * half);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {   // this warp's 32 columns: chunks 4 half .. + 3
+                    const uint4 w4 = xr[(4 * half + c) ^ (row & 7)];
+                    const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
+                    float o[8];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = 8 * c + 2 * e;   // column within the half
+                        // selects, not an indexed pointer (local memory)
+                        const float dlo = half ? __uint_as_float(d1[i]) : __uint_as_float(d0[i]);
+                        const float dhi = half ? __uint_as_float(d1[i + 1]) : __uint_as_float(d0[i + 1]);
+                        o[2 * e] = (dlo - __uint_as_float(ws[e] << 16) * inv * xd) * inv;
+                        o[2 * e + 1] = (dhi - __uint_as_float(ws[e] & 0xFFFF0000u) * inv * xd) * inv;
+                    }
+                    dst[2 * c] = make_float4(o[0], o[1], o[2], o[3]);
+                    dst[2 * c + 1] = make_float4(o[4], o[5], o[6], o[7]);
+                }
+            }
+            warp_arrive(&bar[PB_XE + s]);   // this warp is done with X slot s
+        };
         Ring xring(kXBufs), dr(kRing);
+        int ps = 0;                     // X slot of the tile whose dx is pending
+        float pinv = 1.0f, pnrm = 1.0f;
         for (int k = 0; k < nt; ++k) {
             const int s = xring.slot;
             {
@@ -343,67 +410,13 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
                 tc_fence_before();
                 warp_arrive(&bar[PB_AF + (j & 1)]);
             }
-            // dx of tile k: dX^ (64 columns) -> (dX^ - x^ (x^ . dX^)) / n, this warp's half
-            {
-                uint32_t ph = static_cast<uint32_t>((k >> 1) & 1);
-                wt.wait(&bar[PB_DF + (k & 1)], ph);
-            }
-            tc_fence_after();
-            uint32_t d0[32], d1[32];
-            tmem_ld32(trow + kColDX + 64u * (k & 1), d0);
-            tmem_ld32(trow + kColDX + 64u * (k & 1) + 32, d1);
-            tmem_wait_ld();
-            reg_fence(d0);
-            reg_fence(d1);
-            tc_fence_before();
-            warp_arrive(&bar[PB_DE + (k & 1)]);
-            // x^ of this row from the X tile (bf16, 128-byte swizzle: 16-byte chunk c of the
-            // row at c ^ (row & 7)), read where it is used so that it holds no registers
-            const uint4* xr = reinterpret_cast<const uint4*>(xrow);
-            float dot[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 w4 = xr[c ^ (row & 7)];
-                const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int i = 8 * c + 2 * e;   // element index 0..63
-                    const float lo = __uint_as_float(ws[e] << 16);
-                    const float hi = __uint_as_float(ws[e] & 0xFFFF0000u);
-                    const float dlo = i < 32 ? __uint_as_float(d0[i]) : __uint_as_float(d1[i - 32]);
-                    const float dhi = i < 32 ? __uint_as_float(d0[i + 1]) : __uint_as_float(d1[i - 31]);
-                    dot[e] = fmaf(lo, dlo, dot[e]);
-                    dot[e] = fmaf(hi, dhi, dot[e]);
-                }
-            }
-            // below the 1e-12 norm guard x^ = x / 1e-12 is not a unit vector and its
-            // derivative is the identity / 1e-12: no tangential projection there
-            const float xd = nrm > 1e-12f ? ((dot[0] + dot[1]) + (dot[2] + dot[3])) * inv : 0.0f;
-            const int64_t r = static_cast<int64_t>(k * static_cast<int>(gridDim.x) +
-                                                   static_cast<int>(blockIdx.x)) * kRows + row;
-            if (r < n_rows) {
-                float4* dst = reinterpret_cast<float4*>(dx + r * 64 + 32 * half);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {   // this warp's 32 columns: chunks 4 half .. + 3
-                    const uint4 w4 = xr[(4 * half + c) ^ (row & 7)];
-                    const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
-                    float o[8];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i = 8 * c + 2 * e;   // column within the half
-                        // selects, not an indexed pointer (local memory)
-                        const float dlo = half ? __uint_as_float(d1[i]) : __uint_as_float(d0[i]);
-                        const float dhi = half ? __uint_as_float(d1[i + 1]) : __uint_as_float(d0[i + 1]);
-                        o[2 * e] = (dlo - __uint_as_float(ws[e] << 16) * inv * xd) * inv;
-                        o[2 * e + 1] = (dhi - __uint_as_float(ws[e] & 0xFFFF0000u) * inv * xd) * inv;
-                    }
-                    dst[2 * c] = make_float4(o[0], o[1], o[2], o[3]);
-                    dst[2 * c + 1] = make_float4(o[4], o[5], o[6], o[7]);
-                }
-            }
-            warp_arrive(&bar[PB_XE + s]);   // this warp is done with X slot s
+            if (k >= 1) dx_tile(k - 1, ps, pinv, pnrm);
+            ps = s;
+            pinv = inv;
+            pnrm = nrm;
             xring.next();
         }
+        if (nt > 0) dx_tile(nt - 1, ps, pinv, pnrm);
     }
     wt.report(status);
     drain_after_failure(wt.ok);
