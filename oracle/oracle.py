@@ -78,6 +78,9 @@ def lib():
         L.orc_attn_causal_state.argtypes = [dp, dp, dp, dp, dp] + shp + par + [C.c_double,
                                                                              dp, dp, dp, dp]
         L.orc_attn_causal_state.restype = None
+        L.orc_attn_causal_bwd_state.argtypes = ([dp] * 10 + shp + par +
+                                                [C.c_double, dp, dp, dp, dp, dp])
+        L.orc_attn_causal_bwd_state.restype = None
         L.orc_num_threads.argtypes = []
         L.orc_num_threads.restype = C.c_int
         _lib = L
@@ -356,10 +359,32 @@ def attn_causal_state(q, k, v, P: Params, S0=None, z0=None):
     return out, den, S1, z1
 
 
+def attn_causal_bwd_state(q, k, v, out, den, dout, P: Params, S_in=None, z_in=None, G_in=None,
+                          zg_in=None):
+    """Backward of one piece of a longer causal sequence at its given forward output: S_in
+    [B,H,F,Dv], z_in [B,H,F] sum phi(k)[v, 1] over the tokens before the piece, G_in, zg_in
+    sum phi(q)[dn, delta] over the tokens after it (None = zero).  Returns (dq, dk, dv,
+    G_out, zg_out), the last two the piece's own sum of phi(q)[dn, delta]."""
+    q, k, v, o, dn, g = _d(q), _d(k), _d(v), _d(out), _d(den), _d(dout)
+    B, H, L, D, Dv = _shape4(q, v)
+    F = P.F
+    dq = np.zeros(q.shape)
+    dk = np.zeros(k.shape)
+    dv = np.zeros(v.shape)
+    G_out = np.zeros((B, H, F, Dv))
+    zg_out = np.zeros((B, H, F))
+    st = [None if x is None else _d(x) for x in (S_in, z_in, G_in, zg_in)]
+    lib().orc_attn_causal_bwd_state(_p(q), _p(k), _p(v), _p(o), _p(dn), _p(g),
+                                    *[None if x is None else _p(x) for x in st],
+                                    B, H, L, D, Dv, P.R, P.m, *P.args(), P.eps,
+                                    _p(dq), _p(dk), _p(dv), _p(G_out), _p(zg_out))
+    return dq, dk, dv, G_out, zg_out
+
+
 __all__ = ["lib", "num_threads", "philox4x32_10", "gauss_laguerre", "Params", "sketch_params",
            "yat_kernel", "quad_kernel", "feature_map", "attn_quadratic", "attn_quadratic_rows",
            "attn_recurrent", "decode_step", "attn_causal_bwd", "attn_causal_bwd_rows",
            "attn_causal_bwd_given", "attn_causal_bwd_given_rows", "feature_map_bwd",
            "attn_bidir_bwd", "attn_bidir_bwd_given", "KindParams", "sketch_params_kind",
            "feature_map_kind", "attn_from_phi", "PHI_ANCHOR", "PHI_ORTHOGONAL", "PHI_SIGNED",
-           "PHI_PER_HEAD", "PHI_PERFORMER", "attn_causal_state"]
+           "PHI_PER_HEAD", "PHI_PERFORMER", "attn_causal_state", "attn_causal_bwd_state"]

@@ -650,6 +650,107 @@ void orc_attn_causal_bwd_given(const double* q, const double* k, const double* v
     }
 }
 
+/* The backward of one piece of a longer causal sequence, split over ranks (the prefix state
+ * of the review's "Proposed method", step 6, carried across the split in both directions),
+ * at the piece's given forward output out, den_in (its rows of the whole sequence's
+ * forward).  S_in [BH][F][Dv], z_in [BH][F]: the sum of phi(k_j) [v_j, 1] over the tokens
+ * before the piece; G_in [BH][F][Dv], zg_in [BH][F]: the sum of phi(q_i) [dn_i, delta_i] over
+ * the tokens after it (NULL = zero).  The whole-sequence derivative of
+ * orc_attn_causal_bwd_given, restricted to the piece's rows, is then
+ *   dphi(q_i) = sum_{j<=i in the piece} c_ij phi(k_j) + S_in dn_i + z_in delta_i
+ *   dphi(k_j) = sum_{i>=j in the piece} c_ij phi(q_i) + G_in v_j + zg_in
+ *   dv_j      = sum_{i>=j in the piece} a_ij dn_i + G_in^T phi(k_j)
+ * G_out, zg_out (NULL = not wanted): the piece's own sum of phi(q_i) [dn_i, delta_i], the
+ * G_in of the pieces before it. */
+void orc_attn_causal_bwd_state(const double* q, const double* k, const double* v,
+                               const double* out, const double* den_in, const double* dout,
+                               const double* S_in, const double* z_in,
+                               const double* G_in, const double* zg_in,
+                               int B, int H, int L, int D, int Dv, int R, int m,
+                               const double* omega, const double* anchors,
+                               const double* s, const double* wt, double eps,
+                               double* dq, double* dk, double* dv,
+                               double* G_out, double* zg_out)
+{
+    const int64_t F = (int64_t)R * m;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bh = 0; bh < B * H; ++bh) {
+        const double* qs = q + (int64_t)bh * L * D;
+        const double* ks = k + (int64_t)bh * L * D;
+        const double* vs = v + (int64_t)bh * L * Dv;
+        const double* os = out + (int64_t)bh * L * Dv;
+        const double* ds = den_in + (int64_t)bh * L;
+        const double* gs = dout + (int64_t)bh * L * Dv;
+        const double* Si = S_in ? S_in + (int64_t)bh * F * Dv : NULL;
+        const double* zi = z_in ? z_in + (int64_t)bh * F : NULL;
+        const double* Gi = G_in ? G_in + (int64_t)bh * F * Dv : NULL;
+        const double* zgi = zg_in ? zg_in + (int64_t)bh * F : NULL;
+        double* pq = phi_slice(qs, L, D, R, m, omega, anchors, s, wt);
+        double* pk = phi_slice(ks, L, D, R, m, omega, anchors, s, wt);
+        double* dn = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1) * Dv);
+        double* delta = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+        for (int i = 0; i < L; ++i) {
+            double Z = ds[i] + eps;
+            for (int e = 0; e < Dv; ++e) dn[(int64_t)i * Dv + e] = gs[(int64_t)i * Dv + e] / Z;
+            delta[i] = -dot(gs + (int64_t)i * Dv, os + (int64_t)i * Dv, Dv) / Z;
+        }
+        double* dpq = (double*)calloc((size_t)(L > 0 ? L : 1) * F, sizeof(double));
+        double* dpk = (double*)calloc((size_t)(L > 0 ? L : 1) * F, sizeof(double));
+        double* dvs = dv + (int64_t)bh * L * Dv;
+        for (int64_t t = 0; t < (int64_t)L * Dv; ++t) dvs[t] = 0.0;
+        /* the piece's own pairs */
+        for (int i = 0; i < L; ++i) {
+            for (int j = 0; j <= i; ++j) {
+                double c = dot(vs + (int64_t)j * Dv, dn + (int64_t)i * Dv, Dv) + delta[i];
+                double a = dot(pq + (int64_t)i * F, pk + (int64_t)j * F, F);
+                for (int64_t f = 0; f < F; ++f) {
+                    dpq[(int64_t)i * F + f] += c * pk[(int64_t)j * F + f];
+                    dpk[(int64_t)j * F + f] += c * pq[(int64_t)i * F + f];
+                }
+                for (int e = 0; e < Dv; ++e)
+                    dvs[(int64_t)j * Dv + e] += a * dn[(int64_t)i * Dv + e];
+            }
+        }
+        /* the pairs with tokens before the piece (through S_in, z_in) and after it (G_in,
+         * zg_in) */
+        for (int i = 0; i < L; ++i) {
+            for (int64_t f = 0; f < F; ++f) {
+                double sq = 0.0, sk = 0.0;
+                if (Si) sq = dot(Si + f * Dv, dn + (int64_t)i * Dv, Dv) + zi[f] * delta[i];
+                if (Gi) sk = dot(Gi + f * Dv, vs + (int64_t)i * Dv, Dv) + zgi[f];
+                dpq[(int64_t)i * F + f] += sq;
+                dpk[(int64_t)i * F + f] += sk;
+            }
+            if (Gi)
+                for (int e = 0; e < Dv; ++e) {
+                    double acc = 0.0;
+                    for (int64_t f = 0; f < F; ++f) acc += Gi[f * Dv + e] * pk[(int64_t)i * F + f];
+                    dvs[(int64_t)i * Dv + e] += acc;
+                }
+        }
+        for (int i = 0; i < L; ++i) {
+            phi_backward_row(qs + (int64_t)i * D, dpq + (int64_t)i * F, D, R, m,
+                             omega, anchors, s, wt, dq + ((int64_t)bh * L + i) * D);
+            phi_backward_row(ks + (int64_t)i * D, dpk + (int64_t)i * F, D, R, m,
+                             omega, anchors, s, wt, dk + ((int64_t)bh * L + i) * D);
+        }
+        if (G_out)
+            for (int64_t f = 0; f < F; ++f)
+                for (int e = 0; e < Dv; ++e) {
+                    double acc = 0.0;
+                    for (int i = 0; i < L; ++i) acc += pq[(int64_t)i * F + f] * dn[(int64_t)i * Dv + e];
+                    G_out[((int64_t)bh * F + f) * Dv + e] = acc;
+                }
+        if (zg_out)
+            for (int64_t f = 0; f < F; ++f) {
+                double acc = 0.0;
+                for (int i = 0; i < L; ++i) acc += pq[(int64_t)i * F + f] * delta[i];
+                zg_out[(int64_t)bh * F + f] = acc;
+            }
+        free(pq); free(pk); free(dn); free(delta); free(dpq); free(dpk);
+    }
+}
+
 /* orc_attn_causal_bwd_given at the listed rows only (rows[r] is a query row for dq and a
  * key row for dk, dv), for sequences too long for the full form. */
 void orc_attn_causal_bwd_given_rows(const double* q, const double* k, const double* v,

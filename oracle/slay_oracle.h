@@ -115,6 +115,15 @@ void orc_attn_causal_bwd_given(const double* q, const double* k, const double* v
                                const double* omega, const double* anchors,
                                const double* s, const double* wt, double eps,
                                double* dq, double* dk, double* dv);
+void orc_attn_causal_bwd_state(const double* q, const double* k, const double* v,
+                               const double* out, const double* den_in, const double* dout,
+                               const double* S_in, const double* z_in,
+                               const double* G_in, const double* zg_in,
+                               int B, int H, int L, int D, int Dv, int R, int m,
+                               const double* omega, const double* anchors,
+                               const double* s, const double* wt, double eps,
+                               double* dq, double* dk, double* dv,
+                               double* G_out, double* zg_out);
 void orc_attn_causal_bwd_given_rows(const double* q, const double* k, const double* v,
                                     const double* out, const double* den,
                                     const double* dout,

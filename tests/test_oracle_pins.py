@@ -617,3 +617,47 @@ def test_causal_state_is_the_decode_recurrence():
         np.testing.assert_allclose(out[:, :, i], o, rtol=1e-11, atol=1e-14)
     np.testing.assert_allclose(S1, S, rtol=1e-12, atol=1e-16)
     np.testing.assert_allclose(z1, z, rtol=1e-12)
+
+
+# ---------------------------------------------------- backward of a piece of a sequence
+def test_piece_backward_without_states_is_the_given_backward():
+    # no tokens before or after the piece: the whole-sequence backward at the given output
+    q, k, v = _small(54, B=2, H=1, L=17, D=8, Dv=4)
+    P = O.sketch_params(D=8, R=2, m=5, seed=9, eps=1e-6)
+    out, den = O.attn_quadratic(q, k, v, P, True)
+    g = np.random.default_rng(55).standard_normal(v.shape)
+    want = O.attn_causal_bwd_given(q, k, v, out, den, g, P)
+    got = O.attn_causal_bwd_state(q, k, v, out, den, g, P)
+    for a, b in zip(got[:3], want):
+        np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-15)
+
+
+@pytest.mark.parametrize("cuts", [(7, 16), (1, 22), (11,)])
+def test_piece_backward_chains_to_the_whole_sequence(cuts):
+    # sequence parallelism backward: each piece takes the forward state of the pieces before
+    # it (S_in, z_in) and the sum of the later pieces' phi(q)[dn, delta] (G_in, zg_in); the
+    # pieces' gradients are the whole sequence's (pinned by finite differences)
+    q, k, v = _small(56, B=2, H=1, L=23, D=8, Dv=4)
+    P = O.sketch_params(D=8, R=2, m=5, seed=9, eps=1e-6)
+    g = np.random.default_rng(57).standard_normal(v.shape)
+    out, den = O.attn_quadratic(q, k, v, P, True)
+    want = O.attn_causal_bwd(q, k, v, g, P)
+    bounds = (0,) + tuple(cuts) + (23,)
+    pieces = list(zip(bounds[:-1], bounds[1:]))
+    S_in, S, z = [], None, None
+    for a, b in pieces:                  # forward states entering each piece
+        S_in.append((S, z))
+        _, _, S, z = O.attn_causal_state(q[:, :, a:b], k[:, :, a:b], v[:, :, a:b], P, S, z)
+    got = [None] * len(pieces)
+    G, zg = None, None
+    for p in reversed(range(len(pieces))):   # later pieces first: their G sums the suffix
+        a, b = pieces[p]
+        sl = (slice(None), slice(None), slice(a, b))
+        dq, dk, dv, Go, zgo = O.attn_causal_bwd_state(q[sl], k[sl], v[sl], out[sl], den[sl], g[sl],
+                                                      P, *S_in[p], G, zg)
+        got[p] = (dq, dk, dv)
+        G = Go if G is None else G + Go
+        zg = zgo if zg is None else zg + zgo
+    for i in range(3):
+        np.testing.assert_allclose(np.concatenate([x[i] for x in got], axis=2), want[i],
+                                   rtol=1e-9, atol=1e-12)
