@@ -157,6 +157,13 @@ slay_status slay_causal_state(const void* k, const void* v, const float* S_in, c
 slay_status slay_state_prefix(const float* S_all, const float* z_all, int nranks, int rank,
                               float* S_in, float* z_in, int BH, int F, int Dv, void* stream);
 
+/* The counterpart of slay_state_prefix for the backward (sequence parallelism):
+ *   S_out = sum_{r > rank} S_all[r],  z_out = sum_{r > rank} z_all[r]
+ * the sum of the states of the ranks after this one (zero for the last rank).  Layouts and
+ * limits as slay_state_prefix. */
+slay_status slay_state_suffix(const float* S_all, const float* z_all, int nranks, int rank,
+                              float* S_out, float* z_out, int BH, int F, int Dv, void* stream);
+
 /* Bidirectional SLAY attention forward: as above with S, z summed over all keys
  * (review, "Proposed method", step 6, non-causal form).  Same arguments; workspace
  * size from slay_workspace_bytes(SLAY_OP_BIDIR_FWD, ...). */
@@ -183,6 +190,37 @@ slay_status slay_attn_causal_bwd(const void* q, const void* k, const void* v,
                                  int B, int H, int L, int D, int Dv,
                                  slay_dtype dt, int R, int m, uint64_t seed, float eps,
                                  void* workspace, size_t ws_bytes, void* stream);
+
+/* Backward of one piece of a longer causal sequence (sequence parallelism: the prefix state
+ * of the review's "Proposed method", step 6, split across ranks, in the backward direction).
+ * Arguments as slay_attn_causal_bwd (same workspace size; out, den: this piece's rows of the
+ * whole sequence's forward, e.g. from slay_attn_causal_fwd_state), plus:
+ * S_in, z_in  : device [B,H,R*m,Dv] and [B,H,R*m] fp32, sum_j phi(k_j) [v_j, 1] over the tokens
+ *               before the piece (the forward's S_in), or both NULL;
+ * G_in, zg_in : same shapes, sum_i phi(q_i) [dn_i, delta_i] over the tokens after the piece
+ *               (dn_i = dout_i / (den_i + eps), delta_i = -<dout_i, out_i> / (den_i + eps); the
+ *               later ranks' slay_causal_bwd_state results summed, see slay_state_suffix), or
+ *               both NULL.
+ * Then dq, dk, dv of the piece's rows equal the whole sequence's.  With all four NULL the
+ * call equals slay_attn_causal_bwd.  16-byte aligned. */
+slay_status slay_attn_causal_bwd_state(const void* q, const void* k, const void* v,
+                                       const void* out, const float* den, const void* dout,
+                                       float* dq, float* dk, float* dv, const float* S_in,
+                                       const float* z_in, const float* G_in, const float* zg_in,
+                                       int B, int H, int L, int D, int Dv, slay_dtype dt, int R,
+                                       int m, uint64_t seed, float eps, void* workspace,
+                                       size_t ws_bytes, void* stream);
+
+/* A piece's G state for the pieces before it:
+ *   G_out = sum_i phi(q_i) dn_i^T,  zg_out = sum_i phi(q_i) delta_i
+ * over its L tokens (dn, delta as in slay_attn_causal_bwd_state), G_out [B,H,R*m,Dv] and
+ * zg_out [B,H,R*m] fp32, written (zero when L == 0).  q, out, dout in `dt`, den fp32; workspace
+ * slay_workspace_bytes(SLAY_OP_CAUSAL_BWD, ...).  bf16 at tensor-core sizes: phi(q) and the
+ * running sums on tensor cores; otherwise CUDA cores. */
+slay_status slay_causal_bwd_state(const void* q, const void* out, const float* den,
+                                  const void* dout, float* G_out, float* zg_out, int B, int H,
+                                  int L, int D, int Dv, slay_dtype dt, int R, int m, uint64_t seed,
+                                  float eps, void* workspace, size_t ws_bytes, void* stream);
 
 /* Backward of the bidirectional forward: gradients of sum_i <dout_i, out_i> with respect
  * to q, k, v (the pages give no backward; it is the derivative of slay_attn_bidir_fwd).

@@ -27,7 +27,8 @@ EXPORTS = ["slay_feature_map", "slay_attn_causal_fwd", "slay_attn_bidir_fwd",
            "slay_trace_read", "slay_attn_causal_fwd_noalloc", "slay_kernel_status",
            "slay_debug_expire_wait", "slay_attn_bidir_bwd", "slay_feature_map_bwd",
            "slay_feature_map_ex", "slay_sketch_params_ex", "slay_linear_attn_fwd",
-           "slay_attn_causal_fwd_state", "slay_causal_state", "slay_state_prefix"]
+           "slay_attn_causal_fwd_state", "slay_causal_state", "slay_state_prefix",
+           "slay_state_suffix", "slay_attn_causal_bwd_state", "slay_causal_bwd_state"]
 
 
 class SlayError(RuntimeError):
@@ -73,6 +74,9 @@ def lib():
     L.slay_causal_state.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
                                     u64, f32, vp, sz, vp]
     L.slay_state_prefix.argtypes = [vp, vp, i32, i32, vp, vp, i32, i32, i32, vp]
+    L.slay_state_suffix.argtypes = L.slay_state_prefix.argtypes
+    L.slay_attn_causal_bwd_state.argtypes = [vp] * 13 + [i32] * 8 + [u64, f32, vp, sz, vp]
+    L.slay_causal_bwd_state.argtypes = [vp] * 6 + [i32] * 8 + [u64, f32, vp, sz, vp]
     L.slay_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                    u64, f32, vp]
     L.slay_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32]
@@ -95,7 +99,8 @@ def lib():
                  "slay_attn_causal_bwd", "slay_decode_step", "slay_prepare",
                  "slay_attn_bidir_bwd", "slay_feature_map_bwd", "slay_feature_map_ex",
                  "slay_sketch_params_ex", "slay_linear_attn_fwd", "slay_attn_causal_fwd_state",
-                 "slay_causal_state", "slay_state_prefix",
+                 "slay_causal_state", "slay_state_prefix", "slay_state_suffix",
+                 "slay_attn_causal_bwd_state", "slay_causal_bwd_state",
                  "slay_attn_causal_fwd_noalloc",
                  "slay_sketch_params"):
         getattr(L, name).restype = i32
@@ -393,6 +398,69 @@ def slay_state_prefix(S_all, z_all, rank, S_in, z_in, stream=None):
     _check(z_in, "z_in", torch.float32, (B, H, F))
     _raise(lib().slay_state_prefix(_ptr(S_all), _ptr(z_all), N, rank, _ptr(S_in), _ptr(z_in),
                                    B * H, F, Dv, _stream(stream)), "slay_state_prefix")
+
+
+def slay_state_suffix(S_all, z_all, rank, S_out, z_out, stream=None):
+    """S_out = sum of S_all[r] for r > rank (S_all [N,B,H,F,64], z_all [N,B,H,F])."""
+    _check(S_all, "S_all", torch.float32)
+    N, B, H, F, Dv = S_all.shape
+    _check(z_all, "z_all", torch.float32, (N, B, H, F))
+    _check(S_out, "S_out", torch.float32, (B, H, F, Dv))
+    _check(z_out, "z_out", torch.float32, (B, H, F))
+    _raise(lib().slay_state_suffix(_ptr(S_all), _ptr(z_all), N, rank, _ptr(S_out), _ptr(z_out),
+                                   B * H, F, Dv, _stream(stream)), "slay_state_suffix")
+
+
+def slay_attn_causal_bwd_state(q, k, v, out, den, dout, dq, dk, dv, R, m, seed, eps, S_in=None,
+                               z_in=None, G_in=None, zg_in=None, workspace=None, stream=None):
+    """Backward of one piece of a causal sequence: S_in, z_in [B,H,F,64], [B,H,F] sum
+    phi(k)[v, 1] over the tokens before it, G_in, zg_in sum phi(q)[dn, delta] over the tokens
+    after it (None: zero); returns the workspace it used."""
+    _check(q, "q")
+    B, H, L, D = q.shape
+    Dv = v.shape[-1]
+    for t, name, dt_, shp in ((k, "k", q.dtype, (B, H, L, D)), (v, "v", q.dtype, (B, H, L, Dv)),
+                              (out, "out", q.dtype, (B, H, L, Dv)),
+                              (den, "den", torch.float32, (B, H, L)),
+                              (dout, "dout", q.dtype, (B, H, L, Dv)),
+                              (dq, "dq", torch.float32, (B, H, L, D)),
+                              (dk, "dk", torch.float32, (B, H, L, D)),
+                              (dv, "dv", torch.float32, (B, H, L, Dv))):
+        _check(t, name, dt_, shp)
+    F = R * m
+    si, zi = _state_ptrs(S_in, z_in, (B, H), F, "state before")
+    gi, zgi = _state_ptrs(G_in, zg_in, (B, H), F, "state after")
+    dt = _dt(q)
+    if workspace is None:
+        workspace = alloc_workspace(OP_CAUSAL_BWD, dt, B, H, L, D, Dv, R, m, q.device)
+    wbytes = workspace.numel() * workspace.element_size()
+    _raise(lib().slay_attn_causal_bwd_state(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(den),
+                                            _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), si, zi, gi,
+                                            zgi, B, H, L, D, Dv, dt, R, m, seed, eps,
+                                            _ptr(workspace), wbytes, _stream(stream)),
+           "slay_attn_causal_bwd_state")
+    return workspace
+
+
+def slay_causal_bwd_state(q, out, den, dout, G_out, zg_out, R, m, seed, eps, workspace=None,
+                          stream=None):
+    """G_out = sum phi(q) dn^T, zg_out = sum phi(q) delta over the tokens of a piece."""
+    _check(q, "q")
+    B, H, L, D = q.shape
+    Dv = out.shape[-1]
+    _check(out, "out", q.dtype, (B, H, L, Dv))
+    _check(den, "den", torch.float32, (B, H, L))
+    _check(dout, "dout", q.dtype, (B, H, L, Dv))
+    F = R * m
+    go, zgo = _state_ptrs(G_out, zg_out, (B, H), F, "state out")
+    dt = _dt(q)
+    if workspace is None:
+        workspace = alloc_workspace(OP_CAUSAL_BWD, dt, B, H, L, D, Dv, R, m, q.device)
+    wbytes = workspace.numel() * workspace.element_size()
+    _raise(lib().slay_causal_bwd_state(_ptr(q), _ptr(out), _ptr(den), _ptr(dout), go, zgo, B, H,
+                                       L, D, Dv, dt, R, m, seed, eps, _ptr(workspace), wbytes,
+                                       _stream(stream)), "slay_causal_bwd_state")
+    return workspace
 
 
 def slay_feature_map_bwd(x, dphi, dx, R, m, seed, eps, stream=None):

@@ -333,7 +333,8 @@ namespace {
 slay_status attn_bwd(const void* q, const void* k, const void* v, const void* out,
                      const float* den, const void* dout, float* dq, float* dk, float* dv, int B,
                      int H, int L, int D, int Dv, slay_dtype dt, int R, int m, uint64_t seed,
-                     float eps, void* workspace, size_t ws_bytes, void* stream, bool causal)
+                     float eps, void* workspace, size_t ws_bytes, void* stream, bool causal,
+                     const BwdStateIO* sio = nullptr)
 {
     slay_status s = check_attn(q, k, v, out, B, H, L, D, Dv, dt, R, m, eps);
     if (s != SLAY_OK) return s;
@@ -352,10 +353,12 @@ slay_status attn_bwd(const void* q, const void* k, const void* v, const void* ou
     cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
     char* w = static_cast<char*>(workspace) + kWsHeader;
     if (e == cudaSuccess)
-        e = causal ? simt_attn_causal_bwd(q, k, v, out, den, dout, dq, dk, dv, B, H, L, dt, P, eps,
-                                          w, st)
-                   : simt_attn_bidir_bwd(q, k, v, out, den, dout, dq, dk, dv, B, H, L, dt, P, eps,
-                                         w, st);
+        e = sio ? simt_attn_causal_bwd_state(q, k, v, out, den, dout, dq, dk, dv, B, H, L, dt, P,
+                                             eps, w, *sio, st)
+            : causal ? simt_attn_causal_bwd(q, k, v, out, den, dout, dq, dk, dv, B, H, L, dt, P, eps,
+                                            w, st)
+                     : simt_attn_bidir_bwd(q, k, v, out, den, dout, dq, dk, dv, B, H, L, dt, P, eps,
+                                           w, st);
     return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
 }
 
@@ -548,8 +551,67 @@ slay_status slay_state_prefix(const float* S_all, const float* z_all, int nranks
     if (BH == 0) return SLAY_OK;
     if (!S_all || !z_all || !S_in || !z_in) return SLAY_ERR_INVALID_ARG;
     const int64_t ns = static_cast<int64_t>(BH) * F * Dv, nz = static_cast<int64_t>(BH) * F;
-    cudaError_t e = simt_state_prefix(S_all, z_all, nranks, rank, ns, nz, S_in, z_in,
+    cudaError_t e = simt_state_prefix(S_all, z_all, 0, rank, ns, nz, S_in, z_in,
                                       static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
+}
+
+slay_status slay_state_suffix(const float* S_all, const float* z_all, int nranks, int rank,
+                              float* S_out, float* z_out, int BH, int F, int Dv, void* stream)
+{
+    if (nranks <= 0 || rank < 0 || rank >= nranks || BH < 0 || F <= 0 || Dv <= 0)
+        return SLAY_ERR_INVALID_ARG;
+    if (Dv != kD || F > kMaxF) return SLAY_ERR_UNSUPPORTED;
+    if (BH == 0) return SLAY_OK;
+    if (!S_all || !z_all || !S_out || !z_out) return SLAY_ERR_INVALID_ARG;
+    const int64_t ns = static_cast<int64_t>(BH) * F * Dv, nz = static_cast<int64_t>(BH) * F;
+    cudaError_t e = simt_state_prefix(S_all, z_all, rank + 1, nranks, ns, nz, S_out, z_out,
+                                      static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
+}
+
+slay_status slay_attn_causal_bwd_state(const void* q, const void* k, const void* v,
+                                       const void* out, const float* den, const void* dout,
+                                       float* dq, float* dk, float* dv, const float* S_in,
+                                       const float* z_in, const float* G_in, const float* zg_in,
+                                       int B, int H, int L, int D, int Dv, slay_dtype dt, int R,
+                                       int m, uint64_t seed, float eps, void* workspace,
+                                       size_t ws_bytes, void* stream)
+{
+    slay_status s = check_state_ptrs(S_in, z_in);
+    if (s != SLAY_OK) return s;
+    if ((s = check_state_ptrs(G_in, zg_in)) != SLAY_OK) return s;
+    const BwdStateIO sio{S_in, z_in, G_in, zg_in};
+    return attn_bwd(q, k, v, out, den, dout, dq, dk, dv, B, H, L, D, Dv, dt, R, m, seed, eps,
+                    workspace, ws_bytes, stream, true, &sio);
+}
+
+slay_status slay_causal_bwd_state(const void* q, const void* out, const float* den,
+                                  const void* dout, float* G_out, float* zg_out, int B, int H,
+                                  int L, int D, int Dv, slay_dtype dt, int R, int m, uint64_t seed,
+                                  float eps, void* workspace, size_t ws_bytes, void* stream)
+{
+    slay_status s = check_attn(q, q, out, out, B, H, L, D, Dv, dt, R, m, eps);
+    if (s != SLAY_OK) return s;
+    if (!G_out || !zg_out) return SLAY_ERR_INVALID_ARG;
+    if ((s = check_state_ptrs(G_out, zg_out)) != SLAY_OK) return s;
+    if (static_cast<int64_t>(B) * H == 0) return SLAY_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (L == 0) {   // an empty piece: its sum is zero
+        cudaError_t e = cudaMemsetAsync(G_out, 0, static_cast<size_t>(B) * H * R * m * Dv * sizeof(float), st);
+        if (e == cudaSuccess)
+            e = cudaMemsetAsync(zg_out, 0, static_cast<size_t>(B) * H * R * m * sizeof(float), st);
+        return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
+    }
+    if (!den || !dout || !aligned(den, 4) || !aligned(dout, 16)) return SLAY_ERR_INVALID_ARG;
+    const size_t need = attn_ws(SLAY_OP_CAUSAL_BWD, dt, B, H, L, Dv, R, m);
+    if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return SLAY_ERR_INVALID_ARG;
+    Params P;
+    if ((s = get_params(D, R, m, seed, eps, &P)) != SLAY_OK) return s;
+    cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
+    if (e == cudaSuccess)
+        e = simt_causal_bwd_state(q, out, den, dout, G_out, zg_out, B, H, L, dt, P, eps,
+                                  static_cast<char*>(workspace) + kWsHeader, st);
     return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
 }
 

@@ -100,8 +100,26 @@ cudaError_t simt_attn_fwd(const void* q, const void* k, const void* v, void* out
 size_t simt_ws_state(int B, int H, int L, int F);
 cudaError_t simt_causal_state(const void* k, const void* v, int B, int H, int L, slay_dtype dt,
                               const Params& P, void* ws, cudaStream_t st, const StateIO& sio);
-cudaError_t simt_state_prefix(const float* s_all, const float* z_all, int nranks, int rank,
+cudaError_t simt_state_prefix(const float* s_all, const float* z_all, int r0, int r1,
                               int64_t ns, int64_t nz, float* s_in, float* z_in, cudaStream_t st);
+// The sums outside a piece of a causal sequence for its backward: s_in, z_in over the tokens
+// before it (phi(k) [v, 1]), g_in, zg_in over the tokens after it (phi(q) [dn, delta]);
+// [B,H,F,64] and [B,H,F] fp32, null = zero.
+struct BwdStateIO {
+    const float* s_in;
+    const float* z_in;
+    const float* g_in;
+    const float* zg_in;
+};
+cudaError_t simt_attn_causal_bwd_state(const void* q, const void* k, const void* v,
+                                       const void* out, const float* den, const void* dout,
+                                       float* dq, float* dk, float* dv, int B, int H, int L,
+                                       slay_dtype dt, const Params& P, float eps, void* ws,
+                                       const BwdStateIO& sio, cudaStream_t st);
+cudaError_t simt_causal_bwd_state(const void* q, const void* out, const float* den,
+                                  const void* dout, float* g_out, float* zg_out, int B, int H,
+                                  int L, slay_dtype dt, const Params& P, float eps, void* ws,
+                                  cudaStream_t st);
 cudaError_t simt_attn_causal_bwd(const void* q, const void* k, const void* v,
                                  const void* out, const float* den, const void* dout,
                                  float* dq, float* dk, float* dv, int B, int H, int L,

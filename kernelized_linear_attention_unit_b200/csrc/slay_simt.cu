@@ -298,12 +298,13 @@ __global__ void k_scan(float* __restrict__ stt, float* __restrict__ tot, int BH,
     if (mode == 2) tot[static_cast<int64_t>(bh) * FE + idx] = run;
 }
 
-// Exclusive forward prefix over chunks of st[bh][c][f][65] starting from a given state
-// (s_in [bh][f][64], z_in [bh][f]; null = zero), with the state after the last chunk written
-// to s_out / z_out (each may be null).  One thread per (bh, f, e).
+// Exclusive prefix over chunks of st[bh][c][f][65] (rev: exclusive suffix, chunks from the
+// last) starting from a given state (s_in [bh][f][64], z_in [bh][f]; null = zero), with the
+// state after the last chunk walked written to s_out / z_out (each may be null).  One
+// thread per (bh, f, e).
 __global__ void k_scan_state(float* __restrict__ stt, int BH, int NC, int F,
                              const float* __restrict__ s_in, const float* __restrict__ z_in,
-                             float* __restrict__ s_out, float* __restrict__ z_out)
+                             float* __restrict__ s_out, float* __restrict__ z_out, int rev)
 {
     const int FE = F * E;
     const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -313,7 +314,8 @@ __global__ void k_scan_state(float* __restrict__ stt, int BH, int NC, int F,
     float run = 0.0f;
     if (s_in) run = e < kD ? s_in[(static_cast<int64_t>(bh) * F + f) * kD + e] : z_in[static_cast<int64_t>(bh) * F + f];
     float* base = stt + static_cast<int64_t>(bh) * NC * FE + idx;
-    for (int c = 0; c < NC; ++c) {
+    for (int cc = 0; cc < NC; ++cc) {
+        const int c = rev ? NC - 1 - cc : cc;
         const float x = base[static_cast<int64_t>(c) * FE];
         base[static_cast<int64_t>(c) * FE] = run;
         run += x;
@@ -1066,7 +1068,7 @@ static cudaError_t attn_fwd_t(const void* q, const void* k, const void* v, void*
         TraceScope trace_("simt_scan", st);
         if (causal && sio)
             k_scan_state<<<static_cast<unsigned>((nth + 255) / 256), 256, 0, st>>>(
-                stt, BH, NC, F, sio->s_in, sio->z_in, sio->s_out, sio->z_out);
+                stt, BH, NC, F, sio->s_in, sio->z_in, sio->s_out, sio->z_out, 0);
         else
             k_scan<<<static_cast<unsigned>((nth + 255) / 256), 256, 0, st>>>(stt, tot, BH, NC, FE, causal ? 0 : 2);
     }
@@ -1104,7 +1106,7 @@ static cudaError_t causal_state_t(const void* k, const void* v, int B, int H, in
     const int64_t nth = static_cast<int64_t>(BH) * F * E;
     TraceScope trace_("simt_scan", st);
     k_scan_state<<<static_cast<unsigned>((nth + 255) / 256), 256, 0, st>>>(stt, BH, NC, F, sio.s_in,
-                                                                           sio.z_in, sio.s_out, sio.z_out);
+                                                                           sio.z_in, sio.s_out, sio.z_out, 0);
     return cudaGetLastError();
 }
 
@@ -1125,28 +1127,30 @@ cudaError_t simt_causal_state(const void* k, const void* v, int B, int H, int L,
 // S_in = sum of the per-rank states of the ranks before `rank` (an exclusive prefix over the
 // all-gathered [nranks][BH][F][64] states and [nranks][BH][F] z), one thread per element
 __global__ void k_state_prefix(const float* __restrict__ s_all, const float* __restrict__ z_all,
-                               int nranks, int rank, int64_t ns, int64_t nz,
+                               int r0, int r1, int64_t ns, int64_t nz,
                                float* __restrict__ s_in, float* __restrict__ z_in)
 {
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < ns;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         float a = 0.0f;
-        for (int r = 0; r < rank && r < nranks; ++r) a += s_all[static_cast<int64_t>(r) * ns + i];
+        for (int r = r0; r < r1; ++r) a += s_all[static_cast<int64_t>(r) * ns + i];
         s_in[i] = a;
         if (i < nz) {
             float b = 0.0f;
-            for (int r = 0; r < rank && r < nranks; ++r) b += z_all[static_cast<int64_t>(r) * nz + i];
+            for (int r = r0; r < r1; ++r) b += z_all[static_cast<int64_t>(r) * nz + i];
             z_in[i] = b;
         }
     }
 }
 
-cudaError_t simt_state_prefix(const float* s_all, const float* z_all, int nranks, int rank,
+// The sum of the gathered states of ranks r0 .. r1 - 1 in rank order (the prefix of a rank
+// is r0 = 0, r1 = rank; its suffix r0 = rank + 1, r1 = nranks).
+cudaError_t simt_state_prefix(const float* s_all, const float* z_all, int r0, int r1,
                               int64_t ns, int64_t nz, float* s_in, float* z_in, cudaStream_t st)
 {
     const int grid = static_cast<int>(std::min<int64_t>((ns + 255) / 256, 1184));
     TraceScope trace_("simt_state_prefix", st);
-    k_state_prefix<<<grid, 256, 0, st>>>(s_all, z_all, nranks, rank, ns, nz, s_in, z_in);
+    k_state_prefix<<<grid, 256, 0, st>>>(s_all, z_all, r0, r1, ns, nz, s_in, z_in);
     return cudaGetLastError();
 }
 
@@ -1250,7 +1254,8 @@ template <typename T>
 static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const void* out,
                               const float* den, const void* dout, float* dq, float* dk,
                               float* dv, int B, int H, int L, const Params& P, float eps,
-                              void* ws, cudaStream_t st, bool bidir)
+                              void* ws, cudaStream_t st, bool bidir,
+                              const BwdStateIO* sio = nullptr)
 {
     const int BH = B * H, F = P.F, NC = nchunks(L);
     const int64_t rows = static_cast<int64_t>(BH) * L;
@@ -1309,9 +1314,28 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
     float* stot = reinterpret_cast<float*>(w + simt_ws_bwd(B, H, L, kD, F));
     float* gtot = stot + align256(static_cast<size_t>(BH) * FE * sizeof(float)) / sizeof(float);
     if (tcb) {   // running sums over the tiles, written as the contraction's bf16 operands
+        BwdSeeds seeds;   // a piece of a longer sequence: the sums outside it seed them
+        if (sio) {
+            seeds.s_in = sio->s_in;
+            seeds.z_in = sio->z_in;
+            seeds.g_in = sio->g_in;
+            seeds.zg_in = sio->zg_in;
+        }
         if ((err = tc_bwd_sums(phq, phk, v, dn16, delta, sfw, gbw, stot, gtot, BH, L, F, bidir,
-                               status, st)) != cudaSuccess)
+                               status, st, &seeds)) != cudaSuccess)
             return err;
+    } else if (sio) {   // causal piece: the chunk scans start from the outside sums
+        {
+            TraceScope trace_("simt_scan", st);
+            k_scan_state<<<sgrid, 256, 0, st>>>(sfw, BH, NS, F, sio->s_in, sio->z_in, nullptr,
+                                                nullptr, 0);
+        }
+        {
+            TraceScope trace_("simt_scan", st);
+            k_scan_state<<<sgrid, 256, 0, st>>>(gbw, BH, NS, F, sio->g_in, sio->zg_in, nullptr,
+                                                nullptr, 1);
+        }
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
     } else {
         {
             TraceScope trace_("simt_scan", st);
@@ -1404,6 +1428,85 @@ cudaError_t simt_attn_bidir_bwd(const void* q, const void* k, const void* v, con
         return attn_bwd_t<float>(q, k, v, out, den, dout, dq, dk, dv, B, H, L, P, eps, ws, st, true);
     return attn_bwd_t<__nv_bfloat16>(q, k, v, out, den, dout, dq, dk, dv, B, H, L, P, eps, ws, st,
                                      true);
+}
+
+cudaError_t simt_attn_causal_bwd_state(const void* q, const void* k, const void* v,
+                                       const void* out, const float* den, const void* dout,
+                                       float* dq, float* dk, float* dv, int B, int H, int L,
+                                       slay_dtype dt, const Params& P, float eps, void* ws,
+                                       const BwdStateIO& sio, cudaStream_t st)
+{
+    if (dt == SLAY_F32)
+        return attn_bwd_t<float>(q, k, v, out, den, dout, dq, dk, dv, B, H, L, P, eps, ws, st, false,
+                                 &sio);
+    return attn_bwd_t<__nv_bfloat16>(q, k, v, out, den, dout, dq, dk, dv, B, H, L, P, eps, ws, st,
+                                     false, &sio);
+}
+
+// The piece's G = sum_i phi(q_i) [dn_i, delta_i] ([B,H,F,64] and [B,H,F] fp32): phi(q), the
+// row statistics, then the G sums -- on tensor cores the running-sum kernel for G alone in
+// its total form, else the chunk sums and a suffix scan whose final value is the total.
+template <typename T>
+static cudaError_t bwd_state_t(const void* q, const void* out, const float* den, const void* dout,
+                               float* g_out, float* zg_out, int B, int H, int L, const Params& P,
+                               float eps, void* ws, cudaStream_t st)
+{
+    const int BH = B * H, F = P.F, NC = nchunks(L);
+    const int64_t rows = static_cast<int64_t>(BH) * L;
+    const size_t phb = align256(rows * F * sizeof(float));
+    const size_t stb = align256(static_cast<size_t>(BH) * NC * F * E * sizeof(float));
+    char* w = static_cast<char*>(ws);
+    T* phq = reinterpret_cast<T*>(w);
+    float* gbw = reinterpret_cast<float*>(w + 4 * phb + stb);
+    float* dn = reinterpret_cast<float*>(w + 4 * phb + 2 * stb);
+    cudaError_t err;
+    if ((err = phi_map<T>(q, phq, rows, P, st)) != cudaSuccess) return err;
+    const bool tcb = std::is_same<T, __nv_bfloat16>::value && tc_bwd_tile_supported(F, L);
+    __nv_bfloat16* dn16 = reinterpret_cast<__nv_bfloat16*>(dn);
+    float* delta = reinterpret_cast<float*>(dn16 + rows * kD);
+    {
+        TraceScope trace_("simt_bwd_rowstats", st);
+        if (tcb)
+            k_bwd_rowstats_tc<<<static_cast<unsigned>((rows + 31) / 32), 256, 0, st>>>(
+                reinterpret_cast<const __nv_bfloat16*>(out), den,
+                reinterpret_cast<const __nv_bfloat16*>(dout), dn16, delta, rows, eps);
+        else
+            k_bwd_rowstats<T><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
+                cp<T>(out), den, cp<T>(dout), dn, rows, eps);
+    }
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (tcb) {
+        BwdSeeds only_g;
+        only_g.sums = 2;
+        only_g.g_out = g_out;
+        only_g.zg_out = zg_out;
+        int* status = reinterpret_cast<int*>(w - kWsHeader);
+        // (the S-side operands are placeholders of the right shapes: no S CTA runs)
+        return tc_bwd_sums(phq, phq, dn16, dn16, delta, nullptr, nullptr, nullptr, nullptr, BH, L,
+                           F, true, status, st, &only_g);
+    }
+    const dim3 sg((F + C - 1) / C, NC, BH);
+    {
+        TraceScope trace_("simt_chunk_state", st);
+        k_chunk_state<float, T><<<sg, NT, 0, st>>>(phq, dn, E, gbw, L, F);
+    }
+    const int64_t nth = static_cast<int64_t>(BH) * F * E;
+    {
+        TraceScope trace_("simt_scan", st);
+        k_scan_state<<<static_cast<unsigned>((nth + 255) / 256), 256, 0, st>>>(
+            gbw, BH, NC, F, nullptr, nullptr, g_out, zg_out, 1);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t simt_causal_bwd_state(const void* q, const void* out, const float* den,
+                                  const void* dout, float* g_out, float* zg_out, int B, int H,
+                                  int L, slay_dtype dt, const Params& P, float eps, void* ws,
+                                  cudaStream_t st)
+{
+    if (dt == SLAY_F32)
+        return bwd_state_t<float>(q, out, den, dout, g_out, zg_out, B, H, L, P, eps, ws, st);
+    return bwd_state_t<__nv_bfloat16>(q, out, den, dout, g_out, zg_out, B, H, L, P, eps, ws, st);
 }
 
 template <typename Tin, typename TG>

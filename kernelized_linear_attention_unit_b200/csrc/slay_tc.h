@@ -39,9 +39,23 @@ bool tc_bwd_tile_supported(int F, int L);
 // tiles walked in order with the running sums on chip, written per tile as the contraction's
 // operand slabs: [64 f][64 e] bf16 and z fp32 per 64 features, 65 x 64 floats apart (bidir:
 // the whole-sequence sums into tot_s, tot_g).
+// Sums over the tokens outside a piece of the sequence (sequence parallelism): s_in, z_in
+// the S sums before it, g_in, zg_in the G sums after it ([BH][F][64], [BH][F] fp32; null =
+// zero); g_out, zg_out: the piece's G total in fp32 (null = not wanted); sums: bit 0 S,
+// bit 1 G (only those CTAs run).
+struct BwdSeeds {
+    const float* s_in = nullptr;
+    const float* z_in = nullptr;
+    const float* g_in = nullptr;
+    const float* zg_in = nullptr;
+    float* g_out = nullptr;
+    float* zg_out = nullptr;
+    int sums = 3;
+};
 cudaError_t tc_bwd_sums(const void* phq, const void* phk, const void* v, const void* dn16,
                         const float* delta, float* st_s, float* st_g, float* tot_s, float* tot_g,
-                        int BH, int L, int F, bool bidir, int* err, cudaStream_t st);
+                        int BH, int L, int F, bool bidir, int* err, cudaStream_t st,
+                        const BwdSeeds* seeds = nullptr);
 // bidir: the bidirectional form (no masked term; sfw, gbw are each sequence's whole sums).
 // sfw, gbw hold tc_bwd_sums' operands.
 cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const void* dn16,

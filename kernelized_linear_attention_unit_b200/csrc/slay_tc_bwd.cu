@@ -89,6 +89,16 @@ struct BwParams {
     int dphi_bf16;   // contraction: store dphi(q), dphi(k) as bf16 (else fp32)
     int bidir;       // contraction: the bidirectional form (no masked intra-tile term; sfw,
                      // gbw hold each sequence's whole sums, not each tile's)
+    // running sums (k_tc_bwd_sums): which sums (bit 0 S, bit 1 G), their starting values --
+    // the sums over the tokens before this piece of the sequence (S) and after it (G),
+    // [BH][F][64] and [BH][F] fp32, or null -- and, for G, an fp32 total out (same layout)
+    int sums;
+    const float* seed_s;
+    const float* seed_z;
+    const float* seed_g;
+    const float* seed_zg;
+    float* out_g;
+    float* out_zg;
 };
 
 __global__ void __launch_bounds__(kBwThreads, 1)
@@ -454,8 +464,10 @@ k_tc_bwd_sums(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nb = bp.F / 128, NS = bp.ntiles, nsl = bp.F / 64;
-    const int g = static_cast<int>(blockIdx.x) & 1;   // 0: S (keys, forward), 1: G (queries, backward)
-    const int job = static_cast<int>(blockIdx.x) >> 1;
+    // 0: S (keys, forward), 1: G (queries, backward); one CTA of each per job unless only
+    // one of the sums is wanted
+    const int g = bp.sums == 3 ? static_cast<int>(blockIdx.x) & 1 : bp.sums >> 1;
+    const int job = bp.sums == 3 ? static_cast<int>(blockIdx.x) >> 1 : static_cast<int>(blockIdx.x);
     const int bh = job / nb, mb = job - bh * nb;
     const bool total = bp.bidir != 0;
     auto tile_of = [&](int i) { return (g && !total) ? NS - 1 - i : i; };
@@ -532,8 +544,14 @@ k_tc_bwd_sums(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
         const uint32_t trow = tmem + ((32u * q) << 16);
         const int f = 128 * mb + static_cast<int>(row);
         float run[33];
+        {   // the sum over the tokens outside this piece of the sequence (zero when none)
+            const float* sd = g ? bp.seed_g : bp.seed_s;
+            const float* zd = g ? bp.seed_zg : bp.seed_z;
+            const int64_t o = (static_cast<int64_t>(bh) * bp.F + f) * 64 + 32 * half;
 #pragma unroll
-        for (int c = 0; c < 33; ++c) run[c] = 0.0f;
+            for (int c = 0; c < 32; ++c) run[c] = sd ? sd[o + c] : 0.0f;
+            run[32] = (zd && half) ? zd[static_cast<int64_t>(bh) * bp.F + f] : 0.0f;
+        }
         // delta of this thread's token in its 16-byte chunk `half` of the extension row (the
         // 16 columns the N = 80 operand reads), for walk step i
         auto write_delta = [&](int i) {
@@ -592,9 +610,15 @@ k_tc_bwd_sums(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
             for (int c = 0; c < 32; ++c) run[c] += __uint_as_float(a[c]);
             run[32] += __uint_as_float(z);
         }
-        if (total) {
+        if (total && (g ? tot_g : tot_s)) {
             const int64_t slab = static_cast<int64_t>(bh) * nsl + (f >> 6);
             store(slab, (g ? tot_g : tot_s) + slab * kSlabF);
+        }
+        if (g && bp.out_g) {   // fp32 total of G (a piece's state for the other ranks)
+            float4* o = reinterpret_cast<float4*>(bp.out_g + (static_cast<int64_t>(bh) * bp.F + f) * 64 + 32 * half);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) o[c] = make_float4(run[4 * c], run[4 * c + 1], run[4 * c + 2], run[4 * c + 3]);
+            if (half) bp.out_zg[static_cast<int64_t>(bh) * bp.F + f] = run[32];
         }
         if (lane == 0) bulk_wait<0>();   // this warp's stores have landed
     }
@@ -685,7 +709,7 @@ cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const v
     if (!map_seq(&mq, phq, F, L, BH) || !map_seq(&mk, phk, F, L, BH) || !map_seq(&mv, v, 64, L, BH) ||
         !map_seq(&mdn, dn16, 64, L, BH))
         return cudaErrorInvalidValue;
-    BwParams bp;
+    BwParams bp{};
     bp.L = L;
     bp.F = F;
     bp.ntiles = (L + kT - 1) / kT;
@@ -711,31 +735,45 @@ cudaError_t tc_bwd_tile(const void* phq, const void* phk, const void* v, const v
 
 cudaError_t tc_bwd_sums(const void* phq, const void* phk, const void* v, const void* dn16,
                         const float* delta, float* st_s, float* st_g, float* tot_s, float* tot_g,
-                        int BH, int L, int F, bool bidir, int* err, cudaStream_t st)
+                        int BH, int L, int F, bool bidir, int* err, cudaStream_t st,
+                        const BwdSeeds* seeds)
 {
     if (!tc_bwd_tile_supported(F, L)) return cudaErrorNotSupported;
     CUtensorMap mq, mk, mv, mdn;
     if (!map_seq(&mq, phq, F, L, BH) || !map_seq(&mk, phk, F, L, BH) || !map_seq(&mv, v, 64, L, BH) ||
         !map_seq(&mdn, dn16, 64, L, BH))
         return cudaErrorInvalidValue;
-    BwParams bp;
+    BwParams bp{};
     bp.L = L;
     bp.F = F;
     bp.ntiles = (L + kT - 1) / kT;
     bp.nitems = BH * bp.ntiles;
     bp.dphi_bf16 = 0;
     bp.bidir = bidir ? 1 : 0;
-    // outputs: every tile's slabs (causal) or every sequence's (bidirectional)
+    bp.sums = 3;
+    if (seeds) {
+        bp.sums = seeds->sums;
+        bp.seed_s = seeds->s_in;
+        bp.seed_z = seeds->z_in;
+        bp.seed_g = seeds->g_in;
+        bp.seed_zg = seeds->zg_in;
+        bp.out_g = seeds->g_out;
+        bp.out_zg = seeds->zg_out;
+    }
+    // outputs: every tile's slabs (causal) or every sequence's (bidirectional); a total-only
+    // call (G state of a piece) writes no slabs and passes the inputs' maps as placeholders
     const int64_t nslabs = static_cast<int64_t>(BH) * (bidir ? 1 : bp.ntiles) * (F / 64);
-    CUtensorMap mso, mgo;
-    if (!map_slabs_out(&mso, bidir ? tot_s : st_s, nslabs) || !map_slabs_out(&mgo, bidir ? tot_g : st_g, nslabs))
+    float* so = bidir ? tot_s : st_s;
+    float* go = bidir ? tot_g : st_g;
+    CUtensorMap mso = mq, mgo = mq;
+    if ((so && !map_slabs_out(&mso, so, nslabs)) || (go && !map_slabs_out(&mgo, go, nslabs)))
         return cudaErrorInvalidValue;
     const size_t smem = su_layout().total + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_tc_bwd_sums, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     TraceScope trace_("tc_bwd_sums", st);
-    k_tc_bwd_sums<<<BH * (F / 128) * 2, kSumThreads, smem, st>>>(mq, mk, mv, mdn, mso, mgo, delta, st_s,
+    k_tc_bwd_sums<<<BH * (F / 128) * (bp.sums == 3 ? 2 : 1), kSumThreads, smem, st>>>(mq, mk, mv, mdn, mso, mgo, delta, st_s,
                                                                  st_g, tot_s, tot_g, bp, err);
     return cudaGetLastError();
 }

@@ -1,4 +1,4 @@
-"""Sequence-parallel causal SLAY forward over the ranks of a process group.
+"""Sequence-parallel causal SLAY forward and backward over the ranks of a process group.
 
 The causal contraction's prefix state carries everything earlier tokens contribute
 (review, "Proposed method", step 6), so a long sequence split into contiguous pieces, one
@@ -6,12 +6,15 @@ per rank in rank order, needs one exchange: each rank sums its own piece's state
 (slay_causal_state: sum of phi(k) [v, 1]^T), the ranks all-gather those states (F x (Dv+1)
 fp32 per (b, h)), each rank adds up the states of the ranks before it (slay_state_prefix)
 and runs its piece's causal forward from that state (slay_attn_causal_fwd_state).  The
-collective is NCCL's all-gather over NVLink on GPUs (any backend works: the states are
-ordinary tensors); no kernel waits on another rank's memory.
+backward also needs, for each piece, the sum of phi(q) [dn, delta]^T over the later ranks'
+tokens: one more all-gather of the pieces' such sums (slay_causal_bwd_state), a suffix over
+ranks (slay_state_suffix), then the piece's backward from both states
+(slay_attn_causal_bwd_state).  The collective is NCCL's all-gather over NVLink on GPUs (any
+backend works: the states are ordinary tensors); no kernel waits on another rank's memory.
 
 Every step of the path runs in the library's kernels; this module orders them and calls the
-collective.  The three steps are passed in as an object with methods state, prefix and
-forward (LibraryOps by default), so the same orchestration runs in tests on CPU ranks.
+collective.  The steps are passed in as an object (LibraryOps by default: state, prefix,
+forward, bwd_state, suffix, backward), so the same orchestration runs in tests on CPU ranks.
 """
 from typing import Optional
 
@@ -22,7 +25,7 @@ from . import binding as bd
 
 
 class LibraryOps:
-    """The three steps through libslay.so (device tensors)."""
+    """The steps through libslay.so (device tensors)."""
 
     def __init__(self, R, m, seed, eps):
         self.R, self.m, self.seed, self.eps = R, m, seed, eps
@@ -36,6 +39,18 @@ class LibraryOps:
     def forward(self, q, k, v, out, den, S_in, z_in):
         bd.slay_attn_causal_fwd_state(q, k, v, out, den, self.R, self.m, self.seed, self.eps,
                                       S_in=S_in, z_in=z_in)
+
+    def bwd_state(self, q, out, den, dout, G_out, zg_out):
+        bd.slay_causal_bwd_state(q, out, den, dout, G_out, zg_out, self.R, self.m, self.seed,
+                                 self.eps)
+
+    def suffix(self, G_all, zg_all, rank, G_in, zg_in):
+        bd.slay_state_suffix(G_all, zg_all, rank, G_in, zg_in)
+
+    def backward(self, q, k, v, out, den, dout, dq, dk, dv, S_in, z_in, G_in, zg_in):
+        bd.slay_attn_causal_bwd_state(q, k, v, out, den, dout, dq, dk, dv, self.R, self.m,
+                                      self.seed, self.eps, S_in=S_in, z_in=z_in, G_in=G_in,
+                                      zg_in=zg_in)
 
 
 def gather_states(S_loc: torch.Tensor, z_loc: torch.Tensor, group=None):
@@ -74,3 +89,35 @@ def causal_fwd_seqpar(q, k, v, out, den, F: int, ops, group=None,
     ops.prefix(S_all, z_all, rank, sc["S_in"], sc["z_in"])
     ops.forward(q, k, v, out, den, sc["S_in"], sc["z_in"])
     return out
+
+
+def causal_bwd_seqpar(q, k, v, out, den, dout, dq, dk, dv, F: int, ops, group=None,
+                      scratch: Optional[dict] = None):
+    """This rank's piece of the backward of a sequence split over the group in rank order:
+    dq, dk, dv of the whole sequence's backward at this piece's rows.  out, den are this
+    piece's rows of the forward (causal_fwd_seqpar), dout its upstream gradient.
+
+    Besides the prefix state of the forward (the sum of phi(k)[v, 1] over the earlier
+    ranks), the backward needs the sum of phi(q)[dn, delta] over the later ranks' tokens:
+    each rank computes its piece's (ops.bwd_state), the ranks all-gather them and each adds
+    up those of the ranks after it (ops.suffix) before its local backward (ops.backward)."""
+    rank = dist.get_rank(group) if dist.is_initialized() else 0
+    B, H = q.shape[0], q.shape[1]
+    Dv = v.shape[-1]
+    sc = scratch if scratch is not None else {}
+    shape_s, shape_z = (B, H, F, Dv), (B, H, F)
+    if sc.get("bwd_shape") != (shape_s, q.device):
+        sc["bwd_shape"] = (shape_s, q.device)
+        for name in ("bS_loc", "bS_in", "bG_loc", "bG_in"):
+            sc[name] = torch.empty(shape_s, dtype=torch.float32, device=q.device)
+        for name in ("bz_loc", "bz_in", "bzg_loc", "bzg_in"):
+            sc[name] = torch.empty(shape_z, dtype=torch.float32, device=q.device)
+    ops.state(k, v, sc["bS_loc"], sc["bz_loc"])
+    S_all, z_all = gather_states(sc["bS_loc"], sc["bz_loc"], group)
+    ops.prefix(S_all, z_all, rank, sc["bS_in"], sc["bz_in"])
+    ops.bwd_state(q, out, den, dout, sc["bG_loc"], sc["bzg_loc"])
+    G_all, zg_all = gather_states(sc["bG_loc"], sc["bzg_loc"], group)
+    ops.suffix(G_all, zg_all, rank, sc["bG_in"], sc["bzg_in"])
+    ops.backward(q, k, v, out, den, dout, dq, dk, dv, sc["bS_in"], sc["bz_in"], sc["bG_in"],
+                 sc["bzg_in"])
+    return dq, dk, dv

@@ -136,6 +136,27 @@ class _OracleOps:
         out.copy_(torch_from(o))
         den.copy_(torch_from(d))
 
+    def bwd_state(self, q, out, den, dout, G_out, zg_out):
+        import oracle as O
+        zeros = np.zeros(q.shape)
+        _, _, _, G, zg = O.attn_causal_bwd_state(q.numpy(), zeros, zeros, out.numpy(), den.numpy(),
+                                                 dout.numpy(), self.P)
+        G_out.copy_(torch_from(G))
+        zg_out.copy_(torch_from(zg))
+
+    def suffix(self, G_all, zg_all, rank, G_in, zg_in):
+        G_in.copy_(G_all[rank + 1:].sum(0) if rank + 1 < G_all.shape[0] else torch_zeros_like(G_in))
+        zg_in.copy_(zg_all[rank + 1:].sum(0) if rank + 1 < zg_all.shape[0] else torch_zeros_like(zg_in))
+
+    def backward(self, q, k, v, out, den, dout, dq, dk, dv, S_in, z_in, G_in, zg_in):
+        import oracle as O
+        st = [x.double().numpy() for x in (S_in, z_in, G_in, zg_in)]
+        a, b, c, _, _ = O.attn_causal_bwd_state(q.numpy(), k.numpy(), v.numpy(), out.numpy(),
+                                                den.numpy(), dout.numpy(), self.P, *st)
+        dq.copy_(torch_from(a))
+        dk.copy_(torch_from(b))
+        dv.copy_(torch_from(c))
+
 
 def torch_from(a):
     import torch
@@ -183,3 +204,51 @@ def test_sequence_parallel_orchestration_two_ranks():
     P = O.sketch_params(w.D, w.R, w.m, w.sketch_seed, float(np.float32(w.eps)))
     want, _ = O.attn_quadratic(q, k, v, P, True)
     assert np.abs(got - want).max() < 1e-5 * np.abs(want).max()
+
+
+def _seqpar_bwd_rank(rank, world, port, outdir):
+    import torch
+    import torch.distributed as dist
+    import oracle as O
+    from kernelized_linear_attention_unit_b200 import seqpar
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        w = W.Workload("spb", B=1, H=2, L=60, R=2, m=8, dtype="f32", data_seed=62)
+        q, k, v = W.gen_qkv(w)
+        g = W.gen_dout(w)
+        P = O.sketch_params(w.D, w.R, w.m, w.sketch_seed, float(np.float32(w.eps)))
+        a, b = rank * w.L // world, (rank + 1) * w.L // world
+        sl = (slice(None), slice(None), slice(a, b))
+        piece = [torch.from_numpy(np.ascontiguousarray(x[sl])).double() for x in (q, k, v, g)]
+        ops = _OracleOps(P)
+        out = torch.empty((1, 2, b - a, 64), dtype=torch.float64)
+        den = torch.empty((1, 2, b - a), dtype=torch.float64)
+        seqpar.causal_fwd_seqpar(piece[0], piece[1], piece[2], out, den, w.F, ops)
+        dq, dk, dv = (torch.empty((1, 2, b - a, 64), dtype=torch.float64) for _ in range(3))
+        seqpar.causal_bwd_seqpar(piece[0], piece[1], piece[2], out, den, piece[3], dq, dk, dv, w.F,
+                                 ops)
+        np.save(os.path.join(outdir, "spb%d.npy" % rank), np.stack([dq.numpy(), dk.numpy(),
+                                                                    dv.numpy()]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sequence_parallel_backward_orchestration_two_ranks():
+    # two gloo ranks each hold half of a sequence: forward as above, then each rank's piece
+    # state and phi(q)[dn, delta] sum all-gathered, prefix and suffix over ranks, and the
+    # piece's backward; together they are the whole sequence's gradients
+    import torch.multiprocessing as mp
+    import oracle as O
+    outdir = tempfile.mkdtemp(prefix="slay_spb_")
+    mp.spawn(_seqpar_bwd_rank, args=(2, _free_port(), outdir), nprocs=2, join=True)
+    got = np.concatenate([np.load(os.path.join(outdir, "spb%d.npy" % r)) for r in range(2)], axis=3)
+    w = W.Workload("spb", B=1, H=2, L=60, R=2, m=8, dtype="f32", data_seed=62)
+    q, k, v = W.gen_qkv(w)
+    g = W.gen_dout(w)
+    P = O.sketch_params(w.D, w.R, w.m, w.sketch_seed, float(np.float32(w.eps)))
+    want = O.attn_causal_bwd(q, k, v, g, P)
+    for i in range(3):
+        assert np.abs(got[i] - want[i]).max() < 1e-4 * np.abs(want[i]).max(), i

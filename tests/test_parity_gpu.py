@@ -705,3 +705,73 @@ def test_sequence_pieces_emulating_ranks(dt, R, m, L, cuts):
     check(name + " final z", host(z_fin), wz, TOL[dt])
     check(name + " piece-0 S", host(Ss[0]), O.attn_causal_state(
         q[:, :, :cuts[0]], k[:, :, :cuts[0]], v[:, :, :cuts[0]], P)[2], TOL[dt])
+
+
+@pytest.mark.parametrize("dt,R,m,L,cuts", [("bf16", 4, 64, 1000, (300, 700)),
+                                           ("bf16", 8, 64, 700, (128, 512)),
+                                           ("f32", 2, 16, 300, (1, 150)),
+                                           ("bf16", 2, 16, 257, (64, 65))])
+def test_sequence_pieces_backward_emulating_ranks(dt, R, m, L, cuts):
+    # the sequence-parallel backward on one GPU: every piece's forward state (prefix over
+    # the pieces before it) and its sum of phi(q)[dn, delta] (suffix over the pieces after
+    # it), then each piece's backward from both; the pieces' gradients against the oracle's
+    # whole-sequence backward, and a piece's phi(q)[dn, delta] sum against the oracle's
+    w = small(dt, R, m, L, B=1, H=3, seed=26)
+    q, k, v = W.gen_qkv(w)
+    g = W.gen_dout(w)
+    P = params(w)
+    F, eps = w.F, _eps(w)
+    qt, kt, vt, gt = dev(q, dt), dev(k, dt), dev(v, dt), dev(g, dt)
+    out = torch.empty((1, 3, L, 64), device="cuda", dtype=TDT[dt])
+    den = torch.empty((1, 3, L), device="cuda")
+    bd.slay_attn_causal_fwd(qt, kt, vt, out, den, R, m, w.sketch_seed, eps)
+    bounds = (0,) + tuple(cuts) + (L,)
+    pieces = [(a, b) for a, b in zip(bounds[:-1], bounds[1:])]
+
+    def piece(t, a, b):
+        return t[:, :, a:b].contiguous()
+
+    def state_pair():
+        return torch.empty((1, 3, F, 64), device="cuda"), torch.empty((1, 3, F), device="cuda")
+
+    Ss, zs, Gs, zgs = [], [], [], []
+    for a, b in pieces:
+        S, z = state_pair()
+        bd.slay_kernel_status(bd.slay_causal_state(piece(kt, a, b), piece(vt, a, b), S, z, R, m,
+                                                    w.sketch_seed, eps))
+        G, zg = state_pair()
+        bd.slay_kernel_status(bd.slay_causal_bwd_state(piece(qt, a, b), piece(out, a, b),
+                                                       piece(den, a, b), piece(gt, a, b), G, zg,
+                                                       R, m, w.sketch_seed, eps))
+        Ss.append(S)
+        zs.append(z)
+        Gs.append(G)
+        zgs.append(zg)
+    S_all, z_all, G_all, zg_all = (torch.stack(x) for x in (Ss, zs, Gs, zgs))
+    grads = []
+    for r, (a, b) in enumerate(pieces):
+        S_in, z_in = state_pair()
+        G_in, zg_in = state_pair()
+        bd.slay_state_prefix(S_all, z_all, r, S_in, z_in)
+        bd.slay_state_suffix(G_all, zg_all, r, G_in, zg_in)
+        n = b - a
+        dq = torch.empty((1, 3, n, 64), device="cuda")
+        dk = torch.empty_like(dq)
+        dv = torch.empty_like(dq)
+        ws = bd.slay_attn_causal_bwd_state(piece(qt, a, b), piece(kt, a, b), piece(vt, a, b),
+                                           piece(out, a, b), piece(den, a, b), piece(gt, a, b),
+                                           dq, dk, dv, R, m, w.sketch_seed, eps, S_in=S_in,
+                                           z_in=z_in, G_in=G_in, zg_in=zg_in)
+        bd.slay_kernel_status(ws)
+        grads.append((host(dq), host(dk), host(dv)))
+    torch.cuda.synchronize()
+    name = "bwd pieces %s R%d m%d L%d %s" % (dt, R, m, L, cuts)
+    got = tuple(np.concatenate([x[i] for x in grads], axis=2) for i in range(3))
+    _check_bwd(name, got, _bwd_reference(q, k, v, g, P, dt), TOL[dt])
+    # the first piece's sum of phi(q)[dn, delta] at the library's forward output
+    a, b = pieces[0]
+    ow, dw = host(out)[:, :, a:b], host(den)[:, :, a:b]
+    _, _, _, wG, wzg = O.attn_causal_bwd_state(q[:, :, a:b], k[:, :, a:b], v[:, :, a:b], ow, dw,
+                                                W.to_dtype(g, dt)[:, :, a:b], P)
+    check(name + " piece-0 G", host(Gs[0]), wG, TOL[dt])
+    check(name + " piece-0 zg", host(zgs[0]), wzg, TOL[dt])
