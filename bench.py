@@ -3,10 +3,13 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload causal_16k|causal_2k|bidir_vision|fwd_8k|bwd_8k|bidir_bwd|decode|
-                                feature_map|feature_map_bwd|matched_budget|seqpar_16k]
+                                feature_map|feature_map_bwd|matched_budget|seqpar_16k|
+                                seqpar_bwd_8k]
 
 seqpar_16k splits the headline sequence over the N ranks (strong scaling, one all-gather of
-the pieces' states per step); every other workload gives each rank its own batch (weak).
+the pieces' states per step), seqpar_bwd_8k the fwd/bwd sequence for its backward (two
+all-gathers: the states before and after each piece); every other workload gives each rank
+its own batch (weak).
 
 With --gpus N > 1 outside torchrun, bench.py starts the N ranks itself (torch.distributed.run
 on 127.0.0.1); under torchrun, --gpus must equal WORLD_SIZE.
@@ -49,6 +52,7 @@ WORKLOADS = {
     "feature_map_bwd": (W.CAUSAL_16K, "feature_map_bwd"),
     "matched_budget": (W.CAUSAL_16K, "matched_budget"),
     "seqpar_16k": (W.CAUSAL_16K, "seqpar"),
+    "seqpar_bwd_8k": (W.FWDBWD_8K, "seqpar_bwd"),
     "decode": (W.DECODE, "decode"),
     "feature_map": (W.CAUSAL_16K, "feature_map"),
 }
@@ -261,7 +265,7 @@ def oracle_sample(w, op, max_heads):
     q, k, v = W.gen_qkv(w, B=1, H=h)
     form = "O(L) fp64 form"
     tokens = h / w.H * w.L          # token-equivalents (a token carries H heads)
-    if op == "bwd":
+    if op in ("bwd", "seqpar_bwd"):
         # the causal backward has no O(L) oracle form: its per-row form on a seeded sample of
         # 32 rows of each head (each row sums over all later queries and earlier keys)
         g = W.gen_dout(w, B=1, H=h)
@@ -332,7 +336,8 @@ def run_reference(args, w, op):
 
 OP_NAMES = {"causal": "causal fwd", "bidir": "bidirectional fwd", "bwd": "causal bwd",
             "bidir_bwd": "bidirectional bwd", "decode": "decode", "feature_map": "feature map",
-            "feature_map_bwd": "feature-map bwd", "seqpar": "sequence-parallel causal fwd"}
+            "feature_map_bwd": "feature-map bwd", "seqpar": "sequence-parallel causal fwd",
+            "seqpar_bwd": "sequence-parallel causal bwd"}
 
 
 def metric_of(w, op, unit):
@@ -403,7 +408,7 @@ def run_ours(args, w, op):
 
     # inputs: each rank draws its own batch (data seed offset by rank); the sequence-parallel
     # workload shares one sequence
-    wr = w if op == "seqpar" else rank_workload(w, rank)
+    wr = w if op in ("seqpar", "seqpar_bwd") else rank_workload(w, rank)
     if op == "decode":
         qn, kn, vn, Sn, zn = W.gen_decode(wr)
         q, k, v = to_dev(qn), to_dev(kn), to_dev(vn)
@@ -442,6 +447,28 @@ def run_ours(args, w, op):
 
         def step():
             seqpar.causal_fwd_seqpar(q, k, v, out, den, w.F, ops, scratch=scratch)
+        units_per_step = w.B * (b - a)
+        unit = "tokens/s"
+    elif op == "seqpar_bwd":
+        from kernelized_linear_attention_unit_b200 import seqpar
+        # this rank's piece of one long sequence: its forward (once, untimed) gives out and
+        # den; the timed step is the piece's backward with its two state exchanges
+        qn, kn, vn = W.gen_qkv(w)
+        gn = W.gen_dout(w)
+        a, b = rank * w.L // world, (rank + 1) * w.L // world
+        q, k, v, g = (to_dev(np.ascontiguousarray(x[:, :, a:b])) for x in (qn, kn, vn, gn))
+        out = torch.empty(v.shape, device=dev, dtype=tdt)
+        den = torch.empty(v.shape[:-1], device=dev, dtype=torch.float32)
+        ops = seqpar.LibraryOps(w.R, w.m, w.sketch_seed, eps)
+        scratch = {}
+        seqpar.causal_fwd_seqpar(q, k, v, out, den, w.F, ops, scratch=scratch)
+        dq = torch.empty(q.shape, device=dev, dtype=torch.float32)
+        dk = torch.empty_like(dq)
+        dv = torch.empty(v.shape, device=dev, dtype=torch.float32)
+        host_in, dev_in = [pinned(x.cpu()) for x in (q, k, v, g)], [q, k, v, g]
+
+        def step():
+            seqpar.causal_bwd_seqpar(q, k, v, out, den, g, dq, dk, dv, w.F, ops, scratch=scratch)
         units_per_step = w.B * (b - a)
         unit = "tokens/s"
     elif op == "feature_map_bwd":
@@ -488,7 +515,7 @@ def run_ours(args, w, op):
                 fn(q, k, v, out, den, w.R, w.m, w.sketch_seed, eps, ws)
         units_per_step = w.B * w.L
         unit = "tokens/s"
-    result = dq if op in ("bwd", "bidir_bwd") else out
+    result = dq if op in ("bwd", "bidir_bwd", "seqpar_bwd") else out
     host_out = torch.empty(result.shape, dtype=result.dtype, pin_memory=True)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     bd.slay_prepare(w.D, w.R, w.m, w.sketch_seed, eps)
@@ -589,10 +616,12 @@ def run_ours(args, w, op):
     # Dv = 64, C = 64): causal 16 D F + 10 F Dv + (C+1)(3F + 2Dv); bidirectional
     # 16 D F + 10 F Dv (no masked term)
     step_roofline = None
-    if op in ("bwd", "bidir_bwd"):
+    if op in ("bwd", "bidir_bwd", "seqpar_bwd"):
         D_, Dv_, F_ = w.D, w.Dv, w.F
-        per = 16 * D_ * F_ + 10 * F_ * Dv_ + ((C_CHUNK + 1) * (3 * F_ + 2 * Dv_) if op == "bwd" else 0)
-        flop = per * w.B * w.H * w.L
+        per = 16 * D_ * F_ + 10 * F_ * Dv_ + ((C_CHUNK + 1) * (3 * F_ + 2 * Dv_) if op != "bidir_bwd" else 0)
+        # (the sequence-parallel backward: this rank's tokens)
+        toks = units_per_step if op == "seqpar_bwd" else w.B * w.L
+        flop = per * w.H * toks
         tflops = flop / (total_ms / args.steps / 1e3) / 1e12
         step_roofline = {"bound": "tensor", "algorithmic_flop_per_step": flop,
                          "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
@@ -610,7 +639,7 @@ def run_ours(args, w, op):
                 "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-                "scaling": "strong" if op == "seqpar" else "weak", "vs_baseline": None,
+                "scaling": "strong" if op in ("seqpar", "seqpar_bwd") else "weak", "vs_baseline": None,
                 "dtype": w.dtype, "data": "synthetic",
                 "config": config_of(w, op),
                 "e2e": {"value": e2e, "unit": unit, "h2d_bytes_per_step": h2d,
