@@ -47,7 +47,9 @@ constexpr int kEpiWarps = 8;
 constexpr int kPbThreads = 32 * (2 + kEpiWarps);   // MMA warp, 8 epilogue warps, TMA warp
 constexpr int kNumSMs = 148;
 constexpr int kXBufs = 3;                   // X tiles in flight
-constexpr int kRing = 3;                    // W groups and dphi tiles in flight (slot = job % 3)
+constexpr int kRing = 3;                    // W groups in flight (slot = job % 3)
+constexpr int kDRing = 2;                   // dphi tiles in flight (slot = job % 2)
+constexpr int kStgBytes = 32 * 128;         // per epilogue warp: [32 rows][32 fp32] of dx
 constexpr uint32_t kColU = 0;               // two 128-column projection buffers
 constexpr uint32_t kColDX = 256;            // two 64-column dX^ accumulators
 
@@ -57,8 +59,8 @@ enum {
     PB_WF = PB_XE + kXBufs,     // + slot (TMA: W group)
     PB_WE = PB_WF + kRing,      // + slot (contraction MMA commit: the group's W free)
     PB_GF = PB_WE + kRing,      // + slot (TMA: dphi tile)
-    PB_GE = PB_GF + kRing,      // + slot (8 warp arrivals: dphi read)
-    PB_UF = PB_GE + kRing,      // + buffer (projection MMA commit)
+    PB_GE = PB_GF + kDRing,     // + slot (8 warp arrivals: dphi read)
+    PB_UF = PB_GE + kDRing,     // + buffer (projection MMA commit)
     PB_AF = PB_UF + 2,          // + buffer (8 warp arrivals: [alpha | beta] written)
     PB_AE = PB_AF + 2,          // + buffer (contraction MMA commit: operand free)
     PB_DF = PB_AE + 2,          // + buffer (dX^ of a tile complete)
@@ -67,7 +69,7 @@ enum {
 };
 
 struct PbLayout {
-    uint32_t w, x, a, d, bar, tmem, total;
+    uint32_t w, x, a, d, stg, bar, tmem, total;
 };
 
 __host__ __device__ inline PbLayout pb_layout(int /*F*/)
@@ -76,8 +78,9 @@ __host__ __device__ inline PbLayout pb_layout(int /*F*/)
     l.w = 0;                                // kRing W groups (16 KiB each)
     l.x = l.w + kRing * kGroupBytes;        // kXBufs X tiles
     l.a = l.x + kXBufs * kBoxBytes;         // 2 [alpha | beta] operands
-    l.d = l.a + 2 * kABytes;                // kRing dphi tiles [128 rows][64 features]
-    l.bar = l.d + kRing * kBoxBytes;
+    l.d = l.a + 2 * kABytes;                // kDRing dphi tiles [128 rows][64 features]
+    l.stg = l.d + kDRing * kBoxBytes;       // kEpiWarps dx staging boxes (TMA stores)
+    l.bar = l.stg + kEpiWarps * kStgBytes;
     l.tmem = l.bar + PB_NUM * 8;
     l.total = l.tmem + 16;
     return l;
@@ -115,8 +118,8 @@ struct Ring {
 
 __global__ void __launch_bounds__(kPbThreads, 1)
 k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
-             const __grid_constant__ CUtensorMap tmd, float* __restrict__ dx, int64_t n_rows,
-             PbParams pp, int* status)
+             const __grid_constant__ CUtensorMap tmd, const __grid_constant__ CUtensorMap tmdx,
+             int64_t n_rows, PbParams pp, int* status)
 {
     constexpr int kW = 4;     // 16-byte words per 32 bf16 dphi values
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -135,7 +138,7 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
     if (tid == 0) {
         for (int i = 0; i < PB_NUM; ++i) mbar_init(&bar[i], 1);
         for (int s = 0; s < kXBufs; ++s) mbar_init(&bar[PB_XE + s], kEpiWarps);
-        for (int s = 0; s < kRing; ++s) mbar_init(&bar[PB_GE + s], kEpiWarps);
+        for (int s = 0; s < kDRing; ++s) mbar_init(&bar[PB_GE + s], kEpiWarps);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bar[PB_AF + b], kEpiWarps);
             mbar_init(&bar[PB_DE + b], kEpiWarps);
@@ -163,7 +166,7 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
         // job order: the X tile at each tile's first group, then per job its W group and its
         // dphi tile, each into a slot freed by the job kRing (X: kXBufs tiles) before
         if (lane == 0) {
-            Ring xr(kXBufs), rr(kRing);
+            Ring xr(kXBufs), rr(kRing), gr(kDRing);
             for (int j = 0, k = 0, g = 0; j < njobs && wt.ok; ++j) {
                 if (g == 0) {
                     if (xr.use >= 1) {
@@ -182,13 +185,14 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
                 unsigned char* wd = sm + L.w + rr.slot * kGroupBytes;
                 tma_load_2d(wd, &tmw, &bar[PB_WF + rr.slot], 0, (2 * g) * 64);
                 tma_load_2d(wd + kSubBytes, &tmw, &bar[PB_WF + rr.slot], 0, (2 * g + 1) * 64);
-                if (rr.use >= 1) {
-                    uint32_t ph = static_cast<uint32_t>((rr.use - 1) & 1);
-                    wt.wait(&bar[PB_GE + rr.slot], ph);
-                }
-                mbar_arrive_expect_tx(&bar[PB_GF + rr.slot], kBoxBytes);
-                tma_load_2d(sm + L.d + rr.slot * kBoxBytes, &tmd, &bar[PB_GF + rr.slot], 64 * g, row0_of(k));
                 rr.next();
+                if (gr.use >= 1) {
+                    uint32_t ph = static_cast<uint32_t>((gr.use - 1) & 1);
+                    wt.wait(&bar[PB_GE + gr.slot], ph);
+                }
+                mbar_arrive_expect_tx(&bar[PB_GF + gr.slot], kBoxBytes);
+                tma_load_2d(sm + L.d + gr.slot * kBoxBytes, &tmd, &bar[PB_GF + gr.slot], 64 * g, row0_of(k));
+                gr.next();
                 if (++g == ng) {
                     g = 0;
                     ++k;
@@ -311,31 +315,40 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
             // below the 1e-12 norm guard x^ = x / 1e-12 is not a unit vector and its
             // derivative is the identity / 1e-12: no tangential projection there
             const float xd = nrm > 1e-12f ? ((dot[0] + dot[1]) + (dot[2] + dot[3])) * inv : 0.0f;
-            const int64_t r = static_cast<int64_t>(k * static_cast<int>(gridDim.x) +
-                                                   static_cast<int>(blockIdx.x)) * kRows + row;
-            if (r < n_rows) {
-                float4* dst = reinterpret_cast<float4*>(dx + r * 64 + 32 * half);
+            // this warp's 32 rows x 32 columns through its staging box (128-byte swizzle:
+            // 16-byte chunk c of row r at c ^ (r & 7)) and a TMA store; rows past n_rows are
+            // clipped by the tensor map
+            const uint32_t box = sbase + L.stg + ew * kStgBytes;
+            if (lane == 0) bulk_wait_read<0>();   // the previous tile's store has read it
+            __syncwarp();
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {   // this warp's 32 columns: chunks 4 half .. + 3
-                    const uint4 w4 = xr[(4 * half + c) ^ (row & 7)];
-                    const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
-                    float o[8];
+            for (int c = 0; c < 4; ++c) {   // this warp's 32 columns: chunks 4 half .. + 3
+                const uint4 w4 = xr[(4 * half + c) ^ (row & 7)];
+                const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
+                float o[8];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i = 8 * c + 2 * e;   // column within the half
-                        // selects, not an indexed pointer (local memory)
-                        const float dlo = half ? __uint_as_float(d1[i]) : __uint_as_float(d0[i]);
-                        const float dhi = half ? __uint_as_float(d1[i + 1]) : __uint_as_float(d0[i + 1]);
-                        o[2 * e] = (dlo - __uint_as_float(ws[e] << 16) * inv * xd) * inv;
-                        o[2 * e + 1] = (dhi - __uint_as_float(ws[e] & 0xFFFF0000u) * inv * xd) * inv;
-                    }
-                    dst[2 * c] = make_float4(o[0], o[1], o[2], o[3]);
-                    dst[2 * c + 1] = make_float4(o[4], o[5], o[6], o[7]);
+                for (int e = 0; e < 4; ++e) {
+                    const int i = 8 * c + 2 * e;   // column within the half
+                    // selects, not an indexed pointer (local memory)
+                    const float dlo = half ? __uint_as_float(d1[i]) : __uint_as_float(d0[i]);
+                    const float dhi = half ? __uint_as_float(d1[i + 1]) : __uint_as_float(d0[i + 1]);
+                    o[2 * e] = (dlo - __uint_as_float(ws[e] << 16) * inv * xd) * inv;
+                    o[2 * e + 1] = (dhi - __uint_as_float(ws[e] & 0xFFFF0000u) * inv * xd) * inv;
                 }
+                st_shared_v4(box + sw128_off(lane, 2 * c), __float_as_uint(o[0]), __float_as_uint(o[1]),
+                             __float_as_uint(o[2]), __float_as_uint(o[3]));
+                st_shared_v4(box + sw128_off(lane, 2 * c + 1), __float_as_uint(o[4]), __float_as_uint(o[5]),
+                             __float_as_uint(o[6]), __float_as_uint(o[7]));
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_2d(&tmdx, sm + L.stg + ew * kStgBytes, 32 * half, row0_of(k) + 32 * q);
+                bulk_commit_group();
             }
             warp_arrive(&bar[PB_XE + s]);   // this warp is done with X slot s
         };
-        Ring xring(kXBufs), dr(kRing);
+        Ring xring(kXBufs), dr(kDRing);
         int ps = 0;                     // X slot of the tile whose dx is pending
         float pinv = 1.0f, pnrm = 1.0f;
         for (int k = 0; k < nt; ++k) {
@@ -386,7 +399,10 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
                     const float2 d = make_float2(dphi_val(dp, c), dphi_val(dp, c + 1));
                     const float2 p = make_float2(__uint_as_float(pr[c]), __uint_as_float(pr[c + 1]));
                     const float2 y = ffma2(a2, make_float2(__uint_as_float(ur[c]), __uint_as_float(ur[c + 1])), b2);
-                    const float2 t = fmul2(fmul2(d, make_float2(ex2(y.x), ex2(y.y))), p);
+                    // a quarter of the exp2 (every other pair's second) on the FMA pipe: the
+                    // special-function unit is the busiest pipe of this loop
+                    const float2 e = make_float2(ex2(y.x), (c & 2) ? ex2_poly(y.y) : ex2(y.y));
+                    const float2 t = fmul2(fmul2(d, e), p);
                     const float2 af = fmul2(fmul2(t, p), sq2);
                     const float2 bf = fmul2(t, tn2);
                     al[c >> 1] = pack_bf16(af.x, af.y);
@@ -417,12 +433,28 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
             xring.next();
         }
         if (nt > 0) dx_tile(nt - 1, ps, pinv, pnrm);
+        if (lane == 0) bulk_wait<0>();   // this warp's dx stores have landed
     }
     wt.report(status);
     drain_after_failure(wt.ok);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem0, 512);
+}
+
+// dx [n][64] fp32 for the TMA stores: boxes of 32 columns (128 bytes) x 32 rows, 128-byte
+// swizzle; rows past n are not written.
+bool map_dx(CUtensorMap* m, float* dx, int64_t n)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(n)};
+    const cuuint64_t strides[1] = {64 * 4};
+    const cuuint32_t box[2] = {32, 32};
+    const cuuint32_t es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, dx, dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -439,8 +471,9 @@ cudaError_t tc_phi_bwd(const void* x, const void* dphi, float* dx, int64_t n, co
 {
     const int F = P.F;
     if (!P.wB || !tc_phi_bwd_supported(64, P.R, P.m, n)) return cudaErrorNotSupported;
-    CUtensorMap mx, mw, md;
-    if (!map_2d(&mx, x, 64, static_cast<uint64_t>(n), 64, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+    CUtensorMap mx, mw, md, mdx;
+    if (!map_dx(&mdx, dx, n) ||
+        !map_2d(&mx, x, 64, static_cast<uint64_t>(n), 64, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map_2d(&mw, P.wB, 64, static_cast<uint64_t>(F / 32) * 64, 64, 64,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map_2d(&md, dphi, F, static_cast<uint64_t>(n), 64, kRows, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -464,7 +497,7 @@ cudaError_t tc_phi_bwd(const void* x, const void* dphi, float* dx, int64_t n, co
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     TraceScope trace_("tc_phi_bwd", st);
-    k_tc_phi_bwd<<<grid, kPbThreads, smem, st>>>(mx, mw, md, dx, n, pp, status);
+    k_tc_phi_bwd<<<grid, kPbThreads, smem, st>>>(mx, mw, md, mdx, n, pp, status);
     return cudaGetLastError();
 }
 
