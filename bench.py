@@ -80,17 +80,18 @@ def alu_peak_tflops(sm_mhz):
     return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
 
 
-def profiled_traffic(kernel):
-    """DRAM bytes per launch of `kernel` from the committed ncu summaries under profiles/
-    (lines "traffic: <kernel> <bytes> <sha256[:16] of its sources> <sources>"), or None
-    when no capture exists or the kernel's sources changed since it was taken."""
+def profiled_traffic(kernel, workload):
+    """DRAM bytes per launch of `kernel` in `workload` from the committed ncu summaries under
+    profiles/ (lines "traffic: <kernel> <bytes> <sha256[:16] of its sources> <sources>
+    <workload>"), or None when no capture of that kernel in that workload exists or the
+    kernel's sources changed since it was taken."""
     import glob
     import hashlib
     csrc = os.path.join(ROOT, "kernelized_linear_attention_unit_b200", "csrc")
     for fn in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
         for line in open(fn):
             parts = line.split()
-            if len(parts) != 5 or parts[0] != "traffic:" or parts[1] != kernel:
+            if len(parts) != 6 or parts[0] != "traffic:" or parts[1] != kernel or parts[5] != workload:
                 continue
             h = hashlib.sha256()
             try:
@@ -603,7 +604,8 @@ def run_ours(args, w, op):
                 peak = alu_peak_tflops(peaks.get("sm_max_mhz", 1965.0))
                 u = "TFLOP/s"
             roofline = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak,
-                        "unit": u, "frac": achieved / peak, "traffic": profiled_traffic(dom),
+                        "unit": u, "frac": achieved / peak,
+                        "traffic": profiled_traffic(dom, config_of(w, op)["workload"]),
                         "peak_source": peak_src + (" (fp32 FFMA: 148 SMs x 128 x 2 x max clock)"
                                                    if bound == "alu" else ""),
                         "algorithmic_%s_per_launch" % kind: amount,

@@ -81,3 +81,23 @@ def test_backward_step_flops_are_the_per_token_head_count():
     per = 16 * D * w.F + 10 * w.F * DV + 65 * (3 * w.F + 2 * DV)
     assert per == 960128
     assert abs(per * w.B * w.H * w.L - 2.517e11) < 1e9
+
+
+def test_profiled_traffic_needs_the_same_workload_and_sources(tmp_path, monkeypatch):
+    # a committed ncu figure is reported only for the workload it was captured on and only
+    # while the kernel's sources hash as they did then
+    import hashlib
+    csrc = tmp_path / "kernelized_linear_attention_unit_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "a.cu").write_bytes(b"kernel source one")
+    (tmp_path / "profiles").mkdir()
+    h = hashlib.sha256(b"kernel source one").hexdigest()[:16]
+    (tmp_path / "profiles" / "k.md").write_text(
+        "text\ntraffic: tc_x 1234 %s a.cu wl_big\ntraffic: tc_x 99 %s a.cu wl_small\n" % (h, h))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profiled_traffic("tc_x", "wl_big") == 1234
+    assert bench.profiled_traffic("tc_x", "wl_small") == 99
+    assert bench.profiled_traffic("tc_x", "wl_other") is None
+    assert bench.profiled_traffic("tc_y", "wl_big") is None
+    (csrc / "a.cu").write_bytes(b"kernel source two")
+    assert bench.profiled_traffic("tc_x", "wl_big") is None
