@@ -468,8 +468,13 @@ def run_ours(args, w, op):
         dv = torch.empty(v.shape, device=dev, dtype=torch.float32)
         host_in, dev_in = [pinned(x.cpu()) for x in (q, k, v, g)], [q, k, v, g]
 
+        # the state this piece's forward started from is the forward's (a training step
+        # has it); the backward adds the exchange of the later pieces' phi(q)[dn, delta] sums
+        fwd_state = (scratch["S_in"], scratch["z_in"])
+
         def step():
-            seqpar.causal_bwd_seqpar(q, k, v, out, den, g, dq, dk, dv, w.F, ops, scratch=scratch)
+            seqpar.causal_bwd_seqpar(q, k, v, out, den, g, dq, dk, dv, w.F, ops, scratch=scratch,
+                                     fwd_state=fwd_state)
         units_per_step = w.B * (b - a)
         unit = "tokens/s"
     elif op == "feature_map_bwd":

@@ -92,7 +92,7 @@ def causal_fwd_seqpar(q, k, v, out, den, F: int, ops, group=None,
 
 
 def causal_bwd_seqpar(q, k, v, out, den, dout, dq, dk, dv, F: int, ops, group=None,
-                      scratch: Optional[dict] = None):
+                      scratch: Optional[dict] = None, fwd_state=None):
     """This rank's piece of the backward of a sequence split over the group in rank order:
     dq, dk, dv of the whole sequence's backward at this piece's rows.  out, den are this
     piece's rows of the forward (causal_fwd_seqpar), dout its upstream gradient.
@@ -100,7 +100,9 @@ def causal_bwd_seqpar(q, k, v, out, den, dout, dq, dk, dv, F: int, ops, group=No
     Besides the prefix state of the forward (the sum of phi(k)[v, 1] over the earlier
     ranks), the backward needs the sum of phi(q)[dn, delta] over the later ranks' tokens:
     each rank computes its piece's (ops.bwd_state), the ranks all-gather them and each adds
-    up those of the ranks after it (ops.suffix) before its local backward (ops.backward)."""
+    up those of the ranks after it (ops.suffix) before its local backward (ops.backward).
+    fwd_state: the (S_in, z_in) this rank's forward started from (the scratch of
+    causal_fwd_seqpar on the same q, k, v), which saves recomputing it."""
     rank = dist.get_rank(group) if dist.is_initialized() else 0
     B, H = q.shape[0], q.shape[1]
     Dv = v.shape[-1]
@@ -112,12 +114,15 @@ def causal_bwd_seqpar(q, k, v, out, den, dout, dq, dk, dv, F: int, ops, group=No
             sc[name] = torch.empty(shape_s, dtype=torch.float32, device=q.device)
         for name in ("bz_loc", "bz_in", "bzg_loc", "bzg_in"):
             sc[name] = torch.empty(shape_z, dtype=torch.float32, device=q.device)
-    ops.state(k, v, sc["bS_loc"], sc["bz_loc"])
-    S_all, z_all = gather_states(sc["bS_loc"], sc["bz_loc"], group)
-    ops.prefix(S_all, z_all, rank, sc["bS_in"], sc["bz_in"])
+    if fwd_state is None:
+        ops.state(k, v, sc["bS_loc"], sc["bz_loc"])
+        S_all, z_all = gather_states(sc["bS_loc"], sc["bz_loc"], group)
+        ops.prefix(S_all, z_all, rank, sc["bS_in"], sc["bz_in"])
+        S_in, z_in = sc["bS_in"], sc["bz_in"]
+    else:
+        S_in, z_in = fwd_state
     ops.bwd_state(q, out, den, dout, sc["bG_loc"], sc["bzg_loc"])
     G_all, zg_all = gather_states(sc["bG_loc"], sc["bzg_loc"], group)
     ops.suffix(G_all, zg_all, rank, sc["bG_in"], sc["bzg_in"])
-    ops.backward(q, k, v, out, den, dout, dq, dk, dv, sc["bS_in"], sc["bz_in"], sc["bG_in"],
-                 sc["bzg_in"])
+    ops.backward(q, k, v, out, den, dout, dq, dk, dv, S_in, z_in, sc["bG_in"], sc["bzg_in"])
     return dq, dk, dv

@@ -226,12 +226,16 @@ def _seqpar_bwd_rank(rank, world, port, outdir):
         ops = _OracleOps(P)
         out = torch.empty((1, 2, b - a, 64), dtype=torch.float64)
         den = torch.empty((1, 2, b - a), dtype=torch.float64)
-        seqpar.causal_fwd_seqpar(piece[0], piece[1], piece[2], out, den, w.F, ops)
-        dq, dk, dv = (torch.empty((1, 2, b - a, 64), dtype=torch.float64) for _ in range(3))
-        seqpar.causal_bwd_seqpar(piece[0], piece[1], piece[2], out, den, piece[3], dq, dk, dv, w.F,
-                                 ops)
-        np.save(os.path.join(outdir, "spb%d.npy" % rank), np.stack([dq.numpy(), dk.numpy(),
-                                                                    dv.numpy()]))
+        scratch = {}
+        seqpar.causal_fwd_seqpar(piece[0], piece[1], piece[2], out, den, w.F, ops, scratch=scratch)
+        res = []
+        for reuse in (False, True):   # the forward's state recomputed, or passed in
+            dq, dk, dv = (torch.empty((1, 2, b - a, 64), dtype=torch.float64) for _ in range(3))
+            seqpar.causal_bwd_seqpar(piece[0], piece[1], piece[2], out, den, piece[3], dq, dk, dv,
+                                     w.F, ops, fwd_state=(scratch["S_in"], scratch["z_in"])
+                                     if reuse else None)
+            res.append(np.stack([dq.numpy(), dk.numpy(), dv.numpy()]))
+        np.save(os.path.join(outdir, "spb%d.npy" % rank), np.stack(res))
     finally:
         dist.destroy_process_group()
 
@@ -244,7 +248,9 @@ def test_sequence_parallel_backward_orchestration_two_ranks():
     import oracle as O
     outdir = tempfile.mkdtemp(prefix="slay_spb_")
     mp.spawn(_seqpar_bwd_rank, args=(2, _free_port(), outdir), nprocs=2, join=True)
-    got = np.concatenate([np.load(os.path.join(outdir, "spb%d.npy" % r)) for r in range(2)], axis=3)
+    got2 = np.concatenate([np.load(os.path.join(outdir, "spb%d.npy" % r)) for r in range(2)], axis=4)
+    np.testing.assert_array_equal(got2[0], got2[1])
+    got = got2[0]
     w = W.Workload("spb", B=1, H=2, L=60, R=2, m=8, dtype="f32", data_seed=62)
     q, k, v = W.gen_qkv(w)
     g = W.gen_dout(w)
