@@ -18,15 +18,17 @@
 //            P~ and C~ into shared memory;
 //   phase B: dV = P~^T dn, then per slice s: dphiQ_s = C~ phiK_s + dn S_s^T,
 //            dphiK_s = C~^T phiQ_s + V G_s^T, dV += phiK_s G_s; the epilogue adds the z terms
-//            and writes dphiQ, dphiK (fp32) per slice, dV per tile.
+//            and writes dphiQ, dphiK per slice (bf16 through TMA stores, or fp32), dV per
+//            tile.
 // The ones / delta columns never enter an MMA (their terms are rank one, added in fp32),
 // so every contraction has K a multiple of 64.  The transposed products read the same
 // shared-memory tiles as MN-major operands.
 //
 // Persistent, one CTA per SM over the (b, h, tile) items.  Warp 0 issues the MMAs, warp 9
-// the TMA loads (V and dn (bf16 rows), and the phi slice pairs of both phases through a ring
-// of two), warps 1-8 are the epilogue (lane quadrant w % 4, column half (w - 1) / 4; delta per
-// row from its fp32 array).  Every wait is bounded; a timeout sets the workspace status word.
+// the TMA loads (V and dn (bf16 rows), the phi slice pairs of both phases through a ring of
+// two, and per phase-B slice S_s and G_s from k_tc_bwd_sums' operand slabs), warps 1-8 are
+// the epilogue (lane quadrant w % 4, column half (w - 1) / 4; delta per row from its fp32
+// array).  Every wait is bounded; a timeout sets the workspace status word.
 #include <cuda.h>
 #include <cuda_runtime.h>
 

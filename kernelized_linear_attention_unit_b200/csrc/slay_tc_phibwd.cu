@@ -9,19 +9,22 @@
 //   dx^ = sum_f alpha_f omega_f + beta_f a_f,   t = dphi_f e p,
 //   alpha_f = t p sqrt(2 s_r),  beta_f = 2 n t,
 //   dx = (dx^ - x^ (x^ . dx^)) / n   (dx^ / 1e-12 below the norm guard |x| < 1e-12).
-// Both contractions run on tensor cores: per 128-row tile and 64-feature group g the
+// Both contractions run on tensor cores: per 128-row tile and 64-feature group g (a job) the
 // projections U = X W_g^T (N = 128: 64 omega and 64 anchor columns, as in the forward map),
-// then dX^ += [alpha | beta]_g [Omega_g ; A_g] (K = 128, N = 64) with the same resident W
-// tiles read as an MN-major operand.  The kernel reads x (bf16), dphi (bf16, as the
-// tensor-core contraction stores it) and writes dx (fp32): it is bound by the dphi reads
-// (2F bytes per row).
+// then dX^ += [alpha | beta]_g [Omega_g ; A_g] (K = 128, N = 64) with the same W tiles read
+// as an MN-major operand.  The kernel reads x (bf16), dphi (bf16, as the tensor-core
+// contraction stores it) and writes dx (fp32): its DRAM traffic is dominated by the dphi
+// reads (2F bytes per row).
 //
-// Persistent, one CTA per SM, 128-row tiles round-robin.  Warp 0 issues every TMA load and
-// MMA; warps 1-8 are the epilogue: warp w serves TMEM lanes 32 (w % 4).. (rows of the tile)
-// and the 32-feature half (w - 1) / 4 of every group.  Per group an epilogue warp reads its
-// projections, its rows' dphi (bf16, loaded two groups ahead) and writes its block of
-// [alpha | beta] into a K-major 128-byte-swizzled operand tile; per tile it turns dX^ into
-// dx.  Every wait is bounded; a timeout sets the library's feature-map status word.
+// Persistent, one CTA per SM, 128-row tiles round-robin.  Warp 9 issues the TMA loads: X
+// tiles, and per job the group's W operand (three slots, L2-resident) and the dphi tile
+// [128 rows][64 features] (two slots).  Warp 0 issues the MMAs.  Warps 1-8 are the epilogue:
+// warp w serves TMEM lanes 32 (w % 4).. (rows of the tile) and the 32-feature half
+// (w - 1) / 4 of every group; per job it reads its rows' dphi from the shared-memory tile,
+// its projections from tensor memory, and writes its block of [alpha | beta] into a K-major
+// 128-byte-swizzled operand tile; per tile, after the next tile's jobs, it turns dX^ into
+// dx and stores its 32 x 32 block by TMA.  Every wait is bounded; a timeout sets the
+// library's feature-map status word.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -119,7 +122,7 @@ struct Ring {
 __global__ void __launch_bounds__(kPbThreads, 1)
 k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
              const __grid_constant__ CUtensorMap tmd, const __grid_constant__ CUtensorMap tmdx,
-             int64_t n_rows, PbParams pp, int* status)
+             PbParams pp, int* status)
 {
     constexpr int kW = 4;     // 16-byte words per 32 bf16 dphi values
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -316,8 +319,8 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
             // derivative is the identity / 1e-12: no tangential projection there
             const float xd = nrm > 1e-12f ? ((dot[0] + dot[1]) + (dot[2] + dot[3])) * inv : 0.0f;
             // this warp's 32 rows x 32 columns through its staging box (128-byte swizzle:
-            // 16-byte chunk c of row r at c ^ (r & 7)) and a TMA store; rows past n_rows are
-            // clipped by the tensor map
+            // 16-byte chunk c of row r at c ^ (r & 7)) and a TMA store; rows past the last row
+            // are clipped by the tensor map
             const uint32_t box = sbase + L.stg + ew * kStgBytes;
             if (lane == 0) bulk_wait_read<0>();   // the previous tile's store has read it
             __syncwarp();
@@ -497,7 +500,7 @@ cudaError_t tc_phi_bwd(const void* x, const void* dphi, float* dx, int64_t n, co
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     TraceScope trace_("tc_phi_bwd", st);
-    k_tc_phi_bwd<<<grid, kPbThreads, smem, st>>>(mx, mw, md, mdx, n, pp, status);
+    k_tc_phi_bwd<<<grid, kPbThreads, smem, st>>>(mx, mw, md, mdx, pp, status);
     return cudaGetLastError();
 }
 
