@@ -49,7 +49,9 @@
  *     buffer per (device, D, R, m, seed, eps), created on first use (synchronous
  *     allocation and upload; call slay_prepare before capturing a stream into a CUDA
  *     graph) and held until the process exits.  The cache is thread-safe.
- *   - Empty work (L == 0, n_rows == 0, B*H == 0) returns SLAY_OK and enqueues nothing.
+ *   - Empty work (L == 0, n_rows == 0, B*H == 0) returns SLAY_OK and enqueues nothing (but
+ *     for the calls whose outputs are states, which at L == 0 still write them); it leaves
+ *     the workspace, and so its status word, as it was.
  */
 #ifndef SLAY_H
 #define SLAY_H
@@ -80,7 +82,8 @@ typedef enum {
     SLAY_OP_DECODE = 4,
     SLAY_OP_BIDIR_BWD = 5,
     SLAY_OP_LINEAR_ATTN = 6,    /* slay_linear_attn_fwd: R * m = the number of features */
-    SLAY_OP_CAUSAL_STATE = 7    /* slay_causal_state */
+    SLAY_OP_CAUSAL_STATE = 7,   /* slay_causal_state */
+    SLAY_OP_CAUSAL_FWD_SPLIT = 8 /* slay_attn_causal_fwd_begin / _finish (one workspace) */
 } slay_op;
 
 /* Feature-map variants (slay_feature_map_ex).  The pages leave the form of the anchor
@@ -156,6 +159,39 @@ slay_status slay_causal_state(const void* k, const void* v, const float* S_in, c
  * z_in [BH][F] written (zero for rank 0).  F = R*m <= 1024, Dv == 64. */
 slay_status slay_state_prefix(const float* S_all, const float* z_all, int nranks, int rank,
                               float* S_in, float* z_in, int BH, int F, int Dv, void* stream);
+
+/* The sequence-parallel forward of one piece in two calls that share a workspace, so that the
+ * piece's phi(k) and per-segment state sums are made once, for the exchange and the forward
+ * alike (review, "Proposed method", step 6: the prefix state carries every earlier token, so
+ * only the pieces' totals cross ranks).  Between the calls the caller exchanges the totals
+ * and forms the prefix (slay_state_prefix).
+ *
+ * slay_attn_causal_fwd_begin writes this piece's state
+ *     S_out = sum_j phi(k_j) v_j^T,  z_out = sum_j phi(k_j)   over its L tokens per (b,h)
+ *   (slay_causal_state with S_in NULL; zero when L == 0) and leaves in `workspace` what the
+ *   second call reads.  S_out [B,H,R*m,Dv], z_out [B,H,R*m] fp32, both required.
+ * slay_attn_causal_fwd_finish writes out (and den, if not NULL) of the piece continued from
+ *   S_in, z_in ([B,H,R*m,Dv], [B,H,R*m] fp32, or both NULL for a zero state): the values
+ *   slay_attn_causal_fwd_state writes for the same arguments.  It must come after the first
+ *   call in stream order, with the same k, v, B, H, L, D, Dv, dt, R, m, seed, eps and
+ *   workspace, nothing else writing the workspace in between.  q, k, v, out, den as
+ *   slay_attn_causal_fwd.
+ * workspace: slay_workspace_bytes(SLAY_OP_CAUSAL_FWD_SPLIT, ...) bytes, caller-owned, its
+ *   contents the library's from the first call to the second; its first int is the status
+ *   word of both calls' tensor-core kernels (the first call clears it, the second does not).
+ * bf16 at tensor-core sizes: the first call runs the causal forward's state kernel (phi(k)
+ * stored, every segment's sum) and the totals, the second only its output kernel.  Otherwise
+ * CUDA cores: the first call is slay_causal_state, the second slay_attn_causal_fwd_state.
+ * Errors as slay_attn_causal_fwd; on an error nothing is enqueued. */
+slay_status slay_attn_causal_fwd_begin(const void* k, const void* v, float* S_out, float* z_out,
+                                       int B, int H, int L, int D, int Dv, slay_dtype dt, int R,
+                                       int m, uint64_t seed, float eps, void* workspace,
+                                       size_t ws_bytes, void* stream);
+slay_status slay_attn_causal_fwd_finish(const void* q, const void* k, const void* v, void* out,
+                                        float* den, const float* S_in, const float* z_in, int B,
+                                        int H, int L, int D, int Dv, slay_dtype dt, int R, int m,
+                                        uint64_t seed, float eps, void* workspace,
+                                        size_t ws_bytes, void* stream);
 
 /* The counterpart of slay_state_prefix for the backward (sequence parallelism):
  *   S_out = sum_{r > rank} S_all[r],  z_out = sum_{r > rank} z_all[r]

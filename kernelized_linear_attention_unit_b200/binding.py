@@ -18,7 +18,7 @@ SLAY_OK, SLAY_ERR_INVALID_ARG, SLAY_ERR_UNSUPPORTED, SLAY_ERR_CUDA, SLAY_ERR_TIM
     SLAY_ERR_NO_MEMORY = range(6)
 SLAY_F32, SLAY_BF16 = 0, 1
 OP_FEATURE_MAP, OP_CAUSAL_FWD, OP_BIDIR_FWD, OP_CAUSAL_BWD, OP_DECODE, OP_BIDIR_BWD, \
-    OP_LINEAR_ATTN, OP_CAUSAL_STATE = range(8)
+    OP_LINEAR_ATTN, OP_CAUSAL_STATE, OP_CAUSAL_FWD_SPLIT = range(9)
 PHI_ANCHOR, PHI_ORTHOGONAL, PHI_SIGNED, PHI_PER_HEAD, PHI_PERFORMER = range(5)
 
 EXPORTS = ["slay_feature_map", "slay_attn_causal_fwd", "slay_attn_bidir_fwd",
@@ -28,7 +28,8 @@ EXPORTS = ["slay_feature_map", "slay_attn_causal_fwd", "slay_attn_bidir_fwd",
            "slay_debug_expire_wait", "slay_attn_bidir_bwd", "slay_feature_map_bwd",
            "slay_feature_map_ex", "slay_sketch_params_ex", "slay_linear_attn_fwd",
            "slay_attn_causal_fwd_state", "slay_causal_state", "slay_state_prefix",
-           "slay_state_suffix", "slay_attn_causal_bwd_state", "slay_causal_bwd_state"]
+           "slay_state_suffix", "slay_attn_causal_bwd_state", "slay_causal_bwd_state",
+           "slay_attn_causal_fwd_begin", "slay_attn_causal_fwd_finish"]
 
 
 class SlayError(RuntimeError):
@@ -73,6 +74,8 @@ def lib():
                                              i32, i32, i32, i32, i32, u64, f32, vp, sz, vp]
     L.slay_causal_state.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
                                     u64, f32, vp, sz, vp]
+    L.slay_attn_causal_fwd_begin.argtypes = [vp] * 4 + [i32] * 8 + [u64, f32, vp, sz, vp]
+    L.slay_attn_causal_fwd_finish.argtypes = [vp] * 7 + [i32] * 8 + [u64, f32, vp, sz, vp]
     L.slay_state_prefix.argtypes = [vp, vp, i32, i32, vp, vp, i32, i32, i32, vp]
     L.slay_state_suffix.argtypes = L.slay_state_prefix.argtypes
     L.slay_attn_causal_bwd_state.argtypes = [vp] * 13 + [i32] * 8 + [u64, f32, vp, sz, vp]
@@ -101,7 +104,8 @@ def lib():
                  "slay_sketch_params_ex", "slay_linear_attn_fwd", "slay_attn_causal_fwd_state",
                  "slay_causal_state", "slay_state_prefix", "slay_state_suffix",
                  "slay_attn_causal_bwd_state", "slay_causal_bwd_state",
-                 "slay_attn_causal_fwd_noalloc",
+                 "slay_attn_causal_fwd_noalloc", "slay_attn_causal_fwd_begin",
+                 "slay_attn_causal_fwd_finish",
                  "slay_sketch_params"):
         getattr(L, name).restype = i32
     _lib = L
@@ -152,8 +156,12 @@ def slay_workspace_bytes(op, dtype, B, H, L, D, Dv, R, m) -> int:
 
 
 def alloc_workspace(op, dtype, B, H, L, D, Dv, R, m, device=None):
-    """Caller-owned workspace of the size the library asks for (torch allocation)."""
+    """Caller-owned workspace of the size the library asks for (torch allocation).  When the
+    call needs none (empty work, which enqueues nothing and leaves the workspace as it is),
+    a zeroed 256-byte block, so that slay_kernel_status on it reads a clear status word."""
     n = slay_workspace_bytes(op, dtype, B, H, L, D, Dv, R, m)
+    if n == 0:
+        return torch.zeros(256, dtype=torch.uint8, device=device or "cuda")
     return torch.empty(max(n, 256), dtype=torch.uint8, device=device or "cuda")
 
 
@@ -387,6 +395,47 @@ def slay_causal_state(k, v, S_out, z_out, R, m, seed, eps, S_in=None, z_in=None,
                                    seed, eps, _ptr(workspace), wbytes, _stream(stream)),
            "slay_causal_state")
     return workspace
+
+
+def slay_attn_causal_fwd_begin(k, v, S_out, z_out, R, m, seed, eps, workspace=None,
+                               stream=None):
+    """First call of the two-call forward: this piece's state S_out = sum phi(k) v^T,
+    z_out = sum phi(k) [B,H,F,64], [B,H,F] fp32; the workspace it returns (or the one given)
+    carries phi(k) and the segment sums to slay_attn_causal_fwd_finish."""
+    _check(k, "k")
+    B, H, L, D = k.shape
+    Dv = v.shape[-1]
+    _check(v, "v", k.dtype, (B, H, L, Dv))
+    F = R * m
+    so, zo = _state_ptrs(S_out, z_out, (B, H), F, "state out")
+    dt = _dt(k)
+    if workspace is None:
+        workspace = alloc_workspace(OP_CAUSAL_FWD_SPLIT, dt, B, H, L, D, Dv, R, m, k.device)
+    wbytes = workspace.numel() * workspace.element_size()
+    _raise(lib().slay_attn_causal_fwd_begin(_ptr(k), _ptr(v), so, zo, B, H, L, D, Dv, dt, R, m,
+                                            seed, eps, _ptr(workspace), wbytes, _stream(stream)),
+           "slay_attn_causal_fwd_begin")
+    return workspace
+
+
+def slay_attn_causal_fwd_finish(q, k, v, out, den, R, m, seed, eps, workspace, S_in=None,
+                                z_in=None, stream=None):
+    """Second call of the two-call forward: out (and den) of the piece from the state
+    (S_in, z_in) (None: zero), on the workspace of slay_attn_causal_fwd_begin for k, v."""
+    _check(q, "q")
+    B, H, L, D = q.shape
+    Dv = v.shape[-1]
+    _check(k, "k", q.dtype, (B, H, L, D))
+    _check(v, "v", q.dtype, (B, H, L, Dv))
+    _check(out, "out", q.dtype, (B, H, L, Dv))
+    if den is not None:
+        _check(den, "den", torch.float32, (B, H, L))
+    si, zi = _state_ptrs(S_in, z_in, (B, H), R * m, "state in")
+    wbytes = workspace.numel() * workspace.element_size()
+    _raise(lib().slay_attn_causal_fwd_finish(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(den),
+                                             si, zi, B, H, L, D, Dv, _dt(q), R, m, seed, eps,
+                                             _ptr(workspace), wbytes, _stream(stream)),
+           "slay_attn_causal_fwd_finish")
 
 
 def slay_state_prefix(S_all, z_all, rank, S_in, z_in, stream=None):

@@ -4,6 +4,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstdint>
@@ -235,6 +236,11 @@ size_t attn_ws(slay_op op, slay_dtype dt, int B, int H, int L, int Dv, int R, in
     if (op == SLAY_OP_CAUSAL_STATE) {
         if (dt == SLAY_BF16 && tc_supported(SLAY_OP_CAUSAL_FWD, B, H, L, R, m))
             return tc_state_workspace_bytes(B, H, L, R, m);
+    } else if (op == SLAY_OP_CAUSAL_FWD_SPLIT) {
+        if (dt == SLAY_BF16 && tc_supported(SLAY_OP_CAUSAL_FWD, B, H, L, R, m))
+            return tc_workspace_bytes(op, B, H, L, R, m);
+        // CUDA cores: the piece-state call and the forward, one after the other
+        return kWsHeader + std::max(simt_ws_causal(B, H, L, Dv, F), simt_ws_state(B, H, L, F));
     } else if (dt == SLAY_BF16 && tc_supported(op, B, H, L, R, m)) {
         return tc_workspace_bytes(op, B, H, L, R, m);
     }
@@ -542,6 +548,68 @@ slay_status slay_causal_state(const void* k, const void* v, const float* S_in, c
     return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
 }
 
+slay_status slay_attn_causal_fwd_begin(const void* k, const void* v, float* S_out, float* z_out,
+                                       int B, int H, int L, int D, int Dv, slay_dtype dt, int R,
+                                       int m, uint64_t seed, float eps, void* workspace,
+                                       size_t ws_bytes, void* stream)
+{
+    slay_status s = check_attn(k, k, v, v, B, H, L, D, Dv, dt, R, m, eps);
+    if (s != SLAY_OK) return s;
+    if (!S_out || !z_out) return SLAY_ERR_INVALID_ARG;
+    if ((s = check_state_ptrs(S_out, z_out)) != SLAY_OK) return s;
+    if (static_cast<int64_t>(B) * H == 0) return SLAY_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (L == 0) {   // an empty piece adds nothing to the state
+        const size_t bs = static_cast<size_t>(B) * H * R * m * Dv * sizeof(float);
+        const size_t bz = static_cast<size_t>(B) * H * R * m * sizeof(float);
+        cudaError_t e = cudaMemsetAsync(S_out, 0, bs, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(z_out, 0, bz, st);
+        return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
+    }
+    const size_t need = attn_ws(SLAY_OP_CAUSAL_FWD_SPLIT, dt, B, H, L, Dv, R, m);
+    if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return SLAY_ERR_INVALID_ARG;
+    Params P;
+    if ((s = get_params(D, R, m, seed, eps, &P)) != SLAY_OK) return s;
+    cudaError_t e;
+    if (dt == SLAY_BF16 && tc_supported(SLAY_OP_CAUSAL_FWD, B, H, L, R, m)) {
+        e = tc_attn_fwd_begin(k, v, B, H, L, P, eps, workspace, st, S_out, z_out);
+    } else {
+        const StateIO sio{nullptr, nullptr, S_out, z_out};
+        e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
+        if (e == cudaSuccess)
+            e = simt_causal_state(k, v, B, H, L, dt, P, static_cast<char*>(workspace) + kWsHeader,
+                                  st, sio);
+    }
+    return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
+}
+
+slay_status slay_attn_causal_fwd_finish(const void* q, const void* k, const void* v, void* out,
+                                        float* den, const float* S_in, const float* z_in, int B,
+                                        int H, int L, int D, int Dv, slay_dtype dt, int R, int m,
+                                        uint64_t seed, float eps, void* workspace,
+                                        size_t ws_bytes, void* stream)
+{
+    slay_status s = check_attn(q, k, v, out, B, H, L, D, Dv, dt, R, m, eps);
+    if (s != SLAY_OK) return s;
+    if ((s = check_state_ptrs(S_in, z_in)) != SLAY_OK) return s;
+    if (static_cast<int64_t>(B) * H * L == 0) return SLAY_OK;
+    if (den && !aligned(den, 4)) return SLAY_ERR_INVALID_ARG;
+    const size_t need = attn_ws(SLAY_OP_CAUSAL_FWD_SPLIT, dt, B, H, L, Dv, R, m);
+    if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return SLAY_ERR_INVALID_ARG;
+    Params P;
+    if ((s = get_params(D, R, m, seed, eps, &P)) != SLAY_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (dt == SLAY_BF16 && tc_supported(SLAY_OP_CAUSAL_FWD, B, H, L, R, m)) {
+        e = tc_attn_fwd_finish(q, v, out, den, B, H, L, P, eps, workspace, st, S_in, z_in);
+    } else {
+        const StateIO sio{S_in, z_in, nullptr, nullptr};
+        e = simt_attn_fwd(q, k, v, out, den, B, H, L, dt, P, eps, true,
+                          static_cast<char*>(workspace) + kWsHeader, st, &sio);
+    }
+    return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
+}
+
 slay_status slay_state_prefix(const float* S_all, const float* z_all, int nranks, int rank,
                               float* S_in, float* z_in, int BH, int F, int Dv, void* stream)
 {
@@ -692,7 +760,8 @@ size_t slay_workspace_bytes(slay_op op, slay_dtype dt, int B, int H, int L, int 
     if (check_shape(D, Dv, R, m) != SLAY_OK) return SIZE_MAX;
     if (op == SLAY_OP_FEATURE_MAP || op == SLAY_OP_DECODE) return 0;
     if (op != SLAY_OP_CAUSAL_FWD && op != SLAY_OP_BIDIR_FWD && op != SLAY_OP_CAUSAL_BWD &&
-        op != SLAY_OP_BIDIR_BWD && op != SLAY_OP_LINEAR_ATTN && op != SLAY_OP_CAUSAL_STATE)
+        op != SLAY_OP_BIDIR_BWD && op != SLAY_OP_LINEAR_ATTN && op != SLAY_OP_CAUSAL_STATE &&
+        op != SLAY_OP_CAUSAL_FWD_SPLIT)
         return SIZE_MAX;
     if (op == SLAY_OP_LINEAR_ATTN) {   // the contraction alone: F = R * m features given
         if (static_cast<int64_t>(B) * H * L == 0) return 0;

@@ -1937,22 +1937,25 @@ namespace {
 // Workspace: header | per-segment S [BH][nseg][Fc][64] fp32 | z [BH][nseg][Fc] fp32 | for the
 // causal forward that stores phi(k): phi(k) [BH][L][Fc] bf16 | with more than one feature
 // chunk: partial numerators [BH][L][64] and denominators [BH][L] fp32.  Fc is the chunk
-// width; the chunks run one after another and reuse the per-chunk parts.
+// width; the chunks run one after another and reuse the per-chunk parts, except in the
+// two-call forward (keep_chunks), which keeps every chunk's S, z and phi(k) from the first
+// call to the second: chunk c's parts start c times the per-chunk size in (chunk_parts).
 struct WsLayout {
     size_t s, z, phik, num, den, total;
 };
 
-WsLayout ws_layout(int BH, int L, int F, int nseg, bool with_phik)
+WsLayout ws_layout(int BH, int L, int F, int nseg, bool with_phik, bool keep_chunks = false)
 {
     const int Fc = chunk_features(F);
-    const size_t per = static_cast<size_t>(BH) * nseg * Fc;
+    const int kept = keep_chunks ? F / Fc : 1;
+    const size_t per = static_cast<size_t>(BH) * nseg * Fc * kept;
     const size_t rows = static_cast<size_t>(BH) * L;
     auto up = [](size_t b) { return (b + 255) & ~size_t(255); };
     WsLayout w;
     w.s = kWsHeader;
     w.z = w.s + up(per * 64 * sizeof(float));
     w.phik = w.z + up(per * sizeof(float));
-    w.num = w.phik + up(with_phik ? rows * Fc * sizeof(uint16_t) : 0);
+    w.num = w.phik + up(with_phik ? rows * Fc * kept * sizeof(uint16_t) : 0);
     const bool chunked = Fc < F;
     w.den = w.num + (chunked ? up(rows * 64 * sizeof(float)) : 0);
     w.total = w.den + (chunked ? up(rows * sizeof(float)) : 0);
@@ -1963,9 +1966,10 @@ WsLayout ws_layout(int BH, int L, int F, int nseg, bool with_phik)
 
 size_t tc_workspace_bytes(slay_op op, int B, int H, int L, int R, int m, bool lowmem)
 {
-    if (op != SLAY_OP_CAUSAL_FWD && op != SLAY_OP_BIDIR_FWD) return 0;
     const int BH = B * H;
     const int nseg = choose_nseg(BH, (L + kTile - 1) / kTile);
+    if (op == SLAY_OP_CAUSAL_FWD_SPLIT) return ws_layout(BH, L, R * m, nseg, true, true).total;
+    if (op != SLAY_OP_CAUSAL_FWD && op != SLAY_OP_BIDIR_FWD) return 0;
     return ws_layout(BH, L, R * m, nseg, op == SLAY_OP_CAUSAL_FWD && !lowmem).total;
 }
 
@@ -2059,6 +2063,102 @@ __global__ void k_state_total(const float* __restrict__ wsS, const float* __rest
     }
 }
 
+namespace {
+
+// The parameters of feature chunk c of nch (features [c Fc, (c+1) Fc), packed W sub-slices
+// from c Fc / 32 on): the node scales of its 64-feature slices, where its numerators and
+// denominators go (the chunk sums in the workspace while more chunks follow) and the state
+// entering the sequence (sio->s_in; null: zero).
+KParams chunk_kparams(const Params& P, int L, int Fc, int nch, int nseg, int ntiles, float eps,
+                      int c, char* w, const WsLayout& wl, const StateIO* sio)
+{
+    KParams kp{};
+    kp.L = L; kp.F = Fc; kp.nseg = nseg; kp.ntiles = ntiles; kp.eps = eps;
+    kp.all_segs = 1;
+    for (int t = 0; t < kMaxSlices; ++t) {
+        const int node = t < Fc / kSlice ? (c * Fc + t * kSlice) / P.m : 0;
+        kp.a2[t] = P.a2[node];
+        kp.b2[t] = P.b2[node];
+    }
+    kp.acc_in = c > 0;
+    kp.acc_out = c + 1 < nch;
+    kp.part_num = nch > 1 ? reinterpret_cast<float*>(w + wl.num) : nullptr;
+    kp.part_den = nch > 1 ? reinterpret_cast<float*>(w + wl.den) : nullptr;
+    const int F = Fc * nch;
+    kp.s_in = (sio && sio->s_in) ? sio->s_in + static_cast<size_t>(c) * Fc * 64 : nullptr;
+    kp.z_in = (sio && sio->s_in) ? sio->z_in + static_cast<size_t>(c) * Fc : nullptr;
+    kp.s_stride = F * 64;
+    kp.z_stride = F;
+    return kp;
+}
+
+bool map_chunk_w(CUtensorMap* mw, const Params& P, int Fc, int c)
+{
+    return map_w(mw, P.wB + static_cast<size_t>(c) * (Fc / kSub) * 64 * 64, Fc);
+}
+
+// The causal output kernel on stored phi(k) for one chunk; `dependent`: launched as the
+// dependent of the state kernel just ahead of it in the stream (its prologue overlaps that
+// kernel's tail), else an ordinary launch.
+cudaError_t launch_out_ts(const KParams& kp, int grid, bool dependent, cudaStream_t st,
+                          const CUtensorMap& mq, const CUtensorMap& mpk, const CUtensorMap& mv,
+                          const CUtensorMap& mw, const float* wsS, const float* wsZ,
+                          __nv_bfloat16* o, float* den, int* err)
+{
+    const size_t smo = smem_outts_layout(kp.F).total + 1024;
+    auto kern = k_tc_causal_out_ts<0>;
+    switch ((kp.acc_in ? 1 : 0) | (kp.acc_out ? 2 : 0)) {
+    case 1: kern = k_tc_causal_out_ts<1>; break;
+    case 2: kern = k_tc_causal_out_ts<2>; break;
+    case 3: kern = k_tc_causal_out_ts<3>; break;
+    default: break;
+    }
+    cudaError_t e = set_smem(kern, smo);
+    if (e != cudaSuccess) return e;
+    TraceScope trace_("tc_qphi_out", st);
+    if (dependent) {
+        e = launch_dependent(kern, grid, kOutThreads, smo, st, mq, mpk, mv, mw, kp, wsS, wsZ, o, den, err);
+    } else {
+        kern<<<grid, kOutThreads, smo, st>>>(mq, mpk, mv, mw, kp, wsS, wsZ, o, den, err);
+        e = cudaSuccess;
+    }
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+// The state after the sequence for one chunk: s_out/z_out = s_in + the sum of every segment's
+// sum (null s_in: zero).
+cudaError_t launch_state_total(const float* wsS, const float* wsZ, int BH, int nseg, int Fc, int F,
+                               int c, const float* s_in, const float* z_in, float* s_out,
+                               float* z_out, cudaStream_t st)
+{
+    TraceScope trace_("tc_state_total", st);
+    const int64_t n = static_cast<int64_t>(BH) * Fc * 64;
+    const int grid = static_cast<int>(std::min<int64_t>((n + 255) / 256, 4 * kNumSMs));
+    k_state_total<<<grid, 256, 0, st>>>(wsS, wsZ, BH, nseg, Fc, F, c * Fc, s_in, z_in, s_out, z_out);
+    return cudaGetLastError();
+}
+
+// Chunk c's per-segment sums and phi(k) in the two-call forward's workspace.
+struct ChunkParts {
+    float* s;
+    float* z;
+    void* phik;
+};
+
+ChunkParts chunk_parts(char* w, const WsLayout& wl, int BH, int L, int nseg, int Fc, int c)
+{
+    const size_t per = static_cast<size_t>(BH) * nseg * Fc;
+    const size_t rows = static_cast<size_t>(BH) * L;
+    ChunkParts p;
+    p.s = reinterpret_cast<float*>(w + wl.s) + static_cast<size_t>(c) * per * 64;
+    p.z = reinterpret_cast<float*>(w + wl.z) + static_cast<size_t>(c) * per;
+    p.phik = reinterpret_cast<uint16_t*>(w + wl.phik) + static_cast<size_t>(c) * rows * Fc;
+    return p;
+}
+
+}  // namespace
+
 size_t tc_state_workspace_bytes(int B, int H, int L, int R, int m)
 {
     const int BH = B * H;
@@ -2086,27 +2186,15 @@ cudaError_t tc_causal_state(const void* k, const void* v, int B, int H, int L, c
     if ((e = set_smem(k_tc_causal_state<false>, sms)) != cudaSuccess) return e;
     for (int c = 0; c < nch; ++c) {
         CUtensorMap mw;
-        const uint16_t* wc = P.wB + static_cast<size_t>(c) * (Fc / kSub) * 64 * 64;
-        if (!map_w(&mw, wc, Fc)) return cudaErrorInvalidValue;
-        KParams kp{};
-        kp.L = L; kp.F = Fc; kp.nseg = nseg; kp.ntiles = ntiles;
-        kp.all_segs = 1;
-        for (int t = 0; t < kMaxSlices; ++t) {
-            const int node = t < Fc / kSlice ? (c * Fc + t * kSlice) / P.m : 0;
-            kp.a2[t] = P.a2[node];
-            kp.b2[t] = P.b2[node];
-        }
+        if (!map_chunk_w(&mw, P, Fc, c)) return cudaErrorInvalidValue;
+        const KParams kp = chunk_kparams(P, L, Fc, nch, nseg, ntiles, 0.0f, c, w, wl, nullptr);
         {
             TraceScope trace_("tc_state_sums", st);
             k_tc_causal_state<false><<<BH * nseg, kThreads, sms, st>>>(mk, mv, mw, mpk, kp, wsS, wsZ, err);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
-        TraceScope trace_("tc_state_total", st);
-        const int64_t n = static_cast<int64_t>(BH) * Fc * 64;
-        const int grid = static_cast<int>(std::min<int64_t>((n + 255) / 256, 4 * kNumSMs));
-        k_state_total<<<grid, 256, 0, st>>>(wsS, wsZ, BH, nseg, Fc, F, c * Fc, sio.s_in, sio.z_in,
-                                            sio.s_out, sio.z_out);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        e = launch_state_total(wsS, wsZ, BH, nseg, Fc, F, c, sio.s_in, sio.z_in, sio.s_out, sio.z_out, st);
+        if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
 }
@@ -2138,26 +2226,10 @@ cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, 
     if (e != cudaSuccess) return e;
     const size_t sms = smem_bytes_state(Fc);
     for (int c = 0; c < nch; ++c) {
-        // chunk c: features [c Fc, (c+1) Fc), i.e. packed W sub-slices from c Fc / 32 on
         CUtensorMap mw;
-        const uint16_t* wc = P.wB + static_cast<size_t>(c) * (Fc / kSub) * 64 * 64;
-        if (!map_w(&mw, wc, Fc)) return cudaErrorInvalidValue;
-        KParams kp;
-        kp.L = L; kp.F = Fc; kp.nseg = nseg; kp.ntiles = ntiles; kp.eps = eps;
+        if (!map_chunk_w(&mw, P, Fc, c)) return cudaErrorInvalidValue;
+        KParams kp = chunk_kparams(P, L, Fc, nch, nseg, ntiles, eps, c, w, wl, sio);
         kp.all_segs = (causal && lowmem) ? 0 : 1;
-        for (int t = 0; t < kMaxSlices; ++t) {
-            const int node = t < Fc / kSlice ? (c * Fc + t * kSlice) / P.m : 0;
-            kp.a2[t] = P.a2[node];
-            kp.b2[t] = P.b2[node];
-        }
-        kp.acc_in = c > 0;
-        kp.acc_out = c + 1 < nch;
-        kp.part_num = nch > 1 ? reinterpret_cast<float*>(w + wl.num) : nullptr;
-        kp.part_den = nch > 1 ? reinterpret_cast<float*>(w + wl.den) : nullptr;
-        kp.s_in = (sio && sio->s_in) ? sio->s_in + static_cast<size_t>(c) * Fc * 64 : nullptr;
-        kp.z_in = (sio && sio->s_in) ? sio->z_in + static_cast<size_t>(c) * Fc : nullptr;
-        kp.s_stride = F * 64;
-        kp.z_stride = F;
         if (!causal) {
             // every segment's sum, then the readout against their total
             if ((e = set_smem(k_tc_causal_state<false>, sms)) != cudaSuccess) return e;
@@ -2182,28 +2254,12 @@ cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, 
                 k_tc_causal_state<true><<<BH * nseg, kThreads, sms, st>>>(mk, mv, mw, mpk, kp, wsS, wsZ, err);
                 if ((e = cudaGetLastError()) != cudaSuccess) return e;
             }
-            const size_t smo = smem_outts_layout(Fc).total + 1024;
-            auto kern = k_tc_causal_out_ts<0>;
-            switch ((kp.acc_in ? 1 : 0) | (kp.acc_out ? 2 : 0)) {
-            case 1: kern = k_tc_causal_out_ts<1>; break;
-            case 2: kern = k_tc_causal_out_ts<2>; break;
-            case 3: kern = k_tc_causal_out_ts<3>; break;
-            default: break;
-            }
-            if ((e = set_smem(kern, smo)) != cudaSuccess) return e;
-            {
-                TraceScope trace_("tc_qphi_out", st);
-                e = launch_dependent(kern, BH * nseg, kOutThreads, smo, st, mq, mpk, mv, mw, kp, wsS, wsZ, o, den, err);
-                if (e != cudaSuccess) return e;
-                if ((e = cudaGetLastError()) != cudaSuccess) return e;
-            }
+            e = launch_out_ts(kp, BH * nseg, true, st, mq, mpk, mv, mw, wsS, wsZ, o, den, err);
+            if (e != cudaSuccess) return e;
             if (sio && sio->s_out) {   // the state after the sequence, this chunk's features
-                TraceScope trace_("tc_state_total", st);
-                const int64_t n = static_cast<int64_t>(BH) * Fc * 64;
-                const int grid = static_cast<int>(std::min<int64_t>((n + 255) / 256, 4 * kNumSMs));
-                k_state_total<<<grid, 256, 0, st>>>(wsS, wsZ, BH, nseg, Fc, F, c * Fc, kp.s_in ? sio->s_in : nullptr,
-                                                    kp.s_in ? sio->z_in : nullptr, sio->s_out, sio->z_out);
-                if ((e = cudaGetLastError()) != cudaSuccess) return e;
+                e = launch_state_total(wsS, wsZ, BH, nseg, Fc, F, c, kp.s_in ? sio->s_in : nullptr,
+                                       kp.s_in ? sio->z_in : nullptr, sio->s_out, sio->z_out, st);
+                if (e != cudaSuccess) return e;
             }
             continue;
         }
@@ -2221,6 +2277,66 @@ cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, 
             k_tc_causal_out<<<BH * nseg, kOutThreads, smo, st>>>(mq, mk, mv, mw, kp, wsS, wsZ, o, den, err);
         }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t tc_attn_fwd_begin(const void* k, const void* v, int B, int H, int L, const Params& P,
+                              float eps, void* ws, cudaStream_t st, float* s_out, float* z_out)
+{
+    if (!P.wB) return cudaErrorNotSupported;
+    const int BH = B * H, F = P.F, Fc = chunk_features(F), nch = F / Fc;
+    const int ntiles = (L + kTile - 1) / kTile;
+    const int nseg = choose_nseg(BH, ntiles);
+    const WsLayout wl = ws_layout(BH, L, F, nseg, true, true);
+    char* w = static_cast<char*>(ws);
+    CUtensorMap mk, mv;
+    if (!map_rows(&mk, k, L, BH) || !map_rows(&mv, v, L, BH)) return cudaErrorInvalidValue;
+    int* err = reinterpret_cast<int*>(w);
+    cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), st);
+    if (e != cudaSuccess) return e;
+    const size_t sms = smem_bytes_state(Fc);
+    if ((e = set_smem(k_tc_causal_state<true>, sms)) != cudaSuccess) return e;
+    for (int c = 0; c < nch; ++c) {
+        const ChunkParts cp = chunk_parts(w, wl, BH, L, nseg, Fc, c);
+        CUtensorMap mw, mpk;
+        if (!map_chunk_w(&mw, P, Fc, c) || !map_phik(&mpk, cp.phik, Fc, L, BH)) return cudaErrorInvalidValue;
+        const KParams kp = chunk_kparams(P, L, Fc, nch, nseg, ntiles, eps, c, w, wl, nullptr);
+        {
+            TraceScope trace_("tc_kphi_state", st);
+            k_tc_causal_state<true><<<BH * nseg, kThreads, sms, st>>>(mk, mv, mw, mpk, kp, cp.s, cp.z, err);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+        e = launch_state_total(cp.s, cp.z, BH, nseg, Fc, F, c, nullptr, nullptr, s_out, z_out, st);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t tc_attn_fwd_finish(const void* q, const void* v, void* out, float* den, int B, int H,
+                               int L, const Params& P, float eps, void* ws, cudaStream_t st,
+                               const float* s_in, const float* z_in)
+{
+    if (!P.wB) return cudaErrorNotSupported;
+    const int BH = B * H, F = P.F, Fc = chunk_features(F), nch = F / Fc;
+    const int ntiles = (L + kTile - 1) / kTile;
+    const int nseg = choose_nseg(BH, ntiles);
+    const WsLayout wl = ws_layout(BH, L, F, nseg, true, true);
+    char* w = static_cast<char*>(ws);
+    CUtensorMap mq, mv;
+    if (!map_rows(&mq, q, L, BH) || !map_rows(&mv, v, L, BH)) return cudaErrorInvalidValue;
+    int* err = reinterpret_cast<int*>(w);
+    const StateIO sio{s_in, z_in, nullptr, nullptr};
+    for (int c = 0; c < nch; ++c) {
+        const ChunkParts cp = chunk_parts(w, wl, BH, L, nseg, Fc, c);
+        CUtensorMap mw, mpk;
+        if (!map_chunk_w(&mw, P, Fc, c) || !map_phik(&mpk, cp.phik, Fc, L, BH)) return cudaErrorInvalidValue;
+        const KParams kp = chunk_kparams(P, L, Fc, nch, nseg, ntiles, eps, c, w, wl, &sio);
+        // ordinary launches: whatever runs just ahead (the exchange, the caller's kernels)
+        // may still be writing q, v or the state the prologue reads
+        cudaError_t e = launch_out_ts(kp, BH * nseg, false, st, mq, mpk, mv, mw, cp.s, cp.z,
+                                      static_cast<__nv_bfloat16*>(out), den, err);
+        if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
 }

@@ -79,6 +79,16 @@ struct StateIO {
 cudaError_t tc_attn_fwd(const void* q, const void* k, const void* v, void* out, float* den,
                         int B, int H, int L, const Params& P, float eps, bool causal, void* ws,
                         cudaStream_t st, bool lowmem = false, const StateIO* sio = nullptr);
+// The causal forward in two calls on one workspace (tc_workspace_bytes of
+// SLAY_OP_CAUSAL_FWD_SPLIT): begin runs the state kernel over every segment of every feature
+// chunk (phi(k) and the segment sums kept in the workspace) and writes the sequence's state
+// into s_out, z_out; finish runs the output kernels on them from the state s_in, z_in (null:
+// zero).  finish leaves the status word as begin set it.
+cudaError_t tc_attn_fwd_begin(const void* k, const void* v, int B, int H, int L, const Params& P,
+                              float eps, void* ws, cudaStream_t st, float* s_out, float* z_out);
+cudaError_t tc_attn_fwd_finish(const void* q, const void* v, void* out, float* den, int B, int H,
+                               int L, const Params& P, float eps, void* ws, cudaStream_t st,
+                               const float* s_in, const float* z_in);
 
 // The state of a whole sequence on tensor cores (k projections, phi(k) and per-segment sums
 // by the state kernel over every segment, then their total plus sio.s_in into sio.s_out).

@@ -3,9 +3,10 @@
 The causal contraction's prefix state carries everything earlier tokens contribute
 (review, "Proposed method", step 6), so a long sequence split into contiguous pieces, one
 per rank in rank order, needs one exchange: each rank sums its own piece's state
-(slay_causal_state: sum of phi(k) [v, 1]^T), the ranks all-gather those states (F x (Dv+1)
-fp32 per (b, h)), each rank adds up the states of the ranks before it (slay_state_prefix)
-and runs its piece's causal forward from that state (slay_attn_causal_fwd_state).  The
+(slay_attn_causal_fwd_begin: sum of phi(k) [v, 1]^T, with phi(k) and the segment sums kept
+in its workspace), the ranks all-gather those states (F x (Dv+1) fp32 per (b, h)), each rank
+adds up the states of the ranks before it (slay_state_prefix) and runs its piece's causal
+forward from that state on the kept phi(k) (slay_attn_causal_fwd_finish).  The
 backward also needs, for each piece, the sum of phi(q) [dn, delta]^T over the later ranks'
 tokens: one more all-gather of the pieces' such sums (slay_causal_bwd_state), a suffix over
 ranks (slay_state_suffix), then the piece's backward from both states
@@ -13,8 +14,9 @@ ranks (slay_state_suffix), then the piece's backward from both states
 backend works: the states are ordinary tensors); no kernel waits on another rank's memory.
 
 Every step of the path runs in the library's kernels; this module orders them and calls the
-collective.  The steps are passed in as an object (LibraryOps by default: state, prefix,
-forward, bwd_state, suffix, backward), so the same orchestration runs in tests on CPU ranks.
+collective.  The steps are passed in as an object (LibraryOps by default: begin, prefix,
+finish for the forward; state, bwd_state, suffix, backward for the backward), so the same
+orchestration runs in tests on CPU ranks.
 """
 from typing import Optional
 
@@ -30,15 +32,21 @@ class LibraryOps:
     def __init__(self, R, m, seed, eps):
         self.R, self.m, self.seed, self.eps = R, m, seed, eps
 
+    def begin(self, k, v, S_out, z_out, handle=None):
+        """The piece's state; returns the workspace that carries phi(k) to finish (handle: a
+        workspace of an earlier call on the same sizes, reused)."""
+        return bd.slay_attn_causal_fwd_begin(k, v, S_out, z_out, self.R, self.m, self.seed,
+                                             self.eps, workspace=handle)
+
+    def finish(self, q, k, v, out, den, S_in, z_in, handle):
+        bd.slay_attn_causal_fwd_finish(q, k, v, out, den, self.R, self.m, self.seed, self.eps,
+                                       handle, S_in=S_in, z_in=z_in)
+
     def state(self, k, v, S_out, z_out):
         bd.slay_causal_state(k, v, S_out, z_out, self.R, self.m, self.seed, self.eps)
 
     def prefix(self, S_all, z_all, rank, S_in, z_in):
         bd.slay_state_prefix(S_all, z_all, rank, S_in, z_in)
-
-    def forward(self, q, k, v, out, den, S_in, z_in):
-        bd.slay_attn_causal_fwd_state(q, k, v, out, den, self.R, self.m, self.seed, self.eps,
-                                      S_in=S_in, z_in=z_in)
 
     def bwd_state(self, q, out, den, dout, G_out, zg_out):
         bd.slay_causal_bwd_state(q, out, den, dout, G_out, zg_out, self.R, self.m, self.seed,
@@ -70,24 +78,26 @@ def causal_fwd_seqpar(q, k, v, out, den, F: int, ops, group=None,
     """This rank's piece [B, H, Lr, D] of a sequence split over the group in rank order:
     out (and den, if given) of the causal forward of the whole sequence at this piece's rows.
 
-    F = R * m features; ops: LibraryOps (or an object with the same three methods);
-    scratch: optional dict reused across calls for the state buffers."""
+    F = R * m features; ops: LibraryOps (or an object with its begin, prefix and finish
+    methods); scratch: optional dict reused across calls for the state buffers and the
+    workspace begin hands to finish."""
     rank = dist.get_rank(group) if dist.is_initialized() else 0
-    B, H = q.shape[0], q.shape[1]
+    B, H, Lr = q.shape[0], q.shape[1], q.shape[2]
     Dv = v.shape[-1]
     sc = scratch if scratch is not None else {}
     shape_s, shape_z = (B, H, F, Dv), (B, H, F)
-    if sc.get("shape") != (shape_s, q.device):
+    key = (shape_s, Lr, q.dtype, q.device)
+    if sc.get("shape") != key:
         sc.clear()
-        sc["shape"] = (shape_s, q.device)
+        sc["shape"] = key
         for name in ("S_loc", "S_in"):
             sc[name] = torch.empty(shape_s, dtype=torch.float32, device=q.device)
         for name in ("z_loc", "z_in"):
             sc[name] = torch.empty(shape_z, dtype=torch.float32, device=q.device)
-    ops.state(k, v, sc["S_loc"], sc["z_loc"])
+    sc["handle"] = ops.begin(k, v, sc["S_loc"], sc["z_loc"], sc.get("handle"))
     S_all, z_all = gather_states(sc["S_loc"], sc["z_loc"], group)
     ops.prefix(S_all, z_all, rank, sc["S_in"], sc["z_in"])
-    ops.forward(q, k, v, out, den, sc["S_in"], sc["z_in"])
+    ops.finish(q, k, v, out, den, sc["S_in"], sc["z_in"], sc["handle"])
     return out
 
 

@@ -112,12 +112,29 @@ def test_gpus_flag_must_match_the_launcher(monkeypatch):
 
 
 class _OracleOps:
-    """The three sequence-parallel steps computed by the fp64 oracle on CPU tensors (a
-    stand-in for the library on ranks without a GPU; the orchestration under test is the
-    package's own)."""
+    """The sequence-parallel steps computed by the fp64 oracle on CPU tensors (a stand-in
+    for the library on ranks without a GPU; the orchestration under test is the package's
+    own).  begin's handle records the piece it was made for, and finish checks it was
+    handed that handle for the same k, v (the library's workspace contract)."""
 
     def __init__(self, P):
         self.P = P
+        self.begins = 0
+
+    def begin(self, k, v, S_out, z_out, handle=None):
+        self.state(k, v, S_out, z_out)
+        self.begins += 1
+        h = handle if handle is not None else {}
+        h.update(k=k, v=v, n=self.begins)
+        return h
+
+    def finish(self, q, k, v, out, den, S_in, z_in, handle):
+        import oracle as O
+        assert handle["k"] is k and handle["v"] is v and handle["n"] == self.begins
+        o, d, _, _ = O.attn_causal_state(q.numpy(), k.numpy(), v.numpy(), self.P,
+                                         S_in.double().numpy(), z_in.double().numpy())
+        out.copy_(torch_from(o))
+        den.copy_(torch_from(d))
 
     def state(self, k, v, S_out, z_out):
         import oracle as O
@@ -128,13 +145,6 @@ class _OracleOps:
     def prefix(self, S_all, z_all, rank, S_in, z_in):
         S_in.copy_(S_all[:rank].sum(0) if rank else torch_zeros_like(S_in))
         z_in.copy_(z_all[:rank].sum(0) if rank else torch_zeros_like(z_in))
-
-    def forward(self, q, k, v, out, den, S_in, z_in):
-        import oracle as O
-        o, d, _, _ = O.attn_causal_state(q.numpy(), k.numpy(), v.numpy(), self.P,
-                                         S_in.double().numpy(), z_in.double().numpy())
-        out.copy_(torch_from(o))
-        den.copy_(torch_from(d))
 
     def bwd_state(self, q, out, den, dout, G_out, zg_out):
         import oracle as O
@@ -185,7 +195,13 @@ def _seqpar_rank(rank, world, port, outdir):
         piece = [torch.from_numpy(np.ascontiguousarray(x[:, :, a:b])).double() for x in (q, k, v)]
         out = torch.empty((1, 2, b - a, 64))
         den = torch.empty((1, 2, b - a))
-        seqpar.causal_fwd_seqpar(*piece, out, den, w.F, _OracleOps(P))
+        ops, scratch = _OracleOps(P), {}
+        seqpar.causal_fwd_seqpar(*piece, out, den, w.F, ops, scratch=scratch)
+        first, handle = out.clone(), scratch["handle"]
+        # a second step on the same scratch reuses begin's handle
+        seqpar.causal_fwd_seqpar(*piece, out, den, w.F, ops, scratch=scratch)
+        assert scratch["handle"] is handle and ops.begins == 2
+        assert torch.equal(first, out)
         np.save(os.path.join(outdir, "sp%d.npy" % rank), out.numpy())
     finally:
         dist.destroy_process_group()

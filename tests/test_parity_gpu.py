@@ -709,6 +709,87 @@ def test_sequence_pieces_emulating_ranks(dt, R, m, L, cuts):
 
 @pytest.mark.parametrize("dt,R,m,L,cuts", [("bf16", 4, 64, 1000, (300, 700)),
                                            ("bf16", 8, 64, 700, (128, 512)),
+                                           ("bf16", 4, 64, 600, (0, 600)),
+                                           ("f32", 2, 16, 300, (1, 150)),
+                                           ("bf16", 2, 16, 257, (64, 65))])
+def test_two_call_forward_emulating_ranks(dt, R, m, L, cuts):
+    # the two-call forward: every piece's begin (its state, phi(k) kept in its own
+    # workspace), the prefix over pieces, every piece's finish; the outputs against the
+    # oracle's whole-sequence forward and bit for bit against the one-call continuation on
+    # the same prefix (the same output kernel on the same phi(k) and sums)
+    w = small(dt, R, m, L, B=1, H=3, seed=27)
+    q, k, v = W.gen_qkv(w)
+    P = params(w)
+    want, wden, _, _ = O.attn_causal_state(q, k, v, P)
+    bounds = (0,) + tuple(cuts) + (L,)
+    pieces = [(a, b) for a, b in zip(bounds[:-1], bounds[1:])]
+    F, eps = w.F, _eps(w)
+    qt, kt, vt = dev(q, dt), dev(k, dt), dev(v, dt)
+
+    def piece(t, a, b):
+        return t[:, :, a:b].contiguous()
+
+    Ss, zs, wss = [], [], []
+    for a, b in pieces:
+        S = torch.full((1, 3, F, 64), float("nan"), device="cuda")
+        z = torch.full((1, 3, F), float("nan"), device="cuda")
+        wss.append(bd.slay_attn_causal_fwd_begin(piece(kt, a, b), piece(vt, a, b), S, z, R, m,
+                                                 w.sketch_seed, eps))
+        Ss.append(S)
+        zs.append(z)
+    S_all, z_all = torch.stack(Ss), torch.stack(zs)
+    outs, dens = [], []
+    for r, (a, b) in enumerate(pieces):
+        S_in = torch.empty((1, 3, F, 64), device="cuda")
+        z_in = torch.empty((1, 3, F), device="cuda")
+        bd.slay_state_prefix(S_all, z_all, r, S_in, z_in)
+        out = torch.empty((1, 3, b - a, 64), device="cuda", dtype=TDT[dt])
+        den = torch.empty((1, 3, b - a), device="cuda")
+        bd.slay_attn_causal_fwd_finish(piece(qt, a, b), piece(kt, a, b), piece(vt, a, b), out,
+                                       den, R, m, w.sketch_seed, eps, wss[r], S_in=S_in,
+                                       z_in=z_in)
+        bd.slay_kernel_status(wss[r])
+        ref = torch.empty_like(out)
+        rden = torch.empty_like(den)
+        bd.slay_attn_causal_fwd_state(piece(qt, a, b), piece(kt, a, b), piece(vt, a, b), ref,
+                                      rden, R, m, w.sketch_seed, eps, S_in=S_in, z_in=z_in)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref) and torch.equal(den, rden), (r, a, b)
+        outs.append(host(out))
+        dens.append(host(den))
+    name = "two-call %s R%d m%d L%d %s" % (dt, R, m, L, cuts)
+    _check_fwd(name, np.concatenate(outs, axis=2), np.concatenate(dens, axis=2), want, wden,
+               TOL[dt])
+    for (a, b), S, z in zip(pieces, Ss, zs):
+        if b == a:   # an empty piece: zero state
+            assert not torch.any(S) and not torch.any(z)
+            continue
+        _, _, wS, wz = O.attn_causal_state(q[:, :, a:b], k[:, :, a:b], v[:, :, a:b], P)
+        check(name + " piece S", host(S), wS, TOL[dt])
+        check(name + " piece z", host(z), wz, TOL[dt])
+
+
+def test_two_call_forward_rejects_small_workspace():
+    w = small("bf16", 4, 64, 512, B=1, H=2, seed=28)
+    q, k, v = (dev(x, "bf16") for x in W.gen_qkv(w))
+    S = torch.empty((1, 2, 256, 64), device="cuda")
+    z = torch.empty((1, 2, 256), device="cuda")
+    need = bd.slay_workspace_bytes(bd.OP_CAUSAL_FWD_SPLIT, torch.bfloat16, 1, 2, 512, 64, 64, 4, 64)
+    # the two-call workspace keeps phi(k): larger than the one-call forward's
+    assert need >= bd.slay_workspace_bytes(bd.OP_CAUSAL_FWD, torch.bfloat16, 1, 2, 512, 64, 64,
+                                           4, 64)
+    small_ws = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(bd.SlayError):
+        bd.slay_attn_causal_fwd_begin(k, v, S, z, 4, 64, w.sketch_seed, _eps(w), workspace=small_ws)
+    out = torch.empty((1, 2, 512, 64), device="cuda", dtype=torch.bfloat16)
+    with pytest.raises(bd.SlayError):
+        bd.slay_attn_causal_fwd_finish(q, k, v, out, None, 4, 64, w.sketch_seed, _eps(w), small_ws)
+    with pytest.raises(bd.SlayError):   # the state outputs are required
+        bd.slay_attn_causal_fwd_begin(k, v, None, None, 4, 64, w.sketch_seed, _eps(w))
+
+
+@pytest.mark.parametrize("dt,R,m,L,cuts", [("bf16", 4, 64, 1000, (300, 700)),
+                                           ("bf16", 8, 64, 700, (128, 512)),
                                            ("f32", 2, 16, 300, (1, 150)),
                                            ("bf16", 2, 16, 257, (64, 65))])
 def test_sequence_pieces_backward_emulating_ranks(dt, R, m, L, cuts):
