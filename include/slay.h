@@ -83,7 +83,8 @@ typedef enum {
     SLAY_OP_BIDIR_BWD = 5,
     SLAY_OP_LINEAR_ATTN = 6,    /* slay_linear_attn_fwd: R * m = the number of features */
     SLAY_OP_CAUSAL_STATE = 7,   /* slay_causal_state */
-    SLAY_OP_CAUSAL_FWD_SPLIT = 8 /* slay_attn_causal_fwd_begin / _finish (one workspace) */
+    SLAY_OP_CAUSAL_FWD_SPLIT = 8, /* slay_attn_causal_fwd_begin / _finish (one workspace) */
+    SLAY_OP_FEATURE_MAP_BWD = 9  /* slay_feature_map_bwd (no workspace; for slay_path) */
 } slay_op;
 
 /* Feature-map variants (slay_feature_map_ex).  The pages leave the form of the anchor
@@ -392,6 +393,20 @@ slay_status slay_debug_expire_wait(int on);
  * sizes are unsupported).  Feature map, its backward and decode need none. */
 size_t slay_workspace_bytes(slay_op op, slay_dtype dt, int B, int H, int L, int D, int Dv,
                             int R, int m);
+
+/* Which kernels a call takes at these sizes.  The call decides from its sizes and dtype alone,
+ * by the same rule as this query, and never tells the caller: this is how to find out.
+ * Returns a mask of slay_path_bit values (0: every step on the CUDA-core kernels), or -1 for
+ * an op, size or dtype the call rejects.  Feature map and its backward: the rows are B*H*L
+ * (pass B = H = 1, L = n_rows) and dt is the input and output dtype.  SLAY_OP_LINEAR_ATTN:
+ * R*m is the number of features.  Host-only; enqueues nothing. */
+typedef enum {
+    SLAY_PATH_TC_FEATURE_MAP = 1,   /* phi of q and k (or x) by the tcgen05 projection */
+    SLAY_PATH_TC_CONTRACTION = 2,   /* forward: state and output kernels; backward: the
+                                       running sums and the contraction */
+    SLAY_PATH_TC_PHI_BWD = 4        /* the chain rule through phi */
+} slay_path_bit;
+int slay_path(slay_op op, slay_dtype dt, int B, int H, int L, int D, int Dv, int R, int m);
 
 /* Create (if absent) the device copy of the sketch parameters of this key on the
  * current device: synchronous; lets a caller warm the cache before stream capture. */

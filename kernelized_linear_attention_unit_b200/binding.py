@@ -18,7 +18,8 @@ SLAY_OK, SLAY_ERR_INVALID_ARG, SLAY_ERR_UNSUPPORTED, SLAY_ERR_CUDA, SLAY_ERR_TIM
     SLAY_ERR_NO_MEMORY = range(6)
 SLAY_F32, SLAY_BF16 = 0, 1
 OP_FEATURE_MAP, OP_CAUSAL_FWD, OP_BIDIR_FWD, OP_CAUSAL_BWD, OP_DECODE, OP_BIDIR_BWD, \
-    OP_LINEAR_ATTN, OP_CAUSAL_STATE, OP_CAUSAL_FWD_SPLIT = range(9)
+    OP_LINEAR_ATTN, OP_CAUSAL_STATE, OP_CAUSAL_FWD_SPLIT, OP_FEATURE_MAP_BWD = range(10)
+PATH_TC_FEATURE_MAP, PATH_TC_CONTRACTION, PATH_TC_PHI_BWD = 1, 2, 4
 PHI_ANCHOR, PHI_ORTHOGONAL, PHI_SIGNED, PHI_PER_HEAD, PHI_PERFORMER = range(5)
 
 EXPORTS = ["slay_feature_map", "slay_attn_causal_fwd", "slay_attn_bidir_fwd",
@@ -29,7 +30,7 @@ EXPORTS = ["slay_feature_map", "slay_attn_causal_fwd", "slay_attn_bidir_fwd",
            "slay_feature_map_ex", "slay_sketch_params_ex", "slay_linear_attn_fwd",
            "slay_attn_causal_fwd_state", "slay_causal_state", "slay_state_prefix",
            "slay_state_suffix", "slay_attn_causal_bwd_state", "slay_causal_bwd_state",
-           "slay_attn_causal_fwd_begin", "slay_attn_causal_fwd_finish"]
+           "slay_attn_causal_fwd_begin", "slay_attn_causal_fwd_finish", "slay_path"]
 
 
 class SlayError(RuntimeError):
@@ -84,6 +85,8 @@ def lib():
                                    u64, f32, vp]
     L.slay_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32]
     L.slay_workspace_bytes.restype = sz
+    L.slay_path.argtypes = [i32] * 9
+    L.slay_path.restype = i32
     L.slay_prepare.argtypes = [i32, i32, i32, u64, f32]
     L.slay_sketch_params.argtypes = [i32, i32, i32, u64, f32, vp, vp, vp, vp]
     L.slay_status_string.argtypes = [i32]
@@ -153,6 +156,16 @@ def slay_workspace_bytes(op, dtype, B, H, L, D, Dv, R, m) -> int:
     if n == C.c_size_t(-1).value:
         raise SlayError(SLAY_ERR_UNSUPPORTED, "slay_workspace_bytes")
     return int(n)
+
+
+def slay_path(op, dtype, B, H, L, D, Dv, R, m) -> int:
+    """Mask of PATH_* bits: which steps of `op` run on tensor cores at these sizes (0: all
+    on CUDA cores); raises for sizes the op rejects."""
+    dt = dtype if isinstance(dtype, int) else _dt(torch.empty(0, dtype=dtype))
+    n = lib().slay_path(op, dt, B, H, L, D, Dv, R, m)
+    if n < 0:
+        raise SlayError(SLAY_ERR_UNSUPPORTED, "slay_path")
+    return n
 
 
 def alloc_workspace(op, dtype, B, H, L, D, Dv, R, m, device=None):

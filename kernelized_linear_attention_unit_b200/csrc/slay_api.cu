@@ -758,7 +758,8 @@ size_t slay_workspace_bytes(slay_op op, slay_dtype dt, int B, int H, int L, int 
 {
     if (B < 0 || H < 0 || L < 0 || !dtype_ok(dt)) return SIZE_MAX;
     if (check_shape(D, Dv, R, m) != SLAY_OK) return SIZE_MAX;
-    if (op == SLAY_OP_FEATURE_MAP || op == SLAY_OP_DECODE) return 0;
+    if (op == SLAY_OP_FEATURE_MAP || op == SLAY_OP_DECODE || op == SLAY_OP_FEATURE_MAP_BWD)
+        return 0;
     if (op != SLAY_OP_CAUSAL_FWD && op != SLAY_OP_BIDIR_FWD && op != SLAY_OP_CAUSAL_BWD &&
         op != SLAY_OP_BIDIR_BWD && op != SLAY_OP_LINEAR_ATTN && op != SLAY_OP_CAUSAL_STATE &&
         op != SLAY_OP_CAUSAL_FWD_SPLIT)
@@ -769,6 +770,50 @@ size_t slay_workspace_bytes(slay_op op, slay_dtype dt, int B, int H, int L, int 
     }
     if (static_cast<int64_t>(B) * H * L == 0) return 0;
     return attn_ws(op, dt, B, H, L, Dv, R, m);
+}
+
+int slay_path(slay_op op, slay_dtype dt, int B, int H, int L, int D, int Dv, int R, int m)
+{
+    if (B < 0 || H < 0 || L < 0 || !dtype_ok(dt)) return -1;
+    if (op == SLAY_OP_LINEAR_ATTN) {   // R * m features given; the chunk kernels on CUDA cores
+        if (R <= 0 || m <= 0 || Dv != kD || static_cast<int64_t>(R) * m > kMaxF) return -1;
+        return 0;
+    }
+    if (check_shape(D, Dv, R, m) != SLAY_OK) return -1;
+    const bool bf = dt == SLAY_BF16;
+    const bool wb = tc_wb_elems(D, R, m) > 0;   // the packed projection operand exists
+    const int64_t rows = static_cast<int64_t>(B) * H * L;
+    const int fwd = SLAY_PATH_TC_FEATURE_MAP | SLAY_PATH_TC_CONTRACTION;
+    switch (op) {
+    case SLAY_OP_FEATURE_MAP:   // slay_feature_map: bf16 -> bf16 on tensor cores
+        return bf && wb && tc_fmap_supported(D, R, m, rows) ? SLAY_PATH_TC_FEATURE_MAP : 0;
+    case SLAY_OP_FEATURE_MAP_BWD:
+        return bf && wb && tc_phi_bwd_supported(D, R, m, rows) ? SLAY_PATH_TC_PHI_BWD : 0;
+    case SLAY_OP_CAUSAL_FWD:
+    case SLAY_OP_CAUSAL_STATE:
+    case SLAY_OP_CAUSAL_FWD_SPLIT:   // phi inside the state and output kernels
+        return bf && tc_supported(SLAY_OP_CAUSAL_FWD, B, H, L, R, m) ? fwd : 0;
+    case SLAY_OP_BIDIR_FWD:
+        return bf && tc_supported(SLAY_OP_BIDIR_FWD, B, H, L, R, m) ? fwd : 0;
+    case SLAY_OP_CAUSAL_BWD:
+    case SLAY_OP_BIDIR_BWD: {
+        // the rule of the backward: phi maps, the tile contraction and the chain rule through
+        // phi each on tensor cores where their sizes allow; bf16 dphi (which the tensor-core
+        // chain rule reads) comes from the tile contraction, or the bidirectional chunk kernel
+        if (!bf || rows == 0) return 0;
+        const bool tcb = tc_bwd_tile_supported(R * m, L);
+        const bool tcp = wb && tc_phi_bwd_supported(D, R, m, rows);
+        int mask = 0;
+        if (wb && tc_fmap_supported(D, R, m, rows)) mask |= SLAY_PATH_TC_FEATURE_MAP;
+        if (tcb) mask |= SLAY_PATH_TC_CONTRACTION;
+        if ((tcb || op == SLAY_OP_BIDIR_BWD) && tcp) mask |= SLAY_PATH_TC_PHI_BWD;
+        return mask;
+    }
+    case SLAY_OP_DECODE:
+        return 0;
+    default:
+        return -1;
+    }
 }
 
 slay_status slay_prepare(int D, int R, int m, uint64_t seed, float eps)

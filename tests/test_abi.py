@@ -73,6 +73,44 @@ def test_workspace_bytes():
         f(bd.OP_CAUSAL_FWD, bd.SLAY_F32, 1, 1, 16, 32, 64, 4, 64)
 
 
+@pytest.mark.parametrize("op,dt,B,H,L,R,m,want", [
+    ("CAUSAL_FWD", "BF16", 1, 16, 16384, 4, 64, 3),       # the headline: tensor cores
+    ("CAUSAL_FWD", "F32", 1, 16, 16384, 4, 64, 0),        # fp32: CUDA cores
+    ("CAUSAL_FWD", "BF16", 1, 2, 100, 4, 32, 0),          # m % 64 != 0
+    ("CAUSAL_FWD", "BF16", 2, 16, 8192, 8, 64, 3),        # F = 512 in two chunks
+    ("CAUSAL_FWD", "BF16", 1, 2, 100, 16, 64, 0),         # F = 1024 > 512
+    ("CAUSAL_FWD", "BF16", 0, 2, 100, 4, 64, 0),          # empty
+    ("CAUSAL_STATE", "BF16", 1, 2, 100, 4, 64, 3),
+    ("CAUSAL_FWD_SPLIT", "BF16", 1, 2, 100, 4, 64, 3),
+    ("BIDIR_FWD", "BF16", 32, 12, 1024, 4, 64, 3),
+    ("FEATURE_MAP", "BF16", 1, 1, 1000, 4, 32, 1),        # the map takes m % 32 == 0
+    ("FEATURE_MAP", "F32", 1, 1, 1000, 4, 32, 0),
+    ("FEATURE_MAP", "BF16", 1, 1, 1000, 3, 64, 0),        # F % 128 != 0
+    ("FEATURE_MAP_BWD", "BF16", 1, 1, 1000, 4, 32, 4),
+    ("CAUSAL_BWD", "BF16", 2, 16, 8192, 8, 64, 7),
+    ("CAUSAL_BWD", "BF16", 1, 2, 100, 2, 64, 7),
+    ("CAUSAL_BWD", "BF16", 1, 2, 100, 3, 64, 0),          # F = 192
+    ("CAUSAL_BWD", "BF16", 1, 2, 100, 10, 64, 0),         # F = 640
+    ("CAUSAL_BWD", "F32", 1, 2, 100, 2, 64, 0),
+    ("BIDIR_BWD", "BF16", 32, 12, 1024, 4, 64, 7),
+    ("DECODE", "BF16", 256, 16, 1, 8, 64, 0),
+    ("LINEAR_ATTN", "BF16", 1, 2, 100, 1, 256, 0),
+])
+def test_path_query(op, dt, B, H, L, R, m, want):
+    # the size rules the header states for the tensor-core kernels; host only
+    got = bd.slay_path(getattr(bd, "OP_" + op), getattr(bd, "SLAY_" + dt), B, H, L, 64, 64, R, m)
+    assert got == want
+
+
+def test_path_query_rejects():
+    with pytest.raises(bd.SlayError):
+        bd.slay_path(bd.OP_CAUSAL_FWD, bd.SLAY_BF16, 1, 1, 16, 32, 64, 4, 64)   # D != 64
+    with pytest.raises(bd.SlayError):
+        bd.slay_path(99, bd.SLAY_BF16, 1, 1, 16, 64, 64, 4, 64)
+    with pytest.raises(bd.SlayError):
+        bd.slay_path(bd.OP_CAUSAL_FWD, 7, 1, 1, 16, 64, 64, 4, 64)
+
+
 def _fake(addr=0x10000):
     return C.c_void_p(addr)
 
