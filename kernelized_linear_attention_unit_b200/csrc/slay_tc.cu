@@ -2037,27 +2037,44 @@ cudaError_t set_smem(K kernel, size_t bytes)
 
 // The state after the whole sequence for one feature chunk: S_out[bh][c0 + f][e] = S_in +
 // sum over the nseg per-segment sums (every segment's sum is in the workspace when the state
-// kernel ran over all of them), z likewise.  One thread per (bh, f, e) or (bh, f).
+// kernel ran over all of them), z likewise, added in segment order.  One thread per four
+// consecutive (f, e) with 16-byte loads and stores, four segments' loads in flight before
+// their adds; the thread of e = 0..3 also sums z of its f.
 __global__ void k_state_total(const float* __restrict__ wsS, const float* __restrict__ wsZ, int BH,
                               int nseg, int Fc, int Ftot, int c0, const float* __restrict__ s_in,
                               const float* __restrict__ z_in, float* __restrict__ s_out,
                               float* __restrict__ z_out)
 {
-    const int64_t n = static_cast<int64_t>(BH) * Fc * 64;
+    const int64_t q4 = static_cast<int64_t>(Fc) * 16;   // float4s of one sequence's chunk sum
+    const int64_t n = static_cast<int64_t>(BH) * q4;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int bh = static_cast<int>(i / (static_cast<int64_t>(Fc) * 64));
-        const int fe = static_cast<int>(i % (static_cast<int64_t>(Fc) * 64));
-        const size_t dst = static_cast<size_t>(bh) * Ftot * 64 + static_cast<size_t>(c0) * 64 + fe;
-        float acc = s_in ? s_in[dst] : 0.0f;
-        for (int sgi = 0; sgi < nseg; ++sgi)
-            acc += wsS[(static_cast<size_t>(bh) * nseg + sgi) * Fc * 64 + fe];
-        s_out[dst] = acc;
-        if ((fe & 63) == 0) {
-            const int f = fe >> 6;
-            const size_t dz = static_cast<size_t>(bh) * Ftot + c0 + f;
+        const int bh = static_cast<int>(i / q4);
+        const int j = static_cast<int>(i % q4);   // f = j / 16, e = 4 (j % 16) .. + 3
+        const float4* src = reinterpret_cast<const float4*>(wsS) + static_cast<int64_t>(bh) * nseg * q4 + j;
+        const int64_t dst = (static_cast<int64_t>(bh) * Ftot + c0) * 16 + j;
+        float4 a = s_in ? reinterpret_cast<const float4*>(s_in)[dst] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        int sg = 0;
+        for (; sg + 4 <= nseg; sg += 4) {
+            float4 x[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) x[u] = src[(sg + u) * q4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                a.x += x[u].x; a.y += x[u].y; a.z += x[u].z; a.w += x[u].w;
+            }
+        }
+        for (; sg < nseg; ++sg) {
+            const float4 x = src[sg * q4];
+            a.x += x.x; a.y += x.y; a.z += x.z; a.w += x.w;
+        }
+        reinterpret_cast<float4*>(s_out)[dst] = a;
+        if ((j & 15) == 0) {
+            const int f = j >> 4;
+            const int64_t dz = static_cast<int64_t>(bh) * Ftot + c0 + f;
+            const float* zs = wsZ + static_cast<int64_t>(bh) * nseg * Fc + f;
             float az = z_in ? z_in[dz] : 0.0f;
-            for (int sgi = 0; sgi < nseg; ++sgi) az += wsZ[(static_cast<size_t>(bh) * nseg + sgi) * Fc + f];
+            for (int t = 0; t < nseg; ++t) az += zs[static_cast<int64_t>(t) * Fc];
             z_out[dz] = az;
         }
     }
@@ -2133,8 +2150,8 @@ cudaError_t launch_state_total(const float* wsS, const float* wsZ, int BH, int n
                                float* z_out, cudaStream_t st)
 {
     TraceScope trace_("tc_state_total", st);
-    const int64_t n = static_cast<int64_t>(BH) * Fc * 64;
-    const int grid = static_cast<int>(std::min<int64_t>((n + 255) / 256, 4 * kNumSMs));
+    const int64_t n = static_cast<int64_t>(BH) * Fc * 16;   // one thread per float4
+    const int grid = static_cast<int>(std::min<int64_t>((n + 255) / 256, 8 * kNumSMs));
     k_state_total<<<grid, 256, 0, st>>>(wsS, wsZ, BH, nseg, Fc, F, c * Fc, s_in, z_in, s_out, z_out);
     return cudaGetLastError();
 }
