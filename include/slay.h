@@ -259,6 +259,32 @@ slay_status slay_causal_bwd_state(const void* q, const void* out, const float* d
                                   int L, int D, int Dv, slay_dtype dt, int R, int m, uint64_t seed,
                                   float eps, void* workspace, size_t ws_bytes, void* stream);
 
+/* The sequence-parallel backward of one piece in two calls that share a workspace, so that
+ * phi(q) and the row statistics dn, delta (as in slay_attn_causal_bwd_state) are made once,
+ * for the exchange and the backward alike.  Between the calls the caller
+ * exchanges the G sums and forms the suffix (slay_state_suffix).
+ * slay_attn_causal_bwd_begin: as slay_causal_bwd_state (same arguments, G_out and zg_out
+ *   written), and it leaves phi(q) and the row statistics in `workspace`.
+ * slay_attn_causal_bwd_finish: the gradients slay_attn_causal_bwd_state writes for the same
+ *   arguments (same values), without recomputing phi(q) and the row statistics.  It must come
+ *   after the first call in stream order, with the same q, out, den, dout, B, H, L, D, Dv, dt,
+ *   R, m, seed, eps and workspace, nothing else writing the workspace in between.  It leaves
+ *   the status word as the first call set it.
+ * workspace: slay_workspace_bytes(SLAY_OP_CAUSAL_BWD, ...) bytes, caller-owned, its contents
+ * the library's from the first call to the second.  Errors as slay_attn_causal_bwd_state. */
+slay_status slay_attn_causal_bwd_begin(const void* q, const void* out, const float* den,
+                                       const void* dout, float* G_out, float* zg_out, int B, int H,
+                                       int L, int D, int Dv, slay_dtype dt, int R, int m,
+                                       uint64_t seed, float eps, void* workspace, size_t ws_bytes,
+                                       void* stream);
+slay_status slay_attn_causal_bwd_finish(const void* q, const void* k, const void* v,
+                                        const void* out, const float* den, const void* dout,
+                                        float* dq, float* dk, float* dv, const float* S_in,
+                                        const float* z_in, const float* G_in, const float* zg_in,
+                                        int B, int H, int L, int D, int Dv, slay_dtype dt, int R,
+                                        int m, uint64_t seed, float eps, void* workspace,
+                                        size_t ws_bytes, void* stream);
+
 /* Backward of the bidirectional forward: gradients of sum_i <dout_i, out_i> with respect
  * to q, k, v (the pages give no backward; it is the derivative of slay_attn_bidir_fwd).
  * With Z_i = den_i + eps, dn_i = dout_i / Z_i, delta_i = -<dout_i, out_i> / Z_i and the
@@ -401,7 +427,9 @@ size_t slay_workspace_bytes(slay_op op, slay_dtype dt, int B, int H, int L, int 
  * (pass B = H = 1, L = n_rows) and dt is the input and output dtype.  SLAY_OP_LINEAR_ATTN:
  * R*m is the number of features.  Host-only; enqueues nothing. */
 typedef enum {
-    SLAY_PATH_TC_FEATURE_MAP = 1,   /* phi of q and k (or x) by the tcgen05 projection */
+    SLAY_PATH_TC_FEATURE_MAP = 1,   /* phi of q and k (or x) by the tcgen05 projection: in
+                                       the fused forward kernels, or the feature-map kernel
+                                       ahead of CUDA-core contraction kernels */
     SLAY_PATH_TC_CONTRACTION = 2,   /* forward: state and output kernels; backward: the
                                        running sums and the contraction */
     SLAY_PATH_TC_PHI_BWD = 4        /* the chain rule through phi */

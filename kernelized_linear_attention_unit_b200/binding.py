@@ -30,7 +30,8 @@ EXPORTS = ["slay_feature_map", "slay_attn_causal_fwd", "slay_attn_bidir_fwd",
            "slay_feature_map_ex", "slay_sketch_params_ex", "slay_linear_attn_fwd",
            "slay_attn_causal_fwd_state", "slay_causal_state", "slay_state_prefix",
            "slay_state_suffix", "slay_attn_causal_bwd_state", "slay_causal_bwd_state",
-           "slay_attn_causal_fwd_begin", "slay_attn_causal_fwd_finish", "slay_path"]
+           "slay_attn_causal_fwd_begin", "slay_attn_causal_fwd_finish", "slay_path",
+           "slay_attn_causal_bwd_begin", "slay_attn_causal_bwd_finish"]
 
 
 class SlayError(RuntimeError):
@@ -81,6 +82,8 @@ def lib():
     L.slay_state_suffix.argtypes = L.slay_state_prefix.argtypes
     L.slay_attn_causal_bwd_state.argtypes = [vp] * 13 + [i32] * 8 + [u64, f32, vp, sz, vp]
     L.slay_causal_bwd_state.argtypes = [vp] * 6 + [i32] * 8 + [u64, f32, vp, sz, vp]
+    L.slay_attn_causal_bwd_begin.argtypes = L.slay_causal_bwd_state.argtypes
+    L.slay_attn_causal_bwd_finish.argtypes = L.slay_attn_causal_bwd_state.argtypes
     L.slay_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                    u64, f32, vp]
     L.slay_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32]
@@ -108,7 +111,8 @@ def lib():
                  "slay_causal_state", "slay_state_prefix", "slay_state_suffix",
                  "slay_attn_causal_bwd_state", "slay_causal_bwd_state",
                  "slay_attn_causal_fwd_noalloc", "slay_attn_causal_fwd_begin",
-                 "slay_attn_causal_fwd_finish",
+                 "slay_attn_causal_fwd_finish", "slay_attn_causal_bwd_begin",
+                 "slay_attn_causal_bwd_finish",
                  "slay_sketch_params"):
         getattr(L, name).restype = i32
     _lib = L
@@ -478,6 +482,21 @@ def slay_attn_causal_bwd_state(q, k, v, out, den, dout, dq, dk, dv, R, m, seed, 
     """Backward of one piece of a causal sequence: S_in, z_in [B,H,F,64], [B,H,F] sum
     phi(k)[v, 1] over the tokens before it, G_in, zg_in sum phi(q)[dn, delta] over the tokens
     after it (None: zero); returns the workspace it used."""
+    return _bwd_piece(lib().slay_attn_causal_bwd_state, "slay_attn_causal_bwd_state", q, k, v,
+                      out, den, dout, dq, dk, dv, R, m, seed, eps, S_in, z_in, G_in, zg_in,
+                      workspace, stream)
+
+
+def slay_attn_causal_bwd_finish(q, k, v, out, den, dout, dq, dk, dv, R, m, seed, eps, workspace,
+                                S_in=None, z_in=None, G_in=None, zg_in=None, stream=None):
+    """Second call of the two-call backward: the gradients of slay_attn_causal_bwd_state on
+    the workspace of slay_attn_causal_bwd_begin for the same q, out, den, dout."""
+    _bwd_piece(lib().slay_attn_causal_bwd_finish, "slay_attn_causal_bwd_finish", q, k, v, out,
+               den, dout, dq, dk, dv, R, m, seed, eps, S_in, z_in, G_in, zg_in, workspace, stream)
+
+
+def _bwd_piece(fn, name, q, k, v, out, den, dout, dq, dk, dv, R, m, seed, eps, S_in, z_in, G_in,
+               zg_in, workspace, stream):
     _check(q, "q")
     B, H, L, D = q.shape
     Dv = v.shape[-1]
@@ -496,17 +515,28 @@ def slay_attn_causal_bwd_state(q, k, v, out, den, dout, dq, dk, dv, R, m, seed, 
     if workspace is None:
         workspace = alloc_workspace(OP_CAUSAL_BWD, dt, B, H, L, D, Dv, R, m, q.device)
     wbytes = workspace.numel() * workspace.element_size()
-    _raise(lib().slay_attn_causal_bwd_state(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(den),
-                                            _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), si, zi, gi,
-                                            zgi, B, H, L, D, Dv, dt, R, m, seed, eps,
-                                            _ptr(workspace), wbytes, _stream(stream)),
-           "slay_attn_causal_bwd_state")
+    _raise(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(den), _ptr(dout), _ptr(dq), _ptr(dk),
+              _ptr(dv), si, zi, gi, zgi, B, H, L, D, Dv, dt, R, m, seed, eps, _ptr(workspace),
+              wbytes, _stream(stream)), name)
     return workspace
 
 
 def slay_causal_bwd_state(q, out, den, dout, G_out, zg_out, R, m, seed, eps, workspace=None,
                           stream=None):
     """G_out = sum phi(q) dn^T, zg_out = sum phi(q) delta over the tokens of a piece."""
+    return _g_state(lib().slay_causal_bwd_state, "slay_causal_bwd_state", q, out, den, dout,
+                    G_out, zg_out, R, m, seed, eps, workspace, stream)
+
+
+def slay_attn_causal_bwd_begin(q, out, den, dout, G_out, zg_out, R, m, seed, eps, workspace=None,
+                               stream=None):
+    """First call of the two-call backward: as slay_causal_bwd_state; the workspace it returns
+    (or the one given) carries phi(q) and the row statistics to slay_attn_causal_bwd_finish."""
+    return _g_state(lib().slay_attn_causal_bwd_begin, "slay_attn_causal_bwd_begin", q, out, den,
+                    dout, G_out, zg_out, R, m, seed, eps, workspace, stream)
+
+
+def _g_state(fn, name, q, out, den, dout, G_out, zg_out, R, m, seed, eps, workspace, stream):
     _check(q, "q")
     B, H, L, D = q.shape
     Dv = out.shape[-1]
@@ -519,9 +549,8 @@ def slay_causal_bwd_state(q, out, den, dout, G_out, zg_out, R, m, seed, eps, wor
     if workspace is None:
         workspace = alloc_workspace(OP_CAUSAL_BWD, dt, B, H, L, D, Dv, R, m, q.device)
     wbytes = workspace.numel() * workspace.element_size()
-    _raise(lib().slay_causal_bwd_state(_ptr(q), _ptr(out), _ptr(den), _ptr(dout), go, zgo, B, H,
-                                       L, D, Dv, dt, R, m, seed, eps, _ptr(workspace), wbytes,
-                                       _stream(stream)), "slay_causal_bwd_state")
+    _raise(fn(_ptr(q), _ptr(out), _ptr(den), _ptr(dout), go, zgo, B, H, L, D, Dv, dt, R, m, seed,
+              eps, _ptr(workspace), wbytes, _stream(stream)), name)
     return workspace
 
 

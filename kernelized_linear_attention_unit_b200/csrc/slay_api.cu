@@ -356,7 +356,8 @@ slay_status attn_bwd(const void* q, const void* k, const void* v, const void* ou
     Params P;
     if ((s = get_params(D, R, m, seed, eps, &P)) != SLAY_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
+    // the second call of the two-call backward keeps the status word the first one cleared
+    cudaError_t e = (sio && sio->q_ready) ? cudaSuccess : cudaMemsetAsync(workspace, 0, sizeof(int), st);
     char* w = static_cast<char*>(workspace) + kWsHeader;
     if (e == cudaSuccess)
         e = sio ? simt_attn_causal_bwd_state(q, k, v, out, den, dout, dq, dk, dv, B, H, L, dt, P,
@@ -683,6 +684,34 @@ slay_status slay_causal_bwd_state(const void* q, const void* out, const float* d
     return e == cudaSuccess ? SLAY_OK : cuda_fail(e);
 }
 
+slay_status slay_attn_causal_bwd_begin(const void* q, const void* out, const float* den,
+                                       const void* dout, float* G_out, float* zg_out, int B, int H,
+                                       int L, int D, int Dv, slay_dtype dt, int R, int m,
+                                       uint64_t seed, float eps, void* workspace, size_t ws_bytes,
+                                       void* stream)
+{
+    // slay_causal_bwd_state leaves phi(q) and the row statistics where the backward reads them
+    return slay_causal_bwd_state(q, out, den, dout, G_out, zg_out, B, H, L, D, Dv, dt, R, m, seed,
+                                 eps, workspace, ws_bytes, stream);
+}
+
+slay_status slay_attn_causal_bwd_finish(const void* q, const void* k, const void* v,
+                                        const void* out, const float* den, const void* dout,
+                                        float* dq, float* dk, float* dv, const float* S_in,
+                                        const float* z_in, const float* G_in, const float* zg_in,
+                                        int B, int H, int L, int D, int Dv, slay_dtype dt, int R,
+                                        int m, uint64_t seed, float eps, void* workspace,
+                                        size_t ws_bytes, void* stream)
+{
+    slay_status s = check_state_ptrs(S_in, z_in);
+    if (s != SLAY_OK) return s;
+    if ((s = check_state_ptrs(G_in, zg_in)) != SLAY_OK) return s;
+    BwdStateIO sio{S_in, z_in, G_in, zg_in};
+    sio.q_ready = true;
+    return attn_bwd(q, k, v, out, den, dout, dq, dk, dv, B, H, L, D, Dv, dt, R, m, seed, eps,
+                    workspace, ws_bytes, stream, true, &sio);
+}
+
 slay_status slay_feature_map_bwd(const void* x, const void* dphi, float* dx, int64_t n_rows,
                                  int D, slay_dtype x_dt, slay_dtype dphi_dt, int R, int m,
                                  uint64_t seed, float eps, void* stream)
@@ -784,17 +813,19 @@ int slay_path(slay_op op, slay_dtype dt, int B, int H, int L, int D, int Dv, int
     const bool wb = tc_wb_elems(D, R, m) > 0;   // the packed projection operand exists
     const int64_t rows = static_cast<int64_t>(B) * H * L;
     const int fwd = SLAY_PATH_TC_FEATURE_MAP | SLAY_PATH_TC_CONTRACTION;
+    // the tensor-core feature map, also ahead of the CUDA-core contraction kernels in bf16
+    const int fm = bf && wb && tc_fmap_supported(D, R, m, rows) ? SLAY_PATH_TC_FEATURE_MAP : 0;
     switch (op) {
     case SLAY_OP_FEATURE_MAP:   // slay_feature_map: bf16 -> bf16 on tensor cores
-        return bf && wb && tc_fmap_supported(D, R, m, rows) ? SLAY_PATH_TC_FEATURE_MAP : 0;
+        return fm;
     case SLAY_OP_FEATURE_MAP_BWD:
         return bf && wb && tc_phi_bwd_supported(D, R, m, rows) ? SLAY_PATH_TC_PHI_BWD : 0;
     case SLAY_OP_CAUSAL_FWD:
     case SLAY_OP_CAUSAL_STATE:
-    case SLAY_OP_CAUSAL_FWD_SPLIT:   // phi inside the state and output kernels
-        return bf && tc_supported(SLAY_OP_CAUSAL_FWD, B, H, L, R, m) ? fwd : 0;
+    case SLAY_OP_CAUSAL_FWD_SPLIT:   // phi inside the fused state and output kernels
+        return bf && tc_supported(SLAY_OP_CAUSAL_FWD, B, H, L, R, m) ? fwd : fm;
     case SLAY_OP_BIDIR_FWD:
-        return bf && tc_supported(SLAY_OP_BIDIR_FWD, B, H, L, R, m) ? fwd : 0;
+        return bf && tc_supported(SLAY_OP_BIDIR_FWD, B, H, L, R, m) ? fwd : fm;
     case SLAY_OP_CAUSAL_BWD:
     case SLAY_OP_BIDIR_BWD: {
         // the rule of the backward: phi maps, the tile contraction and the chain rule through
@@ -803,8 +834,7 @@ int slay_path(slay_op op, slay_dtype dt, int B, int H, int L, int D, int Dv, int
         if (!bf || rows == 0) return 0;
         const bool tcb = tc_bwd_tile_supported(R * m, L);
         const bool tcp = wb && tc_phi_bwd_supported(D, R, m, rows);
-        int mask = 0;
-        if (wb && tc_fmap_supported(D, R, m, rows)) mask |= SLAY_PATH_TC_FEATURE_MAP;
+        int mask = fm;
         if (tcb) mask |= SLAY_PATH_TC_CONTRACTION;
         if ((tcb || op == SLAY_OP_BIDIR_BWD) && tcp) mask |= SLAY_PATH_TC_PHI_BWD;
         return mask;

@@ -110,6 +110,9 @@ struct BwdStateIO {
     const float* z_in;
     const float* g_in;
     const float* zg_in;
+    // phi(q) and the row statistics of these q, out, den, dout are already in the workspace
+    // (simt_causal_bwd_state on the same workspace left them there): not recomputed
+    bool q_ready = false;
 };
 cudaError_t simt_attn_causal_bwd_state(const void* q, const void* k, const void* v,
                                        const void* out, const float* den, const void* dout,

@@ -1270,7 +1270,10 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
     float* gbw = reinterpret_cast<float*>(w + 4 * phb + stb);
     float* dn = reinterpret_cast<float*>(w + 4 * phb + 2 * stb);
     cudaError_t err;
-    if ((err = phi_map<T>(q, phq, rows, P, st)) != cudaSuccess) return err;
+    // phi(q) and the row statistics may be in the workspace already (the first call of the
+    // two-call backward computed them at the same places)
+    const bool q_ready = sio && sio->q_ready;
+    if (!q_ready && (err = phi_map<T>(q, phq, rows, P, st)) != cudaSuccess) return err;
     if ((err = phi_map<T>(k, phk, rows, P, st)) != cudaSuccess) return err;
     // bf16 phi: states, contraction on tensor cores over 128-token tiles; else 64-token chunks
     // (the bidirectional form: the same kernels with whole-sequence sums and no masked term)
@@ -1278,7 +1281,7 @@ static cudaError_t attn_bwd_t(const void* q, const void* k, const void* v, const
     // tensor-core path: dn as bf16 rows and delta in the dn region (132 of its 260 bytes a row)
     __nv_bfloat16* dn16 = reinterpret_cast<__nv_bfloat16*>(dn);
     float* delta = reinterpret_cast<float*>(dn16 + rows * kD);
-    {
+    if (!q_ready) {
         TraceScope trace_("simt_bwd_rowstats", st);
         if (tcb)
             k_bwd_rowstats_tc<<<static_cast<unsigned>((rows + 31) / 32), 256, 0, st>>>(

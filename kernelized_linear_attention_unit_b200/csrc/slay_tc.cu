@@ -2039,7 +2039,7 @@ cudaError_t set_smem(K kernel, size_t bytes)
 // sum over the nseg per-segment sums (every segment's sum is in the workspace when the state
 // kernel ran over all of them), z likewise, added in segment order.  One thread per four
 // consecutive (f, e) with 16-byte loads and stores, four segments' loads in flight before
-// their adds; the thread of e = 0..3 also sums z of its f.
+// their adds; the thread of e = 0..3 also sums z of its f, four loads deep as well.
 __global__ void k_state_total(const float* __restrict__ wsS, const float* __restrict__ wsZ, int BH,
                               int nseg, int Fc, int Ftot, int c0, const float* __restrict__ s_in,
                               const float* __restrict__ z_in, float* __restrict__ s_out,
@@ -2074,7 +2074,15 @@ __global__ void k_state_total(const float* __restrict__ wsS, const float* __rest
             const int64_t dz = static_cast<int64_t>(bh) * Ftot + c0 + f;
             const float* zs = wsZ + static_cast<int64_t>(bh) * nseg * Fc + f;
             float az = z_in ? z_in[dz] : 0.0f;
-            for (int t = 0; t < nseg; ++t) az += zs[static_cast<int64_t>(t) * Fc];
+            int t = 0;
+            for (; t + 4 <= nseg; t += 4) {
+                float y[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) y[u] = zs[static_cast<int64_t>(t + u) * Fc];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) az += y[u];
+            }
+            for (; t < nseg; ++t) az += zs[static_cast<int64_t>(t) * Fc];
             z_out[dz] = az;
         }
     }

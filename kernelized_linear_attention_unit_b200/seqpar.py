@@ -8,15 +8,16 @@ in its workspace), the ranks all-gather those states (F x (Dv+1) fp32 per (b, h)
 adds up the states of the ranks before it (slay_state_prefix) and runs its piece's causal
 forward from that state on the kept phi(k) (slay_attn_causal_fwd_finish).  The
 backward also needs, for each piece, the sum of phi(q) [dn, delta]^T over the later ranks'
-tokens: one more all-gather of the pieces' such sums (slay_causal_bwd_state), a suffix over
-ranks (slay_state_suffix), then the piece's backward from both states
-(slay_attn_causal_bwd_state).  The collective is NCCL's all-gather over NVLink on GPUs (any
+tokens: one more all-gather of the pieces' such sums (slay_attn_causal_bwd_begin, which keeps
+phi(q) and the row statistics in its workspace), a suffix over ranks (slay_state_suffix),
+then the piece's backward from both states on the kept values (slay_attn_causal_bwd_finish).  The collective is NCCL's all-gather over NVLink on GPUs (any
 backend works: the states are ordinary tensors); no kernel waits on another rank's memory.
 
 Every step of the path runs in the library's kernels; this module orders them and calls the
 collective.  The steps are passed in as an object (LibraryOps by default: begin, prefix,
-finish for the forward; state, bwd_state, suffix, backward for the backward), so the same
-orchestration runs in tests on CPU ranks.
+finish for the forward; bwd_begin, suffix, bwd_finish, and state when the forward's prefix
+state is not passed in, for the backward), so the same orchestration runs in tests on CPU
+ranks.
 """
 from typing import Optional
 
@@ -48,17 +49,19 @@ class LibraryOps:
     def prefix(self, S_all, z_all, rank, S_in, z_in):
         bd.slay_state_prefix(S_all, z_all, rank, S_in, z_in)
 
-    def bwd_state(self, q, out, den, dout, G_out, zg_out):
-        bd.slay_causal_bwd_state(q, out, den, dout, G_out, zg_out, self.R, self.m, self.seed,
-                                 self.eps)
+    def bwd_begin(self, q, out, den, dout, G_out, zg_out, handle=None):
+        """The piece's phi(q)[dn, delta] sum; returns the workspace that carries phi(q) and
+        the row statistics to bwd_finish."""
+        return bd.slay_attn_causal_bwd_begin(q, out, den, dout, G_out, zg_out, self.R, self.m,
+                                             self.seed, self.eps, workspace=handle)
 
     def suffix(self, G_all, zg_all, rank, G_in, zg_in):
         bd.slay_state_suffix(G_all, zg_all, rank, G_in, zg_in)
 
-    def backward(self, q, k, v, out, den, dout, dq, dk, dv, S_in, z_in, G_in, zg_in):
-        bd.slay_attn_causal_bwd_state(q, k, v, out, den, dout, dq, dk, dv, self.R, self.m,
-                                      self.seed, self.eps, S_in=S_in, z_in=z_in, G_in=G_in,
-                                      zg_in=zg_in)
+    def bwd_finish(self, q, k, v, out, den, dout, dq, dk, dv, S_in, z_in, G_in, zg_in, handle):
+        bd.slay_attn_causal_bwd_finish(q, k, v, out, den, dout, dq, dk, dv, self.R, self.m,
+                                       self.seed, self.eps, handle, S_in=S_in, z_in=z_in,
+                                       G_in=G_in, zg_in=zg_in)
 
 
 def gather_states(S_loc: torch.Tensor, z_loc: torch.Tensor, group=None):
@@ -109,8 +112,9 @@ def causal_bwd_seqpar(q, k, v, out, den, dout, dq, dk, dv, F: int, ops, group=No
 
     Besides the prefix state of the forward (the sum of phi(k)[v, 1] over the earlier
     ranks), the backward needs the sum of phi(q)[dn, delta] over the later ranks' tokens:
-    each rank computes its piece's (ops.bwd_state), the ranks all-gather them and each adds
-    up those of the ranks after it (ops.suffix) before its local backward (ops.backward).
+    each rank computes its piece's (ops.bwd_begin), the ranks all-gather them and each adds
+    up those of the ranks after it (ops.suffix) before its local backward (ops.bwd_finish,
+    on what bwd_begin kept).
     fwd_state: the (S_in, z_in) this rank's forward started from (the scratch of
     causal_fwd_seqpar on the same q, k, v), which saves recomputing it."""
     rank = dist.get_rank(group) if dist.is_initialized() else 0
@@ -118,8 +122,10 @@ def causal_bwd_seqpar(q, k, v, out, den, dout, dq, dk, dv, F: int, ops, group=No
     Dv = v.shape[-1]
     sc = scratch if scratch is not None else {}
     shape_s, shape_z = (B, H, F, Dv), (B, H, F)
-    if sc.get("bwd_shape") != (shape_s, q.device):
-        sc["bwd_shape"] = (shape_s, q.device)
+    key = (shape_s, q.shape[2], q.dtype, q.device)
+    if sc.get("bwd_shape") != key:
+        sc["bwd_shape"] = key
+        sc.pop("bwd_handle", None)
         for name in ("bS_loc", "bS_in", "bG_loc", "bG_in"):
             sc[name] = torch.empty(shape_s, dtype=torch.float32, device=q.device)
         for name in ("bz_loc", "bz_in", "bzg_loc", "bzg_in"):
@@ -131,8 +137,10 @@ def causal_bwd_seqpar(q, k, v, out, den, dout, dq, dk, dv, F: int, ops, group=No
         S_in, z_in = sc["bS_in"], sc["bz_in"]
     else:
         S_in, z_in = fwd_state
-    ops.bwd_state(q, out, den, dout, sc["bG_loc"], sc["bzg_loc"])
+    sc["bwd_handle"] = ops.bwd_begin(q, out, den, dout, sc["bG_loc"], sc["bzg_loc"],
+                                     sc.get("bwd_handle"))
     G_all, zg_all = gather_states(sc["bG_loc"], sc["bzg_loc"], group)
     ops.suffix(G_all, zg_all, rank, sc["bG_in"], sc["bzg_in"])
-    ops.backward(q, k, v, out, den, dout, dq, dk, dv, S_in, z_in, sc["bG_in"], sc["bzg_in"])
+    ops.bwd_finish(q, k, v, out, den, dout, dq, dk, dv, S_in, z_in, sc["bG_in"], sc["bzg_in"],
+                   sc["bwd_handle"])
     return dq, dk, dv

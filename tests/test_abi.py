@@ -76,7 +76,9 @@ def test_workspace_bytes():
 @pytest.mark.parametrize("op,dt,B,H,L,R,m,want", [
     ("CAUSAL_FWD", "BF16", 1, 16, 16384, 4, 64, 3),       # the headline: tensor cores
     ("CAUSAL_FWD", "F32", 1, 16, 16384, 4, 64, 0),        # fp32: CUDA cores
-    ("CAUSAL_FWD", "BF16", 1, 2, 100, 4, 32, 0),          # m % 64 != 0
+    ("CAUSAL_FWD", "BF16", 1, 2, 100, 4, 32, 1),          # m % 64 != 0: CUDA-core contraction
+    ("BIDIR_FWD", "BF16", 1, 2, 100, 4, 32, 1),           # after the tensor-core map
+    ("CAUSAL_FWD", "BF16", 1, 2, 100, 3, 32, 0),          # F % 128 != 0: no tensor cores
     ("CAUSAL_FWD", "BF16", 2, 16, 8192, 8, 64, 3),        # F = 512 in two chunks
     ("CAUSAL_FWD", "BF16", 1, 2, 100, 16, 64, 0),         # F = 1024 > 512
     ("CAUSAL_FWD", "BF16", 0, 2, 100, 4, 64, 0),          # empty

@@ -146,20 +146,25 @@ class _OracleOps:
         S_in.copy_(S_all[:rank].sum(0) if rank else torch_zeros_like(S_in))
         z_in.copy_(z_all[:rank].sum(0) if rank else torch_zeros_like(z_in))
 
-    def bwd_state(self, q, out, den, dout, G_out, zg_out):
+    def bwd_begin(self, q, out, den, dout, G_out, zg_out, handle=None):
         import oracle as O
         zeros = np.zeros(q.shape)
         _, _, _, G, zg = O.attn_causal_bwd_state(q.numpy(), zeros, zeros, out.numpy(), den.numpy(),
                                                  dout.numpy(), self.P)
         G_out.copy_(torch_from(G))
         zg_out.copy_(torch_from(zg))
+        self.bwd_begins = getattr(self, "bwd_begins", 0) + 1
+        h = handle if handle is not None else {}
+        h.update(q=q, dout=dout, n=self.bwd_begins)
+        return h
 
     def suffix(self, G_all, zg_all, rank, G_in, zg_in):
         G_in.copy_(G_all[rank + 1:].sum(0) if rank + 1 < G_all.shape[0] else torch_zeros_like(G_in))
         zg_in.copy_(zg_all[rank + 1:].sum(0) if rank + 1 < zg_all.shape[0] else torch_zeros_like(zg_in))
 
-    def backward(self, q, k, v, out, den, dout, dq, dk, dv, S_in, z_in, G_in, zg_in):
+    def bwd_finish(self, q, k, v, out, den, dout, dq, dk, dv, S_in, z_in, G_in, zg_in, handle):
         import oracle as O
+        assert handle["q"] is q and handle["dout"] is dout and handle["n"] == self.bwd_begins
         st = [x.double().numpy() for x in (S_in, z_in, G_in, zg_in)]
         a, b, c, _, _ = O.attn_causal_bwd_state(q.numpy(), k.numpy(), v.numpy(), out.numpy(),
                                                 den.numpy(), dout.numpy(), self.P, *st)

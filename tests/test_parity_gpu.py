@@ -769,6 +769,73 @@ def test_two_call_forward_emulating_ranks(dt, R, m, L, cuts):
         check(name + " piece z", host(z), wz, TOL[dt])
 
 
+@pytest.mark.parametrize("dt,R,m,L,cuts", [("bf16", 4, 64, 1000, (300, 700)),
+                                           ("bf16", 8, 64, 700, (128, 512)),
+                                           ("bf16", 4, 64, 600, (0, 600)),
+                                           ("f32", 2, 16, 300, (1, 150)),
+                                           ("bf16", 2, 16, 257, (64, 65))])
+def test_two_call_backward_emulating_ranks(dt, R, m, L, cuts):
+    # the two-call backward: every piece's begin (its phi(q)[dn, delta] sum, phi(q) and the
+    # row statistics kept in its own workspace) before any finish; the gradients bit for bit
+    # against the one-call piece backward on the same outside sums, and against the oracle's
+    # whole-sequence backward
+    w = small(dt, R, m, L, B=1, H=3, seed=29)
+    q, k, v = W.gen_qkv(w)
+    g = W.gen_dout(w)
+    P = params(w)
+    F, eps = w.F, _eps(w)
+    qt, kt, vt, gt = dev(q, dt), dev(k, dt), dev(v, dt), dev(g, dt)
+    out = torch.empty((1, 3, L, 64), device="cuda", dtype=TDT[dt])
+    den = torch.empty((1, 3, L), device="cuda")
+    bd.slay_attn_causal_fwd(qt, kt, vt, out, den, R, m, w.sketch_seed, eps)
+    bounds = (0,) + tuple(cuts) + (L,)
+    pieces = [(a, b) for a, b in zip(bounds[:-1], bounds[1:])]
+
+    def piece(t, a, b):
+        return t[:, :, a:b].contiguous()
+
+    def state_pair():
+        return torch.empty((1, 3, F, 64), device="cuda"), torch.empty((1, 3, F), device="cuda")
+
+    Ss, zs, Gs, zgs, wss = [], [], [], [], []
+    for a, b in pieces:
+        S, z = state_pair()
+        bd.slay_kernel_status(bd.slay_causal_state(piece(kt, a, b), piece(vt, a, b), S, z, R, m,
+                                                    w.sketch_seed, eps))
+        G, zg = state_pair()
+        wss.append(bd.slay_attn_causal_bwd_begin(piece(qt, a, b), piece(out, a, b),
+                                                 piece(den, a, b), piece(gt, a, b), G, zg, R, m,
+                                                 w.sketch_seed, eps))
+        Ss.append(S)
+        zs.append(z)
+        Gs.append(G)
+        zgs.append(zg)
+    S_all, z_all, G_all, zg_all = (torch.stack(x) for x in (Ss, zs, Gs, zgs))
+    grads = []
+    for r, (a, b) in enumerate(pieces):
+        S_in, z_in = state_pair()
+        G_in, zg_in = state_pair()
+        bd.slay_state_prefix(S_all, z_all, r, S_in, z_in)
+        bd.slay_state_suffix(G_all, zg_all, r, G_in, zg_in)
+        n = b - a
+        args = [piece(t, a, b) for t in (qt, kt, vt, out, den, gt)]
+        got = [torch.empty((1, 3, n, 64), device="cuda") for _ in range(3)]
+        ref = [torch.empty((1, 3, n, 64), device="cuda") for _ in range(3)]
+        bd.slay_attn_causal_bwd_finish(*args, *got, R, m, w.sketch_seed, eps, wss[r], S_in=S_in,
+                                       z_in=z_in, G_in=G_in, zg_in=zg_in)
+        bd.slay_kernel_status(wss[r])
+        bd.slay_kernel_status(bd.slay_attn_causal_bwd_state(*args, *ref, R, m, w.sketch_seed, eps,
+                                                            S_in=S_in, z_in=z_in, G_in=G_in,
+                                                            zg_in=zg_in))
+        torch.cuda.synchronize()
+        for x, y in zip(got, ref):
+            assert torch.equal(x, y), (r, a, b)
+        grads.append(tuple(host(x) for x in got))
+    name = "two-call bwd %s R%d m%d L%d %s" % (dt, R, m, L, cuts)
+    got = tuple(np.concatenate([x[i] for x in grads], axis=2) for i in range(3))
+    _check_bwd(name, got, _bwd_reference(q, k, v, g, P, dt), TOL[dt])
+
+
 def test_two_call_forward_rejects_small_workspace():
     w = small("bf16", 4, 64, 512, B=1, H=2, seed=28)
     q, k, v = (dev(x, "bf16") for x in W.gen_qkv(w))

@@ -61,9 +61,14 @@ OPS = {"causal": bd.OP_CAUSAL_FWD, "bidir": bd.OP_BIDIR_FWD, "state": bd.OP_CAUS
        "bidir_bwd": bd.OP_BIDIR_BWD, "fmap": bd.OP_FEATURE_MAP, "fmap_bwd": bd.OP_FEATURE_MAP_BWD}
 
 
+# trace names of the fused tensor-core forward kernels (projection and phi inside them)
+FWD_TC = {"tc_kphi_state", "tc_qphi_out", "tc_bidir_state", "tc_bidir_out", "tc_state_sums",
+          "tc_causal_state", "tc_causal_out", "tc_state_total"}
+
+
 def _observed(op, names):
-    if op in FWD_OPS:
-        return 3 if any(n.startswith("tc_") for n in names) else 0
+    if op in FWD_OPS and any(n in FWD_TC for n in names):
+        return bd.PATH_TC_FEATURE_MAP | bd.PATH_TC_CONTRACTION
     mask = 0
     if "tc_feature_map" in names:
         mask |= bd.PATH_TC_FEATURE_MAP
