@@ -11,20 +11,22 @@
 //   dx = (dx^ - x^ (x^ . dx^)) / n   (dx^ / 1e-12 below the norm guard |x| < 1e-12).
 // Both contractions run on tensor cores: per 128-row tile and 64-feature group g (a job) the
 // projections U = X W_g^T (N = 128: 64 omega and 64 anchor columns, as in the forward map),
-// then dX^ += [alpha | beta]_g [Omega_g ; A_g] (K = 128, N = 64) with the same W tiles read
-// as an MN-major operand.  The kernel reads x (bf16), dphi (bf16, as the tensor-core
+// then dX^ += [alpha | beta]_g [Omega_g ; A_g] (K = 128, N = 64) with [alpha | beta] read from
+// tensor memory and the same W tiles read as an MN-major shared-memory operand.  The kernel reads x (bf16), dphi (bf16, as the tensor-core
 // contraction stores it) and writes dx (fp32): its DRAM traffic is dominated by the dphi
 // reads (2F bytes per row).
 //
 // Persistent, one CTA per SM, 128-row tiles round-robin.  Warp 9 issues the TMA loads: X
-// tiles, and per job the group's W operand (three slots, L2-resident) and the dphi tile
-// [128 rows][64 features] (two slots).  Warp 0 issues the MMAs.  Warps 1-8 are the epilogue:
-// warp w serves TMEM lanes 32 (w % 4).. (rows of the tile) and the 32-feature half
-// (w - 1) / 4 of every group; per job it reads its rows' dphi from the shared-memory tile,
-// its projections from tensor memory, and writes its block of [alpha | beta] into a K-major
-// 128-byte-swizzled operand tile; per tile, after the next tile's jobs, it turns dX^ into
-// dx and stores its 32 x 32 block by TMA.  Every wait is bounded; a timeout sets the
-// library's feature-map status word.
+// tiles, and per job the group's W operand (five slots, L2-resident) and the dphi tile
+// [128 rows][64 features] (four slots: the dphi stream is the kernel's DRAM traffic, and the
+// loads run up to four jobs ahead of the epilogue so that enough of it is in flight).  Warp 0
+// issues the MMAs.  Warps 1-8 are the epilogue: warp w serves TMEM lanes 32 (w % 4).. (rows
+// of the tile) and the 32-feature half (w - 1) / 4 of every group; per job it reads its rows'
+// dphi from the shared-memory tile, its projections from tensor memory, and writes its block
+// of [alpha | beta] back into tensor memory as the contraction's A operand (bf16 pairs, one
+// row per lane); per tile, after the next tile's jobs, it turns dX^ into dx and stores its
+// 32 x 32 block by TMA.  Every wait is bounded; a timeout sets the library's feature-map
+// status word.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -45,16 +47,16 @@ constexpr int kRows = 128;                  // rows per tile (MMA M)
 constexpr int kBoxBytes = kRows * 128;      // [128 rows][64 bf16] swizzled X tile = 16 KiB
 constexpr int kSubBytes = 64 * 128;         // packed W of 32 features = 8 KiB
 constexpr int kGroupBytes = 2 * kSubBytes;  // 64 features = 16 KiB
-constexpr int kABytes = 2 * kBoxBytes;      // [alpha | beta] of one group: two 16 KiB K-tiles
 constexpr int kEpiWarps = 8;
 constexpr int kPbThreads = 32 * (2 + kEpiWarps);   // MMA warp, 8 epilogue warps, TMA warp
 constexpr int kNumSMs = 148;
 constexpr int kXBufs = 3;                   // X tiles in flight
-constexpr int kRing = 3;                    // W groups in flight (slot = job % 3)
-constexpr int kDRing = 2;                   // dphi tiles in flight (slot = job % 2)
+constexpr int kRing = 5;                    // W groups in flight (slot = job % 5)
+constexpr int kDRing = 4;                   // dphi tiles in flight (slot = job % 4)
 constexpr int kStgBytes = 32 * 128;         // per epilogue warp: [32 rows][32 fp32] of dx
 constexpr uint32_t kColU = 0;               // two 128-column projection buffers
 constexpr uint32_t kColDX = 256;            // two 64-column dX^ accumulators
+constexpr uint32_t kColA = 384;             // two 64-column [alpha | beta] operands (bf16 pairs)
 
 enum {
     PB_XF = 0,                  // + slot (TMA: X tile)
@@ -64,7 +66,7 @@ enum {
     PB_GF = PB_WE + kRing,      // + slot (TMA: dphi tile)
     PB_GE = PB_GF + kDRing,     // + slot (8 warp arrivals: dphi read)
     PB_UF = PB_GE + kDRing,     // + buffer (projection MMA commit)
-    PB_AF = PB_UF + 2,          // + buffer (8 warp arrivals: [alpha | beta] written)
+    PB_AF = PB_UF + 2,          // + buffer (8 warp arrivals: [alpha | beta] in tensor memory)
     PB_AE = PB_AF + 2,          // + buffer (contraction MMA commit: operand free)
     PB_DF = PB_AE + 2,          // + buffer (dX^ of a tile complete)
     PB_DE = PB_DF + 2,          // + buffer (8 warp arrivals: dX^ read)
@@ -72,7 +74,7 @@ enum {
 };
 
 struct PbLayout {
-    uint32_t w, x, a, d, stg, bar, tmem, total;
+    uint32_t w, x, d, stg, bar, tmem, total;
 };
 
 __host__ __device__ inline PbLayout pb_layout(int /*F*/)
@@ -80,8 +82,7 @@ __host__ __device__ inline PbLayout pb_layout(int /*F*/)
     PbLayout l;
     l.w = 0;                                // kRing W groups (16 KiB each)
     l.x = l.w + kRing * kGroupBytes;        // kXBufs X tiles
-    l.a = l.x + kXBufs * kBoxBytes;         // 2 [alpha | beta] operands
-    l.d = l.a + 2 * kABytes;                // kDRing dphi tiles [128 rows][64 features]
+    l.d = l.x + kXBufs * kBoxBytes;         // kDRing dphi tiles [128 rows][64 features]
     l.stg = l.d + kDRing * kBoxBytes;       // kEpiWarps dx staging boxes (TMA stores)
     l.bar = l.stg + kEpiWarps * kStgBytes;
     l.tmem = l.bar + PB_NUM * 8;
@@ -166,8 +167,9 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
 
     if (warp == 9) {
         // ---------------------------------------------------------------- TMA loads, in
-        // job order: the X tile at each tile's first group, then per job its W group and its
-        // dphi tile, each into a slot freed by the job kRing (X: kXBufs tiles) before
+        // job order: the X tile at each tile's first group (into the slot the tile kXBufs
+        // before released), then per job its W group and its dphi tile (into the slots the
+        // jobs kRing and kDRing before released)
         if (lane == 0) {
             Ring xr(kXBufs), rr(kRing), gr(kDRing);
             for (int j = 0, k = 0, g = 0; j < njobs && wt.ok; ++j) {
@@ -210,7 +212,6 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
             constexpr uint32_t idD = idesc_bf16(128, 64, 0, 1);    // [alpha|beta] x W (MN-major)
             const uint64_t dx0 = sdesc(sbase + L.x, 16, 1024, kLayoutSW128);
             const uint64_t dw0 = sdesc(sbase + L.w, 16, 1024, kLayoutSW128);
-            const uint64_t da0 = sdesc(sbase + L.a, 16, 1024, kLayoutSW128);
             // projection job jp = (tile pk, group pg) from X slot px and W slot pw
             int jp = 0, pg = 0;
             Ring px(kXBufs), pw(kRing);
@@ -251,15 +252,15 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
                     wt.wait(&bar[PB_DE + (k & 1)], ph);
                 }
                 tc_fence_after();
-                // dX^_k += [alpha|beta]_j [Omega_g ; A_g]: K = 128 (two 64-wide K-tiles of
-                // the operand; the W rows of the group 2 KiB per 16-row K step)
-                const uint64_t da = da0 + (((j & 1) * kABytes) >> 4);
+                // dX^_k += [alpha|beta]_j [Omega_g ; A_g]: K = 128, 16 per MMA (eight columns of
+                // bf16 pairs of the tensor-memory operand; the W rows of the group 2 KiB per
+                // 16-row K step)
+                const uint32_t ta = tmem0 + kColA + 64u * (j & 1);
                 const uint64_t dwm = dw0 + ((cw.slot * kGroupBytes) >> 4);   // same tiles, MN-major
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    umma_bf16(tmem0 + kColDX + 64u * (k & 1),
-                              da + (kk >> 2) * (kBoxBytes >> 4) + 2 * (kk & 3), dwm + 128 * kk, idD,
-                              (g > 0 || kk > 0) ? 1u : 0u);
+                    umma_bf16_ts(tmem0 + kColDX + 64u * (k & 1), ta + 8 * kk, dwm + 128 * kk, idD,
+                                 (g > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(&bar[PB_AE + (j & 1)]);
                 umma_commit(&bar[PB_WE + cw.slot]);   // the group's W (projection and contraction) done
                 if (g == ng - 1) umma_commit(&bar[PB_DF + (k & 1)]);
@@ -276,7 +277,6 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
         const int ew = warp - 1, q = warp & 3, half = ew >> 2;
         const uint32_t row = 32u * q + lane;
         const uint32_t trow = tmem0 + ((32u * q) << 16);
-        const uint32_t abase = sbase + L.a + half * kBoxBytes;
         // dx of tile k (X slot s, its rows' 1/|x| and |x|): dX^ (64 columns) -> (dX^ - x^
         // (x^ . dX^)) / n, this warp's half.  It runs after the next tile's jobs, so the wait
         // for the tile's last contraction is hidden behind them (dX^ is double buffered; the
@@ -415,17 +415,13 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
                     uint32_t ph = static_cast<uint32_t>(((j - 2) >> 1) & 1);
                     wt.wait(&bar[PB_AE + (j & 1)], ph);
                 }
-                // K order of the operand: [alpha | beta] of sub-slice 2g in K-tile 0, of 2g+1
-                // in K-tile 1 -- the row order of the group's packed W (32 omega, 32 anchor)
-                const uint32_t arow = abase + (j & 1) * kABytes;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    st_shared_v4(arow + sw128_off(row, c), al[4 * c], al[4 * c + 1], al[4 * c + 2],
-                                 al[4 * c + 3]);
-                    st_shared_v4(arow + sw128_off(row, 4 + c), be[4 * c], be[4 * c + 1],
-                                 be[4 * c + 2], be[4 * c + 3]);
-                }
-                fence_async_smem();
+                // K order of the operand: alpha then beta of sub-slice 2g in K 0..63 (columns
+                // 0..31), of 2g+1 in K 64..127 -- the row order of the group's packed W (32
+                // omega, 32 anchor); this warp writes its rows' 32 columns of sub-slice 2g+half
+                const uint32_t acol = trow + kColA + 64u * (j & 1) + 32u * half;
+                tmem_st16(acol, al);
+                tmem_st16(acol + 16, be);
+                tmem_wait_st();
                 tc_fence_before();
                 warp_arrive(&bar[PB_AF + (j & 1)]);
             }
