@@ -161,6 +161,41 @@ def test_argument_errors_before_any_device_work():
               None) == bd.SLAY_ERR_INVALID_ARG
 
 
+def test_two_call_argument_errors_before_any_device_work():
+    # the sequence-parallel two-call pairs check their arguments on the host like the rest
+    L = bd.lib()
+    F, big, ws = _fake(0x30000), 1 << 40, _fake(0x20000)
+    sz = [1, 1, 128, 64, 64, bd.SLAY_BF16, 4, 64, 1234, 1e-6]
+    fb = L.slay_attn_causal_fwd_begin
+    assert fb(_fake(), _fake(), None, None, *sz, ws, big, None) == bd.SLAY_ERR_INVALID_ARG
+    assert fb(_fake(), _fake(), _fake(0x30004), _fake(), *sz, ws, big, None) == bd.SLAY_ERR_INVALID_ARG
+    assert fb(None, _fake(), F, _fake(), *sz, ws, big, None) == bd.SLAY_ERR_INVALID_ARG
+    assert fb(_fake(), _fake(), F, _fake(), *sz, None, big, None) == bd.SLAY_ERR_INVALID_ARG
+    assert fb(_fake(), _fake(), F, _fake(), *sz, ws, 256, None) == bd.SLAY_ERR_INVALID_ARG
+    assert fb(_fake(), _fake(), F, _fake(), *sz, _fake(0x20010), big, None) == bd.SLAY_ERR_INVALID_ARG
+    assert fb(_fake(), _fake(), F, _fake(), 0, *sz[1:], None, 0, None) == bd.SLAY_OK   # B = 0
+    ff = L.slay_attn_causal_fwd_finish
+    q5 = [_fake()] * 4
+    assert ff(None, _fake(), _fake(), _fake(), None, None, None, *sz, ws, big, None) == bd.SLAY_ERR_INVALID_ARG
+    assert ff(*q5, None, F, None, *sz, ws, big, None) == bd.SLAY_ERR_INVALID_ARG          # S_in without z_in
+    assert ff(*q5, _fake(0x10002), None, None, *sz, ws, big, None) == bd.SLAY_ERR_INVALID_ARG
+    assert ff(*q5, None, None, None, *sz, ws, 256, None) == bd.SLAY_ERR_INVALID_ARG
+    sz0 = list(sz)
+    sz0[2] = 0
+    assert ff(None, None, None, None, None, None, None, *sz0, None, 0, None) == bd.SLAY_OK   # L = 0
+    bb = L.slay_attn_causal_bwd_begin
+    assert bb(_fake(), _fake(), _fake(), _fake(), None, None, *sz, ws, big, None) == bd.SLAY_ERR_INVALID_ARG
+    assert bb(_fake(), _fake(), None, _fake(), F, _fake(), *sz, ws, big, None) == bd.SLAY_ERR_INVALID_ARG
+    assert bb(_fake(), _fake(), _fake(), _fake(), F, _fake(), *sz, ws, 256, None) == bd.SLAY_ERR_INVALID_ARG
+    bf = L.slay_attn_causal_bwd_finish
+    nine = [_fake()] * 9
+    assert bf(*nine, None, None, F, None, *sz, ws, big, None) == bd.SLAY_ERR_INVALID_ARG  # G_in without zg_in
+    assert bf(*nine[:6], None, _fake(), _fake(), None, None, None, None, *sz, ws, big,
+              None) == bd.SLAY_ERR_INVALID_ARG                                         # dq missing
+    assert bf(*nine, None, None, None, None, *sz, ws, 256, None) == bd.SLAY_ERR_INVALID_ARG
+    assert bf(*([None] * 13), *sz0, None, 0, None) == bd.SLAY_OK                         # L = 0
+
+
 def test_sketch_params_rejects_bad_args():
     L = bd.lib()
     assert L.slay_sketch_params(64, 0, 4, 1, 1e-6, None, None, None, None) == bd.SLAY_ERR_INVALID_ARG
