@@ -212,14 +212,17 @@ def _seqpar_rank(rank, world, port, outdir):
         dist.destroy_process_group()
 
 
-def test_sequence_parallel_orchestration_two_ranks():
-    # two gloo ranks each hold half of a sequence; the package's orchestration (piece state,
-    # all-gather, prefix over earlier ranks, forward from it) reproduces the whole sequence
+@pytest.mark.parametrize("world", [2, 3])
+def test_sequence_parallel_orchestration(world):
+    # gloo ranks each hold a contiguous piece of a sequence; the package's orchestration (piece
+    # state, all-gather, prefix over earlier ranks, forward from it) reproduces the whole
+    # sequence (with three ranks the middle one starts from a non-zero, non-total prefix)
     import torch.multiprocessing as mp
     import oracle as O
     outdir = tempfile.mkdtemp(prefix="slay_sp_")
-    mp.spawn(_seqpar_rank, args=(2, _free_port(), outdir), nprocs=2, join=True)
-    got = np.concatenate([np.load(os.path.join(outdir, "sp%d.npy" % r)) for r in range(2)], axis=2)
+    mp.spawn(_seqpar_rank, args=(world, _free_port(), outdir), nprocs=world, join=True)
+    got = np.concatenate([np.load(os.path.join(outdir, "sp%d.npy" % r)) for r in range(world)],
+                         axis=2)
     w = W.Workload("sp", B=1, H=2, L=90, R=2, m=8, dtype="f32", data_seed=61)
     q, k, v = W.gen_qkv(w)
     P = O.sketch_params(w.D, w.R, w.m, w.sketch_seed, float(np.float32(w.eps)))
@@ -261,15 +264,18 @@ def _seqpar_bwd_rank(rank, world, port, outdir):
         dist.destroy_process_group()
 
 
-def test_sequence_parallel_backward_orchestration_two_ranks():
-    # two gloo ranks each hold half of a sequence: forward as above, then each rank's piece
+@pytest.mark.parametrize("world", [2, 3])
+def test_sequence_parallel_backward_orchestration(world):
+    # gloo ranks each hold a piece of a sequence: forward as above, then each rank's piece
     # state and phi(q)[dn, delta] sum all-gathered, prefix and suffix over ranks, and the
-    # piece's backward; together they are the whole sequence's gradients
+    # piece's backward; together they are the whole sequence's gradients (with three ranks
+    # the middle one has both a non-zero prefix and a non-zero suffix)
     import torch.multiprocessing as mp
     import oracle as O
     outdir = tempfile.mkdtemp(prefix="slay_spb_")
-    mp.spawn(_seqpar_bwd_rank, args=(2, _free_port(), outdir), nprocs=2, join=True)
-    got2 = np.concatenate([np.load(os.path.join(outdir, "spb%d.npy" % r)) for r in range(2)], axis=4)
+    mp.spawn(_seqpar_bwd_rank, args=(world, _free_port(), outdir), nprocs=world, join=True)
+    got2 = np.concatenate([np.load(os.path.join(outdir, "spb%d.npy" % r)) for r in range(world)],
+                          axis=4)
     np.testing.assert_array_equal(got2[0], got2[1])
     got = got2[0]
     w = W.Workload("spb", B=1, H=2, L=60, R=2, m=8, dtype="f32", data_seed=62)
