@@ -402,9 +402,9 @@ k_tc_phi_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CU
                     const float2 d = make_float2(dphi_val(dp, c), dphi_val(dp, c + 1));
                     const float2 p = make_float2(__uint_as_float(pr[c]), __uint_as_float(pr[c + 1]));
                     const float2 y = ffma2(a2, make_float2(__uint_as_float(ur[c]), __uint_as_float(ur[c + 1])), b2);
-                    // a quarter of the exp2 (every other pair's second) on the FMA pipe: the
-                    // special-function unit is the busiest pipe of this loop
-                    const float2 e = make_float2(ex2(y.x), (c & 2) ? ex2_poly(y.y) : ex2(y.y));
+                    // every exp2 on the special-function unit: moving a share onto the FMA pipe
+                    // as a polynomial made this loop issue-bound (measured slower)
+                    const float2 e = make_float2(ex2(y.x), ex2(y.y));
                     const float2 t = fmul2(fmul2(d, e), p);
                     const float2 af = fmul2(fmul2(t, p), sq2);
                     const float2 bf = fmul2(t, tn2);
