@@ -183,6 +183,48 @@ def torch_zeros_like(t):
     return torch.zeros_like(t)
 
 
+def test_seqpar_scratch_reuses_the_handle_only_for_the_same_piece():
+    # without a process group (one rank): begin's workspace handle is kept in the scratch and
+    # handed back to begin on the next step of the same sizes; a new piece length or dtype
+    # starts a new one (the library's workspace size depends on both)
+    import torch
+    from kernelized_linear_attention_unit_b200 import seqpar
+
+    class CountingOps:
+        def __init__(self):
+            self.given, self.made = [], 0
+
+        def begin(self, k, v, S_out, z_out, handle=None):
+            self.given.append(handle)
+            if handle is None:
+                self.made += 1
+                handle = {"id": self.made}
+            S_out.zero_()
+            z_out.zero_()
+            return handle
+
+        def prefix(self, S_all, z_all, rank, S_in, z_in):
+            S_in.zero_()
+            z_in.zero_()
+
+        def finish(self, q, k, v, out, den, S_in, z_in, handle):
+            out.zero_()
+
+    ops, sc = CountingOps(), {}
+
+    def step(L, dtype=torch.float64):
+        q, k, v = (torch.zeros((1, 2, L, 64), dtype=dtype) for _ in range(3))
+        seqpar.causal_fwd_seqpar(q, k, v, torch.empty_like(v), torch.empty((1, 2, L)), 16,
+                                 ops, scratch=sc)
+
+    step(40)
+    step(40)
+    step(41)
+    step(41, torch.float32)
+    assert [h["id"] if h else None for h in ops.given] == [None, 1, None, None]
+    assert ops.made == 3
+
+
 def _seqpar_rank(rank, world, port, outdir):
     import torch
     import torch.distributed as dist
