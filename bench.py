@@ -7,9 +7,10 @@
                                 seqpar_bwd_8k]
 
 seqpar_16k splits the headline sequence over the N ranks (strong scaling, one all-gather of
-the pieces' states per step), seqpar_bwd_8k the fwd/bwd sequence for its backward (two
-all-gathers: the states before and after each piece); every other workload gives each rank
-its own batch (weak).
+the pieces' states per step), seqpar_bwd_8k the fwd/bwd sequence for its backward (one
+all-gather per step, of the pieces' phi(q)[dn, delta] sums; the prefix state comes from the
+untimed forward); every other workload gives each rank its own batch (weak).  For those two
+the dominant kernel's work is counted over the rank's piece.
 
 With --gpus N > 1 outside torchrun, bench.py starts the N ranks itself (torch.distributed.run
 on 127.0.0.1); under torchrun, --gpus must equal WORLD_SIZE.
@@ -25,6 +26,7 @@ Prints one JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle (th
 reference this method has) on the host cores instead.
 """
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -410,6 +412,8 @@ def run_ours(args, w, op):
     # inputs: each rank draws its own batch (data seed offset by rank); the sequence-parallel
     # workload shares one sequence
     wr = w if op in ("seqpar", "seqpar_bwd") else rank_workload(w, rank)
+    # the sizes one launch of this rank works on (the sequence-parallel ops: its piece)
+    w_launch = w
     if op == "decode":
         qn, kn, vn, Sn, zn = W.gen_decode(wr)
         q, k, v = to_dev(qn), to_dev(kn), to_dev(vn)
@@ -449,6 +453,7 @@ def run_ours(args, w, op):
         def step():
             seqpar.causal_fwd_seqpar(q, k, v, out, den, w.F, ops, scratch=scratch)
         units_per_step = w.B * (b - a)
+        w_launch = dataclasses.replace(w, L=b - a)
         unit = "tokens/s"
     elif op == "seqpar_bwd":
         from kernelized_linear_attention_unit_b200 import seqpar
@@ -476,6 +481,7 @@ def run_ours(args, w, op):
             seqpar.causal_bwd_seqpar(q, k, v, out, den, g, dq, dk, dv, w.F, ops, scratch=scratch,
                                      fwd_state=fwd_state)
         units_per_step = w.B * (b - a)
+        w_launch = dataclasses.replace(w, L=b - a)
         unit = "tokens/s"
     elif op == "feature_map_bwd":
         qn, kn, _ = W.gen_qkv(wr)
@@ -597,7 +603,7 @@ def run_ours(args, w, op):
     if per:
         dom = max(per, key=lambda n: sum(per[n]))
         avg_s = sum(per[dom]) / len(per[dom]) / 1e3
-        wk = kernel_work(dom, w, op)
+        wk = kernel_work(dom, w_launch, op)
         if wk is not None:
             amount, kind, bound = wk
             if bound == "hbm":
